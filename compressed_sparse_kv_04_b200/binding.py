@@ -1,0 +1,185 @@
+"""Thin ctypes binding of libcsa.so (include/csa.h), same entry-point names.
+
+Argument marshalling only: every step runs in the library's CUDA kernels.
+Tensors are torch tensors on the current CUDA device; the current torch
+stream is passed as the `stream` argument.  Loading fails loudly when the
+library has not been built: there is no CPU fallback.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libcsa.so")
+
+CSA_OK = 0
+STATUS_NAMES = {0: "CSA_OK", 1: "CSA_ERR_INVALID_ARG", 2: "CSA_ERR_UNSUPPORTED_SHAPE",
+                3: "CSA_ERR_CAPACITY", 4: "CSA_ERR_WORKSPACE", 5: "CSA_ERR_CUDA",
+                6: "CSA_ERR_DEVICE_TIMEOUT", 7: "CSA_ERR_DEVICE_INDEX"}
+OP_INDEX_TOPK, OP_SPARSE_MQA, OP_DENSE_MQA, OP_PREFILL = 1, 2, 3, 4
+
+EXPORTS = ["csa_version", "csa_last_error", "csa_workspace_bytes", "hca_compress",
+           "csa_compress", "lightning_index_topk", "sparse_mqa_decode", "dense_mqa_decode",
+           "csa_prefill_chunk"]
+
+
+class CsaError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"{STATUS_NAMES.get(status, status)}: {msg}")
+        self.status = status
+
+
+class csa_params(C.Structure):
+    _fields_ = [("B", C.c_int), ("d", C.c_int), ("H", C.c_int), ("H_I", C.c_int),
+                ("D_I", C.c_int), ("k", C.c_int), ("window", C.c_int), ("rope_dim", C.c_int),
+                ("m", C.c_int), ("eps", C.c_float), ("softmax_scale", C.c_float),
+                ("rope_inv_freq", C.POINTER(C.c_double))]
+
+
+_lib = None
+
+
+def lib():
+    """The loaded libcsa.so (raises if it was not built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"libcsa.so not found at {LIB_PATH}; build it with "
+                               "`python -m compressed_sparse_kv_04_b200.build`")
+        L = C.CDLL(LIB_PATH)
+        _declare(L)
+        _lib = L
+    return _lib
+
+
+def _declare(L):
+    vp, i32, i64, sz = C.c_void_p, C.c_int, C.c_int64, C.c_size_t
+    P = C.POINTER(csa_params)
+    L.csa_version.restype = i32
+    L.csa_last_error.restype = C.c_char_p
+    L.csa_workspace_bytes.argtypes = [P, i32, i32, i64]
+    L.csa_workspace_bytes.restype = sz
+    L.hca_compress.argtypes = [P, vp, i64, vp, vp, vp, vp, i64, i64, vp, i64, vp, vp]
+    L.csa_compress.argtypes = [P, vp, i64, vp, vp, vp, vp, i64, i64, vp, i64, vp, vp, vp, vp,
+                               vp, vp, vp]
+    L.lightning_index_topk.argtypes = [P, i32, vp, vp, vp, vp, vp, i64, vp, vp, vp, vp, vp, sz,
+                                       vp, vp]
+    L.sparse_mqa_decode.argtypes = [P, vp, vp, vp, i64, vp, vp, vp, i64, vp, vp, vp, vp, vp, vp,
+                                    sz, vp, vp]
+    L.dense_mqa_decode.argtypes = [P, vp, vp, vp, i64, vp, i64, vp, vp, vp, vp, vp, vp, sz, vp,
+                                   vp]
+    L.csa_prefill_chunk.argtypes = [P, i64, i32, vp, vp, i64, vp, vp, vp, vp, vp, vp, vp, vp,
+                                    i64, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp, vp]
+    for name in EXPORTS[3:]:
+        getattr(L, name).restype = i32
+
+
+def make_params(B, d, H=0, H_I=0, D_I=0, k=0, window=0, rope_dim=0, m=4, eps=1e-6,
+                softmax_scale=0.0, rope_inv_freq=None):
+    p = csa_params(B, d, H, H_I, D_I, k, window, rope_dim, m, eps, softmax_scale, None)
+    if rope_inv_freq is not None:
+        arr = (C.c_double * len(rope_inv_freq))(*rope_inv_freq)
+        p.rope_inv_freq = C.cast(arr, C.POINTER(C.c_double))
+        p._keep = arr
+    return p
+
+
+def params_for(w, B=None, **kw):
+    """csa_params for a Workload (compressed_sparse_kv_04_b200.configs)."""
+    return make_params(B or w.B, w.d, w.H, w.H_I, w.D_I, w.k, w.W, w.rope_dim, w.m, **kw)
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"expected a torch.Tensor, got {type(t)}")
+    if not t.is_cuda:
+        raise ValueError("tensors must be on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("tensors must be contiguous")
+    return C.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return C.c_void_p(s.cuda_stream)
+
+
+def _check(status):
+    if status != CSA_OK:
+        raise CsaError(status, lib().csa_last_error().decode())
+
+
+def version():
+    return lib().csa_version()
+
+
+def workspace_bytes(p, op, Q, N_cap):
+    n = lib().csa_workspace_bytes(C.byref(p), op, Q, N_cap)
+    if n == 0:
+        raise CsaError(1, lib().csa_last_error().decode())
+    return n
+
+
+def workspace(p, op, Q, N_cap, device=None):
+    return torch.empty(workspace_bytes(p, op, Q, N_cap), dtype=torch.uint8,
+                       device=device or torch.cuda.current_device())
+
+
+def hca_compress(p, kv_tok, ctx_len, w_s, b_pos, gamma, first_block, n_blocks, kv_c,
+                 dev_status=None, stream=None):
+    _check(lib().hca_compress(C.byref(p), _ptr(kv_tok), kv_tok.shape[1], _ptr(ctx_len),
+                              _ptr(w_s), _ptr(b_pos), _ptr(gamma), first_block, n_blocks,
+                              _ptr(kv_c), kv_c.shape[1], _ptr(dev_status), _stream(stream)))
+
+
+def csa_compress(p, kv_tok, ctx_len, w_s, b_pos, gamma, first_block, n_blocks, kv_c,
+                 idx_tok=None, w_s_idx=None, b_pos_idx=None, idx_key=None, idx_scale=None,
+                 dev_status=None, stream=None):
+    _check(lib().csa_compress(C.byref(p), _ptr(kv_tok), kv_tok.shape[1], _ptr(ctx_len),
+                              _ptr(w_s), _ptr(b_pos), _ptr(gamma), first_block, n_blocks,
+                              _ptr(kv_c), kv_c.shape[1], _ptr(idx_tok), _ptr(w_s_idx),
+                              _ptr(b_pos_idx), _ptr(idx_key), _ptr(idx_scale),
+                              _ptr(dev_status), _stream(stream)))
+
+
+def lightning_index_topk(p, Q, q_idx, q_scale, w, idx_key, idx_scale, pos_q, topk_idx,
+                         topk_cnt, scores_out=None, ws=None, dev_status=None, stream=None):
+    _check(lib().lightning_index_topk(
+        C.byref(p), Q, _ptr(q_idx), _ptr(q_scale), _ptr(w), _ptr(idx_key), _ptr(idx_scale),
+        idx_key.shape[1], _ptr(pos_q), _ptr(topk_idx), _ptr(topk_cnt), _ptr(scores_out),
+        _ptr(ws), 0 if ws is None else ws.numel() * ws.element_size(), _ptr(dev_status),
+        _stream(stream)))
+
+
+def sparse_mqa_decode(p, q, pos_q, kv_c, topk_idx, topk_cnt, kv_tok, sink, out, gamma_q=None,
+                      gamma_kv=None, lse=None, ws=None, dev_status=None, stream=None):
+    _check(lib().sparse_mqa_decode(
+        C.byref(p), _ptr(q), _ptr(pos_q), _ptr(kv_c), kv_c.shape[1], _ptr(topk_idx),
+        _ptr(topk_cnt), _ptr(kv_tok), kv_tok.shape[1], _ptr(sink), _ptr(gamma_q),
+        _ptr(gamma_kv), _ptr(out), _ptr(lse), _ptr(ws),
+        0 if ws is None else ws.numel() * ws.element_size(), _ptr(dev_status), _stream(stream)))
+
+
+def dense_mqa_decode(p, q, pos_q, kv_c, kv_tok, sink, out, gamma_q=None, gamma_kv=None,
+                     lse=None, ws=None, dev_status=None, stream=None):
+    _check(lib().dense_mqa_decode(
+        C.byref(p), _ptr(q), _ptr(pos_q), _ptr(kv_c), kv_c.shape[1], _ptr(kv_tok),
+        kv_tok.shape[1], _ptr(sink), _ptr(gamma_q), _ptr(gamma_kv), _ptr(out), _ptr(lse),
+        _ptr(ws), 0 if ws is None else ws.numel() * ws.element_size(), _ptr(dev_status),
+        _stream(stream)))
+
+
+def csa_prefill_chunk(p, P, T, kv_tok, idx_tok, w_s, b_pos, gamma, w_s_idx, b_pos_idx, kv_c,
+                      idx_key, idx_scale, q, q_idx, q_scale, w, sink, topk_idx, topk_cnt, out,
+                      gamma_q=None, gamma_kv=None, ws=None, dev_status=None, stream=None):
+    _check(lib().csa_prefill_chunk(
+        C.byref(p), P, T, _ptr(kv_tok), _ptr(idx_tok), kv_tok.shape[1], _ptr(w_s), _ptr(b_pos),
+        _ptr(gamma), _ptr(w_s_idx), _ptr(b_pos_idx), _ptr(kv_c), _ptr(idx_key), _ptr(idx_scale),
+        kv_c.shape[1], _ptr(q), _ptr(q_idx), _ptr(q_scale), _ptr(w), _ptr(sink), _ptr(gamma_q),
+        _ptr(gamma_kv), _ptr(topk_idx), _ptr(topk_cnt), _ptr(out), _ptr(ws),
+        0 if ws is None else ws.numel() * ws.element_size(), _ptr(dev_status), _stream(stream)))

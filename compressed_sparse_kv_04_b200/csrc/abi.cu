@@ -1,0 +1,493 @@
+// C ABI of libcsa.so: argument validation, workspace carving and launches.
+// Every entry point is declared and documented in include/csa.h.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+
+#include "../../include/csa.h"
+#include "kernels.h"
+
+namespace {
+
+thread_local char g_err[512] = "";
+
+csa_status fail(csa_status s, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return s;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+#define REQ_PTR(p)                                                                     \
+  do {                                                                                 \
+    if ((p) == nullptr) return fail(CSA_ERR_INVALID_ARG, "%s: %s is null", fn, #p);    \
+    if (!aligned16(p)) return fail(CSA_ERR_INVALID_ARG, "%s: %s is not 16-byte aligned", fn, #p); \
+  } while (0)
+#define OPT_PTR(p)                                                                     \
+  do {                                                                                 \
+    if ((p) != nullptr && !aligned16(p))                                               \
+      return fail(CSA_ERR_INVALID_ARG, "%s: %s is not 16-byte aligned", fn, #p);      \
+  } while (0)
+// 4-byte alignment suffices for small fp32 parameter vectors.
+#define REQ_PTR4(p)                                                                    \
+  do {                                                                                 \
+    if ((p) == nullptr) return fail(CSA_ERR_INVALID_ARG, "%s: %s is null", fn, #p);    \
+    if ((reinterpret_cast<uintptr_t>(p) & 3u) != 0)                                    \
+      return fail(CSA_ERR_INVALID_ARG, "%s: %s is not 4-byte aligned", fn, #p);       \
+  } while (0)
+#define OPT_PTR4(p)                                                                    \
+  do {                                                                                 \
+    if ((p) != nullptr && (reinterpret_cast<uintptr_t>(p) & 3u) != 0)                  \
+      return fail(CSA_ERR_INVALID_ARG, "%s: %s is not 4-byte aligned", fn, #p);       \
+  } while (0)
+
+csa_status check_common(const char* fn, const csa_params* p) {
+  if (!p) return fail(CSA_ERR_INVALID_ARG, "%s: params is null", fn);
+  if (p->B < 1) return fail(CSA_ERR_INVALID_ARG, "%s: B=%d must be >= 1", fn, p->B);
+  if (p->d != 128 && p->d != 512)
+    return fail(CSA_ERR_UNSUPPORTED_SHAPE, "%s: d=%d (supported: 128, 512)", fn, p->d);
+  if (p->m < 1 || p->m > 128)
+    return fail(CSA_ERR_UNSUPPORTED_SHAPE, "%s: m=%d (supported: 1..128)", fn, p->m);
+  if (!(p->eps > 0.f) || !std::isfinite(p->eps))
+    return fail(CSA_ERR_INVALID_ARG, "%s: eps must be finite and > 0", fn);
+  return CSA_OK;
+}
+
+csa_status check_indexer(const char* fn, const csa_params* p) {
+  if (p->D_I != 64 && p->D_I != 128)
+    return fail(CSA_ERR_UNSUPPORTED_SHAPE, "%s: D_I=%d (supported: 64, 128)", fn, p->D_I);
+  if (p->H_I < 1 || p->H_I > 64)
+    return fail(CSA_ERR_UNSUPPORTED_SHAPE, "%s: H_I=%d (supported: 1..64)", fn, p->H_I);
+  if (p->k < 1 || p->k > 2048)
+    return fail(CSA_ERR_UNSUPPORTED_SHAPE, "%s: k=%d (supported: 1..2048)", fn, p->k);
+  return CSA_OK;
+}
+
+csa_status check_attention(const char* fn, const csa_params* p) {
+  if (p->H < 1 || p->H > 128)
+    return fail(CSA_ERR_UNSUPPORTED_SHAPE, "%s: H=%d (supported: 1..128)", fn, p->H);
+  if (p->window < 0 || p->window > 1024)
+    return fail(CSA_ERR_UNSUPPORTED_SHAPE, "%s: window=%d (supported: 0..1024)", fn, p->window);
+  if (p->rope_dim < 0 || (p->rope_dim & 1) || p->rope_dim > 128 || p->rope_dim > p->d / 2)
+    return fail(CSA_ERR_UNSUPPORTED_SHAPE,
+                "%s: rope_dim=%d (supported: even, <= 128, within the upper half of d)", fn,
+                p->rope_dim);
+  if (p->softmax_scale < 0.f || !std::isfinite(p->softmax_scale))
+    return fail(CSA_ERR_INVALID_ARG, "%s: softmax_scale must be finite and >= 0", fn);
+  return CSA_OK;
+}
+
+csa_status cuda_fail(const char* fn, cudaError_t e) {
+  return fail(CSA_ERR_CUDA, "%s: %s", fn, cudaGetErrorString(e));
+}
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+size_t scores_bytes(int64_t rows, int64_t N_cap) {
+  return round_up((size_t)rows * (size_t)N_cap * sizeof(float), 256);
+}
+
+void fill_inv_freq(const csa_params* p, double* out) {
+  int half = p->rope_dim / 2;
+  for (int j = 0; j < 64; ++j) out[j] = 0.0;
+  for (int j = 0; j < half; ++j)
+    out[j] = p->rope_inv_freq ? p->rope_inv_freq[j]
+                              : std::pow(10000.0, -2.0 * j / (double)p->rope_dim);
+}
+
+float softmax_scale_of(const csa_params* p) {
+  return p->softmax_scale > 0.f ? p->softmax_scale : (float)(1.0 / std::sqrt((double)p->d));
+}
+
+int64_t max_kv_rows(const csa_params* p, csa_op op, int64_t N_cap) {
+  int64_t n = (op == CSA_OP_DENSE_MQA) ? N_cap : (int64_t)p->k;
+  return n + p->window;
+}
+
+int splits_for(const csa_params* p, csa_op op, int rows, int64_t N_cap) {
+  return csa::mqa_choose_splits(rows, max_kv_rows(p, op, N_cap), csa::device_sm_count());
+}
+
+}  // namespace
+
+extern "C" {
+
+int csa_version(void) { return 100; }
+
+const char* csa_last_error(void) { return g_err; }
+
+size_t csa_workspace_bytes(const csa_params* p, csa_op op, int Q, int64_t N_cap) {
+  const char* fn = "csa_workspace_bytes";
+  if (check_common(fn, p) != CSA_OK) return 0;
+  if (Q < 1 || N_cap < 0) {
+    fail(CSA_ERR_INVALID_ARG, "%s: Q=%d, N_cap=%lld", fn, Q, (long long)N_cap);
+    return 0;
+  }
+  switch (op) {
+    case CSA_OP_INDEX_TOPK:
+      return scores_bytes((int64_t)p->B * Q, N_cap) + 256;
+    case CSA_OP_SPARSE_MQA:
+    case CSA_OP_DENSE_MQA: {
+      int rows = p->B;
+      return csa::mqa_workspace_bytes(rows, splits_for(p, op, rows, N_cap), p->H, p->d) + 256;
+    }
+    case CSA_OP_PREFILL: {
+      int rows = Q;
+      return scores_bytes(rows, N_cap) +
+             csa::mqa_workspace_bytes(rows, splits_for(p, CSA_OP_SPARSE_MQA, rows, N_cap), p->H,
+                                      p->d) +
+             512;
+    }
+  }
+  fail(CSA_ERR_INVALID_ARG, "%s: unknown op %d", fn, (int)op);
+  return 0;
+}
+
+static csa_status compress_common(const char* fn, const csa_params* p, const void* kv_tok,
+                                  int64_t L_cap, const int64_t* ctx_len, int64_t ctx_len_value,
+                                  const float* w_s, const float* b_pos, const float* gamma,
+                                  int64_t first_block, int64_t n_blocks, void* kv_c,
+                                  int64_t N_cap, const void* idx_tok, const float* w_s_idx,
+                                  const float* b_pos_idx, uint8_t* idx_key, float* idx_scale,
+                                  int32_t* dev_status, void* stream) {
+  csa_status st = check_common(fn, p);
+  if (st != CSA_OK) return st;
+  REQ_PTR(kv_tok);
+  REQ_PTR(kv_c);
+  REQ_PTR4(w_s);
+  REQ_PTR4(b_pos);
+  OPT_PTR4(gamma);
+  OPT_PTR4(dev_status);
+  if (ctx_len) OPT_PTR(ctx_len);
+  if (L_cap < 1 || N_cap < 1)
+    return fail(CSA_ERR_INVALID_ARG, "%s: L_cap=%lld N_cap=%lld", fn, (long long)L_cap,
+                (long long)N_cap);
+  if (first_block < 0 || n_blocks < 0 || first_block + n_blocks > N_cap)
+    return fail(CSA_ERR_CAPACITY, "%s: blocks [%lld, %lld) outside N_cap=%lld", fn,
+                (long long)first_block, (long long)(first_block + n_blocks), (long long)N_cap);
+  if (idx_tok) {
+    st = check_indexer(fn, p);
+    if (st != CSA_OK) return st;
+    REQ_PTR(idx_tok);
+    REQ_PTR4(w_s_idx);
+    REQ_PTR4(b_pos_idx);
+    REQ_PTR(idx_key);
+    REQ_PTR4(idx_scale);
+  }
+  csa::CompressLaunch c{};
+  c.B = p->B;
+  c.d = p->d;
+  c.D_I = p->D_I;
+  c.m = p->m;
+  c.L_cap = L_cap;
+  c.N_cap = N_cap;
+  c.kv_tok = kv_tok;
+  c.idx_tok = idx_tok;
+  c.ctx_len = ctx_len;
+  c.ctx_len_value = ctx_len_value;
+  c.w_s = w_s;
+  c.b_pos = b_pos;
+  c.gamma = gamma;
+  c.w_s_idx = w_s_idx;
+  c.b_pos_idx = b_pos_idx;
+  c.first_block = first_block;
+  c.n_blocks = n_blocks;
+  c.kv_c = kv_c;
+  c.idx_key = idx_key;
+  c.idx_scale = idx_scale;
+  c.eps = p->eps;
+  c.status = dev_status;
+  cudaError_t e = csa::launch_compress(c, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(fn, e);
+  return CSA_OK;
+}
+
+csa_status hca_compress(const csa_params* p, const void* kv_tok, int64_t L_cap,
+                        const int64_t* ctx_len, const float* w_s, const float* b_pos,
+                        const float* gamma, int64_t first_block, int64_t n_blocks, void* kv_c,
+                        int64_t N_cap, int32_t* dev_status, void* stream) {
+  const char* fn = "hca_compress";
+  csa_status st = check_common(fn, p);
+  if (st != CSA_OK) return st;
+  REQ_PTR(ctx_len);
+  return compress_common(fn, p, kv_tok, L_cap, ctx_len, 0, w_s, b_pos, gamma, first_block,
+                         n_blocks, kv_c, N_cap, nullptr, nullptr, nullptr, nullptr, nullptr,
+                         dev_status, stream);
+}
+
+csa_status csa_compress(const csa_params* p, const void* kv_tok, int64_t L_cap,
+                        const int64_t* ctx_len, const float* w_s, const float* b_pos,
+                        const float* gamma, int64_t first_block, int64_t n_blocks, void* kv_c,
+                        int64_t N_cap, const void* idx_tok, const float* w_s_idx,
+                        const float* b_pos_idx, uint8_t* idx_key, float* idx_scale,
+                        int32_t* dev_status, void* stream) {
+  const char* fn = "csa_compress";
+  csa_status st = check_common(fn, p);
+  if (st != CSA_OK) return st;
+  REQ_PTR(ctx_len);
+  return compress_common(fn, p, kv_tok, L_cap, ctx_len, 0, w_s, b_pos, gamma, first_block,
+                         n_blocks, kv_c, N_cap, idx_tok, w_s_idx, b_pos_idx, idx_key,
+                         idx_scale, dev_status, stream);
+}
+
+static csa_status index_topk_common(const char* fn, const csa_params* p, int Q,
+                                    const uint8_t* q_idx, const float* q_scale, const float* w,
+                                    const uint8_t* idx_key, const float* idx_scale,
+                                    int64_t N_cap, const int64_t* pos_q, int64_t pos_base,
+                                    int32_t* topk_idx, int32_t* topk_cnt, float* scores,
+                                    int32_t* dev_status, cudaStream_t stream) {
+  csa::IndexLaunch a{};
+  a.B = p->B;
+  a.Q = Q;
+  a.H_I = p->H_I;
+  a.D_I = p->D_I;
+  a.m = p->m;
+  a.N_cap = N_cap;
+  a.q_idx = q_idx;
+  a.q_scale = q_scale;
+  a.w = w;
+  a.key = idx_key;
+  a.key_scale = idx_scale;
+  a.pos_q = pos_q;
+  a.pos_base = pos_base;
+  a.scores = scores;
+  a.status = dev_status;
+  a.num_sms = csa::device_sm_count();
+  cudaError_t e = csa::launch_index_scores(a, stream);
+  if (e != cudaSuccess) return cuda_fail(fn, e);
+  csa::TopkLaunch t{};
+  t.rows = p->B * Q;
+  t.Q = Q;
+  t.m = p->m;
+  t.N_cap = N_cap;
+  t.scores = scores;
+  t.pos_q = pos_q;
+  t.pos_base = pos_base;
+  t.k = p->k;
+  t.idx = topk_idx;
+  t.cnt = topk_cnt;
+  t.status = dev_status;
+  e = csa::launch_topk(t, stream);
+  if (e != cudaSuccess) return cuda_fail(fn, e);
+  return CSA_OK;
+}
+
+csa_status lightning_index_topk(const csa_params* p, int Q, const uint8_t* q_idx,
+                                const float* q_scale, const float* w, const uint8_t* idx_key,
+                                const float* idx_scale, int64_t N_cap, const int64_t* pos_q,
+                                int32_t* topk_idx, int32_t* topk_cnt, float* scores_out,
+                                void* ws, size_t ws_bytes, int32_t* dev_status, void* stream) {
+  const char* fn = "lightning_index_topk";
+  csa_status st = check_common(fn, p);
+  if (st != CSA_OK) return st;
+  st = check_indexer(fn, p);
+  if (st != CSA_OK) return st;
+  if (Q < 1) return fail(CSA_ERR_INVALID_ARG, "%s: Q=%d", fn, Q);
+  if (N_cap < 1 || N_cap > (int64_t)1 << 22)
+    return fail(CSA_ERR_UNSUPPORTED_SHAPE, "%s: N_cap=%lld (supported: 1..4194304)", fn,
+                (long long)N_cap);
+  REQ_PTR(q_idx);
+  REQ_PTR4(q_scale);
+  REQ_PTR4(w);
+  REQ_PTR(idx_key);
+  REQ_PTR4(idx_scale);
+  REQ_PTR(pos_q);
+  REQ_PTR(topk_idx);
+  REQ_PTR4(topk_cnt);
+  OPT_PTR(scores_out);
+  OPT_PTR4(dev_status);
+  if (((N_cap * p->D_I) & 15) != 0)
+    return fail(CSA_ERR_UNSUPPORTED_SHAPE, "%s: N_cap*D_I must be a multiple of 16", fn);
+  float* scores = scores_out;
+  if (!scores) {
+    size_t need = csa_workspace_bytes(p, CSA_OP_INDEX_TOPK, Q, N_cap);
+    if (!ws || ws_bytes < need)
+      return fail(CSA_ERR_WORKSPACE, "%s: workspace of %zu bytes needed, %zu given", fn, need,
+                  ws ? ws_bytes : (size_t)0);
+    if (!aligned16(ws)) return fail(CSA_ERR_INVALID_ARG, "%s: ws is not 16-byte aligned", fn);
+    scores = static_cast<float*>(ws);
+  }
+  return index_topk_common(fn, p, Q, q_idx, q_scale, w, idx_key, idx_scale, N_cap, pos_q, 0,
+                           topk_idx, topk_cnt, scores, dev_status,
+                           static_cast<cudaStream_t>(stream));
+}
+
+static csa_status mqa_common(const char* fn, const csa_params* p, csa_op op, int rows, int Q,
+                             const void* q, const int64_t* pos_q, int64_t pos_base,
+                             const void* kv_c, int64_t N_cap, const int32_t* sel_idx,
+                             const int32_t* sel_cnt, const void* kv_tok, int64_t L_cap,
+                             const float* sink, const float* gamma_q, const float* gamma_kv,
+                             void* out, float* lse, void* ws, size_t ws_bytes,
+                             int32_t* dev_status, cudaStream_t stream) {
+  int splits = splits_for(p, op, rows, N_cap);
+  size_t need = csa::mqa_workspace_bytes(rows, splits, p->H, p->d);
+  if (!ws || ws_bytes < need)
+    return fail(CSA_ERR_WORKSPACE, "%s: workspace of %zu bytes needed, %zu given", fn, need,
+                ws ? ws_bytes : (size_t)0);
+  if (!aligned16(ws)) return fail(CSA_ERR_INVALID_ARG, "%s: ws is not 16-byte aligned", fn);
+  csa::MqaLaunch a{};
+  a.B = p->B;
+  a.Q = Q;
+  a.H = p->H;
+  a.D = p->d;
+  a.m = p->m;
+  a.W = p->window;
+  a.rope_dim = p->rope_dim;
+  a.N_cap = N_cap;
+  a.L_cap = L_cap;
+  a.q = q;
+  a.pos_q = pos_q;
+  a.pos_base = pos_base;
+  a.kv_c = kv_c;
+  a.sel_idx = sel_idx;
+  a.sel_cnt = sel_cnt;
+  a.kmax = p->k;
+  a.kv_tok = kv_tok;
+  a.sink = sink;
+  a.gamma_q = gamma_q;
+  a.gamma_kv = gamma_kv;
+  a.eps = p->eps;
+  a.scale = softmax_scale_of(p);
+  fill_inv_freq(p, a.inv_freq);
+  a.out = out;
+  a.lse = lse;
+  a.splits = splits;
+  a.part_o = static_cast<float*>(ws);
+  a.part_ml = reinterpret_cast<float*>(static_cast<char*>(ws) +
+                                       round_up((size_t)rows * splits * p->H * p->d * 4, 256));
+  a.status = dev_status;
+  cudaError_t e = csa::launch_mqa(a, stream);
+  if (e != cudaSuccess) return cuda_fail(fn, e);
+  return CSA_OK;
+}
+
+static csa_status check_mqa_args(const char* fn, const csa_params* p, const void* q,
+                                 const int64_t* pos_q, const void* kv_c, int64_t N_cap,
+                                 const void* kv_tok, int64_t L_cap, const float* sink,
+                                 const float* gamma_q, const float* gamma_kv, void* out,
+                                 float* lse, int32_t* dev_status) {
+  csa_status st = check_common(fn, p);
+  if (st != CSA_OK) return st;
+  st = check_attention(fn, p);
+  if (st != CSA_OK) return st;
+  REQ_PTR(q);
+  REQ_PTR(pos_q);
+  REQ_PTR(kv_c);
+  REQ_PTR(kv_tok);
+  REQ_PTR4(sink);
+  OPT_PTR4(gamma_q);
+  OPT_PTR4(gamma_kv);
+  REQ_PTR(out);
+  OPT_PTR4(lse);
+  OPT_PTR4(dev_status);
+  if (N_cap < 1 || L_cap < 1 || N_cap > ((int64_t)1 << 31) - 1 || L_cap > ((int64_t)1 << 31) - 1)
+    return fail(CSA_ERR_INVALID_ARG, "%s: N_cap=%lld L_cap=%lld", fn, (long long)N_cap,
+                (long long)L_cap);
+  if ((int64_t)p->B * N_cap > ((int64_t)1 << 31) - 1 || (int64_t)p->B * L_cap > ((int64_t)1 << 31) - 1)
+    return fail(CSA_ERR_UNSUPPORTED_SHAPE, "%s: B*N_cap and B*L_cap must fit in int32 rows", fn);
+  return CSA_OK;
+}
+
+csa_status sparse_mqa_decode(const csa_params* p, const void* q, const int64_t* pos_q,
+                             const void* kv_c, int64_t N_cap, const int32_t* topk_idx,
+                             const int32_t* topk_cnt, const void* kv_tok, int64_t L_cap,
+                             const float* sink, const float* gamma_q, const float* gamma_kv,
+                             void* out, float* lse, void* ws, size_t ws_bytes,
+                             int32_t* dev_status, void* stream) {
+  const char* fn = "sparse_mqa_decode";
+  csa_status st = check_mqa_args(fn, p, q, pos_q, kv_c, N_cap, kv_tok, L_cap, sink, gamma_q,
+                                 gamma_kv, out, lse, dev_status);
+  if (st != CSA_OK) return st;
+  if (p->k < 1 || p->k > 2048)
+    return fail(CSA_ERR_UNSUPPORTED_SHAPE, "%s: k=%d (supported: 1..2048)", fn, p->k);
+  REQ_PTR(topk_idx);
+  REQ_PTR4(topk_cnt);
+  return mqa_common(fn, p, CSA_OP_SPARSE_MQA, p->B, 1, q, pos_q, 0, kv_c, N_cap, topk_idx,
+                    topk_cnt, kv_tok, L_cap, sink, gamma_q, gamma_kv, out, lse, ws, ws_bytes,
+                    dev_status, static_cast<cudaStream_t>(stream));
+}
+
+csa_status dense_mqa_decode(const csa_params* p, const void* q, const int64_t* pos_q,
+                            const void* kv_c, int64_t N_cap, const void* kv_tok, int64_t L_cap,
+                            const float* sink, const float* gamma_q, const float* gamma_kv,
+                            void* out, float* lse, void* ws, size_t ws_bytes,
+                            int32_t* dev_status, void* stream) {
+  const char* fn = "dense_mqa_decode";
+  csa_status st = check_mqa_args(fn, p, q, pos_q, kv_c, N_cap, kv_tok, L_cap, sink, gamma_q,
+                                 gamma_kv, out, lse, dev_status);
+  if (st != CSA_OK) return st;
+  return mqa_common(fn, p, CSA_OP_DENSE_MQA, p->B, 1, q, pos_q, 0, kv_c, N_cap, nullptr,
+                    nullptr, kv_tok, L_cap, sink, gamma_q, gamma_kv, out, lse, ws, ws_bytes,
+                    dev_status, static_cast<cudaStream_t>(stream));
+}
+
+csa_status csa_prefill_chunk(const csa_params* p, int64_t P, int T, const void* kv_tok,
+                             const void* idx_tok, int64_t L_cap, const float* w_s,
+                             const float* b_pos, const float* gamma, const float* w_s_idx,
+                             const float* b_pos_idx, void* kv_c, uint8_t* idx_key,
+                             float* idx_scale, int64_t N_cap, const void* q,
+                             const uint8_t* q_idx, const float* q_scale, const float* w,
+                             const float* sink, const float* gamma_q, const float* gamma_kv,
+                             int32_t* topk_idx, int32_t* topk_cnt, void* out, void* ws,
+                             size_t ws_bytes, int32_t* dev_status, void* stream) {
+  const char* fn = "csa_prefill_chunk";
+  csa_status st = check_common(fn, p);
+  if (st != CSA_OK) return st;
+  if (p->B != 1) return fail(CSA_ERR_UNSUPPORTED_SHAPE, "%s: B=%d (supported: 1)", fn, p->B);
+  st = check_indexer(fn, p);
+  if (st != CSA_OK) return st;
+  st = check_attention(fn, p);
+  if (st != CSA_OK) return st;
+  if (P < 0 || T < 1 || P % p->m != 0)
+    return fail(CSA_ERR_INVALID_ARG, "%s: P=%lld must be a multiple of m=%d, T=%d >= 1", fn,
+                (long long)P, p->m, T);
+  if (P + T > L_cap)
+    return fail(CSA_ERR_CAPACITY, "%s: P+T=%lld exceeds L_cap=%lld", fn, (long long)(P + T),
+                (long long)L_cap);
+  int64_t nblk_total = (P + T + p->m - 1) / p->m;
+  if (nblk_total > N_cap)
+    return fail(CSA_ERR_CAPACITY, "%s: %lld compressed entries exceed N_cap=%lld", fn,
+                (long long)nblk_total, (long long)N_cap);
+  REQ_PTR(q);
+  REQ_PTR(q_idx);
+  REQ_PTR4(q_scale);
+  REQ_PTR4(w);
+  REQ_PTR4(sink);
+  REQ_PTR(topk_idx);
+  REQ_PTR4(topk_cnt);
+  REQ_PTR(out);
+  REQ_PTR(kv_c);
+  REQ_PTR(kv_tok);
+  if (((N_cap * p->D_I) & 15) != 0)
+    return fail(CSA_ERR_UNSUPPORTED_SHAPE, "%s: N_cap*D_I must be a multiple of 16", fn);
+  size_t need = csa_workspace_bytes(p, CSA_OP_PREFILL, T, N_cap);
+  if (!ws || ws_bytes < need)
+    return fail(CSA_ERR_WORKSPACE, "%s: workspace of %zu bytes needed, %zu given", fn, need,
+                ws ? ws_bytes : (size_t)0);
+  if (!aligned16(ws)) return fail(CSA_ERR_INVALID_ARG, "%s: ws is not 16-byte aligned", fn);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // 1. Compress the blocks the new tokens touch.
+  int64_t b0 = P / p->m;
+  st = compress_common(fn, p, kv_tok, L_cap, nullptr, P + T, w_s, b_pos, gamma, b0,
+                       nblk_total - b0, kv_c, N_cap, idx_tok, w_s_idx, b_pos_idx, idx_key,
+                       idx_scale, dev_status, stream);
+  if (st != CSA_OK) return st;
+  // 2-3. Causal indexer and top-k for the T queries at positions P .. P+T-1.
+  float* scores = static_cast<float*>(ws);
+  csa_params p1 = *p;
+  st = index_topk_common(fn, &p1, T, q_idx, q_scale, w, idx_key, idx_scale, N_cap, nullptr, P,
+                         topk_idx, topk_cnt, scores, dev_status, s);
+  if (st != CSA_OK) return st;
+  // 4. Sparse MQA per query, each with its own causal window.
+  char* rest = static_cast<char*>(ws) + scores_bytes(T, N_cap);
+  size_t rest_bytes = ws_bytes - scores_bytes(T, N_cap);
+  return mqa_common(fn, p, CSA_OP_SPARSE_MQA, T, T, q, nullptr, P, kv_c, N_cap, topk_idx,
+                    topk_cnt, kv_tok, L_cap, sink, gamma_q, gamma_kv, out, nullptr, rest,
+                    rest_bytes, dev_status, s);
+}
+
+}  // extern "C"

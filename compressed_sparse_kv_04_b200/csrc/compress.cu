@@ -1,0 +1,310 @@
+// KV compression (CSA m=4, HCA m'=128): learned softmax pooling of each
+// block of m token vectors, RMSNorm, bf16 storage; for the indexer-key
+// stream, E4M3 row quantisation with one fp32 scale per row.
+//
+// "DeepSeek V4 technical report" (agentupdate.ai), hybrid attention: CSA step
+// 1 (m tokens merged with learned attention-like weights) and the HCA
+// paragraph (m' = 128, no overlap); "DeepSeek V4-Pro" (llm-arch-kb), "Hybrid
+// attention" CSA / HCA bullets.  Weight form (the build's reading):
+// softmax_j(c_t . w_s + b_pos[j]) over the present tokens of the block.
+//
+// Design: pure HBM streaming on CUDA cores.  A warp owns up to 16 tokens of
+// a block and keeps an online-softmax accumulator of the block row in
+// registers (16 fp32 per lane at d = 512); token rows are read with 16-byte
+// coalesced loads, four rows in flight per warp.  m <= 16: one warp per
+// block, 8 blocks per 256-thread CTA.  m > 16: 8 warps per block, merged
+// through shared memory.  Both streams of csa_compress run in one launch
+// (blockIdx.y selects the stream).
+#include "common.cuh"
+#include "kernels.h"
+
+namespace csa {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+
+struct StreamArgs {
+  const __nv_bfloat16* tok;  // [B, L_cap, dim]
+  const float* w_s;          // [dim]
+  const float* b_pos;        // [m]
+  const float* gamma;        // [dim] or null
+  __nv_bfloat16* out_bf16;   // [B, N_cap, dim] or null
+  uint8_t* out_e4m3;         // [B, N_cap, dim] or null
+  float* out_scale;          // [B, N_cap] (with out_e4m3)
+  int dim;
+};
+
+struct PoolArgs {
+  StreamArgs s[2];
+  int nstreams;
+  int B, m;
+  int64_t L_cap, N_cap;
+  const int64_t* ctx_len;  // [B] device, or null -> ctx_len_value
+  int64_t ctx_len_value;
+  int64_t first_block, n_blocks;
+  float eps;
+  int32_t* status;
+};
+
+// Lane l holds elements  part * (32 * VEC) + l * VEC + v,  v < VEC.
+template <int DIM>
+struct Lane {
+  static constexpr int E = DIM / 32;
+  static constexpr int VEC = E < 8 ? E : 8;
+  static constexpr int NPART = E / VEC;
+  CSA_DEV static int elem(int lane, int part, int v) { return part * (32 * VEC) + lane * VEC + v; }
+};
+
+template <int DIM>
+CSA_DEV void load_row(const __nv_bfloat16* row, int lane, float (&x)[DIM / 32]) {
+  using LN = Lane<DIM>;
+#pragma unroll
+  for (int p = 0; p < LN::NPART; ++p) {
+    const __nv_bfloat16* src = row + LN::elem(lane, p, 0);
+    if constexpr (LN::VEC == 8) {
+      uint4 u = __ldg(reinterpret_cast<const uint4*>(src));
+      uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        x[p * 8 + 2 * q] = bf16_lo(w[q]);
+        x[p * 8 + 2 * q + 1] = bf16_hi(w[q]);
+      }
+    } else if constexpr (LN::VEC == 4) {
+      uint2 u = __ldg(reinterpret_cast<const uint2*>(src));
+      x[p * 4 + 0] = bf16_lo(u.x);
+      x[p * 4 + 1] = bf16_hi(u.x);
+      x[p * 4 + 2] = bf16_lo(u.y);
+      x[p * 4 + 3] = bf16_hi(u.y);
+    } else {
+      uint32_t u = __ldg(reinterpret_cast<const uint32_t*>(src));
+      x[p * 2 + 0] = bf16_lo(u);
+      x[p * 2 + 1] = bf16_hi(u);
+    }
+  }
+}
+
+// Online-softmax pooling of tokens [j0, j1) of one block by one warp.
+template <int DIM>
+CSA_DEV void pool_tokens(const __nv_bfloat16* blk, int j0, int j1, int lane,
+                         const float (&ws)[DIM / 32], const float* b_pos, float& mx, float& l,
+                         float (&acc)[DIM / 32]) {
+  constexpr int E = DIM / 32;
+  mx = -INFINITY;
+  l = 0.f;
+#pragma unroll
+  for (int e = 0; e < E; ++e) acc[e] = 0.f;
+  for (int j = j0; j < j1; j += 4) {
+    float x[4][E];
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      if (j + u < j1) load_row<DIM>(blk + (int64_t)(j + u) * DIM, lane, x[u]);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      if (j + u >= j1) break;
+      float dot = 0.f;
+#pragma unroll
+      for (int e = 0; e < E; ++e) dot = fmaf(x[u][e], ws[e], dot);
+      float s = warp_sum(dot) + __ldg(b_pos + j + u);
+      float mn = fmaxf(mx, s);
+      float corr = __expf(mx - mn);
+      float p = __expf(s - mn);
+      l = l * corr + p;
+#pragma unroll
+      for (int e = 0; e < E; ++e) acc[e] = fmaf(acc[e], corr, p * x[u][e]);
+      mx = mn;
+    }
+  }
+}
+
+template <int DIM>
+CSA_DEV void finish_row(const StreamArgs& sa, int64_t row, int lane, float (&p)[DIM / 32],
+                        float eps) {
+  using LN = Lane<DIM>;
+  constexpr int E = DIM / 32;
+  float ss = 0.f;
+#pragma unroll
+  for (int e = 0; e < E; ++e) ss = fmaf(p[e], p[e], ss);
+  ss = warp_sum(ss);
+  float inv = 1.0f / sqrtf(ss / (float)DIM + eps);
+#pragma unroll
+  for (int part = 0; part < LN::NPART; ++part)
+#pragma unroll
+    for (int v = 0; v < LN::VEC; ++v) {
+      int e = part * LN::VEC + v;
+      float g = sa.gamma ? __ldg(sa.gamma + LN::elem(lane, part, v)) : 1.f;
+      p[e] = p[e] * inv * g;
+    }
+  if (sa.out_bf16) {
+    __nv_bfloat16* dst = sa.out_bf16 + row * DIM;
+#pragma unroll
+    for (int part = 0; part < LN::NPART; ++part) {
+      uint32_t w[LN::VEC / 2];
+#pragma unroll
+      for (int q = 0; q < LN::VEC / 2; ++q)
+        w[q] = pack_bf16(p[part * LN::VEC + 2 * q], p[part * LN::VEC + 2 * q + 1]);
+      __nv_bfloat16* d = dst + LN::elem(lane, part, 0);
+      if constexpr (LN::VEC == 8)
+        *reinterpret_cast<uint4*>(d) = make_uint4(w[0], w[1], w[2], w[3]);
+      else if constexpr (LN::VEC == 4)
+        *reinterpret_cast<uint2*>(d) = make_uint2(w[0], w[1]);
+      else
+        *reinterpret_cast<uint32_t*>(d) = w[0];
+    }
+  }
+  if (sa.out_e4m3) {
+    float amax = 0.f;
+#pragma unroll
+    for (int e = 0; e < E; ++e) amax = fmaxf(amax, fabsf(p[e]));
+    amax = warp_max(amax);
+    float scale = amax > 0.f ? __fdiv_rn(amax, 448.0f) : 1.0f;
+    uint8_t* dst = sa.out_e4m3 + row * DIM;
+#pragma unroll
+    for (int part = 0; part < LN::NPART; ++part) {
+      uint8_t codes[LN::VEC];
+#pragma unroll
+      for (int v = 0; v < LN::VEC; v += 2) {
+        float2 f = make_float2(__fdiv_rn(p[part * LN::VEC + v], scale),
+                               __fdiv_rn(p[part * LN::VEC + v + 1], scale));
+        __nv_fp8x2_storage_t c2 = __nv_cvt_float2_to_fp8x2(f, __NV_SATFINITE, __NV_E4M3);
+        codes[v] = (uint8_t)(c2 & 0xFF);
+        codes[v + 1] = (uint8_t)(c2 >> 8);
+      }
+      uint8_t* d = dst + LN::elem(lane, part, 0);
+      if constexpr (LN::VEC == 8) {
+        uint2 w;
+        w.x = codes[0] | (codes[1] << 8) | (codes[2] << 16) | ((uint32_t)codes[3] << 24);
+        w.y = codes[4] | (codes[5] << 8) | (codes[6] << 16) | ((uint32_t)codes[7] << 24);
+        *reinterpret_cast<uint2*>(d) = w;
+      } else if constexpr (LN::VEC == 4) {
+        *reinterpret_cast<uint32_t*>(d) =
+            codes[0] | (codes[1] << 8) | (codes[2] << 16) | ((uint32_t)codes[3] << 24);
+      } else {
+        *reinterpret_cast<uint16_t*>(d) = (uint16_t)(codes[0] | (codes[1] << 8));
+      }
+    }
+    if (lane == 0) sa.out_scale[row] = scale;
+  }
+}
+
+template <int DIM>
+CSA_DEV void pool_stream(const PoolArgs& a, const StreamArgs& sa, float* smem) {
+  constexpr int E = DIM / 32;
+  using LN = Lane<DIM>;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int G = a.m <= 16 ? 1 : kWarps;           // warps per block
+  const int per_cta = kWarps / G;                  // blocks per CTA
+  const int64_t unit = (int64_t)blockIdx.x * per_cta + warp / G;  // (b, block) pair
+  const int64_t total = (int64_t)a.B * a.n_blocks;
+  const bool active = unit < total;
+  int64_t b = 0, i = 0;
+  int present = 0;
+  if (active) {
+    b = unit / a.n_blocks;
+    i = a.first_block + unit % a.n_blocks;
+    int64_t L = a.ctx_len ? a.ctx_len[b] : a.ctx_len_value;
+    if (L > a.L_cap) L = a.L_cap;
+    int64_t rem = L - i * a.m;
+    present = rem <= 0 ? 0 : (rem < a.m ? (int)rem : a.m);
+  }
+  float ws[E];
+#pragma unroll
+  for (int part = 0; part < LN::NPART; ++part)
+#pragma unroll
+    for (int v = 0; v < LN::VEC; ++v) ws[part * LN::VEC + v] = __ldg(sa.w_s + LN::elem(lane, part, v));
+
+  const __nv_bfloat16* blk = sa.tok + ((int64_t)b * a.L_cap + i * a.m) * DIM;
+  float mx, l, acc[E];
+  const int g = warp % G;
+  const int per_warp = (a.m + G - 1) / G;
+  int j0 = g * per_warp, j1 = min(present, j0 + per_warp);
+  pool_tokens<DIM>(blk, j0, j1 > j0 ? j1 : j0, lane, ws, sa.b_pos, mx, l, acc);
+
+  if (G == 1) {
+    if (!active || present == 0) return;
+#pragma unroll
+    for (int e = 0; e < E; ++e) acc[e] = acc[e] / l;
+    finish_row<DIM>(sa, b * a.N_cap + i, lane, acc, a.eps);
+    return;
+  }
+  // Merge the G warp partials of the one block of this CTA.
+  float* s_acc = smem;                 // [kWarps][DIM]
+  float* s_ml = smem + kWarps * DIM;   // [kWarps][2]
+#pragma unroll
+  for (int part = 0; part < LN::NPART; ++part)
+#pragma unroll
+    for (int v = 0; v < LN::VEC; ++v)
+      s_acc[warp * DIM + LN::elem(lane, part, v)] = acc[part * LN::VEC + v];
+  if (lane == 0) {
+    s_ml[2 * warp] = mx;
+    s_ml[2 * warp + 1] = l;
+  }
+  __syncthreads();
+  if (warp != 0 || !active || present == 0) return;
+  float M = -INFINITY;
+  for (int w = 0; w < G; ++w) M = fmaxf(M, s_ml[2 * w]);
+  float L = 0.f, p[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) p[e] = 0.f;
+  for (int w = 0; w < G; ++w) {
+    float mw = s_ml[2 * w];
+    if (mw == -INFINITY) continue;
+    float c = __expf(mw - M);
+    L = fmaf(s_ml[2 * w + 1], c, L);
+#pragma unroll
+    for (int part = 0; part < LN::NPART; ++part)
+#pragma unroll
+      for (int v = 0; v < LN::VEC; ++v)
+        p[part * LN::VEC + v] = fmaf(s_acc[w * DIM + LN::elem(lane, part, v)], c,
+                                     p[part * LN::VEC + v]);
+  }
+#pragma unroll
+  for (int e = 0; e < E; ++e) p[e] = p[e] / L;
+  finish_row<DIM>(sa, b * a.N_cap + i, lane, p, a.eps);
+}
+
+__global__ void __launch_bounds__(kThreads) compress_kernel(const PoolArgs a) {
+  extern __shared__ float smem[];
+  const StreamArgs& sa = a.s[blockIdx.y];
+  switch (sa.dim) {
+    case 512: pool_stream<512>(a, sa, smem); break;
+    case 128: pool_stream<128>(a, sa, smem); break;
+    case 64: pool_stream<64>(a, sa, smem); break;
+    default: report(a.status, CSA_ERR_UNSUPPORTED_SHAPE); break;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_compress(const CompressLaunch& c, cudaStream_t stream) {
+  PoolArgs a{};
+  a.nstreams = c.idx_tok ? 2 : 1;
+  a.s[0] = StreamArgs{reinterpret_cast<const __nv_bfloat16*>(c.kv_tok), c.w_s, c.b_pos, c.gamma,
+                      reinterpret_cast<__nv_bfloat16*>(c.kv_c), nullptr, nullptr, c.d};
+  if (c.idx_tok)
+    a.s[1] = StreamArgs{reinterpret_cast<const __nv_bfloat16*>(c.idx_tok), c.w_s_idx, c.b_pos_idx,
+                        nullptr, nullptr, c.idx_key, c.idx_scale, c.D_I};
+  a.B = c.B;
+  a.m = c.m;
+  a.L_cap = c.L_cap;
+  a.N_cap = c.N_cap;
+  a.ctx_len = c.ctx_len;
+  a.ctx_len_value = c.ctx_len_value;
+  a.first_block = c.first_block;
+  a.n_blocks = c.n_blocks;
+  a.eps = c.eps;
+  a.status = c.status;
+  int G = c.m <= 16 ? 1 : kWarps;
+  int per_cta = kWarps / G;
+  int64_t units = (int64_t)c.B * c.n_blocks;
+  if (units == 0) return cudaSuccess;
+  int64_t grid_x = (units + per_cta - 1) / per_cta;
+  if (grid_x > 0x7FFFFFFF) return cudaErrorInvalidConfiguration;
+  int maxdim = c.idx_tok && c.D_I > c.d ? c.D_I : c.d;
+  size_t smem = G == 1 ? 0 : (size_t)kWarps * (maxdim + 2) * sizeof(float);
+  dim3 grid((unsigned)grid_x, a.nstreams);
+  compress_kernel<<<grid, kThreads, smem, stream>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace csa

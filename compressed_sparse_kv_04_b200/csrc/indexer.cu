@@ -1,0 +1,314 @@
+// Lightning Indexer scores on the 5th-generation tensor cores.
+//
+// "DeepSeek V4 technical report" (agentupdate.ai), hybrid attention, CSA step
+// 2: a light indexer scores each query against every compressed block;
+// "DeepSeek V4-Pro" (llm-arch-kb), "Hybrid attention" CSA bullet: 64 indexer
+// heads of dim 128; "KV Cache Compression ... Visualised" (webconsulting.at),
+// "Dual Compression and Indexing": a low-precision pass.  Score form (the
+// DSA reading): score_i = sum_h w_h ReLU(q_h . k_i) on dequantised E4M3
+// values, computed as
+//     score_i = s_k[i] * sum_h (w_h s_q[h]) * ReLU(sum_d q8[h,d] k8[i,d])
+// which is the same number because every scale is >= 0.
+//
+// Design (swap-AB): A = a 128-entry tile of E4M3 keys (K-major, TMA with
+// 128B/64B swizzle), B = the G queries' H_I heads (N = G * roundup16(H_I) <=
+// 256 rows, K-major, loaded once per CTA), D = 128 entries x N in TMEM (fp32).
+// With one TMEM lane per entry, the epilogue's reduction over heads is a
+// per-thread loop over columns: no shuffles.  Warp roles: 0 = TMA producer,
+// 1 = MMA issuer, 2..5 = epilogue (TMEM -> score).  The key ring is 6-8 stages
+// deep and the accumulator is double-buffered, so loads, MMAs and the
+// epilogue of consecutive tiles overlap.  Each CTA owns one query group and
+// a contiguous range of tiles; the grid is sized to fill every SM.
+#include <algorithm>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "tma.h"
+
+namespace csa {
+namespace {
+
+constexpr int kTileRows = 128;
+constexpr int kThreads = 192;
+
+template <int DI>
+struct Cfg {
+  static constexpr int kStageBytes = kTileRows * DI;
+  static constexpr int kStages = DI == 128 ? 6 : 8;
+  static constexpr uint32_t kSBO = 8 * DI;               // 8 rows per swizzle atom
+  static constexpr uint32_t kSwzMask = DI == 128 ? 7 : 3;  // 128B / 64B swizzle
+  static constexpr uint64_t kLayout = DI == 128 ? 2 : 4;   // descriptor layout type
+};
+
+struct Params {
+  int B, Q, H_I, HP, G, N, m;
+  int64_t N_cap;
+  int tiles_per_chunk, ntiles, qgroups;
+  const uint8_t* q_idx;
+  const float* q_scale;
+  const float* w;
+  const float* key_scale;
+  const int64_t* pos_q;
+  int64_t pos_base;
+  float* scores;
+  int32_t* status;
+  uint32_t tmem_cols;
+};
+
+template <int DI>
+CSA_DEV uint64_t desc_kmajor(uint32_t saddr) {
+  uint64_t d = sdesc_sw128(saddr, 16, Cfg<DI>::kSBO);
+  d &= ~(7ull << 61);
+  d |= Cfg<DI>::kLayout << 61;
+  return d;
+}
+
+template <int DI>
+__global__ void __launch_bounds__(kThreads, 1)
+    index_score_kernel(const __grid_constant__ CUtensorMap kmap, const Params p) {
+  using C = Cfg<DI>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* ring = smem;                                      // kStages x kStageBytes
+  uint8_t* qtile = ring + C::kStages * C::kStageBytes;       // N x DI
+  float* wq = reinterpret_cast<float*>(qtile + p.N * DI);    // N
+  uint64_t* bars = reinterpret_cast<uint64_t*>(wq + 256);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + C::kStages;
+  uint64_t* tfull = empty + C::kStages;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_slot + 1);
+  int* consumed = const_cast<int*>(abort_flag + 1);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int group = blockIdx.y;
+  const int b = group / p.qgroups;
+  const int q0 = (group % p.qgroups) * p.G;
+  const int nq = min(p.G, p.Q - q0);
+
+  // Visible entries per query of the group (causal), clamped to capacity.
+  int64_t nv_max = 0;
+  for (int g = 0; g < nq; ++g) {
+    int64_t pos = p.pos_q ? p.pos_q[(int64_t)b * p.Q + q0 + g] : p.pos_base + q0 + g;
+    int64_t nv = pos < 0 ? 0 : (pos + 1) / p.m;
+    if (nv > p.N_cap) nv = p.N_cap;
+    nv_max = max(nv_max, nv);
+  }
+  const int t_begin = blockIdx.x * p.tiles_per_chunk;
+  const int t_vis = (int)((nv_max + kTileRows - 1) / kTileRows);
+  const int t_end = min(min(t_begin + p.tiles_per_chunk, p.ntiles), t_vis);
+  if (t_begin >= t_end) return;  // uniform over the CTA
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 128);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    *consumed = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_base_slot, p.tmem_cols);
+    tmem_relinquish();
+  }
+  // Query tile (B operand): row g*HP + h holds head h of query q0+g; rows of
+  // padding heads / absent queries are zero.  Written with the swizzle the
+  // MMA descriptor expects.
+  for (int c = threadIdx.x; c < p.N * (DI / 16); c += kThreads) {
+    int row = c / (DI / 16), chunk = c % (DI / 16);
+    int g = row / p.HP, h = row % p.HP;
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (g < nq && h < p.H_I)
+      v = __ldg(reinterpret_cast<const uint4*>(
+          p.q_idx + (((int64_t)b * p.Q + q0 + g) * p.H_I + h) * DI + chunk * 16));
+    uint32_t lin = row * DI + chunk * 16;
+    uint32_t phys = lin ^ (((lin >> 7) & C::kSwzMask) << 4);
+    *reinterpret_cast<uint4*>(qtile + phys) = v;
+  }
+  for (int r = threadIdx.x; r < p.N; r += kThreads) {
+    int g = r / p.HP, h = r % p.HP;
+    float v = 0.f;
+    if (g < nq && h < p.H_I) {
+      int64_t o = ((int64_t)b * p.Q + q0 + g) * p.H_I + h;
+      v = __ldg(p.w + o) * __ldg(p.q_scale + o);
+    }
+    wq[r] = v;
+  }
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_base_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------- TMA producer --
+    if (elect_one()) {
+      tma_prefetch_desc(&kmap);
+      int it = 0;
+      for (int t = t_begin; t < t_end; ++t, ++it) {
+        int s = it % C::kStages;
+        uint32_t ph = (it / C::kStages) & 1;
+        if (!mbar_wait(&empty[s], ph ^ 1, p.status, abort_flag)) break;
+        mbar_expect_tx(&full[s], C::kStageBytes);
+        tma_load_2d(ring + s * C::kStageBytes, &kmap, &full[s], 0,
+                    (int32_t)((int64_t)b * p.N_cap + (int64_t)t * kTileRows));
+      }
+      // On abort, wait for the copies still in flight before the CTA exits.
+      if (*abort_flag) {
+        int issued = it;
+        for (int j = max(0, issued - C::kStages); j < issued; ++j)
+          mbar_wait(&full[j % C::kStages], (j / C::kStages) & 1, p.status);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------- MMA issuer --
+    if (elect_one()) {
+      const uint32_t idesc = idesc_e4m3(128, p.N);
+      const uint32_t q_addr = smem_u32(qtile);
+      int it = 0;
+      bool issued_any = false;
+      for (int t = t_begin; t < t_end; ++t, ++it) {
+        int s = it % C::kStages;
+        uint32_t ph = (it / C::kStages) & 1;
+        if (!mbar_wait(&full[s], ph, p.status, abort_flag)) break;
+        int a = it & 1;
+        uint32_t aph = (it >> 1) & 1;
+        if (!mbar_wait(&tempty[a], aph ^ 1, p.status, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t a_addr = smem_u32(ring + s * C::kStageBytes);
+#pragma unroll
+        for (int k = 0; k < DI / 32; ++k)
+          mma_e4m3_ss(tmem + a * p.N, desc_kmajor<DI>(a_addr + k * 32),
+                      desc_kmajor<DI>(q_addr + k * 32), idesc, k > 0 ? 1u : 0u);
+        mma_commit(&empty[s]);
+        mma_commit(&tfull[a]);
+        issued_any = true;
+      }
+      if (*abort_flag && issued_any) {
+        mma_commit(drain);
+        mbar_wait(drain, 0, p.status);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue --
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    int64_t nv[8];
+#pragma unroll
+    for (int g = 0; g < 8; ++g) nv[g] = 0;
+    for (int g = 0; g < nq && g < 8; ++g) {
+      int64_t pos = p.pos_q ? p.pos_q[(int64_t)b * p.Q + q0 + g] : p.pos_base + q0 + g;
+      int64_t v = pos < 0 ? 0 : (pos + 1) / p.m;
+      if (v > p.N_cap) {
+        v = p.N_cap;
+        if (row == 0 && t_begin == 0) report(p.status, CSA_ERR_CAPACITY);
+      }
+      nv[g] = v;
+    }
+    int it = 0;
+    for (int t = t_begin; t < t_end; ++t, ++it) {
+      int a = it & 1;
+      uint32_t aph = (it >> 1) & 1;
+      bool ok = mbar_wait(&tfull[a], aph, p.status, abort_flag);
+      if (!__all_sync(0xffffffffu, ok)) break;  // keep the warp converged for tcgen05.ld
+      tc_fence_after();
+      const int64_t entry = (int64_t)t * kTileRows + row;
+      const float ks = entry < p.N_cap ? __ldg(p.key_scale + (int64_t)b * p.N_cap + entry) : 0.f;
+      for (int g = 0; g < nq; ++g) {
+        float acc = 0.f;
+        for (int c = 0; c < p.HP; c += 16) {
+          uint32_t v[16];
+          tmem_ld16(tmem_addr(tmem, quarter * 32, a * p.N + g * p.HP + c), v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            acc = fmaf(wq[g * p.HP + c + j], fmaxf(__uint_as_float(v[j]), 0.f), acc);
+        }
+        if (entry < nv[g < 8 ? g : 7])
+          p.scores[((int64_t)b * p.Q + q0 + g) * p.N_cap + entry] = acc * ks;
+      }
+      tc_fence_before();
+      mbar_arrive(&tempty[a]);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, p.tmem_cols);
+  }
+}
+
+template <int DI>
+cudaError_t launch_impl(const IndexLaunch& a, cudaStream_t stream) {
+  using C = Cfg<DI>;
+  Params p{};
+  p.B = a.B;
+  p.Q = a.Q;
+  p.H_I = a.H_I;
+  p.HP = (a.H_I + 15) / 16 * 16;
+  p.G = std::max(1, std::min(std::min(a.Q, 256 / p.HP), 8));
+  p.N = p.G * p.HP;
+  p.m = a.m;
+  p.N_cap = a.N_cap;
+  p.ntiles = (int)((a.N_cap + kTileRows - 1) / kTileRows);
+  p.qgroups = (a.Q + p.G - 1) / p.G;
+  p.q_idx = a.q_idx;
+  p.q_scale = a.q_scale;
+  p.w = a.w;
+  p.key_scale = a.key_scale;
+  p.pos_q = a.pos_q;
+  p.pos_base = a.pos_base;
+  p.scores = a.scores;
+  p.status = a.status;
+  uint32_t cols = 32;
+  while (cols < (uint32_t)(2 * p.N)) cols <<= 1;
+  p.tmem_cols = cols;
+
+  size_t smem = 1024 + (size_t)C::kStages * C::kStageBytes + (size_t)p.N * DI + 256 * 4 +
+                (2 * C::kStages + 5) * 8 + 16;
+  auto kern = index_score_kernel<DI>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
+  if (e != cudaSuccess) return e;
+  int occ = 1;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kThreads, smem);
+  if (e != cudaSuccess) return e;
+  occ = std::max(1, std::min(occ, 2));
+  if (2 * cols > 512) occ = 1;  // two CTAs would contend for tensor memory
+  int64_t groups = (int64_t)a.B * p.qgroups;
+  if (groups > 65535) return cudaErrorInvalidConfiguration;
+  int64_t slots = (int64_t)a.num_sms * occ;
+  int chunks = 1;
+  if (groups < slots) chunks = (int)std::max<int64_t>(1, std::min<int64_t>(p.ntiles, slots / groups));
+  p.tiles_per_chunk = (p.ntiles + chunks - 1) / chunks;
+  chunks = (p.ntiles + p.tiles_per_chunk - 1) / p.tiles_per_chunk;
+
+  CUtensorMap kmap;
+  e = make_tmap_2d(&kmap, a.key, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)a.B * a.N_cap, DI,
+                   kTileRows, DI, DI == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B);
+  if (e != cudaSuccess) return e;
+  dim3 grid(chunks, (unsigned)groups);
+  kern<<<grid, kThreads, smem, stream>>>(kmap, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_index_scores(const IndexLaunch& a, cudaStream_t stream) {
+  if (a.B * (int64_t)a.N_cap > 0x7FFFFFFF) return cudaErrorInvalidValue;
+  if (a.D_I == 128) return launch_impl<128>(a, stream);
+  if (a.D_I == 64) return launch_impl<64>(a, stream);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace csa

@@ -1,0 +1,93 @@
+// Internal launch interface between the C ABI (abi.cu) and the kernels.
+// Host-side only types: plain pointers and sizes.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace csa {
+
+struct CompressLaunch {
+  int B, d, D_I, m;
+  int64_t L_cap, N_cap;
+  const void* kv_tok;
+  const void* idx_tok;  // null: KV stream only
+  const int64_t* ctx_len;
+  int64_t ctx_len_value;  // used when ctx_len is null
+  const float *w_s, *b_pos, *gamma, *w_s_idx, *b_pos_idx;
+  int64_t first_block, n_blocks;
+  void* kv_c;
+  uint8_t* idx_key;
+  float* idx_scale;
+  float eps;
+  int32_t* status;
+};
+cudaError_t launch_compress(const CompressLaunch& c, cudaStream_t stream);
+
+// Lightning Indexer scores (tcgen05 kind::f8f6f4) over every (query, entry
+// tile).  Queries are grouped G per MMA (N = G * H_I <= 256).
+struct IndexLaunch {
+  int B, Q, H_I, D_I, m;
+  int64_t N_cap;
+  const uint8_t* q_idx;     // [B, Q, H_I, D_I]
+  const float* q_scale;     // [B, Q, H_I]
+  const float* w;           // [B, Q, H_I]
+  const uint8_t* key;       // [B, N_cap, D_I]
+  const float* key_scale;   // [B, N_cap]
+  const int64_t* pos_q;     // [B, Q] or null -> pos_base + q
+  int64_t pos_base;
+  float* scores;            // [B, Q, N_cap]
+  int32_t* status;
+  int num_sms;
+};
+cudaError_t launch_index_scores(const IndexLaunch& a, cudaStream_t stream);
+
+// Exact top-k over fp32 scores, one cluster of CTAs per query row.
+struct TopkLaunch {
+  int rows;                 // B * Q
+  int Q, m;
+  int64_t N_cap;
+  const float* scores;      // [rows, N_cap]
+  const int64_t* pos_q;     // [rows] or null -> pos_base + (row % Q)
+  int64_t pos_base;
+  int k;
+  int32_t* idx;             // [rows, k]
+  int32_t* cnt;             // [rows]
+  int32_t* status;
+};
+cudaError_t launch_topk(const TopkLaunch& a, cudaStream_t stream);
+
+// Shared-KV MQA decode (sparse or dense) with window and sink: a pair of
+// CTAs (cluster of 2) per (query row, split), each owning half of the head
+// dim; split partials are merged by the combine kernel.
+struct MqaLaunch {
+  int B, Q, H, D, m, W, rope_dim;
+  int64_t N_cap, L_cap;
+  const void* q;            // [B*Q, H, D] bf16
+  const int64_t* pos_q;     // [B*Q] or null -> pos_base + (row % Q)
+  int64_t pos_base;
+  const void* kv_c;         // [B, N_cap, D]
+  const int32_t* sel_idx;   // [B*Q, kmax] or null (dense)
+  const int32_t* sel_cnt;   // [B*Q]
+  int kmax;
+  const void* kv_tok;       // [B, L_cap, D]
+  const float* sink;        // [H]
+  const float* gamma_q;     // [D] or null
+  const float* gamma_kv;    // [D] or null
+  float eps, scale;
+  double inv_freq[64];      // rope_dim/2 entries
+  void* out;                // [B*Q, H, D] bf16
+  float* lse;               // [B*Q, H] or null
+  float* part_o;            // workspace [rows, S, H, D] fp32
+  float* part_ml;           // workspace [rows, S, 2, H] fp32
+  int splits;               // S
+  int32_t* status;
+};
+size_t mqa_workspace_bytes(int rows, int splits, int H, int D);
+int mqa_choose_splits(int rows, int64_t max_kv, int num_sms);
+cudaError_t launch_mqa(const MqaLaunch& a, cudaStream_t stream);
+
+int device_sm_count();
+
+}  // namespace csa

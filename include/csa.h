@@ -1,0 +1,242 @@
+/*
+ * csa.h - C ABI of libcsa.so, the B200 (sm_100a) DeepSeek-V4 hybrid-attention
+ * hot path: Compressed Sparse Attention (CSA) and Heavily Compressed
+ * Attention (HCA).
+ *
+ * Sources, cited by page title and section:
+ *   [P2] "DeepSeek V4 technical report" (agentupdate.ai, Chinese), hybrid
+ *        attention section: CSA steps 1 (KV compression), 2 (Lightning
+ *        Indexer + top-k), 3 (core multi-query attention); HCA paragraph.
+ *   [P3] "DeepSeek V4-Pro Architecture: KV Cache Compression and
+ *        Hyper-Connections Visualised" (webconsulting.at), "Key points" and
+ *        "Dual Compression and Indexing".
+ *   [P5] "DeepSeek V4-Pro" (lizeman.github.io llm-arch-kb), "What's new in
+ *        V4 / 1. Hybrid attention: CSA + HCA replace MLA".
+ *
+ * Conventions shared by every entry point
+ *   - Tensor pointers are DEVICE pointers owned by the caller (the binding
+ *     allocates them with PyTorch).  The library never allocates or frees
+ *     device memory; scratch comes from a caller-provided workspace whose
+ *     size csa_workspace_bytes() reports.  Host pointers are marked "host".
+ *   - Every tensor is dense, row-major, in the layout written beside it, and
+ *     its base address is 16-byte aligned (CSA_ERR_INVALID_ARG otherwise).
+ *   - bf16 tensors are passed as void* holding IEEE bfloat16 values; E4M3
+ *     tensors as uint8_t* holding OCP FP8 E4M3 ("fn") codes.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Calls only enqueue work; they are stream-ordered, keep no
+ *     state between calls and may be captured into a CUDA graph.
+ *   - Argument checks are synchronous and return an error before anything
+ *     is enqueued.  A failed launch returns CSA_ERR_CUDA.  csa_last_error()
+ *     returns a thread-local message for the last failure on that thread.
+ *   - `dev_status` (optional, device int32) receives the first error a
+ *     kernel detects on the device (an index outside the buffers it was
+ *     given, a visible-entry count above the capacity, a bounded wait that
+ *     gave up).  The offending access is skipped; nothing traps.  The caller
+ *     reads and clears it.
+ *   - No exceptions cross the ABI and there is no CPU fallback.
+ */
+#ifndef CSA_H_
+#define CSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  CSA_OK = 0,
+  CSA_ERR_INVALID_ARG = 1,       /* null/misaligned pointer, negative size, ... */
+  CSA_ERR_UNSUPPORTED_SHAPE = 2, /* a size outside the supported set below */
+  CSA_ERR_CAPACITY = 3,          /* a range that does not fit the given capacity */
+  CSA_ERR_WORKSPACE = 4,         /* workspace missing or smaller than required */
+  CSA_ERR_CUDA = 5,              /* a CUDA runtime/driver call failed */
+  CSA_ERR_DEVICE_TIMEOUT = 6,    /* (dev_status) a bounded device wait gave up */
+  CSA_ERR_DEVICE_INDEX = 7       /* (dev_status) an index outside its buffer */
+} csa_status;
+
+/* Shapes and constants shared by the calls of one layer.
+ * Supported: d in {128, 512}; 1 <= H <= 128; H_I in {1..64}, D_I in {64, 128}
+ * (indexer calls only); 1 <= k <= 2048; 0 <= window <= 1024; rope_dim even,
+ * 0 <= rope_dim <= min(d, 128); 1 <= m <= 128 (CSA uses 4, HCA 128); eps > 0. */
+typedef struct {
+  int B;               /* sequences in the batch */
+  int d;               /* KV entry dim == attention head dim D ([P5]: 512) */
+  int H;               /* query heads ([P5]: 128) */
+  int H_I;             /* Lightning-Indexer heads ([P5]: 64) */
+  int D_I;             /* Lightning-Indexer head dim ([P5]: 128) */
+  int k;               /* entries kept per query ([P5]: 1024) */
+  int window;          /* uncompressed sliding window W ([P5]: 128) */
+  int rope_dim;        /* rotated trailing dims r ([P5]: 64) */
+  int m;               /* compression ratio ([P5]: 4 for CSA, 128 for HCA) */
+  float eps;           /* RMSNorm epsilon (1e-6 in the build's tests) */
+  float softmax_scale; /* logit scale; 0 selects 1/sqrt(d) */
+  const double* rope_inv_freq; /* host, [rope_dim/2] angle per position for
+                                  pair j; NULL selects 10000^(-2j/rope_dim) */
+} csa_params;
+
+/* Operation selector for csa_workspace_bytes(). */
+typedef enum {
+  CSA_OP_INDEX_TOPK = 1,
+  CSA_OP_SPARSE_MQA = 2,
+  CSA_OP_DENSE_MQA = 3,
+  CSA_OP_PREFILL = 4
+} csa_op;
+
+/* Library version (major*100 + minor). */
+int csa_version(void);
+
+/* Thread-local message for the last non-OK status returned on this thread. */
+const char* csa_last_error(void);
+
+/* Workspace bytes that `op` needs for these params.
+ *   Q     queries per sequence (1 for decode; T for CSA_OP_PREFILL),
+ *   N_cap capacity of the compressed cache (entries per sequence).
+ * Returns 0 for invalid arguments (and sets csa_last_error). */
+size_t csa_workspace_bytes(const csa_params* p, csa_op op, int Q, int64_t N_cap);
+
+/* ---------------------------------------------------------------------------
+ * KV compression, HCA form ([P2] HCA: m' = 128, blocks do not overlap;
+ * [P3] "Dual Compression and Indexing": a learned weighted average per
+ * block; [P5] "Hybrid attention": HCA bullet).
+ *
+ * For every sequence b and block i in [first_block, first_block+n_blocks)
+ * the present tokens t = i*m + j (j < m, t < ctx_len[b]) are pooled:
+ *   s_j   = kv_tok[b,t,:] . w_s + b_pos[j]
+ *   alpha = softmax over the present j of s_j
+ *   e     = RMSNorm(sum_j alpha_j kv_tok[b,t,:]) * gamma      (eps = p->eps)
+ * and e is stored as bf16 in kv_c[b,i,:].  A block with no present token is
+ * left untouched.  (The weight form is the build's reading: the pages do
+ * not fix it.)
+ *
+ *   kv_tok  [B, L_cap, d] bf16 (device)     token KV stream
+ *   ctx_len [B] int64 (device)              tokens present per sequence
+ *   w_s [d], b_pos [m], gamma [d] or NULL (ones)   fp32 (device)
+ *   kv_c    [B, N_cap, d] bf16 (device)     compressed cache (written)
+ * Errors: CSA_ERR_CAPACITY if first_block < 0 or first_block + n_blocks > N_cap
+ *         (checked on the host); tokens at or beyond L_cap are never read.
+ * ------------------------------------------------------------------------- */
+csa_status hca_compress(const csa_params* p, const void* kv_tok, int64_t L_cap,
+                        const int64_t* ctx_len, const float* w_s, const float* b_pos,
+                        const float* gamma, int64_t first_block, int64_t n_blocks,
+                        void* kv_c, int64_t N_cap, int32_t* dev_status, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * KV compression, CSA form ([P2] CSA step 1; [P5] CSA bullet: m = 4).
+ * The KV stream is pooled exactly as hca_compress does.  When idx_tok is not
+ * NULL, the indexer-key stream idx_tok [B, L_cap, D_I] bf16 is pooled by the
+ * same operation with its own w_s_idx [D_I] and b_pos_idx [m] (no gain),
+ * and each pooled row x is stored in E4M3 ([P3]: the indexer is low
+ * precision): scale = max|x| / 448 in binary32 (1 when the row is zero),
+ * code = E4M3 round-to-nearest-even, saturating, of x / scale.
+ *   idx_key   [B, N_cap, D_I] uint8 E4M3 codes (written)
+ *   idx_scale [B, N_cap] fp32 (written)
+ * ------------------------------------------------------------------------- */
+csa_status csa_compress(const csa_params* p, const void* kv_tok, int64_t L_cap,
+                        const int64_t* ctx_len, const float* w_s, const float* b_pos,
+                        const float* gamma, int64_t first_block, int64_t n_blocks,
+                        void* kv_c, int64_t N_cap, const void* idx_tok,
+                        const float* w_s_idx, const float* b_pos_idx, uint8_t* idx_key,
+                        float* idx_scale, int32_t* dev_status, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Lightning Indexer + top-k ([P2] CSA step 2; [P5] CSA bullet: 64 heads of
+ * dim 128, k = 1024; [P3] "Key points": ~262,000 entries narrowed to 1,024).
+ *
+ * For every sequence b and query q (position pos_q[b,q]) the visible
+ * entries are i < n_vis = floor((pos_q+1)/m) (the block holding the query is
+ * not complete and is not visible, [P5] sliding-window bullet).  Score
+ * (reading of the DSA form the pages cite):
+ *   score_i = sum_h w[h] * ReLU( (q_idx[h,:]*q_scale[h]) . (key[i,:]*key_scale[i]) )
+ * evaluated as key_scale[i] * sum_h (w[h]*q_scale[h]) * ReLU(q_idx[h,:] . key[i,:])
+ * with E4M3 products accumulated in fp32 on the tensor cores.  The k entries
+ * with the largest score are kept (ties: lower index first; NaN lowest;
+ * -0 == +0) and written as ascending indices, padded with -1;
+ * topk_cnt = min(k, n_vis).
+ *
+ *   q_idx    [B, Q, H_I, D_I] uint8 E4M3 (device)
+ *   q_scale  [B, Q, H_I] fp32 (device, >= 0)    w [B, Q, H_I] fp32 (device)
+ *   idx_key  [B, N_cap, D_I] uint8, idx_scale [B, N_cap] fp32 (device, >= 0)
+ *   pos_q    [B, Q] int64 (device)
+ *   topk_idx [B, Q, k] int32 (written)          topk_cnt [B, Q] int32 (written)
+ *   scores_out [B, Q, N_cap] fp32 or NULL: when given, entries i < n_vis
+ *              receive the fp32 scores (others are not written).
+ * Device errors: n_vis > N_cap -> CSA_ERR_CAPACITY in dev_status, clamped.
+ * ------------------------------------------------------------------------- */
+csa_status lightning_index_topk(const csa_params* p, int Q, const uint8_t* q_idx,
+                                const float* q_scale, const float* w,
+                                const uint8_t* idx_key, const float* idx_scale, int64_t N_cap,
+                                const int64_t* pos_q, int32_t* topk_idx, int32_t* topk_cnt,
+                                float* scores_out, void* ws, size_t ws_bytes,
+                                int32_t* dev_status, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Shared-KV multi-query attention over selected entries + window + sink
+ * ([P2] CSA step 3; [P5] "Hybrid attention": shared-KV MQA with 128 heads
+ * of dim 512, sliding-window branch of 128 tokens, per-head sink logits in
+ * the softmax denominator, QK RMSNorm, RoPE on the last 64 dims with inverse
+ * RoPE on the output).  One query per sequence at position pos = pos_q[b].
+ *
+ *   qhat_h = RoPE_pos(RMSNorm(q[b,h,:]) * gamma_q)
+ *   KV set = { RoPE_{(i+1)m-1}(kv_c[b,i,:]) : i in topk_idx[b, 0..topk_cnt) }
+ *          U { RoPE_t(RMSNorm(kv_tok[b,t,:]) * gamma_kv) : max(0,pos-W+1) <= t <= pos }
+ *   s_hj = softmax_scale * qhat_h . v_j;  M_h = max(max_j s_hj, sink[h])
+ *   out[b,h,:] = RoPE_{-pos}( sum_j e^{s_hj-M_h} v_j / (sum_j e^{s_hj-M_h} + e^{sink[h]-M_h}) )
+ * stored as bf16; lse[b,h] = M_h + log(denominator) when lse is not NULL.
+ * Readings (pages silent): one joint softmax over window and entries, no
+ * de-duplication; compressed entries are used as stored (their pooling
+ * RMSNorm is the KV norm); entry i sits at position (i+1)*m-1; rotate-half
+ * pairing over the last rope_dim dims.  sink = -inf drops the sink; +inf
+ * gives a zero output.
+ *
+ *   q [B, H, d] bf16; pos_q [B] int64; kv_c [B, N_cap, d] bf16;
+ *   topk_idx [B, k] int32, topk_cnt [B] int32 (entries must be < n_vis);
+ *   kv_tok [B, L_cap, d] bf16; sink [H] fp32; gamma_q, gamma_kv [d] or NULL;
+ *   out [B, H, d] bf16 (written); lse [B, H] fp32 or NULL.
+ * Device errors: an index >= n_vis or < -1 -> CSA_ERR_DEVICE_INDEX, skipped.
+ * ------------------------------------------------------------------------- */
+csa_status sparse_mqa_decode(const csa_params* p, const void* q, const int64_t* pos_q,
+                             const void* kv_c, int64_t N_cap, const int32_t* topk_idx,
+                             const int32_t* topk_cnt, const void* kv_tok, int64_t L_cap,
+                             const float* sink, const float* gamma_q, const float* gamma_kv,
+                             void* out, float* lse, void* ws, size_t ws_bytes,
+                             int32_t* dev_status, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * HCA dense decode ([P2] HCA: dense attention over every compressed entry;
+ * [P5] HCA bullet).  As sparse_mqa_decode with the KV set
+ * { entries 0 .. n_vis-1 } U window, n_vis = min(floor((pos+1)/m), N_cap).
+ * ------------------------------------------------------------------------- */
+csa_status dense_mqa_decode(const csa_params* p, const void* q, const int64_t* pos_q,
+                            const void* kv_c, int64_t N_cap, const void* kv_tok, int64_t L_cap,
+                            const float* sink, const float* gamma_q, const float* gamma_kv,
+                            void* out, float* lse, void* ws, size_t ws_bytes,
+                            int32_t* dev_status, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * CSA prefill chunk (B = 1): T new tokens at positions P .. P+T-1 whose KV
+ * rows (kv_tok) and indexer-stream rows (idx_tok) the caller has already
+ * written.  Runs, in order: csa_compress of blocks P/m .. ceil((P+T)/m)-1
+ * (ctx_len = P+T); the Lightning Indexer for every new query t with its own
+ * causal visible count floor((t+1)/m); top-k per query; and the sparse MQA
+ * per query with its own window [max(0,t-W+1), t].  P must be a multiple
+ * of m.
+ *   q [T, H, d] bf16, q_idx [T, H_I, D_I] E4M3, q_scale/w [T, H_I] fp32,
+ *   out [T, H, d] bf16 (written), topk_idx [T, k] / topk_cnt [T] (written).
+ * ------------------------------------------------------------------------- */
+csa_status csa_prefill_chunk(const csa_params* p, int64_t P, int T, const void* kv_tok,
+                             const void* idx_tok, int64_t L_cap, const float* w_s,
+                             const float* b_pos, const float* gamma, const float* w_s_idx,
+                             const float* b_pos_idx, void* kv_c, uint8_t* idx_key,
+                             float* idx_scale, int64_t N_cap, const void* q,
+                             const uint8_t* q_idx, const float* q_scale, const float* w,
+                             const float* sink, const float* gamma_q, const float* gamma_kv,
+                             int32_t* topk_idx, int32_t* topk_cnt, void* out, void* ws,
+                             size_t ws_bytes, int32_t* dev_status, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CSA_H_ */

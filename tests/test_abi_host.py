@@ -1,0 +1,115 @@
+"""Host-only checks of the C ABI: the library builds, loads and exports every
+symbol include/csa.h declares, and argument validation rejects bad calls
+before anything reaches a device.  No test here passes a non-null device
+pointer, so nothing can be launched.
+"""
+import ctypes as C
+import os
+import re
+
+import pytest
+
+from compressed_sparse_kv_04_b200 import binding
+from compressed_sparse_kv_04_b200 import build as csa_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    csa_build.build()
+    return binding.lib()
+
+
+def declared_functions():
+    names = []
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if not fn.endswith(".h"):
+            continue
+        text = open(os.path.join(ROOT, "include", fn)).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        for m in re.finditer(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\*?\s*([a-z_][a-z0-9_]*)\s*\(",
+                             text, flags=re.M):
+            names.append(m.group(1))
+    return sorted(set(names))
+
+
+def test_header_declares_the_six_entry_points():
+    names = declared_functions()
+    for n in ["hca_compress", "csa_compress", "lightning_index_topk", "sparse_mqa_decode",
+              "dense_mqa_decode", "csa_prefill_chunk"]:
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in declared_functions():
+        assert hasattr(L, name), name
+    assert set(binding.EXPORTS) <= set(declared_functions())
+
+
+def test_version_and_error_string(L):
+    assert L.csa_version() >= 100
+    assert isinstance(L.csa_last_error(), bytes)
+
+
+def P(**kw):
+    base = dict(B=1, d=512, H=128, H_I=64, D_I=128, k=1024, window=128, rope_dim=64, m=4)
+    base.update(kw)
+    return binding.make_params(**base)
+
+
+def test_null_params_rejected(L):
+    assert L.hca_compress(None, None, 1, None, None, None, None, 0, 1, None, 1, None, None) == 1
+    assert L.csa_workspace_bytes(None, 1, 1, 1) == 0
+
+
+@pytest.mark.parametrize("kw,code", [(dict(d=256), 2), (dict(m=0), 2), (dict(m=200), 2),
+                                     (dict(B=0), 1), (dict(eps=0.0), 1)])
+def test_bad_shapes_rejected(L, kw, code):
+    p = P(**kw)
+    st = L.hca_compress(C.byref(p), None, 1, None, None, None, None, 0, 1, None, 1, None, None)
+    assert st == code, binding.lib().csa_last_error()
+
+
+def test_null_tensor_rejected_before_launch(L):
+    p = P()
+    st = L.lightning_index_topk(C.byref(p), 1, None, None, None, None, None, 1024, None, None,
+                                None, None, None, 0, None, None)
+    assert st == 1
+    assert b"q_idx" in L.csa_last_error()
+
+
+def test_indexer_shape_limits(L):
+    for kw in (dict(D_I=96), dict(H_I=65), dict(k=4096), dict(k=0)):
+        p = P(**kw)
+        st = L.lightning_index_topk(C.byref(p), 1, None, None, None, None, None, 1024, None,
+                                    None, None, None, None, 0, None, None)
+        assert st == 2, kw
+
+
+def test_attention_shape_limits(L):
+    for kw in (dict(H=129), dict(rope_dim=63), dict(rope_dim=512), dict(window=-1)):
+        p = P(**kw)
+        st = L.dense_mqa_decode(C.byref(p), None, None, None, 1, None, 1, None, None, None,
+                                None, None, None, 0, None, None)
+        assert st == 2, kw
+
+
+def test_prefill_argument_checks(L):
+    p = P(B=2)
+    args = [None] * 2 + [1] + [None] * 8 + [1] + [None] * 10 + [None, 0, None, None]
+    st = L.csa_prefill_chunk(C.byref(p), 0, 4, *args)
+    assert st == 2  # B must be 1
+    p = P(B=1)
+    st = L.csa_prefill_chunk(C.byref(p), 3, 4, *args)
+    assert st == 1  # P not a multiple of m
+
+
+def test_workspace_sizes_are_monotone(L):
+    p = P(B=8)
+    a = L.csa_workspace_bytes(C.byref(p), 1, 1, 32768)
+    b = L.csa_workspace_bytes(C.byref(p), 1, 1, 65536)
+    assert 0 < a < b
+    assert L.csa_workspace_bytes(C.byref(p), 2, 1, 32768) > 0
+    assert L.csa_workspace_bytes(C.byref(p), 3, 1, 8192) > 0
+    assert L.csa_workspace_bytes(C.byref(p), 9, 1, 8192) == 0
