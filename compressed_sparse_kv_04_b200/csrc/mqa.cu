@@ -1,8 +1,40 @@
-// Shared-KV MQA decode (placeholder until the tcgen05 kernel lands).
+// Shared-KV multi-query attention for decode (CSA sparse / HCA dense) with
+// the sliding window and per-head sink, on the 5th-generation tensor cores.
+//
+// "DeepSeek V4 technical report" (agentupdate.ai), hybrid attention: CSA step
+// 3 (multi-query attention over the selected compressed entries) and the HCA
+// paragraph (dense attention over every compressed entry); "DeepSeek V4-Pro"
+// (llm-arch-kb), "Hybrid attention": 128 query heads of dim 512 sharing one
+// KV head, a 128-token uncompressed window branch, a learnable sink logit per
+// head in the softmax denominator, RMSNorm on queries and KV, RoPE on the
+// last 64 dims of query / KV / output with the inverse rotation on the output.
+//
+// Design.  The 128 x 512 fp32 output accumulator alone would fill the whole
+// tensor memory of an SM, so a pair of CTAs (a cluster of 2) shares every
+// (query, split): CTA r owns head-dim half r.  Per 64-entry tile:
+//   - the producer warp gathers the tile's rows with TMA tile::gather4 (only
+//     this CTA's half of each row; 128-byte swizzle), K = V = that tile;
+//   - transform warps RoPE the rotated dims in place (the half that holds
+//     them) and, for window tokens, compute the half-row sum of squares that
+//     the token RMSNorm needs;
+//   - the MMA warp issues S_r = Qhat_r . K_r^T (A = this CTA's half of the
+//     normalised, roped query, resident in TMEM; B = the tile, K-major) into
+//     one of two TMEM S buffers, then P . V_r into the O half (A = P in TMEM,
+//     B = the same tile read MN-major);
+//   - softmax warps (thread = head) exchange the partial S rows with the peer
+//     through distributed shared memory, sum them in a fixed order (so both
+//     CTAs hold bit-identical logits), apply the window-token norm factors,
+//     run an online softmax with lazy rescaling (O is rescaled in TMEM only
+//     when the running max grows by more than 8), and write P (bf16) back
+//     into the S buffer for the P.V MMA.
+// Splits of the KV list run on different pairs; their (m, l, O) partials are
+// merged by mqa_combine_kernel, which also folds in the sink and applies the
+// inverse RoPE.  Every wait is bounded and reports CSA_ERR_DEVICE_TIMEOUT.
 #include <algorithm>
 
 #include "common.cuh"
 #include "kernels.h"
+#include "tma.h"
 
 namespace csa {
 
@@ -13,13 +45,691 @@ size_t mqa_workspace_bytes(int rows, int splits, int H, int D) {
 }
 
 int mqa_choose_splits(int rows, int64_t max_kv, int num_sms) {
-  int64_t tiles = (max_kv + 63) / 64;
+  int64_t tiles = (max_kv + 63) / 64 + 1;
   int pairs = std::max(1, num_sms / 2);
   int64_t s = (pairs + rows - 1) / rows;
-  s = std::min<int64_t>(s, std::max<int64_t>(1, tiles));
+  s = std::min<int64_t>(s, tiles);
   return (int)std::max<int64_t>(1, s);
 }
 
-cudaError_t launch_mqa(const MqaLaunch&, cudaStream_t) { return cudaErrorNotSupported; }
+namespace {
+
+constexpr int TN = 64;           // KV rows per tile
+constexpr int kThreads = 320;    // 10 warps
+constexpr int kXStride = 68;     // padded row (floats) of the S exchange buffer
+constexpr float kRescaleThreshold = 8.0f;
+
+template <int D>
+struct MCfg {
+  static constexpr int Dh = D / 2;             // head-dim half per CTA
+  static constexpr int NC = Dh / 64;           // 128-byte chunks per half row
+  static constexpr int kChunkBytes = TN * 128;
+  static constexpr int kStageBytes = NC * kChunkBytes;
+  static constexpr int kStages = D == 512 ? 3 : 4;
+  static constexpr int kQCols = Dh / 2;        // bf16 pairs
+  static constexpr int kSCol0 = kQCols;        // two S buffers of TN columns
+  static constexpr int kOCol = kQCols + 2 * TN;
+  static constexpr int kCols = kOCol + Dh;     // 512 for D = 512
+  static constexpr uint32_t kAlloc = kCols <= 256 ? 256 : 512;
+};
+
+struct Meta {
+  int32_t grow[TN];   // row coordinate in the tensor map
+  int32_t pos[TN];    // RoPE position
+  float ss[TN];       // half-row sum of squares (window tiles)
+  uint32_t valid[2];  // bit r: row r holds a real KV vector
+  int32_t window;     // 1: window tokens; 0: compressed entries
+  int32_t pad;
+};
+
+struct XSlot {
+  float s[128 * kXStride];
+  float ss[TN];
+};
+
+struct Params {
+  int Q, H, m, W, R, splits;
+  int64_t N_cap, L_cap;
+  const __nv_bfloat16* q;
+  const int64_t* pos_q;
+  int64_t pos_base;
+  const int32_t* sel_idx;
+  const int32_t* sel_cnt;
+  int kmax;
+  const float* gamma_q;
+  const float* gamma_kv;
+  float eps, scale_log2;  // softmax scale * log2(e)
+  float* part_o;
+  float* part_ml;
+  int32_t* status;
+  double inv_freq[64];
+};
+
+// Byte offset of (row r, local dim d) inside a stage (128B-swizzled chunks).
+CSA_DEV uint32_t tile_off(int r, int d) {
+  uint32_t lin = (uint32_t)r * 128u + (uint32_t)(d & 63) * 2u;
+  return (uint32_t)(d >> 6) * (TN * 128u) + (lin ^ (((lin >> 7) & 7u) << 4));
+}
+
+CSA_DEV uint64_t desc_k(uint32_t saddr) { return sdesc_sw128(saddr, 16, 1024); }
+template <int D>
+CSA_DEV uint64_t desc_mn(uint32_t saddr) {
+  return sdesc_sw128(saddr, MCfg<D>::kChunkBytes, 1024);
+}
+
+CSA_DEV int64_t row_pos(const Params& p, int row) {
+  return p.pos_q ? p.pos_q[row] : p.pos_base + row % p.Q;
+}
+
+template <bool kCluster = false>
+CSA_DEV bool wait_all(uint64_t* bar, uint32_t parity, const Params& p, volatile int* abort_flag) {
+  bool ok = mbar_wait<kCluster>(bar, parity, p.status, abort_flag);
+  return __all_sync(0xffffffffu, ok);
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    mqa_pair_kernel(const __grid_constant__ CUtensorMap map_c,
+                    const __grid_constant__ CUtensorMap map_t, const Params p) {
+  using C = MCfg<D>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* stages = smem;
+  XSlot* xs = reinterpret_cast<XSlot*>(stages + C::kStages * C::kStageBytes);
+  Meta* meta = reinterpret_cast<Meta*>(xs + 2);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(meta + C::kStages);
+  uint64_t* full = bars;
+  uint64_t* ready = full + C::kStages;
+  uint64_t* empty = ready + C::kStages;
+  uint64_t* sfull = empty + C::kStages;
+  uint64_t* pready = sfull + 2;
+  uint64_t* xfull = pready + 2;
+  uint64_t* xempty = xfull + 2;
+  uint64_t* pvdone = xempty + 2;
+  uint64_t* qready = pvdone + 1;
+  uint64_t* drain = qready + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const uint32_t rank = cluster_ctarank();
+  const uint32_t peer = rank ^ 1u;
+  const int split = blockIdx.x >> 1;
+  const int row = blockIdx.y;
+  const int b = row / p.Q;
+
+  // The KV list of this query row: n_c compressed entries, then the window.
+  const int64_t pos = row_pos(p, row);
+  int64_t n_vis = pos < 0 ? 0 : (pos + 1) / p.m;
+  if (n_vis > p.N_cap) n_vis = p.N_cap;
+  int n_c;
+  if (p.sel_idx) {
+    int c = p.sel_cnt[row];
+    n_c = c < 0 ? 0 : (c > p.kmax ? p.kmax : c);
+  } else {
+    n_c = (int)n_vis;
+  }
+  const int64_t w0 = pos - p.W + 1 < 0 ? 0 : pos - p.W + 1;
+  const int nwin = (p.W > 0 && pos >= 0) ? (int)(pos - w0 + 1) : 0;
+  const int tiles_c = (n_c + TN - 1) / TN;
+  const int tiles_all = tiles_c + (nwin + TN - 1) / TN;
+  const int tps = (tiles_all + p.splits - 1) / p.splits;
+  const int t0 = std::min(split * tps, tiles_all);
+  const int t1 = std::min(t0 + tps, tiles_all);
+  const int ntile = t1 - t0;
+
+  float* po = p.part_o + (((int64_t)row * p.splits + split) * p.H) * D + rank * C::Dh;
+  float* pml = p.part_ml + ((int64_t)row * p.splits + split) * 2 * p.H;
+  if (ntile <= 0) {  // empty split: an empty partial (uniform over the pair)
+    if (rank == 0)
+      for (int h = threadIdx.x; h < p.H; h += kThreads) {
+        pml[h] = -INFINITY;
+        pml[p.H + h] = 0.f;
+      }
+    return;
+  }
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&ready[s], 128);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&sfull[a], 1);
+      mbar_init(&pready[a], 128);
+      mbar_init(&xfull[a], 128);
+      mbar_init(&xempty[a], 128);
+    }
+    mbar_init(pvdone, 1);
+    mbar_init(qready, 128);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, C::kAlloc);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  cluster_sync();  // the peer's barriers are initialised before any remote arrive
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t t_q = tmem, t_s = tmem + C::kSCol0, t_o = tmem + C::kOCol;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------- producer --
+    int it = 0;
+    for (int t = t0; t < t1; ++t, ++it) {
+      const int s = it % C::kStages;
+      const uint32_t ph = (it / C::kStages) & 1;
+      if (!wait_all(&empty[s], ph ^ 1, p, abort_flag)) break;
+      const bool win = t >= tiles_c;
+      Meta& M = meta[s];
+      uint32_t vbits[2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int r = lane + 32 * h;
+        bool valid;
+        int32_t grow, rpos;
+        if (!win) {
+          const int j = t * TN + r;
+          valid = j < n_c;
+          int64_t i = j;
+          if (valid && p.sel_idx) {
+            i = p.sel_idx[(int64_t)row * p.kmax + j];
+            if (i < 0 || i >= n_vis) {
+              report(p.status, CSA_ERR_DEVICE_INDEX);
+              valid = false;
+            }
+          }
+          if (!valid) i = 0;
+          grow = (int32_t)((int64_t)b * p.N_cap + i);
+          rpos = (int32_t)((i + 1) * p.m - 1);
+        } else {
+          const int j = (t - tiles_c) * TN + r;
+          valid = j < nwin;
+          if (valid && w0 + j >= p.L_cap) {  // query position beyond the token buffer
+            report(p.status, CSA_ERR_CAPACITY);
+            valid = false;
+          }
+          const int64_t tok = valid ? w0 + j : 0;
+          grow = (int32_t)((int64_t)b * p.L_cap + tok);
+          rpos = (int32_t)tok;
+        }
+        M.grow[r] = grow;
+        M.pos[r] = rpos;
+        vbits[h] = __ballot_sync(0xffffffffu, valid);
+      }
+      if (lane == 0) {
+        M.valid[0] = vbits[0];
+        M.valid[1] = vbits[1];
+        M.window = win ? 1 : 0;
+      }
+      __syncwarp();
+      if (lane == 0) {
+        const CUtensorMap* map = win ? &map_t : &map_c;
+        mbar_expect_tx(&full[s], C::kStageBytes);
+        uint8_t* dst = stages + s * C::kStageBytes;
+#pragma unroll
+        for (int c = 0; c < C::NC; ++c)
+          for (int g = 0; g < TN / 4; ++g)
+            tma_gather4(dst + c * C::kChunkBytes + g * 4 * 128, map, &full[s],
+                        (int32_t)(rank * C::Dh + c * 64), M.grow[4 * g], M.grow[4 * g + 1],
+                        M.grow[4 * g + 2], M.grow[4 * g + 3]);
+      }
+    }
+    if (*abort_flag && lane == 0) {  // copies still in flight must land first
+      for (int j = std::max(0, it - C::kStages); j < it; ++j)
+        mbar_wait(&full[j % C::kStages], (j / C::kStages) & 1, p.status);
+    }
+  } else if (warp == 1) {
+    // -------------------------------------------------------- MMA issuer --
+    const uint32_t idesc_s = idesc_bf16(128, TN, 0, 0);
+    const uint32_t idesc_pv = idesc_bf16(128, C::Dh, 0, 1);
+    bool ok = wait_all(qready, 0, p, abort_flag);
+    tc_fence_after();
+    bool issued = false;
+    auto issue_pv = [&](int jt) -> bool {
+      const int a = jt & 1, s = jt % C::kStages;
+      if (!wait_all(&pready[a], (jt >> 1) & 1, p, abort_flag)) return false;
+      tc_fence_after();
+      if (elect_one()) {
+        const uint32_t base = smem_u32(stages + s * C::kStageBytes);
+#pragma unroll
+        for (int kk = 0; kk < TN / 16; ++kk)
+          mma_bf16_ts(t_o, t_s + a * TN + kk * 8, desc_mn<D>(base + kk * 16 * 128), idesc_pv,
+                      (jt > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(&empty[s]);
+        mma_commit(pvdone);
+      }
+      __syncwarp();
+      return true;
+    };
+    int it = 0;
+    for (; ok && it < ntile; ++it) {
+      const int s = it % C::kStages, a = it & 1;
+      if (!wait_all(&ready[s], (it / C::kStages) & 1, p, abort_flag)) break;
+      tc_fence_after();
+      if (elect_one()) {
+        const uint32_t base = smem_u32(stages + s * C::kStageBytes);
+#pragma unroll
+        for (int kk = 0; kk < C::Dh / 16; ++kk)
+          mma_bf16_ts(t_s + a * TN, t_q + kk * 8,
+                      desc_k(base + (kk >> 2) * C::kChunkBytes + (kk & 3) * 32), idesc_s,
+                      kk > 0 ? 1u : 0u);
+        mma_commit(&sfull[a]);
+      }
+      __syncwarp();
+      issued = true;
+      if (it > 0 && !issue_pv(it - 1)) break;
+    }
+    if (it == ntile && ntile > 0 && !*abort_flag) issue_pv(ntile - 1);
+    if (*abort_flag && issued) {
+      if (elect_one()) mma_commit(drain);
+      __syncwarp();
+      mbar_wait(drain, 0, p.status);
+    }
+  } else if (warp < 6) {
+    // ----------------------------------------------------------- transform --
+    // Two threads per tile row: `half` 0 takes the window-norm sum and the
+    // first half of the rotated pairs, `half` 1 the second half.
+    const int tid = threadIdx.x - 64;  // 0..127
+    const int r = tid >> 1, hf = tid & 1;
+    const bool rope_here = (p.R > 0) && rank == 1;
+    for (int it = 0; it < ntile; ++it) {
+      const int s = it % C::kStages;
+      if (!wait_all(&full[s], (it / C::kStages) & 1, p, abort_flag)) break;
+      const Meta& M = meta[s];
+      uint8_t* st = stages + s * C::kStageBytes;
+      const bool valid = (M.valid[r >> 5] >> (r & 31)) & 1u;
+      float ss = 0.f;
+      if (valid && M.window) {
+        for (int c = hf; c < C::Dh / 8; c += 2) {  // 16-byte units
+          uint4 u = *reinterpret_cast<const uint4*>(st + tile_off(r, c * 8));
+          uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            float lo = bf16_lo(w4[q]), hi = bf16_hi(w4[q]);
+            ss = fmaf(lo, lo, fmaf(hi, hi, ss));
+          }
+          if (p.gamma_kv) {
+            const float* g = p.gamma_kv + rank * C::Dh + c * 8;
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              w4[q] = pack_bf16(bf16_lo(w4[q]) * __ldg(g + 2 * q),
+                                bf16_hi(w4[q]) * __ldg(g + 2 * q + 1));
+            *reinterpret_cast<uint4*>(st + tile_off(r, c * 8)) =
+                make_uint4(w4[0], w4[1], w4[2], w4[3]);
+          }
+        }
+      }
+      ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+      if (hf == 0) meta[s].ss[r] = ss;
+      __syncwarp();  // gain-scaled values are in place before the rotation reads them
+      if (valid && rope_here) {
+        const int half = p.R / 2;
+        const int d0 = C::Dh - p.R;
+        const double ppos = (double)M.pos[r];
+        for (int j = hf; j < half; j += 2) {
+          float sn, cs;
+          sincos_reduced(ppos * p.inv_freq[j], &sn, &cs);
+          __nv_bfloat16* a1 = reinterpret_cast<__nv_bfloat16*>(st + tile_off(r, d0 + j));
+          __nv_bfloat16* a2 = reinterpret_cast<__nv_bfloat16*>(st + tile_off(r, d0 + j + half));
+          float x1 = __bfloat162float(*a1), x2 = __bfloat162float(*a2);
+          *a1 = __float2bfloat16_rn(x1 * cs - x2 * sn);
+          *a2 = __float2bfloat16_rn(x2 * cs + x1 * sn);
+        }
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(&ready[s]);
+    }
+  } else {
+    // ------------------------------------------------- softmax / epilogue --
+    const int quarter = warp & 3;
+    const int h = quarter * 32 + lane;  // head == TMEM lane
+    const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+    const bool head_ok = h < p.H;
+    // Query prologue: qhat = RoPE(RMSNorm(q) * gamma_q), this CTA's half -> TMEM.
+    {
+      const __nv_bfloat16* qr = p.q + ((int64_t)row * p.H + (head_ok ? h : 0)) * D;
+      float ss = 0.f;
+      for (int c = 0; c < D / 8; ++c) {
+        uint4 u = __ldg(reinterpret_cast<const uint4*>(qr) + c);
+        uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          float lo = bf16_lo(w4[q]), hi = bf16_hi(w4[q]);
+          ss = fmaf(lo, lo, fmaf(hi, hi, ss));
+        }
+      }
+      const float inv = head_ok ? 1.0f / sqrtf(ss / (float)D + p.eps) : 0.f;
+      const int dbase = rank * C::Dh;
+      const int d_rope = C::Dh - ((rank == 1) ? p.R : 0);  // local start of rotated dims
+      // Plain dims in chunks of 32.
+      for (int c0 = 0; c0 < d_rope; c0 += 32) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          uint4 v = __ldg(reinterpret_cast<const uint4*>(qr + dbase + c0 + u * 8));
+          uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int d = dbase + c0 + u * 8 + 2 * q;
+            float g0 = p.gamma_q ? __ldg(p.gamma_q + d) : 1.f;
+            float g1 = p.gamma_q ? __ldg(p.gamma_q + d + 1) : 1.f;
+            pk[u * 4 + q] = pack_bf16(bf16_lo(w4[q]) * inv * g0, bf16_hi(w4[q]) * inv * g1);
+          }
+        }
+        tmem_st16(t_q + lane_base + c0 / 2, pk);
+      }
+      // Rotated dims (this CTA holds them only when rank == 1).
+      if (d_rope < C::Dh) {
+        const int half = p.R / 2;
+        for (int j0 = 0; j0 < half; j0 += 16) {
+          // pairs j0..j0+15: dims d_rope+j and d_rope+half+j
+          float x1[16], x2[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int d1 = dbase + d_rope + j0 + j, d2 = d1 + half;
+            float g1 = p.gamma_q ? __ldg(p.gamma_q + d1) : 1.f;
+            float g2 = p.gamma_q ? __ldg(p.gamma_q + d2) : 1.f;
+            x1[j] = __bfloat162float(qr[d1]) * inv * g1;
+            x2[j] = __bfloat162float(qr[d2]) * inv * g2;
+          }
+          uint32_t pk1[8], pk2[8];
+#pragma unroll
+          for (int j = 0; j < 16; j += 2) {
+            float s0, c0, s1, c1;
+            sincos_reduced((double)pos * p.inv_freq[j0 + j], &s0, &c0);
+            sincos_reduced((double)pos * p.inv_freq[j0 + j + 1], &s1, &c1);
+            pk1[j / 2] = pack_bf16(x1[j] * c0 - x2[j] * s0, x1[j + 1] * c1 - x2[j + 1] * s1);
+            pk2[j / 2] = pack_bf16(x2[j] * c0 + x1[j] * s0, x2[j + 1] * c1 + x1[j + 1] * s1);
+          }
+          // Columns hold bf16 pairs: local dim d -> column d/2 (8 columns each).
+          tmem_st8(t_q + lane_base + (d_rope + j0) / 2, pk1);
+          tmem_st8(t_q + lane_base + (d_rope + half + j0) / 2, pk2);
+        }
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(qready);
+    }
+
+    float m_run = -INFINITY, l_run = 0.f;
+    const uint32_t x_peer_base = mapa(smem_u32(&xs[0]), peer);
+    const uint32_t xfull_peer = mapa(smem_u32(&xfull[0]), peer);
+    const uint32_t xempty_peer = mapa(smem_u32(&xempty[0]), peer);
+    bool alive = true;
+    for (int it = 0; it < ntile && alive; ++it) {
+      const int s = it % C::kStages, a = it & 1;
+      if (!wait_all(&sfull[a], (it >> 1) & 1, p, abort_flag)) break;
+      tc_fence_after();
+      float sv[TN];
+      {
+        uint32_t v[32];
+        tmem_ld32(t_s + lane_base + a * TN, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 32; ++j) sv[j] = __uint_as_float(v[j]);
+        tmem_ld32(t_s + lane_base + a * TN + 32, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 32; ++j) sv[32 + j] = __uint_as_float(v[j]);
+      }
+      if (!wait_all(&ready[s], (it / C::kStages) & 1, p, abort_flag)) break;
+      // Exchange partial logits with the peer (slot a).
+      if (!wait_all<true>(&xempty[a], ((it >> 1) & 1) ^ 1, p, abort_flag)) break;
+      {
+        const uint32_t dst = x_peer_base + (uint32_t)(a * sizeof(XSlot)) + (uint32_t)(h * kXStride * 4);
+#pragma unroll
+        for (int j = 0; j < TN; j += 4) st_cluster_v4(dst + j * 4, sv[j], sv[j + 1], sv[j + 2], sv[j + 3]);
+        if (h < TN) {
+          const uint32_t dss = x_peer_base + (uint32_t)(a * sizeof(XSlot)) +
+                               (uint32_t)offsetof(XSlot, ss) + (uint32_t)(h * 4);
+          asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(dss), "f"(meta[s].ss[h]) : "memory");
+        }
+        mbar_arrive_remote(xfull_peer + a * 8);
+      }
+      if (!wait_all<true>(&xfull[a], (it >> 1) & 1, p, abort_flag)) break;
+      const Meta& M = meta[s];
+      const bool win = M.window != 0;
+      // Window-token RMSNorm factor 1/rms(c_t) of column j: the two half sums
+      // are added in rank order, so both CTAs get the same bits.  No CTA-wide
+      // barrier is used here: every wait in this loop must stay bounded.
+      auto norm_factor = [&](int j) -> float {
+        const float ssum = rank == 0 ? M.ss[j] + xs[a].ss[j] : xs[a].ss[j] + M.ss[j];
+        return 1.0f / sqrtf(ssum / (float)D + p.eps);
+      };
+      const float* xr = xs[a].s + h * kXStride;
+      float mt = -INFINITY;
+#pragma unroll
+      for (int j = 0; j < TN; ++j) {
+        const float other = xr[j];
+        float v = rank == 0 ? sv[j] + other : other + sv[j];
+        if (win) v *= norm_factor(j);
+        const bool valid = (M.valid[j >> 5] >> (j & 31)) & 1u;
+        v = valid ? v * p.scale_log2 : -INFINITY;  // log2 domain
+        sv[j] = v;
+        mt = fmaxf(mt, v);
+      }
+      // Online softmax with lazy rescaling (log2 domain).
+      const bool grow = mt > m_run + kRescaleThreshold * 1.4426950408889634f || m_run == -INFINITY;
+      const float m_new = grow ? fmaxf(mt, m_run) : m_run;
+      const bool need = grow && m_run != -INFINITY;
+      // P.V of the previous tile must be complete before O may be rescaled.
+      // This wait happens on every tile, before pready(it) is released, so
+      // the pvdone phase can never run two phases ahead of this check.
+      if (it > 0) {
+        if (!wait_all(pvdone, (it - 1) & 1, p, abort_flag)) break;
+        tc_fence_after();
+      }
+      if (__any_sync(0xffffffffu, need) && it > 0) {
+        const float f = need ? exp2f(m_run - m_new) : 1.f;
+        for (int c = 0; c < C::Dh; c += 32) {
+          uint32_t v[32];
+          tmem_ld32(t_o + lane_base + c, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * f);
+          uint32_t v0[16], v1[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            v0[j] = v[j];
+            v1[j] = v[16 + j];
+          }
+          tmem_st16(t_o + lane_base + c, v0);
+          tmem_st16(t_o + lane_base + c + 16, v1);
+        }
+        tmem_wait_st();
+      }
+      if (need) l_run *= exp2f(m_run - m_new);
+      m_run = m_new;
+      float lsum = 0.f;
+      uint32_t pk[32];
+#pragma unroll
+      for (int j = 0; j < TN; j += 2) {
+        float p0 = m_run == -INFINITY ? 0.f : exp2f(sv[j] - m_run);
+        float p1 = m_run == -INFINITY ? 0.f : exp2f(sv[j + 1] - m_run);
+        lsum += p0 + p1;
+        if (win) {
+          p0 *= norm_factor(j);
+          p1 *= norm_factor(j + 1);
+        }
+        pk[j / 2] = pack_bf16(p0, p1);
+      }
+      l_run += lsum;
+      {
+        uint32_t v0[16], v1[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          v0[j] = pk[j];
+          v1[j] = pk[16 + j];
+        }
+        tmem_st16(t_s + lane_base + a * TN, v0);
+        tmem_st16(t_s + lane_base + a * TN + 16, v1);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&pready[a]);
+      mbar_arrive_remote(xempty_peer + a * 8);  // slot a may now be refilled by the peer
+    }
+    // Epilogue: the O half and (rank 0) the running max / sum.
+    if (!*abort_flag && wait_all(pvdone, (ntile - 1) & 1, p, abort_flag)) {
+      tc_fence_after();
+      float* dst = po + (int64_t)h * D;
+      for (int c = 0; c < C::Dh; c += 32) {
+        uint32_t v[32];
+        tmem_ld32(t_o + lane_base + c, v);
+        tmem_wait_ld();
+        if (head_ok)
+#pragma unroll
+          for (int j = 0; j < 32; j += 4)
+            *reinterpret_cast<float4*>(dst + c + j) =
+                make_float4(__uint_as_float(v[j]), __uint_as_float(v[j + 1]),
+                            __uint_as_float(v[j + 2]), __uint_as_float(v[j + 3]));
+      }
+      if (rank == 0 && head_ok) {
+        pml[h] = m_run;  // log2 domain
+        pml[p.H + h] = l_run;
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // no CTA leaves while its peer may still touch its shared memory
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kAlloc);
+  }
+}
+
+// Merge the split partials of one (row, head), fold in the sink, normalise,
+// apply the inverse rotation, store bf16 (and the log-sum-exp).
+__global__ void mqa_combine_kernel(const Params p, int D, const float* __restrict__ sink,
+                                   __nv_bfloat16* __restrict__ out, float* __restrict__ lse) {
+  extern __shared__ float so[];  // D floats
+  const int row = blockIdx.x, h = blockIdx.y;
+  const float* ml = p.part_ml + (int64_t)row * p.splits * 2 * p.H;
+  const float LOG2E = 1.4426950408889634f;
+  const float z = sink[h];
+  __nv_bfloat16* o = out + ((int64_t)row * p.H + h) * D;
+  if (z == INFINITY) {
+    for (int d = threadIdx.x; d < D; d += blockDim.x) o[d] = __float2bfloat16_rn(0.f);
+    if (lse && threadIdx.x == 0) lse[(int64_t)row * p.H + h] = INFINITY;
+    return;
+  }
+  const float z2 = z * LOG2E;  // log2 domain
+  float M = z2;
+  for (int s = 0; s < p.splits; ++s) M = fmaxf(M, ml[(int64_t)s * 2 * p.H + h]);
+  if (M == -INFINITY) {
+    for (int d = threadIdx.x; d < D; d += blockDim.x) o[d] = __float2bfloat16_rn(0.f);
+    if (lse && threadIdx.x == 0) lse[(int64_t)row * p.H + h] = -INFINITY;
+    return;
+  }
+  float L = z2 == -INFINITY ? 0.f : exp2f(z2 - M);
+  for (int s = 0; s < p.splits; ++s) {
+    const float ms = ml[(int64_t)s * 2 * p.H + h];
+    if (ms != -INFINITY) L += ml[(int64_t)s * 2 * p.H + p.H + h] * exp2f(ms - M);
+  }
+  const float invL = 1.0f / L;
+  for (int d = threadIdx.x; d < D; d += blockDim.x) {
+    float acc = 0.f;
+    for (int s = 0; s < p.splits; ++s) {
+      const float ms = ml[(int64_t)s * 2 * p.H + h];
+      if (ms == -INFINITY) continue;
+      acc = fmaf(p.part_o[(((int64_t)row * p.splits + s) * p.H + h) * D + d], exp2f(ms - M), acc);
+    }
+    so[d] = acc * invL;
+  }
+  __syncthreads();
+  const int64_t pos = row_pos(p, row);
+  const int half = p.R / 2, d0 = D - p.R;
+  for (int d = threadIdx.x; d < D; d += blockDim.x) {
+    float v = so[d];
+    if (d >= d0 && p.R > 0) {
+      const int j = (d - d0) % half;
+      float sn, cs;
+      sincos_reduced((double)pos * p.inv_freq[j], &sn, &cs);
+      if (d - d0 < half)
+        v = so[d] * cs + so[d + half] * sn;  // rotation by -angle
+      else
+        v = so[d] * cs - so[d - half] * sn;
+    }
+    o[d] = __float2bfloat16_rn(v);
+  }
+  if (lse && threadIdx.x == 0) lse[(int64_t)row * p.H + h] = (M + log2f(L)) / LOG2E;
+}
+
+template <int D>
+cudaError_t launch_impl(const MqaLaunch& a, cudaStream_t stream) {
+  using C = MCfg<D>;
+  Params p{};
+  p.Q = a.Q;
+  p.H = a.H;
+  p.m = a.m;
+  p.W = a.W;
+  p.R = a.rope_dim;
+  p.splits = a.splits;
+  p.N_cap = a.N_cap;
+  p.L_cap = a.L_cap;
+  p.q = reinterpret_cast<const __nv_bfloat16*>(a.q);
+  p.pos_q = a.pos_q;
+  p.pos_base = a.pos_base;
+  p.sel_idx = a.sel_idx;
+  p.sel_cnt = a.sel_cnt;
+  p.kmax = a.kmax;
+  p.gamma_q = a.gamma_q;
+  p.gamma_kv = a.gamma_kv;
+  p.eps = a.eps;
+  p.scale_log2 = a.scale * 1.4426950408889634f;
+  p.part_o = a.part_o;
+  p.part_ml = a.part_ml;
+  p.status = a.status;
+  for (int j = 0; j < 64; ++j) p.inv_freq[j] = a.inv_freq[j];
+  const int rows = a.B * a.Q;
+  if (rows > 65535 || a.splits * 2 > 65535) return cudaErrorInvalidConfiguration;
+
+  CUtensorMap map_c, map_t;
+  cudaError_t e = make_tmap_2d(&map_c, a.kv_c, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                               (uint64_t)a.B * a.N_cap, D, 1, 64, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (e != cudaSuccess) return e;
+  e = make_tmap_2d(&map_t, a.kv_tok, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)a.B * a.L_cap,
+                   D, 1, 64, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (e != cudaSuccess) return e;
+
+  const size_t smem = 1024 + (size_t)C::kStages * C::kStageBytes + 2 * sizeof(XSlot) +
+                      C::kStages * sizeof(Meta) + 32 * 8 + 16;
+  auto kern = mqa_pair_kernel<D>;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(2 * a.splits, rows, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, kern, map_c, map_t, p);
+  if (e != cudaSuccess) return e;
+  mqa_combine_kernel<<<dim3(rows, a.H), 128, D * sizeof(float), stream>>>(
+      p, D, a.sink, reinterpret_cast<__nv_bfloat16*>(a.out), a.lse);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_mqa(const MqaLaunch& a, cudaStream_t stream) {
+  if (a.D == 512) return launch_impl<512>(a, stream);
+  if (a.D == 128) return launch_impl<128>(a, stream);
+  return cudaErrorInvalidValue;
+}
 
 }  // namespace csa

@@ -336,11 +336,14 @@ void orc_topk(int64_t BQ, int64_t N_cap, const double* scores, const int64_t* n_
 //
 // sel_idx == nullptr selects the dense form (entries 0..n_vis-1); otherwise
 // entries sel_idx[bq, 0..sel_cnt[bq]) are used (negative ones are skipped).
+// kv_tok holds token rows tok_base .. tok_base+L_cap-1 (a window of a long
+// stream; pure storage offset, no effect on the arithmetic).
 void orc_mqa(int B, int Q, int H, int D, int m, int W, int rope_dim, double rope_base,
              const uint16_t* q, const int64_t* pos_q, const uint16_t* kv_c, int64_t N_cap,
              const int32_t* sel_idx, const int32_t* sel_cnt, int kmax, const uint16_t* kv_tok,
-             int64_t L_cap, const float* sink, const float* gamma_q, const float* gamma_kv,
-             double eps, double scale, double* out, double* lse, int nthreads) {
+             int64_t L_cap, int64_t tok_base, const float* sink, const float* gamma_q,
+             const float* gamma_kv, double eps, double scale, double* out, double* lse,
+             int nthreads) {
   const double inf = std::numeric_limits<double>::infinity();
   for (int64_t bq = 0; bq < (int64_t)B * Q; ++bq) {
     int64_t b = bq / Q;
@@ -369,7 +372,7 @@ void orc_mqa(int B, int Q, int H, int D, int m, int W, int rope_dim, double rope
         rope_apply(v, D, rope_dim, rope_base, (double)((i + 1) * m - 1), +1.0);
       } else {
         int64_t t = w0 + (j - (int64_t)ent.size());
-        const uint16_t* row = kv_tok + (b * L_cap + t) * D;
+        const uint16_t* row = kv_tok + (b * L_cap + (t - tok_base)) * D;
         for (int d = 0; d < D; ++d) v[d] = bf16_decode(row[d]);
         rms_norm(v, D, gamma_kv, eps);
         rope_apply(v, D, rope_dim, rope_base, (double)t, +1.0);

@@ -64,7 +64,7 @@ def _declare(L):
     L.orc_topk.argtypes = [i64, i64, P(f64), P(i64), i32, P(C.c_int32), P(C.c_int32), i32]
     L.orc_mqa.argtypes = [i32, i32, i32, i32, i32, i32, i32, f64, P(C.c_uint16), P(i64),
                           P(C.c_uint16), i64, P(C.c_int32), P(C.c_int32), i32, P(C.c_uint16),
-                          i64, P(f32), P(f32), P(f32), f64, f64, P(f64), P(f64), i32]
+                          i64, i64, P(f32), P(f32), P(f32), f64, f64, P(f64), P(f64), i32]
 
 
 def _c(a, dt):
@@ -152,10 +152,12 @@ def topk(scores, n_vis, k, nthreads=0):
 
 
 def mqa(q, pos_q, kv_c, kv_tok, sink, m, W, rope_dim, sel_idx=None, sel_cnt=None,
-        gamma_q=None, gamma_kv=None, eps=1e-6, scale=None, rope_base=10000.0, nthreads=0):
+        gamma_q=None, gamma_kv=None, eps=1e-6, scale=None, rope_base=10000.0, nthreads=0,
+        tok_base=0):
     """Shared-KV MQA with window and sink (a4 sparse when sel_idx is given, else a5 dense).
 
-    q [B,Q,H,D] bf16 bits; pos_q [B,Q]; kv_c [B,N_cap,D]; kv_tok [B,L_cap,D].
+    q [B,Q,H,D] bf16 bits; pos_q [B,Q]; kv_c [B,N_cap,D]; kv_tok [B,L_cap,D] holding
+    token rows tok_base .. tok_base+L_cap-1.
     Returns (out fp64 [B,Q,H,D], lse fp64 [B,Q,H]).
     """
     q = _c(q, np.uint16)
@@ -175,7 +177,7 @@ def mqa(q, pos_q, kv_c, kv_tok, sink, m, W, rope_dim, sel_idx=None, sel_cnt=None
     lib().orc_mqa(B, Q, H, D, m, W, rope_dim, rope_base, _p(q, C.c_uint16),
                   _p(_c(pos_q, np.int64), C.c_int64), _p(kv_c, C.c_uint16), N_cap,
                   _p(sel_idx, C.c_int32), _p(sel_cnt, C.c_int32), kmax,
-                  _p(kv_tok, C.c_uint16), L_cap, _p(_c(sink, np.float32), C.c_float),
+                  _p(kv_tok, C.c_uint16), L_cap, tok_base, _p(_c(sink, np.float32), C.c_float),
                   _p(None if gamma_q is None else _c(gamma_q, np.float32), C.c_float),
                   _p(None if gamma_kv is None else _c(gamma_kv, np.float32), C.c_float),
                   eps, scale, _p(out, C.c_double), _p(lse, C.c_double), nthreads)
