@@ -1,0 +1,620 @@
+#!/usr/bin/env python
+"""Benchmark of the CSA/HCA hybrid-attention decode layer on B200.
+
+Metric: decode-layer query-tokens/s (one new query token per sequence per
+step) and the achieved fraction of the HBM roofline.  A step is one pass of
+the whole hot path over one batch:
+  CSA: compress the block the new token completes (KV + indexer streams),
+       Lightning-Indexer scores, top-k, sparse shared-KV MQA (+ combine);
+  HCA: compress the newest block, dense shared-KV MQA (+ combine).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+    python bench.py --impl reference ...   (the fp64 CPU oracle, same metric)
+
+Timing: W untimed warm-up steps, then exactly K steps replayed as CUDA graphs,
+bracketed by a barrier and torch.cuda.synchronize() on both sides, CUDA
+events on the launching stream, max over ranks.  Inputs rotate over R
+independent device-resident sets whose combined per-step traffic exceeds
+four times the 126 MB L2, so every step reads its data from HBM.  A second,
+instrumented pass over the same sets records CUDA events between the stages
+of every step; it gives each kernel's average launch time, from which the
+dominant kernel's roofline fraction is computed.  The e2e figure runs the
+same steps through the same calls with the step's new inputs copied from
+pinned host memory and the output copied back, inside the timed region.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from compressed_sparse_kv_04_b200 import configs  # noqa: E402
+
+L2_BYTES = 126 * 2 ** 20
+METRIC = "CSA/HCA decode layer query-tokens/s at 128K and 1M ctx; % of HBM roofline"
+DEFAULT_WORKLOAD = configs.CSA_128K.name
+
+
+# ----------------------------------------------------------- byte accounting --
+def algorithmic_bytes(w) -> dict:
+    """Algorithmic HBM bytes per step (whole batch) of each kernel.
+
+    Only bytes the method must move are counted: inputs read once, outputs
+    written once.  Intermediates the library materialises (indexer scores,
+    split partials) are implementation overhead and are not counted, except
+    as the input of the kernel whose job is to read them (top-k reads the
+    scores it ranks)."""
+    B, d, m, W, H = w.B, w.d, w.m, w.W, w.H
+    out = {}
+    blk_in = B * m * d * 2 + (B * m * w.D_I * 2 if w.csa else 0)
+    blk_out = B * d * 2 + (B * (w.D_I + 4) if w.csa else 0)
+    out["compress"] = blk_in + blk_out + (d + m) * 4 * (2 if w.csa else 1)
+    q_bytes = B * H * d * 2
+    o_bytes = B * H * d * 2
+    if w.csa:
+        n = w.N_c
+        out["index_scores"] = B * n * (w.D_I + 4) + B * w.H_I * (w.D_I + 8)
+        out["topk"] = B * n * 4 + B * w.k * 4 + B * 4
+        kv = B * (w.k + W) * d * 2
+        out["mqa"] = kv + q_bytes + B * w.k * 4 + H * 4
+    else:
+        kv = B * (w.N_c + W) * d * 2
+        out["mqa"] = kv + q_bytes + H * 4
+    out["combine"] = o_bytes
+    out["step"] = sum(out.values())
+    return out
+
+
+def step_flops(w) -> dict:
+    f = {}
+    if w.csa:
+        f["index_scores"] = 2.0 * w.B * w.N_c * w.H_I * w.D_I
+        f["mqa"] = 4.0 * w.B * w.H * (w.k + w.W) * w.d
+    else:
+        f["mqa"] = 4.0 * w.B * w.H * (w.N_c + w.W) * w.d
+    return f
+
+
+# ------------------------------------------------------------ peak figures --
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return dict(hbm_gbs=float(d["hbm_gbs"]), bf16_tflops=float(d["bf16_tflops"]),
+                    source="measured")
+    return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, source="fallback")
+
+
+def kernel_source_sha(kernel: str) -> str:
+    src = {"index_scores": "indexer.cu", "topk": "topk.cu", "mqa": "mqa.cu",
+           "combine": "mqa.cu", "compress": "compress.cu"}[kernel]
+    h = hashlib.sha256()
+    for f in (src, "common.cuh"):
+        with open(os.path.join(ROOT, "compressed_sparse_kv_04_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def stored_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from a committed ncu capture, if it is still current."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    e = d.get(kernel, {}).get(workload)
+    if not e or e.get("source_sha") != kernel_source_sha(kernel):
+        return None
+    return e.get("bytes_per_launch")
+
+
+# ------------------------------------------------------------------ clocks --
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in self.lines:
+            f = [x.strip() for x in l.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                mhz = float(f[1])
+                smax = float(f[2])
+            except ValueError:
+                continue
+            sm.append(mhz)
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        loaded = [x for x in sm if smax and x > 0.5 * smax] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None,
+                "sm_max_mhz": smax, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------- aggregation --
+def aggregate(units_per_rank: float, elapsed_ms: float, world: int, reduce_max, reduce_sum):
+    """Whole-job throughput: all ranks' units over the slowest rank's time."""
+    t = reduce_max(elapsed_ms)
+    u = reduce_sum(units_per_rank)
+    return u / (t / 1e3), t
+
+
+# ------------------------------------------------------------- GPU workload --
+class Decode:
+    """Device state for R rotating input sets of one decode workload."""
+
+    def __init__(self, w, R, device):
+        import torch
+
+        from compressed_sparse_kv_04_b200 import binding, synth
+        self.torch, self.binding = torch, binding
+        self.w, self.R, self.dev = w, R, device
+        B, L, d, N = w.B, w.L, w.d, w.N_c
+        self.p = binding.params_for(w)
+        self.w_s, self.b_pos = synth.pool_params(w, device)
+        if w.csa:
+            self.w_si, self.b_pi = synth.pool_params(w, device, indexer=True)
+        qi = synth.queries(w, Q=1, device=device)
+        self.sink = qi["sink"]
+        self.ctx = torch.full((B,), L, dtype=torch.int64, device=device)
+        self.pos = self.ctx - 1
+        self.pos2 = self.pos.view(B, 1)
+        # One source stream and its whole-context compression (setup, untimed).
+        kv_src, idx_src = synth.token_streams(w, device=device)
+        kv_c_src = torch.empty(B, N, d, dtype=torch.bfloat16, device=device)
+        if w.csa:
+            key_src = torch.empty(B, N, w.D_I, dtype=torch.uint8, device=device)
+            ksc_src = torch.empty(B, N, dtype=torch.float32, device=device)
+            binding.csa_compress(self.p, kv_src, self.ctx, self.w_s, self.b_pos, None, 0, N,
+                                 kv_c_src, idx_src, self.w_si, self.b_pi, key_src, ksc_src)
+        else:
+            binding.hca_compress(self.p, kv_src, self.ctx, self.w_s, self.b_pos, None, 0, N,
+                                 kv_c_src)
+        tail = max(w.W, w.m)
+        self.tail = tail
+        self.sets = []
+        for r in range(R):
+            s = {}
+            # Full-size token buffers; only the tail the step reads is filled.
+            s["kv_tok"] = torch.empty(B, L, d, dtype=torch.bfloat16, device=device)
+            s["kv_tok"][:, L - tail:] = kv_src[:, L - tail:]
+            s["kv_c"] = kv_c_src.clone()
+            s["q"] = synth.normal_bf16((B, w.H, d), w.seed + 1000 + r, "q", device)
+            s["out"] = torch.empty(B, w.H, d, dtype=torch.bfloat16, device=device)
+            if w.csa:
+                s["idx_tok"] = torch.empty(B, L, w.D_I, dtype=torch.bfloat16, device=device)
+                s["idx_tok"][:, L - tail:] = idx_src[:, L - tail:]
+                s["key"] = key_src.clone()
+                s["ksc"] = ksc_src.clone()
+                qr = synth.queries(configs.scaled(w, seed=w.seed + 1000 + r), Q=1, device=device)
+                s["q_idx"], s["q_scale"], s["w"] = qr["q_idx"], qr["q_scale"], qr["w"]
+                s["scores"] = torch.empty(B, 1, N, dtype=torch.float32, device=device)
+                s["tidx"] = torch.empty(B, 1, w.k, dtype=torch.int32, device=device)
+                s["tcnt"] = torch.empty(B, 1, dtype=torch.int32, device=device)
+                s["ws"] = binding.workspace(self.p, binding.OP_SPARSE_MQA, 1, N, device)
+            else:
+                s["ws"] = binding.workspace(self.p, binding.OP_DENSE_MQA, 1, N, device)
+            self.sets.append(s)
+        del kv_src, idx_src
+        self.status = torch.zeros(1, dtype=torch.int32, device=device)
+        torch.cuda.synchronize()
+
+    # The stages of one step, in order; each is one library call.
+    def stages(self, s):
+        b, w, p, N = self.binding, self.w, self.p, self.w.N_c
+        st = self.status
+        if w.csa:
+            return [
+                ("compress", lambda: b.csa_compress(p, s["kv_tok"], self.ctx, self.w_s, self.b_pos,
+                                                    None, N - 1, 1, s["kv_c"], s["idx_tok"],
+                                                    self.w_si, self.b_pi, s["key"], s["ksc"],
+                                                    dev_status=st)),
+                ("index_scores", lambda: b.lightning_index_scores(p, 1, s["q_idx"], s["q_scale"],
+                                                                  s["w"], s["key"], s["ksc"],
+                                                                  self.pos2, s["scores"],
+                                                                  dev_status=st)),
+                ("topk", lambda: b.topk_select(p, 1, s["scores"], self.pos2, s["tidx"], s["tcnt"],
+                                               dev_status=st)),
+                ("mqa", lambda: b.sparse_mqa_decode(p, s["q"], self.pos, s["kv_c"],
+                                                    s["tidx"].view(w.B, w.k),
+                                                    s["tcnt"].view(w.B), s["kv_tok"], self.sink,
+                                                    s["out"], ws=s["ws"], dev_status=st)),
+            ]
+        return [
+            ("compress", lambda: b.hca_compress(p, s["kv_tok"], self.ctx, self.w_s, self.b_pos,
+                                                None, N - 1, 1, s["kv_c"], dev_status=st)),
+            ("mqa", lambda: b.dense_mqa_decode(p, s["q"], self.pos, s["kv_c"], s["kv_tok"],
+                                               self.sink, s["out"], ws=s["ws"], dev_status=st)),
+        ]
+
+    def launches_per_step(self):
+        # compress 1, (index 1, top-k 1), attention pair 1 + combine 1
+        return 5 if self.w.csa else 3
+
+    def capture(self, instrumented=False):
+        """One CUDA graph per input set (optionally with stage events)."""
+        torch = self.torch
+        graphs, events = [], []
+        stream = torch.cuda.Stream()
+        stream.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(stream):
+            for s in self.sets:  # warm the launch path outside capture
+                for _, fn in self.stages(s):
+                    fn()
+        torch.cuda.current_stream().wait_stream(stream)
+        torch.cuda.synchronize()
+        for s in self.sets:
+            g = torch.cuda.CUDAGraph()
+            ev = []
+            with torch.cuda.graph(g, stream=stream):
+                if instrumented:
+                    e = torch.cuda.Event(enable_timing=True, external=True)
+                    e.record()
+                    ev.append(e)
+                for _, fn in self.stages(s):
+                    fn()
+                    if instrumented:
+                        e = torch.cuda.Event(enable_timing=True, external=True)
+                        e.record()
+                        ev.append(e)
+            graphs.append(g)
+            events.append(ev)
+        return graphs, events
+
+    def step_input_bytes(self):
+        w = self.w
+        b = w.B * w.H * w.d * 2 + w.B * w.m * w.d * 2
+        if w.csa:
+            b += w.B * w.H_I * (w.D_I + 8) + w.B * w.m * w.D_I * 2
+        return b
+
+
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    def rmax(x):
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return t.item()
+
+    def rsum(x):
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.SUM)
+        return t.item()
+
+    w = configs.BY_NAME[args.workload]
+    ab = algorithmic_bytes(w)
+    R = args.rotate or max(2, math.ceil(4 * L2_BYTES / ab["step"]) + 1)
+    st = Decode(w, R, dev)
+    graphs, _ = st.capture(instrumented=False)
+    K, W = args.steps, args.warmup
+    torch.cuda.synchronize()
+
+    with ClockSampler(local) as clocks:
+        for i in range(W):
+            graphs[i % R].replay()
+        barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for i in range(K):
+            graphs[(W + i) % R].replay()
+        e1.record()
+        barrier()
+        elapsed = e0.elapsed_time(e1)
+        value, t_max = aggregate(w.B * K, elapsed, world, rmax, rsum)
+        status = int(st.status.item())
+
+        # Instrumented pass: stage durations of K steps (events inside graphs).
+        igraphs, ievents = st.capture(instrumented=True)
+        names = [n for n, _ in st.stages(st.sets[0])]
+        sums = {n: 0.0 for n in names}
+        done = 0
+        while done < K:
+            batch = min(R, K - done)
+            for j in range(batch):
+                igraphs[j].replay()
+            torch.cuda.synchronize()
+            for j in range(batch):
+                ev = ievents[j]
+                for n, a, b in zip(names, ev[:-1], ev[1:]):
+                    sums[n] += a.elapsed_time(b)
+            done += batch
+        stage_ms = {n: sums[n] / K for n in names}
+
+        # e2e: the step's new inputs from pinned host memory, output back.
+        e2e = None
+        if not args.no_e2e:
+            e2e = run_e2e(st, graphs, K, W, barrier, rmax, rsum, world)
+    clk = clocks.summary()
+
+    # Dominant kernel (largest average stage time) and its roofline.
+    peaks = measured_peaks()
+    dom = max(stage_ms, key=stage_ms.get)
+    dom_kernel = dom
+    dom_ms = stage_ms[dom]
+    if dom == "mqa":
+        # the attention call is the pair kernel + the combine kernel
+        bytes_dom = ab["mqa"] + ab["combine"]
+    else:
+        bytes_dom = ab[dom]
+    achieved = bytes_dom / (dom_ms * 1e-3) / 1e9
+    traffic = stored_traffic(dom_kernel, w.name)
+    launches = st.launches_per_step() * K
+
+    if rank != 0:
+        if world > 1:
+            dist.destroy_process_group()
+        return
+    ms_per_step = t_max / K
+    line = {
+        "metric": METRIC,
+        "value": round(value, 1),
+        "unit": "query-tokens/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": W,
+        "ms_per_step": round(ms_per_step, 6),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16+e4m3",
+        "data": "synthetic (seeded N(0,1) token streams, random query/indexer inputs)",
+        "config": {"workload": w.name, "batch": w.B, "context": w.L, "compressed_entries": w.N_c,
+                   "m": w.m, "heads": w.H, "head_dim": w.d, "window": w.W,
+                   "top_k": w.k if w.csa else None, "indexer": [w.H_I, w.D_I] if w.csa else None,
+                   "parallelism": f"replicas x{world} (independent sequences per GPU)",
+                   "l2": f"rotating {R} resident input sets (~{R * ab['step'] / 1e6:.0f} MB of "
+                         f"step traffic per rotation, > 4x the 126 MB L2)"},
+        "roofline": {"bound": "hbm", "kernel": dom_kernel, "achieved": round(achieved, 1),
+                     "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": round(achieved / peaks["hbm_gbs"], 4),
+                     "peak_source": peaks["source"], "traffic": traffic,
+                     "algorithmic_bytes_per_launch": bytes_dom,
+                     "avg_launch_ms": round(dom_ms, 6)},
+        "step_roofline": {"algorithmic_bytes": ab["step"],
+                          "achieved_GBps": round(ab["step"] / (ms_per_step * 1e-3) / 1e9, 1),
+                          "frac": round(ab["step"] / (ms_per_step * 1e-3) / 1e9 / peaks["hbm_gbs"], 4)},
+        "kernels_ms": {k: round(v, 6) for k, v in stage_ms.items()},
+        "e2e": e2e,
+        "gpu_launches": launches,
+        "clocks": clk,
+        "device_status": status,
+    }
+    if not args.no_cpu_baseline and world == 1:
+        line["cpu_baseline"] = cpu_baseline(w, st, args.cpu_seconds)
+    print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def run_e2e(st, graphs, K, W, barrier, rmax, rsum, world):
+    """Same steps; the new query and token rows come from pinned host memory
+    and the output goes back to it, inside the timed region."""
+    torch = st.torch
+    w, R = st.w, st.R
+    L, m = w.L, w.m
+    hq = [s["q"].cpu().pin_memory() for s in st.sets]
+    hkv = [s["kv_tok"][:, L - m:].cpu().pin_memory() for s in st.sets]
+    hout = torch.empty_like(st.sets[0]["out"], device="cpu").pin_memory()
+    extra = []
+    if w.csa:
+        extra = [(s, s["q_idx"].cpu().pin_memory(), s["q_scale"].cpu().pin_memory(),
+                  s["w"].cpu().pin_memory(), s["idx_tok"][:, L - m:].cpu().pin_memory())
+                 for s in st.sets]
+    h2d = sum(t.numel() * t.element_size() for t in (hq[0], hkv[0]))
+    if w.csa:
+        h2d += sum(t.numel() * t.element_size() for t in extra[0][1:])
+    d2h = hout.numel() * hout.element_size()
+
+    def one(i):
+        r = i % R
+        s = st.sets[r]
+        s["q"].copy_(hq[r], non_blocking=True)
+        s["kv_tok"][:, L - m:].copy_(hkv[r], non_blocking=True)
+        if w.csa:
+            _, a, b, c, d = extra[r]
+            s["q_idx"].copy_(a, non_blocking=True)
+            s["q_scale"].copy_(b, non_blocking=True)
+            s["w"].copy_(c, non_blocking=True)
+            s["idx_tok"][:, L - m:].copy_(d, non_blocking=True)
+        graphs[r].replay()
+        hout.copy_(s["out"], non_blocking=True)
+
+    for i in range(W):
+        one(i)
+    barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(K):
+        one(i)
+    e1.record()
+    barrier()
+    val, _ = aggregate(w.B * K, e0.elapsed_time(e1), world, rmax, rsum)
+    return {"value": round(val, 1), "unit": "query-tokens/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h}
+
+
+# ------------------------------------------------------------ CPU oracle --
+def oracle_sample(w, seconds, state=None):
+    """Time the fp64 oracle on one sequence's decode step, repeated for about
+    `seconds` (at least once).  Returns (query-tokens/s, steps, threads)."""
+    import numpy as np
+
+    from oracle import oracle as orc
+    rng = np.random.default_rng(w.seed)
+    d, N, L, m = w.d, w.N_c, w.L, w.m
+
+    def bf16(shape):
+        x = rng.standard_normal(shape).astype(np.float32)
+        return (x.view(np.uint32) >> 16).astype(np.uint16)
+
+    tail = max(w.W, m)
+    if state is not None:
+        import torch
+        s = state.sets[0]
+        kv_c = s["kv_c"][0:1].contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+        tok = s["kv_tok"][0:1, L - tail:].contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+    else:
+        kv_c = bf16((1, N, d))
+        tok = bf16((1, tail, d))
+    q = bf16((1, 1, w.H, d))
+    sink = rng.standard_normal(w.H).astype(np.float32)
+    w_s = (rng.standard_normal(d) * 0.02).astype(np.float32)
+    b_pos = (rng.standard_normal(m) * 0.1).astype(np.float32)
+    pos = np.array([[L - 1]])
+    if w.csa:
+        keys = rng.integers(0, 0x7E, (1, N, w.D_I)).astype(np.uint8)
+        ksc = rng.uniform(0.005, 0.015, (1, N)).astype(np.float32)
+        q_idx = rng.integers(0, 0x7E, (1, 1, w.H_I, w.D_I)).astype(np.uint8)
+        q_scale = rng.uniform(0.005, 0.02, (1, 1, w.H_I)).astype(np.float32)
+        wh = rng.uniform(0, 1, (1, 1, w.H_I)).astype(np.float32)
+        itok = bf16((1, tail, w.D_I))
+    threads = os.cpu_count() or 1
+    steps = 0
+    t0 = time.perf_counter()
+    while True:
+        # compress the newest block (the step's first stage)
+        orc.pool(tok, [tail], w_s, b_pos, None, m, tail // m - 1, 1, tail // m)
+        if w.csa:
+            orc.pool(itok, [tail], (rng.standard_normal(w.D_I) * 0.02).astype(np.float32),
+                     b_pos, None, m, tail // m - 1, 1, tail // m)
+            sc = orc.index_scores(q_idx, q_scale, wh, keys, ksc, pos, m)
+            idx, cnt = orc.topk(sc, np.array([[N]]), w.k)
+            orc.mqa(q, pos, kv_c, tok, sink, m, w.W, w.rope_dim, idx, cnt, tok_base=L - tail)
+        else:
+            orc.mqa(q, pos, kv_c, tok, sink, m, w.W, w.rope_dim, tok_base=L - tail)
+        steps += 1
+        el = time.perf_counter() - t0
+        if el >= seconds:
+            break
+    return steps / el, steps, threads, el
+
+
+def cpu_baseline(w, state, seconds):
+    v, steps, threads, el = oracle_sample(w, seconds, state)
+    return {"value": round(v, 4), "unit": "query-tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"{steps} decode step(s) of one sequence ({w.name}: {w.N_c} compressed "
+                      f"entries), {el:.1f} s wall on {threads} host threads"}
+
+
+def run_reference(args):
+    """The reference arm: the fp64 oracle as it stands, on the host cores."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    w = configs.BY_NAME[args.workload]
+    from oracle import oracle as orc
+    orc.lib()
+    for _ in range(args.warmup):
+        oracle_sample(w, 0.0)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_sample(w, 0.0)
+    el = time.perf_counter() - t0
+    value = args.steps / el  # one query token per step
+    threads = os.cpu_count() or 1
+    line = {
+        "metric": METRIC, "impl": "reference", "value": round(value, 4),
+        "unit": "query-tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(el / args.steps * 1e3, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": w.name},
+        "cpu_baseline": {"value": round(value, 4), "unit": "query-tokens/s", "cores": threads,
+                         "kind": "oracle",
+                         "sample": f"each step = one sequence's decode step of {w.name}"},
+        "e2e": {"value": round(value, 4), "unit": "query-tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=200)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(configs.BY_NAME))
+    ap.add_argument("--rotate", type=int, default=0, help="input sets (default: from L2 size)")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    if args.workload == configs.CSA_PREFILL.name or args.workload == configs.TINY_CSA.name:
+        ap.error("the benchmark times the decode workloads; prefill and the tiny case are "
+                 "parity-test cases")
+    run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -22,8 +22,8 @@ STATUS_NAMES = {0: "CSA_OK", 1: "CSA_ERR_INVALID_ARG", 2: "CSA_ERR_UNSUPPORTED_S
 OP_INDEX_TOPK, OP_SPARSE_MQA, OP_DENSE_MQA, OP_PREFILL = 1, 2, 3, 4
 
 EXPORTS = ["csa_version", "csa_last_error", "csa_workspace_bytes", "hca_compress",
-           "csa_compress", "lightning_index_topk", "sparse_mqa_decode", "dense_mqa_decode",
-           "csa_prefill_chunk"]
+           "csa_compress", "lightning_index_topk", "lightning_index_scores", "topk_select",
+           "sparse_mqa_decode", "dense_mqa_decode", "csa_prefill_chunk"]
 
 
 class CsaError(RuntimeError):
@@ -67,6 +67,8 @@ def _declare(L):
                                vp, vp, vp]
     L.lightning_index_topk.argtypes = [P, i32, vp, vp, vp, vp, vp, i64, vp, vp, vp, vp, vp, sz,
                                        vp, vp]
+    L.lightning_index_scores.argtypes = [P, i32, vp, vp, vp, vp, vp, i64, vp, vp, vp, vp]
+    L.topk_select.argtypes = [P, i32, vp, i64, vp, vp, vp, vp, vp]
     L.sparse_mqa_decode.argtypes = [P, vp, vp, vp, i64, vp, vp, vp, i64, vp, vp, vp, vp, vp, vp,
                                     sz, vp, vp]
     L.dense_mqa_decode.argtypes = [P, vp, vp, vp, i64, vp, i64, vp, vp, vp, vp, vp, vp, sz, vp,
@@ -154,6 +156,18 @@ def lightning_index_topk(p, Q, q_idx, q_scale, w, idx_key, idx_scale, pos_q, top
         idx_key.shape[1], _ptr(pos_q), _ptr(topk_idx), _ptr(topk_cnt), _ptr(scores_out),
         _ptr(ws), 0 if ws is None else ws.numel() * ws.element_size(), _ptr(dev_status),
         _stream(stream)))
+
+
+def lightning_index_scores(p, Q, q_idx, q_scale, w, idx_key, idx_scale, pos_q, scores,
+                           dev_status=None, stream=None):
+    _check(lib().lightning_index_scores(
+        C.byref(p), Q, _ptr(q_idx), _ptr(q_scale), _ptr(w), _ptr(idx_key), _ptr(idx_scale),
+        idx_key.shape[1], _ptr(pos_q), _ptr(scores), _ptr(dev_status), _stream(stream)))
+
+
+def topk_select(p, Q, scores, pos_q, topk_idx, topk_cnt, dev_status=None, stream=None):
+    _check(lib().topk_select(C.byref(p), Q, _ptr(scores), scores.shape[-1], _ptr(pos_q),
+                             _ptr(topk_idx), _ptr(topk_cnt), _ptr(dev_status), _stream(stream)))
 
 
 def sparse_mqa_decode(p, q, pos_q, kv_c, topk_idx, topk_cnt, kv_tok, sink, out, gamma_q=None,

@@ -20,6 +20,8 @@ csa_status fail(csa_status s, const char* fmt, ...) {
   return s;
 }
 
+constexpr int64_t kMaxIndexEntries = 262144;  // one 8-CTA cluster holds a score row
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 #define REQ_PTR(p)                                                                     \
@@ -234,12 +236,11 @@ csa_status csa_compress(const csa_params* p, const void* kv_tok, int64_t L_cap,
                          idx_scale, dev_status, stream);
 }
 
-static csa_status index_topk_common(const char* fn, const csa_params* p, int Q,
-                                    const uint8_t* q_idx, const float* q_scale, const float* w,
-                                    const uint8_t* idx_key, const float* idx_scale,
-                                    int64_t N_cap, const int64_t* pos_q, int64_t pos_base,
-                                    int32_t* topk_idx, int32_t* topk_cnt, float* scores,
-                                    int32_t* dev_status, cudaStream_t stream) {
+static csa_status index_common(const char* fn, const csa_params* p, int Q,
+                               const uint8_t* q_idx, const float* q_scale, const float* w,
+                               const uint8_t* idx_key, const float* idx_scale, int64_t N_cap,
+                               const int64_t* pos_q, int64_t pos_base, float* scores,
+                               int32_t* dev_status, cudaStream_t stream) {
   csa::IndexLaunch a{};
   a.B = p->B;
   a.Q = Q;
@@ -259,6 +260,13 @@ static csa_status index_topk_common(const char* fn, const csa_params* p, int Q,
   a.num_sms = csa::device_sm_count();
   cudaError_t e = csa::launch_index_scores(a, stream);
   if (e != cudaSuccess) return cuda_fail(fn, e);
+  return CSA_OK;
+}
+
+static csa_status topk_common(const char* fn, const csa_params* p, int Q, const float* scores,
+                              int64_t N_cap, const int64_t* pos_q, int64_t pos_base,
+                              int32_t* topk_idx, int32_t* topk_cnt, int32_t* dev_status,
+                              cudaStream_t stream) {
   csa::TopkLaunch t{};
   t.rows = p->B * Q;
   t.Q = Q;
@@ -271,8 +279,36 @@ static csa_status index_topk_common(const char* fn, const csa_params* p, int Q,
   t.idx = topk_idx;
   t.cnt = topk_cnt;
   t.status = dev_status;
-  e = csa::launch_topk(t, stream);
+  cudaError_t e = csa::launch_topk(t, stream);
   if (e != cudaSuccess) return cuda_fail(fn, e);
+  return CSA_OK;
+}
+
+static csa_status index_topk_common(const char* fn, const csa_params* p, int Q,
+                                    const uint8_t* q_idx, const float* q_scale, const float* w,
+                                    const uint8_t* idx_key, const float* idx_scale,
+                                    int64_t N_cap, const int64_t* pos_q, int64_t pos_base,
+                                    int32_t* topk_idx, int32_t* topk_cnt, float* scores,
+                                    int32_t* dev_status, cudaStream_t stream) {
+  csa_status st = index_common(fn, p, Q, q_idx, q_scale, w, idx_key, idx_scale, N_cap, pos_q,
+                               pos_base, scores, dev_status, stream);
+  if (st != CSA_OK) return st;
+  return topk_common(fn, p, Q, scores, N_cap, pos_q, pos_base, topk_idx, topk_cnt, dev_status,
+                     stream);
+}
+
+static csa_status check_index_args(const char* fn, const csa_params* p, int Q, int64_t N_cap) {
+  csa_status st = check_common(fn, p);
+  if (st != CSA_OK) return st;
+  st = check_indexer(fn, p);
+  if (st != CSA_OK) return st;
+  if (Q < 1) return fail(CSA_ERR_INVALID_ARG, "%s: Q=%d", fn, Q);
+  if (N_cap < 1 || N_cap > kMaxIndexEntries)
+    return fail(CSA_ERR_UNSUPPORTED_SHAPE, "%s: N_cap=%lld (supported: 1..%lld)", fn,
+                (long long)N_cap, (long long)kMaxIndexEntries);
+  if ((int64_t)p->B * Q > 65535)
+    return fail(CSA_ERR_UNSUPPORTED_SHAPE, "%s: B*Q=%lld (supported: <= 65535)", fn,
+                (long long)p->B * Q);
   return CSA_OK;
 }
 
@@ -282,14 +318,8 @@ csa_status lightning_index_topk(const csa_params* p, int Q, const uint8_t* q_idx
                                 int32_t* topk_idx, int32_t* topk_cnt, float* scores_out,
                                 void* ws, size_t ws_bytes, int32_t* dev_status, void* stream) {
   const char* fn = "lightning_index_topk";
-  csa_status st = check_common(fn, p);
+  csa_status st = check_index_args(fn, p, Q, N_cap);
   if (st != CSA_OK) return st;
-  st = check_indexer(fn, p);
-  if (st != CSA_OK) return st;
-  if (Q < 1) return fail(CSA_ERR_INVALID_ARG, "%s: Q=%d", fn, Q);
-  if (N_cap < 1 || N_cap > (int64_t)1 << 22)
-    return fail(CSA_ERR_UNSUPPORTED_SHAPE, "%s: N_cap=%lld (supported: 1..4194304)", fn,
-                (long long)N_cap);
   REQ_PTR(q_idx);
   REQ_PTR4(q_scale);
   REQ_PTR4(w);
@@ -300,8 +330,6 @@ csa_status lightning_index_topk(const csa_params* p, int Q, const uint8_t* q_idx
   REQ_PTR4(topk_cnt);
   OPT_PTR(scores_out);
   OPT_PTR4(dev_status);
-  if (((N_cap * p->D_I) & 15) != 0)
-    return fail(CSA_ERR_UNSUPPORTED_SHAPE, "%s: N_cap*D_I must be a multiple of 16", fn);
   float* scores = scores_out;
   if (!scores) {
     size_t need = csa_workspace_bytes(p, CSA_OP_INDEX_TOPK, Q, N_cap);
@@ -314,6 +342,40 @@ csa_status lightning_index_topk(const csa_params* p, int Q, const uint8_t* q_idx
   return index_topk_common(fn, p, Q, q_idx, q_scale, w, idx_key, idx_scale, N_cap, pos_q, 0,
                            topk_idx, topk_cnt, scores, dev_status,
                            static_cast<cudaStream_t>(stream));
+}
+
+csa_status lightning_index_scores(const csa_params* p, int Q, const uint8_t* q_idx,
+                                  const float* q_scale, const float* w, const uint8_t* idx_key,
+                                  const float* idx_scale, int64_t N_cap, const int64_t* pos_q,
+                                  float* scores, int32_t* dev_status, void* stream) {
+  const char* fn = "lightning_index_scores";
+  csa_status st = check_index_args(fn, p, Q, N_cap);
+  if (st != CSA_OK) return st;
+  REQ_PTR(q_idx);
+  REQ_PTR4(q_scale);
+  REQ_PTR4(w);
+  REQ_PTR(idx_key);
+  REQ_PTR4(idx_scale);
+  REQ_PTR(pos_q);
+  REQ_PTR(scores);
+  OPT_PTR4(dev_status);
+  return index_common(fn, p, Q, q_idx, q_scale, w, idx_key, idx_scale, N_cap, pos_q, 0, scores,
+                      dev_status, static_cast<cudaStream_t>(stream));
+}
+
+csa_status topk_select(const csa_params* p, int Q, const float* scores, int64_t N_cap,
+                       const int64_t* pos_q, int32_t* topk_idx, int32_t* topk_cnt,
+                       int32_t* dev_status, void* stream) {
+  const char* fn = "topk_select";
+  csa_status st = check_index_args(fn, p, Q, N_cap);
+  if (st != CSA_OK) return st;
+  REQ_PTR(scores);
+  REQ_PTR(pos_q);
+  REQ_PTR(topk_idx);
+  REQ_PTR4(topk_cnt);
+  OPT_PTR4(dev_status);
+  return topk_common(fn, p, Q, scores, N_cap, pos_q, 0, topk_idx, topk_cnt, dev_status,
+                     static_cast<cudaStream_t>(stream));
 }
 
 static csa_status mqa_common(const char* fn, const csa_params* p, csa_op op, int rows, int Q,
@@ -462,8 +524,6 @@ csa_status csa_prefill_chunk(const csa_params* p, int64_t P, int T, const void* 
   REQ_PTR(out);
   REQ_PTR(kv_c);
   REQ_PTR(kv_tok);
-  if (((N_cap * p->D_I) & 15) != 0)
-    return fail(CSA_ERR_UNSUPPORTED_SHAPE, "%s: N_cap*D_I must be a multiple of 16", fn);
   size_t need = csa_workspace_bytes(p, CSA_OP_PREFILL, T, N_cap);
   if (!ws || ws_bytes < need)
     return fail(CSA_ERR_WORKSPACE, "%s: workspace of %zu bytes needed, %zu given", fn, need,

@@ -277,13 +277,11 @@ cudaError_t launch_impl(const IndexLaunch& a, cudaStream_t stream) {
   size_t smem = 1024 + (size_t)C::kStages * C::kStageBytes + (size_t)p.N * DI + 256 * 4 +
                 (2 * C::kStages + 5) * 8 + 16;
   auto kern = index_score_kernel<DI>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)smem);
+  cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kern), DI == 128 ? 0 : 1,
+                                   smem);
   if (e != cudaSuccess) return e;
-  int occ = 1;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kThreads, smem);
-  if (e != cudaSuccess) return e;
-  occ = std::max(1, std::min(occ, 2));
+  // Two CTAs per SM when shared memory allows it (228 KB per SM).
+  int occ = (2 * (smem + 1024) <= 228 * 1024) ? 2 : 1;
   if (2 * cols > 512) occ = 1;  // two CTAs would contend for tensor memory
   int64_t groups = (int64_t)a.B * p.qgroups;
   if (groups > 65535) return cudaErrorInvalidConfiguration;

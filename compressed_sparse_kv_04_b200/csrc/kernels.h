@@ -90,4 +90,8 @@ cudaError_t launch_mqa(const MqaLaunch& a, cudaStream_t stream);
 
 int device_sm_count();
 
+// Sets the dynamic shared-memory limit of `func` once per device (the call
+// is then skipped, which keeps launches legal inside CUDA-graph capture).
+cudaError_t ensure_smem_attr(const void* func, int slot, size_t bytes);
+
 }  // namespace csa

@@ -703,7 +703,7 @@ cudaError_t launch_impl(const MqaLaunch& a, cudaStream_t stream) {
   const size_t smem = 1024 + (size_t)C::kStages * C::kStageBytes + 2 * sizeof(XSlot) +
                       C::kStages * sizeof(Meta) + 32 * 8 + 16;
   auto kern = mqa_pair_kernel<D>;
-  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  e = ensure_smem_attr(reinterpret_cast<const void*>(kern), D == 512 ? 3 : 4, smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(2 * a.splits, rows, 1);

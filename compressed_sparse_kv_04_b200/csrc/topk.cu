@@ -25,7 +25,6 @@ namespace csa {
 namespace {
 
 constexpr int kThreads = 1024;
-constexpr int kWarps = kThreads / 32;
 
 struct Params {
   int Q, m, k, C;
@@ -245,8 +244,7 @@ cudaError_t launch_topk(const TopkLaunch& a, cudaStream_t stream) {
   p.cnt = a.cnt;
   p.status = a.status;
   size_t smem = (256 + 256 + 32 + 8) * 4 + (size_t)p.slice * 4;
-  cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)smem);
+  cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(topk_kernel), 2, smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(C, a.rows, 1);

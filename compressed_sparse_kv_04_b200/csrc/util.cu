@@ -1,6 +1,7 @@
 // Host utilities shared by the launchers: SM count and TMA tensor maps.
 #include <mutex>
 
+#include "kernels.h"
 #include "tma.h"
 
 namespace csa {
@@ -16,6 +17,19 @@ int device_sm_count() {
     cached[dev] = n;
   }
   return cached[dev];
+}
+
+cudaError_t ensure_smem_attr(const void* func, int slot, size_t bytes) {
+  static size_t done[64][16] = {};
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64 || slot < 0 || slot >= 16)
+    return cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  std::lock_guard<std::mutex> lock(mu);
+  if (done[dev][slot] >= bytes) return cudaSuccess;
+  cudaError_t e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e == cudaSuccess) done[dev][slot] = bytes;
+  return e;
 }
 
 namespace {

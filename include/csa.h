@@ -163,6 +163,7 @@ csa_status csa_compress(const csa_params* p, const void* kv_tok, int64_t L_cap,
  *   scores_out [B, Q, N_cap] fp32 or NULL: when given, entries i < n_vis
  *              receive the fp32 scores (others are not written).
  * Device errors: n_vis > N_cap -> CSA_ERR_CAPACITY in dev_status, clamped.
+ * Sizes: N_cap <= 262144 (one cluster of 8 CTAs holds a row of scores).
  * ------------------------------------------------------------------------- */
 csa_status lightning_index_topk(const csa_params* p, int Q, const uint8_t* q_idx,
                                 const float* q_scale, const float* w,
@@ -170,6 +171,24 @@ csa_status lightning_index_topk(const csa_params* p, int Q, const uint8_t* q_idx
                                 const int64_t* pos_q, int32_t* topk_idx, int32_t* topk_cnt,
                                 float* scores_out, void* ws, size_t ws_bytes,
                                 int32_t* dev_status, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * The two halves of lightning_index_topk, for callers that want the scores
+ * themselves or their own selection: lightning_index_scores writes the fp32
+ * scores of the visible entries (others untouched); topk_select ranks the
+ * first n_vis = floor((pos_q+1)/m) scores of every row with the same rule
+ * and output as lightning_index_topk.  Running the two in order gives the
+ * same result as lightning_index_topk.
+ *   scores [B, Q, N_cap] fp32 (device; written / read).
+ * ------------------------------------------------------------------------- */
+csa_status lightning_index_scores(const csa_params* p, int Q, const uint8_t* q_idx,
+                                  const float* q_scale, const float* w, const uint8_t* idx_key,
+                                  const float* idx_scale, int64_t N_cap, const int64_t* pos_q,
+                                  float* scores, int32_t* dev_status, void* stream);
+
+csa_status topk_select(const csa_params* p, int Q, const float* scores, int64_t N_cap,
+                       const int64_t* pos_q, int32_t* topk_idx, int32_t* topk_cnt,
+                       int32_t* dev_status, void* stream);
 
 /* ---------------------------------------------------------------------------
  * Shared-KV multi-query attention over selected entries + window + sink
