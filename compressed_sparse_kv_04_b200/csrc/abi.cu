@@ -74,10 +74,9 @@ csa_status check_attention(const char* fn, const csa_params* p) {
     return fail(CSA_ERR_UNSUPPORTED_SHAPE, "%s: H=%d (supported: 1..128)", fn, p->H);
   if (p->window < 0 || p->window > 1024)
     return fail(CSA_ERR_UNSUPPORTED_SHAPE, "%s: window=%d (supported: 0..1024)", fn, p->window);
-  if (p->rope_dim < 0 || (p->rope_dim & 1) || p->rope_dim > 128 || p->rope_dim > p->d / 2)
+  if ((p->rope_dim != 0 && p->rope_dim != 32 && p->rope_dim != 64) || p->rope_dim > p->d / 4)
     return fail(CSA_ERR_UNSUPPORTED_SHAPE,
-                "%s: rope_dim=%d (supported: even, <= 128, within the upper half of d)", fn,
-                p->rope_dim);
+                "%s: rope_dim=%d (supported: 0, 32, 64, and at most d/4)", fn, p->rope_dim);
   if (p->softmax_scale < 0.f || !std::isfinite(p->softmax_scale))
     return fail(CSA_ERR_INVALID_ARG, "%s: softmax_scale must be finite and >= 0", fn);
   return CSA_OK;

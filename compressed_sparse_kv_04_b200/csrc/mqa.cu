@@ -127,8 +127,102 @@ CSA_DEV bool wait_all(uint64_t* bar, uint32_t parity, const Params& p, volatile 
   return __all_sync(0xffffffffu, ok);
 }
 
-template <int D>
-__global__ void __launch_bounds__(kThreads, 1)
+
+// Query prologue: qhat = RoPE(RMSNorm(q) * gamma_q), this CTA's half of every
+// head row, into TMEM (bf16 pairs, the A operand of S = Qhat K^T).  Two
+// threads share a head row: part 0 (a transform-warp thread) takes the first
+// quarter of the row, part 1 (a softmax-warp thread, which also owns the
+// rotated dims) the second; both sit in warps of the head's TMEM lane
+// quarter.  All loads of a thread are in flight at once.  The half-row sums
+// of squares are combined in the CTA (part 0 + part 1) and then with the peer
+// CTA through distributed shared memory, always in rank order, so both CTAs
+// normalise with the same bits.
+template <int D, int R>
+CSA_DEV void q_prologue(const Params& p, int part, int h, int row, uint32_t rank, uint32_t peer,
+                        int64_t pos, uint32_t t_q, float* pss, float* qss_in, uint64_t* qssbar,
+                        uint64_t* qready, volatile int* abort_flag) {
+  using C = MCfg<D>;
+  constexpr int NU = C::Dh / 16;  // 16-byte units per quarter row
+  const bool head_ok = h < p.H;
+  const int e0 = part * (C::Dh / 2);  // first element of this thread's quarter
+  const __nv_bfloat16* qr =
+      p.q + ((int64_t)row * p.H + (head_ok ? h : 0)) * D + rank * C::Dh + e0;
+  uint4 u[NU];
+#pragma unroll
+  for (int c = 0; c < NU; ++c) u[c] = __ldg(reinterpret_cast<const uint4*>(qr) + c);
+  float ss = 0.f;
+#pragma unroll
+  for (int c = 0; c < NU; ++c) {
+    const uint32_t w4[4] = {u[c].x, u[c].y, u[c].z, u[c].w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float lo = bf16_lo(w4[q]), hi = bf16_hi(w4[q]);
+      ss = fmaf(lo, lo, fmaf(hi, hi, ss));
+    }
+  }
+  pss[part * 128 + h] = ss;
+  named_barrier_sync(2, 256);  // the 128 part-0 and 128 part-1 threads
+  const float half_ss = pss[h] + pss[128 + h];
+  if (part == 1) {
+    const uint32_t dst = mapa(smem_u32(&qss_in[h]), peer);
+    asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(dst), "f"(half_ss) : "memory");
+    mbar_arrive_remote(mapa(smem_u32(qssbar), peer));
+  }
+  mbar_wait<true>(qssbar, 0, p.status, abort_flag);
+  const float other = qss_in[h];
+  const float tot = rank == 0 ? half_ss + other : other + half_ss;
+  const float inv = head_ok ? 1.0f / sqrtf(tot / (float)D + p.eps) : 0.f;
+  const int dbase = rank * C::Dh + e0;
+  const uint32_t lane_base = (uint32_t)(h & ~31) << 16;
+  // Element e of the quarter row: unit e/8, word (e%8)/2, low/high half.
+  auto elem = [&](int e) -> float {
+    const uint4& v = u[e >> 3];
+    const int wi = (e >> 1) & 3;
+    const uint32_t wd = wi == 0 ? v.x : wi == 1 ? v.y : wi == 2 ? v.z : v.w;
+    const float x = (e & 1) ? bf16_hi(wd) : bf16_lo(wd);
+    return x * inv * (p.gamma_q ? __ldg(p.gamma_q + dbase + e) : 1.f);
+  };
+  constexpr int Qn = C::Dh / 2;                              // elements per quarter row
+  const bool roped = R > 0 && rank == 1 && part == 1;      // rotated dims: end of the half
+  const int plain_end = roped ? Qn - R : Qn;
+#pragma unroll
+  for (int c0 = 0; c0 < Qn; c0 += 32) {
+    if (c0 >= plain_end) continue;
+    uint32_t pk[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) pk[j] = pack_bf16(elem(c0 + 2 * j), elem(c0 + 2 * j + 1));
+    tmem_st16(t_q + lane_base + (e0 + c0) / 2, pk);
+  }
+  if constexpr (R > 0) {
+    if (roped) {
+      constexpr int half = R / 2;
+      constexpr int b0 = Qn - R;
+#pragma unroll
+      for (int j0 = 0; j0 < half; j0 += 16) {
+        uint32_t pk1[8], pk2[8];
+#pragma unroll
+        for (int j = 0; j < 16; j += 2) {
+          float s0, c0, s1, c1;
+          sincos_reduced((double)pos * p.inv_freq[j0 + j], &s0, &c0);
+          sincos_reduced((double)pos * p.inv_freq[j0 + j + 1], &s1, &c1);
+          const float a0 = elem(b0 + j0 + j), b0v = elem(b0 + half + j0 + j);
+          const float a1 = elem(b0 + j0 + j + 1), b1v = elem(b0 + half + j0 + j + 1);
+          pk1[j / 2] = pack_bf16(a0 * c0 - b0v * s0, a1 * c1 - b1v * s1);
+          pk2[j / 2] = pack_bf16(b0v * c0 + a0 * s0, b1v * c1 + a1 * s1);
+        }
+        // Columns hold bf16 pairs: local dim d -> column d/2 (8 columns each).
+        tmem_st8(t_q + lane_base + (e0 + b0 + j0) / 2, pk1);
+        tmem_st8(t_q + lane_base + (e0 + b0 + half + j0) / 2, pk2);
+      }
+    }
+  }
+  tmem_wait_st();
+  tc_fence_before();
+  mbar_arrive(qready);
+}
+
+template <int D, int R>
+__global__ void __maxnreg__(200)
     mqa_pair_kernel(const __grid_constant__ CUtensorMap map_c,
                     const __grid_constant__ CUtensorMap map_t, const Params p) {
   using C = MCfg<D>;
@@ -149,7 +243,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* pvdone = xempty + 2;
   uint64_t* qready = pvdone + 1;
   uint64_t* drain = qready + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* qssbar = drain + 1;
+  float* qss_in = reinterpret_cast<float*>(qssbar + 1);  // [128] peer's half-row sums
+  float* pss = qss_in + 128;                               // [2][128] quarter-row sums
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(pss + 256);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -203,8 +300,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&xempty[a], 128);
     }
     mbar_init(pvdone, 1);
-    mbar_init(qready, 128);
+    mbar_init(qready, 256);
     mbar_init(drain, 1);
+    mbar_init(qssbar, 128);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -337,8 +435,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Two threads per tile row: `half` 0 takes the window-norm sum and the
     // first half of the rotated pairs, `half` 1 the second half.
     const int tid = threadIdx.x - 64;  // 0..127
+    q_prologue<D, R>(p, 0, (warp & 3) * 32 + lane, row, rank, peer, pos, tmem, pss, qss_in,
+                     qssbar, qready, abort_flag);
     const int r = tid >> 1, hf = tid & 1;
-    const bool rope_here = (p.R > 0) && rank == 1;
+    const bool rope_here = (R > 0) && rank == 1;
     for (int it = 0; it < ntile; ++it) {
       const int s = it % C::kStages;
       if (!wait_all(&full[s], (it / C::kStages) & 1, p, abort_flag)) break;
@@ -370,8 +470,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (hf == 0) meta[s].ss[r] = ss;
       __syncwarp();  // gain-scaled values are in place before the rotation reads them
       if (valid && rope_here) {
-        const int half = p.R / 2;
-        const int d0 = C::Dh - p.R;
+        constexpr int half = R / 2;
+        constexpr int d0 = C::Dh - R;
         const double ppos = (double)M.pos[r];
         for (int j = hf; j < half; j += 2) {
           float sn, cs;
@@ -392,71 +492,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int h = quarter * 32 + lane;  // head == TMEM lane
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
     const bool head_ok = h < p.H;
-    // Query prologue: qhat = RoPE(RMSNorm(q) * gamma_q), this CTA's half -> TMEM.
-    {
-      const __nv_bfloat16* qr = p.q + ((int64_t)row * p.H + (head_ok ? h : 0)) * D;
-      float ss = 0.f;
-      for (int c = 0; c < D / 8; ++c) {
-        uint4 u = __ldg(reinterpret_cast<const uint4*>(qr) + c);
-        uint32_t w4[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          float lo = bf16_lo(w4[q]), hi = bf16_hi(w4[q]);
-          ss = fmaf(lo, lo, fmaf(hi, hi, ss));
-        }
-      }
-      const float inv = head_ok ? 1.0f / sqrtf(ss / (float)D + p.eps) : 0.f;
-      const int dbase = rank * C::Dh;
-      const int d_rope = C::Dh - ((rank == 1) ? p.R : 0);  // local start of rotated dims
-      // Plain dims in chunks of 32.
-      for (int c0 = 0; c0 < d_rope; c0 += 32) {
-        uint32_t pk[16];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          uint4 v = __ldg(reinterpret_cast<const uint4*>(qr + dbase + c0 + u * 8));
-          uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const int d = dbase + c0 + u * 8 + 2 * q;
-            float g0 = p.gamma_q ? __ldg(p.gamma_q + d) : 1.f;
-            float g1 = p.gamma_q ? __ldg(p.gamma_q + d + 1) : 1.f;
-            pk[u * 4 + q] = pack_bf16(bf16_lo(w4[q]) * inv * g0, bf16_hi(w4[q]) * inv * g1);
-          }
-        }
-        tmem_st16(t_q + lane_base + c0 / 2, pk);
-      }
-      // Rotated dims (this CTA holds them only when rank == 1).
-      if (d_rope < C::Dh) {
-        const int half = p.R / 2;
-        for (int j0 = 0; j0 < half; j0 += 16) {
-          // pairs j0..j0+15: dims d_rope+j and d_rope+half+j
-          float x1[16], x2[16];
-#pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const int d1 = dbase + d_rope + j0 + j, d2 = d1 + half;
-            float g1 = p.gamma_q ? __ldg(p.gamma_q + d1) : 1.f;
-            float g2 = p.gamma_q ? __ldg(p.gamma_q + d2) : 1.f;
-            x1[j] = __bfloat162float(qr[d1]) * inv * g1;
-            x2[j] = __bfloat162float(qr[d2]) * inv * g2;
-          }
-          uint32_t pk1[8], pk2[8];
-#pragma unroll
-          for (int j = 0; j < 16; j += 2) {
-            float s0, c0, s1, c1;
-            sincos_reduced((double)pos * p.inv_freq[j0 + j], &s0, &c0);
-            sincos_reduced((double)pos * p.inv_freq[j0 + j + 1], &s1, &c1);
-            pk1[j / 2] = pack_bf16(x1[j] * c0 - x2[j] * s0, x1[j + 1] * c1 - x2[j + 1] * s1);
-            pk2[j / 2] = pack_bf16(x2[j] * c0 + x1[j] * s0, x2[j + 1] * c1 + x1[j + 1] * s1);
-          }
-          // Columns hold bf16 pairs: local dim d -> column d/2 (8 columns each).
-          tmem_st8(t_q + lane_base + (d_rope + j0) / 2, pk1);
-          tmem_st8(t_q + lane_base + (d_rope + half + j0) / 2, pk2);
-        }
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(qready);
-    }
+    q_prologue<D, R>(p, 1, h, row, rank, peer, pos, t_q, pss, qss_in, qssbar, qready,
+                     abort_flag);
 
     float m_run = -INFINITY, l_run = 0.f;
     const uint32_t x_peer_base = mapa(smem_u32(&xs[0]), peer);
@@ -663,7 +700,7 @@ __global__ void mqa_combine_kernel(const Params p, int D, const float* __restric
   if (lse && threadIdx.x == 0) lse[(int64_t)row * p.H + h] = (M + log2f(L)) / LOG2E;
 }
 
-template <int D>
+template <int D, int R>
 cudaError_t launch_impl(const MqaLaunch& a, cudaStream_t stream) {
   using C = MCfg<D>;
   Params p{};
@@ -701,9 +738,9 @@ cudaError_t launch_impl(const MqaLaunch& a, cudaStream_t stream) {
   if (e != cudaSuccess) return e;
 
   const size_t smem = 1024 + (size_t)C::kStages * C::kStageBytes + 2 * sizeof(XSlot) +
-                      C::kStages * sizeof(Meta) + 32 * 8 + 16;
-  auto kern = mqa_pair_kernel<D>;
-  e = ensure_smem_attr(reinterpret_cast<const void*>(kern), D == 512 ? 3 : 4, smem);
+                      C::kStages * sizeof(Meta) + 32 * 8 + 384 * 4 + 16;
+  auto kern = mqa_pair_kernel<D, R>;
+  e = ensure_smem_attr(reinterpret_cast<const void*>(kern), 3 + (D == 512 ? 0 : 3) + R / 32, smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(2 * a.splits, rows, 1);
@@ -727,8 +764,14 @@ cudaError_t launch_impl(const MqaLaunch& a, cudaStream_t stream) {
 }  // namespace
 
 cudaError_t launch_mqa(const MqaLaunch& a, cudaStream_t stream) {
-  if (a.D == 512) return launch_impl<512>(a, stream);
-  if (a.D == 128) return launch_impl<128>(a, stream);
+  if (a.D == 512) {
+    if (a.rope_dim == 64) return launch_impl<512, 64>(a, stream);
+    if (a.rope_dim == 32) return launch_impl<512, 32>(a, stream);
+    if (a.rope_dim == 0) return launch_impl<512, 0>(a, stream);
+  } else if (a.D == 128) {
+    if (a.rope_dim == 32) return launch_impl<128, 32>(a, stream);
+    if (a.rope_dim == 0) return launch_impl<128, 0>(a, stream);
+  }
   return cudaErrorInvalidValue;
 }
 

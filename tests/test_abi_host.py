@@ -88,7 +88,7 @@ def test_indexer_shape_limits(L):
 
 
 def test_attention_shape_limits(L):
-    for kw in (dict(H=129), dict(rope_dim=63), dict(rope_dim=512), dict(window=-1)):
+    for kw in (dict(H=129), dict(rope_dim=63), dict(rope_dim=512), dict(rope_dim=128), dict(window=-1)):
         p = P(**kw)
         st = L.dense_mqa_decode(C.byref(p), None, None, None, 1, None, 1, None, None, None,
                                 None, None, None, 0, None, None)
