@@ -222,7 +222,7 @@ CSA_DEV void q_prologue(const Params& p, int part, int h, int row, uint32_t rank
 }
 
 template <int D, int R>
-__global__ void __maxnreg__(200)
+__global__ void __launch_bounds__(kThreads, 1)
     mqa_pair_kernel(const __grid_constant__ CUtensorMap map_c,
                     const __grid_constant__ CUtensorMap map_t, const Params p) {
   using C = MCfg<D>;
