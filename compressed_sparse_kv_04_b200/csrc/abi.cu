@@ -104,13 +104,9 @@ float softmax_scale_of(const csa_params* p) {
   return p->softmax_scale > 0.f ? p->softmax_scale : (float)(1.0 / std::sqrt((double)p->d));
 }
 
-int64_t max_kv_rows(const csa_params* p, csa_op op, int64_t N_cap) {
-  int64_t n = (op == CSA_OP_DENSE_MQA) ? N_cap : (int64_t)p->k;
-  return n + p->window;
-}
-
 int splits_for(const csa_params* p, csa_op op, int rows, int64_t N_cap) {
-  return csa::mqa_choose_splits(rows, max_kv_rows(p, op, N_cap), csa::device_sm_count());
+  const int64_t compressed_max = (op == CSA_OP_DENSE_MQA) ? N_cap : (int64_t)p->k;
+  return csa::mqa_choose_splits(rows, compressed_max, p->window, csa::device_sm_count());
 }
 
 }  // namespace

@@ -326,13 +326,19 @@ CSA_DEV uint32_t pack_bf16(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-// Reduce an angle (radians, fp64) into [-pi, pi] and return its sine/cosine
-// in fp32.  The reduction is done in fp64 so that positions up to 2^20 keep
-// their phase.
+// sin / cos of a RoPE angle (radians, fp64).  The angle is reduced to
+// [-pi, pi] in fp64 with a two-constant Cody-Waite step (2*pi split into its
+// fp64 value and the remainder), so positions up to 2^20 keep their phase;
+// the reduced angle is then evaluated with the fast single-precision
+// intrinsic, whose absolute error on [-pi, pi] is about 2^-21.
 CSA_DEV void sincos_reduced(double ang, float* s, float* c) {
-  const double two_pi = 6.283185307179586476925286766559;
-  double r = ang - two_pi * rint(ang / two_pi);
-  sincosf((float)r, s, c);
+  const double kInv2Pi = 0.15915494309189533577;
+  const double k2PiHi = 6.283185307179586232;     // fp64 nearest to 2*pi
+  const double k2PiLo = 2.4492935982947064e-16;   // 2*pi - k2PiHi
+  const double k = rint(ang * kInv2Pi);
+  double r = fma(-k, k2PiHi, ang);
+  r = fma(-k, k2PiLo, r);
+  __sincosf((float)r, s, c);
 }
 
 }  // namespace csa

@@ -85,7 +85,7 @@ struct MqaLaunch {
   int32_t* status;
 };
 size_t mqa_workspace_bytes(int rows, int splits, int H, int D);
-int mqa_choose_splits(int rows, int64_t max_kv, int num_sms);
+int mqa_choose_splits(int rows, int64_t compressed_max, int window, int num_sms);
 cudaError_t launch_mqa(const MqaLaunch& a, cudaStream_t stream);
 
 int device_sm_count();

@@ -44,12 +44,16 @@ size_t mqa_workspace_bytes(int rows, int splits, int H, int D) {
   return o + (size_t)rows * splits * 2 * H * 4;
 }
 
-int mqa_choose_splits(int rows, int64_t max_kv, int num_sms) {
-  int64_t tiles = (max_kv + 63) / 64 + 1;
-  int pairs = std::max(1, num_sms / 2);
-  int64_t s = (pairs + rows - 1) / rows;
-  s = std::min<int64_t>(s, tiles);
-  return (int)std::max<int64_t>(1, s);
+// Splits of each row's KV list over CTA pairs: at most one wave of pairs
+// (rows * splits <= SMs / 2), no split left without a tile.
+int mqa_choose_splits(int rows, int64_t compressed_max, int window, int num_sms) {
+  const int64_t tiles = (compressed_max + 63) / 64 + (window + 63) / 64;
+  const int64_t pairs = std::max(1, num_sms / 2);
+  int64_t s = std::max<int64_t>(1, pairs / std::max(1, rows));
+  s = std::min<int64_t>(s, std::max<int64_t>(1, tiles));
+  const int64_t tps = (tiles + s - 1) / s;
+  s = std::max<int64_t>(1, (tiles + tps - 1) / tps);
+  return (int)s;
 }
 
 namespace {
@@ -174,41 +178,57 @@ CSA_DEV void q_prologue(const Params& p, int part, int h, int row, uint32_t rank
   const float inv = head_ok ? 1.0f / sqrtf(tot / (float)D + p.eps) : 0.f;
   const int dbase = rank * C::Dh + e0;
   const uint32_t lane_base = (uint32_t)(h & ~31) << 16;
-  // Element e of the quarter row: unit e/8, word (e%8)/2, low/high half.
-  auto elem = [&](int e) -> float {
-    const uint4& v = u[e >> 3];
-    const int wi = (e >> 1) & 3;
-    const uint32_t wd = wi == 0 ? v.x : wi == 1 ? v.y : wi == 2 ? v.z : v.w;
-    const float x = (e & 1) ? bf16_hi(wd) : bf16_lo(wd);
-    return x * inv * (p.gamma_q ? __ldg(p.gamma_q + dbase + e) : 1.f);
-  };
-  constexpr int Qn = C::Dh / 2;                              // elements per quarter row
-  const bool roped = R > 0 && rank == 1 && part == 1;      // rotated dims: end of the half
-  const int plain_end = roped ? Qn - R : Qn;
+  const float* gq = p.gamma_q ? p.gamma_q + dbase : nullptr;
+  // 8 normalised elements of unit c (re-read: the lines are in L1 by now).
+  auto unit8 = [&](int c, float (&x)[8]) {
+    const uint4 v = __ldg(reinterpret_cast<const uint4*>(qr) + c);
+    const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-  for (int c0 = 0; c0 < Qn; c0 += 32) {
-    if (c0 >= plain_end) continue;
+    for (int q = 0; q < 4; ++q) {
+      x[2 * q] = bf16_lo(w4[q]) * inv;
+      x[2 * q + 1] = bf16_hi(w4[q]) * inv;
+    }
+    if (gq) {
+      const float4 g0 = __ldg(reinterpret_cast<const float4*>(gq + 8 * c));
+      const float4 g1 = __ldg(reinterpret_cast<const float4*>(gq + 8 * c + 4));
+      x[0] *= g0.x; x[1] *= g0.y; x[2] *= g0.z; x[3] *= g0.w;
+      x[4] *= g1.x; x[5] *= g1.y; x[6] *= g1.z; x[7] *= g1.w;
+    }
+  };
+  constexpr int Qn = C::Dh / 2;                         // elements per quarter row
+  const bool roped = R > 0 && rank == 1 && part == 1;  // rotated dims: end of the half
+  const int plain_end = roped ? Qn - R : Qn;
+#pragma unroll 1
+  for (int c0 = 0; c0 < plain_end; c0 += 32) {
     uint32_t pk[16];
 #pragma unroll
-    for (int j = 0; j < 16; ++j) pk[j] = pack_bf16(elem(c0 + 2 * j), elem(c0 + 2 * j + 1));
+    for (int u4 = 0; u4 < 4; ++u4) {
+      float x[8];
+      unit8(c0 / 8 + u4, x);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) pk[u4 * 4 + q] = pack_bf16(x[2 * q], x[2 * q + 1]);
+    }
     tmem_st16(t_q + lane_base + (e0 + c0) / 2, pk);
   }
   if constexpr (R > 0) {
     if (roped) {
       constexpr int half = R / 2;
       constexpr int b0 = Qn - R;
-#pragma unroll
+#pragma unroll 1
       for (int j0 = 0; j0 < half; j0 += 16) {
+        float a[16], b[16];
+        unit8((b0 + j0) / 8, *reinterpret_cast<float(*)[8]>(a));
+        unit8((b0 + j0) / 8 + 1, *reinterpret_cast<float(*)[8]>(a + 8));
+        unit8((b0 + half + j0) / 8, *reinterpret_cast<float(*)[8]>(b));
+        unit8((b0 + half + j0) / 8 + 1, *reinterpret_cast<float(*)[8]>(b + 8));
         uint32_t pk1[8], pk2[8];
 #pragma unroll
         for (int j = 0; j < 16; j += 2) {
           float s0, c0, s1, c1;
           sincos_reduced((double)pos * p.inv_freq[j0 + j], &s0, &c0);
           sincos_reduced((double)pos * p.inv_freq[j0 + j + 1], &s1, &c1);
-          const float a0 = elem(b0 + j0 + j), b0v = elem(b0 + half + j0 + j);
-          const float a1 = elem(b0 + j0 + j + 1), b1v = elem(b0 + half + j0 + j + 1);
-          pk1[j / 2] = pack_bf16(a0 * c0 - b0v * s0, a1 * c1 - b1v * s1);
-          pk2[j / 2] = pack_bf16(b0v * c0 + a0 * s0, b1v * c1 + a1 * s1);
+          pk1[j / 2] = pack_bf16(a[j] * c0 - b[j] * s0, a[j + 1] * c1 - b[j + 1] * s1);
+          pk2[j / 2] = pack_bf16(b[j] * c0 + a[j] * s0, b[j + 1] * c1 + a[j + 1] * s1);
         }
         // Columns hold bf16 pairs: local dim d -> column d/2 (8 columns each).
         tmem_st8(t_q + lane_base + (e0 + b0 + j0) / 2, pk1);
@@ -499,58 +519,61 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t x_peer_base = mapa(smem_u32(&xs[0]), peer);
     const uint32_t xfull_peer = mapa(smem_u32(&xfull[0]), peer);
     const uint32_t xempty_peer = mapa(smem_u32(&xempty[0]), peer);
-    bool alive = true;
-    for (int it = 0; it < ntile && alive; ++it) {
+    for (int it = 0; it < ntile; ++it) {
       const int s = it % C::kStages, a = it & 1;
+      const uint32_t t_sa = t_s + lane_base + a * TN;
       if (!wait_all(&sfull[a], (it >> 1) & 1, p, abort_flag)) break;
       tc_fence_after();
-      float sv[TN];
-      {
-        uint32_t v[32];
-        tmem_ld32(t_s + lane_base + a * TN, v);
-        tmem_wait_ld();
-#pragma unroll
-        for (int j = 0; j < 32; ++j) sv[j] = __uint_as_float(v[j]);
-        tmem_ld32(t_s + lane_base + a * TN + 32, v);
-        tmem_wait_ld();
-#pragma unroll
-        for (int j = 0; j < 32; ++j) sv[32 + j] = __uint_as_float(v[j]);
-      }
       if (!wait_all(&ready[s], (it / C::kStages) & 1, p, abort_flag)) break;
-      // Exchange partial logits with the peer (slot a).
+      // Send this CTA's partial logits (and window half-row sums) to the peer.
       if (!wait_all<true>(&xempty[a], ((it >> 1) & 1) ^ 1, p, abort_flag)) break;
       {
-        const uint32_t dst = x_peer_base + (uint32_t)(a * sizeof(XSlot)) + (uint32_t)(h * kXStride * 4);
+        const uint32_t dst =
+            x_peer_base + (uint32_t)(a * sizeof(XSlot)) + (uint32_t)(h * kXStride * 4);
+#pragma unroll 1
+        for (int c = 0; c < TN; c += 16) {
+          uint32_t v[16];
+          tmem_ld16(t_sa + c, v);
+          tmem_wait_ld();
 #pragma unroll
-        for (int j = 0; j < TN; j += 4) st_cluster_v4(dst + j * 4, sv[j], sv[j + 1], sv[j + 2], sv[j + 3]);
+          for (int j = 0; j < 16; j += 4)
+            st_cluster_v4(dst + (c + j) * 4, __uint_as_float(v[j]), __uint_as_float(v[j + 1]),
+                          __uint_as_float(v[j + 2]), __uint_as_float(v[j + 3]));
+        }
         if (h < TN) {
           const uint32_t dss = x_peer_base + (uint32_t)(a * sizeof(XSlot)) +
                                (uint32_t)offsetof(XSlot, ss) + (uint32_t)(h * 4);
-          asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(dss), "f"(meta[s].ss[h]) : "memory");
+          asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(dss), "f"(meta[s].ss[h])
+                       : "memory");
         }
         mbar_arrive_remote(xfull_peer + a * 8);
       }
       if (!wait_all<true>(&xfull[a], (it >> 1) & 1, p, abort_flag)) break;
       const Meta& M = meta[s];
       const bool win = M.window != 0;
-      // Window-token RMSNorm factor 1/rms(c_t) of column j: the two half sums
-      // are added in rank order, so both CTAs get the same bits.  No CTA-wide
-      // barrier is used here: every wait in this loop must stay bounded.
-      auto norm_factor = [&](int j) -> float {
-        const float ssum = rank == 0 ? M.ss[j] + xs[a].ss[j] : xs[a].ss[j] + M.ss[j];
-        return 1.0f / sqrtf(ssum / (float)D + p.eps);
-      };
       const float* xr = xs[a].s + h * kXStride;
-      float mt = -INFINITY;
-#pragma unroll
-      for (int j = 0; j < TN; ++j) {
+      const float* xss = xs[a].ss;
+      // Logit of column j from this CTA's partial (own) and the peer's; the
+      // two halves are added in rank order so both CTAs get the same bits,
+      // and the window-token norm 1/rms(c_t) uses the half sums the same way.
+      auto logit = [&](float own, int j) -> float {
         const float other = xr[j];
-        float v = rank == 0 ? sv[j] + other : other + sv[j];
-        if (win) v *= norm_factor(j);
+        float v = rank == 0 ? __fadd_rn(own, other) : __fadd_rn(other, own);
+        if (win) {
+          const float ssum = rank == 0 ? __fadd_rn(M.ss[j], xss[j]) : __fadd_rn(xss[j], M.ss[j]);
+          v = __fmul_rn(v, rsqrtf(__fadd_rn(__fmul_rn(ssum, 1.0f / (float)D), p.eps)));
+        }
         const bool valid = (M.valid[j >> 5] >> (j & 31)) & 1u;
-        v = valid ? v * p.scale_log2 : -INFINITY;  // log2 domain
-        sv[j] = v;
-        mt = fmaxf(mt, v);
+        return valid ? __fmul_rn(v, p.scale_log2) : -INFINITY;  // log2 domain
+      };
+      float mt = -INFINITY;
+#pragma unroll 1
+      for (int c = 0; c < TN; c += 16) {
+        uint32_t v[16];
+        tmem_ld16(t_sa + c, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 16; ++j) mt = fmaxf(mt, logit(__uint_as_float(v[j]), c + j));
       }
       // Online softmax with lazy rescaling (log2 domain).
       const bool grow = mt > m_run + kRescaleThreshold * 1.4426950408889634f || m_run == -INFINITY;
@@ -565,49 +588,47 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (__any_sync(0xffffffffu, need) && it > 0) {
         const float f = need ? exp2f(m_run - m_new) : 1.f;
-        for (int c = 0; c < C::Dh; c += 32) {
-          uint32_t v[32];
-          tmem_ld32(t_o + lane_base + c, v);
+#pragma unroll 1
+        for (int c = 0; c < C::Dh; c += 16) {
+          uint32_t v[16];
+          tmem_ld16(t_o + lane_base + c, v);
           tmem_wait_ld();
 #pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * f);
-          uint32_t v0[16], v1[16];
-#pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            v0[j] = v[j];
-            v1[j] = v[16 + j];
-          }
-          tmem_st16(t_o + lane_base + c, v0);
-          tmem_st16(t_o + lane_base + c + 16, v1);
+          for (int j = 0; j < 16; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * f);
+          tmem_st16(t_o + lane_base + c, v);
         }
         tmem_wait_st();
       }
       if (need) l_run *= exp2f(m_run - m_new);
       m_run = m_new;
+      // P = exp2(logit - m) in bf16 (times the window norm, since V = norm *
+      // the stored row), written over the consumed S columns.
       float lsum = 0.f;
-      uint32_t pk[32];
+#pragma unroll 1
+      for (int c = 0; c < TN; c += 16) {
+        uint32_t v[16];
+        tmem_ld16(t_sa + c, v);
+        tmem_wait_ld();
+        uint32_t pk[8];
 #pragma unroll
-      for (int j = 0; j < TN; j += 2) {
-        float p0 = m_run == -INFINITY ? 0.f : exp2f(sv[j] - m_run);
-        float p1 = m_run == -INFINITY ? 0.f : exp2f(sv[j + 1] - m_run);
-        lsum += p0 + p1;
-        if (win) {
-          p0 *= norm_factor(j);
-          p1 *= norm_factor(j + 1);
+        for (int j = 0; j < 16; j += 2) {
+          const float l0 = logit(__uint_as_float(v[j]), c + j);
+          const float l1 = logit(__uint_as_float(v[j + 1]), c + j + 1);
+          float p0 = m_run == -INFINITY ? 0.f : exp2f(l0 - m_run);
+          float p1 = m_run == -INFINITY ? 0.f : exp2f(l1 - m_run);
+          lsum += p0 + p1;
+          if (win) {
+            const int j0 = c + j, j1 = c + j + 1;
+            const float s0 = rank == 0 ? __fadd_rn(M.ss[j0], xss[j0]) : __fadd_rn(xss[j0], M.ss[j0]);
+            const float s1 = rank == 0 ? __fadd_rn(M.ss[j1], xss[j1]) : __fadd_rn(xss[j1], M.ss[j1]);
+            p0 *= rsqrtf(__fadd_rn(__fmul_rn(s0, 1.0f / (float)D), p.eps));
+            p1 *= rsqrtf(__fadd_rn(__fmul_rn(s1, 1.0f / (float)D), p.eps));
+          }
+          pk[j / 2] = pack_bf16(p0, p1);
         }
-        pk[j / 2] = pack_bf16(p0, p1);
+        tmem_st8(t_sa + c / 2, pk);  // columns c/2 .. c/2+7: already consumed
       }
       l_run += lsum;
-      {
-        uint32_t v0[16], v1[16];
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          v0[j] = pk[j];
-          v1[j] = pk[16 + j];
-        }
-        tmem_st16(t_s + lane_base + a * TN, v0);
-        tmem_st16(t_s + lane_base + a * TN + 16, v1);
-      }
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&pready[a]);
