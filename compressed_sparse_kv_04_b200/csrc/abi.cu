@@ -64,8 +64,8 @@ csa_status check_indexer(const char* fn, const csa_params* p) {
     return fail(CSA_ERR_UNSUPPORTED_SHAPE, "%s: D_I=%d (supported: 64, 128)", fn, p->D_I);
   if (p->H_I < 1 || p->H_I > 64)
     return fail(CSA_ERR_UNSUPPORTED_SHAPE, "%s: H_I=%d (supported: 1..64)", fn, p->H_I);
-  if (p->k < 1 || p->k > 2048)
-    return fail(CSA_ERR_UNSUPPORTED_SHAPE, "%s: k=%d (supported: 1..2048)", fn, p->k);
+  if (p->k < 1 || p->k > 1024)
+    return fail(CSA_ERR_UNSUPPORTED_SHAPE, "%s: k=%d (supported: 1..1024)", fn, p->k);
   return CSA_OK;
 }
 
@@ -459,8 +459,8 @@ csa_status sparse_mqa_decode(const csa_params* p, const void* q, const int64_t* 
   csa_status st = check_mqa_args(fn, p, q, pos_q, kv_c, N_cap, kv_tok, L_cap, sink, gamma_q,
                                  gamma_kv, out, lse, dev_status);
   if (st != CSA_OK) return st;
-  if (p->k < 1 || p->k > 2048)
-    return fail(CSA_ERR_UNSUPPORTED_SHAPE, "%s: k=%d (supported: 1..2048)", fn, p->k);
+  if (p->k < 1 || p->k > 1024)
+    return fail(CSA_ERR_UNSUPPORTED_SHAPE, "%s: k=%d (supported: 1..1024)", fn, p->k);
   REQ_PTR(topk_idx);
   REQ_PTR4(topk_cnt);
   return mqa_common(fn, p, CSA_OP_SPARSE_MQA, p->B, 1, q, pos_q, 0, kv_c, N_cap, topk_idx,

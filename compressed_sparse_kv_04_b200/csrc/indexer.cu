@@ -216,23 +216,31 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     int it = 0;
     for (int t = t_begin; t < t_end; ++t, ++it) {
-      int a = it & 1;
-      uint32_t aph = (it >> 1) & 1;
+      const int a = it & 1;
+      const uint32_t aph = (it >> 1) & 1;
+      const int64_t entry = (int64_t)t * kTileRows + row;
+      // Issued before the wait so that its latency overlaps the MMA.
+      const float ks = entry < p.N_cap ? __ldg(p.key_scale + (int64_t)b * p.N_cap + entry) : 0.f;
       bool ok = mbar_wait(&tfull[a], aph, p.status, abort_flag);
       if (!__all_sync(0xffffffffu, ok)) break;  // keep the warp converged for tcgen05.ld
       tc_fence_after();
-      const int64_t entry = (int64_t)t * kTileRows + row;
-      const float ks = entry < p.N_cap ? __ldg(p.key_scale + (int64_t)b * p.N_cap + entry) : 0.f;
       for (int g = 0; g < nq; ++g) {
-        float acc = 0.f;
-        for (int c = 0; c < p.HP; c += 16) {
-          uint32_t v[16];
-          tmem_ld16(tmem_addr(tmem, quarter * 32, a * p.N + g * p.HP + c), v);
-          tmem_wait_ld();
+        // All of this query's head columns (<= 64) in flight, one wait.
+        uint32_t v[4][16];
+        const uint32_t col = tmem_addr(tmem, quarter * 32, a * p.N + g * p.HP);
 #pragma unroll
-          for (int j = 0; j < 16; ++j)
-            acc = fmaf(wq[g * p.HP + c + j], fmaxf(__uint_as_float(v[j]), 0.f), acc);
-        }
+        for (int c = 0; c < 4; ++c)
+          if (c * 16 < p.HP) tmem_ld16(col + c * 16, v[c]);
+        tmem_wait_ld();
+        float acc = 0.f;
+        const float* wg = wq + g * p.HP;
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          if (c * 16 < p.HP) {
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+              acc = fmaf(wg[c * 16 + j], fmaxf(__uint_as_float(v[c][j]), 0.f), acc);
+          }
         if (entry < nv[g < 8 ? g : 7])
           p.scores[((int64_t)b * p.Q + q0 + g) * p.N_cap + entry] = acc * ks;
       }

@@ -58,7 +58,7 @@ typedef enum {
 
 /* Shapes and constants shared by the calls of one layer.
  * Supported: d in {128, 512}; 1 <= H <= 128; H_I in {1..64}, D_I in {64, 128}
- * (indexer calls only); 1 <= k <= 2048; 0 <= window <= 1024; rope_dim in
+ * (indexer calls only); 1 <= k <= 1024; 0 <= window <= 1024; rope_dim in
  * {0, 32, 64} and <= d/4 (attention calls); 1 <= m <= 128 (CSA uses 4, HCA
  * 128); eps > 0. */
 typedef struct {

@@ -80,7 +80,7 @@ def test_null_tensor_rejected_before_launch(L):
 
 
 def test_indexer_shape_limits(L):
-    for kw in (dict(D_I=96), dict(H_I=65), dict(k=4096), dict(k=0)):
+    for kw in (dict(D_I=96), dict(H_I=65), dict(k=1025), dict(k=0)):
         p = P(**kw)
         st = L.lightning_index_topk(C.byref(p), 1, None, None, None, None, None, 1024, None,
                                     None, None, None, None, 0, None, None)
