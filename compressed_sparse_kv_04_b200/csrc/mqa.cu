@@ -60,7 +60,7 @@ namespace {
 
 constexpr int TN = 64;           // KV rows per tile
 constexpr int kThreads = 320;    // 10 warps
-constexpr int kXStride = 68;     // padded row (floats) of the S exchange buffer
+constexpr int kXRow = TN;        // floats per head row in an exchange slot
 constexpr float kRescaleThreshold = 8.0f;
 
 template <int D>
@@ -86,10 +86,17 @@ struct Meta {
   int32_t pad;
 };
 
+// One tile's partial logits of all 128 heads (+ the window half-row sums),
+// as staged locally and as received from the peer.  Within a row the 16-byte
+// chunks are XOR-swizzled by the row index so that the 128 threads' vector
+// stores and loads hit distinct banks.
 struct XSlot {
-  float s[128 * kXStride];
+  float s[128 * kXRow];
   float ss[TN];
 };
+CSA_DEV int xoff(int h, int j) {  // float offset of (head h, column j)
+  return h * kXRow + ((((j >> 2) ^ (h & 15)) << 2) | (j & 3));
+}
 
 struct Params {
   int Q, H, m, W, R, splits;
@@ -244,14 +251,17 @@ CSA_DEV void q_prologue(const Params& p, int part, int h, int row, uint32_t rank
 template <int D, int R>
 __global__ void __launch_bounds__(kThreads, 1)
     mqa_pair_kernel(const __grid_constant__ CUtensorMap map_c,
-                    const __grid_constant__ CUtensorMap map_t, const Params p) {
+                    const __grid_constant__ CUtensorMap map_t,
+                    const __grid_constant__ CUtensorMap box_c,
+                    const __grid_constant__ CUtensorMap box_t, const Params p) {
   using C = MCfg<D>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   uint8_t* stages = smem;
   XSlot* xs = reinterpret_cast<XSlot*>(stages + C::kStages * C::kStageBytes);
-  Meta* meta = reinterpret_cast<Meta*>(xs + 2);
+  XSlot* xst = xs + 2;  // local staging of this CTA's partial logits
+  Meta* meta = reinterpret_cast<Meta*>(xs + 3);
   uint64_t* bars = reinterpret_cast<uint64_t*>(meta + C::kStages);
   uint64_t* full = bars;
   uint64_t* ready = full + C::kStages;
@@ -263,7 +273,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* pvdone = xempty + 2;
   uint64_t* qready = pvdone + 1;
   uint64_t* drain = qready + 1;
-  uint64_t* qssbar = drain + 1;
+  uint64_t* staged = drain + 1;
+  uint64_t* qssbar = staged + 1;
   float* qss_in = reinterpret_cast<float*>(qssbar + 1);  // [128] peer's half-row sums
   float* pss = qss_in + 128;                               // [2][128] quarter-row sums
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(pss + 256);
@@ -316,13 +327,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int a = 0; a < 2; ++a) {
       mbar_init(&sfull[a], 1);
       mbar_init(&pready[a], 128);
-      mbar_init(&xfull[a], 128);
-      mbar_init(&xempty[a], 128);
+      mbar_init(&xfull[a], 1);    // own expect_tx + the peer's bulk copy
+      mbar_init(&xempty[a], 128); // the peer's softmax threads
     }
     mbar_init(pvdone, 1);
     mbar_init(qready, 256);
     mbar_init(drain, 1);
     mbar_init(qssbar, 128);
+    mbar_init(staged, 128);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -339,64 +351,79 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     // ---------------------------------------------------------- producer --
+    // Contiguous tiles (dense entries, window tokens) are fetched with four
+    // 64-row box copies; selected entries with row gathers (tile::gather4),
+    // two per lane so the whole warp issues them.
     int it = 0;
     for (int t = t0; t < t1; ++t, ++it) {
       const int s = it % C::kStages;
       const uint32_t ph = (it / C::kStages) & 1;
-      if (!wait_all(&empty[s], ph ^ 1, p, abort_flag)) break;
       const bool win = t >= tiles_c;
-      Meta& M = meta[s];
-      uint32_t vbits[2];
+      const bool gathered = !win && p.sel_idx != nullptr;
+      // Row metadata (loads issued before the slot wait so they overlap it).
+      int32_t grow[2], rpos[2];
+      bool valid[2];
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int r = lane + 32 * h;
-        bool valid;
-        int32_t grow, rpos;
+      for (int hh = 0; hh < 2; ++hh) {
+        const int r = lane + 32 * hh;
         if (!win) {
           const int j = t * TN + r;
-          valid = j < n_c;
+          valid[hh] = j < n_c;
           int64_t i = j;
-          if (valid && p.sel_idx) {
+          if (valid[hh] && gathered) {
             i = p.sel_idx[(int64_t)row * p.kmax + j];
             if (i < 0 || i >= n_vis) {
               report(p.status, CSA_ERR_DEVICE_INDEX);
-              valid = false;
+              valid[hh] = false;
             }
           }
-          if (!valid) i = 0;
-          grow = (int32_t)((int64_t)b * p.N_cap + i);
-          rpos = (int32_t)((i + 1) * p.m - 1);
+          if (!valid[hh] && gathered) i = 0;
+          grow[hh] = (int32_t)((int64_t)b * p.N_cap + i);
+          rpos[hh] = (int32_t)((i + 1) * p.m - 1);
         } else {
           const int j = (t - tiles_c) * TN + r;
-          valid = j < nwin;
-          if (valid && w0 + j >= p.L_cap) {  // query position beyond the token buffer
+          valid[hh] = j < nwin;
+          if (valid[hh] && w0 + j >= p.L_cap) {  // query position beyond the token buffer
             report(p.status, CSA_ERR_CAPACITY);
-            valid = false;
+            valid[hh] = false;
           }
-          const int64_t tok = valid ? w0 + j : 0;
-          grow = (int32_t)((int64_t)b * p.L_cap + tok);
-          rpos = (int32_t)tok;
+          const int64_t tok = w0 + j;
+          grow[hh] = (int32_t)((int64_t)b * p.L_cap + tok);
+          rpos[hh] = (int32_t)tok;
         }
-        M.grow[r] = grow;
-        M.pos[r] = rpos;
-        vbits[h] = __ballot_sync(0xffffffffu, valid);
       }
+      const uint32_t vb0 = __ballot_sync(0xffffffffu, valid[0]);
+      const uint32_t vb1 = __ballot_sync(0xffffffffu, valid[1]);
+      if (!wait_all(&empty[s], ph ^ 1, p, abort_flag)) break;
+      Meta& M = meta[s];
+      M.grow[lane] = grow[0];
+      M.grow[lane + 32] = grow[1];
+      M.pos[lane] = rpos[0];
+      M.pos[lane + 32] = rpos[1];
       if (lane == 0) {
-        M.valid[0] = vbits[0];
-        M.valid[1] = vbits[1];
+        M.valid[0] = vb0;
+        M.valid[1] = vb1;
         M.window = win ? 1 : 0;
+        mbar_expect_tx(&full[s], C::kStageBytes);
       }
       __syncwarp();
-      if (lane == 0) {
-        const CUtensorMap* map = win ? &map_t : &map_c;
-        mbar_expect_tx(&full[s], C::kStageBytes);
-        uint8_t* dst = stages + s * C::kStageBytes;
-#pragma unroll
-        for (int c = 0; c < C::NC; ++c)
-          for (int g = 0; g < TN / 4; ++g)
-            tma_gather4(dst + c * C::kChunkBytes + g * 4 * 128, map, &full[s],
-                        (int32_t)(rank * C::Dh + c * 64), M.grow[4 * g], M.grow[4 * g + 1],
-                        M.grow[4 * g + 2], M.grow[4 * g + 3]);
+      uint8_t* dst = stages + s * C::kStageBytes;
+      if (!gathered) {
+        // Rows grow[0] .. grow[0]+63 are consecutive (rows past the list are
+        // fetched too and masked; rows past the tensor are zero-filled).
+        const int32_t y0 = __shfl_sync(0xffffffffu, grow[0], 0);
+        if (lane < C::NC)
+          tma_load_2d(dst + lane * C::kChunkBytes, win ? &box_t : &box_c, &full[s],
+                      (int32_t)(rank * C::Dh + lane * 64), y0);
+      } else {
+        // 16 groups of 4 rows per 128-byte chunk: lane -> (chunk, 2 groups).
+        constexpr int kGroups = C::NC * (TN / 4);
+        for (int q = lane; q < kGroups; q += 32) {
+          const int c = q / (TN / 4), g = q % (TN / 4);
+          tma_gather4(dst + c * C::kChunkBytes + g * 4 * 128, &map_c, &full[s],
+                      (int32_t)(rank * C::Dh + c * 64), M.grow[4 * g], M.grow[4 * g + 1],
+                      M.grow[4 * g + 2], M.grow[4 * g + 3]);
+        }
       }
     }
     if (*abort_flag && lane == 0) {  // copies still in flight must land first
@@ -490,17 +517,31 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (hf == 0) meta[s].ss[r] = ss;
       __syncwarp();  // gain-scaled values are in place before the rotation reads them
       if (valid && rope_here) {
+        // The rotated dims are the last R of this half row: pairs (j, j+R/2).
+        // Thread half hf rotates pairs [hf*R/4, hf*R/4 + R/4) with 16-byte
+        // shared-memory accesses (8 bf16 per access).
         constexpr int half = R / 2;
         constexpr int d0 = C::Dh - R;
         const double ppos = (double)M.pos[r];
-        for (int j = hf; j < half; j += 2) {
-          float sn, cs;
-          sincos_reduced(ppos * p.inv_freq[j], &sn, &cs);
-          __nv_bfloat16* a1 = reinterpret_cast<__nv_bfloat16*>(st + tile_off(r, d0 + j));
-          __nv_bfloat16* a2 = reinterpret_cast<__nv_bfloat16*>(st + tile_off(r, d0 + j + half));
-          float x1 = __bfloat162float(*a1), x2 = __bfloat162float(*a2);
-          *a1 = __float2bfloat16_rn(x1 * cs - x2 * sn);
-          *a2 = __float2bfloat16_rn(x2 * cs + x1 * sn);
+#pragma unroll
+        for (int q = 0; q < R / 32; ++q) {  // R/4 pairs per thread, 8 per access
+          const int j0 = hf * (half / 2) + q * 8;
+          uint4* pa = reinterpret_cast<uint4*>(st + tile_off(r, d0 + j0));
+          uint4* pb = reinterpret_cast<uint4*>(st + tile_off(r, d0 + half + j0));
+          uint4 ua = *pa, ub = *pb;
+          uint32_t wa[4] = {ua.x, ua.y, ua.z, ua.w}, wb[4] = {ub.x, ub.y, ub.z, ub.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            float s0, c0, s1, c1;
+            sincos_reduced(ppos * p.inv_freq[j0 + 2 * e], &s0, &c0);
+            sincos_reduced(ppos * p.inv_freq[j0 + 2 * e + 1], &s1, &c1);
+            const float x10 = bf16_lo(wa[e]), x11 = bf16_hi(wa[e]);
+            const float x20 = bf16_lo(wb[e]), x21 = bf16_hi(wb[e]);
+            wa[e] = pack_bf16(x10 * c0 - x20 * s0, x11 * c1 - x21 * s1);
+            wb[e] = pack_bf16(x20 * c0 + x10 * s0, x21 * c1 + x11 * s1);
+          }
+          *pa = make_uint4(wa[0], wa[1], wa[2], wa[3]);
+          *pb = make_uint4(wb[0], wb[1], wb[2], wb[3]);
         }
       }
       fence_proxy_async_smem();
@@ -516,64 +557,76 @@ __global__ void __launch_bounds__(kThreads, 1)
                      abort_flag);
 
     float m_run = -INFINITY, l_run = 0.f;
-    const uint32_t x_peer_base = mapa(smem_u32(&xs[0]), peer);
+    const uint32_t xs_peer = mapa(smem_u32(&xs[0]), peer);
     const uint32_t xfull_peer = mapa(smem_u32(&xfull[0]), peer);
     const uint32_t xempty_peer = mapa(smem_u32(&xempty[0]), peer);
+    const bool leader = h == 0;  // issues the bulk copy of the staged logits
     for (int it = 0; it < ntile; ++it) {
       const int s = it % C::kStages, a = it & 1;
       const uint32_t t_sa = t_s + lane_base + a * TN;
       if (!wait_all(&sfull[a], (it >> 1) & 1, p, abort_flag)) break;
       tc_fence_after();
-      if (!wait_all(&ready[s], (it / C::kStages) & 1, p, abort_flag)) break;
-      // Send this CTA's partial logits (and window half-row sums) to the peer.
-      if (!wait_all<true>(&xempty[a], ((it >> 1) & 1) ^ 1, p, abort_flag)) break;
+      float sv[TN];
       {
-        const uint32_t dst =
-            x_peer_base + (uint32_t)(a * sizeof(XSlot)) + (uint32_t)(h * kXStride * 4);
-#pragma unroll 1
-        for (int c = 0; c < TN; c += 16) {
-          uint32_t v[16];
-          tmem_ld16(t_sa + c, v);
-          tmem_wait_ld();
+        uint32_t v[4][16];
 #pragma unroll
-          for (int j = 0; j < 16; j += 4)
-            st_cluster_v4(dst + (c + j) * 4, __uint_as_float(v[j]), __uint_as_float(v[j + 1]),
-                          __uint_as_float(v[j + 2]), __uint_as_float(v[j + 3]));
-        }
-        if (h < TN) {
-          const uint32_t dss = x_peer_base + (uint32_t)(a * sizeof(XSlot)) +
-                               (uint32_t)offsetof(XSlot, ss) + (uint32_t)(h * 4);
-          asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(dss), "f"(meta[s].ss[h])
-                       : "memory");
-        }
-        mbar_arrive_remote(xfull_peer + a * 8);
+        for (int c = 0; c < 4; ++c) tmem_ld16(t_sa + 16 * c, v[c]);
+        tmem_wait_ld();
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+          for (int j = 0; j < 16; ++j) sv[16 * c + j] = __uint_as_float(v[c][j]);
+      }
+      if (!wait_all(&ready[s], (it / C::kStages) & 1, p, abort_flag)) break;
+      // Stage this CTA's partial logits locally, then one bulk copy moves
+      // them into the peer's receive slot a (completing on its xfull[a]).
+      // The staging buffer is free once the peer has consumed the previous
+      // tile (its xempty arrival for tile it-1).
+      if (it > 0 && !wait_all<true>(&xempty[(it - 1) & 1], ((it - 1) >> 1) & 1, p, abort_flag))
+        break;
+      {
+        float* row = xst->s;
+#pragma unroll
+        for (int j = 0; j < TN; j += 4)
+          *reinterpret_cast<float4*>(row + xoff(h, j)) =
+              make_float4(sv[j], sv[j + 1], sv[j + 2], sv[j + 3]);
+        if (h < TN) xst->ss[h] = meta[s].ss[h];
+        fence_proxy_async_smem();
+        mbar_arrive(staged);
+      }
+      if (leader) {
+        // Own receive slot: expect the peer's bytes.
+        mbar_expect_tx(&xfull[a], (uint32_t)sizeof(XSlot));
+        bool ok = mbar_wait(staged, it & 1, p.status, abort_flag);
+        // The peer's slot a is free once it consumed tile it-2.
+        ok = ok && mbar_wait<true>(&xempty[a], ((it >> 1) & 1) ^ 1, p.status, abort_flag);
+        if (ok)
+          asm volatile(
+              "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes"
+              " [%0], [%1], %2, [%3];" ::"r"(xs_peer + (uint32_t)(a * sizeof(XSlot))),
+              "r"(smem_u32(xst)), "r"((uint32_t)sizeof(XSlot)), "r"(xfull_peer + a * 8)
+              : "memory");
       }
       if (!wait_all<true>(&xfull[a], (it >> 1) & 1, p, abort_flag)) break;
       const Meta& M = meta[s];
       const bool win = M.window != 0;
-      const float* xr = xs[a].s + h * kXStride;
-      const float* xss = xs[a].ss;
-      // Logit of column j from this CTA's partial (own) and the peer's; the
-      // two halves are added in rank order so both CTAs get the same bits,
-      // and the window-token norm 1/rms(c_t) uses the half sums the same way.
-      auto logit = [&](float own, int j) -> float {
-        const float other = xr[j];
-        float v = rank == 0 ? __fadd_rn(own, other) : __fadd_rn(other, own);
+      const XSlot& X = xs[a];
+      // Full logits: the two partial sums added in rank order (bit-identical
+      // in both CTAs); window tokens scaled by 1/rms(c_t) from the two half
+      // sums of squares, also added in rank order.
+      float mt = -INFINITY;
+#pragma unroll
+      for (int j = 0; j < TN; ++j) {
+        const float other = X.s[xoff(h, j)];
+        float v = rank == 0 ? __fadd_rn(sv[j], other) : __fadd_rn(other, sv[j]);
         if (win) {
-          const float ssum = rank == 0 ? __fadd_rn(M.ss[j], xss[j]) : __fadd_rn(xss[j], M.ss[j]);
+          const float ssum = rank == 0 ? __fadd_rn(M.ss[j], X.ss[j]) : __fadd_rn(X.ss[j], M.ss[j]);
           v = __fmul_rn(v, rsqrtf(__fadd_rn(__fmul_rn(ssum, 1.0f / (float)D), p.eps)));
         }
         const bool valid = (M.valid[j >> 5] >> (j & 31)) & 1u;
-        return valid ? __fmul_rn(v, p.scale_log2) : -INFINITY;  // log2 domain
-      };
-      float mt = -INFINITY;
-#pragma unroll 1
-      for (int c = 0; c < TN; c += 16) {
-        uint32_t v[16];
-        tmem_ld16(t_sa + c, v);
-        tmem_wait_ld();
-#pragma unroll
-        for (int j = 0; j < 16; ++j) mt = fmaxf(mt, logit(__uint_as_float(v[j]), c + j));
+        v = valid ? __fmul_rn(v, p.scale_log2) : -INFINITY;  // log2 domain
+        sv[j] = v;
+        mt = fmaxf(mt, v);
       }
       // Online softmax with lazy rescaling (log2 domain).
       const bool grow = mt > m_run + kRescaleThreshold * 1.4426950408889634f || m_run == -INFINITY;
@@ -601,38 +654,39 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (need) l_run *= exp2f(m_run - m_new);
       m_run = m_new;
-      // P = exp2(logit - m) in bf16 (times the window norm, since V = norm *
-      // the stored row), written over the consumed S columns.
+      // P = exp2(logit - m) in bf16, times the window norm (V = norm * the
+      // stored row), written over the consumed S columns.
       float lsum = 0.f;
-#pragma unroll 1
-      for (int c = 0; c < TN; c += 16) {
-        uint32_t v[16];
-        tmem_ld16(t_sa + c, v);
-        tmem_wait_ld();
-        uint32_t pk[8];
+      uint32_t pk[TN / 2];
 #pragma unroll
-        for (int j = 0; j < 16; j += 2) {
-          const float l0 = logit(__uint_as_float(v[j]), c + j);
-          const float l1 = logit(__uint_as_float(v[j + 1]), c + j + 1);
-          float p0 = m_run == -INFINITY ? 0.f : exp2f(l0 - m_run);
-          float p1 = m_run == -INFINITY ? 0.f : exp2f(l1 - m_run);
-          lsum += p0 + p1;
-          if (win) {
-            const int j0 = c + j, j1 = c + j + 1;
-            const float s0 = rank == 0 ? __fadd_rn(M.ss[j0], xss[j0]) : __fadd_rn(xss[j0], M.ss[j0]);
-            const float s1 = rank == 0 ? __fadd_rn(M.ss[j1], xss[j1]) : __fadd_rn(xss[j1], M.ss[j1]);
-            p0 *= rsqrtf(__fadd_rn(__fmul_rn(s0, 1.0f / (float)D), p.eps));
-            p1 *= rsqrtf(__fadd_rn(__fmul_rn(s1, 1.0f / (float)D), p.eps));
-          }
-          pk[j / 2] = pack_bf16(p0, p1);
+      for (int j = 0; j < TN; j += 2) {
+        float p0 = m_run == -INFINITY ? 0.f : exp2f(sv[j] - m_run);
+        float p1 = m_run == -INFINITY ? 0.f : exp2f(sv[j + 1] - m_run);
+        lsum += p0 + p1;
+        if (win) {
+          const float s0 = rank == 0 ? __fadd_rn(M.ss[j], X.ss[j]) : __fadd_rn(X.ss[j], M.ss[j]);
+          const float s1 = rank == 0 ? __fadd_rn(M.ss[j + 1], X.ss[j + 1])
+                                     : __fadd_rn(X.ss[j + 1], M.ss[j + 1]);
+          p0 *= rsqrtf(__fadd_rn(__fmul_rn(s0, 1.0f / (float)D), p.eps));
+          p1 *= rsqrtf(__fadd_rn(__fmul_rn(s1, 1.0f / (float)D), p.eps));
         }
-        tmem_st8(t_sa + c / 2, pk);  // columns c/2 .. c/2+7: already consumed
+        pk[j / 2] = pack_bf16(p0, p1);
       }
       l_run += lsum;
+      mbar_arrive_remote(xempty_peer + a * 8);  // receive slot a consumed
+      {
+        uint32_t v0[16], v1[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          v0[j] = pk[j];
+          v1[j] = pk[16 + j];
+        }
+        tmem_st16(t_sa, v0);
+        tmem_st16(t_sa + 16, v1);
+      }
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&pready[a]);
-      mbar_arrive_remote(xempty_peer + a * 8);  // slot a may now be refilled by the peer
     }
     // Epilogue: the O half and (rank 0) the running max / sum.
     if (!*abort_flag && wait_all(pvdone, (ntile - 1) & 1, p, abort_flag)) {
@@ -750,16 +804,23 @@ cudaError_t launch_impl(const MqaLaunch& a, cudaStream_t stream) {
   const int rows = a.B * a.Q;
   if (rows > 65535 || a.splits * 2 > 65535) return cudaErrorInvalidConfiguration;
 
-  CUtensorMap map_c, map_t;
+  // Row-gather maps (one-row boxes) and 64-row box maps, 128-byte swizzle.
+  CUtensorMap map_c, map_t, box_c, box_t;
   cudaError_t e = make_tmap_2d(&map_c, a.kv_c, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
                                (uint64_t)a.B * a.N_cap, D, 1, 64, CU_TENSOR_MAP_SWIZZLE_128B);
   if (e != cudaSuccess) return e;
   e = make_tmap_2d(&map_t, a.kv_tok, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)a.B * a.L_cap,
                    D, 1, 64, CU_TENSOR_MAP_SWIZZLE_128B);
   if (e != cudaSuccess) return e;
+  e = make_tmap_2d(&box_c, a.kv_c, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)a.B * a.N_cap,
+                   D, TN, 64, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (e != cudaSuccess) return e;
+  e = make_tmap_2d(&box_t, a.kv_tok, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)a.B * a.L_cap,
+                   D, TN, 64, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (e != cudaSuccess) return e;
 
-  const size_t smem = 1024 + (size_t)C::kStages * C::kStageBytes + 2 * sizeof(XSlot) +
-                      C::kStages * sizeof(Meta) + 32 * 8 + 384 * 4 + 16;
+  const size_t smem = 1024 + (size_t)C::kStages * C::kStageBytes + 3 * sizeof(XSlot) +
+                      C::kStages * sizeof(Meta) + 40 * 8 + 384 * 4 + 16;
   auto kern = mqa_pair_kernel<D, R>;
   e = ensure_smem_attr(reinterpret_cast<const void*>(kern), 3 + (D == 512 ? 0 : 3) + R / 32, smem);
   if (e != cudaSuccess) return e;
@@ -775,7 +836,7 @@ cudaError_t launch_impl(const MqaLaunch& a, cudaStream_t stream) {
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, kern, map_c, map_t, p);
+  e = cudaLaunchKernelEx(&cfg, kern, map_c, map_t, box_c, box_t, p);
   if (e != cudaSuccess) return e;
   mqa_combine_kernel<<<dim3(rows, a.H), 128, D * sizeof(float), stream>>>(
       p, D, a.sink, reinterpret_cast<__nv_bfloat16*>(a.out), a.lse);
