@@ -611,22 +611,43 @@ __global__ void __launch_bounds__(kThreads, 1)
       const Meta& M = meta[s];
       const bool win = M.window != 0;
       const XSlot& X = xs[a];
-      // Full logits: the two partial sums added in rank order (bit-identical
-      // in both CTAs); window tokens scaled by 1/rms(c_t) from the two half
-      // sums of squares, also added in rank order.
-      float mt = -INFINITY;
+      // Logit of column j: the two partial sums added in rank order (own
+      // partial from the local staging copy, the peer's from the receive
+      // slot), bit-identical in both CTAs; window tokens scaled by
+      // 1/rms(c_t) from the two half sums of squares, also in rank order.
+      // Loops stay rolled over 16-column chunks (small code, four
+      // independent accumulators).
+      auto logit4 = [&](int j, float (&v)[4]) {
+        const float4 mine = *reinterpret_cast<const float4*>(xst->s + xoff(h, j));
+        const float4 theirs = *reinterpret_cast<const float4*>(X.s + xoff(h, j));
+        const float a4[4] = {mine.x, mine.y, mine.z, mine.w};
+        const float b4[4] = {theirs.x, theirs.y, theirs.z, theirs.w};
 #pragma unroll
-      for (int j = 0; j < TN; ++j) {
-        const float other = X.s[xoff(h, j)];
-        float v = rank == 0 ? __fadd_rn(sv[j], other) : __fadd_rn(other, sv[j]);
-        if (win) {
-          const float ssum = rank == 0 ? __fadd_rn(M.ss[j], X.ss[j]) : __fadd_rn(X.ss[j], M.ss[j]);
-          v = __fmul_rn(v, rsqrtf(__fadd_rn(__fmul_rn(ssum, 1.0f / (float)D), p.eps)));
+        for (int e = 0; e < 4; ++e) {
+          float x = rank == 0 ? __fadd_rn(a4[e], b4[e]) : __fadd_rn(b4[e], a4[e]);
+          if (win) {
+            const float ssum = rank == 0 ? __fadd_rn(M.ss[j + e], X.ss[j + e])
+                                         : __fadd_rn(X.ss[j + e], M.ss[j + e]);
+            x = __fmul_rn(x, rsqrtf(__fadd_rn(__fmul_rn(ssum, 1.0f / (float)D), p.eps)));
+          }
+          const bool valid = (M.valid[(j + e) >> 5] >> ((j + e) & 31)) & 1u;
+          v[e] = valid ? __fmul_rn(x, p.scale_log2) : -INFINITY;  // log2 domain
         }
-        const bool valid = (M.valid[j >> 5] >> (j & 31)) & 1u;
-        v = valid ? __fmul_rn(v, p.scale_log2) : -INFINITY;  // log2 domain
-        sv[j] = v;
-        mt = fmaxf(mt, v);
+      };
+      float mt;
+      {
+        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll 1
+        for (int j = 0; j < TN; j += 16) {
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            float v[4];
+            logit4(j + 4 * q, v);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) m4[e] = fmaxf(m4[e], v[e]);
+          }
+        }
+        mt = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
       }
       // Online softmax with lazy rescaling (log2 domain).
       const bool grow = mt > m_run + kRescaleThreshold * 1.4426950408889634f || m_run == -INFINITY;
@@ -656,34 +677,32 @@ __global__ void __launch_bounds__(kThreads, 1)
       m_run = m_new;
       // P = exp2(logit - m) in bf16, times the window norm (V = norm * the
       // stored row), written over the consumed S columns.
-      float lsum = 0.f;
-      uint32_t pk[TN / 2];
+      float l4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 1
+      for (int j = 0; j < TN; j += 16) {
+        uint32_t pk[8];
 #pragma unroll
-      for (int j = 0; j < TN; j += 2) {
-        float p0 = m_run == -INFINITY ? 0.f : exp2f(sv[j] - m_run);
-        float p1 = m_run == -INFINITY ? 0.f : exp2f(sv[j + 1] - m_run);
-        lsum += p0 + p1;
-        if (win) {
-          const float s0 = rank == 0 ? __fadd_rn(M.ss[j], X.ss[j]) : __fadd_rn(X.ss[j], M.ss[j]);
-          const float s1 = rank == 0 ? __fadd_rn(M.ss[j + 1], X.ss[j + 1])
-                                     : __fadd_rn(X.ss[j + 1], M.ss[j + 1]);
-          p0 *= rsqrtf(__fadd_rn(__fmul_rn(s0, 1.0f / (float)D), p.eps));
-          p1 *= rsqrtf(__fadd_rn(__fmul_rn(s1, 1.0f / (float)D), p.eps));
+        for (int q = 0; q < 4; ++q) {
+          float v[4];
+          logit4(j + 4 * q, v);
+          float pe[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            pe[e] = m_run == -INFINITY ? 0.f : exp2f(v[e] - m_run);
+            l4[e] += pe[e];
+            if (win) {
+              const float ssum = rank == 0 ? __fadd_rn(M.ss[j + 4 * q + e], X.ss[j + 4 * q + e])
+                                           : __fadd_rn(X.ss[j + 4 * q + e], M.ss[j + 4 * q + e]);
+              pe[e] *= rsqrtf(__fadd_rn(__fmul_rn(ssum, 1.0f / (float)D), p.eps));
+            }
+          }
+          pk[2 * q] = pack_bf16(pe[0], pe[1]);
+          pk[2 * q + 1] = pack_bf16(pe[2], pe[3]);
         }
-        pk[j / 2] = pack_bf16(p0, p1);
+        tmem_st8(t_sa + j / 2, pk);  // columns j/2 .. j/2+7 (S there is consumed)
       }
-      l_run += lsum;
+      l_run += (l4[0] + l4[1]) + (l4[2] + l4[3]);
       mbar_arrive_remote(xempty_peer + a * 8);  // receive slot a consumed
-      {
-        uint32_t v0[16], v1[16];
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          v0[j] = pk[j];
-          v1[j] = pk[16 + j];
-        }
-        tmem_st16(t_sa, v0);
-        tmem_st16(t_sa + 16, v1);
-      }
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&pready[a]);
