@@ -319,6 +319,13 @@ CSA_DEV float warp_max(float v) {
   return v;
 }
 
+// 2^x with the hardware approximation (relative error ~2^-22; 2^-inf = 0).
+CSA_DEV float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 CSA_DEV float bf16_lo(uint32_t u) { return __uint_as_float(u << 16); }
 CSA_DEV float bf16_hi(uint32_t u) { return __uint_as_float(u & 0xFFFF0000u); }
 CSA_DEV uint32_t pack_bf16(float lo, float hi) {

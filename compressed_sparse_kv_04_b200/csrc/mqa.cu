@@ -69,7 +69,7 @@ struct MCfg {
   static constexpr int NC = Dh / 64;           // 128-byte chunks per half row
   static constexpr int kChunkBytes = TN * 128;
   static constexpr int kStageBytes = NC * kChunkBytes;
-  static constexpr int kStages = D == 512 ? 3 : 4;
+  static constexpr int kStages = D == 512 ? 2 : 4;
   static constexpr int kQCols = Dh / 2;        // bf16 pairs
   static constexpr int kSCol0 = kQCols;        // two S buffers of TN columns
   static constexpr int kOCol = kQCols + 2 * TN;
@@ -260,8 +260,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                                              ~uintptr_t(1023));
   uint8_t* stages = smem;
   XSlot* xs = reinterpret_cast<XSlot*>(stages + C::kStages * C::kStageBytes);
-  XSlot* xst = xs + 2;  // local staging of this CTA's partial logits
-  Meta* meta = reinterpret_cast<Meta*>(xs + 3);
+  XSlot* xst = xs + 2;  // [2] local staging of this CTA's partial logits
+  Meta* meta = reinterpret_cast<Meta*>(xs + 4);
   uint64_t* bars = reinterpret_cast<uint64_t*>(meta + C::kStages);
   uint64_t* full = bars;
   uint64_t* ready = full + C::kStages;
@@ -560,15 +560,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t xs_peer = mapa(smem_u32(&xs[0]), peer);
     const uint32_t xfull_peer = mapa(smem_u32(&xfull[0]), peer);
     const uint32_t xempty_peer = mapa(smem_u32(&xempty[0]), peer);
-    const bool leader = h == 0;  // issues the bulk copy of the staged logits
-    for (int it = 0; it < ntile; ++it) {
+    const bool leader = h == 0;  // issues the bulk copies of the staged logits
+    // Software pipeline with a lag of one tile: iteration it sends tile it's
+    // partial logits to the peer, then computes the softmax of tile it-1,
+    // whose exchange has had a whole iteration to land.
+    //
+    // send(it): S(it) from TMEM -> local staging slot a -> one bulk copy into
+    // the peer's receive slot a (completes on the peer's xfull[a]).  Staging
+    // slot a and the peer's receive slot a are both free once the peer has
+    // consumed tile it-2 (its xempty[a] arrivals).
+    auto send = [&](int it) -> bool {
       const int s = it % C::kStages, a = it & 1;
-      const uint32_t t_sa = t_s + lane_base + a * TN;
-      if (!wait_all(&sfull[a], (it >> 1) & 1, p, abort_flag)) break;
+      if (!wait_all(&sfull[a], (it >> 1) & 1, p, abort_flag)) return false;
       tc_fence_after();
       float sv[TN];
       {
         uint32_t v[4][16];
+        const uint32_t t_sa = t_s + lane_base + a * TN;
 #pragma unroll
         for (int c = 0; c < 4; ++c) tmem_ld16(t_sa + 16 * c, v[c]);
         tmem_wait_ld();
@@ -577,61 +585,55 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int j = 0; j < 16; ++j) sv[16 * c + j] = __uint_as_float(v[c][j]);
       }
-      if (!wait_all(&ready[s], (it / C::kStages) & 1, p, abort_flag)) break;
-      // Stage this CTA's partial logits locally, then one bulk copy moves
-      // them into the peer's receive slot a (completing on its xfull[a]).
-      // The staging buffer is free once the peer has consumed the previous
-      // tile (its xempty arrival for tile it-1).
-      if (it > 0 && !wait_all<true>(&xempty[(it - 1) & 1], ((it - 1) >> 1) & 1, p, abort_flag))
-        break;
-      {
-        float* row = xst->s;
+      if (!wait_all(&ready[s], (it / C::kStages) & 1, p, abort_flag)) return false;
+      if (!wait_all<true>(&xempty[a], ((it >> 1) & 1) ^ 1, p, abort_flag)) return false;
+      XSlot& st = xst[a];
 #pragma unroll
-        for (int j = 0; j < TN; j += 4)
-          *reinterpret_cast<float4*>(row + xoff(h, j)) =
-              make_float4(sv[j], sv[j + 1], sv[j + 2], sv[j + 3]);
-        if (h < TN) xst->ss[h] = meta[s].ss[h];
-        fence_proxy_async_smem();
-        mbar_arrive(staged);
-      }
+      for (int j = 0; j < TN; j += 4)
+        *reinterpret_cast<float4*>(st.s + xoff(h, j)) =
+            make_float4(sv[j], sv[j + 1], sv[j + 2], sv[j + 3]);
+      if (h < TN) st.ss[h] = meta[s].ss[h];
+      fence_proxy_async_smem();
+      mbar_arrive(staged);
       if (leader) {
-        // Own receive slot: expect the peer's bytes.
-        mbar_expect_tx(&xfull[a], (uint32_t)sizeof(XSlot));
-        bool ok = mbar_wait(staged, it & 1, p.status, abort_flag);
-        // The peer's slot a is free once it consumed tile it-2.
-        ok = ok && mbar_wait<true>(&xempty[a], ((it >> 1) & 1) ^ 1, p.status, abort_flag);
-        if (ok)
+        mbar_expect_tx(&xfull[a], (uint32_t)sizeof(XSlot));  // own receive slot
+        if (mbar_wait(staged, it & 1, p.status, abort_flag))
           asm volatile(
               "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes"
               " [%0], [%1], %2, [%3];" ::"r"(xs_peer + (uint32_t)(a * sizeof(XSlot))),
-              "r"(smem_u32(xst)), "r"((uint32_t)sizeof(XSlot)), "r"(xfull_peer + a * 8)
+              "r"(smem_u32(&st)), "r"((uint32_t)sizeof(XSlot)), "r"(xfull_peer + a * 8)
               : "memory");
       }
-      if (!wait_all<true>(&xfull[a], (it >> 1) & 1, p, abort_flag)) break;
+      return true;
+    };
+    // compute(it): logits, online softmax (lazy rescale), P into TMEM.
+    auto compute = [&](int it) -> bool {
+      const int s = it % C::kStages, a = it & 1;
+      const uint32_t t_sa = t_s + lane_base + a * TN;
+      if (!wait_all<true>(&xfull[a], (it >> 1) & 1, p, abort_flag)) return false;
       const Meta& M = meta[s];
       const bool win = M.window != 0;
+      const uint32_t vw0 = M.valid[0], vw1 = M.valid[1];
       const XSlot& X = xs[a];
-      // Logit of column j: the two partial sums added in rank order (own
-      // partial from the local staging copy, the peer's from the receive
-      // slot), bit-identical in both CTAs; window tokens scaled by
-      // 1/rms(c_t) from the two half sums of squares, also in rank order.
-      // Loops stay rolled over 16-column chunks (small code, four
-      // independent accumulators).
+      const XSlot& Y = xst[a];
+      // Logit of column j: the two partial sums added in rank order (bit-
+      // identical in both CTAs); window tokens scaled by 1/rms(c_t) from the
+      // two half sums of squares, also in rank order.
       auto logit4 = [&](int j, float (&v)[4]) {
-        const float4 mine = *reinterpret_cast<const float4*>(xst->s + xoff(h, j));
+        const float4 mine = *reinterpret_cast<const float4*>(Y.s + xoff(h, j));
         const float4 theirs = *reinterpret_cast<const float4*>(X.s + xoff(h, j));
         const float a4[4] = {mine.x, mine.y, mine.z, mine.w};
         const float b4[4] = {theirs.x, theirs.y, theirs.z, theirs.w};
+        const uint32_t vw = j < 32 ? vw0 : vw1;
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           float x = rank == 0 ? __fadd_rn(a4[e], b4[e]) : __fadd_rn(b4[e], a4[e]);
           if (win) {
-            const float ssum = rank == 0 ? __fadd_rn(M.ss[j + e], X.ss[j + e])
-                                         : __fadd_rn(X.ss[j + e], M.ss[j + e]);
+            const float ssum = rank == 0 ? __fadd_rn(Y.ss[j + e], X.ss[j + e])
+                                         : __fadd_rn(X.ss[j + e], Y.ss[j + e]);
             x = __fmul_rn(x, rsqrtf(__fadd_rn(__fmul_rn(ssum, 1.0f / (float)D), p.eps)));
           }
-          const bool valid = (M.valid[(j + e) >> 5] >> ((j + e) & 31)) & 1u;
-          v[e] = valid ? __fmul_rn(x, p.scale_log2) : -INFINITY;  // log2 domain
+          v[e] = ((vw >> ((j + e) & 31)) & 1u) ? __fmul_rn(x, p.scale_log2) : -INFINITY;
         }
       };
       float mt;
@@ -657,11 +659,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       // This wait happens on every tile, before pready(it) is released, so
       // the pvdone phase can never run two phases ahead of this check.
       if (it > 0) {
-        if (!wait_all(pvdone, (it - 1) & 1, p, abort_flag)) break;
+        if (!wait_all(pvdone, (it - 1) & 1, p, abort_flag)) return false;
         tc_fence_after();
       }
       if (__any_sync(0xffffffffu, need) && it > 0) {
-        const float f = need ? exp2f(m_run - m_new) : 1.f;
+        const float f = need ? fast_exp2(m_run - m_new) : 1.f;
 #pragma unroll 1
         for (int c = 0; c < C::Dh; c += 16) {
           uint32_t v[16];
@@ -673,11 +675,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tmem_wait_st();
       }
-      if (need) l_run *= exp2f(m_run - m_new);
+      if (need) l_run *= fast_exp2(m_run - m_new);
       m_run = m_new;
-      // P = exp2(logit - m) in bf16, times the window norm (V = norm * the
+      // P = 2^(logit - m) in bf16, times the window norm (V = norm * the
       // stored row), written over the consumed S columns.
       float l4[4] = {0.f, 0.f, 0.f, 0.f};
+      const bool live = m_run != -INFINITY;
 #pragma unroll 1
       for (int j = 0; j < TN; j += 16) {
         uint32_t pk[8];
@@ -688,11 +691,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           float pe[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            pe[e] = m_run == -INFINITY ? 0.f : exp2f(v[e] - m_run);
+            pe[e] = live ? fast_exp2(v[e] - m_run) : 0.f;
             l4[e] += pe[e];
             if (win) {
-              const float ssum = rank == 0 ? __fadd_rn(M.ss[j + 4 * q + e], X.ss[j + 4 * q + e])
-                                           : __fadd_rn(X.ss[j + 4 * q + e], M.ss[j + 4 * q + e]);
+              const int jj = j + 4 * q + e;
+              const float ssum = rank == 0 ? __fadd_rn(Y.ss[jj], X.ss[jj])
+                                           : __fadd_rn(X.ss[jj], Y.ss[jj]);
               pe[e] *= rsqrtf(__fadd_rn(__fmul_rn(ssum, 1.0f / (float)D), p.eps));
             }
           }
@@ -706,7 +710,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&pready[a]);
-    }
+      return true;
+    };
+    bool alive = ntile > 0 && send(0);
+    for (int it = 1; alive && it < ntile; ++it) alive = send(it) && compute(it - 1);
+    if (alive) compute(ntile - 1);
     // Epilogue: the O half and (rank 0) the running max / sum.
     if (!*abort_flag && wait_all(pvdone, (ntile - 1) & 1, p, abort_flag)) {
       tc_fence_after();
@@ -838,7 +846,7 @@ cudaError_t launch_impl(const MqaLaunch& a, cudaStream_t stream) {
                    D, TN, 64, CU_TENSOR_MAP_SWIZZLE_128B);
   if (e != cudaSuccess) return e;
 
-  const size_t smem = 1024 + (size_t)C::kStages * C::kStageBytes + 3 * sizeof(XSlot) +
+  const size_t smem = 1024 + (size_t)C::kStages * C::kStageBytes + 4 * sizeof(XSlot) +
                       C::kStages * sizeof(Meta) + 40 * 8 + 384 * 4 + 16;
   auto kern = mqa_pair_kernel<D, R>;
   e = ensure_smem_attr(reinterpret_cast<const void*>(kern), 3 + (D == 512 ? 0 : 3) + R / 32, smem);
