@@ -6,21 +6,22 @@
 // ascending; NaN below every number; -0 == +0.  Output: ascending indices,
 // padded with -1, and the count min(k, n_vis).
 //
-// Design: a cluster of C CTAs (1024 threads each) per query row, C = 1..8.
-//   Stage 1: CTA r holds its slice of the row in shared memory as
-//     order-preserving 32-bit keys and selects the exact top-k of the slice
-//     with a radix select: the digits start just below the bits common to
-//     every key of the slice (min/max reduction), 11 bits per pass,
-//     histograms with warp-aggregated shared atomics, and the passes stop as
-//     soon as the threshold digit's bin is taken whole.  The selected
-//     (key, index) pairs are compacted in index order.
-//   Stage 2 (C > 1): every CTA pushes its list into the leader CTA's shared
-//     memory (distributed shared memory stores) and arrives on the leader's
-//     mbarrier; the leader selects the final top-k among the C*k candidates
-//     with the same routine.  The global top-k of a row is contained in the
-//     union of the slices' top-k under the same total order, so the result is
-//     exact.  The leader's wait is bounded.
-// No global atomics, no inter-CTA spin on memory; deterministic.
+// Design: one thread-block cluster of C CTAs (C = 1..8) per query row.  CTA r
+// keeps its slice of the row in shared memory as order-preserving 32-bit
+// keys.  A radix select finds the exact k-th largest key over the whole row:
+//   - every exchange is a "push": each CTA adds its contribution into the
+//     shared memory of every CTA of the cluster (remote atomics), then
+//     arrives on each CTA's mbarrier; every CTA waits for the C arrivals of
+//     the round (bounded wait) and so holds the cluster-wide sum -- one
+//     one-way hop per round, no cluster-wide barrier;
+//   - round 0 exchanges min / max; the digits then start right below the
+//     bits common to every key of the row, 11 bits per round, histograms
+//     built with warp-aggregated shared atomics; the rounds stop as soon as
+//     the threshold digit's bin is taken whole;
+//   - a last round exchanges the per-CTA counts of keys above / equal to the
+//     threshold, which gives every CTA its offset in the index-ordered
+//     output (keys above the threshold, then the lowest-index equal keys).
+// No global atomics; deterministic.
 #include <algorithm>
 
 #include "common.cuh"
@@ -32,6 +33,7 @@ namespace {
 constexpr int kThreads = 1024;
 constexpr int kBins = 2048;  // 11-bit digits
 constexpr int kMaxK = 1024;
+constexpr int kMaxRounds = 8;  // min/max + at most 3 digit rounds + counts (+ slack)
 
 struct Params {
   int Q, m, k, C;
@@ -51,197 +53,51 @@ CSA_DEV uint32_t orderable(float s) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-struct Scratch {
-  uint32_t hist[kBins];
-  uint32_t warp_a[32];
-  uint32_t warp_b[32];
+struct Shared {
+  uint32_t hist[2][kBins];  // cluster-wide histograms (double-buffered by round)
+  uint32_t local[kBins];    // this CTA's histogram of the round
+  uint32_t gmin, gmax;      // cluster-wide min / max key
+  uint32_t gt_before, eq_before;  // counts of lower-rank CTAs
+  uint32_t warp_a[32], warp_b[32];
   uint32_t bcast[4];
+  uint64_t bar[kMaxRounds];  // one mbarrier per round, C arrivals each
 };
 
-// Inclusive block-wide scan helpers (1024 threads).
-CSA_DEV uint32_t block_excl_scan(uint32_t v, Scratch& sc, uint32_t* total) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  uint32_t x = v;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
-    if (lane >= o) x += y;
-  }
-  if (lane == 31) sc.warp_a[warp] = x;
-  __syncthreads();
-  if (warp == 0) {
-    uint32_t t = sc.warp_a[lane], s = t;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      uint32_t y = __shfl_up_sync(0xffffffffu, s, o);
-      if (lane >= o) s += y;
-    }
-    sc.warp_a[lane] = s - t;
-    if (lane == 31) sc.bcast[3] = s;
-  }
-  __syncthreads();
-  const uint32_t r = sc.warp_a[warp] + x - v;
-  if (total) *total = sc.bcast[3];
-  __syncthreads();
-  return r;
+CSA_DEV void red_add_remote(uint32_t caddr, uint32_t v) {
+  asm volatile("red.relaxed.cluster.shared::cluster.add.u32 [%0], %1;" ::"r"(caddr), "r"(v)
+               : "memory");
+}
+CSA_DEV void red_min_remote(uint32_t caddr, uint32_t v) {
+  asm volatile("red.relaxed.cluster.shared::cluster.min.u32 [%0], %1;" ::"r"(caddr), "r"(v)
+               : "memory");
+}
+CSA_DEV void red_max_remote(uint32_t caddr, uint32_t v) {
+  asm volatile("red.relaxed.cluster.shared::cluster.max.u32 [%0], %1;" ::"r"(caddr), "r"(v)
+               : "memory");
 }
 
-CSA_DEV uint32_t block_min_max(uint32_t lo, uint32_t hi, Scratch& sc, uint32_t* out_hi) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, o));
-    hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, o));
-  }
-  if (lane == 0) {
-    sc.warp_a[warp] = lo;
-    sc.warp_b[warp] = hi;
-  }
+// End of a round: every thread's remote contributions are issued; one thread
+// arrives on round `rd`'s barrier of every CTA, then everyone waits for the C
+// arrivals of the round.  Returns false when the (bounded) wait gave up.
+CSA_DEV bool round_sync(Shared& sh, int rd, int C, int32_t* status) {
   __syncthreads();
-  if (warp == 0) {
-    lo = sc.warp_a[lane];
-    hi = sc.warp_b[lane];
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, o));
-      hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, o));
-    }
-    if (lane == 0) {
-      sc.bcast[0] = lo;
-      sc.bcast[1] = hi;
-    }
+  if (threadIdx.x == 0) {
+    const uint32_t a = smem_u32(&sh.bar[rd]);
+    for (int c = 0; c < C; ++c) mbar_arrive_remote(mapa(a, c));
   }
-  __syncthreads();
-  lo = sc.bcast[0];
-  *out_hi = sc.bcast[1];
-  __syncthreads();
-  return lo;
-}
-
-// Radix select over keys[0..n) (shared memory; `valid` filters slots).
-// Result: prefix T and mask M such that the selection is every key with
-// (key & M) > T, plus the first `need_eq` keys (in position order) with
-// (key & M) == T.  |selection| = min(k, count of valid keys).
-template <typename Valid>
-CSA_DEV void radix_select(const uint32_t* keys, int n, int k, Valid valid, Scratch& sc,
-                          uint32_t& T, uint32_t& M, uint32_t& need_eq) {
-  const int tid = threadIdx.x, lane = tid & 31;
-  uint32_t lo = 0xFFFFFFFFu, hi = 0u;
-  for (int i = tid; i < n; i += kThreads)
-    if (valid(i)) {
-      lo = min(lo, keys[i]);
-      hi = max(hi, keys[i]);
-    }
-  uint32_t gmax;
-  const uint32_t gmin = block_min_max(lo, hi, sc, &gmax);
-  uint32_t prefix = gmin & gmax, mask = 0u;
-  uint32_t k_rem = (uint32_t)k;
-  if (gmin == gmax) {  // every key equal (or a single key)
-    T = gmin;
-    M = 0xFFFFFFFFu;
-    need_eq = k_rem;
-    return;
-  }
-  int top = 31 - __clz(gmin ^ gmax);  // highest bit that differs
-  mask = top == 31 ? 0u : (0xFFFFFFFFu << (top + 1));
-  prefix &= mask;
-  int shift = top + 1;
-  while (shift > 0) {
-    const int width = shift >= 11 ? 11 : shift;
-    shift -= width;
-    const uint32_t dmask = (1u << width) - 1u;
-    for (int b = tid; b < kBins; b += kThreads) sc.hist[b] = 0;
-    __syncthreads();
-    for (int i0 = 0; i0 < n; i0 += kThreads) {
-      const int i = i0 + tid;
-      bool act = false;
-      uint32_t bin = 0;
-      if (i < n && valid(i)) {
-        const uint32_t key = keys[i];
-        act = (key & mask) == prefix;
-        bin = (key >> shift) & dmask;
-      }
-      const uint32_t am = __ballot_sync(0xffffffffu, act);
-      if (act) {
-        const uint32_t peers = __match_any_sync(am, bin);
-        if (lane == __ffs(peers) - 1) atomicAdd(&sc.hist[bin], __popc(peers));
-      }
-    }
-    __syncthreads();
-    // Suffix sums over the digits: thread t owns digits 2t, 2t+1 (descending
-    // digit = ascending thread from the top).
-    const int nb = (int)dmask + 1;
-    uint32_t c1 = 0, c0 = 0;  // counts of digits (nb-1-2t) and (nb-2-2t)
-    const int d1 = nb - 1 - 2 * tid, d0 = nb - 2 - 2 * tid;
-    if (d1 >= 0) c1 = sc.hist[d1];
-    if (d0 >= 0) c0 = sc.hist[d0];
-    uint32_t tot;
-    const uint32_t above = block_excl_scan(c1 + c0, sc, &tot);  // keys in larger digits
-    // Exactly one digit d satisfies above(d) < k_rem <= above(d) + count(d).
-    if (d1 >= 0 && above < k_rem && above + c1 >= k_rem) {
-      sc.bcast[0] = (uint32_t)d1;
-      sc.bcast[1] = above;
-      sc.bcast[2] = c1;
-    }
-    if (d0 >= 0 && above + c1 < k_rem && above + c1 + c0 >= k_rem) {
-      sc.bcast[0] = (uint32_t)d0;
-      sc.bcast[1] = above + c1;
-      sc.bcast[2] = c0;
-    }
-    __syncthreads();
-    const uint32_t d = sc.bcast[0], abv = sc.bcast[1], cnt_d = sc.bcast[2];
-    __syncthreads();
-    k_rem -= abv;
-    prefix |= d << shift;
-    mask |= dmask << shift;
-    if (cnt_d == k_rem) break;  // the whole bin is taken: no need to resolve lower bits
-  }
-  T = prefix;
-  M = mask;
-  need_eq = k_rem;
-}
-
-// Index-ordered compaction of the selection; calls emit(position, out_slot).
-template <typename Valid, typename Emit>
-CSA_DEV uint32_t compact(const uint32_t* keys, int n, uint32_t T, uint32_t M, uint32_t need_eq,
-                         Valid valid, Scratch& sc, Emit emit) {
-  const int tid = threadIdx.x;
-  const int E = (n + kThreads - 1) / kThreads;
-  const int i0 = min(n, tid * E), i1 = min(n, i0 + E);
-  uint32_t n_gt = 0, n_eq = 0;
-  for (int i = i0; i < i1; ++i)
-    if (valid(i)) {
-      const uint32_t km = keys[i] & M;
-      n_gt += km > T;
-      n_eq += km == T;
-    }
-  const uint32_t eq_base = block_excl_scan(n_eq, sc, nullptr);
-  const uint32_t take_eq = need_eq > eq_base ? min(need_eq - eq_base, n_eq) : 0u;
-  uint32_t total;
-  uint32_t o = block_excl_scan(n_gt + take_eq, sc, &total);
-  uint32_t eq_seen = 0;
-  for (int i = i0; i < i1; ++i) {
-    if (!valid(i)) continue;
-    const uint32_t km = keys[i] & M;
-    bool take = km > T;
-    if (km == T) take = eq_seen++ < take_eq;
-    if (take) emit(i, o++);
-  }
-  return total;
+  const bool ok = mbar_wait<true>(&sh.bar[rd], 0, status);
+  return __syncthreads_and(ok) != 0;
 }
 
 __global__ void __launch_bounds__(kThreads, 1) topk_kernel(const Params p) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
-  Scratch& sc = *reinterpret_cast<Scratch*>(smem_raw);
-  uint64_t* bar = reinterpret_cast<uint64_t*>(smem_raw + sizeof(Scratch));
-  uint32_t* cand_cnt = reinterpret_cast<uint32_t*>(bar + 1);         // [8]
-  uint32_t* keys = cand_cnt + 8;                                      // slice
-  uint32_t* cand_key = keys + p.slice;                                // [C][k] (leader)
-  int32_t* cand_idx = reinterpret_cast<int32_t*>(cand_key + (p.C > 1 ? p.C * p.k : 0));
+  Shared& sh = *reinterpret_cast<Shared*>(smem_raw);
+  uint32_t* keys = reinterpret_cast<uint32_t*>(smem_raw + sizeof(Shared));
 
   const int row = blockIdx.y;
+  const int C = p.C;
   const uint32_t r = cluster_ctarank();
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int64_t pos = p.pos_q ? p.pos_q[row] : p.pos_base + row % p.Q;
   int64_t n = pos < 0 ? 0 : (pos + 1) / p.m;
   if (n > p.N_cap) {
@@ -256,57 +112,203 @@ __global__ void __launch_bounds__(kThreads, 1) topk_kernel(const Params p) {
     }
     return;
   }
-  if (p.C > 1) {
-    if (tid == 0) {
-      mbar_init(bar, p.C);
-      fence_mbar_init();
-    }
-    cluster_sync();  // the leader's barrier exists before anyone arrives on it
+  // Initial state, visible cluster-wide before any remote update.
+  for (int b = tid; b < kBins; b += kThreads) sh.hist[0][b] = sh.hist[1][b] = 0;
+  if (tid == 0) {
+    sh.gmin = 0xFFFFFFFFu;
+    sh.gmax = 0u;
+    sh.gt_before = sh.eq_before = 0u;
+    for (int rd = 0; rd < kMaxRounds; ++rd) mbar_init(&sh.bar[rd], C);
+    fence_mbar_init();
   }
+  cluster_sync();
+
   const int64_t lo = (int64_t)r * p.slice;
-  const int64_t hi = std::min<int64_t>(lo + p.slice, n);
+  const int64_t hi = lo + p.slice < n ? lo + p.slice : n;
   const int len = hi > lo ? (int)(hi - lo) : 0;
   const float* src = p.scores + (int64_t)row * p.N_cap + lo;
-  for (int i = tid; i < len; i += kThreads) keys[i] = orderable(__ldg(src + i));
+  uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
+#pragma unroll 4
+  for (int i = tid; i < len; i += kThreads) {
+    const uint32_t key = orderable(__ldg(src + i));
+    keys[i] = key;
+    kmin = min(kmin, key);
+    kmax = max(kmax, key);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
+    kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
+  }
+  // Round 0: min / max into every CTA.
+  if (lane == 0 && len > 0) {
+    const uint32_t amin = smem_u32(&sh.gmin), amax = smem_u32(&sh.gmax);
+    for (int c = 0; c < C; ++c) {
+      red_min_remote(mapa(amin, c), kmin);
+      red_max_remote(mapa(amax, c), kmax);
+    }
+  }
+  int rd = 0;
+  if (!round_sync(sh, rd++, C, p.status)) return;
+  const uint32_t gmin = sh.gmin, gmax = sh.gmax;
+
+  // Radix rounds below the common prefix.
+  uint32_t prefix, mask;
+  uint32_t k_rem = (uint32_t)p.k;
+  if (gmin == gmax) {
+    prefix = gmin;
+    mask = 0xFFFFFFFFu;
+  } else {
+    const int top = 31 - __clz(gmin ^ gmax);
+    mask = top == 31 ? 0u : (0xFFFFFFFFu << (top + 1));
+    prefix = gmin & mask;
+    int shift = top + 1;
+    int buf = 0;
+    while (shift > 0) {
+      const int width = shift >= 11 ? 11 : shift;
+      shift -= width;
+      const uint32_t dmask = (1u << width) - 1u;
+      for (int b = tid; b < kBins; b += kThreads) sh.local[b] = 0;
+      __syncthreads();
+      for (int i0 = 0; i0 < len; i0 += kThreads) {
+        const int i = i0 + tid;
+        bool act = false;
+        uint32_t bin = 0;
+        if (i < len) {
+          const uint32_t key = keys[i];
+          act = (key & mask) == prefix;
+          bin = (key >> shift) & dmask;
+        }
+        const uint32_t am = __ballot_sync(0xffffffffu, act);
+        if (act) {
+          const uint32_t peers = __match_any_sync(am, bin);
+          if (lane == __ffs(peers) - 1) atomicAdd(&sh.local[bin], __popc(peers));
+        }
+      }
+      __syncthreads();
+      // Clear the other buffer before arriving (the next round's adds only
+      // come from CTAs that have seen this round's arrival of this CTA).
+      for (int b = tid; b < kBins; b += kThreads) sh.hist[buf ^ 1][b] = 0;
+      const uint32_t base = smem_u32(&sh.hist[buf][0]);
+      for (int b = tid; b <= (int)dmask; b += kThreads) {
+        const uint32_t v = sh.local[b];
+        if (v)
+          for (int c = 0; c < C; ++c) red_add_remote(mapa(base + 4u * b, c), v);
+      }
+      if (!round_sync(sh, rd++, C, p.status)) return;
+      // Warp 0 finds the digit d with above(d) < k_rem <= above(d) + count(d),
+      // scanning from the top digit down (64 digits per lane).
+      if (warp == 0) {
+        const int nb = (int)dmask + 1;
+        const int per = (nb + 31) / 32;
+        const int d_hi = nb - 1 - lane * per;  // this lane's digits: d_hi down to d_hi-per+1
+        uint32_t sum = 0;
+        for (int j = 0; j < per; ++j) {
+          const int d = d_hi - j;
+          if (d >= 0) sum += sh.hist[buf][d];
+        }
+        uint32_t incl = sum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += y;
+        }
+        uint32_t above = incl - sum;  // keys in digits owned by lower lanes (larger digits)
+        if (above < k_rem && incl >= k_rem) {
+          for (int j = 0; j < per; ++j) {
+            const int d = d_hi - j;
+            if (d < 0) break;
+            const uint32_t cd = sh.hist[buf][d];
+            if (above + cd >= k_rem) {
+              sh.bcast[0] = (uint32_t)d;
+              sh.bcast[1] = above;
+              sh.bcast[2] = cd;
+              break;
+            }
+            above += cd;
+          }
+        }
+      }
+      __syncthreads();
+      const uint32_t d = sh.bcast[0], abv = sh.bcast[1], cnt_d = sh.bcast[2];
+      k_rem -= abv;
+      prefix |= d << shift;
+      mask |= dmask << shift;
+      buf ^= 1;
+      __syncthreads();
+      if (cnt_d == k_rem) break;  // the whole bin is taken
+    }
+  }
+  const uint32_t T = prefix, M = mask, need_eq = k_rem;
+
+  // Index-ordered output.  Warp w owns the slice elements
+  // [w*chunk, (w+1)*chunk) (chunk a multiple of 32); lane l reads element
+  // j*32 + l of the chunk, so a ballot gives each element its rank.
+  const int chunk = (((len + 31) / 32) + 31) & ~31;
+  const int w0 = min(len, warp * chunk), w1 = min(len, w0 + chunk);
+  uint32_t n_gt = 0, n_eq = 0;
+  for (int i = w0 + lane; i < w1; i += 32) {
+    const uint32_t km = keys[i] & M;
+    n_gt += km > T;
+    n_eq += km == T;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    n_gt += __shfl_xor_sync(0xffffffffu, n_gt, o);
+    n_eq += __shfl_xor_sync(0xffffffffu, n_eq, o);
+  }
+  if (lane == 0) {
+    sh.warp_a[warp] = n_gt;
+    sh.warp_b[warp] = n_eq;
+  }
   __syncthreads();
-  auto all_valid = [](int) { return true; };
-
-  // Stage 1: the exact top-k of this slice.
-  const int kl = std::min(p.k, len);
-  uint32_t T = 0, M = 0xFFFFFFFFu, need_eq = (uint32_t)len;
-  if (len > kl) radix_select(keys, len, kl, all_valid, sc, T, M, need_eq);
-  if (p.C == 1) {
-    compact(keys, len, T, M, need_eq, all_valid, sc,
-            [&](int i, uint32_t o) { out[o] = (int32_t)(lo + i); });
-    if (tid == 0) p.cnt[row] = p.k;
-    return;
+  if (warp == 0) {
+    const uint32_t a = sh.warp_a[lane], b = sh.warp_b[lane];
+    uint32_t sa = a, sb = b;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t ya = __shfl_up_sync(0xffffffffu, sa, o);
+      const uint32_t yb = __shfl_up_sync(0xffffffffu, sb, o);
+      if (lane >= o) {
+        sa += ya;
+        sb += yb;
+      }
+    }
+    sh.warp_a[lane] = sa - a;
+    sh.warp_b[lane] = sb - b;
+    if (lane == 31) {
+      sh.bcast[0] = sa;
+      sh.bcast[1] = sb;
+    }
   }
-  // Push the slice's list (index order) to the leader: slots r*k ...
-  const uint32_t ck = mapa(smem_u32(cand_key), 0) + r * p.k * 4u;
-  const uint32_t ci = mapa(smem_u32(cand_idx), 0) + r * p.k * 4u;
-  const uint32_t total = compact(keys, len, T, M, need_eq, all_valid, sc, [&](int i, uint32_t o) {
-    asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(ck + o * 4u), "r"(keys[i]) : "memory");
-    asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(ci + o * 4u), "r"((uint32_t)(lo + i))
-                 : "memory");
-  });
+  __syncthreads();
+  // Last round: this CTA's totals into every higher-rank CTA.
   if (tid == 0) {
-    asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(mapa(smem_u32(&cand_cnt[r]), 0)),
-                 "r"(total)
-                 : "memory");
+    const uint32_t ag = smem_u32(&sh.gt_before), ae = smem_u32(&sh.eq_before);
+    for (int c = (int)r + 1; c < C; ++c) {
+      red_add_remote(mapa(ag, c), sh.bcast[0]);
+      red_add_remote(mapa(ae, c), sh.bcast[1]);
+    }
   }
-  __syncthreads();  // every store of this CTA precedes the release below
-  if (tid == 0) mbar_arrive_remote(mapa(smem_u32(bar), 0));
-  if (r != 0) return;
-
-  // Stage 2 (leader): the top-k of the C lists.
-  const bool ok = mbar_wait<true>(bar, 0, p.status);
-  if (!__syncthreads_and(ok)) return;
-  const int nc = p.C * p.k;
-  auto cand_valid = [&](int j) { return (uint32_t)(j % p.k) < cand_cnt[j / p.k]; };
-  radix_select(cand_key, nc, p.k, cand_valid, sc, T, M, need_eq);
-  compact(cand_key, nc, T, M, need_eq, cand_valid, sc,
-          [&](int j, uint32_t o) { out[o] = cand_idx[j]; });
-  if (tid == 0) p.cnt[row] = p.k;
+  if (!round_sync(sh, rd++, C, p.status)) return;
+  uint32_t gt_run = sh.gt_before + sh.warp_a[warp];
+  uint32_t eq_run = sh.eq_before + sh.warp_b[warp];
+  const uint32_t lt = (1u << lane) - 1u;
+  for (int i = w0 + lane; i - lane < w1; i += 32) {
+    const uint32_t km = i < w1 ? keys[i] & M : 0u;
+    const bool gt = i < w1 && km > T;
+    const bool eq = i < w1 && km == T;
+    const uint32_t bg = __ballot_sync(0xffffffffu, gt);
+    const uint32_t be = __ballot_sync(0xffffffffu, eq);
+    const uint32_t eq_rank = eq_run + __popc(be & lt);
+    if (gt || (eq && eq_rank < need_eq)) {
+      const uint32_t o = gt_run + __popc(bg & lt) + min(need_eq, eq_rank);
+      if (o < (uint32_t)p.k) out[o] = (int32_t)(lo + i);
+    }
+    gt_run += __popc(bg);
+    eq_run += __popc(be);
+  }
+  if (r == 0 && tid == 0) p.cnt[row] = p.k;
 }
 
 }  // namespace
@@ -336,8 +338,7 @@ cudaError_t launch_topk(const TopkLaunch& a, cudaStream_t stream) {
   p.idx = a.idx;
   p.cnt = a.cnt;
   p.status = a.status;
-  const size_t smem = sizeof(Scratch) + 8 + 8 * 4 + (size_t)p.slice * 4 +
-                      (C > 1 ? (size_t)C * a.k * 8 : 0);
+  const size_t smem = sizeof(Shared) + (size_t)p.slice * 4;
   if (smem > 227 * 1024) return cudaErrorInvalidConfiguration;
   cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(topk_kernel), 2, smem);
   if (e != cudaSuccess) return e;
