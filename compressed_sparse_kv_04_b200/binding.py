@@ -23,7 +23,8 @@ OP_INDEX_TOPK, OP_SPARSE_MQA, OP_DENSE_MQA, OP_PREFILL = 1, 2, 3, 4
 
 EXPORTS = ["csa_version", "csa_last_error", "csa_workspace_bytes", "hca_compress",
            "csa_compress", "lightning_index_topk", "lightning_index_scores", "topk_select",
-           "sparse_mqa_decode", "dense_mqa_decode", "csa_prefill_chunk"]
+           "sparse_mqa_decode", "dense_mqa_decode", "csa_prefill_chunk",
+           "lightning_index_topk_static"]
 
 
 class CsaError(RuntimeError):
@@ -75,6 +76,8 @@ def _declare(L):
                                    vp]
     L.csa_prefill_chunk.argtypes = [P, i64, i32, vp, vp, i64, vp, vp, vp, vp, vp, vp, vp, vp,
                                     i64, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp, vp]
+    L.lightning_index_topk_static.argtypes = [P, i32, vp, vp, vp, vp, vp, i64, vp, vp, vp, vp,
+                                              vp]
     for name in EXPORTS[3:]:
         getattr(L, name).restype = i32
 
@@ -155,6 +158,16 @@ def lightning_index_topk(p, Q, q_idx, q_scale, w, idx_key, idx_scale, pos_q, top
         C.byref(p), Q, _ptr(q_idx), _ptr(q_scale), _ptr(w), _ptr(idx_key), _ptr(idx_scale),
         idx_key.shape[1], _ptr(pos_q), _ptr(topk_idx), _ptr(topk_cnt), _ptr(scores_out),
         _ptr(ws), 0 if ws is None else ws.numel() * ws.element_size(), _ptr(dev_status),
+        _stream(stream)))
+
+
+def lightning_index_topk_static(p, Q, q_idx, q_scale, w, idx_key, idx_scale, pos_q, topk_idx,
+                                topk_cnt, dev_status=None, stream=None):
+    """lightning_index_topk with the scores in the library's own device array
+    (no workspace; B*Q*N_cap <= 2**21)."""
+    _check(lib().lightning_index_topk_static(
+        C.byref(p), Q, _ptr(q_idx), _ptr(q_scale), _ptr(w), _ptr(idx_key), _ptr(idx_scale),
+        idx_key.shape[1], _ptr(pos_q), _ptr(topk_idx), _ptr(topk_cnt), _ptr(dev_status),
         _stream(stream)))
 
 

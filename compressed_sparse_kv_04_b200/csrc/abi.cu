@@ -111,6 +111,18 @@ int splits_for(const csa_params* p, csa_op op, int rows, int64_t N_cap) {
 
 }  // namespace
 
+namespace csa {
+// Records the message returned by csa_last_error (for entry points defined
+// in other files of the library).
+csa_status set_error(csa_status s, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return s;
+}
+}  // namespace csa
+
 extern "C" {
 
 int csa_version(void) { return 100; }

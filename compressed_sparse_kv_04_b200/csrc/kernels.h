@@ -6,6 +6,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "../../include/csa.h"
+
 namespace csa {
 
 struct CompressLaunch {
@@ -89,6 +91,9 @@ int mqa_choose_splits(int rows, int64_t compressed_max, int window, int num_sms)
 cudaError_t launch_mqa(const MqaLaunch& a, cudaStream_t stream);
 
 int device_sm_count();
+
+// Sets the message that csa_last_error returns and passes `s` through.
+csa_status set_error(csa_status s, const char* fmt, ...);
 
 // Sets the dynamic shared-memory limit of `func` once per device (the call
 // is then skipped, which keeps launches legal inside CUDA-graph capture).

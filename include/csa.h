@@ -192,6 +192,37 @@ csa_status topk_select(const csa_params* p, int Q, const float* scores, int64_t 
                        int32_t* dev_status, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * lightning_index_topk without a workspace.  The paper has no counterpart:
+ * this is an interface variant of this library, not a step of the method.
+ *
+ * Same arguments, result and errors as lightning_index_topk minus scores_out,
+ * ws and ws_bytes: the fp32 score matrix lives in an array that the library
+ * itself holds on every device it is loaded on (8 MiB each, kept until the
+ * process exits).  The call allocates no device or host memory, so callers
+ * that cannot allocate can use it: code running under another memory
+ * manager that has reserved the device's memory (an engine that pre-reserves
+ * the HBM for its KV cache), code that may not stall the device (freeing
+ * memory synchronises it), or code whose fixed interface has no workspace
+ * to hand over.
+ *
+ * Limit: B * Q * N_cap <= 2^21 (2097152) scores -- e.g. B = 8 at N_cap =
+ * 32768 or B = 4 at N_cap = 262144, one query each.  Larger calls return
+ * CSA_ERR_WORKSPACE and launch nothing.
+ * The first call on each device looks up the array's device address (with
+ * that device current); make that first call before any stream capture.
+ * Every call on a device uses the same array, which keeps the last call's
+ * scores; nothing in it has to start at zero (each call writes every score
+ * it then ranks).  Calls that can overlap on one device -- on two streams,
+ * or from two host threads -- race on the array and give wrong results:
+ * order them on one stream.
+ * ------------------------------------------------------------------------- */
+csa_status lightning_index_topk_static(const csa_params* p, int Q, const uint8_t* q_idx,
+                                       const float* q_scale, const float* w,
+                                       const uint8_t* idx_key, const float* idx_scale,
+                                       int64_t N_cap, const int64_t* pos_q, int32_t* topk_idx,
+                                       int32_t* topk_cnt, int32_t* dev_status, void* stream);
+
+/* ---------------------------------------------------------------------------
  * Shared-KV multi-query attention over selected entries + window + sink
  * ([P2] CSA step 3; [P5] "Hybrid attention": shared-KV MQA with 128 heads
  * of dim 512, sliding-window branch of 128 tokens, per-head sink logits in
