@@ -312,6 +312,17 @@ CSA_DEV void tmem_st_16x32bx2_x32(uint32_t taddr, const uint32_t (&r)[32]) {
 }
 
 // ------------------------------------------------------------------ cluster --
+// Programmatic dependent launch.  A kernel launched with programmatic stream
+// serialization may start while its predecessor in the stream is still
+// running; pdl_wait() blocks the calling thread until every prerequisite
+// grid has completed and its memory is visible (a no-op for a kernel
+// launched without the attribute).  Rule used by every kernel here: global
+// writes, and reads of anything a kernel of this library writes, come after
+// pdl_wait(); only reads of caller inputs and on-chip set-up come before.
+// pdl_trigger() lets the next kernel in the stream be scheduled early.
+CSA_DEV void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+CSA_DEV void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 CSA_DEV void named_barrier_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }

@@ -135,6 +135,7 @@ CSA_DEV void finish_row(const StreamArgs& sa, int64_t row, int lane, float (&p)[
       float g = sa.gamma ? __ldg(sa.gamma + LN::elem(lane, part, v)) : 1.f;
       p[e] = p[e] * inv * g;
     }
+  pdl_wait();  // stores come after every earlier kernel of the stream
   if (sa.out_bf16) {
     __nv_bfloat16* dst = sa.out_bf16 + row * DIM;
 #pragma unroll
@@ -265,12 +266,16 @@ CSA_DEV void pool_stream(const PoolArgs& a, const StreamArgs& sa, float* smem) {
 
 __global__ void __launch_bounds__(kThreads) compress_kernel(const PoolArgs a) {
   extern __shared__ float smem[];
+  pdl_trigger();
   const StreamArgs& sa = a.s[blockIdx.y];
   switch (sa.dim) {
     case 512: pool_stream<512>(a, sa, smem); break;
     case 128: pool_stream<128>(a, sa, smem); break;
     case 64: pool_stream<64>(a, sa, smem); break;
-    default: report(a.status, CSA_ERR_UNSUPPORTED_SHAPE); break;
+    default:
+      pdl_wait();
+      report(a.status, CSA_ERR_UNSUPPORTED_SHAPE);
+      break;
   }
 }
 
@@ -303,8 +308,7 @@ cudaError_t launch_compress(const CompressLaunch& c, cudaStream_t stream) {
   int maxdim = c.idx_tok && c.D_I > c.d ? c.D_I : c.d;
   size_t smem = G == 1 ? 0 : (size_t)kWarps * (maxdim + 2) * sizeof(float);
   dim3 grid((unsigned)grid_x, a.nstreams);
-  compress_kernel<<<grid, kThreads, smem, stream>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(compress_kernel, grid, dim3(kThreads), smem, stream, 0, a);
 }
 
 }  // namespace csa

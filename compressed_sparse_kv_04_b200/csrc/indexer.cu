@@ -84,6 +84,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   int* consumed = const_cast<int*>(abort_flag + 1);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  pdl_trigger();
   const int group = blockIdx.y;
   const int b = group / p.qgroups;
   const int q0 = (group % p.qgroups) * p.G;
@@ -153,6 +154,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------- TMA producer --
     if (elect_one()) {
       tma_prefetch_desc(&kmap);
+      pdl_wait();  // the keys are written by the compression kernel
       int it = 0;
       for (int t = t_begin; t < t_end; ++t, ++it) {
         int s = it % C::kStages;
@@ -202,6 +204,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ epilogue --
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
+    pdl_wait();  // key scales are read and scores written below
     int64_t nv[8];
 #pragma unroll
     for (int g = 0; g < 8; ++g) nv[g] = 0;
@@ -304,8 +307,7 @@ cudaError_t launch_impl(const IndexLaunch& a, cudaStream_t stream) {
                    kTileRows, DI, DI == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B);
   if (e != cudaSuccess) return e;
   dim3 grid(chunks, (unsigned)groups);
-  kern<<<grid, kThreads, smem, stream>>>(kmap, p);
-  return cudaGetLastError();
+  return launch_pdl(kern, grid, dim3(kThreads), smem, stream, 0, kmap, p);
 }
 
 }  // namespace

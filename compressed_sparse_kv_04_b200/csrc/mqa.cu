@@ -151,6 +151,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  pdl_trigger();
   const int hg0 = (blockIdx.x & 1) * HC;  // first head of this CTA
   const int split = blockIdx.x >> 1;
   const int row = blockIdx.y;
@@ -160,32 +161,28 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int64_t pos = row_pos(p, row);
   int64_t n_vis = pos < 0 ? 0 : (pos + 1) / p.m;
   if (n_vis > p.N_cap) n_vis = p.N_cap;
-  int n_c;
-  if (p.sel_idx) {
-    const int c = p.sel_cnt[row];
-    n_c = c < 0 ? 0 : (c > p.kmax ? p.kmax : c);
-  } else {
-    n_c = (int)n_vis;
-  }
   const int64_t w0 = pos - p.W + 1 < 0 ? 0 : pos - p.W + 1;
   const int nwin = (p.W > 0 && pos >= 0) ? (int)(pos - w0 + 1) : 0;
-  const int tiles_c = (n_c + TN - 1) / TN;
-  const int tiles_all = tiles_c + (nwin + TN - 1) / TN;
-  const int tps = (tiles_all + p.splits - 1) / p.splits;
-  const int t0 = std::min(split * tps, tiles_all);
-  const int t1 = std::min(t0 + tps, tiles_all);
-  const int ntile = t1 - t0;
+  // This split's tiles [t0, t1) of the list; the selection count comes from
+  // the top-k kernel, so every role calls this after pdl_wait().
+  int n_c = 0, tiles_c = 0, t0 = 0, t1 = 0, ntile = 0;
+  auto tile_range = [&]() {
+    if (p.sel_idx) {
+      const int c = p.sel_cnt[row];
+      n_c = c < 0 ? 0 : (c > p.kmax ? p.kmax : c);
+    } else {
+      n_c = (int)n_vis;
+    }
+    tiles_c = (n_c + TN - 1) / TN;
+    const int tiles_all = tiles_c + (nwin + TN - 1) / TN;
+    const int tps = (tiles_all + p.splits - 1) / p.splits;
+    t0 = std::min(split * tps, tiles_all);
+    t1 = std::min(t0 + tps, tiles_all);
+    ntile = t1 - t0;
+  };
 
   float* pml = p.part_ml + ((int64_t)row * p.splits + split) * 2 * p.H;
   if (hg0 >= p.H) return;  // this CTA has no heads (H <= 64)
-  if (ntile <= 0) {        // empty split: an empty partial for this CTA's heads
-    for (int h = threadIdx.x; h < HC; h += kThreads)
-      if (hg0 + h < p.H) {
-        pml[hg0 + h] = -INFINITY;
-        pml[p.H + hg0 + h] = 0.f;
-      }
-    return;
-  }
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) {
@@ -220,6 +217,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Contiguous tiles (dense entries, window tokens): one 64-row box per
     // 128-byte chunk.  Selected entries: row gathers (tile::gather4), issued
     // by every lane of the warp.
+    pdl_wait();
+    tile_range();
     int it = 0;
     for (int t = t0; t < t1; ++t, ++it) {
       const int s = it % C::kStages;
@@ -298,6 +297,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr int kPvN = D >= 256 ? 256 : D;  // N of one P.V instruction
     const uint32_t idesc_s = idesc_bf16(64, TN, 0, 0);
     const uint32_t idesc_pv = idesc_bf16(64, kPvN, 0, 1);
+    pdl_wait();
+    tile_range();
     const bool ok = wait_all(qready, 0, p, abort_flag);
     tc_fence_after();
     bool issued = false;
@@ -351,6 +352,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // and the KV gain in place.  Every real row: RoPE on the rotated dims.
     const int tid = threadIdx.x - 64;  // 0..127
     const int r = tid >> 1, hf = tid & 1;
+    pdl_wait();
+    tile_range();
     for (int it = 0; it < ntile; ++it) {
       const int s = it % C::kStages;
       if (!wait_all(&full[s], (it / C::kStages) & 1, p, abort_flag)) break;
@@ -492,6 +495,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       mbar_arrive(qready);
     }
+    pdl_wait();  // the query prologue above overlaps the previous kernel
+    tile_range();
 
     float m_run = -INFINITY, l_run = 0.f;
     for (int it = 0; it < ntile; ++it) {
@@ -581,8 +586,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       mbar_arrive(&pfull[a]);
     }
-    // Epilogue: this CTA's O rows and running max / sum.
-    if (!*abort_flag && wait_all(pvdone, (ntile - 1) & 1, p, abort_flag)) {
+    // Epilogue: this CTA's O rows and running max / sum (an empty split
+    // leaves an empty partial).
+    if (ntile <= 0) {
+      if (head_ok && hf == 0) {
+        pml[hg] = -INFINITY;
+        pml[p.H + hg] = 0.f;
+      }
+    } else if (!*abort_flag && wait_all(pvdone, (ntile - 1) & 1, p, abort_flag)) {
       tc_fence_after();
       float* po = p.part_o + (((int64_t)row * p.splits + split) * p.H + (head_ok ? hg : 0)) * D +
                   hf * (D / 2);
@@ -614,58 +625,108 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // Merge the split partials of one (row, head), fold in the sink, normalise,
-// apply the inverse rotation, store bf16 (and the log-sum-exp).
-__global__ void mqa_combine_kernel(const Params p, int D, const float* __restrict__ sink,
-                                   __nv_bfloat16* __restrict__ out, float* __restrict__ lse) {
-  extern __shared__ float so[];  // D floats
+// apply the inverse rotation, store bf16 (and the log-sum-exp).  Warp 0
+// turns the S (max, sum) pairs into one weight per split; then thread t
+// accumulates dims [4t, 4t+4) over the splits with independent 16-byte
+// loads.
+__global__ void __launch_bounds__(128) mqa_combine_kernel(const Params p, int D,
+                                                          const float* __restrict__ sink,
+                                                          __nv_bfloat16* __restrict__ out,
+                                                          float* __restrict__ lse) {
+  extern __shared__ float so[];  // D floats, then one weight per split
+  pdl_trigger();
+  pdl_wait();  // the partials come from the attention kernel
+  float* wsplit = so + D;
+  __shared__ float s_ml[2];
   const int row = blockIdx.x, h = blockIdx.y;
-  const float* ml = p.part_ml + (int64_t)row * p.splits * 2 * p.H;
+  const int S = p.splits;
+  const float* ml = p.part_ml + (int64_t)row * S * 2 * p.H;
   const float LOG2E = 1.4426950408889634f;
   const float z = sink[h];
-  __nv_bfloat16* o = out + ((int64_t)row * p.H + h) * D;
-  if (z == INFINITY) {
-    for (int d = threadIdx.x; d < D; d += blockDim.x) o[d] = __float2bfloat16_rn(0.f);
-    if (lse && threadIdx.x == 0) lse[(int64_t)row * p.H + h] = INFINITY;
-    return;
-  }
   const float z2 = z * LOG2E;  // log2 domain
-  float M = z2;
-  for (int s = 0; s < p.splits; ++s) M = fmaxf(M, ml[(int64_t)s * 2 * p.H + h]);
-  if (M == -INFINITY) {
-    for (int d = threadIdx.x; d < D; d += blockDim.x) o[d] = __float2bfloat16_rn(0.f);
-    if (lse && threadIdx.x == 0) lse[(int64_t)row * p.H + h] = -INFINITY;
-    return;
+  __nv_bfloat16* o = out + ((int64_t)row * p.H + h) * D;
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
+    float M = z2;
+    for (int s = lane; s < S; s += 32) M = fmaxf(M, ml[(int64_t)s * 2 * p.H + h]);
+    M = warp_max(M);
+    float L = 0.f;
+    if (M != -INFINITY && z != INFINITY) {
+      for (int s = lane; s < S; s += 32) {
+        const float ms = ml[(int64_t)s * 2 * p.H + h];
+        const float w = ms == -INFINITY ? 0.f : exp2f(ms - M);
+        wsplit[s] = w;
+        L = fmaf(ml[(int64_t)s * 2 * p.H + p.H + h], w, L);
+      }
+      L = warp_sum(L);
+      if (z2 != -INFINITY) L += exp2f(z2 - M);
+    }
+    if (lane == 0) {
+      s_ml[0] = M;
+      s_ml[1] = L;
+    }
   }
-  float L = z2 == -INFINITY ? 0.f : exp2f(z2 - M);
-  for (int s = 0; s < p.splits; ++s) {
-    const float ms = ml[(int64_t)s * 2 * p.H + h];
-    if (ms != -INFINITY) L += ml[(int64_t)s * 2 * p.H + p.H + h] * exp2f(ms - M);
+  __syncthreads();
+  const float M = s_ml[0], L = s_ml[1];
+  if (z == INFINITY || M == -INFINITY) {  // +inf sink, or nothing to attend
+    for (int d = threadIdx.x; d < D; d += blockDim.x) o[d] = __float2bfloat16_rn(0.f);
+    if (lse && threadIdx.x == 0)
+      lse[(int64_t)row * p.H + h] = z == INFINITY ? INFINITY : -INFINITY;
+    return;
   }
   const float invL = 1.0f / L;
-  for (int d = threadIdx.x; d < D; d += blockDim.x) {
-    float acc = 0.f;
-    for (int s = 0; s < p.splits; ++s) {
-      const float ms = ml[(int64_t)s * 2 * p.H + h];
-      if (ms == -INFINITY) continue;
-      acc = fmaf(p.part_o[(((int64_t)row * p.splits + s) * p.H + h) * D + d], exp2f(ms - M), acc);
+  for (int d4 = threadIdx.x; d4 < D / 4; d4 += blockDim.x) {
+    const float* src = p.part_o + ((int64_t)row * S * p.H + h) * D + 4 * d4;
+    const int64_t stride = (int64_t)p.H * D;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    int s = 0;
+    for (; s + 4 <= S; s += 4) {
+      float4 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) v[u] = __ldg(reinterpret_cast<const float4*>(src + (s + u) * stride));
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float w = wsplit[s + u];
+        acc.x = fmaf(v[u].x, w, acc.x);
+        acc.y = fmaf(v[u].y, w, acc.y);
+        acc.z = fmaf(v[u].z, w, acc.z);
+        acc.w = fmaf(v[u].w, w, acc.w);
+      }
     }
-    so[d] = acc * invL;
+    for (; s < S; ++s) {
+      const float4 v = __ldg(reinterpret_cast<const float4*>(src + s * stride));
+      const float w = wsplit[s];
+      acc.x = fmaf(v.x, w, acc.x);
+      acc.y = fmaf(v.y, w, acc.y);
+      acc.z = fmaf(v.z, w, acc.z);
+      acc.w = fmaf(v.w, w, acc.w);
+    }
+    so[4 * d4] = acc.x * invL;
+    so[4 * d4 + 1] = acc.y * invL;
+    so[4 * d4 + 2] = acc.z * invL;
+    so[4 * d4 + 3] = acc.w * invL;
   }
   __syncthreads();
   const int64_t pos = row_pos(p, row);
   const int half = p.R / 2, d0 = D - p.R;
-  for (int d = threadIdx.x; d < D; d += blockDim.x) {
-    float v = so[d];
-    if (d >= d0 && p.R > 0) {
-      const int j = (d - d0) % half;
-      float sn, cs;
-      sincos_reduced((double)pos * p.inv_freq[j], &sn, &cs);
-      if (d - d0 < half)
-        v = so[d] * cs + so[d + half] * sn;  // rotation by -angle
-      else
-        v = so[d] * cs - so[d - half] * sn;
+  for (int d2 = threadIdx.x; d2 < D / 2; d2 += blockDim.x) {
+    float v2[2];
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int d = 2 * d2 + e;
+      float v = so[d];
+      if (p.R > 0 && d >= d0) {
+        const int j = (d - d0) % half;
+        float sn, cs;
+        sincos_reduced((double)pos * p.inv_freq[j], &sn, &cs);
+        if (d - d0 < half)
+          v = so[d] * cs + so[d + half] * sn;  // rotation by -angle
+        else
+          v = so[d] * cs - so[d - half] * sn;
+      }
+      v2[e] = v;
     }
-    o[d] = __float2bfloat16_rn(v);
+    reinterpret_cast<uint32_t*>(o)[d2] = pack_bf16(v2[0], v2[1]);
   }
   if (lse && threadIdx.x == 0) lse[(int64_t)row * p.H + h] = (M + log2f(L)) / LOG2E;
 }
@@ -720,12 +781,11 @@ cudaError_t launch_impl(const MqaLaunch& a, cudaStream_t stream) {
   e = ensure_smem_attr(reinterpret_cast<const void*>(kern), 3 + (D == 512 ? 0 : 3) + R / 32, smem);
   if (e != cudaSuccess) return e;
   dim3 grid(2 * a.splits, rows, 1);
-  kern<<<grid, kThreads, smem, stream>>>(map_c, map_t, box_c, box_t, p);
-  e = cudaGetLastError();
+  e = launch_pdl(kern, grid, dim3(kThreads), smem, stream, 0, map_c, map_t, box_c, box_t, p);
   if (e != cudaSuccess) return e;
-  mqa_combine_kernel<<<dim3(rows, a.H), 128, D * sizeof(float), stream>>>(
-      p, D, a.sink, reinterpret_cast<__nv_bfloat16*>(a.out), a.lse);
-  return cudaGetLastError();
+  return launch_pdl(mqa_combine_kernel, dim3(rows, a.H), dim3(128),
+                    (size_t)(D + a.splits) * sizeof(float), stream, 0, p, D, a.sink,
+                    reinterpret_cast<__nv_bfloat16*>(a.out), a.lse);
 }
 
 }  // namespace

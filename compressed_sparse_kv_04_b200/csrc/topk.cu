@@ -9,18 +9,20 @@
 // Design: one thread-block cluster of C CTAs (C = 1..8) per query row.  CTA r
 // keeps its slice of the row in shared memory as order-preserving 32-bit
 // keys.  A radix select finds the exact k-th largest key over the whole row:
-//   - every exchange is a "push": each CTA adds its contribution into the
-//     shared memory of every CTA of the cluster (remote atomics), then
-//     arrives on each CTA's mbarrier; every CTA waits for the C arrivals of
-//     the round (bounded wait) and so holds the cluster-wide sum -- one
-//     one-way hop per round, no cluster-wide barrier;
+//   - every exchange is a push of plain 16-byte stores: each CTA writes its
+//     contribution into its own slot of every CTA's receive buffer, then one
+//     hardware cluster barrier (arrive.release / wait.acquire) makes all
+//     slots visible; each CTA sums the C slots itself.  (Remote atomics and
+//     mbarrier hops cost several times more per round on this part.)
 //   - round 0 exchanges min / max; the digits then start right below the
-//     bits common to every key of the row, 11 bits per round, histograms
-//     built with warp-aggregated shared atomics; the rounds stop as soon as
-//     the threshold digit's bin is taken whole;
+//     bits common to every key of the row, kDigitBits per round; the rounds
+//     stop as soon as the threshold digit's bin is taken whole;
 //   - a last round exchanges the per-CTA counts of keys above / equal to the
 //     threshold, which gives every CTA its offset in the index-ordered
 //     output (keys above the threshold, then the lowest-index equal keys).
+// Every decision that steers the control flow (early exit, number of
+// rounds) is computed from cluster-wide sums that all CTAs of the cluster
+// hold identically, so all of them reach every cluster barrier.
 // No global atomics; deterministic.
 #include <algorithm>
 
@@ -31,9 +33,9 @@ namespace csa {
 namespace {
 
 constexpr int kThreads = 1024;
-constexpr int kBins = 2048;  // 11-bit digits
+constexpr int kDigitBits = 8;  // radix digit width (256 bins)
 constexpr int kMaxK = 1024;
-constexpr int kMaxRounds = 8;  // min/max + at most 3 digit rounds + counts (+ slack)
+constexpr int kMaxC = 16;      // CTAs per cluster (16 needs the non-portable size)
 
 struct Params {
   int Q, m, k, C;
@@ -53,104 +55,103 @@ CSA_DEV uint32_t orderable(float s) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
+template <int kBins>
 struct Shared {
-  uint32_t hist[2][kBins];  // cluster-wide histograms (double-buffered by round)
-  uint32_t local[kBins];    // this CTA's histogram of the round
-  uint32_t gmin, gmax;      // cluster-wide min / max key
-  uint32_t gt_before, eq_before;  // counts of lower-rank CTAs
+  uint32_t recv[2][kMaxC][kBins];  // per-source histograms, by round parity
+  uint32_t local[2][kBins];        // this CTA's histogram, by round parity
+  uint32_t mm[kMaxC][2];           // per-source (min, max) key
+  uint32_t cn[kMaxC][2];           // per-source (above, equal) counts
   uint32_t warp_a[32], warp_b[32];
   uint32_t bcast[4];
-  uint64_t bar[kMaxRounds];  // one mbarrier per round, C arrivals each
 };
 
-CSA_DEV void red_add_remote(uint32_t caddr, uint32_t v) {
-  asm volatile("red.relaxed.cluster.shared::cluster.add.u32 [%0], %1;" ::"r"(caddr), "r"(v)
+CSA_DEV void cluster_arrive() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+CSA_DEV void cluster_wait() { asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory"); }
+CSA_DEV void st_remote_v2(uint32_t caddr, uint32_t a, uint32_t b) {
+  asm volatile("st.shared::cluster.v2.u32 [%0], {%1, %2};" ::"r"(caddr), "r"(a), "r"(b)
                : "memory");
 }
-CSA_DEV void red_min_remote(uint32_t caddr, uint32_t v) {
-  asm volatile("red.relaxed.cluster.shared::cluster.min.u32 [%0], %1;" ::"r"(caddr), "r"(v)
-               : "memory");
-}
-CSA_DEV void red_max_remote(uint32_t caddr, uint32_t v) {
-  asm volatile("red.relaxed.cluster.shared::cluster.max.u32 [%0], %1;" ::"r"(caddr), "r"(v)
+CSA_DEV void st_remote_v4(uint32_t caddr, uint4 v) {
+  asm volatile("st.shared::cluster.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(caddr), "r"(v.x),
+               "r"(v.y), "r"(v.z), "r"(v.w)
                : "memory");
 }
 
-// End of a round: every thread's remote contributions are issued; one thread
-// arrives on round `rd`'s barrier of every CTA, then everyone waits for the C
-// arrivals of the round.  Returns false when the (bounded) wait gave up.
-CSA_DEV bool round_sync(Shared& sh, int rd, int C, int32_t* status) {
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    const uint32_t a = smem_u32(&sh.bar[rd]);
-    for (int c = 0; c < C; ++c) mbar_arrive_remote(mapa(a, c));
-  }
-  const bool ok = mbar_wait<true>(&sh.bar[rd], 0, status);
-  return __syncthreads_and(ok) != 0;
-}
-
+template <int kBits, bool kAggregate>
 __global__ void __launch_bounds__(kThreads, 1) topk_kernel(const Params p) {
+  constexpr int kBins = 1 << kBits;
+  using S = Shared<kBins>;
   extern __shared__ __align__(16) uint8_t smem_raw[];
-  Shared& sh = *reinterpret_cast<Shared*>(smem_raw);
-  uint32_t* keys = reinterpret_cast<uint32_t*>(smem_raw + sizeof(Shared));
+  S& sh = *reinterpret_cast<S*>(smem_raw);
+  uint32_t* keys = reinterpret_cast<uint32_t*>(smem_raw + sizeof(S));
 
   const int row = blockIdx.y;
   const int C = p.C;
   const uint32_t r = cluster_ctarank();
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  pdl_trigger();
   const int64_t pos = p.pos_q ? p.pos_q[row] : p.pos_base + row % p.Q;
+  pdl_wait();  // the scores come from the indexer kernel
+  // The slice's scores are loaded before the visible count is known (the
+  // row holds N_cap scores, so every address is in bounds).
+  const int64_t lo = (int64_t)r * p.slice;
+  const int cap = (int)(p.N_cap - lo < p.slice ? (p.N_cap - lo > 0 ? p.N_cap - lo : 0) : p.slice);
+  const float* src = p.scores + (int64_t)row * p.N_cap + lo;
+#pragma unroll 8
+  for (int i = tid; i < cap; i += kThreads) keys[i] = orderable(__ldg(src + i));
   int64_t n = pos < 0 ? 0 : (pos + 1) / p.m;
   if (n > p.N_cap) {
     n = p.N_cap;
     if (r == 0 && tid == 0) report(p.status, CSA_ERR_CAPACITY);
   }
   int32_t* out = p.idx + (int64_t)row * p.k;
-  if (n <= p.k) {  // every visible entry is kept (uniform over the cluster)
+  if (n <= p.k) {  // every visible entry is kept (the whole cluster returns)
     if (r == 0) {
       for (int j = tid; j < p.k; j += kThreads) out[j] = j < n ? j : -1;
       if (tid == 0) p.cnt[row] = (int32_t)n;
     }
     return;
   }
-  // Initial state, visible cluster-wide before any remote update.
-  for (int b = tid; b < kBins; b += kThreads) sh.hist[0][b] = sh.hist[1][b] = 0;
-  if (tid == 0) {
-    sh.gmin = 0xFFFFFFFFu;
-    sh.gmax = 0u;
-    sh.gt_before = sh.eq_before = 0u;
-    for (int rd = 0; rd < kMaxRounds; ++rd) mbar_init(&sh.bar[rd], C);
-    fence_mbar_init();
-  }
-  cluster_sync();
+  cluster_arrive();  // paired with the wait before the first remote store
 
-  const int64_t lo = (int64_t)r * p.slice;
-  const int64_t hi = lo + p.slice < n ? lo + p.slice : n;
-  const int len = hi > lo ? (int)(hi - lo) : 0;
-  const float* src = p.scores + (int64_t)row * p.N_cap + lo;
+  const int len = (int)(n - lo < cap ? (n - lo > 0 ? n - lo : 0) : cap);
+  for (int b = tid; b < kBins; b += kThreads) sh.local[0][b] = 0;
   uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
-#pragma unroll 4
-  for (int i = tid; i < len; i += kThreads) {
-    const uint32_t key = orderable(__ldg(src + i));
-    keys[i] = key;
-    kmin = min(kmin, key);
-    kmax = max(kmax, key);
+  for (int i = tid; i < len; i += kThreads) {  // the keys this thread wrote
+    kmin = min(kmin, keys[i]);
+    kmax = max(kmax, keys[i]);
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
     kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
     kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
   }
-  // Round 0: min / max into every CTA.
-  if (lane == 0 && len > 0) {
-    const uint32_t amin = smem_u32(&sh.gmin), amax = smem_u32(&sh.gmax);
-    for (int c = 0; c < C; ++c) {
-      red_min_remote(mapa(amin, c), kmin);
-      red_max_remote(mapa(amax, c), kmax);
-    }
+  if (lane == 0) {
+    sh.warp_a[warp] = kmin;
+    sh.warp_b[warp] = kmax;
   }
-  int rd = 0;
-  if (!round_sync(sh, rd++, C, p.status)) return;
-  const uint32_t gmin = sh.gmin, gmax = sh.gmax;
+  __syncthreads();
+  cluster_wait();  // every CTA of the cluster is running
+  // Round 0: (min, max) of this CTA into slot r of every CTA.
+  if (warp == 0) {
+    kmin = sh.warp_a[lane];
+    kmax = sh.warp_b[lane];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
+      kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
+    }
+    if (lane < C) st_remote_v2(mapa(smem_u32(&sh.mm[r][0]), lane), kmin, kmax);
+  }
+  cluster_arrive();
+  cluster_wait();
+  uint32_t gmin = 0xFFFFFFFFu, gmax = 0u;
+  for (int c = 0; c < C; ++c) {
+    gmin = min(gmin, sh.mm[c][0]);
+    gmax = max(gmax, sh.mm[c][1]);
+  }
 
   // Radix rounds below the common prefix.
   uint32_t prefix, mask;
@@ -163,70 +164,62 @@ __global__ void __launch_bounds__(kThreads, 1) topk_kernel(const Params p) {
     mask = top == 31 ? 0u : (0xFFFFFFFFu << (top + 1));
     prefix = gmin & mask;
     int shift = top + 1;
-    int buf = 0;
+    int par = 0;
     while (shift > 0) {
-      const int width = shift >= 11 ? 11 : shift;
+      const int width = shift >= kBits ? kBits : shift;
       shift -= width;
       const uint32_t dmask = (1u << width) - 1u;
-      for (int b = tid; b < kBins; b += kThreads) sh.local[b] = 0;
-      __syncthreads();
-      for (int i0 = 0; i0 < len; i0 += kThreads) {
-        const int i = i0 + tid;
-        bool act = false;
-        uint32_t bin = 0;
-        if (i < len) {
-          const uint32_t key = keys[i];
-          act = (key & mask) == prefix;
-          bin = (key >> shift) & dmask;
-        }
-        const uint32_t am = __ballot_sync(0xffffffffu, act);
-        if (act) {
-          const uint32_t peers = __match_any_sync(am, bin);
-          if (lane == __ffs(peers) - 1) atomicAdd(&sh.local[bin], __popc(peers));
+      uint32_t* loc = sh.local[par];
+      for (int i = tid; i < len; i += kThreads) {
+        const uint32_t key = keys[i];
+        const bool act = (key & mask) == prefix;
+        const uint32_t bin = (key >> shift) & dmask;
+        if (kAggregate) {
+          const uint32_t am = __ballot_sync(__activemask(), act);
+          if (act) {
+            const uint32_t peers = __match_any_sync(am, bin);
+            if (lane == __ffs(peers) - 1) atomicAdd(&loc[bin], __popc(peers));
+          }
+        } else if (act) {
+          atomicAdd(&loc[bin], 1u);
         }
       }
       __syncthreads();
-      // Clear the other buffer before arriving (the next round's adds only
-      // come from CTAs that have seen this round's arrival of this CTA).
-      for (int b = tid; b < kBins; b += kThreads) sh.hist[buf ^ 1][b] = 0;
-      const uint32_t base = smem_u32(&sh.hist[buf][0]);
-      for (int b = tid; b <= (int)dmask; b += kThreads) {
-        const uint32_t v = sh.local[b];
-        if (v)
-          for (int c = 0; c < C; ++c) red_add_remote(mapa(base + 4u * b, c), v);
+      // Push: this CTA's histogram into slot r of every CTA (16-byte stores);
+      // the other threads clear next round's local histogram.
+      constexpr int kVec = kBins / 4;
+      for (int t = tid; t < C * kVec; t += kThreads) {
+        const int c = t / kVec, j = t % kVec;
+        const uint4 v = reinterpret_cast<const uint4*>(loc)[j];
+        st_remote_v4(mapa(smem_u32(&sh.recv[par][r][4 * j]), c), v);
       }
-      if (!round_sync(sh, rd++, C, p.status)) return;
-      // Warp 0 finds the digit d with above(d) < k_rem <= above(d) + count(d),
-      // scanning from the top digit down (64 digits per lane).
-      if (warp == 0) {
-        const int nb = (int)dmask + 1;
-        const int per = (nb + 31) / 32;
-        const int d_hi = nb - 1 - lane * per;  // this lane's digits: d_hi down to d_hi-per+1
-        uint32_t sum = 0;
-        for (int j = 0; j < per; ++j) {
-          const int d = d_hi - j;
-          if (d >= 0) sum += sh.hist[buf][d];
-        }
-        uint32_t incl = sum;
+      for (int b = tid; b < kBins; b += kThreads) sh.local[par ^ 1][b] = 0;
+      cluster_arrive();
+      cluster_wait();
+      // Thread t < nb owns digit d = nb-1-t: its cluster-wide count, then a
+      // scan over t gives the keys in digits >= d; the one thread with
+      // above(d) < k_rem <= above(d) + count(d) publishes d.
+      const int nb = (int)dmask + 1;
+      uint32_t cnt_t = 0;
+      if (tid < nb)
+        for (int c = 0; c < C; ++c) cnt_t += sh.recv[par][c][nb - 1 - tid];
+      uint32_t incl = cnt_t;
+      if (warp < kBins / 32) {
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
           const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
           if (lane >= o) incl += y;
         }
-        uint32_t above = incl - sum;  // keys in digits owned by lower lanes (larger digits)
+        if (lane == 31) sh.warp_a[warp] = incl;
+      }
+      __syncthreads();
+      if (tid < nb) {
+        for (int w2 = 0; w2 < warp; ++w2) incl += sh.warp_a[w2];
+        const uint32_t above = incl - cnt_t;
         if (above < k_rem && incl >= k_rem) {
-          for (int j = 0; j < per; ++j) {
-            const int d = d_hi - j;
-            if (d < 0) break;
-            const uint32_t cd = sh.hist[buf][d];
-            if (above + cd >= k_rem) {
-              sh.bcast[0] = (uint32_t)d;
-              sh.bcast[1] = above;
-              sh.bcast[2] = cd;
-              break;
-            }
-            above += cd;
-          }
+          sh.bcast[0] = (uint32_t)(nb - 1 - tid);
+          sh.bcast[1] = above;
+          sh.bcast[2] = cnt_t;
         }
       }
       __syncthreads();
@@ -234,8 +227,7 @@ __global__ void __launch_bounds__(kThreads, 1) topk_kernel(const Params p) {
       k_rem -= abv;
       prefix |= d << shift;
       mask |= dmask << shift;
-      buf ^= 1;
-      __syncthreads();
+      par ^= 1;
       if (cnt_d == k_rem) break;  // the whole bin is taken
     }
   }
@@ -257,6 +249,7 @@ __global__ void __launch_bounds__(kThreads, 1) topk_kernel(const Params p) {
     n_gt += __shfl_xor_sync(0xffffffffu, n_gt, o);
     n_eq += __shfl_xor_sync(0xffffffffu, n_eq, o);
   }
+  __syncthreads();  // bcast / warp slots of the last round are read
   if (lane == 0) {
     sh.warp_a[warp] = n_gt;
     sh.warp_b[warp] = n_eq;
@@ -276,23 +269,17 @@ __global__ void __launch_bounds__(kThreads, 1) topk_kernel(const Params p) {
     }
     sh.warp_a[lane] = sa - a;
     sh.warp_b[lane] = sb - b;
-    if (lane == 31) {
-      sh.bcast[0] = sa;
-      sh.bcast[1] = sb;
-    }
+    // Last round: this CTA's totals into slot r of every higher-rank CTA.
+    const uint32_t ga = __shfl_sync(0xffffffffu, sa, 31), gb = __shfl_sync(0xffffffffu, sb, 31);
+    if (lane > (int)r && lane < C) st_remote_v2(mapa(smem_u32(&sh.cn[r][0]), lane), ga, gb);
   }
-  __syncthreads();
-  // Last round: this CTA's totals into every higher-rank CTA.
-  if (tid == 0) {
-    const uint32_t ag = smem_u32(&sh.gt_before), ae = smem_u32(&sh.eq_before);
-    for (int c = (int)r + 1; c < C; ++c) {
-      red_add_remote(mapa(ag, c), sh.bcast[0]);
-      red_add_remote(mapa(ae, c), sh.bcast[1]);
-    }
+  cluster_arrive();
+  cluster_wait();
+  uint32_t gt_run = sh.warp_a[warp], eq_run = sh.warp_b[warp];
+  for (int c = 0; c < (int)r; ++c) {
+    gt_run += sh.cn[c][0];
+    eq_run += sh.cn[c][1];
   }
-  if (!round_sync(sh, rd++, C, p.status)) return;
-  uint32_t gt_run = sh.gt_before + sh.warp_a[warp];
-  uint32_t eq_run = sh.eq_before + sh.warp_b[warp];
   const uint32_t lt = (1u << lane) - 1u;
   for (int i = w0 + lane; i - lane < w1; i += 32) {
     const uint32_t km = i < w1 ? keys[i] & M : 0u;
@@ -313,17 +300,62 @@ __global__ void __launch_bounds__(kThreads, 1) topk_kernel(const Params p) {
 
 }  // namespace
 
+// Largest cluster size (8 or 16) that can be resident for this kernel and
+// shared-memory size on the current device; cached per device.
+int max_cluster(const void* kern, size_t smem) {
+  static int cached[64][2] = {};
+  static size_t cached_smem[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 8;
+  if (cached[dev][0] && cached_smem[dev] == smem) return cached[dev][1];
+  int best = 8;
+  bool failed = true;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
+      cudaSuccess) {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(16, 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 16;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) == cudaSuccess) {
+      failed = false;
+      if (n >= 1) best = 16;
+    }
+  }
+  if (failed) cudaGetLastError();  // a refused query is not the caller's error
+  cached[dev][0] = 1;
+  cached[dev][1] = best;
+  cached_smem[dev] = smem;
+  return best;
+}
+
 cudaError_t launch_topk(const TopkLaunch& a, cudaStream_t stream) {
   if (a.rows < 1) return cudaSuccess;
   if (a.rows > 65535 || a.k > kMaxK) return cudaErrorInvalidConfiguration;
   const int sms = device_sm_count();
   const int need = (int)((a.N_cap + 32767) / 32768);
   if (need > 8) return cudaErrorInvalidValue;
+  auto kern = topk_kernel<kDigitBits, false>;
+  using S = Shared<(1 << kDigitBits)>;
+  // Slices of at most 32768 scores; small batches spread each row over more
+  // CTAs (slices of at least 4096 scores), up to 16 where 16-CTA clusters fit.
+  const int64_t slice_max = (a.N_cap + need - 1) / need;
+  cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kern), 2,
+                                   sizeof(S) + (size_t)slice_max * 4);
+  if (e != cudaSuccess) return e;
+  const int limit = max_cluster(reinterpret_cast<const void*>(kern), sizeof(S) + slice_max * 4);
   int C = 1;
   while (C < need) C <<= 1;
-  if (a.rows < sms) {  // spread small batches: slices of at least 4096 scores
+  if (a.rows < sms) {
     const int fill = std::max(1, sms / a.rows);
-    while (C * 2 <= 8 && C * 2 <= fill && a.N_cap / (C * 2) >= 4096) C *= 2;
+    while (C * 2 <= limit && C * 2 <= fill && a.N_cap / (C * 2) >= 4096) C *= 2;
   }
   Params p{};
   p.Q = a.Q;
@@ -338,25 +370,8 @@ cudaError_t launch_topk(const TopkLaunch& a, cudaStream_t stream) {
   p.idx = a.idx;
   p.cnt = a.cnt;
   p.status = a.status;
-  const size_t smem = sizeof(Shared) + (size_t)p.slice * 4;
-  if (smem > 227 * 1024) return cudaErrorInvalidConfiguration;
-  cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(topk_kernel), 2, smem);
-  if (e != cudaSuccess) return e;
-  cudaLaunchConfig_t cfg{};
-  cfg.gridDim = dim3(C, a.rows, 1);
-  cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = C;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, topk_kernel, p);
-  if (e != cudaSuccess) return e;
-  return cudaGetLastError();
+  const size_t smem = sizeof(S) + (size_t)p.slice * 4;
+  return launch_pdl(kern, dim3(C, a.rows, 1), dim3(kThreads), smem, stream, C, p);
 }
 
 }  // namespace csa
