@@ -116,6 +116,19 @@ CSA_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, int32_t* status,
   }
 }
 
+// 16-byte global -> shared copy through L2 (LSU path), and an mbarrier
+// arrival that fires once this thread's earlier copies have landed (counts
+// as one of the barrier's expected arrivals).
+CSA_DEV void cp_async_16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src)
+               : "memory");
+}
+CSA_DEV void cp_async_arrive(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+CSA_DEV void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
 // --------------------------------------------------------------------- TMA --
 CSA_DEV void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");

@@ -79,7 +79,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* tfull = empty + C::kStages;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
-  uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* done = drain + 1;  // one arrival per warp when its role is over
+  uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_slot + 1);
   int* consumed = const_cast<int*>(abort_flag + 1);
 
@@ -113,10 +114,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&tempty[a], 128);
     }
     mbar_init(drain, 1);
+    mbar_init(done, kThreads / 32);
     *abort_flag = 0;
     *consumed = 0;
     fence_mbar_init();
   }
+  __syncwarp();
   if (warp == 0) {
     tmem_alloc(tmem_base_slot, p.tmem_cols);
     tmem_relinquish();
@@ -251,9 +254,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive(&tempty[a]);
     }
   }
+  // Teardown: every warp reports (converged) that it is done with tensor
+  // memory; warp 0 frees it after all of them (bounded wait).
+  __syncwarp();
   tc_fence_before();
-  __syncthreads();
+  if (lane == 0) mbar_arrive(done);
   if (warp == 0) {
+    mbar_wait(done, 0, p.status);
+    __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, p.tmem_cols);
   }
@@ -286,7 +294,7 @@ cudaError_t launch_impl(const IndexLaunch& a, cudaStream_t stream) {
   p.tmem_cols = cols;
 
   size_t smem = 1024 + (size_t)C::kStages * C::kStageBytes + (size_t)p.N * DI + 256 * 4 +
-                (2 * C::kStages + 5) * 8 + 16;
+                (2 * C::kStages + 6) * 8 + 16;
   auto kern = index_score_kernel<DI>;
   cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kern), DI == 128 ? 0 : 1,
                                    smem);

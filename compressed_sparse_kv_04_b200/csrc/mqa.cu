@@ -19,9 +19,11 @@
 //     Qhat (64 heads x D bf16 pairs)   lane half 1, columns 128 .. 128+D/2-1
 // (the A operand of S = Qhat K^T is read from TMEM in the same lane half as
 // the accumulator it feeds).  Per 64-entry tile:
-//   - the producer warp fetches the tile's full rows (TMA boxes for
-//     contiguous tiles, tile::gather4 row gathers for selected entries;
-//     128-byte swizzle), K = V = that tile;
+//   - contiguous tiles (dense entries, window tokens) arrive by TMA boxes
+//     issued by the producer warp; selected entries are gathered by the four
+//     transform warps with 16-byte cp.async (two threads per row, a few
+//     tiles ahead), which keeps many more rows in flight than per-row TMA
+//     gathers; 128-byte swizzle either way, K = V = that tile;
 //   - transform warps RoPE the rotated dims in place and, for window tokens,
 //     compute 1/rms(c_t) and apply the KV gain;
 //   - the MMA warp issues S = Qhat K^T (TS form) into one of two S buffers,
@@ -97,6 +99,7 @@ struct Params {
   const int32_t* sel_idx;
   const int32_t* sel_cnt;
   int kmax;
+  const __nv_bfloat16* kv_c;
   const float* gamma_q;
   const float* gamma_kv;
   float eps, scale_log2;  // softmax scale * log2(e)
@@ -147,7 +150,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* pvdone = pfull + 2;
   uint64_t* qready = pvdone + 1;
   uint64_t* drain = qready + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* done = drain + 1;  // one arrival per warp when its role is over
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -186,7 +190,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) {
-      mbar_init(&full[s], 1);
+      mbar_init(&full[s], 1 + 128);  // producer + the transform threads
       mbar_init(&ready[s], 128);
       mbar_init(&empty[s], 1);
     }
@@ -197,9 +201,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(pvdone, 1);
     mbar_init(qready, 128);
     mbar_init(drain, 1);
+    mbar_init(done, kThreads / 32);
     *abort_flag = 0;
     fence_mbar_init();
   }
+  __syncwarp();
   if (warp == 0) {
     tmem_alloc(tmem_slot, C::kAlloc);
     tmem_relinquish();
@@ -268,29 +274,26 @@ __global__ void __launch_bounds__(kThreads, 1)
         M.valid[0] = vb0;
         M.valid[1] = vb1;
         M.window = win ? 1 : 0;
-        mbar_expect_tx(&full[s], C::kStageBytes);
+        if (gathered)
+          mbar_arrive(&full[s]);  // the transform warps gather the rows
+        else
+          mbar_expect_tx(&full[s], C::kStageBytes);
       }
       __syncwarp();
-      uint8_t* dst = stages + s * C::kStageBytes;
       if (!gathered) {
         // Rows grow[0] .. grow[0]+63 are consecutive (rows past the list are
         // fetched too and masked; rows past the tensor are zero-filled).
+        uint8_t* dst = stages + s * C::kStageBytes;
         const int32_t y0 = __shfl_sync(0xffffffffu, grow[0], 0);
         if (lane < C::NC)
           tma_load_2d(dst + lane * C::kChunkBytes, win ? &box_t : &box_c, &full[s],
                       (int32_t)(lane * 64), y0);
-      } else {
-        constexpr int kGroups = C::NC * (TN / 4);  // 4-row groups per tile
-        for (int q = lane; q < kGroups; q += 32) {
-          const int c = q / (TN / 4), g = q % (TN / 4);
-          tma_gather4(dst + c * C::kChunkBytes + g * 4 * 128, &map_c, &full[s], (int32_t)(c * 64),
-                      M.grow[4 * g], M.grow[4 * g + 1], M.grow[4 * g + 2], M.grow[4 * g + 3]);
-        }
       }
     }
-    if (*abort_flag && lane == 0) {  // copies still in flight must land first
+    if (*abort_flag && lane == 0) {  // box copies still in flight must land first
       for (int j = std::max(0, it - C::kStages); j < it; ++j)
-        mbar_wait(&full[j % C::kStages], (j / C::kStages) & 1, p.status);
+        if (t0 + j >= tiles_c || p.sel_idx == nullptr)
+          mbar_wait(&full[j % C::kStages], (j / C::kStages) & 1, p.status);
     }
   } else if (warp == 1) {
     // -------------------------------------------------------- MMA issuer --
@@ -354,7 +357,31 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int r = tid >> 1, hf = tid & 1;
     pdl_wait();
     tile_range();
-    for (int it = 0; it < ntile; ++it) {
+    // Tile `it`: selected entries are fetched here (thread pair r gathers
+    // row r, half hf each, 16 bytes per cp.async) once the stage is free;
+    // every thread then arrives on full[s] (after its copies land).
+    auto fetch = [&](int it) -> bool {
+      const int s = it % C::kStages;
+      const int t = t0 + it;
+      if (p.sel_idx != nullptr && t < tiles_c) {
+        const int j = t * TN + r;
+        int64_t i = j < n_c ? (int64_t)p.sel_idx[(int64_t)row * p.kmax + j] : 0;
+        if (i < 0 || i >= n_vis) i = 0;  // invalid rows: any real row (masked)
+        if (!wait_all(&empty[s], ((it / C::kStages) & 1) ^ 1, p, abort_flag)) return false;
+        const __nv_bfloat16* src = p.kv_c + ((int64_t)b * p.N_cap + i) * D + hf * (D / 2);
+        uint8_t* st = stages + s * C::kStageBytes;
+#pragma unroll
+        for (int c = 0; c < D / 16; ++c) cp_async_16(st + tile_off(r, hf * (D / 2) + 8 * c), src + 8 * c);
+        cp_async_arrive(&full[s]);
+      } else {
+        mbar_arrive(&full[s]);
+      }
+      return true;
+    };
+    constexpr int kAhead = C::kStages - 1;
+    bool fetch_ok = true;
+    for (int it = 0; it < kAhead && it < ntile && fetch_ok; ++it) fetch_ok = fetch(it);
+    for (int it = 0; it < ntile && fetch_ok; ++it) {
       const int s = it % C::kStages;
       if (!wait_all(&full[s], (it / C::kStages) & 1, p, abort_flag)) break;
       Meta& M = meta[s];
@@ -415,7 +442,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       fence_proxy_async_smem();
       mbar_arrive(&ready[s]);
+      if (it + kAhead < ntile) fetch_ok = fetch(it + kAhead);
     }
+    cp_async_wait_all();  // no copy may still target shared memory at exit
   } else {
     // ------------------------------------------------- softmax / epilogue --
     // The warp with TMEM lane quarter q serves heads 16q .. 16q+15 of this
@@ -616,9 +645,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   }
+  // Teardown: every warp reports (converged) that it is done with tensor
+  // memory; warp 0 frees it after all of them (bounded wait).
+  __syncwarp();
   tc_fence_before();
-  __syncthreads();
+  if (lane == 0) mbar_arrive(done);
   if (warp == 0) {
+    wait_all(done, 0, p, nullptr);
     tc_fence_after();
     tmem_dealloc(tmem, C::kAlloc);
   }
@@ -748,6 +781,7 @@ cudaError_t launch_impl(const MqaLaunch& a, cudaStream_t stream) {
   p.pos_base = a.pos_base;
   p.sel_idx = a.sel_idx;
   p.sel_cnt = a.sel_cnt;
+  p.kv_c = reinterpret_cast<const __nv_bfloat16*>(a.kv_c);
   p.kmax = a.kmax;
   p.gamma_q = a.gamma_q;
   p.gamma_kv = a.gamma_kv;

@@ -65,10 +65,20 @@ struct Shared {
   uint32_t bcast[4];
 };
 
+// The aligned barriers below need converged warps: each helper reconverges
+// its warp first.
 CSA_DEV void cluster_arrive() {
+  __syncwarp();
   asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
 }
-CSA_DEV void cluster_wait() { asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory"); }
+CSA_DEV void cluster_wait() {
+  __syncwarp();
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+CSA_DEV void cta_sync() {
+  __syncwarp();
+  __syncthreads();
+}
 CSA_DEV void st_remote_v2(uint32_t caddr, uint32_t a, uint32_t b) {
   asm volatile("st.shared::cluster.v2.u32 [%0], {%1, %2};" ::"r"(caddr), "r"(a), "r"(b)
                : "memory");
@@ -132,7 +142,7 @@ __global__ void __launch_bounds__(kThreads, 1) topk_kernel(const Params p) {
     sh.warp_a[warp] = kmin;
     sh.warp_b[warp] = kmax;
   }
-  __syncthreads();
+  cta_sync();
   cluster_wait();  // every CTA of the cluster is running
   // Round 0: (min, max) of this CTA into slot r of every CTA.
   if (warp == 0) {
@@ -184,7 +194,7 @@ __global__ void __launch_bounds__(kThreads, 1) topk_kernel(const Params p) {
           atomicAdd(&loc[bin], 1u);
         }
       }
-      __syncthreads();
+      cta_sync();
       // Push: this CTA's histogram into slot r of every CTA (16-byte stores);
       // the other threads clear next round's local histogram.
       constexpr int kVec = kBins / 4;
@@ -212,7 +222,7 @@ __global__ void __launch_bounds__(kThreads, 1) topk_kernel(const Params p) {
         }
         if (lane == 31) sh.warp_a[warp] = incl;
       }
-      __syncthreads();
+      cta_sync();
       if (tid < nb) {
         for (int w2 = 0; w2 < warp; ++w2) incl += sh.warp_a[w2];
         const uint32_t above = incl - cnt_t;
@@ -222,7 +232,7 @@ __global__ void __launch_bounds__(kThreads, 1) topk_kernel(const Params p) {
           sh.bcast[2] = cnt_t;
         }
       }
-      __syncthreads();
+      cta_sync();
       const uint32_t d = sh.bcast[0], abv = sh.bcast[1], cnt_d = sh.bcast[2];
       k_rem -= abv;
       prefix |= d << shift;
@@ -249,12 +259,12 @@ __global__ void __launch_bounds__(kThreads, 1) topk_kernel(const Params p) {
     n_gt += __shfl_xor_sync(0xffffffffu, n_gt, o);
     n_eq += __shfl_xor_sync(0xffffffffu, n_eq, o);
   }
-  __syncthreads();  // bcast / warp slots of the last round are read
+  cta_sync();  // bcast / warp slots of the last round are read
   if (lane == 0) {
     sh.warp_a[warp] = n_gt;
     sh.warp_b[warp] = n_eq;
   }
-  __syncthreads();
+  cta_sync();
   if (warp == 0) {
     const uint32_t a = sh.warp_a[lane], b = sh.warp_b[lane];
     uint32_t sa = a, sb = b;
