@@ -116,6 +116,16 @@ CSA_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, int32_t* status,
   }
 }
 
+// Bulk copy of `bytes` (multiple of 16, both addresses 16-byte aligned)
+// from shared to global memory, tracked by this thread's bulk group.
+CSA_DEV void bulk_store(void* gdst, const void* ssrc, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst),
+               "r"(smem_u32(ssrc)), "r"(bytes)
+               : "memory");
+}
+CSA_DEV void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+CSA_DEV void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 // 16-byte global -> shared copy through L2 (LSU path), and an mbarrier
 // arrival that fires once this thread's earlier copies have landed (counts
 // as one of the barrier's expected arrivals).

@@ -130,7 +130,7 @@ CSA_DEV bool wait_all(uint64_t* bar, uint32_t parity, const Params& p, volatile 
 
 template <int D, int R>
 __global__ void __launch_bounds__(kThreads, 1)
-    mqa_heads_kernel(const __grid_constant__ CUtensorMap map_c,
+    mqa_heads_kernel(const __grid_constant__ CUtensorMap map_q,
                      const __grid_constant__ CUtensorMap map_t,
                      const __grid_constant__ CUtensorMap box_c,
                      const __grid_constant__ CUtensorMap box_t, const Params p) {
@@ -151,7 +151,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* qready = pvdone + 1;
   uint64_t* drain = qready + 1;
   uint64_t* done = drain + 1;  // one arrival per warp when its role is over
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+  uint64_t* qfull = done + 1;  // the query block landed in the last stage
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(qfull + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -169,20 +170,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int nwin = (p.W > 0 && pos >= 0) ? (int)(pos - w0 + 1) : 0;
   // This split's tiles [t0, t1) of the list; the selection count comes from
   // the top-k kernel, so every role calls this after pdl_wait().
-  int n_c = 0, tiles_c = 0, t0 = 0, t1 = 0, ntile = 0;
-  auto tile_range = [&]() {
-    if (p.sel_idx) {
-      const int c = p.sel_cnt[row];
-      n_c = c < 0 ? 0 : (c > p.kmax ? p.kmax : c);
-    } else {
-      n_c = (int)n_vis;
-    }
-    tiles_c = (n_c + TN - 1) / TN;
-    const int tiles_all = tiles_c + (nwin + TN - 1) / TN;
-    const int tps = (tiles_all + p.splits - 1) / p.splits;
-    t0 = std::min(split * tps, tiles_all);
-    t1 = std::min(t0 + tps, tiles_all);
-    ntile = t1 - t0;
+  // With a selection the list is laid out for kmax entries (the tiles past
+  // the selection count hold only masked rows), so the tile range does not
+  // wait for the count; the count is read after pdl_wait() where needed.
+  const int n_list = p.sel_idx ? p.kmax : (int)n_vis;
+  const int tiles_c = (n_list + TN - 1) / TN;
+  const int tiles_all = tiles_c + (nwin + TN - 1) / TN;
+  const int tps = (tiles_all + p.splits - 1) / p.splits;
+  const int t0 = std::min(split * tps, tiles_all);
+  const int t1 = std::min(t0 + tps, tiles_all);
+  const int ntile = t1 - t0;
+  auto sel_count = [&]() -> int {
+    if (!p.sel_idx) return (int)n_vis;
+    const int c = p.sel_cnt[row];
+    return c < 0 ? 0 : (c > p.kmax ? p.kmax : c);
   };
 
   float* pml = p.part_ml + ((int64_t)row * p.splits + split) * 2 * p.H;
@@ -202,6 +203,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(qready, 128);
     mbar_init(drain, 1);
     mbar_init(done, kThreads / 32);
+    mbar_init(qfull, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -223,12 +225,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Contiguous tiles (dense entries, window tokens): one 64-row box per
     // 128-byte chunk.  Selected entries: row gathers (tile::gather4), issued
     // by every lane of the warp.
+    // The query block first (a caller input: no need to wait for the
+    // previous kernel): 64 heads x D into the last stage, freed by qready.
+    if (lane == 0) {
+      mbar_expect_tx(qfull, C::kStageBytes);
+      for (int c = 0; c < C::NC; ++c)
+        tma_load_2d(stages + (C::kStages - 1) * C::kStageBytes + c * C::kChunkBytes, &map_q, qfull,
+                    c * 64, row * p.H + hg0);
+    }
     pdl_wait();
-    tile_range();
+    const int n_c = sel_count();
     int it = 0;
     for (int t = t0; t < t1; ++t, ++it) {
       const int s = it % C::kStages;
       const uint32_t ph = (it / C::kStages) & 1;
+      // The last stage holds the query block until the prologue is done.
+      if (it == C::kStages - 1 && !wait_all(qready, 0, p, abort_flag)) break;
       const bool win = t >= tiles_c;
       const bool gathered = !win && p.sel_idx != nullptr;
       int32_t grow[2], rpos[2];
@@ -300,8 +312,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr int kPvN = D >= 256 ? 256 : D;  // N of one P.V instruction
     const uint32_t idesc_s = idesc_bf16(64, TN, 0, 0);
     const uint32_t idesc_pv = idesc_bf16(64, kPvN, 0, 1);
-    pdl_wait();
-    tile_range();
     const bool ok = wait_all(qready, 0, p, abort_flag);
     tc_fence_after();
     bool issued = false;
@@ -356,7 +366,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int tid = threadIdx.x - 64;  // 0..127
     const int r = tid >> 1, hf = tid & 1;
     pdl_wait();
-    tile_range();
+    const int n_c = sel_count();
     // Tile `it`: selected entries are fetched here (thread pair r gathers
     // row r, half hf each, 16 bytes per cp.async) once the stage is free;
     // every thread then arrives on full[s] (after its copies land).
@@ -368,6 +378,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         int64_t i = j < n_c ? (int64_t)p.sel_idx[(int64_t)row * p.kmax + j] : 0;
         if (i < 0 || i >= n_vis) i = 0;  // invalid rows: any real row (masked)
         if (!wait_all(&empty[s], ((it / C::kStages) & 1) ^ 1, p, abort_flag)) return false;
+        if (it == C::kStages - 1 && !wait_all(qready, 0, p, abort_flag)) return false;
         const __nv_bfloat16* src = p.kv_c + ((int64_t)b * p.N_cap + i) * D + hf * (D / 2);
         uint8_t* st = stages + s * C::kStageBytes;
 #pragma unroll
@@ -461,13 +472,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     // columns) writes 64 dims of both halves.  The rotated dims (the last R)
     // all sit in the last 64-dim chunk of half 1.
     {
-      const __nv_bfloat16* qr =
-          p.q + ((int64_t)row * p.H + (head_ok ? hg : 0)) * D + hf * (D / 2);
+      // The block is in the last stage (TMA, 128-byte swizzled chunks):
+      // row hl, dims [hf*D/2, hf*D/2 + D/2).
+      const uint8_t* qs = stages + (C::kStages - 1) * C::kStageBytes;
+      const int d_half = hf * (D / 2);
       constexpr int NU = D / 16;  // 16-byte units of a half row
+      const bool qok = wait_all(qfull, 0, p, abort_flag);
       float ss = 0.f;
 #pragma unroll 8
       for (int c = 0; c < NU; ++c) {
-        const uint4 v = __ldg(reinterpret_cast<const uint4*>(qr) + c);
+        const uint4 v = *reinterpret_cast<const uint4*>(qs + tile_off(hl, d_half + 8 * c));
         const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
@@ -476,7 +490,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       ss += __shfl_xor_sync(0xffffffffu, ss, 16);  // the row's other half
-      const float inv = head_ok ? 1.0f / sqrtf(ss / (float)D + p.eps) : 0.f;
+      const float inv = (head_ok && qok) ? 1.0f / sqrtf(ss / (float)D + p.eps) : 0.f;
       const float* gq = p.gamma_q ? p.gamma_q + hf * (D / 2) : nullptr;
       constexpr int kChunks = D / 128;  // 64-dim chunks per half row
 #pragma unroll 1
@@ -484,7 +498,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         float x[64];
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
-          const uint4 v = __ldg(reinterpret_cast<const uint4*>(qr) + 8 * c + u);
+          const uint4 v =
+              *reinterpret_cast<const uint4*>(qs + tile_off(hl, d_half + 64 * c + 8 * u));
           const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
@@ -525,7 +540,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive(qready);
     }
     pdl_wait();  // the query prologue above overlaps the previous kernel
-    tile_range();
 
     float m_run = -INFINITY, l_run = 0.f;
     for (int it = 0; it < ntile; ++it) {
@@ -624,20 +638,28 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     } else if (!*abort_flag && wait_all(pvdone, (ntile - 1) & 1, p, abort_flag)) {
       tc_fence_after();
+      // O rows go through shared memory (the stages are free now: every
+      // MMA has completed) and leave as one bulk copy per half row.
       float* po = p.part_o + (((int64_t)row * p.splits + split) * p.H + (head_ok ? hg : 0)) * D +
                   hf * (D / 2);
+      constexpr int kORow = D * 4 + 16;  // padded row: 4-way bank spread
+      float* ob = reinterpret_cast<float*>(stages + hl * kORow) + hf * (D / 2);
 #pragma unroll 1
       for (int c = 0; c < D / 2; c += 32) {
         uint32_t v[32];
         tmem_ld_16x32bx2_x32<D / 2>(t_o + lq + c, v);
         tmem_wait_ld();
-        if (head_ok) {
 #pragma unroll
-          for (int j = 0; j < 32; j += 4)
-            *reinterpret_cast<float4*>(po + c + j) =
-                make_float4(__uint_as_float(v[j]), __uint_as_float(v[j + 1]),
-                            __uint_as_float(v[j + 2]), __uint_as_float(v[j + 3]));
-        }
+        for (int j = 0; j < 32; j += 4)
+          *reinterpret_cast<float4*>(ob + c + j) =
+              make_float4(__uint_as_float(v[j]), __uint_as_float(v[j + 1]),
+                          __uint_as_float(v[j + 2]), __uint_as_float(v[j + 3]));
+      }
+      if (head_ok) {
+        fence_proxy_async_smem();
+        bulk_store(po, ob, (D / 2) * 4);
+        bulk_commit();
+        bulk_wait_all();
       }
       if (head_ok && hf == 0) {
         pml[hg] = m_run;  // log2 domain
@@ -795,9 +817,9 @@ cudaError_t launch_impl(const MqaLaunch& a, cudaStream_t stream) {
   if (rows > 65535 || a.splits * 2 > 65535) return cudaErrorInvalidConfiguration;
 
   // Row-gather maps (one-row boxes) and 64-row box maps, 128-byte swizzle.
-  CUtensorMap map_c, map_t, box_c, box_t;
-  cudaError_t e = make_tmap_2d(&map_c, a.kv_c, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
-                               (uint64_t)a.B * a.N_cap, D, 1, 64, CU_TENSOR_MAP_SWIZZLE_128B);
+  CUtensorMap map_q, map_t, box_c, box_t;
+  cudaError_t e = make_tmap_2d(&map_q, a.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                               (uint64_t)rows * a.H, D, TN, 64, CU_TENSOR_MAP_SWIZZLE_128B);
   if (e != cudaSuccess) return e;
   e = make_tmap_2d(&map_t, a.kv_tok, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)a.B * a.L_cap,
                    D, 1, 64, CU_TENSOR_MAP_SWIZZLE_128B);
@@ -815,7 +837,7 @@ cudaError_t launch_impl(const MqaLaunch& a, cudaStream_t stream) {
   e = ensure_smem_attr(reinterpret_cast<const void*>(kern), 3 + (D == 512 ? 0 : 3) + R / 32, smem);
   if (e != cudaSuccess) return e;
   dim3 grid(2 * a.splits, rows, 1);
-  e = launch_pdl(kern, grid, dim3(kThreads), smem, stream, 0, map_c, map_t, box_c, box_t, p);
+  e = launch_pdl(kern, grid, dim3(kThreads), smem, stream, 0, map_q, map_t, box_c, box_t, p);
   if (e != cudaSuccess) return e;
   return launch_pdl(mqa_combine_kernel, dim3(rows, a.H), dim3(128),
                     (size_t)(D + a.splits) * sizeof(float), stream, 0, p, D, a.sink,
