@@ -234,9 +234,22 @@ __global__ void __launch_bounds__(kThreads, 1)
                     c * 64, row * p.H + hg0);
     }
     pdl_wait();
+    // Selected indices of the next tile are loaded one tile ahead, and
+    // independently of the selection count (both round trips overlap).
+    auto load_idx = [&](int t, int hh) -> int64_t {
+      const int j = t * TN + lane + 32 * hh;
+      return (p.sel_idx && t < tiles_c && j < p.kmax) ? (int64_t)p.sel_idx[(int64_t)row * p.kmax + j]
+                                                       : 0;
+    };
+    int64_t nxt0 = load_idx(t0, 0), nxt1 = load_idx(t0, 1);
     const int n_c = sel_count();
     int it = 0;
     for (int t = t0; t < t1; ++t, ++it) {
+      const int64_t cur[2] = {nxt0, nxt1};
+      if (t + 1 < t1) {
+        nxt0 = load_idx(t + 1, 0);
+        nxt1 = load_idx(t + 1, 1);
+      }
       const int s = it % C::kStages;
       const uint32_t ph = (it / C::kStages) & 1;
       // The last stage holds the query block until the prologue is done.
@@ -253,7 +266,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           valid[hh] = j < n_c;
           int64_t i = j;
           if (valid[hh] && gathered) {
-            i = p.sel_idx[(int64_t)row * p.kmax + j];
+            i = cur[hh];
             if (i < 0 || i >= n_vis) {
               report(p.status, CSA_ERR_DEVICE_INDEX);
               valid[hh] = false;
@@ -370,13 +383,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Tile `it`: selected entries are fetched here (thread pair r gathers
     // row r, half hf each, 16 bytes per cp.async) once the stage is free;
     // every thread then arrives on full[s] (after its copies land).
-    auto fetch = [&](int it) -> bool {
+    // Row index of thread pair r in tile `it` (loaded ahead of the fetch).
+    auto row_index = [&](int it) -> int64_t {
+      const int t = t0 + it, j = t * TN + r;
+      return (p.sel_idx && t < tiles_c && j < p.kmax) ? (int64_t)p.sel_idx[(int64_t)row * p.kmax + j]
+                                                       : 0;
+    };
+    auto fetch = [&](int it, int64_t i) -> bool {
       const int s = it % C::kStages;
       const int t = t0 + it;
       if (p.sel_idx != nullptr && t < tiles_c) {
         const int j = t * TN + r;
-        int64_t i = j < n_c ? (int64_t)p.sel_idx[(int64_t)row * p.kmax + j] : 0;
-        if (i < 0 || i >= n_vis) i = 0;  // invalid rows: any real row (masked)
+        if (j >= n_c || i < 0 || i >= n_vis) i = 0;  // masked rows: any real row
         if (!wait_all(&empty[s], ((it / C::kStages) & 1) ^ 1, p, abort_flag)) return false;
         if (it == C::kStages - 1 && !wait_all(qready, 0, p, abort_flag)) return false;
         const __nv_bfloat16* src = p.kv_c + ((int64_t)b * p.N_cap + i) * D + hf * (D / 2);
@@ -391,7 +409,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
     constexpr int kAhead = C::kStages - 1;
     bool fetch_ok = true;
-    for (int it = 0; it < kAhead && it < ntile && fetch_ok; ++it) fetch_ok = fetch(it);
+    {
+      int64_t ri[kAhead];
+#pragma unroll
+      for (int u = 0; u < kAhead; ++u) ri[u] = u < ntile ? row_index(u) : 0;
+#pragma unroll
+      for (int u = 0; u < kAhead; ++u)
+        if (u < ntile && fetch_ok) fetch_ok = fetch(u, ri[u]);
+    }
+    int64_t nxt = kAhead < ntile ? row_index(kAhead) : 0;
     for (int it = 0; it < ntile && fetch_ok; ++it) {
       const int s = it % C::kStages;
       if (!wait_all(&full[s], (it / C::kStages) & 1, p, abort_flag)) break;
@@ -453,7 +479,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       fence_proxy_async_smem();
       mbar_arrive(&ready[s]);
-      if (it + kAhead < ntile) fetch_ok = fetch(it + kAhead);
+      if (it + kAhead < ntile) {
+        const int64_t cur = nxt;
+        if (it + kAhead + 1 < ntile) nxt = row_index(it + kAhead + 1);
+        fetch_ok = fetch(it + kAhead, cur);
+      }
     }
     cp_async_wait_all();  // no copy may still target shared memory at exit
   } else {
@@ -477,6 +507,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint8_t* qs = stages + (C::kStages - 1) * C::kStageBytes;
       const int d_half = hf * (D / 2);
       constexpr int NU = D / 16;  // 16-byte units of a half row
+      // The query's rotation angles (one position for every head): lane j
+      // of each softmax warp computes pair j into the (still unused) P
+      // buffer, so the rotating threads read them instead of each
+      // recomputing all of them.
+      float2* qang = reinterpret_cast<float2*>(pbuf) + 32 * q;
+      if constexpr (R > 0) {
+        if (lane < R / 2) {
+          float sn, cs;
+          sincos_reduced((double)pos * p.inv_freq[lane], &sn, &cs);
+          qang[lane] = make_float2(sn, cs);
+        }
+        __syncwarp();
+      }
       const bool qok = wait_all(qfull, 0, p, abort_flag);
       float ss = 0.f;
 #pragma unroll 8
@@ -522,8 +565,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             constexpr int half = R / 2, b0 = 64 - R;
 #pragma unroll
             for (int j = 0; j < half; ++j) {
-              float sn, cs;
-              sincos_reduced((double)pos * p.inv_freq[j], &sn, &cs);
+              const float2 sc = qang[j];
+              const float sn = sc.x, cs = sc.y;
               const float a1 = x[b0 + j], a2 = x[b0 + half + j];
               x[b0 + j] = a1 * cs - a2 * sn;
               x[b0 + half + j] = a2 * cs + a1 * sn;
