@@ -425,9 +425,9 @@ static csa_status mqa_common(const char* fn, const csa_params* p, csa_op op, int
   a.out = out;
   a.lse = lse;
   a.splits = splits;
-  a.part_o = static_cast<float*>(ws);
+  a.part_o = ws;
   a.part_ml = reinterpret_cast<float*>(static_cast<char*>(ws) +
-                                       round_up((size_t)rows * splits * p->H * p->d * 4, 256));
+                                       round_up((size_t)rows * splits * p->H * p->d * 2, 256));
   a.status = dev_status;
   cudaError_t e = csa::launch_mqa(a, stream);
   if (e != cudaSuccess) return cuda_fail(fn, e);

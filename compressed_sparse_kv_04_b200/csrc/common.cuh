@@ -5,6 +5,7 @@
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_fp8.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -392,6 +393,7 @@ CSA_DEV float fast_exp2(float x) {
 
 CSA_DEV float bf16_lo(uint32_t u) { return __uint_as_float(u << 16); }
 CSA_DEV float bf16_hi(uint32_t u) { return __uint_as_float(u & 0xFFFF0000u); }
+CSA_DEV uint32_t h2_bits(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
 CSA_DEV uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);

@@ -238,15 +238,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int c = 0; c < 4; ++c)
           if (c * 16 < p.HP) tmem_ld16(col + c * 16, v[c]);
         tmem_wait_ld();
-        float acc = 0.f;
+        float a4[4] = {0.f, 0.f, 0.f, 0.f};  // independent FMA chains
         const float* wg = wq + g * p.HP;
 #pragma unroll
         for (int c = 0; c < 4; ++c)
           if (c * 16 < p.HP) {
 #pragma unroll
             for (int j = 0; j < 16; ++j)
-              acc = fmaf(wg[c * 16 + j], fmaxf(__uint_as_float(v[c][j]), 0.f), acc);
+              a4[j & 3] = fmaf(wg[c * 16 + j], fmaxf(__uint_as_float(v[c][j]), 0.f), a4[j & 3]);
           }
+        const float acc = (a4[0] + a4[1]) + (a4[2] + a4[3]);
         if (entry < nv[g < 8 ? g : 7])
           p.scores[((int64_t)b * p.Q + q0 + g) * p.N_cap + entry] = acc * ks;
       }

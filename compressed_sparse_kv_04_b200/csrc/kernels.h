@@ -81,7 +81,7 @@ struct MqaLaunch {
   double inv_freq[64];      // rope_dim/2 entries
   void* out;                // [B*Q, H, D] bf16
   float* lse;               // [B*Q, H] or null
-  float* part_o;            // workspace [rows, S, H, D] fp32
+  void* part_o;             // workspace [rows, S, H, D] fp16: split output / split sum
   float* part_ml;           // workspace [rows, S, 2, H] fp32
   int splits;               // S
   int32_t* status;

@@ -45,7 +45,7 @@
 namespace csa {
 
 size_t mqa_workspace_bytes(int rows, int splits, int H, int D) {
-  size_t o = (size_t)rows * splits * H * D * 4;
+  size_t o = (size_t)rows * splits * H * D * 2;  // fp16 partial outputs
   o = (o + 255) / 256 * 256;
   return o + (size_t)rows * splits * 2 * H * 4;
 }
@@ -103,7 +103,7 @@ struct Params {
   const float* gamma_q;
   const float* gamma_kv;
   float eps, scale_log2;  // softmax scale * log2(e)
-  float* part_o;
+  __half* part_o;  // [rows, S, H, D]: the split's output divided by its sum
   float* part_ml;
   int32_t* status;
   double inv_freq[64];
@@ -383,9 +383,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Tile `it`: selected entries are fetched here (thread pair r gathers
     // row r, half hf each, 16 bytes per cp.async) once the stage is free;
     // every thread then arrives on full[s] (after its copies land).
-    // Row index of thread pair r in tile `it` (loaded ahead of the fetch).
+    // Gathers: transform warp tw copies rows tw, tw+4, ..., tw+60 of the
+    // tile, a whole row per pair of instructions (lane l: 16 bytes at
+    // 16*l and 512+16*l), so each instruction reads 512 contiguous bytes.
+    // Lane l (< 16) holds the index of row tw + 4*l, loaded ahead.
+    const int tw = tid >> 5, tl = tid & 31;
     auto row_index = [&](int it) -> int64_t {
-      const int t = t0 + it, j = t * TN + r;
+      const int t = t0 + it, j = t * TN + tw + 4 * (tl & 15);
       return (p.sel_idx && t < tiles_c && j < p.kmax) ? (int64_t)p.sel_idx[(int64_t)row * p.kmax + j]
                                                        : 0;
     };
@@ -393,14 +397,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int s = it % C::kStages;
       const int t = t0 + it;
       if (p.sel_idx != nullptr && t < tiles_c) {
-        const int j = t * TN + r;
-        if (j >= n_c || i < 0 || i >= n_vis) i = 0;  // masked rows: any real row
+        const int j = t * TN + tw + 4 * (tl & 15);
+        if (j >= n_c || i < 0 || i >= n_vis) i = -1;  // masked row: not fetched (zeroed later)
         if (!wait_all(&empty[s], ((it / C::kStages) & 1) ^ 1, p, abort_flag)) return false;
         if (it == C::kStages - 1 && !wait_all(qready, 0, p, abort_flag)) return false;
-        const __nv_bfloat16* src = p.kv_c + ((int64_t)b * p.N_cap + i) * D + hf * (D / 2);
         uint8_t* st = stages + s * C::kStageBytes;
+        constexpr int kUnits = D / 8;  // 16-byte units per row
+#pragma unroll 4
+        for (int u = 0; u < TN / 4; ++u) {
+          const int64_t iu = __shfl_sync(0xffffffffu, i, u);
+          if (iu < 0) continue;
+          const int rr = tw + 4 * u;
+          const __nv_bfloat16* src = p.kv_c + ((int64_t)b * p.N_cap + iu) * D;
 #pragma unroll
-        for (int c = 0; c < D / 16; ++c) cp_async_16(st + tile_off(r, hf * (D / 2) + 8 * c), src + 8 * c);
+          for (int h = 0; h < (kUnits + 31) / 32; ++h) {
+            const int unit = 32 * h + tl;
+            if (unit < kUnits) cp_async_16(st + tile_off(rr, 8 * unit), src + 8 * unit);
+          }
+        }
         cp_async_arrive(&full[s]);
       } else {
         mbar_arrive(&full[s]);
@@ -424,15 +438,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       Meta& M = meta[s];
       uint8_t* st = stages + s * C::kStageBytes;
       const bool valid = (M.valid[r >> 5] >> (r & 31)) & 1u;
+      if (!valid) {  // masked rows enter P.V with P = 0: make them finite zeros
+        for (int c = hf; c < D / 8; c += 2)
+          *reinterpret_cast<uint4*>(st + tile_off(r, c * 8)) = make_uint4(0u, 0u, 0u, 0u);
+      }
       float ss = 0.f;
       if (valid && M.window) {
+        float a4[4] = {0.f, 0.f, 0.f, 0.f};  // independent chains, loads in flight
+#pragma unroll 8
         for (int c = hf; c < D / 8; c += 2) {  // 16-byte units
           uint4 u = *reinterpret_cast<const uint4*>(st + tile_off(r, c * 8));
           uint32_t w4[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const float lo = bf16_lo(w4[e]), hi = bf16_hi(w4[e]);
-            ss = fmaf(lo, lo, fmaf(hi, hi, ss));
+            a4[e] = fmaf(lo, lo, fmaf(hi, hi, a4[e]));
           }
           if (p.gamma_kv) {
             const float* g = p.gamma_kv + c * 8;
@@ -444,6 +464,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 make_uint4(w4[0], w4[1], w4[2], w4[3]);
           }
         }
+        ss = (a4[0] + a4[1]) + (a4[2] + a4[3]);
       }
       ss += __shfl_xor_sync(0xffffffffu, ss, 1);
       if (hf == 0) M.rn[r] = (valid && M.window) ? 1.0f / sqrtf(ss / (float)D + p.eps) : 1.0f;
@@ -521,7 +542,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
       }
       const bool qok = wait_all(qfull, 0, p, abort_flag);
-      float ss = 0.f;
+      float a4[4] = {0.f, 0.f, 0.f, 0.f};  // independent chains, loads in flight
 #pragma unroll 8
       for (int c = 0; c < NU; ++c) {
         const uint4 v = *reinterpret_cast<const uint4*>(qs + tile_off(hl, d_half + 8 * c));
@@ -529,9 +550,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const float lo = bf16_lo(w4[e]), hi = bf16_hi(w4[e]);
-          ss = fmaf(lo, lo, fmaf(hi, hi, ss));
+          a4[e] = fmaf(lo, lo, fmaf(hi, hi, a4[e]));
         }
       }
+      float ss = (a4[0] + a4[1]) + (a4[2] + a4[3]);
       ss += __shfl_xor_sync(0xffffffffu, ss, 16);  // the row's other half
       const float inv = (head_ok && qok) ? 1.0f / sqrtf(ss / (float)D + p.eps) : 0.f;
       const float* gq = p.gamma_q ? p.gamma_q + hf * (D / 2) : nullptr;
@@ -681,26 +703,32 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     } else if (!*abort_flag && wait_all(pvdone, (ntile - 1) & 1, p, abort_flag)) {
       tc_fence_after();
-      // O rows go through shared memory (the stages are free now: every
-      // MMA has completed) and leave as one bulk copy per half row.
-      float* po = p.part_o + (((int64_t)row * p.splits + split) * p.H + (head_ok ? hg : 0)) * D +
-                  hf * (D / 2);
-      constexpr int kORow = D * 4 + 16;  // padded row: 4-way bank spread
-      float* ob = reinterpret_cast<float*>(stages + hl * kORow) + hf * (D / 2);
+      // O / l rows (fp16: |O / l| is at most the largest |v|) go through
+      // shared memory (the stages are free now: every MMA has completed)
+      // and leave as one bulk copy per half row.
+      __half* po = p.part_o + (((int64_t)row * p.splits + split) * p.H + (head_ok ? hg : 0)) * D +
+                   hf * (D / 2);
+      constexpr int kORow = D * 2 + 16;  // padded row: spreads the banks
+      __half* ob = reinterpret_cast<__half*>(stages + hl * kORow) + hf * (D / 2);
+      const float inv_l = l_run > 0.f ? 1.0f / l_run : 0.f;
 #pragma unroll 1
       for (int c = 0; c < D / 2; c += 32) {
         uint32_t v[32];
         tmem_ld_16x32bx2_x32<D / 2>(t_o + lq + c, v);
         tmem_wait_ld();
 #pragma unroll
-        for (int j = 0; j < 32; j += 4)
-          *reinterpret_cast<float4*>(ob + c + j) =
-              make_float4(__uint_as_float(v[j]), __uint_as_float(v[j + 1]),
-                          __uint_as_float(v[j + 2]), __uint_as_float(v[j + 3]));
+        for (int j = 0; j < 32; j += 8) {
+          uint4 u;
+          u.x = h2_bits(__floats2half2_rn(__uint_as_float(v[j]) * inv_l, __uint_as_float(v[j + 1]) * inv_l));
+          u.y = h2_bits(__floats2half2_rn(__uint_as_float(v[j + 2]) * inv_l, __uint_as_float(v[j + 3]) * inv_l));
+          u.z = h2_bits(__floats2half2_rn(__uint_as_float(v[j + 4]) * inv_l, __uint_as_float(v[j + 5]) * inv_l));
+          u.w = h2_bits(__floats2half2_rn(__uint_as_float(v[j + 6]) * inv_l, __uint_as_float(v[j + 7]) * inv_l));
+          *reinterpret_cast<uint4*>(ob + c + j) = u;
+        }
       }
       if (head_ok) {
         fence_proxy_async_smem();
-        bulk_store(po, ob, (D / 2) * 4);
+        bulk_store(po, ob, (D / 2) * 2);
         bulk_commit();
         bulk_wait_all();
       }
@@ -752,9 +780,9 @@ __global__ void __launch_bounds__(128) mqa_combine_kernel(const Params p, int D,
     if (M != -INFINITY && z != INFINITY) {
       for (int s = lane; s < S; s += 32) {
         const float ms = ml[(int64_t)s * 2 * p.H + h];
-        const float w = ms == -INFINITY ? 0.f : exp2f(ms - M);
-        wsplit[s] = w;
-        L = fmaf(ml[(int64_t)s * 2 * p.H + p.H + h], w, L);
+        const float w = ms == -INFINITY ? 0.f : ml[(int64_t)s * 2 * p.H + p.H + h] * exp2f(ms - M);
+        wsplit[s] = w;  // the split's stored output is O / l
+        L += w;
       }
       L = warp_sum(L);
       if (z2 != -INFINITY) L += exp2f(z2 - M);
@@ -774,31 +802,27 @@ __global__ void __launch_bounds__(128) mqa_combine_kernel(const Params p, int D,
   }
   const float invL = 1.0f / L;
   for (int d4 = threadIdx.x; d4 < D / 4; d4 += blockDim.x) {
-    const float* src = p.part_o + ((int64_t)row * S * p.H + h) * D + 4 * d4;
+    const __half* src = p.part_o + ((int64_t)row * S * p.H + h) * D + 4 * d4;
     const int64_t stride = (int64_t)p.H * D;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    auto add = [&](uint2 u, float w) {
+      if (w == 0.f) return;  // empty split: its partial was never written
+      const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&u.x));
+      const float2 c = __half22float2(*reinterpret_cast<const __half2*>(&u.y));
+      acc.x = fmaf(a.x, w, acc.x);
+      acc.y = fmaf(a.y, w, acc.y);
+      acc.z = fmaf(c.x, w, acc.z);
+      acc.w = fmaf(c.y, w, acc.w);
+    };
     int s = 0;
     for (; s + 4 <= S; s += 4) {
-      float4 v[4];
+      uint2 v[4];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) v[u] = __ldg(reinterpret_cast<const float4*>(src + (s + u) * stride));
+      for (int u = 0; u < 4; ++u) v[u] = __ldg(reinterpret_cast<const uint2*>(src + (s + u) * stride));
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const float w = wsplit[s + u];
-        acc.x = fmaf(v[u].x, w, acc.x);
-        acc.y = fmaf(v[u].y, w, acc.y);
-        acc.z = fmaf(v[u].z, w, acc.z);
-        acc.w = fmaf(v[u].w, w, acc.w);
-      }
+      for (int u = 0; u < 4; ++u) add(v[u], wsplit[s + u]);
     }
-    for (; s < S; ++s) {
-      const float4 v = __ldg(reinterpret_cast<const float4*>(src + s * stride));
-      const float w = wsplit[s];
-      acc.x = fmaf(v.x, w, acc.x);
-      acc.y = fmaf(v.y, w, acc.y);
-      acc.z = fmaf(v.z, w, acc.z);
-      acc.w = fmaf(v.w, w, acc.w);
-    }
+    for (; s < S; ++s) add(__ldg(reinterpret_cast<const uint2*>(src + s * stride)), wsplit[s]);
     so[4 * d4] = acc.x * invL;
     so[4 * d4 + 1] = acc.y * invL;
     so[4 * d4 + 2] = acc.z * invL;
@@ -852,7 +876,7 @@ cudaError_t launch_impl(const MqaLaunch& a, cudaStream_t stream) {
   p.gamma_kv = a.gamma_kv;
   p.eps = a.eps;
   p.scale_log2 = a.scale * 1.4426950408889634f;
-  p.part_o = a.part_o;
+  p.part_o = reinterpret_cast<__half*>(a.part_o);
   p.part_ml = a.part_ml;
   p.status = a.status;
   for (int j = 0; j < 64; ++j) p.inv_freq[j] = a.inv_freq[j];

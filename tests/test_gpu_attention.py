@@ -213,3 +213,39 @@ def test_dense_hca_1m_shape(orc):
     ref, rlse = oracle_attention(orc, w, q, [w.L - 1] * w.B, kv_c, tail, sink, tok_base=w.L - w.W)
     mx, rl2 = assert_attention_close(out_values(out), ref, "HCA 1M")
     assert np.allclose(f32(lse), rlse, atol=2e-2)
+
+
+@pytest.mark.parametrize("dense", [False, True])
+def test_garbage_workspace_and_unwritten_cache_rows(orc, dense):
+    """Workspace bytes and cache rows the method never reads may hold any
+    bits (here NaN): empty splits, masked rows of a partial tile and unused
+    selection slots must not leak into the output."""
+    w = configs.scaled(configs.CSA_128K, B=2, k=100)
+    B, N_cap, L_cap = 2, 300, 1200
+    kv_c, kv_tok = random_cache(w, B, N_cap, L_cap, 77)
+    q = synth.normal_bf16((B, w.H, w.D), 78, "q", DEV)
+    sink = synth.normal_f32((w.H,), 79, "sink", 1.0, DEV)
+    pos = [5, 190]  # 1 and 47 visible entries: mostly masked tiles
+    n_vis = [(x + 1) // w.m for x in pos]
+    for b in range(B):
+        kv_c[b, n_vis[b]:] = float("nan")
+    p = binding.params_for(w, B=B)
+    op = binding.OP_DENSE_MQA if dense else binding.OP_SPARSE_MQA
+    ws = binding.workspace(p, op, 1, N_cap)
+    ws.fill_(0xFF)
+    out = torch.empty(B, w.H, w.D, dtype=torch.bfloat16, device=DEV)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    pos_t = torch.tensor(pos, dtype=torch.int64, device=DEV)
+    if dense:
+        binding.dense_mqa_decode(p, q, pos_t, kv_c, kv_tok, sink, out, ws=ws, dev_status=status)
+        sel = cnt = None
+    else:
+        sel, cnt = random_selection(B, w.k, n_vis, 80)
+        binding.sparse_mqa_decode(p, q, pos_t, kv_c, sel, cnt, kv_tok, sink, out, ws=ws,
+                                  dev_status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    got = out_values(out)
+    assert np.isfinite(got).all()
+    ref, _ = oracle_attention(orc, w, q, pos, kv_c, kv_tok, sink, sel, cnt)
+    assert_attention_close(got, ref, "garbage workspace")
