@@ -84,34 +84,67 @@ CSA_DEV void load_row(const __nv_bfloat16* row, int lane, float (&x)[DIM / 32]) 
   }
 }
 
-// Online-softmax pooling of tokens [j0, j1) of one block by one warp.
+// A row's elements of this lane, still packed as bf16 pairs.
 template <int DIM>
-CSA_DEV void pool_tokens(const __nv_bfloat16* blk, int j0, int j1, int lane,
+CSA_DEV void load_row_packed(const __nv_bfloat16* row, int lane, uint32_t (&w)[DIM / 64]) {
+  using LN = Lane<DIM>;
+#pragma unroll
+  for (int p = 0; p < LN::NPART; ++p) {
+    const __nv_bfloat16* src = row + LN::elem(lane, p, 0);
+    if constexpr (LN::VEC == 8) {
+      const uint4 u = __ldg(reinterpret_cast<const uint4*>(src));
+      w[p * 4] = u.x;
+      w[p * 4 + 1] = u.y;
+      w[p * 4 + 2] = u.z;
+      w[p * 4 + 3] = u.w;
+    } else if constexpr (LN::VEC == 4) {
+      const uint2 u = __ldg(reinterpret_cast<const uint2*>(src));
+      w[p * 2] = u.x;
+      w[p * 2 + 1] = u.y;
+    } else {
+      w[p] = __ldg(reinterpret_cast<const uint32_t*>(src));
+    }
+  }
+}
+
+// Online-softmax pooling of tokens [j0, j_use) of one block by one warp.
+// Rows are fetched up to 8 at a time (packed, so 8 rows of d = 512 take 64
+// registers); rows [j_use, j_load) may be fetched too (they are in bounds)
+// so that the loads need not wait for the context length.
+template <int DIM>
+CSA_DEV void pool_tokens(const __nv_bfloat16* blk, int j0, int j_load, int j_use, int lane,
                          const float (&ws)[DIM / 32], const float* b_pos, float& mx, float& l,
                          float (&acc)[DIM / 32]) {
   constexpr int E = DIM / 32;
+  constexpr int RB = 8;
   mx = -INFINITY;
   l = 0.f;
 #pragma unroll
   for (int e = 0; e < E; ++e) acc[e] = 0.f;
-  for (int j = j0; j < j1; j += 4) {
-    float x[4][E];
+  for (int j = j0; j < j_load; j += RB) {
+    uint32_t w[RB][E / 2];
 #pragma unroll
-    for (int u = 0; u < 4; ++u)
-      if (j + u < j1) load_row<DIM>(blk + (int64_t)(j + u) * DIM, lane, x[u]);
+    for (int u = 0; u < RB; ++u)
+      if (j + u < j_load) load_row_packed<DIM>(blk + (int64_t)(j + u) * DIM, lane, w[u]);
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      if (j + u >= j1) break;
-      float dot = 0.f;
+    for (int u = 0; u < RB; ++u) {
+      if (j + u >= j_use) break;
+      float x[E];
 #pragma unroll
-      for (int e = 0; e < E; ++e) dot = fmaf(x[u][e], ws[e], dot);
-      float s = warp_sum(dot) + __ldg(b_pos + j + u);
+      for (int e = 0; e < E / 2; ++e) {
+        x[2 * e] = bf16_lo(w[u][e]);
+        x[2 * e + 1] = bf16_hi(w[u][e]);
+      }
+      float d4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int e = 0; e < E; ++e) d4[e & 3] = fmaf(x[e], ws[e], d4[e & 3]);
+      float s = warp_sum((d4[0] + d4[1]) + (d4[2] + d4[3])) + __ldg(b_pos + j + u);
       float mn = fmaxf(mx, s);
       float corr = __expf(mx - mn);
       float p = __expf(s - mn);
       l = l * corr + p;
 #pragma unroll
-      for (int e = 0; e < E; ++e) acc[e] = fmaf(acc[e], corr, p * x[u][e]);
+      for (int e = 0; e < E; ++e) acc[e] = fmaf(acc[e], corr, p * x[e]);
       mx = mn;
     }
   }
@@ -218,8 +251,13 @@ CSA_DEV void pool_stream(const PoolArgs& a, const StreamArgs& sa, float* smem) {
   float mx, l, acc[E];
   const int g = warp % G;
   const int per_warp = (a.m + G - 1) / G;
-  int j0 = g * per_warp, j1 = min(present, j0 + per_warp);
-  pool_tokens<DIM>(blk, j0, j1 > j0 ? j1 : j0, lane, ws, sa.b_pos, mx, l, acc);
+  // Rows in the buffer (fetched at once) and rows present (pooled).
+  const int64_t in_buf = active ? a.L_cap - i * a.m : 0;
+  const int avail = in_buf <= 0 ? 0 : (in_buf < a.m ? (int)in_buf : a.m);
+  const int j0 = g * per_warp;
+  const int j_load = max(j0, min(avail, j0 + per_warp));
+  const int j_use = max(j0, min(present, j0 + per_warp));
+  pool_tokens<DIM>(blk, j0, j_load, j_use, lane, ws, sa.b_pos, mx, l, acc);
 
   if (G == 1) {
     if (!active || present == 0) return;

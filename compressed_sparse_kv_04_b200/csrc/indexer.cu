@@ -220,13 +220,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       nv[g] = v;
     }
+    // Key scales are loaded a tile ahead so that their latency hides behind
+    // the previous tile's work.
+    auto load_ks = [&](int t) -> float {
+      const int64_t e = (int64_t)t * kTileRows + row;
+      return e < p.N_cap ? __ldg(p.key_scale + (int64_t)b * p.N_cap + e) : 0.f;
+    };
+    float ks_next = load_ks(t_begin);
     int it = 0;
     for (int t = t_begin; t < t_end; ++t, ++it) {
       const int a = it & 1;
       const uint32_t aph = (it >> 1) & 1;
       const int64_t entry = (int64_t)t * kTileRows + row;
-      // Issued before the wait so that its latency overlaps the MMA.
-      const float ks = entry < p.N_cap ? __ldg(p.key_scale + (int64_t)b * p.N_cap + entry) : 0.f;
+      const float ks = ks_next;
+      if (t + 1 < t_end) ks_next = load_ks(t + 1);
       bool ok = mbar_wait(&tfull[a], aph, p.status, abort_flag);
       if (!__all_sync(0xffffffffu, ok)) break;  // keep the warp converged for tcgen05.ld
       tc_fence_after();

@@ -147,8 +147,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* empty = ready + C::kStages;
   uint64_t* sfull = empty + C::kStages;
   uint64_t* pfull = sfull + 2;
-  uint64_t* pvdone = pfull + 2;
-  uint64_t* qready = pvdone + 1;
+  uint64_t* pvdone = pfull + 2;  // [2]: P.V of tiles with parity 0 / 1
+  uint64_t* qready = pvdone + 2;
   uint64_t* drain = qready + 1;
   uint64_t* done = drain + 1;  // one arrival per warp when its role is over
   uint64_t* qfull = done + 1;  // the query block landed in the last stage
@@ -199,7 +199,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&sfull[a], 1);
       mbar_init(&pfull[a], 128);
     }
-    mbar_init(pvdone, 1);
+    mbar_init(&pvdone[0], 1);
+    mbar_init(&pvdone[1], 1);
     mbar_init(qready, 128);
     mbar_init(drain, 1);
     mbar_init(done, kThreads / 32);
@@ -343,7 +344,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         desc_mn(vbase + (n * kPvN / 64) * C::kChunkBytes + kk * 16 * 128),
                         idesc_pv, (jt > 0 || kk > 0) ? 1u : 0u);
         mma_commit(&empty[s]);
-        mma_commit(pvdone);
+        mma_commit(&pvdone[jt & 1]);
       }
       __syncwarp();
       return true;
@@ -639,15 +640,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool grow = mt > m_run + kRescaleThreshold * 1.4426950408889634f || m_run == -INFINITY;
       const float m_new = grow ? fmaxf(mt, m_run) : m_run;
       const bool need = grow && m_run != -INFINITY;
-      // P.V of the previous tile must be complete before O may be rescaled
-      // and before P buffer a (read by P.V two tiles back) is rewritten.
-      // This wait happens on every tile, before pfull(it) is released, so
-      // the pvdone phase can never run two phases ahead of this check.
-      if (it > 0) {
-        if (!wait_all(pvdone, (it - 1) & 1, p, abort_flag)) break;
+      // P buffer a was last read by P.V of tile it-2; rescaling O needs
+      // every earlier P.V complete (the latest is tile it-1).  pvdone[x]
+      // completes once per tile of parity x, and tile it's P.V cannot be
+      // issued before pfull(it) below, so neither wait can see its barrier
+      // two phases ahead.  Without a rescale, P.V(it-1) overlaps this tile.
+      const bool rescale = __any_sync(0xffffffffu, need) && it > 0;
+      if (rescale) {
+        if (!wait_all(&pvdone[(it - 1) & 1], ((it - 1) >> 1) & 1, p, abort_flag)) break;
         tc_fence_after();
+      } else if (it >= 2) {
+        if (!wait_all(&pvdone[it & 1], ((it - 2) >> 1) & 1, p, abort_flag)) break;
       }
-      if (__any_sync(0xffffffffu, need) && it > 0) {
+      if (rescale) {
         const float f = need ? fast_exp2(m_run - m_new) : 1.f;
 #pragma unroll 1
         for (int c = 0; c < D / 2; c += 32) {
@@ -701,7 +706,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         pml[hg] = -INFINITY;
         pml[p.H + hg] = 0.f;
       }
-    } else if (!*abort_flag && wait_all(pvdone, (ntile - 1) & 1, p, abort_flag)) {
+    } else if (!*abort_flag &&
+               wait_all(&pvdone[(ntile - 1) & 1], ((ntile - 1) >> 1) & 1, p, abort_flag)) {
       tc_fence_after();
       // O / l rows (fp16: |O / l| is at most the largest |v|) go through
       // shared memory (the stages are free now: every MMA has completed)
