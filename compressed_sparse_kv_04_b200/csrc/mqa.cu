@@ -820,15 +820,24 @@ __global__ void __launch_bounds__(128) mqa_combine_kernel(const Params p, int D,
       acc.z = fmaf(c.x, w, acc.z);
       acc.w = fmaf(c.y, w, acc.w);
     };
-    int s = 0;
-    for (; s + 4 <= S; s += 4) {
-      uint2 v[4];
+    // Groups of 4 splits, the next group's loads issued before this
+    // group's use (two groups in flight).
+    auto load4 = [&](int s0, uint2 (&v)[4]) {
 #pragma unroll
-      for (int u = 0; u < 4; ++u) v[u] = __ldg(reinterpret_cast<const uint2*>(src + (s + u) * stride));
+      for (int u = 0; u < 4; ++u)
+        v[u] = s0 + u < S ? __ldg(reinterpret_cast<const uint2*>(src + (s0 + u) * stride))
+                          : make_uint2(0u, 0u);
+    };
+    uint2 cur[4], nxt[4];
+    load4(0, cur);
+    for (int s0 = 0; s0 < S; s0 += 4) {
+      if (s0 + 4 < S) load4(s0 + 4, nxt);
 #pragma unroll
-      for (int u = 0; u < 4; ++u) add(v[u], wsplit[s + u]);
+      for (int u = 0; u < 4; ++u)
+        if (s0 + u < S) add(cur[u], wsplit[s0 + u]);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) cur[u] = nxt[u];
     }
-    for (; s < S; ++s) add(__ldg(reinterpret_cast<const uint2*>(src + s * stride)), wsplit[s]);
     so[4 * d4] = acc.x * invL;
     so[4 * d4 + 1] = acc.y * invL;
     so[4 * d4 + 2] = acc.z * invL;
