@@ -126,6 +126,9 @@ CSA_DEV void bulk_store(void* gdst, const void* ssrc, uint32_t bytes) {
 }
 CSA_DEV void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 CSA_DEV void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+// Waits only until the source shared memory has been read (the writes are
+// visible to later kernels once this one completes).
+CSA_DEV void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 
 // 16-byte global -> shared copy through L2 (LSU path), and an mbarrier
 // arrival that fires once this thread's earlier copies have landed (counts

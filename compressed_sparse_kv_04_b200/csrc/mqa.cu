@@ -718,12 +718,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       __half* ob = reinterpret_cast<__half*>(stages + hl * kORow) + hf * (D / 2);
       const float inv_l = l_run > 0.f ? 1.0f / l_run : 0.f;
 #pragma unroll 1
-      for (int c = 0; c < D / 2; c += 32) {
-        uint32_t v[32];
-        tmem_ld_16x32bx2_x32<D / 2>(t_o + lq + c, v);
+      for (int c = 0; c < D / 2; c += 64) {  // two 32-column loads per wait
+        uint32_t v[64];
+        tmem_ld_16x32bx2_x32<D / 2>(t_o + lq + c, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+        tmem_ld_16x32bx2_x32<D / 2>(t_o + lq + c + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
         tmem_wait_ld();
 #pragma unroll
-        for (int j = 0; j < 32; j += 8) {
+        for (int j = 0; j < 64; j += 8) {
           uint4 u;
           u.x = h2_bits(__floats2half2_rn(__uint_as_float(v[j]) * inv_l, __uint_as_float(v[j + 1]) * inv_l));
           u.y = h2_bits(__floats2half2_rn(__uint_as_float(v[j + 2]) * inv_l, __uint_as_float(v[j + 3]) * inv_l));
@@ -736,7 +737,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         fence_proxy_async_smem();
         bulk_store(po, ob, (D / 2) * 2);
         bulk_commit();
-        bulk_wait_all();
+        bulk_wait_read();  // shared memory may be released; the kernel end publishes the data
       }
       if (head_ok && hf == 0) {
         pml[hg] = m_run;  // log2 domain
@@ -777,6 +778,20 @@ __global__ void __launch_bounds__(128) mqa_combine_kernel(const Params p, int D,
   const float z = sink[h];
   const float z2 = z * LOG2E;  // log2 domain
   __nv_bfloat16* o = out + ((int64_t)row * p.H + h) * D;
+  // Thread t merges dims [4t, 4t+4) (D <= 512).  Its first group of
+  // partials is requested before the weights are known.
+  const int d4 = threadIdx.x;
+  const bool dims = d4 < D / 4;
+  const __half* src = p.part_o + ((int64_t)row * S * p.H + h) * D + 4 * d4;
+  const int64_t stride = (int64_t)p.H * D;
+  auto load4 = [&](int s0, uint2 (&v)[4]) {
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      v[u] = (dims && s0 + u < S) ? __ldg(reinterpret_cast<const uint2*>(src + (s0 + u) * stride))
+                                  : make_uint2(0u, 0u);
+  };
+  uint2 cur[4], nxt[4];
+  load4(0, cur);
   if (threadIdx.x < 32) {
     const int lane = threadIdx.x;
     float M = z2;
@@ -807,9 +822,7 @@ __global__ void __launch_bounds__(128) mqa_combine_kernel(const Params p, int D,
     return;
   }
   const float invL = 1.0f / L;
-  for (int d4 = threadIdx.x; d4 < D / 4; d4 += blockDim.x) {
-    const __half* src = p.part_o + ((int64_t)row * S * p.H + h) * D + 4 * d4;
-    const int64_t stride = (int64_t)p.H * D;
+  if (dims) {
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     auto add = [&](uint2 u, float w) {
       if (w == 0.f) return;  // empty split: its partial was never written
@@ -820,16 +833,8 @@ __global__ void __launch_bounds__(128) mqa_combine_kernel(const Params p, int D,
       acc.z = fmaf(c.x, w, acc.z);
       acc.w = fmaf(c.y, w, acc.w);
     };
-    // Groups of 4 splits, the next group's loads issued before this
-    // group's use (two groups in flight).
-    auto load4 = [&](int s0, uint2 (&v)[4]) {
-#pragma unroll
-      for (int u = 0; u < 4; ++u)
-        v[u] = s0 + u < S ? __ldg(reinterpret_cast<const uint2*>(src + (s0 + u) * stride))
-                          : make_uint2(0u, 0u);
-    };
-    uint2 cur[4], nxt[4];
-    load4(0, cur);
+    // Groups of 4 splits, the next group's loads in flight during this
+    // group's use.
     for (int s0 = 0; s0 < S; s0 += 4) {
       if (s0 + 4 < S) load4(s0 + 4, nxt);
 #pragma unroll
