@@ -516,28 +516,57 @@ def run_e2e(st, graphs, K, W, barrier, rmax, rsum, world):
         h2d += sum(t.numel() * t.element_size() for t in extra[0][1:])
     d2h = hout.numel() * hout.element_size()
 
-    def one(i):
+    # Copies run on their own streams: the inputs of step i+1 travel while
+    # step i computes, and the output of step i returns while step i+1
+    # computes (each step has its own input set, so nothing is overwritten
+    # while in use).
+    comp = torch.cuda.current_stream()
+    up, down = torch.cuda.Stream(), torch.cuda.Stream()
+    copied = [torch.cuda.Event() for _ in range(R)]
+    done = [torch.cuda.Event() for _ in range(R)]
+    used = [False] * R
+
+    def upload(i):
         r = i % R
         s = st.sets[r]
-        s["q"].copy_(hq[r], non_blocking=True)
-        s["kv_tok"][:, L - m:].copy_(hkv[r], non_blocking=True)
-        if w.csa:
-            _, a, b, c, d = extra[r]
-            s["q_idx"].copy_(a, non_blocking=True)
-            s["q_scale"].copy_(b, non_blocking=True)
-            s["w"].copy_(c, non_blocking=True)
-            s["idx_tok"][:, L - m:].copy_(d, non_blocking=True)
-        graphs[r].replay()
-        hout.copy_(s["out"], non_blocking=True)
+        with torch.cuda.stream(up):
+            if used[r]:
+                up.wait_event(done[r])  # the set's previous step has finished
+            s["q"].copy_(hq[r], non_blocking=True)
+            s["kv_tok"][:, L - m:].copy_(hkv[r], non_blocking=True)
+            if w.csa:
+                _, a, b, c, d = extra[r]
+                s["q_idx"].copy_(a, non_blocking=True)
+                s["q_scale"].copy_(b, non_blocking=True)
+                s["w"].copy_(c, non_blocking=True)
+                s["idx_tok"][:, L - m:].copy_(d, non_blocking=True)
+            copied[r].record(up)
 
-    for i in range(W):
-        one(i)
+    def compute(i):
+        r = i % R
+        comp.wait_event(copied[r])
+        graphs[r].replay()
+        done[r].record(comp)
+        used[r] = True
+        with torch.cuda.stream(down):
+            down.wait_event(done[r])
+            hout.copy_(st.sets[r]["out"], non_blocking=True)
+
+    def run(n):
+        up.wait_stream(comp)
+        upload(0)
+        for i in range(n):
+            if i + 1 < n:
+                upload(i + 1)
+            compute(i)
+        comp.wait_stream(down)
+
+    run(W)
     barrier()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record()
-    for i in range(K):
-        one(i)
+    run(K)
     e1.record()
     barrier()
     val, _ = aggregate(w.B * K, e0.elapsed_time(e1), world, rmax, rsum)
