@@ -732,7 +732,8 @@ class OracleStep:
         n_sub = N if n_sub is None else max(1, min(N, n_sub))
         h_sub = w.H if h_sub is None else max(1, min(w.H, h_sub))
         t0 = time.perf_counter()
-        orc.pool(self.tok, [tail], self.w_s, self.b_pos, None, m, tail // m - 1, 1, tail // m)
+        orc.pool(self.tok, [tail], self.w_s, self.b_pos, None, m, tail // m - 1, 1, tail // m,
+                 rope_dim=w.rope_dim)
         if w.csa:
             orc.pool(self.itok, [tail], self.w_si, self.b_pos, None, m, tail // m - 1, 1,
                      tail // m)

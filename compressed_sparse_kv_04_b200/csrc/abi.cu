@@ -178,6 +178,9 @@ static csa_status compress_common(const char* fn, const csa_params* p, const voi
   if (first_block < 0 || n_blocks < 0 || first_block + n_blocks > N_cap)
     return fail(CSA_ERR_CAPACITY, "%s: blocks [%lld, %lld) outside N_cap=%lld", fn,
                 (long long)first_block, (long long)(first_block + n_blocks), (long long)N_cap);
+  if ((p->rope_dim != 0 && p->rope_dim != 32 && p->rope_dim != 64) || p->rope_dim > p->d / 4)
+    return fail(CSA_ERR_UNSUPPORTED_SHAPE,
+                "%s: rope_dim=%d (supported: 0, 32, 64, and at most d/4)", fn, p->rope_dim);
   if (idx_tok) {
     st = check_indexer(fn, p);
     if (st != CSA_OK) return st;
@@ -209,6 +212,8 @@ static csa_status compress_common(const char* fn, const csa_params* p, const voi
   c.idx_key = idx_key;
   c.idx_scale = idx_scale;
   c.eps = p->eps;
+  c.rope_dim = p->rope_dim;
+  fill_inv_freq(p, c.inv_freq);
   c.status = dev_status;
   cudaError_t e = csa::launch_compress(c, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(fn, e);

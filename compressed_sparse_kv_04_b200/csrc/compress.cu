@@ -8,11 +8,16 @@
 // attention" CSA / HCA bullets.  Weight form (the build's reading):
 // softmax_j(c_t . w_s + b_pos[j]) over the present tokens of the block.
 //
+// Storage (the build's reading): a KV entry is stored already rotated (RoPE
+// on the last rope_dim dims, "DeepSeek V4-Pro" (llm-arch-kb), "Hybrid
+// attention") to its own position (i+1)*m - 1, so attention uses it as
+// stored; indexer keys are not rotated.
+//
 // Design: pure HBM streaming on CUDA cores.  A warp owns up to 16 tokens of
 // a block and keeps an online-softmax accumulator of the block row in
 // registers (16 fp32 per lane at d = 512); token rows are read with 16-byte
-// coalesced loads, four rows in flight per warp.  m <= 16: one warp per
-// block, 8 blocks per 256-thread CTA.  m > 16: 8 warps per block, merged
+// coalesced loads, up to eight rows in flight per warp.  m <= 16: one warp
+// per block, 8 blocks per 256-thread CTA.  m > 16: 8 warps per block, merged
 // through shared memory.  Both streams of csa_compress run in one launch
 // (blockIdx.y selects the stream).
 #include "common.cuh"
@@ -33,6 +38,7 @@ struct StreamArgs {
   uint8_t* out_e4m3;         // [B, N_cap, dim] or null
   float* out_scale;          // [B, N_cap] (with out_e4m3)
   int dim;
+  int rope_dim;              // > 0: the entry is stored rotated to (i+1)*m - 1
 };
 
 struct PoolArgs {
@@ -44,6 +50,7 @@ struct PoolArgs {
   int64_t ctx_len_value;
   int64_t first_block, n_blocks;
   float eps;
+  double inv_freq[64];  // rotation frequencies (rope_dim/2 entries)
   int32_t* status;
 };
 
@@ -151,8 +158,8 @@ CSA_DEV void pool_tokens(const __nv_bfloat16* blk, int j0, int j_load, int j_use
 }
 
 template <int DIM>
-CSA_DEV void finish_row(const StreamArgs& sa, int64_t row, int lane, float (&p)[DIM / 32],
-                        float eps) {
+CSA_DEV void finish_row(const StreamArgs& sa, const PoolArgs& a, int64_t row, int64_t pos,
+                        int lane, float (&p)[DIM / 32], float eps) {
   using LN = Lane<DIM>;
   constexpr int E = DIM / 32;
   float ss = 0.f;
@@ -168,6 +175,29 @@ CSA_DEV void finish_row(const StreamArgs& sa, int64_t row, int lane, float (&p)[
       float g = sa.gamma ? __ldg(sa.gamma + LN::elem(lane, part, v)) : 1.f;
       p[e] = p[e] * inv * g;
     }
+  if (sa.rope_dim > 0) {
+    // Rotate-half over the last R dims, to the entry's position.  Those dims
+    // sit in the last part of lanes 32 - R/VEC .. 31; the partner of dim d
+    // (d +- R/2) is held by lane ^ (R/2 / VEC).
+    const int R = sa.rope_dim, half = R / 2;
+    constexpr int lp = LN::NPART - 1;
+    float other[LN::VEC];
+#pragma unroll
+    for (int v = 0; v < LN::VEC; ++v)
+      other[v] = __shfl_xor_sync(0xffffffffu, p[lp * LN::VEC + v], half / LN::VEC);
+    const int d0 = LN::elem(lane, lp, 0);
+    if (d0 >= DIM - R) {
+      const bool first = d0 < DIM - half;
+#pragma unroll
+      for (int v = 0; v < LN::VEC; ++v) {
+        const int j = (d0 + v - (DIM - R)) % half;
+        float sn, cs;
+        sincos_reduced((double)pos * a.inv_freq[j], &sn, &cs);
+        const float x = p[lp * LN::VEC + v], y = other[v];
+        p[lp * LN::VEC + v] = first ? x * cs - y * sn : x * cs + y * sn;
+      }
+    }
+  }
   pdl_wait();  // stores come after every earlier kernel of the stream
   if (sa.out_bf16) {
     __nv_bfloat16* dst = sa.out_bf16 + row * DIM;
@@ -263,7 +293,7 @@ CSA_DEV void pool_stream(const PoolArgs& a, const StreamArgs& sa, float* smem) {
     if (!active || present == 0) return;
 #pragma unroll
     for (int e = 0; e < E; ++e) acc[e] = acc[e] / l;
-    finish_row<DIM>(sa, b * a.N_cap + i, lane, acc, a.eps);
+    finish_row<DIM>(sa, a, b * a.N_cap + i, (i + 1) * a.m - 1, lane, acc, a.eps);
     return;
   }
   // Merge the G warp partials of the one block of this CTA.
@@ -299,7 +329,7 @@ CSA_DEV void pool_stream(const PoolArgs& a, const StreamArgs& sa, float* smem) {
   }
 #pragma unroll
   for (int e = 0; e < E; ++e) p[e] = p[e] / L;
-  finish_row<DIM>(sa, b * a.N_cap + i, lane, p, a.eps);
+  finish_row<DIM>(sa, a, b * a.N_cap + i, (i + 1) * a.m - 1, lane, p, a.eps);
 }
 
 __global__ void __launch_bounds__(kThreads) compress_kernel(const PoolArgs a) {
@@ -323,10 +353,11 @@ cudaError_t launch_compress(const CompressLaunch& c, cudaStream_t stream) {
   PoolArgs a{};
   a.nstreams = c.idx_tok ? 2 : 1;
   a.s[0] = StreamArgs{reinterpret_cast<const __nv_bfloat16*>(c.kv_tok), c.w_s, c.b_pos, c.gamma,
-                      reinterpret_cast<__nv_bfloat16*>(c.kv_c), nullptr, nullptr, c.d};
+                      reinterpret_cast<__nv_bfloat16*>(c.kv_c), nullptr, nullptr, c.d, c.rope_dim};
   if (c.idx_tok)
     a.s[1] = StreamArgs{reinterpret_cast<const __nv_bfloat16*>(c.idx_tok), c.w_s_idx, c.b_pos_idx,
-                        nullptr, nullptr, c.idx_key, c.idx_scale, c.D_I};
+                        nullptr, nullptr, c.idx_key, c.idx_scale, c.D_I, 0};
+  for (int j = 0; j < 64; ++j) a.inv_freq[j] = c.inv_freq[j];
   a.B = c.B;
   a.m = c.m;
   a.L_cap = c.L_cap;

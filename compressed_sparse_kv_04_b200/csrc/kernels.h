@@ -23,6 +23,8 @@ struct CompressLaunch {
   uint8_t* idx_key;
   float* idx_scale;
   float eps;
+  int rope_dim;             // KV entries are stored rotated to (i+1)*m - 1
+  double inv_freq[64];      // rope_dim/2 entries
   int32_t* status;
 };
 cudaError_t launch_compress(const CompressLaunch& c, cudaStream_t stream);

@@ -24,8 +24,9 @@
 //     transform warps with 16-byte cp.async (two threads per row, a few
 //     tiles ahead), which keeps many more rows in flight than per-row TMA
 //     gathers; 128-byte swizzle either way, K = V = that tile;
-//   - transform warps RoPE the rotated dims in place and, for window tokens,
-//     compute 1/rms(c_t) and apply the KV gain;
+//   - transform warps zero masked rows and, for window tokens, compute
+//     1/rms(c_t), apply the KV gain and rotate the last R dims to the token
+//     position (compressed entries are stored already rotated to theirs);
 //   - the MMA warp issues S = Qhat K^T (TS form) into one of two S buffers,
 //     then P V into O (P from shared memory, V = the same tile read
 //     MN-major, in N <= 256 pieces);
@@ -471,7 +472,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (hf == 0) M.rn[r] = (valid && M.window) ? 1.0f / sqrtf(ss / (float)D + p.eps) : 1.0f;
       __syncwarp();  // gain-scaled values are in place before the rotation reads them
       if constexpr (R > 0) {
-        if (valid) {
+        if (valid && M.window) {  // compressed entries are stored rotated
           // Pairs (j, j+R/2) of the last R dims; thread half hf rotates pairs
           // [hf*R/4, hf*R/4 + R/4) with 16-byte accesses (8 bf16 each).
           constexpr int half = R / 2;

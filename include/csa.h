@@ -107,9 +107,12 @@ size_t csa_workspace_bytes(const csa_params* p, csa_op op, int Q, int64_t N_cap)
  *   s_j   = kv_tok[b,t,:] . w_s + b_pos[j]
  *   alpha = softmax over the present j of s_j
  *   e     = RMSNorm(sum_j alpha_j kv_tok[b,t,:]) * gamma      (eps = p->eps)
- * and e is stored as bf16 in kv_c[b,i,:].  A block with no present token is
- * left untouched.  (The weight form is the build's reading: the pages do
- * not fix it.)
+ * and RoPE_{(i+1)m-1}(e) -- e rotated on its last p->rope_dim dims to the
+ * position of the block's last token ([P5]: RoPE on the last 64 dims of the
+ * KV) -- is stored as bf16 in kv_c[b,i,:], so that attention uses entries
+ * as stored.  A block with no present token is left untouched.  (The weight
+ * form and the place of the rotation are the build's readings: the pages
+ * fix neither.)  rope_dim must be 0, 32 or 64 and at most d/4.
  *
  *   kv_tok  [B, L_cap, d] bf16 (device)     token KV stream
  *   ctx_len [B] int64 (device)              tokens present per sequence
@@ -230,15 +233,15 @@ csa_status lightning_index_topk_static(const csa_params* p, int Q, const uint8_t
  * RoPE on the output).  One query per sequence at position pos = pos_q[b].
  *
  *   qhat_h = RoPE_pos(RMSNorm(q[b,h,:]) * gamma_q)
- *   KV set = { RoPE_{(i+1)m-1}(kv_c[b,i,:]) : i in topk_idx[b, 0..topk_cnt) }
+ *   KV set = { kv_c[b,i,:] (stored rotated, see hca_compress) : i in topk_idx[b, 0..topk_cnt) }
  *          U { RoPE_t(RMSNorm(kv_tok[b,t,:]) * gamma_kv) : max(0,pos-W+1) <= t <= pos }
  *   s_hj = softmax_scale * qhat_h . v_j;  M_h = max(max_j s_hj, sink[h])
  *   out[b,h,:] = RoPE_{-pos}( sum_j e^{s_hj-M_h} v_j / (sum_j e^{s_hj-M_h} + e^{sink[h]-M_h}) )
  * stored as bf16; lse[b,h] = M_h + log(denominator) when lse is not NULL.
  * Readings (pages silent): one joint softmax over window and entries, no
  * de-duplication; compressed entries are used as stored (their pooling
- * RMSNorm is the KV norm); entry i sits at position (i+1)*m-1; rotate-half
- * pairing over the last rope_dim dims.  sink = -inf drops the sink; +inf
+ * RMSNorm is the KV norm, and they are stored rotated to their position
+ * (i+1)*m-1); rotate-half pairing over the last rope_dim dims.  sink = -inf drops the sink; +inf
  * gives a zero output.
  *
  *   q [B, H, d] bf16; pos_q [B] int64; kv_c [B, N_cap, d] bf16;

@@ -192,10 +192,16 @@ void orc_bf16_encode_array(int64_t n, const double* x, uint16_t* out) {
 // of the QK-Norm that [P5] places on the one shared compressed KV head).  Blocks do not
 // overlap for either ratio.  A block with no present token is not written.
 // `normalize` = 0 skips the RMSNorm (a test hook only).
+//
+// Storage reading for the KV stream ([P5] puts RoPE on the last dimensions
+// of the KV; where it is applied is not fixed): the entry is stored already
+// rotated to its own position (i+1)*m - 1, the last token of the block, so
+// that attention uses it as stored.  rope_dim = 0 stores it unrotated (the
+// indexer stream, which the pages do not rotate).
 void orc_pool(int B, int64_t L_cap, int d, int m, const uint16_t* tok, const int64_t* ctx_len,
               const float* w_s, const float* b_pos, const float* gamma, double eps, int normalize,
-              int64_t first_block, int64_t n_blocks, int64_t N_cap, double* out, uint8_t* written,
-              int nthreads) {
+              int rope_dim, double rope_base, int64_t first_block, int64_t n_blocks,
+              int64_t N_cap, double* out, uint8_t* written, int nthreads) {
   parallel_for((int64_t)B * n_blocks, nthreads, [&](int64_t w) {
     int64_t b = w / n_blocks, i = first_block + w % n_blocks;
     if (i < 0 || i >= N_cap) return;
@@ -221,6 +227,7 @@ void orc_pool(int B, int64_t L_cap, int d, int m, const uint16_t* tok, const int
       for (int k = 0; k < d; ++k) p[k] += a * bf16_decode(row[k]);
     }
     if (normalize) rms_norm(p.data(), d, gamma, eps);
+    rope_apply(p.data(), d, rope_dim, rope_base, (double)((i + 1) * m - 1), +1.0);
     double* o = out + ((int64_t)b * N_cap + i) * d;
     for (int k = 0; k < d; ++k) o[k] = p[k];
     if (written) written[(int64_t)b * N_cap + i] = 1;
@@ -327,9 +334,10 @@ void orc_topk(int64_t BQ, int64_t N_cap, const double* scores, const int64_t* n_
 //
 // Readings: window and compressed entries share one softmax and are not
 // de-duplicated; the window holds tokens max(0, pos-W+1) .. pos (the query
-// token itself included); compressed entries are used as stored (their
-// pooling RMSNorm is the KV norm), window tokens get RMSNorm with gamma_kv;
-// entry i sits at position (i+1)*m - 1; the logit scale is `scale`
+// token itself included); compressed entries are used as stored: their
+// pooling RMSNorm is the KV norm and they are stored already rotated to
+// their position (i+1)*m - 1 (see orc_pool); window tokens get RMSNorm with
+// gamma_kv and the rotation to their position t; the logit scale is `scale`
 // (1/sqrt(D) in the library); K = V = the roped vector; the output is
 // RoPE(-pos) of the normalised weighted sum.  A sink of -inf drops out; a
 // sink of +inf gives a zero output.
@@ -368,8 +376,7 @@ void orc_mqa(int B, int Q, int H, int D, int m, int W, int rope_dim, double rope
       if (j < (int64_t)ent.size()) {
         int64_t i = ent[j];
         const uint16_t* row = kv_c + (b * N_cap + i) * D;
-        for (int d = 0; d < D; ++d) v[d] = bf16_decode(row[d]);
-        rope_apply(v, D, rope_dim, rope_base, (double)((i + 1) * m - 1), +1.0);
+        for (int d = 0; d < D; ++d) v[d] = bf16_decode(row[d]);  // stored rotated
       } else {
         int64_t t = w0 + (j - (int64_t)ent.size());
         const uint16_t* row = kv_tok + (b * L_cap + (t - tok_base)) * D;

@@ -70,7 +70,8 @@ def test_csa_compress_tiny(orc, L_ctx):
     r = run_compress(w, L_ctx)
     n = math.ceil(L_ctx / w.m)
     ref_bits, written, vals = orc.compress_kv(bits16(r["kv_tok"]), [L_ctx], f32(r["w_s"]), f32(r["b_pos"]),
-                                              None, w.m, 0, r["N_cap"], r["N_cap"])
+                                              None, w.m, 0, r["N_cap"], r["N_cap"],
+                                              rope_dim=w.rope_dim)
     assert written[0, :n].all() and not written[0, n:].any()
     assert_bf16_storage_close(bits16(r["kv_c"])[:, :n], vals[:, :n], "kv_c")
     assert not bits16(r["kv_c"])[:, n:].any()  # blocks past the context untouched
@@ -87,7 +88,8 @@ def test_hca_compress_ragged_with_gain(orc):
     gamma = synth.gains(w.d, w.seed, DEV)
     r = run_compress(w, lens, gamma=gamma)
     _, written, vals = orc.compress_kv(bits16(r["kv_tok"]), lens, f32(r["w_s"]), f32(r["b_pos"]),
-                                       f32(gamma), w.m, 0, r["N_cap"], r["N_cap"])
+                                       f32(gamma), w.m, 0, r["N_cap"], r["N_cap"],
+                                       rope_dim=w.rope_dim)
     got = bits16(r["kv_c"])
     for b, L in enumerate(lens):
         n = math.ceil(L / w.m)
@@ -102,7 +104,7 @@ def test_compress_newest_block_only(orc):
     got = bits16(r["kv_c"])
     assert not got[:, :1023].any()
     _, _, vals = orc.compress_kv(bits16(r["kv_tok"]), [4096, 4096], f32(r["w_s"]), f32(r["b_pos"]),
-                                 None, w.m, 1023, 1, r["N_cap"])
+                                 None, w.m, 1023, 1, r["N_cap"], rope_dim=w.rope_dim)
     assert_bf16_storage_close(got[:, 1023:], vals[:, 1023:], "newest block")
 
 

@@ -46,7 +46,8 @@ def run_prefill(orc, w, P, T):
     qi = synth.queries(w, Q=T)
     kv_bits, idx_bits = bits16(kv_tok), bits16(idx_tok)
     # Cached blocks 0 .. b0-1 from the oracle.
-    kv_c0, _, _ = orc.compress_kv(kv_bits, [P], f32(w_s), f32(b_pos), None, m, 0, b0, N_cap)
+    kv_c0, _, _ = orc.compress_kv(kv_bits, [P], f32(w_s), f32(b_pos), None, m, 0, b0, N_cap,
+                                  rope_dim=w.rope_dim)
     key0, ks0, _, _ = orc.compress_index(idx_bits, [P], f32(w_si), f32(b_pi), m, 0, b0, N_cap)
     kv_c = torch.from_numpy(kv_c0.view(np.int16)).view(torch.bfloat16).to(DEV)
     idx_key = torch.from_numpy(key0).to(DEV)
@@ -79,7 +80,7 @@ def check_prefill(orc, w, r, rows):
     assert np.array_equal(r["kv_c"][:, :b0], r["kv_c0"][:, :b0])
     assert np.array_equal(r["idx_key"][:, :b0], r["key0"][:, :b0])
     _, _, vals = orc.compress_kv(r["kv_bits"], [P + T], f32(r["w_s"]), f32(r["b_pos"]), None, m,
-                                 b0, N_cap - b0, N_cap)
+                                 b0, N_cap - b0, N_cap, rope_dim=w.rope_dim)
     assert_bf16_storage_close(r["kv_c"][:, b0:], vals[:, b0:], "new KV entries")
     _, ks_ref, kvals, _ = orc.compress_index(r["idx_bits"], [P + T], f32(r["w_si"]),
                                              f32(r["b_pi"]), m, b0, N_cap - b0, N_cap)

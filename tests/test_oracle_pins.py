@@ -353,34 +353,75 @@ def test_sink_limits_and_closed_form(orc):
     assert np.allclose(lse[0, 0], np.logaddexp(s, z.astype(np.float64)), rtol=1e-13)
 
 
-def test_rope_relative_rotation_closed_form(orc):
-    # One compressed entry, no window, sink -inf: the output is the entry
-    # rotated by (entry position - query position) on the last r dims.
+def _rotate(v, pos, r_dim, base=10000.0):
+    """Rotate-half rotation of the last r_dim dims of v by position pos (the
+    textbook form, written out here to check the oracle against it)."""
+    D = v.shape[-1]
+    half = r_dim // 2
+    th = base ** (-2.0 * np.arange(half) / r_dim)
+    c, s = np.cos(pos * th), np.sin(pos * th)
+    out = v.copy()
+    x1, x2 = v[..., D - r_dim: D - half], v[..., D - half:]
+    out[..., D - r_dim: D - half] = x1 * c - x2 * s
+    out[..., D - half:] = x2 * c + x1 * s
+    return out
+
+
+def test_rope_inverse_on_output_closed_form(orc):
+    # One stored entry (stored already rotated to its position), no window,
+    # sink -inf: the output is that stored vector rotated back by the query
+    # position.
     B, Q, H, D, m, r_dim = 1, 1, 2, 32, 4, 16
     q, kv_tok, kv_c, sink = _mqa_case(B, Q, H, D, 16, m, 26)
     sink[:] = -np.inf
-    pos = np.array([[11]])  # n_vis = 3; entry 0 sits at position 3
-    sel = np.array([[[0, -1]]], np.int32)
+    pos = np.array([[11]])  # n_vis = 3
     cnt = np.array([[1]], np.int32)
-    out, _ = orc.mqa(q, pos, kv_c, kv_tok, sink, m, 0, r_dim, sel, cnt)
-    e = orc.bf16_decode(kv_c)[0, 0]
-    delta = 3 - 11
-    half = r_dim // 2
-    th = 10000.0 ** (-2.0 * np.arange(half) / r_dim)
-    c, s = np.cos(delta * th), np.sin(delta * th)
-    ref = e.copy()
-    x1, x2 = e[D - r_dim: D - half], e[D - half:]
-    ref[D - r_dim: D - half] = x1 * c - x2 * s
-    ref[D - half:] = x2 * c + x1 * s
-    assert np.allclose(out[0, 0], np.broadcast_to(ref, (H, D)), rtol=1e-12, atol=1e-12)
-    # Entry 2 sits at the query position: no rotation at all.
-    out, _ = orc.mqa(q, pos, kv_c, kv_tok, sink, m, 0, r_dim, np.array([[[2, -1]]], np.int32), cnt)
-    assert np.allclose(out[0, 0], np.broadcast_to(orc.bf16_decode(kv_c)[0, 2], (H, D)), rtol=1e-13, atol=1e-13)
+    for ent in (0, 2):
+        out, _ = orc.mqa(q, pos, kv_c, kv_tok, sink, m, 0, r_dim, np.array([[[ent, -1]]], np.int32),
+                         cnt)
+        ref = _rotate(orc.bf16_decode(kv_c)[0, ent], -11.0, r_dim)
+        assert np.allclose(out[0, 0], np.broadcast_to(ref, (H, D)), rtol=1e-12, atol=1e-12)
+    # Window token t (one token window at the query position): rotated to t
+    # and back, so the output is the normalised token itself.
+    x = orc.bf16_decode(kv_tok)[0, 11]
+    v = x / np.sqrt(np.mean(x * x) + 1e-6)
+    out_w, _ = orc.mqa(q, pos, kv_c, kv_tok, sink, m, 1, r_dim, np.array([[[-1, -1]]], np.int32),
+                       np.array([[0]], np.int32))
+    assert np.allclose(out_w[0, 0], np.broadcast_to(v, (H, D)), rtol=1e-12, atol=1e-12)
+
+
+def test_compression_stores_entry_rotated_to_its_position(orc):
+    # m = 1 with uniform weights: the entry is RMSNorm(c_t) rotated to t.
+    B, L, d, r_dim = 1, 6, 32, 16
+    r = rng(31)
+    tok = bf16_bits(r.standard_normal((B, L, d)))
+    vals, _ = orc.pool(tok, np.array([L]), np.zeros(d), np.zeros(1), None, 1, 0, L, L,
+                       rope_dim=r_dim)
+    x = orc.bf16_decode(tok)[0]
+    nrm = x / np.sqrt(np.mean(x * x, axis=1, keepdims=True) + 1e-6)
+    for t in range(L):
+        assert np.allclose(vals[0, t], _rotate(nrm[t], float(t), r_dim), rtol=1e-12, atol=1e-13)
+    # m = 4: block i is rotated to its last token, 4i + 3 (and only the last
+    # r_dim dims move).
+    m, N = 4, 3
+    tok = bf16_bits(r.standard_normal((B, m * N, d)))
+    w_s = (r.standard_normal(d) * 0.1).astype(np.float32)
+    b_pos = (r.standard_normal(m) * 0.1).astype(np.float32)
+    plain, _ = orc.pool(tok, np.array([m * N]), w_s, b_pos, None, m, 0, N, N)
+    roped, _ = orc.pool(tok, np.array([m * N]), w_s, b_pos, None, m, 0, N, N, rope_dim=r_dim)
+    for i in range(N):
+        assert np.allclose(roped[0, i], _rotate(plain[0, i], float(4 * i + 3), r_dim), rtol=1e-12,
+                           atol=1e-13)
+    assert np.array_equal(roped[0, :, : d - r_dim], plain[0, :, : d - r_dim])
 
 
 def test_rope_translation_invariance(orc):
+    # Shifting every position (query, window, entries) by S leaves the output
+    # unchanged.  Stored entries are kept exactly: their rotated dims are
+    # zero, so re-rotating them to the shifted positions is exact in bf16.
     B, Q, H, D, L, m, W, r_dim = 1, 1, 4, 64, 64, 4, 16, 32
     q, kv_tok, kv_c, sink = _mqa_case(B, Q, H, D, L, m, 27)
+    kv_c[..., D - r_dim:] = 0
     pos = np.array([[59]])
     sel = np.array([[[1, 5, 9, 14]]], np.int32)
     cnt = np.array([[4]], np.int32)
