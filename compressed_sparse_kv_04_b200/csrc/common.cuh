@@ -1,5 +1,5 @@
 // Shared device helpers for the sm_100a kernels: status reporting, bounded
-// waits, mbarriers, TMA (tiled and gather4), tcgen05 (TMEM alloc, MMA,
+// waits, mbarriers, TMA (tiled), bulk and cp.async copies, tcgen05 (TMEM alloc, MMA,
 // commit, ld/st) and cluster primitives, written as inline PTX.
 #pragma once
 
@@ -161,17 +161,6 @@ CSA_DEV void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int32
       : "memory");
 }
 
-// Row gather: four rows y0..y3 of the one-row box starting at column x,
-// landing at dst, dst+row_bytes, ... (the box must be one row high).
-CSA_DEV void tma_gather4(void* dst, const CUtensorMap* map, uint64_t* bar, int32_t x, int32_t y0,
-                         int32_t y1, int32_t y2, int32_t y3) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y0), "r"(y1),
-      "r"(y2), "r"(y3)
-      : "memory");
-}
 
 // ----------------------------------------------------------------- tcgen05 --
 // Tensor-memory address: lane in bits 31..16, column in 15..0.

@@ -62,9 +62,10 @@ struct TopkLaunch {
 };
 cudaError_t launch_topk(const TopkLaunch& a, cudaStream_t stream);
 
-// Shared-KV MQA decode (sparse or dense) with window and sink: a pair of
-// CTAs (cluster of 2) per (query row, split), each owning half of the head
-// dim; split partials are merged by the combine kernel.
+// Shared-KV MQA decode (sparse or dense) with window and sink: two CTAs per
+// (query row, split), each owning 64 of the heads at the full head dim;
+// split partials (fp16 O/l plus max and sum) are merged by the combine
+// kernel.
 struct MqaLaunch {
   int B, Q, H, D, m, W, rope_dim;
   int64_t N_cap, L_cap;

@@ -132,7 +132,6 @@ CSA_DEV bool wait_all(uint64_t* bar, uint32_t parity, const Params& p, volatile 
 template <int D, int R>
 __global__ void __launch_bounds__(kThreads, 1)
     mqa_heads_kernel(const __grid_constant__ CUtensorMap map_q,
-                     const __grid_constant__ CUtensorMap map_t,
                      const __grid_constant__ CUtensorMap box_c,
                      const __grid_constant__ CUtensorMap box_t, const Params p) {
   using C = MCfg<D>;
@@ -225,8 +224,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ---------------------------------------------------------- producer --
     // Contiguous tiles (dense entries, window tokens): one 64-row box per
-    // 128-byte chunk.  Selected entries: row gathers (tile::gather4), issued
-    // by every lane of the warp.
+    // 128-byte chunk.  Selected entries: this warp only writes the row
+    // metadata; the transform warps gather the rows.
     // The query block first (a caller input: no need to wait for the
     // previous kernel): 64 heads x D into the last stage, freed by qready.
     if (lane == 0) {
@@ -905,12 +904,9 @@ cudaError_t launch_impl(const MqaLaunch& a, cudaStream_t stream) {
   if (rows > 65535 || a.splits * 2 > 65535) return cudaErrorInvalidConfiguration;
 
   // Row-gather maps (one-row boxes) and 64-row box maps, 128-byte swizzle.
-  CUtensorMap map_q, map_t, box_c, box_t;
+  CUtensorMap map_q, box_c, box_t;
   cudaError_t e = make_tmap_2d(&map_q, a.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
                                (uint64_t)rows * a.H, D, TN, 64, CU_TENSOR_MAP_SWIZZLE_128B);
-  if (e != cudaSuccess) return e;
-  e = make_tmap_2d(&map_t, a.kv_tok, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)a.B * a.L_cap,
-                   D, 1, 64, CU_TENSOR_MAP_SWIZZLE_128B);
   if (e != cudaSuccess) return e;
   e = make_tmap_2d(&box_c, a.kv_c, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)a.B * a.N_cap,
                    D, TN, 64, CU_TENSOR_MAP_SWIZZLE_128B);
@@ -925,7 +921,7 @@ cudaError_t launch_impl(const MqaLaunch& a, cudaStream_t stream) {
   e = ensure_smem_attr(reinterpret_cast<const void*>(kern), 3 + (D == 512 ? 0 : 3) + R / 32, smem);
   if (e != cudaSuccess) return e;
   dim3 grid(2 * a.splits, rows, 1);
-  e = launch_pdl(kern, grid, dim3(kThreads), smem, stream, 0, map_q, map_t, box_c, box_t, p);
+  e = launch_pdl(kern, grid, dim3(kThreads), smem, stream, 0, map_q, box_c, box_t, p);
   if (e != cudaSuccess) return e;
   return launch_pdl(mqa_combine_kernel, dim3(rows, a.H), dim3(128),
                     (size_t)(D + a.splits) * sizeof(float), stream, 0, p, D, a.sink,
