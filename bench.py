@@ -721,6 +721,12 @@ class OracleStep:
             self.itok = bf16((1, tail, w.D_I))
             self.w_si = (rng.standard_normal(w.D_I) * 0.02).astype(np.float32)
         self.threads = os.cpu_count() or 1
+        # RoPE frequencies and logit scale: the oracle's own YaRN table for a
+        # workload with YaRN settings, else plain RoPE and 1/sqrt(d).
+        self.freq, self.scale = None, None
+        if w.yarn is not None:
+            self.freq = orc.yarn_inv_freq(w.rope_dim, *w.yarn)
+            self.scale = orc.yarn_logit_gain(w.yarn[0]) / d ** 0.5
 
     def run(self, n_sub=None, h_sub=None, a_sub=None):
         """Returns (compress_s, index_s, attention_s).  A sample covers the
@@ -733,7 +739,7 @@ class OracleStep:
         h_sub = w.H if h_sub is None else max(1, min(w.H, h_sub))
         t0 = time.perf_counter()
         orc.pool(self.tok, [tail], self.w_s, self.b_pos, None, m, tail // m - 1, 1, tail // m,
-                 rope_dim=w.rope_dim)
+                 rope_dim=w.rope_dim, rope_freq=self.freq)
         if w.csa:
             orc.pool(self.itok, [tail], self.w_si, self.b_pos, None, m, tail // m - 1, 1,
                      tail // m)
@@ -748,16 +754,17 @@ class OracleStep:
             if a_sub is not None:
                 cnt = np.minimum(cnt, a_sub).astype(np.int32)
             orc.mqa(q, self.pos, self.kv_c, self.tok, sink, m, w.W, w.rope_dim, idx, cnt,
-                    tok_base=w.L - tail)
+                    tok_base=w.L - tail, rope_freq=self.freq, scale=self.scale)
         else:
             t2 = t1
             if a_sub is None:
                 orc.mqa(q, self.pos, self.kv_c, self.tok, sink, m, w.W, w.rope_dim,
-                        tok_base=w.L - tail)
+                        tok_base=w.L - tail, rope_freq=self.freq, scale=self.scale)
             else:
                 sel = np.arange(min(a_sub, N), dtype=np.int32).reshape(1, 1, -1)
                 orc.mqa(q, self.pos, self.kv_c, self.tok, sink, m, w.W, w.rope_dim, sel,
-                        np.full((1, 1), sel.shape[-1], np.int32), tok_base=w.L - tail)
+                        np.full((1, 1), sel.shape[-1], np.int32), tok_base=w.L - tail,
+                        rope_freq=self.freq, scale=self.scale)
         t3 = time.perf_counter()
         return t1 - t0, t2 - t1, t3 - t2
 

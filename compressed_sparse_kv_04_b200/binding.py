@@ -24,7 +24,7 @@ OP_INDEX_TOPK, OP_SPARSE_MQA, OP_DENSE_MQA, OP_PREFILL = 1, 2, 3, 4
 EXPORTS = ["csa_version", "csa_last_error", "csa_workspace_bytes", "hca_compress",
            "csa_compress", "lightning_index_topk", "lightning_index_scores", "topk_select",
            "sparse_mqa_decode", "dense_mqa_decode", "csa_prefill_chunk",
-           "lightning_index_topk_static"]
+           "lightning_index_topk_static", "csa_rope_yarn"]
 
 
 class CsaError(RuntimeError):
@@ -78,6 +78,8 @@ def _declare(L):
                                     i64, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp, vp]
     L.lightning_index_topk_static.argtypes = [P, i32, vp, vp, vp, vp, vp, i64, vp, vp, vp, vp,
                                               vp]
+    L.csa_rope_yarn.argtypes = [i32, C.c_double, C.c_double, C.c_double, C.c_double,
+                                C.c_double, C.POINTER(C.c_double), C.POINTER(C.c_double)]
     for name in EXPORTS[3:]:
         getattr(L, name).restype = i32
 
@@ -93,7 +95,13 @@ def make_params(B, d, H=0, H_I=0, D_I=0, k=0, window=0, rope_dim=0, m=4, eps=1e-
 
 
 def params_for(w, B=None, **kw):
-    """csa_params for a Workload (compressed_sparse_kv_04_b200.configs)."""
+    """csa_params for a Workload (compressed_sparse_kv_04_b200.configs).  A
+    workload with YaRN settings gets the library's YaRN frequency table and
+    the logit scale gain / sqrt(d), unless the caller passes its own."""
+    if w.yarn is not None and w.rope_dim > 0 and "rope_inv_freq" not in kw:
+        tab, gain = rope_yarn(w.rope_dim, *w.yarn)
+        kw["rope_inv_freq"] = tab
+        kw.setdefault("softmax_scale", gain / w.d ** 0.5)
     return make_params(B or w.B, w.d, w.H, w.H_I, w.D_I, w.k, w.W, w.rope_dim, w.m, **kw)
 
 
@@ -169,6 +177,16 @@ def lightning_index_topk_static(p, Q, q_idx, q_scale, w, idx_key, idx_scale, pos
         C.byref(p), Q, _ptr(q_idx), _ptr(q_scale), _ptr(w), _ptr(idx_key), _ptr(idx_scale),
         idx_key.shape[1], _ptr(pos_q), _ptr(topk_idx), _ptr(topk_cnt), _ptr(dev_status),
         _stream(stream)))
+
+
+def rope_yarn(rope_dim, factor, beta_fast, beta_slow, original_len, base=10000.0):
+    """YaRN frequency table and logit gain (host only): returns (list of
+    rope_dim/2 frequencies for make_params(rope_inv_freq=...), logit gain)."""
+    tab = (C.c_double * (rope_dim // 2))()
+    gain = C.c_double()
+    _check(lib().csa_rope_yarn(rope_dim, base, factor, beta_fast, beta_slow, original_len, tab,
+                               C.byref(gain)))
+    return list(tab), gain.value
 
 
 def lightning_index_scores(p, Q, q_idx, q_scale, w, idx_key, idx_scale, pos_q, scores,

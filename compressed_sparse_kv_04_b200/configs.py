@@ -30,6 +30,7 @@ class Workload:
     P: int = 0           # prefill: prior tokens
     T: int = 0           # prefill: new tokens
     seed: int = 0
+    yarn: tuple | None = None  # (factor, beta_fast, beta_slow, original_len) or plain RoPE
 
     @property
     def D(self) -> int:
@@ -57,7 +58,16 @@ CSA_PREFILL = Workload("csa_prefill_4096_after_65536", "csa_prefill", B=1, L=655
                        d=512, m=4, H=128, rope_dim=64, W=128, H_I=64, D_I=128, k=1024,
                        P=65536, T=4096, seed=20260005)
 
-ALL = [TINY_CSA, CSA_128K, HCA_1M, CSA_1M, CSA_PREFILL]
+# V4-Flash attention ("DeepSeek V4-Pro" (llm-arch-kb), "Family"): 64 query
+# heads and top-k 512, the rest as V4-Pro; RoPE with the YaRN frequencies of
+# "5. 1M context, gradually" (factor 16, beta_fast 32, beta_slow 1) over an
+# original context of 1,048,576 / 16 tokens.
+YARN_V4 = (16.0, 32.0, 1.0, 1048576 / 16)
+CSA_FLASH_128K = Workload("csa_flash_decode_128k_b8", "csa_decode", B=8, L=131072, d=512, m=4,
+                          H=64, rope_dim=64, W=128, H_I=64, D_I=128, k=512, seed=20260006,
+                          yarn=YARN_V4)
+
+ALL = [TINY_CSA, CSA_128K, HCA_1M, CSA_1M, CSA_PREFILL, CSA_FLASH_128K]
 BY_NAME = {w.name: w for w in ALL}
 
 

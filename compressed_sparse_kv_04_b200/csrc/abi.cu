@@ -106,7 +106,8 @@ float softmax_scale_of(const csa_params* p) {
 
 int splits_for(const csa_params* p, csa_op op, int rows, int64_t N_cap) {
   const int64_t compressed_max = (op == CSA_OP_DENSE_MQA) ? N_cap : (int64_t)p->k;
-  return csa::mqa_choose_splits(rows, compressed_max, p->window, csa::device_sm_count());
+  return csa::mqa_choose_splits(rows, compressed_max, p->window, csa::device_sm_count(),
+                                p->H);
 }
 
 }  // namespace
@@ -125,7 +126,37 @@ csa_status set_error(csa_status s, const char* fmt, ...) {
 
 extern "C" {
 
-int csa_version(void) { return 100; }
+int csa_version(void) { return 101; }
+
+csa_status csa_rope_yarn(int rope_dim, double base, double factor, double beta_fast,
+                         double beta_slow, double original_len, double* inv_freq,
+                         double* logit_gain) {
+  const char* fn = "csa_rope_yarn";
+  if (rope_dim < 2 || rope_dim > 128 || rope_dim % 2)
+    return fail(CSA_ERR_UNSUPPORTED_SHAPE, "%s: rope_dim=%d (supported: even, 2..128)", fn,
+                rope_dim);
+  if (!inv_freq) return fail(CSA_ERR_INVALID_ARG, "%s: inv_freq is NULL", fn);
+  if (!(base > 1.0) || !std::isfinite(base) || !(factor >= 1.0) || !std::isfinite(factor) ||
+      !(beta_slow >= 0.0) || !(beta_fast > beta_slow) || !std::isfinite(beta_fast) ||
+      !(original_len > 0.0) || !std::isfinite(original_len))
+    return fail(CSA_ERR_INVALID_ARG,
+                "%s: need base > 1, factor >= 1, 0 <= beta_slow < beta_fast, original_len > 0",
+                fn);
+  const double kTwoPi = 6.283185307179586;
+  for (int j = 0; j < rope_dim / 2; ++j) {
+    const double theta = std::pow(base, -2.0 * j / (double)rope_dim);
+    // Turns of this pair over the original context place it on the ramp:
+    // 1 keeps the frequency, 0 divides it by the factor.
+    double ramp = (original_len * theta / kTwoPi - beta_slow) / (beta_fast - beta_slow);
+    ramp = ramp < 0.0 ? 0.0 : (ramp > 1.0 ? 1.0 : ramp);
+    inv_freq[j] = theta / factor + ramp * (theta - theta / factor);
+  }
+  if (logit_gain) {
+    const double t = 1.0 + 0.1 * std::log(factor);
+    *logit_gain = t * t;
+  }
+  return CSA_OK;
+}
 
 const char* csa_last_error(void) { return g_err; }
 

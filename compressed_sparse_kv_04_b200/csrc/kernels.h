@@ -62,8 +62,9 @@ struct TopkLaunch {
 };
 cudaError_t launch_topk(const TopkLaunch& a, cudaStream_t stream);
 
-// Shared-KV MQA decode (sparse or dense) with window and sink: two CTAs per
-// (query row, split), each owning 64 of the heads at the full head dim;
+// Shared-KV MQA decode (sparse or dense) with window and sink: one CTA per
+// (query row, split) for H <= 64, two for H > 64 (64 heads each), at the
+// full head dim;
 // split partials (fp16 O/l plus max and sum) are merged by the combine
 // kernel.
 struct MqaLaunch {
@@ -90,7 +91,7 @@ struct MqaLaunch {
   int32_t* status;
 };
 size_t mqa_workspace_bytes(int rows, int splits, int H, int D);
-int mqa_choose_splits(int rows, int64_t compressed_max, int window, int num_sms);
+int mqa_choose_splits(int rows, int64_t compressed_max, int window, int num_sms, int H);
 cudaError_t launch_mqa(const MqaLaunch& a, cudaStream_t stream);
 
 int device_sm_count();

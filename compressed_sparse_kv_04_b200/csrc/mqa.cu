@@ -53,10 +53,11 @@ size_t mqa_workspace_bytes(int rows, int splits, int H, int D) {
 
 // Splits of each row's KV list over CTA pairs: at most one wave of pairs
 // (rows * splits <= SMs / 2), no split left without a tile.
-int mqa_choose_splits(int rows, int64_t compressed_max, int window, int num_sms) {
+int mqa_choose_splits(int rows, int64_t compressed_max, int window, int num_sms, int H) {
   const int64_t tiles = (compressed_max + 63) / 64 + (window + 63) / 64;
-  const int64_t pairs = std::max(1, num_sms / 2);
-  int64_t s = std::max<int64_t>(1, pairs / std::max(1, rows));
+  // One CTA per (row, split) owns up to 64 heads: H > 64 takes two.
+  const int64_t units = std::max(1, num_sms / (H > 64 ? 2 : 1));
+  int64_t s = std::max<int64_t>(1, units / std::max(1, rows));
   s = std::min<int64_t>(s, std::max<int64_t>(1, tiles));
   const int64_t tps = (tiles + s - 1) / s;
   s = std::max<int64_t>(1, (tiles + tps - 1) / tps);
@@ -157,8 +158,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   pdl_trigger();
-  const int hg0 = (blockIdx.x & 1) * HC;  // first head of this CTA
-  const int split = blockIdx.x >> 1;
+  // H > 64: CTAs 2s and 2s+1 of split s own heads 0..63 and 64..H-1.
+  const bool pair = p.H > HC;
+  const int hg0 = pair ? (blockIdx.x & 1) * HC : 0;  // first head of this CTA
+  const int split = pair ? blockIdx.x >> 1 : blockIdx.x;
   const int row = blockIdx.y;
   const int b = row / p.Q;
 
@@ -187,7 +190,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   };
 
   float* pml = p.part_ml + ((int64_t)row * p.splits + split) * 2 * p.H;
-  if (hg0 >= p.H) return;  // this CTA has no heads (H <= 64)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) {
@@ -901,7 +903,8 @@ cudaError_t launch_impl(const MqaLaunch& a, cudaStream_t stream) {
   p.status = a.status;
   for (int j = 0; j < 64; ++j) p.inv_freq[j] = a.inv_freq[j];
   const int rows = a.B * a.Q;
-  if (rows > 65535 || a.splits * 2 > 65535) return cudaErrorInvalidConfiguration;
+  const int cps = a.H > HC ? 2 : 1;  // CTAs per (row, split)
+  if (rows > 65535 || a.splits * cps > 65535) return cudaErrorInvalidConfiguration;
 
   // Row-gather maps (one-row boxes) and 64-row box maps, 128-byte swizzle.
   CUtensorMap map_q, box_c, box_t;
@@ -920,7 +923,7 @@ cudaError_t launch_impl(const MqaLaunch& a, cudaStream_t stream) {
   auto kern = mqa_heads_kernel<D, R>;
   e = ensure_smem_attr(reinterpret_cast<const void*>(kern), 3 + (D == 512 ? 0 : 3) + R / 32, smem);
   if (e != cudaSuccess) return e;
-  dim3 grid(2 * a.splits, rows, 1);
+  dim3 grid(cps * a.splits, rows, 1);
   e = launch_pdl(kern, grid, dim3(kThreads), smem, stream, 0, map_q, box_c, box_t, p);
   if (e != cudaSuccess) return e;
   return launch_pdl(mqa_combine_kernel, dim3(rows, a.H), dim3(128),

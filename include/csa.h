@@ -11,7 +11,8 @@
  *        Hyper-Connections Visualised" (webconsulting.at), "Key points" and
  *        "Dual Compression and Indexing".
  *   [P5] "DeepSeek V4-Pro" (lizeman.github.io llm-arch-kb), "What's new in
- *        V4 / 1. Hybrid attention: CSA + HCA replace MLA".
+ *        V4 / 1. Hybrid attention: CSA + HCA replace MLA"; "5. 1M context,
+ *        gradually" (YaRN extension); "Family" (V4-Flash shapes).
  *
  * Conventions shared by every entry point
  *   - Tensor pointers are DEVICE pointers owned by the caller (the binding
@@ -90,6 +91,33 @@ int csa_version(void);
 
 /* Thread-local message for the last non-OK status returned on this thread. */
 const char* csa_last_error(void);
+
+/* ---------------------------------------------------------------------------
+ * YaRN RoPE frequency table (host only; no device work).  [P5] "5. 1M
+ * context, gradually": the context is extended to 1,048,576 tokens with
+ * YaRN, factor 16, beta_fast 32, beta_slow 1.  The pages give no formula;
+ * this follows the published method (Peng et al. 2023, "YaRN: Efficient
+ * Context Window Extension of Large Language Models", NTK-by-parts):
+ *   theta_j  = base^(-2j/rope_dim)                 j < rope_dim/2
+ *   turns_j  = original_len * theta_j / (2 pi)
+ *   ramp_j   = clamp((turns_j - beta_slow) / (beta_fast - beta_slow), 0, 1)
+ *   inv_freq[j] = ramp_j * theta_j + (1 - ramp_j) * theta_j / factor
+ *   *logit_gain = (1 + 0.1 ln factor)^2   (the method's attention
+ *                 temperature; multiply 1/sqrt(d) by it for softmax_scale)
+ * Pass the table as csa_params.rope_inv_freq: compression, the window
+ * rotation, the query rotation and the inverse rotation of the output all
+ * use it.  (original_len = 1,048,576 / 16 = 65,536 is the reading for the
+ * pages' schedule.)
+ *   inv_freq   host, [rope_dim/2] doubles (written)
+ *   logit_gain host, one double (written) or NULL
+ * Errors: CSA_ERR_UNSUPPORTED_SHAPE for rope_dim odd or outside 2..128;
+ *         CSA_ERR_INVALID_ARG for inv_freq NULL, base <= 1, factor < 1,
+ *         beta_slow < 0, beta_fast <= beta_slow, original_len <= 0 or any
+ *         non-finite value.
+ * ------------------------------------------------------------------------- */
+csa_status csa_rope_yarn(int rope_dim, double base, double factor, double beta_fast,
+                         double beta_slow, double original_len, double* inv_freq,
+                         double* logit_gain);
 
 /* Workspace bytes that `op` needs for these params.
  *   Q     queries per sequence (1 for decode; T for CSA_OP_PREFILL),

@@ -143,12 +143,15 @@ uint8_t e4m3_encode(float xf) {
 // [P5] rotates only the last 64 dimensions of query, KV and output.
 // Reading: rotate-half pairing over the last r dimensions, (D-r+j, D-r+j+r/2) for
 // j < r/2, frequency theta_j = base^(-2j/r), angle = position * theta_j.
-// The pages give neither the pairing nor the base; 10000 is used.
-void rope_apply(double* v, int D, int r, double base, double pos, double sign) {
+// The pages give neither the pairing nor the base; 10000 is used.  A
+// caller-given table freq[j] replaces base^(-2j/r) (a context-extension
+// rescaling such as YaRN changes only these per-pair frequencies).
+void rope_apply(double* v, int D, int r, double base, const double* freq, double pos,
+                double sign) {
   if (r <= 0) return;
   int b0 = D - r, half = r / 2;
   for (int j = 0; j < half; ++j) {
-    double theta = std::pow(base, -2.0 * j / (double)r);
+    double theta = freq ? freq[j] : std::pow(base, -2.0 * j / (double)r);
     double ang = sign * pos * theta;
     double c = std::cos(ang), s = std::sin(ang);
     double x1 = v[b0 + j], x2 = v[b0 + j + half];
@@ -168,7 +171,7 @@ void rms_norm(double* v, int D, const float* gamma, double eps) {
 
 extern "C" {
 
-int orc_abi_version(void) { return 1; }
+int orc_abi_version(void) { return 2; }
 
 double orc_bf16_decode(uint16_t h) { return bf16_decode(h); }
 uint16_t orc_bf16_encode(double x) { return bf16_encode(x); }
@@ -200,7 +203,8 @@ void orc_bf16_encode_array(int64_t n, const double* x, uint16_t* out) {
 // indexer stream, which the pages do not rotate).
 void orc_pool(int B, int64_t L_cap, int d, int m, const uint16_t* tok, const int64_t* ctx_len,
               const float* w_s, const float* b_pos, const float* gamma, double eps, int normalize,
-              int rope_dim, double rope_base, int64_t first_block, int64_t n_blocks,
+              int rope_dim, double rope_base, const double* rope_freq, int64_t first_block,
+              int64_t n_blocks,
               int64_t N_cap, double* out, uint8_t* written, int nthreads) {
   parallel_for((int64_t)B * n_blocks, nthreads, [&](int64_t w) {
     int64_t b = w / n_blocks, i = first_block + w % n_blocks;
@@ -227,7 +231,7 @@ void orc_pool(int B, int64_t L_cap, int d, int m, const uint16_t* tok, const int
       for (int k = 0; k < d; ++k) p[k] += a * bf16_decode(row[k]);
     }
     if (normalize) rms_norm(p.data(), d, gamma, eps);
-    rope_apply(p.data(), d, rope_dim, rope_base, (double)((i + 1) * m - 1), +1.0);
+    rope_apply(p.data(), d, rope_dim, rope_base, rope_freq, (double)((i + 1) * m - 1), +1.0);
     double* o = out + ((int64_t)b * N_cap + i) * d;
     for (int k = 0; k < d; ++k) o[k] = p[k];
     if (written) written[(int64_t)b * N_cap + i] = 1;
@@ -347,7 +351,7 @@ void orc_topk(int64_t BQ, int64_t N_cap, const double* scores, const int64_t* n_
 // kv_tok holds token rows tok_base .. tok_base+L_cap-1 (a window of a long
 // stream; pure storage offset, no effect on the arithmetic).
 void orc_mqa(int B, int Q, int H, int D, int m, int W, int rope_dim, double rope_base,
-             const uint16_t* q, const int64_t* pos_q, const uint16_t* kv_c, int64_t N_cap,
+             const double* rope_freq, const uint16_t* q, const int64_t* pos_q, const uint16_t* kv_c, int64_t N_cap,
              const int32_t* sel_idx, const int32_t* sel_cnt, int kmax, const uint16_t* kv_tok,
              int64_t L_cap, int64_t tok_base, const float* sink, const float* gamma_q,
              const float* gamma_kv, double eps, double scale, double* out, double* lse,
@@ -382,7 +386,7 @@ void orc_mqa(int B, int Q, int H, int D, int m, int W, int rope_dim, double rope
         const uint16_t* row = kv_tok + (b * L_cap + (t - tok_base)) * D;
         for (int d = 0; d < D; ++d) v[d] = bf16_decode(row[d]);
         rms_norm(v, D, gamma_kv, eps);
-        rope_apply(v, D, rope_dim, rope_base, (double)t, +1.0);
+        rope_apply(v, D, rope_dim, rope_base, rope_freq, (double)t, +1.0);
       }
     }
     parallel_for(H, nthreads, [&](int64_t h) {
@@ -390,7 +394,7 @@ void orc_mqa(int B, int Q, int H, int D, int m, int W, int rope_dim, double rope
       const uint16_t* qr = q + (bq * H + h) * D;
       for (int d = 0; d < D; ++d) qh[d] = bf16_decode(qr[d]);
       rms_norm(qh.data(), D, gamma_q, eps);
-      rope_apply(qh.data(), D, rope_dim, rope_base, (double)pos, +1.0);
+      rope_apply(qh.data(), D, rope_dim, rope_base, rope_freq, (double)pos, +1.0);
       std::vector<double> s(T);
       double smax = -inf;
       for (int64_t j = 0; j < T; ++j) {
@@ -420,7 +424,7 @@ void orc_mqa(int B, int Q, int H, int D, int m, int W, int rope_dim, double rope
         for (int d = 0; d < D; ++d) acc[d] += p * kv[j * D + d];
       }
       for (int d = 0; d < D; ++d) acc[d] /= L;
-      rope_apply(acc.data(), D, rope_dim, rope_base, (double)pos, -1.0);
+      rope_apply(acc.data(), D, rope_dim, rope_base, rope_freq, (double)pos, -1.0);
       for (int d = 0; d < D; ++d) o[d] = acc[d];
       if (lse) lse[bq * H + h] = M + std::log(L);
     });

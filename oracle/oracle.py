@@ -57,12 +57,13 @@ def _declare(L):
     L.orc_e4m3_encode.restype = C.c_uint8
     L.orc_bf16_encode_array.argtypes = [i64, P(f64), P(C.c_uint16)]
     L.orc_pool.argtypes = [i32, i64, i32, i32, P(C.c_uint16), P(i64), P(f32), P(f32), P(f32),
-                           f64, i32, i32, f64, i64, i64, i64, P(f64), P(C.c_uint8), i32]
+                           f64, i32, i32, f64, P(f64), i64, i64, i64, P(f64), P(C.c_uint8),
+                           i32]
     L.orc_quant_rows_e4m3.argtypes = [i64, i32, P(f64), P(C.c_uint8), P(f32)]
     L.orc_index_scores.argtypes = [i32, i32, i32, i32, i32, P(C.c_uint8), P(f32), P(f32),
                                    P(C.c_uint8), P(f32), i64, P(i64), P(f64), i32]
     L.orc_topk.argtypes = [i64, i64, P(f64), P(i64), i32, P(C.c_int32), P(C.c_int32), i32]
-    L.orc_mqa.argtypes = [i32, i32, i32, i32, i32, i32, i32, f64, P(C.c_uint16), P(i64),
+    L.orc_mqa.argtypes = [i32, i32, i32, i32, i32, i32, i32, f64, P(f64), P(C.c_uint16), P(i64),
                           P(C.c_uint16), i64, P(C.c_int32), P(C.c_int32), i32, P(C.c_uint16),
                           i64, i64, P(f32), P(f32), P(f32), f64, f64, P(f64), P(f64), i32]
 
@@ -93,11 +94,57 @@ def e4m3_encode_scalar(x: float) -> int:
     return int(lib().orc_e4m3_encode(float(np.float32(x))))
 
 
+# ------------------------------------------------- RoPE frequency tables --
+def rope_inv_freq(rope_dim, base=10000.0):
+    """Plain RoPE frequencies theta_j = base^(-2j/r), j < r/2."""
+    j = np.arange(rope_dim // 2, dtype=np.float64)
+    return base ** (-2.0 * j / rope_dim)
+
+
+def yarn_inv_freq(rope_dim, factor, beta_fast, beta_slow, original_len, base=10000.0):
+    """YaRN context-extension frequencies (the DeepSeek-V4 pages' training
+    section: YaRN with factor 16, beta_fast 32 and beta_slow 1 extends the
+    context to 1,048,576 tokens), following the published method (Peng et
+    al., "YaRN: Efficient Context Window Extension of Large Language Models",
+    2023, the "NTK-by-parts" interpolation):
+
+      theta_j   = base^(-2j/r)                  plain frequency of pair j
+      rot_j     = original_len * theta_j / 2pi  full turns of pair j over the
+                                                original context
+      gamma_j   = clamp((rot_j - beta_slow) / (beta_fast - beta_slow), 0, 1)
+      theta'_j  = gamma_j * theta_j + (1 - gamma_j) * theta_j / factor
+
+    Pairs that turn many times over the original context keep their
+    frequency; pairs that turn less than once are interpolated by `factor`;
+    the ones between are blended linearly in rot_j."""
+    theta = rope_inv_freq(rope_dim, base)
+    rot = original_len * theta / (2.0 * math.pi)
+    g = np.clip((rot - beta_slow) / (beta_fast - beta_slow), 0.0, 1.0)
+    return g * theta + (1.0 - g) * theta / factor
+
+
+def yarn_logit_gain(factor):
+    """YaRN attention temperature: q and k are both scaled by
+    sqrt(1/t) = 0.1 ln(factor) + 1 (same paper), i.e. the logits by its square."""
+    return (0.1 * math.log(factor) + 1.0) ** 2
+
+
 # -------------------------------------------------------------------- steps --
+def _freq(rope_freq, rope_dim):
+    if rope_freq is None:
+        return None
+    f = _c(rope_freq, np.float64)
+    if f.shape != (rope_dim // 2,):
+        raise ValueError(f"rope_freq must hold rope_dim/2 = {rope_dim // 2} values")
+    return f
+
+
 def pool(tok, ctx_len, w_s, b_pos, gamma, m, first_block, n_blocks, N_cap, eps=1e-6,
-         normalize=True, nthreads=0, rope_dim=0, rope_base=10000.0):
+         normalize=True, nthreads=0, rope_dim=0, rope_base=10000.0, rope_freq=None):
     """Compression step (a1) in fp64.  Returns (values[B,N_cap,d], written[B,N_cap]).
-    rope_dim > 0: each entry is stored rotated to its position (i+1)*m - 1."""
+    rope_dim > 0: each entry is stored rotated to its position (i+1)*m - 1.
+    rope_freq [rope_dim/2] replaces the frequencies rope_base^(-2j/rope_dim)."""
+    rope_freq = _freq(rope_freq, rope_dim)
     tok = _c(tok, np.uint16)
     B, L_cap, d = tok.shape
     ctx_len = _c(ctx_len, np.int64)
@@ -106,7 +153,8 @@ def pool(tok, ctx_len, w_s, b_pos, gamma, m, first_block, n_blocks, N_cap, eps=1
     lib().orc_pool(B, L_cap, d, m, _p(tok, C.c_uint16), _p(ctx_len, C.c_int64),
                    _p(_c(w_s, np.float32), C.c_float), _p(_c(b_pos, np.float32), C.c_float),
                    _p(None if gamma is None else _c(gamma, np.float32), C.c_float),
-                   eps, 1 if normalize else 0, rope_dim, rope_base, first_block, n_blocks, N_cap,
+                   eps, 1 if normalize else 0, rope_dim, rope_base, _p(rope_freq, C.c_double),
+                   first_block, n_blocks, N_cap,
                    _p(out, C.c_double), _p(written, C.c_uint8), nthreads)
     return out, written.astype(bool)
 
@@ -154,13 +202,15 @@ def topk(scores, n_vis, k, nthreads=0):
 
 def mqa(q, pos_q, kv_c, kv_tok, sink, m, W, rope_dim, sel_idx=None, sel_cnt=None,
         gamma_q=None, gamma_kv=None, eps=1e-6, scale=None, rope_base=10000.0, nthreads=0,
-        tok_base=0):
+        tok_base=0, rope_freq=None):
     """Shared-KV MQA with window and sink (a4 sparse when sel_idx is given, else a5 dense).
 
     q [B,Q,H,D] bf16 bits; pos_q [B,Q]; kv_c [B,N_cap,D]; kv_tok [B,L_cap,D] holding
-    token rows tok_base .. tok_base+L_cap-1.
+    token rows tok_base .. tok_base+L_cap-1.  rope_freq [rope_dim/2] replaces
+    the frequencies rope_base^(-2j/rope_dim).
     Returns (out fp64 [B,Q,H,D], lse fp64 [B,Q,H]).
     """
+    rope_freq = _freq(rope_freq, rope_dim)
     q = _c(q, np.uint16)
     B, Q, H, D = q.shape
     kv_c = _c(kv_c, np.uint16)
@@ -175,7 +225,8 @@ def mqa(q, pos_q, kv_c, kv_tok, sink, m, W, rope_dim, sel_idx=None, sel_cnt=None
         sel_cnt = _c(sel_cnt, np.int32)
     out = np.empty((B, Q, H, D), np.float64)
     lse = np.empty((B, Q, H), np.float64)
-    lib().orc_mqa(B, Q, H, D, m, W, rope_dim, rope_base, _p(q, C.c_uint16),
+    lib().orc_mqa(B, Q, H, D, m, W, rope_dim, rope_base, _p(rope_freq, C.c_double),
+                  _p(q, C.c_uint16),
                   _p(_c(pos_q, np.int64), C.c_int64), _p(kv_c, C.c_uint16), N_cap,
                   _p(sel_idx, C.c_int32), _p(sel_cnt, C.c_int32), kmax,
                   _p(kv_tok, C.c_uint16), L_cap, tok_base, _p(_c(sink, np.float32), C.c_float),
@@ -187,11 +238,11 @@ def mqa(q, pos_q, kv_c, kv_tok, sink, m, W, rope_dim, sel_idx=None, sel_cnt=None
 
 # --------------------------------------------------------------- composites --
 def compress_kv(tok, ctx_len, w_s, b_pos, gamma, m, first_block, n_blocks, N_cap, eps=1e-6,
-                nthreads=0, rope_dim=0, rope_base=10000.0):
+                nthreads=0, rope_dim=0, rope_base=10000.0, rope_freq=None):
     """a1 for the KV stream with bfloat16 storage (entries stored rotated to
     their position when rope_dim > 0): returns (bf16 bits, written mask, fp64 values)."""
     vals, written = pool(tok, ctx_len, w_s, b_pos, gamma, m, first_block, n_blocks, N_cap,
-                         eps, True, nthreads, rope_dim, rope_base)
+                         eps, True, nthreads, rope_dim, rope_base, rope_freq)
     return bf16_encode(vals), written, vals
 
 

@@ -113,3 +113,32 @@ def test_workspace_sizes_are_monotone(L):
     assert L.csa_workspace_bytes(C.byref(p), 2, 1, 32768) > 0
     assert L.csa_workspace_bytes(C.byref(p), 3, 1, 8192) > 0
     assert L.csa_workspace_bytes(C.byref(p), 9, 1, 8192) == 0
+
+
+# ---------------------------------------------- YaRN frequency table (host) --
+@pytest.mark.parametrize("args", [(64, 16.0, 32.0, 1.0, 65536.0), (32, 4.0, 32.0, 1.0, 4096.0),
+                                  (64, 1.0, 32.0, 1.0, 4096.0), (64, 40.0, 16.0, 2.0, 1.0e6),
+                                  (2, 16.0, 32.0, 1.0, 100.0)])
+def test_yarn_table_matches_the_oracle(L, orc, args):
+    import math
+
+    import numpy as np
+    tab, gain = binding.rope_yarn(*args)
+    assert np.allclose(tab, orc.yarn_inv_freq(*args), rtol=1e-14, atol=0)
+    assert math.isclose(gain, orc.yarn_logit_gain(args[1]), rel_tol=1e-14)
+
+
+@pytest.mark.parametrize("args,code", [((63, 16.0, 32.0, 1.0, 65536.0), 2),
+                                       ((0, 16.0, 32.0, 1.0, 65536.0), 2),
+                                       ((130, 16.0, 32.0, 1.0, 65536.0), 2),
+                                       ((64, 0.5, 32.0, 1.0, 65536.0), 1),
+                                       ((64, 16.0, 1.0, 1.0, 65536.0), 1),
+                                       ((64, 16.0, 32.0, -1.0, 65536.0), 1),
+                                       ((64, 16.0, 32.0, 1.0, 0.0), 1),
+                                       ((64, 16.0, 32.0, 1.0, float("nan")), 1),
+                                       ((64, float("inf"), 32.0, 1.0, 65536.0), 1)])
+def test_yarn_argument_checks(L, args, code):
+    with pytest.raises(binding.CsaError) as e:
+        binding.rope_yarn(*args)
+    assert e.value.status == code
+    assert L.csa_rope_yarn(64, 1e4, 16.0, 32.0, 1.0, 65536.0, None, None) == 1

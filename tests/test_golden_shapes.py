@@ -29,3 +29,15 @@ def test_one_million_context_entry_counts():
     assert configs.HCA_1M.N_c == 8192
     # The double reduction of CSA: n -> n/m -> k.
     assert n_csa // v("top_k") == 256
+
+
+def test_flash_and_yarn_settings():
+    w = configs.CSA_FLASH_128K
+    assert (w.H, w.k) == (v("flash_query_heads"), v("flash_top_k"))
+    assert (w.m, w.H_I, w.D_I, w.D, w.rope_dim, w.W) == (
+        v("csa_ratio_m"), v("indexer_heads"), v("indexer_head_dim"), v("head_dim"), v("rope_dims"),
+        v("window"))
+    factor, beta_fast, beta_slow, original_len = w.yarn
+    assert (factor, beta_fast, beta_slow) == (
+        v("yarn_factor"), v("yarn_beta_fast"), v("yarn_beta_slow"))
+    assert original_len * factor == v("context_tokens")

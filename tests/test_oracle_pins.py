@@ -353,12 +353,13 @@ def test_sink_limits_and_closed_form(orc):
     assert np.allclose(lse[0, 0], np.logaddexp(s, z.astype(np.float64)), rtol=1e-13)
 
 
-def _rotate(v, pos, r_dim, base=10000.0):
+def _rotate(v, pos, r_dim, base=10000.0, theta=None):
     """Rotate-half rotation of the last r_dim dims of v by position pos (the
-    textbook form, written out here to check the oracle against it)."""
+    textbook form, written out here to check the oracle against it); theta
+    overrides the per-pair frequencies."""
     D = v.shape[-1]
     half = r_dim // 2
-    th = base ** (-2.0 * np.arange(half) / r_dim)
+    th = base ** (-2.0 * np.arange(half) / r_dim) if theta is None else np.asarray(theta)
     c, s = np.cos(pos * th), np.sin(pos * th)
     out = v.copy()
     x1, x2 = v[..., D - r_dim: D - half], v[..., D - half:]
@@ -452,3 +453,75 @@ def test_incomplete_block_is_invisible(orc):
     kv_c2[0, 1] = bf16_bits(np.full(D, 5.0))
     o3, _ = orc.mqa(q, pos, kv_c2, kv_tok, sink, m, W, 8)
     assert not np.allclose(o3, o1)
+
+
+# ------------------------------------------------------ YaRN (context extension)
+def test_yarn_factor_one_is_plain_rope(orc):
+    plain = 10000.0 ** (-np.arange(32) / 32.0)
+    assert np.allclose(orc.yarn_inv_freq(64, 1.0, 32.0, 1.0, 4096), plain, rtol=1e-15, atol=0)
+    assert orc.yarn_logit_gain(1.0) == 1.0
+
+
+def test_yarn_regions_kept_interpolated_and_blended(orc):
+    # r = 64, base 1e4, original context 4096: pair j turns 4096 * 1e4^(-j/32)
+    # / 2pi times.  It keeps its frequency while that is >= 32 turns, i.e. for
+    # j <= 8 log10(4096 / (64 pi)); it is divided by the factor once it is <= 1
+    # turn, i.e. for j >= 8 log10(4096 / (2 pi)); between, the ratio falls
+    # strictly from 1 to 1/factor.
+    s = 16.0
+    tab = orc.yarn_inv_freq(64, s, 32.0, 1.0, 4096)
+    ratio = tab / 10000.0 ** (-np.arange(32) / 32.0)
+    j_keep = math.floor(8 * math.log10(4096 / (64 * math.pi)))
+    j_interp = math.ceil(8 * math.log10(4096 / (2 * math.pi)))
+    assert 0 < j_keep < j_interp < 31
+    assert np.allclose(ratio[: j_keep + 1], 1.0, rtol=1e-14, atol=0)
+    assert np.allclose(ratio[j_interp:], 1.0 / s, rtol=1e-14, atol=0)
+    mid = ratio[j_keep + 1: j_interp]
+    assert ((mid < 1.0) & (mid > 1.0 / s)).all() and (np.diff(ratio[j_keep: j_interp + 1]) < 0).all()
+
+
+def test_yarn_ramp_midpoint(orc):
+    # An original context on which pair 5 turns exactly (32 + 1) / 2 times sits
+    # half way up the ramp: its frequency is the mean of theta and theta / s.
+    s, th5 = 16.0, 10000.0 ** (-10.0 / 64)
+    L0 = 16.5 * 2 * math.pi / th5
+    tab = orc.yarn_inv_freq(64, s, 32.0, 1.0, L0)
+    assert math.isclose(tab[5], th5 * (1 + 1 / s) / 2, rel_tol=1e-13)
+
+
+def test_yarn_logit_gain_factor_16(orc):
+    # sqrt(1/t) = 1 + 0.1 ln 16 = 1 + 0.4 ln 2.
+    assert math.isclose(orc.yarn_logit_gain(16.0), (1 + 0.4 * math.log(2.0)) ** 2, rel_tol=1e-15)
+
+
+def test_frequency_table_reaches_compression_and_attention(orc):
+    # m = 1: the stored entry of token t is RMSNorm(c_t) rotated by t * theta'_j
+    # with the table's frequencies.
+    B, L, d, r_dim = 1, 5, 32, 16
+    r = rng(41)
+    tab = orc.yarn_inv_freq(r_dim, 16.0, 32.0, 1.0, 64)
+    tok = bf16_bits(r.standard_normal((B, L, d)))
+    vals, _ = orc.pool(tok, np.array([L]), np.zeros(d), np.zeros(1), None, 1, 0, L, L,
+                       rope_dim=r_dim, rope_freq=tab)
+    x = orc.bf16_decode(tok)[0]
+    nrm = x / np.sqrt(np.mean(x * x, axis=1, keepdims=True) + 1e-6)
+    for t in range(L):
+        assert np.allclose(vals[0, t], _rotate(nrm[t], float(t), r_dim, theta=tab),
+                           rtol=1e-12, atol=1e-13)
+    # Attention: shifting every position leaves the output unchanged under any
+    # frequency table, and the table does change the output.
+    B, Q, H, D, L, m, W, r_dim = 1, 1, 4, 64, 64, 4, 16, 32
+    q, kv_tok, kv_c, sink = _mqa_case(B, Q, H, D, L, m, 43)
+    kv_c[..., D - r_dim:] = 0
+    tab = orc.yarn_inv_freq(r_dim, 16.0, 32.0, 1.0, 256)
+    pos = np.array([[59]])
+    sel = np.array([[[2, 6, 11]]], np.int32)
+    cnt = np.array([[3]], np.int32)
+    base, lb = orc.mqa(q, pos, kv_c, kv_tok, sink, m, W, r_dim, sel, cnt, rope_freq=tab)
+    S = 4 * 777
+    out, l2 = orc.mqa(q, pos + S, np.concatenate([np.zeros((B, 777, D), np.uint16), kv_c], 1),
+                      np.concatenate([np.zeros((B, S, D), np.uint16), kv_tok], 1), sink, m, W,
+                      r_dim, sel + 777, cnt, rope_freq=tab)
+    assert np.allclose(out, base, rtol=1e-9, atol=1e-9) and np.allclose(l2, lb, rtol=1e-9, atol=1e-9)
+    plain, _ = orc.mqa(q, pos, kv_c, kv_tok, sink, m, W, r_dim, sel, cnt)
+    assert not np.allclose(plain, base, rtol=1e-6, atol=1e-6)
