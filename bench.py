@@ -674,6 +674,83 @@ def run_prefill(args):
     print(json.dumps(line), flush=True)
 
 
+HCA_PREFILL_METRIC = "HCA prefill chunk query-tokens/s; % of BF16 tensor roofline"
+
+
+def hca_prefill_flops(w):
+    """Causal attention flops of one HCA chunk: every query against its
+    visible entries and its window (QK^T and PV, 2 flops per MAC)."""
+    import numpy as np
+    t = w.P + np.arange(w.T, dtype=np.int64)
+    nv = (t + 1) // w.m
+    win = np.minimum(t + 1, w.W)
+    return 4.0 * w.H * w.d * float((nv + win).sum())
+
+
+def run_hca_prefill(args):
+    """One HCA prefill chunk per step (hca_prefill_chunk: compression of the
+    chunk's blocks, dense attention per query, merge), B = 1.  The step's
+    split partials and output (2 x T x H x d x 2 bytes) exceed the L2, so no
+    rotation."""
+    import torch
+
+    from compressed_sparse_kv_04_b200 import binding as b
+    from compressed_sparse_kv_04_b200 import synth
+    w = configs.HCA_PREFILL
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    L_cap = w.P + w.T
+    N_cap = -(-L_cap // w.m)
+    kv_tok, _ = synth.token_streams(w, L_cap=L_cap, device=dev)
+    w_s, b_pos = synth.pool_params(w, dev)
+    qi = synth.queries(w, Q=w.T, device=dev)
+    q = qi["q"][0].contiguous()
+    p = b.params_for(w, B=1)
+    kv_c = torch.zeros(1, N_cap, w.d, dtype=torch.bfloat16, device=dev)
+    ctx = torch.full((1,), w.P, dtype=torch.int64, device=dev)
+    b.hca_compress(p, kv_tok, ctx, w_s, b_pos, None, 0, w.P // w.m, kv_c)  # the cached part
+    ws = b.workspace(p, b.OP_HCA_PREFILL, w.T, N_cap, device=dev)
+    out = torch.empty(w.T, w.H, w.d, dtype=torch.bfloat16, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    def chunk():
+        b.hca_prefill_chunk(p, w.P, w.T, kv_tok, w_s, b_pos, None, kv_c, q, qi["sink"], out,
+                            ws=ws, dev_status=status)
+
+    K, W = args.steps, args.warmup
+    with ClockSampler(0) as clocks:
+        for _ in range(W):
+            chunk()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(K):
+            chunk()
+        e1.record()
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / K
+    flops = hca_prefill_flops(w)
+    peaks = measured_peaks()
+    tf = flops / (ms * 1e-3) / 1e12
+    line = {
+        "metric": HCA_PREFILL_METRIC, "value": round(w.T / (ms * 1e-3), 1),
+        "unit": "query-tokens/s", "n_gpus": 1, "steps": K, "warmup": W,
+        "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) token streams and queries)",
+        "config": {"workload": w.name, "prior_tokens": w.P, "chunk_tokens": w.T, "heads": w.H,
+                   "head_dim": w.d, "m": w.m, "window": w.W,
+                   "l2": "no rotation: the chunk's partials and output exceed the L2"},
+        "roofline": {"bound": "tensor", "kernel": "hca_prefill_chunk (compress + attention + merge)",
+                     "achieved": round(tf, 1), "peak": round(peaks["bf16_tflops"], 1),
+                     "unit": "TFLOP/s", "frac": round(tf / peaks["bf16_tflops"], 4),
+                     "peak_source": peaks["source"], "avg_launch_ms": round(ms, 4),
+                     "algorithmic_flops": flops},
+        "gpu_launches": 3 * K, "clocks": clocks.summary(), "device_status": int(status.item()),
+    }
+    print(json.dumps(line), flush=True)
+
+
 # ------------------------------------------------------------ CPU oracle --
 class OracleStep:
     """One sequence's decode step through the fp64 oracle, as it stands:
@@ -872,11 +949,15 @@ def main(argv=None):
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
+        if configs.BY_NAME[args.workload].kind.endswith("prefill"):
+            ap.error("the reference arm times decode workloads")
         return run_reference(args)
     if args.workload == configs.TINY_CSA.name:
         ap.error("the tiny case is a parity-test case")
     if args.workload == configs.CSA_PREFILL.name:  # explicit request only; not the default line
         return run_prefill(args)
+    if args.workload == configs.HCA_PREFILL.name:
+        return run_hca_prefill(args)
     run_gpu(args)
 
 

@@ -19,12 +19,12 @@ CSA_OK = 0
 STATUS_NAMES = {0: "CSA_OK", 1: "CSA_ERR_INVALID_ARG", 2: "CSA_ERR_UNSUPPORTED_SHAPE",
                 3: "CSA_ERR_CAPACITY", 4: "CSA_ERR_WORKSPACE", 5: "CSA_ERR_CUDA",
                 6: "CSA_ERR_DEVICE_TIMEOUT", 7: "CSA_ERR_DEVICE_INDEX"}
-OP_INDEX_TOPK, OP_SPARSE_MQA, OP_DENSE_MQA, OP_PREFILL = 1, 2, 3, 4
+OP_INDEX_TOPK, OP_SPARSE_MQA, OP_DENSE_MQA, OP_PREFILL, OP_HCA_PREFILL = 1, 2, 3, 4, 5
 
 EXPORTS = ["csa_version", "csa_last_error", "csa_workspace_bytes", "hca_compress",
            "csa_compress", "lightning_index_topk", "lightning_index_scores", "topk_select",
            "sparse_mqa_decode", "dense_mqa_decode", "csa_prefill_chunk",
-           "lightning_index_topk_static", "csa_rope_yarn"]
+           "lightning_index_topk_static", "csa_rope_yarn", "hca_prefill_chunk"]
 
 
 class CsaError(RuntimeError):
@@ -78,6 +78,8 @@ def _declare(L):
                                     i64, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp, vp]
     L.lightning_index_topk_static.argtypes = [P, i32, vp, vp, vp, vp, vp, i64, vp, vp, vp, vp,
                                               vp]
+    L.hca_prefill_chunk.argtypes = [P, i64, i32, vp, i64, vp, vp, vp, vp, i64, vp, vp, vp, vp, vp,
+                                    vp, vp, sz, vp, vp]
     L.csa_rope_yarn.argtypes = [i32, C.c_double, C.c_double, C.c_double, C.c_double,
                                 C.c_double, C.POINTER(C.c_double), C.POINTER(C.c_double)]
     for name in EXPORTS[3:]:
@@ -228,3 +230,14 @@ def csa_prefill_chunk(p, P, T, kv_tok, idx_tok, w_s, b_pos, gamma, w_s_idx, b_po
         kv_c.shape[1], _ptr(q), _ptr(q_idx), _ptr(q_scale), _ptr(w), _ptr(sink), _ptr(gamma_q),
         _ptr(gamma_kv), _ptr(topk_idx), _ptr(topk_cnt), _ptr(out), _ptr(ws),
         0 if ws is None else ws.numel() * ws.element_size(), _ptr(dev_status), _stream(stream)))
+
+
+def hca_prefill_chunk(p, P, T, kv_tok, w_s, b_pos, gamma, kv_c, q, sink, out, gamma_q=None,
+                      gamma_kv=None, lse=None, ws=None, dev_status=None, stream=None):
+    """HCA prefill chunk (B = 1): compression of the chunk's blocks, then dense
+    MQA per new query.  kv_tok [1, L_cap, d]; kv_c [1, N_cap, d]; q/out [T, H, d]."""
+    _check(lib().hca_prefill_chunk(
+        C.byref(p), P, T, _ptr(kv_tok), kv_tok.shape[1], _ptr(w_s), _ptr(b_pos), _ptr(gamma),
+        _ptr(kv_c), kv_c.shape[1], _ptr(q), _ptr(sink), _ptr(gamma_q), _ptr(gamma_kv), _ptr(out),
+        _ptr(lse), _ptr(ws), 0 if ws is None else ws.numel() * ws.element_size(),
+        _ptr(dev_status), _stream(stream)))

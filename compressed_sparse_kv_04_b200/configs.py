@@ -16,7 +16,7 @@ from dataclasses import dataclass, replace
 @dataclass(frozen=True)
 class Workload:
     name: str
-    kind: str            # "csa_decode" | "hca_decode" | "csa_prefill"
+    kind: str            # "csa_decode" | "hca_decode" | "csa_prefill" | "hca_prefill"
     B: int               # sequences
     L: int               # context tokens per sequence (decode: the query is token L-1)
     d: int               # KV entry dim == head dim D
@@ -67,7 +67,13 @@ CSA_FLASH_128K = Workload("csa_flash_decode_128k_b8", "csa_decode", B=8, L=13107
                           H=64, rope_dim=64, W=128, H_I=64, D_I=128, k=512, seed=20260006,
                           yarn=YARN_V4)
 
-ALL = [TINY_CSA, CSA_128K, HCA_1M, CSA_1M, CSA_PREFILL, CSA_FLASH_128K]
+# HCA prefill: the same 4096-token chunk after 65,536 cached tokens as the CSA
+# prefill, through the HCA layer (m' = 128: 512 cached + 32 new entries).
+HCA_PREFILL = Workload("hca_prefill_4096_after_65536", "hca_prefill", B=1, L=65536 + 4096,
+                       d=512, m=128, H=128, rope_dim=64, W=128, P=65536, T=4096,
+                       seed=20260007)
+
+ALL = [TINY_CSA, CSA_128K, HCA_1M, CSA_1M, CSA_PREFILL, CSA_FLASH_128K, HCA_PREFILL]
 BY_NAME = {w.name: w for w in ALL}
 
 

@@ -182,6 +182,12 @@ size_t csa_workspace_bytes(const csa_params* p, csa_op op, int Q, int64_t N_cap)
                                       p->d) +
              512;
     }
+    case CSA_OP_HCA_PREFILL: {
+      int rows = Q;
+      return csa::mqa_workspace_bytes(rows, splits_for(p, CSA_OP_DENSE_MQA, rows, N_cap), p->H,
+                                      p->d) +
+             256;
+    }
   }
   fail(CSA_ERR_INVALID_ARG, "%s: unknown op %d", fn, (int)op);
   return 0;
@@ -591,6 +597,54 @@ csa_status csa_prefill_chunk(const csa_params* p, int64_t P, int T, const void* 
   return mqa_common(fn, p, CSA_OP_SPARSE_MQA, T, T, q, nullptr, P, kv_c, N_cap, topk_idx,
                     topk_cnt, kv_tok, L_cap, sink, gamma_q, gamma_kv, out, nullptr, rest,
                     rest_bytes, dev_status, s);
+}
+
+csa_status hca_prefill_chunk(const csa_params* p, int64_t P, int T, const void* kv_tok,
+                             int64_t L_cap, const float* w_s, const float* b_pos,
+                             const float* gamma, void* kv_c, int64_t N_cap, const void* q,
+                             const float* sink, const float* gamma_q, const float* gamma_kv,
+                             void* out, float* lse, void* ws, size_t ws_bytes,
+                             int32_t* dev_status, void* stream) {
+  const char* fn = "hca_prefill_chunk";
+  csa_status st = check_common(fn, p);
+  if (st != CSA_OK) return st;
+  if (p->B != 1) return fail(CSA_ERR_UNSUPPORTED_SHAPE, "%s: B=%d (supported: 1)", fn, p->B);
+  st = check_attention(fn, p);
+  if (st != CSA_OK) return st;
+  if (P < 0 || T < 1 || P % p->m != 0)
+    return fail(CSA_ERR_INVALID_ARG, "%s: P=%lld must be a multiple of m=%d, T=%d >= 1", fn,
+                (long long)P, p->m, T);
+  if (T > 65535) return fail(CSA_ERR_UNSUPPORTED_SHAPE, "%s: T=%d (supported: <= 65535)", fn, T);
+  if (P + T > L_cap)
+    return fail(CSA_ERR_CAPACITY, "%s: P+T=%lld exceeds L_cap=%lld", fn, (long long)(P + T),
+                (long long)L_cap);
+  if (L_cap > ((int64_t)1 << 31) - 1 || N_cap > ((int64_t)1 << 31) - 1)
+    return fail(CSA_ERR_UNSUPPORTED_SHAPE, "%s: N_cap and L_cap must fit in int32 rows", fn);
+  const int64_t nblk_total = (P + T + p->m - 1) / p->m;
+  if (nblk_total > N_cap)
+    return fail(CSA_ERR_CAPACITY, "%s: %lld compressed entries exceed N_cap=%lld", fn,
+                (long long)nblk_total, (long long)N_cap);
+  REQ_PTR(q);
+  REQ_PTR4(sink);
+  OPT_PTR4(gamma_q);
+  OPT_PTR4(gamma_kv);
+  REQ_PTR(out);
+  OPT_PTR4(lse);
+  size_t need = csa_workspace_bytes(p, CSA_OP_HCA_PREFILL, T, N_cap);
+  if (!ws || ws_bytes < need)
+    return fail(CSA_ERR_WORKSPACE, "%s: workspace of %zu bytes needed, %zu given", fn, need,
+                ws ? ws_bytes : (size_t)0);
+  if (!aligned16(ws)) return fail(CSA_ERR_INVALID_ARG, "%s: ws is not 16-byte aligned", fn);
+  // 1. Compress the blocks the new tokens touch (ctx_len = P+T for all).
+  const int64_t b0 = P / p->m;
+  st = compress_common(fn, p, kv_tok, L_cap, nullptr, P + T, w_s, b_pos, gamma, b0,
+                       nblk_total - b0, kv_c, N_cap, nullptr, nullptr, nullptr, nullptr, nullptr,
+                       dev_status, stream);
+  if (st != CSA_OK) return st;
+  // 2. Dense MQA per query over its visible entries and its causal window.
+  return mqa_common(fn, p, CSA_OP_DENSE_MQA, T, T, q, nullptr, P, kv_c, N_cap, nullptr, nullptr,
+                    kv_tok, L_cap, sink, gamma_q, gamma_kv, out, lse, ws, ws_bytes, dev_status,
+                    static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

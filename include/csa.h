@@ -83,7 +83,8 @@ typedef enum {
   CSA_OP_INDEX_TOPK = 1,
   CSA_OP_SPARSE_MQA = 2,
   CSA_OP_DENSE_MQA = 3,
-  CSA_OP_PREFILL = 4
+  CSA_OP_PREFILL = 4,
+  CSA_OP_HCA_PREFILL = 5
 } csa_op;
 
 /* Library version (major*100 + minor). */
@@ -120,7 +121,8 @@ csa_status csa_rope_yarn(int rope_dim, double base, double factor, double beta_f
                          double* logit_gain);
 
 /* Workspace bytes that `op` needs for these params.
- *   Q     queries per sequence (1 for decode; T for CSA_OP_PREFILL),
+ *   Q     queries per sequence (1 for decode; T for CSA_OP_PREFILL and
+ *         CSA_OP_HCA_PREFILL),
  *   N_cap capacity of the compressed cache (entries per sequence).
  * Returns 0 for invalid arguments (and sets csa_last_error). */
 size_t csa_workspace_bytes(const csa_params* p, csa_op op, int Q, int64_t N_cap);
@@ -316,6 +318,33 @@ csa_status csa_prefill_chunk(const csa_params* p, int64_t P, int T, const void* 
                              const float* sink, const float* gamma_q, const float* gamma_kv,
                              int32_t* topk_idx, int32_t* topk_cnt, void* out, void* ws,
                              size_t ws_bytes, int32_t* dev_status, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * HCA prefill chunk (B = 1; [P2] HCA paragraph: dense attention over every
+ * compressed entry, m' = 128, no overlap; [P5] "Hybrid attention": HCA
+ * bullet and the sliding-window branch).  T new tokens at positions
+ * P .. P+T-1 whose KV rows (kv_tok) the caller has already written.  Runs,
+ * in order: hca_compress of blocks P/m .. ceil((P+T)/m)-1 with ctx_len = P+T
+ * (a partial last block is pooled over its present tokens and stays
+ * invisible), then for every new query t the dense MQA over its visible
+ * entries 0 .. floor((t+1)/m)-1 and its window [max(0, t-W+1), t], one joint
+ * softmax with the sink, inverse RoPE on the output.  P must be a multiple
+ * of m; entries before P/m must already be in kv_c.
+ *   kv_tok [1, L_cap, d] bf16; w_s [d], b_pos [m], gamma [d] or NULL fp32;
+ *   kv_c [1, N_cap, d] bf16 (blocks P/m .. written); q [T, H, d] bf16;
+ *   sink [H] fp32; gamma_q, gamma_kv [d] or NULL; out [T, H, d] bf16
+ *   (written); lse [T, H] fp32 or NULL.
+ * Workspace: csa_workspace_bytes(p, CSA_OP_HCA_PREFILL, T, N_cap).
+ * Errors: CSA_ERR_UNSUPPORTED_SHAPE for B != 1 or T > 65535;
+ *         CSA_ERR_INVALID_ARG when P is not a multiple of m or T < 1;
+ *         CSA_ERR_CAPACITY when P+T > L_cap or ceil((P+T)/m) > N_cap.
+ * ------------------------------------------------------------------------- */
+csa_status hca_prefill_chunk(const csa_params* p, int64_t P, int T, const void* kv_tok,
+                             int64_t L_cap, const float* w_s, const float* b_pos,
+                             const float* gamma, void* kv_c, int64_t N_cap, const void* q,
+                             const float* sink, const float* gamma_q, const float* gamma_kv,
+                             void* out, float* lse, void* ws, size_t ws_bytes,
+                             int32_t* dev_status, void* stream);
 
 #ifdef __cplusplus
 }

@@ -105,6 +105,21 @@ def test_prefill_argument_checks(L):
     assert st == 1  # P not a multiple of m
 
 
+def test_hca_prefill_argument_checks(L):
+    def call(p, P_, T, L_cap=1 << 20, N_cap=1 << 13):
+        return L.hca_prefill_chunk(C.byref(p), P_, T, None, L_cap, None, None, None, None, N_cap,
+                                   None, None, None, None, None, None, None, 0, None, None)
+    assert call(P(B=2, m=128), 0, 4) == 2          # B must be 1
+    p = P(B=1, m=128)
+    assert call(p, 3, 4) == 1                      # P not a multiple of m
+    assert call(p, 0, 0) == 1                      # T >= 1
+    assert call(p, 0, 70000) == 2                  # T <= 65535
+    assert call(p, 128, 10, L_cap=100) == 3        # P+T > L_cap
+    assert call(p, 0, 300, L_cap=1024, N_cap=2) == 3  # ceil(300/128) > N_cap
+    assert call(p, 0, 300, L_cap=1024, N_cap=3) == 1  # q is NULL
+    assert L.csa_workspace_bytes(C.byref(p), 5, 4096, 544) > 0
+
+
 def test_workspace_sizes_are_monotone(L):
     p = P(B=8)
     a = L.csa_workspace_bytes(C.byref(p), 1, 1, 32768)

@@ -140,3 +140,74 @@ def test_prefill_full_shape_sampled(orc):
     w = configs.CSA_PREFILL
     r = run_prefill(orc, w, w.P, w.T)
     check_prefill(orc, w, r, _sample_rows(w.T, w.m, 6, 7))
+
+
+# ------------------------------------------------------------ HCA prefill --
+def run_hca_prefill(orc, w, P, T, gamma=False):
+    m = w.m
+    L_cap = P + T
+    N_cap = math.ceil(L_cap / m)
+    b0 = P // m
+    kv_tok, _ = synth.token_streams(w, L_cap=L_cap)
+    w_s, b_pos = synth.pool_params(w)
+    qi = synth.queries(w, Q=T)
+    kv_bits = bits16(kv_tok)
+    g = synth.gains(w.d, w.seed) if gamma else None
+    # Cached blocks 0 .. b0-1 from the oracle.
+    kv_c0, _, _ = orc.compress_kv(kv_bits, [P], f32(w_s), f32(b_pos), None if g is None else f32(g),
+                                  m, 0, b0, N_cap, rope_dim=w.rope_dim)
+    kv_c = torch.from_numpy(kv_c0.view(np.int16)).view(torch.bfloat16).to(DEV)
+    p = binding.params_for(w, B=1)
+    ws = binding.workspace(p, binding.OP_HCA_PREFILL, T, N_cap)
+    out = torch.full((T, w.H, w.D), float("nan"), dtype=torch.bfloat16, device=DEV)
+    lse = torch.full((T, w.H), float("nan"), dtype=torch.float32, device=DEV)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    binding.hca_prefill_chunk(p, P, T, kv_tok.to(DEV), w_s.to(DEV), b_pos.to(DEV),
+                              None if g is None else g.to(DEV), kv_c, qi["q"][0].contiguous().to(DEV),
+                              qi["sink"].to(DEV), out, lse=lse, ws=ws, dev_status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    return dict(P=P, T=T, N_cap=N_cap, b0=b0, kv_bits=kv_bits, w_s=w_s, b_pos=b_pos, g=g, qi=qi,
+                kv_c0=kv_c0, kv_c=bits16(kv_c), out=f32(out).astype(np.float64),
+                lse=f32(lse).astype(np.float64))
+
+
+def check_hca_prefill(orc, w, r, rows):
+    m, P, T, N_cap, b0 = w.m, r["P"], r["T"], r["N_cap"], r["b0"]
+    g = None if r["g"] is None else f32(r["g"])
+    # 1. Compression: cached rows untouched, new rows (partial last block
+    # included) against the oracle.
+    assert np.array_equal(r["kv_c"][:, :b0], r["kv_c0"][:, :b0])
+    _, _, vals = orc.compress_kv(r["kv_bits"], [P + T], f32(r["w_s"]), f32(r["b_pos"]), g, m, b0,
+                                 N_cap - b0, N_cap, rope_dim=w.rope_dim)
+    assert_bf16_storage_close(r["kv_c"][:, b0:], vals[:, b0:], "new HCA entries")
+    # 2. Dense attention of the sampled rows with the GPU's entries.
+    pos = (P + np.arange(T)).reshape(1, T)
+    ref, rlse = orc.mqa(bits16(r["qi"]["q"])[:, rows], pos[:, rows], r["kv_c"], r["kv_bits"],
+                        f32(r["qi"]["sink"]), m, w.W, w.rope_dim)
+    got = r["out"][rows]
+    assert np.isfinite(got).all()
+    assert_attention_close(got, ref[0], "HCA prefill attention")
+    gl, rl = r["lse"][rows], rlse[0]
+    assert np.allclose(gl, rl, rtol=0, atol=2e-2), np.abs(gl - rl).max()
+
+
+@pytest.mark.parametrize("P,T,gamma", [(128 * 10, 300, False), (0, 260, True), (128 * 3, 128, False)])
+def test_hca_prefill_small(orc, P, T, gamma):
+    """Ragged chunks through the HCA layer: a partial last block, a chunk that
+    starts the sequence (queries before the first complete block see only
+    their window), one that ends on a block boundary; with and without a gain."""
+    w = configs.scaled(configs.HCA_PREFILL, L=P + T, P=P, T=T)
+    r = run_hca_prefill(orc, w, P, T, gamma)
+    rows = _sample_rows(T, w.m, 24, P + T)
+    rows = np.union1d(rows, [t for t in (126, 127, 128, 255, 256) if t < T])
+    check_hca_prefill(orc, w, r, rows)
+
+
+@pytest.mark.slow
+def test_hca_prefill_full_shape_sampled(orc):
+    """The 4096-token chunk after 65,536 cached tokens: the 32 new entries and
+    sampled rows' attention."""
+    w = configs.HCA_PREFILL
+    r = run_hca_prefill(orc, w, w.P, w.T)
+    check_hca_prefill(orc, w, r, _sample_rows(w.T, w.m, 8, 11))
