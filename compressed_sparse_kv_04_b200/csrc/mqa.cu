@@ -759,120 +759,129 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-// Merge the split partials of one (row, head), fold in the sink, normalise,
-// apply the inverse rotation, store bf16 (and the log-sum-exp).  Warp 0
-// turns the S (max, sum) pairs into one weight per split; then thread t
-// accumulates dims [4t, 4t+4) over the splits with independent 16-byte
-// loads.
-__global__ void __launch_bounds__(128) mqa_combine_kernel(const Params p, int D,
+// Merge the split partials of one (row, head) per warp: fold in the sink,
+// normalise, apply the inverse rotation, store bf16 (and the log-sum-exp).
+// Lane l owns dims [l*VPL, (l+1)*VPL) (VPL = D/32), so the output row leaves
+// as one coalesced 32-lane store and the rotated pairs (d, d + R/2) sit in
+// lanes l and l ^ (R/2/VPL).  The S (max, sum) pairs become one weight per
+// split (per-warp shared memory); the partials are read G splits at a time
+// with the next group's loads in flight, the first group before the weights
+// are known.  Four warps per CTA.
+template <int D, int R, int G>
+__global__ void __launch_bounds__(128) mqa_combine_kernel(const Params p, int rows,
                                                           const float* __restrict__ sink,
                                                           __nv_bfloat16* __restrict__ out,
                                                           float* __restrict__ lse) {
-  extern __shared__ float so[];  // D floats, then one weight per split
+  constexpr int VPL = D / 32;     // dims per lane: 16 (D = 512) or 4 (D = 128)
+  constexpr int NW = VPL / 2;     // 32-bit words (fp16 pairs) per lane and split
+  static_assert(VPL == 16 || VPL == 4, "D must be 512 or 128");
+  extern __shared__ float wsm[];  // [4 warps][S] split weights
   pdl_trigger();
   pdl_wait();  // the partials come from the attention kernel
-  float* wsplit = so + D;
-  __shared__ float s_ml[2];
-  const int row = blockIdx.x, h = blockIdx.y;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t gw = (int64_t)blockIdx.x * 4 + warp;
+  if (gw >= (int64_t)rows * p.H) return;
+  const int row = (int)(gw / p.H), h = (int)(gw % p.H);
   const int S = p.splits;
+  float* wsplit = wsm + warp * S;
   const float* ml = p.part_ml + (int64_t)row * S * 2 * p.H;
+  const __half* src = p.part_o + ((int64_t)row * S * p.H + h) * D + lane * VPL;
+  const int64_t stride = (int64_t)p.H * D;
+  auto load = [&](int s, uint32_t (&v)[NW]) {
+    const __half* a = src + (int64_t)s * stride;
+    if constexpr (VPL == 16) {
+      *reinterpret_cast<uint4*>(&v[0]) = __ldg(reinterpret_cast<const uint4*>(a));
+      *reinterpret_cast<uint4*>(&v[4]) = __ldg(reinterpret_cast<const uint4*>(a) + 1);
+    } else {
+      *reinterpret_cast<uint2*>(&v[0]) = __ldg(reinterpret_cast<const uint2*>(a));
+    }
+  };
+  uint32_t cur[G][NW], nxt[G][NW];
+#pragma unroll
+  for (int u = 0; u < G; ++u)
+    if (u < S) load(u, cur[u]);
   const float LOG2E = 1.4426950408889634f;
   const float z = sink[h];
   const float z2 = z * LOG2E;  // log2 domain
-  __nv_bfloat16* o = out + ((int64_t)row * p.H + h) * D;
-  // Thread t merges dims [4t, 4t+4) (D <= 512).  Its first group of
-  // partials is requested before the weights are known.
-  const int d4 = threadIdx.x;
-  const bool dims = d4 < D / 4;
-  const __half* src = p.part_o + ((int64_t)row * S * p.H + h) * D + 4 * d4;
-  const int64_t stride = (int64_t)p.H * D;
-  auto load4 = [&](int s0, uint2 (&v)[4]) {
+  float M = z2;
+  for (int s = lane; s < S; s += 32) M = fmaxf(M, ml[(int64_t)s * 2 * p.H + h]);
+  M = warp_max(M);
+  const bool zero = z == INFINITY || M == -INFINITY;  // +inf sink, or nothing to attend
+  float L = 0.f;
+  if (!zero) {
+    for (int s = lane; s < S; s += 32) {
+      const float ms = ml[(int64_t)s * 2 * p.H + h];
+      const float w = ms == -INFINITY ? 0.f : ml[(int64_t)s * 2 * p.H + p.H + h] * exp2f(ms - M);
+      wsplit[s] = w;  // the split's stored output is O / l
+      L += w;
+    }
+    L = warp_sum(L);
+    if (z2 != -INFINITY) L += exp2f(z2 - M);
+  }
+  __syncwarp();
+  __nv_bfloat16* o = out + ((int64_t)row * p.H + h) * D + lane * VPL;
+  float acc[VPL];
 #pragma unroll
-    for (int u = 0; u < 4; ++u)
-      v[u] = (dims && s0 + u < S) ? __ldg(reinterpret_cast<const uint2*>(src + (s0 + u) * stride))
-                                  : make_uint2(0u, 0u);
-  };
-  uint2 cur[4], nxt[4];
-  load4(0, cur);
-  if (threadIdx.x < 32) {
-    const int lane = threadIdx.x;
-    float M = z2;
-    for (int s = lane; s < S; s += 32) M = fmaxf(M, ml[(int64_t)s * 2 * p.H + h]);
-    M = warp_max(M);
-    float L = 0.f;
-    if (M != -INFINITY && z != INFINITY) {
-      for (int s = lane; s < S; s += 32) {
-        const float ms = ml[(int64_t)s * 2 * p.H + h];
-        const float w = ms == -INFINITY ? 0.f : ml[(int64_t)s * 2 * p.H + p.H + h] * exp2f(ms - M);
-        wsplit[s] = w;  // the split's stored output is O / l
-        L += w;
+  for (int e = 0; e < VPL; ++e) acc[e] = 0.f;
+  if (!zero) {
+    for (int s0 = 0; s0 < S; s0 += G) {
+      if (s0 + G < S) {
+#pragma unroll
+        for (int u = 0; u < G; ++u)
+          if (s0 + G + u < S) load(s0 + G + u, nxt[u]);
       }
-      L = warp_sum(L);
-      if (z2 != -INFINITY) L += exp2f(z2 - M);
-    }
-    if (lane == 0) {
-      s_ml[0] = M;
-      s_ml[1] = L;
-    }
-  }
-  __syncthreads();
-  const float M = s_ml[0], L = s_ml[1];
-  if (z == INFINITY || M == -INFINITY) {  // +inf sink, or nothing to attend
-    for (int d = threadIdx.x; d < D; d += blockDim.x) o[d] = __float2bfloat16_rn(0.f);
-    if (lse && threadIdx.x == 0)
-      lse[(int64_t)row * p.H + h] = z == INFINITY ? INFINITY : -INFINITY;
-    return;
-  }
-  const float invL = 1.0f / L;
-  if (dims) {
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    auto add = [&](uint2 u, float w) {
-      if (w == 0.f) return;  // empty split: its partial was never written
-      const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&u.x));
-      const float2 c = __half22float2(*reinterpret_cast<const __half2*>(&u.y));
-      acc.x = fmaf(a.x, w, acc.x);
-      acc.y = fmaf(a.y, w, acc.y);
-      acc.z = fmaf(c.x, w, acc.z);
-      acc.w = fmaf(c.y, w, acc.w);
-    };
-    // Groups of 4 splits, the next group's loads in flight during this
-    // group's use.
-    for (int s0 = 0; s0 < S; s0 += 4) {
-      if (s0 + 4 < S) load4(s0 + 4, nxt);
 #pragma unroll
-      for (int u = 0; u < 4; ++u)
-        if (s0 + u < S) add(cur[u], wsplit[s0 + u]);
+      for (int u = 0; u < G; ++u) {
+        if (s0 + u >= S) break;
+        const float w = wsplit[s0 + u];
+        if (w == 0.f) continue;  // empty split: its partial was never written
 #pragma unroll
-      for (int u = 0; u < 4; ++u) cur[u] = nxt[u];
-    }
-    so[4 * d4] = acc.x * invL;
-    so[4 * d4 + 1] = acc.y * invL;
-    so[4 * d4 + 2] = acc.z * invL;
-    so[4 * d4 + 3] = acc.w * invL;
-  }
-  __syncthreads();
-  const int64_t pos = row_pos(p, row);
-  const int half = p.R / 2, d0 = D - p.R;
-  for (int d2 = threadIdx.x; d2 < D / 2; d2 += blockDim.x) {
-    float v2[2];
-#pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      const int d = 2 * d2 + e;
-      float v = so[d];
-      if (p.R > 0 && d >= d0) {
-        const int j = (d - d0) % half;
-        float sn, cs;
-        sincos_reduced((double)pos * p.inv_freq[j], &sn, &cs);
-        if (d - d0 < half)
-          v = so[d] * cs + so[d + half] * sn;  // rotation by -angle
-        else
-          v = so[d] * cs - so[d - half] * sn;
+        for (int i = 0; i < NW; ++i) {
+          const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&cur[u][i]));
+          acc[2 * i] = fmaf(f.x, w, acc[2 * i]);
+          acc[2 * i + 1] = fmaf(f.y, w, acc[2 * i + 1]);
+        }
       }
-      v2[e] = v;
+#pragma unroll
+      for (int u = 0; u < G; ++u)
+#pragma unroll
+        for (int i = 0; i < NW; ++i) cur[u][i] = nxt[u][i];
     }
-    reinterpret_cast<uint32_t*>(o)[d2] = pack_bf16(v2[0], v2[1]);
+    const float invL = 1.0f / L;
+#pragma unroll
+    for (int e = 0; e < VPL; ++e) acc[e] *= invL;
+    if constexpr (R > 0) {
+      // Rotation by -pos: pair j of the last R dims is (d0 + j, d0 + j + R/2).
+      constexpr int K = R / 2 / VPL;  // lanes per rotated half
+      constexpr int L0 = 32 - 2 * K;  // first lane holding rotated dims
+      static_assert(K >= 1 && (K & (K - 1)) == 0, "rotated halves must span whole lanes");
+      const int64_t pos = row_pos(p, row);
+      float sn = 0.f, cs = 1.f;
+      if (lane < R / 2) sincos_reduced((double)pos * p.inv_freq[lane], &sn, &cs);
+      const bool rot = lane >= L0;
+      const bool first = rot && lane - L0 < K;
+      const int jb = rot ? ((lane - L0) % K) * VPL : 0;
+#pragma unroll
+      for (int e = 0; e < VPL; ++e) {
+        const float c = __shfl_sync(0xffffffffu, cs, jb + e);
+        const float sj = __shfl_sync(0xffffffffu, sn, jb + e);
+        const float other = __shfl_xor_sync(0xffffffffu, acc[e], K);
+        if (rot) acc[e] = first ? acc[e] * c + other * sj : acc[e] * c - other * sj;
+      }
+    }
   }
-  if (lse && threadIdx.x == 0) lse[(int64_t)row * p.H + h] = (M + log2f(L)) / LOG2E;
+  uint32_t packed[NW];
+#pragma unroll
+  for (int i = 0; i < NW; ++i) packed[i] = pack_bf16(acc[2 * i], acc[2 * i + 1]);
+  if constexpr (VPL == 16) {
+    reinterpret_cast<uint4*>(o)[0] = *reinterpret_cast<const uint4*>(&packed[0]);
+    reinterpret_cast<uint4*>(o)[1] = *reinterpret_cast<const uint4*>(&packed[4]);
+  } else {
+    *reinterpret_cast<uint2*>(o) = *reinterpret_cast<const uint2*>(&packed[0]);
+  }
+  if (lse && lane == 0)
+    lse[(int64_t)row * p.H + h] =
+        zero ? (z == INFINITY ? INFINITY : -INFINITY) : (M + log2f(L)) / LOG2E;
 }
 
 template <int D, int R>
@@ -926,8 +935,10 @@ cudaError_t launch_impl(const MqaLaunch& a, cudaStream_t stream) {
   dim3 grid(cps * a.splits, rows, 1);
   e = launch_pdl(kern, grid, dim3(kThreads), smem, stream, 0, map_q, box_c, box_t, p);
   if (e != cudaSuccess) return e;
-  return launch_pdl(mqa_combine_kernel, dim3(rows, a.H), dim3(128),
-                    (size_t)(D + a.splits) * sizeof(float), stream, 0, p, D, a.sink,
+  const unsigned nblk = (unsigned)(((int64_t)rows * a.H + 3) / 4);
+  const size_t wsm = (size_t)4 * a.splits * sizeof(float);
+  auto merge = a.splits == 1 ? mqa_combine_kernel<D, R, 1> : mqa_combine_kernel<D, R, 4>;
+  return launch_pdl(merge, dim3(nblk), dim3(128), wsm, stream, 0, p, rows, a.sink,
                     reinterpret_cast<__nv_bfloat16*>(a.out), a.lse);
 }
 
