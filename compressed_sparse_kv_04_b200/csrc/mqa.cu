@@ -108,6 +108,13 @@ struct Params {
   __half* part_o;  // [rows, S, H, D]: the split's output divided by its sum
   float* part_ml;
   int32_t* status;
+  // One split per row: the attention kernel finishes the rows itself (sink,
+  // normalisation, inverse rotation, bf16 output and log-sum-exp) and no
+  // merge runs.
+  int fused;
+  const float* sink;
+  __nv_bfloat16* out;
+  float* lse;
   double inv_freq[64];
 };
 
@@ -702,9 +709,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive(&pfull[a]);
     }
     // Epilogue: this CTA's O rows and running max / sum (an empty split
-    // leaves an empty partial).
+    // leaves an empty partial).  With one split (p.fused) the rows are
+    // finished here: out = RoPE^-1(O * 2^(m - M) / L) with M = max(m, z) and
+    // L = l * 2^(m - M) + 2^(z - M) (log2 domain; z the head's sink).
+    const float LOG2E = 1.4426950408889634f;
+    const float zs = (p.fused && head_ok) ? p.sink[hg] : 0.f;
+    const float z2 = zs * LOG2E;
     if (ntile <= 0) {
-      if (head_ok && hf == 0) {
+      if (p.fused) {
+        // Nothing to attend: a zero row; the log-sum-exp is the sink's.
+        if (head_ok) {
+          uint4* o4 = reinterpret_cast<uint4*>(p.out + ((int64_t)row * p.H + hg) * D + hf * (D / 2));
+          for (int i = 0; i < D / 16; ++i) o4[i] = make_uint4(0u, 0u, 0u, 0u);
+          if (p.lse && hf == 0) p.lse[(int64_t)row * p.H + hg] = zs;
+        }
+      } else if (head_ok && hf == 0) {
         pml[hg] = -INFINITY;
         pml[p.H + hg] = 0.f;
       }
@@ -714,25 +733,74 @@ __global__ void __launch_bounds__(kThreads, 1)
       // O / l rows (fp16: |O / l| is at most the largest |v|) go through
       // shared memory (the stages are free now: every MMA has completed)
       // and leave as one bulk copy per half row.
-      __half* po = p.part_o + (((int64_t)row * p.splits + split) * p.H + (head_ok ? hg : 0)) * D +
-                   hf * (D / 2);
+      void* po = p.fused
+                     ? static_cast<void*>(p.out + ((int64_t)row * p.H + (head_ok ? hg : 0)) * D +
+                                          hf * (D / 2))
+                     : static_cast<void*>(p.part_o + (((int64_t)row * p.splits + split) * p.H +
+                                                      (head_ok ? hg : 0)) * D + hf * (D / 2));
       constexpr int kORow = D * 2 + 16;  // padded row: spreads the banks
-      __half* ob = reinterpret_cast<__half*>(stages + hl * kORow) + hf * (D / 2);
-      const float inv_l = l_run > 0.f ? 1.0f / l_run : 0.f;
+      uint8_t* ob = stages + hl * kORow + hf * D;
+      float scale = l_run > 0.f ? 1.0f / l_run : 0.f;
+      float M = m_run, L = l_run;
+      bool zero = false;
+      float ang_s = 0.f, ang_c = 1.f;
+      if (p.fused) {
+        M = fmaxf(m_run, z2);
+        zero = zs == INFINITY || M == -INFINITY;
+        if (!zero) {
+          const float wm = m_run == -INFINITY ? 0.f : exp2f(m_run - M);
+          L = l_run * wm + (z2 == -INFINITY ? 0.f : exp2f(z2 - M));
+          scale = wm / L;
+        } else {
+          scale = 0.f;
+        }
+        if constexpr (R > 0) {
+          if (lane < R / 2) sincos_reduced((double)pos * p.inv_freq[lane], &ang_s, &ang_c);
+        }
+      }
 #pragma unroll 1
       for (int c = 0; c < D / 2; c += 64) {  // two 32-column loads per wait
         uint32_t v[64];
         tmem_ld_16x32bx2_x32<D / 2>(t_o + lq + c, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
         tmem_ld_16x32bx2_x32<D / 2>(t_o + lq + c + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
         tmem_wait_ld();
+        if (p.fused) {
+          if constexpr (R > 0) {
+            // The rotated dims (the last R) are the end of this chunk in
+            // half 1: pair j is (v[64-R+j], v[64-R/2+j]); rotation by -pos.
+            if (c == D / 2 - 64) {
 #pragma unroll
-        for (int j = 0; j < 64; j += 8) {
-          uint4 u;
-          u.x = h2_bits(__floats2half2_rn(__uint_as_float(v[j]) * inv_l, __uint_as_float(v[j + 1]) * inv_l));
-          u.y = h2_bits(__floats2half2_rn(__uint_as_float(v[j + 2]) * inv_l, __uint_as_float(v[j + 3]) * inv_l));
-          u.z = h2_bits(__floats2half2_rn(__uint_as_float(v[j + 4]) * inv_l, __uint_as_float(v[j + 5]) * inv_l));
-          u.w = h2_bits(__floats2half2_rn(__uint_as_float(v[j + 6]) * inv_l, __uint_as_float(v[j + 7]) * inv_l));
-          *reinterpret_cast<uint4*>(ob + c + j) = u;
+              for (int j = 0; j < R / 2; ++j) {
+                const float cs = __shfl_sync(0xffffffffu, ang_c, j);
+                const float sn = __shfl_sync(0xffffffffu, ang_s, j);
+                if (hf == 1) {
+                  const float x1 = __uint_as_float(v[64 - R + j]);
+                  const float x2 = __uint_as_float(v[64 - R / 2 + j]);
+                  v[64 - R + j] = __float_as_uint(x1 * cs + x2 * sn);
+                  v[64 - R / 2 + j] = __float_as_uint(x2 * cs - x1 * sn);
+                }
+              }
+            }
+          }
+#pragma unroll
+          for (int j = 0; j < 64; j += 8) {
+            uint4 u;
+            u.x = pack_bf16(__uint_as_float(v[j]) * scale, __uint_as_float(v[j + 1]) * scale);
+            u.y = pack_bf16(__uint_as_float(v[j + 2]) * scale, __uint_as_float(v[j + 3]) * scale);
+            u.z = pack_bf16(__uint_as_float(v[j + 4]) * scale, __uint_as_float(v[j + 5]) * scale);
+            u.w = pack_bf16(__uint_as_float(v[j + 6]) * scale, __uint_as_float(v[j + 7]) * scale);
+            *reinterpret_cast<uint4*>(ob + 2 * (c + j)) = u;
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < 64; j += 8) {
+            uint4 u;
+            u.x = h2_bits(__floats2half2_rn(__uint_as_float(v[j]) * scale, __uint_as_float(v[j + 1]) * scale));
+            u.y = h2_bits(__floats2half2_rn(__uint_as_float(v[j + 2]) * scale, __uint_as_float(v[j + 3]) * scale));
+            u.z = h2_bits(__floats2half2_rn(__uint_as_float(v[j + 4]) * scale, __uint_as_float(v[j + 5]) * scale));
+            u.w = h2_bits(__floats2half2_rn(__uint_as_float(v[j + 6]) * scale, __uint_as_float(v[j + 7]) * scale));
+            *reinterpret_cast<uint4*>(ob + 2 * (c + j)) = u;
+          }
         }
       }
       if (head_ok) {
@@ -742,8 +810,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         bulk_wait_read();  // shared memory may be released; the kernel end publishes the data
       }
       if (head_ok && hf == 0) {
-        pml[hg] = m_run;  // log2 domain
-        pml[p.H + hg] = l_run;
+        if (p.fused) {
+          if (p.lse)
+            p.lse[(int64_t)row * p.H + hg] =
+                zero ? (zs == INFINITY ? INFINITY : -INFINITY) : (M + log2f(L)) / LOG2E;
+        } else {
+          pml[hg] = m_run;  // log2 domain
+          pml[p.H + hg] = l_run;
+        }
       }
     }
   }
@@ -910,6 +984,10 @@ cudaError_t launch_impl(const MqaLaunch& a, cudaStream_t stream) {
   p.part_o = reinterpret_cast<__half*>(a.part_o);
   p.part_ml = a.part_ml;
   p.status = a.status;
+  p.fused = a.splits == 1 ? 1 : 0;
+  p.sink = a.sink;
+  p.out = reinterpret_cast<__nv_bfloat16*>(a.out);
+  p.lse = a.lse;
   for (int j = 0; j < 64; ++j) p.inv_freq[j] = a.inv_freq[j];
   const int rows = a.B * a.Q;
   const int cps = a.H > HC ? 2 : 1;  // CTAs per (row, split)
@@ -935,9 +1013,10 @@ cudaError_t launch_impl(const MqaLaunch& a, cudaStream_t stream) {
   dim3 grid(cps * a.splits, rows, 1);
   e = launch_pdl(kern, grid, dim3(kThreads), smem, stream, 0, map_q, box_c, box_t, p);
   if (e != cudaSuccess) return e;
+  if (p.fused) return cudaSuccess;  // the attention kernel finished the rows
   const unsigned nblk = (unsigned)(((int64_t)rows * a.H + 3) / 4);
   const size_t wsm = (size_t)4 * a.splits * sizeof(float);
-  auto merge = a.splits == 1 ? mqa_combine_kernel<D, R, 1> : mqa_combine_kernel<D, R, 4>;
+  auto merge = mqa_combine_kernel<D, R, 4>;
   return launch_pdl(merge, dim3(nblk), dim3(128), wsm, stream, 0, p, rows, a.sink,
                     reinterpret_cast<__nv_bfloat16*>(a.out), a.lse);
 }

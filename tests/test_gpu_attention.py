@@ -249,3 +249,35 @@ def test_garbage_workspace_and_unwritten_cache_rows(orc, dense):
     assert np.isfinite(got).all()
     ref, _ = oracle_attention(orc, w, q, pos, kv_c, kv_tok, sink, sel, cnt)
     assert_attention_close(got, ref, "garbage workspace")
+
+
+@pytest.mark.parametrize("dense", [False, True])
+def test_one_split_rows_finish_in_the_attention_kernel(orc, dense):
+    """80 sequences give one split per row, so the attention kernel itself
+    folds in the sink, normalises, inverse-rotates and writes bf16 (no merge
+    launch).  Sinks include +inf and -inf; some rows see no complete block."""
+    w = configs.scaled(configs.CSA_128K, B=80, k=64)
+    B, N_cap, L_cap = 80, 200, 800
+    kv_c, kv_tok = random_cache(w, B, N_cap, L_cap, 90 + dense)
+    q = synth.normal_bf16((B, w.H, w.D), 91, "q", DEV)
+    sink = synth.normal_f32((w.H,), 92, "sink", 1.0, DEV)
+    sink[3], sink[5] = float("inf"), float("-inf")
+    rng = np.random.default_rng(93)
+    pos = rng.integers(0, L_cap, B)
+    pos[:3] = [0, 2, L_cap - 1]
+    n_vis = [min((int(t) + 1) // w.m, N_cap) for t in pos]
+    sel, cnt = (None, None) if dense else random_selection(B, w.k, n_vis, 94)
+    check(orc, w, q, pos.tolist(), kv_c, kv_tok, sink, sel, cnt, what=f"one split, dense={dense}")
+
+
+def test_one_split_rows_with_nothing_to_attend(orc):
+    """No window and positions before the first complete block: an empty KV
+    set, a zero output, and the sink's own log-sum-exp (one split per row)."""
+    w = configs.scaled(configs.HCA_1M, B=80, W=0)
+    B, N_cap, L_cap = 80, 8, 1024
+    kv_c, kv_tok = random_cache(w, B, N_cap, L_cap, 95)
+    q = synth.normal_bf16((B, w.H, w.D), 96, "q", DEV)
+    sink = synth.normal_f32((w.H,), 97, "sink", 1.0, DEV)
+    sink[7], sink[9] = float("inf"), float("-inf")
+    pos = [t % 128 if t % 3 else 128 * (1 + t % 7) + 5 for t in range(B)]
+    check(orc, w, q, pos, kv_c, kv_tok, sink, what="one split, empty KV sets")
