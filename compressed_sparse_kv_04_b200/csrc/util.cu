@@ -1,4 +1,5 @@
 // Host utilities shared by the launchers: SM count and TMA tensor maps.
+#include <atomic>
 #include <mutex>
 
 #include "kernels.h"
@@ -7,16 +8,16 @@
 namespace csa {
 
 int device_sm_count() {
-  static int cached[64] = {0};
+  static std::atomic<int> cached[64] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
-  if (cached[dev] == 0) {
-    int n = 0;
+  int n = cached[dev].load(std::memory_order_relaxed);
+  if (n == 0) {
     if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1)
       n = 148;
-    cached[dev] = n;
+    cached[dev].store(n, std::memory_order_relaxed);
   }
-  return cached[dev];
+  return n;
 }
 
 cudaError_t ensure_smem_attr(const void* func, int slot, size_t bytes) {
