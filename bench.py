@@ -52,8 +52,8 @@ def algorithmic_bytes(w) -> dict:
     Only bytes the method must move are counted: inputs read once, outputs
     written once.  Intermediates the library materialises (indexer scores,
     split partials) are implementation overhead and are not counted, except
-    as the input of the kernel whose job is to read them (top-k reads the
-    scores it ranks)."""
+    as the input of the kernel whose job is to read them: the top-k stage's
+    own figure counts the scores it ranks, the step total does not."""
     B, d, m, W, H = w.B, w.d, w.m, w.W, w.H
     out = {}
     blk_in = B * m * d * 2 + (B * m * w.D_I * 2 if w.csa else 0)
@@ -71,7 +71,7 @@ def algorithmic_bytes(w) -> dict:
         kv = B * (w.N_c + W) * d * 2
         out["mqa"] = kv + q_bytes + H * 4
     out["combine"] = o_bytes
-    out["step"] = sum(out.values())
+    out["step"] = sum(out.values()) - (B * w.N_c * 4 if w.csa else 0)
     return out
 
 

@@ -157,3 +157,28 @@ def test_yarn_argument_checks(L, args, code):
         binding.rope_yarn(*args)
     assert e.value.status == code
     assert L.csa_rope_yarn(64, 1e4, 16.0, 32.0, 1.0, 65536.0, None, None) == 1
+
+
+# ------------------------------------------- bench accounting (no GPU) --
+def test_step_algorithmic_bytes_per_query():
+    """Per query of a decode step: indexer keys N (D_I + 4), gathered entries
+    k d 2, window W d 2, newest-block compression (m d 2 + d 2 for the KV,
+    m D_I 2 + D_I + 4 for the indexer), q and out H d 2 each, the indexer
+    query H_I (D_I + 8), the selection k 4 written and read, its count; once
+    per step (shared by the batch): the sinks H 4 and the pooling weights.
+    The fp32 scores are implementation traffic (not counted)."""
+    import sys
+    sys.argv = ["bench"]
+    import bench
+    from compressed_sparse_kv_04_b200 import configs
+    for w in (configs.CSA_128K, configs.CSA_1M):
+        N, d, k, W, m, H, HI, DI = w.N_c, w.d, w.k, w.W, w.m, w.H, w.H_I, w.D_I
+        per_q = (N * (DI + 4) + k * d * 2 + W * d * 2 + (m * d * 2 + d * 2) + (m * DI * 2 + DI + 4)
+                 + 2 * H * d * 2 + HI * (DI + 8) + 2 * k * 4 + 4)
+        weights = ((d + m) * 4 * 2 + H * 4) / w.B  # pooling weights and sinks, once per step
+        got = bench.algorithmic_bytes(w)["step"] / w.B
+        assert abs(got - (per_q + weights)) <= 8, (w.name, got, per_q + weights)
+    w = configs.HCA_1M
+    per_q = (w.N_c + w.W) * w.d * 2 + w.m * w.d * 2 + w.d * 2 + 2 * w.H * w.d * 2 + w.H * 4 / w.B
+    got = bench.algorithmic_bytes(w)["step"] / w.B
+    assert abs(got - per_q - (w.d + w.m) * 4 / w.B) <= 8, (got, per_q)
