@@ -20,11 +20,13 @@ STATUS_NAMES = {0: "CSA_OK", 1: "CSA_ERR_INVALID_ARG", 2: "CSA_ERR_UNSUPPORTED_S
                 3: "CSA_ERR_CAPACITY", 4: "CSA_ERR_WORKSPACE", 5: "CSA_ERR_CUDA",
                 6: "CSA_ERR_DEVICE_TIMEOUT", 7: "CSA_ERR_DEVICE_INDEX"}
 OP_INDEX_TOPK, OP_SPARSE_MQA, OP_DENSE_MQA, OP_PREFILL, OP_HCA_PREFILL = 1, 2, 3, 4, 5
+OP_CSA_DECODE_STEP, OP_HCA_DECODE_STEP = 6, 7
 
 EXPORTS = ["csa_version", "csa_last_error", "csa_workspace_bytes", "hca_compress",
            "csa_compress", "lightning_index_topk", "lightning_index_scores", "topk_select",
            "sparse_mqa_decode", "dense_mqa_decode", "csa_prefill_chunk",
-           "lightning_index_topk_static", "csa_rope_yarn", "hca_prefill_chunk"]
+           "lightning_index_topk_static", "csa_rope_yarn", "hca_prefill_chunk",
+           "csa_decode_step", "hca_decode_step"]
 
 
 class CsaError(RuntimeError):
@@ -80,6 +82,10 @@ def _declare(L):
                                               vp]
     L.hca_prefill_chunk.argtypes = [P, i64, i32, vp, i64, vp, vp, vp, vp, i64, vp, vp, vp, vp, vp,
                                     vp, vp, sz, vp, vp]
+    L.csa_decode_step.argtypes = [P, vp, vp, vp, i64, vp, vp, vp, vp, vp, vp, vp, vp, i64, vp, vp,
+                                  vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp, vp]
+    L.hca_decode_step.argtypes = [P, vp, vp, i64, vp, vp, vp, vp, i64, vp, vp, vp, vp, vp, vp, vp,
+                                  sz, vp, vp]
     L.csa_rope_yarn.argtypes = [i32, C.c_double, C.c_double, C.c_double, C.c_double,
                                 C.c_double, C.POINTER(C.c_double), C.POINTER(C.c_double)]
     for name in EXPORTS[3:]:
@@ -241,3 +247,28 @@ def hca_prefill_chunk(p, P, T, kv_tok, w_s, b_pos, gamma, kv_c, q, sink, out, ga
         _ptr(kv_c), kv_c.shape[1], _ptr(q), _ptr(sink), _ptr(gamma_q), _ptr(gamma_kv), _ptr(out),
         _ptr(lse), _ptr(ws), 0 if ws is None else ws.numel() * ws.element_size(),
         _ptr(dev_status), _stream(stream)))
+
+
+def csa_decode_step(p, pos_q, kv_tok, idx_tok, w_s, b_pos, gamma, w_s_idx, b_pos_idx, kv_c,
+                    idx_key, idx_scale, q, q_idx, q_scale, w, sink, topk_idx, topk_cnt, out,
+                    gamma_q=None, gamma_kv=None, lse=None, ws=None, dev_status=None, stream=None):
+    """One CSA decode step (newest-block compression, indexer, top-k, sparse
+    MQA) for B sequences at positions pos_q [B]."""
+    _check(lib().csa_decode_step(
+        C.byref(p), _ptr(pos_q), _ptr(kv_tok), _ptr(idx_tok), kv_tok.shape[1], _ptr(w_s),
+        _ptr(b_pos), _ptr(gamma), _ptr(w_s_idx), _ptr(b_pos_idx), _ptr(kv_c), _ptr(idx_key),
+        _ptr(idx_scale), kv_c.shape[1], _ptr(q), _ptr(q_idx), _ptr(q_scale), _ptr(w), _ptr(sink),
+        _ptr(gamma_q), _ptr(gamma_kv), _ptr(topk_idx), _ptr(topk_cnt), _ptr(out), _ptr(lse),
+        _ptr(ws), 0 if ws is None else ws.numel() * ws.element_size(), _ptr(dev_status),
+        _stream(stream)))
+
+
+def hca_decode_step(p, pos_q, kv_tok, w_s, b_pos, gamma, kv_c, q, sink, out, gamma_q=None,
+                    gamma_kv=None, lse=None, ws=None, dev_status=None, stream=None):
+    """One HCA decode step (newest-block compression, dense MQA) for B
+    sequences at positions pos_q [B]."""
+    _check(lib().hca_decode_step(
+        C.byref(p), _ptr(pos_q), _ptr(kv_tok), kv_tok.shape[1], _ptr(w_s), _ptr(b_pos),
+        _ptr(gamma), _ptr(kv_c), kv_c.shape[1], _ptr(q), _ptr(sink), _ptr(gamma_q),
+        _ptr(gamma_kv), _ptr(out), _ptr(lse), _ptr(ws),
+        0 if ws is None else ws.numel() * ws.element_size(), _ptr(dev_status), _stream(stream)))

@@ -182,6 +182,15 @@ size_t csa_workspace_bytes(const csa_params* p, csa_op op, int Q, int64_t N_cap)
                                       p->d) +
              512;
     }
+    case CSA_OP_CSA_DECODE_STEP:
+      return scores_bytes(p->B, N_cap) +
+             csa::mqa_workspace_bytes(p->B, splits_for(p, CSA_OP_SPARSE_MQA, p->B, N_cap), p->H,
+                                      p->d) +
+             512;
+    case CSA_OP_HCA_DECODE_STEP:
+      return csa::mqa_workspace_bytes(p->B, splits_for(p, CSA_OP_DENSE_MQA, p->B, N_cap), p->H,
+                                      p->d) +
+             256;
     case CSA_OP_HCA_PREFILL: {
       int rows = Q;
       return csa::mqa_workspace_bytes(rows, splits_for(p, CSA_OP_DENSE_MQA, rows, N_cap), p->H,
@@ -199,7 +208,8 @@ static csa_status compress_common(const char* fn, const csa_params* p, const voi
                                   int64_t first_block, int64_t n_blocks, void* kv_c,
                                   int64_t N_cap, const void* idx_tok, const float* w_s_idx,
                                   const float* b_pos_idx, uint8_t* idx_key, float* idx_scale,
-                                  int32_t* dev_status, void* stream) {
+                                  int32_t* dev_status, void* stream,
+                                  const int64_t* pos_newest = nullptr) {
   csa_status st = check_common(fn, p);
   if (st != CSA_OK) return st;
   REQ_PTR(kv_tok);
@@ -245,6 +255,7 @@ static csa_status compress_common(const char* fn, const csa_params* p, const voi
   c.b_pos_idx = b_pos_idx;
   c.first_block = first_block;
   c.n_blocks = n_blocks;
+  c.pos_newest = pos_newest;
   c.kv_c = kv_c;
   c.idx_key = idx_key;
   c.idx_scale = idx_scale;
@@ -597,6 +608,76 @@ csa_status csa_prefill_chunk(const csa_params* p, int64_t P, int T, const void* 
   return mqa_common(fn, p, CSA_OP_SPARSE_MQA, T, T, q, nullptr, P, kv_c, N_cap, topk_idx,
                     topk_cnt, kv_tok, L_cap, sink, gamma_q, gamma_kv, out, nullptr, rest,
                     rest_bytes, dev_status, s);
+}
+
+csa_status csa_decode_step(const csa_params* p, const int64_t* pos_q, const void* kv_tok,
+                           const void* idx_tok, int64_t L_cap, const float* w_s,
+                           const float* b_pos, const float* gamma, const float* w_s_idx,
+                           const float* b_pos_idx, void* kv_c, uint8_t* idx_key,
+                           float* idx_scale, int64_t N_cap, const void* q, const uint8_t* q_idx,
+                           const float* q_scale, const float* w, const float* sink,
+                           const float* gamma_q, const float* gamma_kv, int32_t* topk_idx,
+                           int32_t* topk_cnt, void* out, float* lse, void* ws, size_t ws_bytes,
+                           int32_t* dev_status, void* stream) {
+  const char* fn = "csa_decode_step";
+  csa_status st = check_index_args(fn, p, 1, N_cap);
+  if (st != CSA_OK) return st;
+  st = check_mqa_args(fn, p, q, pos_q, kv_c, N_cap, kv_tok, L_cap, sink, gamma_q, gamma_kv, out,
+                      lse, dev_status);
+  if (st != CSA_OK) return st;
+  if (p->k < 1 || p->k > 1024)
+    return fail(CSA_ERR_UNSUPPORTED_SHAPE, "%s: k=%d (supported: 1..1024)", fn, p->k);
+  REQ_PTR(idx_tok);
+  REQ_PTR(q_idx);
+  REQ_PTR4(q_scale);
+  REQ_PTR4(w);
+  REQ_PTR(topk_idx);
+  REQ_PTR4(topk_cnt);
+  size_t need = csa_workspace_bytes(p, CSA_OP_CSA_DECODE_STEP, 1, N_cap);
+  if (!ws || ws_bytes < need)
+    return fail(CSA_ERR_WORKSPACE, "%s: workspace of %zu bytes needed, %zu given", fn, need,
+                ws ? ws_bytes : (size_t)0);
+  if (!aligned16(ws)) return fail(CSA_ERR_INVALID_ARG, "%s: ws is not 16-byte aligned", fn);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // 1. Each sequence's newest block: the one holding its query token,
+  // pooled over the tokens up to it.
+  st = compress_common(fn, p, kv_tok, L_cap, nullptr, 0, w_s, b_pos, gamma, 0, 1, kv_c, N_cap,
+                       idx_tok, w_s_idx, b_pos_idx, idx_key, idx_scale, dev_status, stream, pos_q);
+  if (st != CSA_OK) return st;
+  // 2-3. Indexer and top-k over each sequence's visible entries.
+  float* scores = static_cast<float*>(ws);
+  st = index_topk_common(fn, p, 1, q_idx, q_scale, w, idx_key, idx_scale, N_cap, pos_q, 0,
+                         topk_idx, topk_cnt, scores, dev_status, s);
+  if (st != CSA_OK) return st;
+  // 4. Sparse MQA over the selection, the window and the sink.
+  char* rest = static_cast<char*>(ws) + scores_bytes(p->B, N_cap);
+  return mqa_common(fn, p, CSA_OP_SPARSE_MQA, p->B, 1, q, pos_q, 0, kv_c, N_cap, topk_idx,
+                    topk_cnt, kv_tok, L_cap, sink, gamma_q, gamma_kv, out, lse, rest,
+                    ws_bytes - scores_bytes(p->B, N_cap), dev_status, s);
+}
+
+csa_status hca_decode_step(const csa_params* p, const int64_t* pos_q, const void* kv_tok,
+                           int64_t L_cap, const float* w_s, const float* b_pos,
+                           const float* gamma, void* kv_c, int64_t N_cap, const void* q,
+                           const float* sink, const float* gamma_q, const float* gamma_kv,
+                           void* out, float* lse, void* ws, size_t ws_bytes,
+                           int32_t* dev_status, void* stream) {
+  const char* fn = "hca_decode_step";
+  csa_status st = check_mqa_args(fn, p, q, pos_q, kv_c, N_cap, kv_tok, L_cap, sink, gamma_q,
+                                 gamma_kv, out, lse, dev_status);
+  if (st != CSA_OK) return st;
+  size_t need = csa_workspace_bytes(p, CSA_OP_HCA_DECODE_STEP, 1, N_cap);
+  if (!ws || ws_bytes < need)
+    return fail(CSA_ERR_WORKSPACE, "%s: workspace of %zu bytes needed, %zu given", fn, need,
+                ws ? ws_bytes : (size_t)0);
+  if (!aligned16(ws)) return fail(CSA_ERR_INVALID_ARG, "%s: ws is not 16-byte aligned", fn);
+  // 1. Each sequence's newest block, then 2. dense MQA with window and sink.
+  st = compress_common(fn, p, kv_tok, L_cap, nullptr, 0, w_s, b_pos, gamma, 0, 1, kv_c, N_cap,
+                       nullptr, nullptr, nullptr, nullptr, nullptr, dev_status, stream, pos_q);
+  if (st != CSA_OK) return st;
+  return mqa_common(fn, p, CSA_OP_DENSE_MQA, p->B, 1, q, pos_q, 0, kv_c, N_cap, nullptr, nullptr,
+                    kv_tok, L_cap, sink, gamma_q, gamma_kv, out, lse, ws, ws_bytes, dev_status,
+                    static_cast<cudaStream_t>(stream));
 }
 
 csa_status hca_prefill_chunk(const csa_params* p, int64_t P, int T, const void* kv_tok,

@@ -49,6 +49,9 @@ struct PoolArgs {
   const int64_t* ctx_len;  // [B] device, or null -> ctx_len_value
   int64_t ctx_len_value;
   int64_t first_block, n_blocks;
+  // [B] device, or null.  Set: one block per sequence, the one holding
+  // position pos_newest[b], pooled over tokens up to pos_newest[b].
+  const int64_t* pos_newest;
   float eps;
   double inv_freq[64];  // rotation frequencies (rope_dim/2 entries)
   int32_t* status;
@@ -260,13 +263,29 @@ CSA_DEV void pool_stream(const PoolArgs& a, const StreamArgs& sa, float* smem) {
   const int per_cta = kWarps / G;                  // blocks per CTA
   const int64_t unit = (int64_t)blockIdx.x * per_cta + warp / G;  // (b, block) pair
   const int64_t total = (int64_t)a.B * a.n_blocks;
-  const bool active = unit < total;
+  bool active = unit < total;
   int64_t b = 0, i = 0;
   int present = 0;
   if (active) {
     b = unit / a.n_blocks;
-    i = a.first_block + unit % a.n_blocks;
-    int64_t L = a.ctx_len ? a.ctx_len[b] : a.ctx_len_value;
+    int64_t L;
+    if (a.pos_newest) {
+      const int64_t t = a.pos_newest[b];
+      L = t + 1;
+      i = t < 0 ? 0 : t / a.m;
+      if (t < 0 || i >= a.N_cap) {  // no block, or one outside the cache
+        active = false;
+        L = 0;
+        i = 0;
+        if (t >= 0 && threadIdx.x % 32 == 0) {
+          pdl_wait();
+          report(a.status, CSA_ERR_DEVICE_INDEX);
+        }
+      }
+    } else {
+      i = a.first_block + unit % a.n_blocks;
+      L = a.ctx_len ? a.ctx_len[b] : a.ctx_len_value;
+    }
     if (L > a.L_cap) L = a.L_cap;
     int64_t rem = L - i * a.m;
     present = rem <= 0 ? 0 : (rem < a.m ? (int)rem : a.m);
@@ -365,12 +384,13 @@ cudaError_t launch_compress(const CompressLaunch& c, cudaStream_t stream) {
   a.ctx_len = c.ctx_len;
   a.ctx_len_value = c.ctx_len_value;
   a.first_block = c.first_block;
-  a.n_blocks = c.n_blocks;
+  a.n_blocks = c.pos_newest ? 1 : c.n_blocks;
+  a.pos_newest = c.pos_newest;
   a.eps = c.eps;
   a.status = c.status;
   int G = c.m <= 16 ? 1 : kWarps;
   int per_cta = kWarps / G;
-  int64_t units = (int64_t)c.B * c.n_blocks;
+  int64_t units = (int64_t)c.B * a.n_blocks;
   if (units == 0) return cudaSuccess;
   int64_t grid_x = (units + per_cta - 1) / per_cta;
   if (grid_x > 0x7FFFFFFF) return cudaErrorInvalidConfiguration;

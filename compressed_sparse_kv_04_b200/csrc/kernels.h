@@ -19,6 +19,7 @@ struct CompressLaunch {
   int64_t ctx_len_value;  // used when ctx_len is null
   const float *w_s, *b_pos, *gamma, *w_s_idx, *b_pos_idx;
   int64_t first_block, n_blocks;
+  const int64_t* pos_newest;  // [B] or null: one block per sequence, the one holding pos
   void* kv_c;
   uint8_t* idx_key;
   float* idx_scale;

@@ -84,7 +84,9 @@ typedef enum {
   CSA_OP_SPARSE_MQA = 2,
   CSA_OP_DENSE_MQA = 3,
   CSA_OP_PREFILL = 4,
-  CSA_OP_HCA_PREFILL = 5
+  CSA_OP_HCA_PREFILL = 5,
+  CSA_OP_CSA_DECODE_STEP = 6,
+  CSA_OP_HCA_DECODE_STEP = 7
 } csa_op;
 
 /* Library version (major*100 + minor). */
@@ -318,6 +320,54 @@ csa_status csa_prefill_chunk(const csa_params* p, int64_t P, int T, const void* 
                              const float* sink, const float* gamma_q, const float* gamma_kv,
                              int32_t* topk_idx, int32_t* topk_cnt, void* out, void* ws,
                              size_t ws_bytes, int32_t* dev_status, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * One CSA decode step for B sequences, each at its own position ([P2] CSA
+ * steps 1-3; [P5] "Hybrid attention": CSA bullet).  The caller has written
+ * each sequence's new token rows (kv_tok, idx_tok row pos_q[b]); the call
+ * then runs, in order:
+ *   1. compression of each sequence's newest block, the one holding its
+ *      query token: block pos_q[b]/m pooled over tokens up to pos_q[b] (as
+ *      csa_compress; a block that is still partial is written but stays
+ *      invisible until it is complete, and a later step rewrites it);
+ *   2. the Lightning Indexer and top-k over the visible entries
+ *      floor((pos_q[b]+1)/m) (as lightning_index_topk);
+ *   3. the sparse MQA over the selection, the window and the sink (as
+ *      sparse_mqa_decode).
+ * Calling it for consecutive positions is the decode loop: the caches grow
+ * by one compressed entry every m steps.
+ *   pos_q [B] int64 (device); q [B, H, d]; q_idx [B, H_I, D_I]; q_scale, w
+ *   [B, H_I]; topk_idx [B, k], topk_cnt [B] (written); out [B, H, d] bf16
+ *   and lse [B, H] or NULL (written); other tensors as csa_compress and
+ *   sparse_mqa_decode.
+ * Workspace: csa_workspace_bytes(p, CSA_OP_CSA_DECODE_STEP, 1, N_cap).
+ * Device errors: a newest block at or beyond N_cap -> CSA_ERR_DEVICE_INDEX
+ * (not written).
+ * ------------------------------------------------------------------------- */
+csa_status csa_decode_step(const csa_params* p, const int64_t* pos_q, const void* kv_tok,
+                           const void* idx_tok, int64_t L_cap, const float* w_s,
+                           const float* b_pos, const float* gamma, const float* w_s_idx,
+                           const float* b_pos_idx, void* kv_c, uint8_t* idx_key,
+                           float* idx_scale, int64_t N_cap, const void* q, const uint8_t* q_idx,
+                           const float* q_scale, const float* w, const float* sink,
+                           const float* gamma_q, const float* gamma_kv, int32_t* topk_idx,
+                           int32_t* topk_cnt, void* out, float* lse, void* ws, size_t ws_bytes,
+                           int32_t* dev_status, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * One HCA decode step for B sequences, each at its own position ([P2] HCA
+ * paragraph; [P5] "Hybrid attention": HCA bullet): compression of each
+ * sequence's newest block (block pos_q[b]/m, pooled over tokens up to
+ * pos_q[b], as hca_compress), then the dense MQA over the visible entries,
+ * the window and the sink (as dense_mqa_decode).
+ * Workspace: csa_workspace_bytes(p, CSA_OP_HCA_DECODE_STEP, 1, N_cap).
+ * ------------------------------------------------------------------------- */
+csa_status hca_decode_step(const csa_params* p, const int64_t* pos_q, const void* kv_tok,
+                           int64_t L_cap, const float* w_s, const float* b_pos,
+                           const float* gamma, void* kv_c, int64_t N_cap, const void* q,
+                           const float* sink, const float* gamma_q, const float* gamma_kv,
+                           void* out, float* lse, void* ws, size_t ws_bytes,
+                           int32_t* dev_status, void* stream);
 
 /* ---------------------------------------------------------------------------
  * HCA prefill chunk (B = 1; [P2] HCA paragraph: dense attention over every

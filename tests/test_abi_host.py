@@ -120,6 +120,24 @@ def test_hca_prefill_argument_checks(L):
     assert L.csa_workspace_bytes(C.byref(p), 5, 4096, 544) > 0
 
 
+def test_decode_step_argument_checks(L):
+    p = P(B=2)
+    n = [None] * 29
+    n[0] = C.byref(p)
+    n[4], n[13], n[26] = 1 << 12, 1 << 10, 0  # L_cap, N_cap, ws_bytes
+    assert L.csa_decode_step(*n) == 1            # pos_q (and the rest) NULL
+    p = P(B=2, k=4096)
+    n[0] = C.byref(p)
+    assert L.csa_decode_step(*n) in (1, 2)       # k outside 1..1024 or NULL pointers
+    h = [None] * 19
+    h[0] = C.byref(P(B=2, m=128))
+    h[3], h[8], h[16] = 1 << 12, 32, 0
+    assert L.hca_decode_step(*h) == 1            # NULL tensors
+    assert L.csa_workspace_bytes(C.byref(P(B=8)), 6, 1, 32768) > \
+        L.csa_workspace_bytes(C.byref(P(B=8)), 2, 1, 32768)
+    assert L.csa_workspace_bytes(C.byref(P(B=8, m=128)), 7, 1, 8192) > 0
+
+
 def test_workspace_sizes_are_monotone(L):
     p = P(B=8)
     a = L.csa_workspace_bytes(C.byref(p), 1, 1, 32768)

@@ -1,0 +1,159 @@
+"""GPU parity of the decode loop: csa_decode_step / hca_decode_step called for
+consecutive positions, each sequence at its own position, against the fp64
+oracle through the C ABI.
+
+The caches start with the blocks the oracle compresses from the tokens
+before each sequence's first step, so no oracle input comes from the GPU.
+Every step is checked layer by layer: the newest block of every sequence
+against the oracle's compression of the tokens up to its position; scores
+against the oracle fed the GPU's E4M3 keys; the top-k bit-exact against the
+oracle ranking the GPU's scores; attention against the oracle fed the GPU's
+selection and cache.  After the loop the whole cache is checked."""
+import numpy as np
+import pytest
+import torch
+
+from compressed_sparse_kv_04_b200 import binding, configs, synth
+from gpuhelp import assert_attention_close, assert_bf16_storage_close, bits8, bits16, f32
+from test_gpu_compress_index import check_keys
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    binding.lib()
+
+
+def _to_bf16(bits):
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(DEV)
+
+
+def _check_lse(lse, rlse):
+    gl = f32(lse).astype(np.float64)
+    fin = np.isfinite(rlse)
+    assert np.array_equal(np.isfinite(gl), fin)
+    assert np.allclose(gl[fin], rlse[fin], rtol=0, atol=2e-2), np.abs(gl[fin] - rlse[fin]).max()
+
+
+def test_csa_decode_loop(orc):
+    """Three sequences at positions 301, 514 and 127, six steps each: blocks
+    complete mid-loop (at 303, 515/519, 127/131), and the third sequence
+    starts with fewer visible entries (32) than k (64)."""
+    w = configs.scaled(configs.CSA_128K, B=3, k=64, L=2048)
+    B, m, L_cap = w.B, w.m, 2048
+    N_cap = L_cap // m
+    start = np.array([301, 514, 127])
+    kv_tok, idx_tok = synth.token_streams(w, L_cap=L_cap, device=DEV)
+    kv_bits, idx_bits = bits16(kv_tok), bits16(idx_tok)
+    w_s, b_pos = synth.pool_params(w, DEV)
+    w_si, b_pi = synth.pool_params(w, DEV, indexer=True)
+    kv_c0, _, _ = orc.compress_kv(kv_bits, start, f32(w_s), f32(b_pos), None, m, 0, N_cap, N_cap,
+                                  rope_dim=w.rope_dim)
+    key0, ks0, _, _ = orc.compress_index(idx_bits, start, f32(w_si), f32(b_pi), m, 0, N_cap, N_cap)
+    kv_c = _to_bf16(kv_c0)
+    idx_key = torch.from_numpy(key0).to(DEV)
+    idx_scale = torch.from_numpy(ks0).to(DEV)
+    p = binding.params_for(w, B=B)
+    ws = binding.workspace(p, binding.OP_CSA_DECODE_STEP, 1, N_cap)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    for step in range(6):
+        pos = start + step
+        qi = synth.queries(configs.scaled(w, seed=w.seed + 100 + step), Q=1, device=DEV)
+        q = qi["q"][:, 0].contiguous()
+        out = torch.full((B, w.H, w.D), float("nan"), dtype=torch.bfloat16, device=DEV)
+        lse = torch.full((B, w.H), float("nan"), dtype=torch.float32, device=DEV)
+        tidx = torch.full((B, w.k), -7, dtype=torch.int32, device=DEV)
+        tcnt = torch.full((B,), -7, dtype=torch.int32, device=DEV)
+        ws.fill_(0xFF)  # unwritten scores read as NaN
+        pos_t = torch.from_numpy(pos).to(DEV)
+        binding.csa_decode_step(p, pos_t, kv_tok, idx_tok, w_s, b_pos, None, w_si, b_pi, kv_c,
+                                idx_key, idx_scale, q, qi["q_idx"][:, 0].contiguous(),
+                                qi["q_scale"][:, 0].contiguous(), qi["w"][:, 0].contiguous(),
+                                qi["sink"], tidx, tcnt, out, lse=lse, ws=ws, dev_status=status)
+        torch.cuda.synchronize()
+        assert status.item() == 0, status.item()
+        # 1. Each sequence's newest block (pooled over tokens up to pos).
+        got_c, got_k, got_s = bits16(kv_c), bits8(idx_key), f32(idx_scale)
+        for b in range(B):
+            i = pos[b] // m
+            _, _, vals = orc.compress_kv(kv_bits[b: b + 1], [pos[b] + 1], f32(w_s), f32(b_pos),
+                                         None, m, i, 1, N_cap, rope_dim=w.rope_dim)
+            assert_bf16_storage_close(got_c[b: b + 1, i], vals[:, i], f"step {step} seq {b} entry")
+            _, _, kvals, _ = orc.compress_index(idx_bits[b: b + 1], [pos[b] + 1], f32(w_si),
+                                                f32(b_pi), m, i, 1, N_cap)
+            check_keys(orc, got_k[b: b + 1, i], got_s[b: b + 1, i], kvals[:, i],
+                       f"step {step} seq {b} key")
+        # 2. Scores of the visible entries against the oracle on the GPU's keys.
+        nv = (pos + 1) // m
+        scores = f32(ws[: B * N_cap * 4].view(torch.float32).view(B, N_cap)).astype(np.float64)
+        ref = orc.index_scores(bits8(qi["q_idx"]), f32(qi["q_scale"]), f32(qi["w"]), got_k, got_s,
+                               pos.reshape(B, 1), m)[:, 0]
+        for b in range(B):
+            g, r = scores[b, : nv[b]], ref[b, : nv[b]]
+            assert np.allclose(g, r, rtol=2e-5, atol=1e-6 * np.abs(r).mean()), (step, b)
+        # 3. Top-k bit-exact on the GPU's scores.
+        gs = np.where(np.isnan(scores), -np.inf, scores)
+        ridx, rcnt = orc.topk(gs, nv, w.k)
+        assert np.array_equal(tcnt.cpu().numpy(), rcnt), step
+        assert np.array_equal(tidx.cpu().numpy(), ridx), step
+        # 4. Attention with the GPU's selection and cache.
+        ro, rl = orc.mqa(bits16(q).reshape(B, 1, w.H, w.D), pos.reshape(B, 1), got_c, kv_bits,
+                         f32(qi["sink"]), m, w.W, w.rope_dim, tidx.cpu().numpy()[:, None],
+                         tcnt.cpu().numpy()[:, None])
+        got = out.double().cpu().numpy()
+        assert np.isfinite(got).all()
+        assert_attention_close(got, ro[:, 0], f"step {step}")
+        _check_lse(lse, rl[:, 0])
+    # The whole cache after the loop: every block of tokens up to the last
+    # position, the partial newest one included.
+    last = start + 5
+    _, _, vals = orc.compress_kv(kv_bits, last + 1, f32(w_s), f32(b_pos), None, m, 0, N_cap, N_cap,
+                                 rope_dim=w.rope_dim)
+    got_c = bits16(kv_c)
+    for b in range(B):
+        n = last[b] // m + 1
+        assert_bf16_storage_close(got_c[b, :n], vals[b, :n], f"seq {b} cache")
+
+
+def test_hca_decode_loop(orc):
+    """Two sequences at positions 125 and 640, six steps each: the first
+    block of the first sequence completes at 127 (its first visible entry)."""
+    w = configs.scaled(configs.HCA_1M, B=2, L=1536)
+    B, m, L_cap = w.B, w.m, 1536
+    N_cap = L_cap // m
+    start = np.array([125, 640])
+    kv_tok, _ = synth.token_streams(w, L_cap=L_cap, device=DEV)
+    kv_bits = bits16(kv_tok)
+    w_s, b_pos = synth.pool_params(w, DEV)
+    kv_c0, _, _ = orc.compress_kv(kv_bits, start, f32(w_s), f32(b_pos), None, m, 0, N_cap, N_cap,
+                                  rope_dim=w.rope_dim)
+    kv_c = _to_bf16(kv_c0)
+    p = binding.params_for(w, B=B)
+    ws = binding.workspace(p, binding.OP_HCA_DECODE_STEP, 1, N_cap)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    for step in range(6):
+        pos = start + step
+        qi = synth.queries(configs.scaled(w, seed=w.seed + 100 + step), Q=1, device=DEV)
+        q = qi["q"][:, 0].contiguous()
+        out = torch.full((B, w.H, w.D), float("nan"), dtype=torch.bfloat16, device=DEV)
+        lse = torch.full((B, w.H), float("nan"), dtype=torch.float32, device=DEV)
+        binding.hca_decode_step(p, torch.from_numpy(pos).to(DEV), kv_tok, w_s, b_pos, None, kv_c,
+                                q, qi["sink"], out, lse=lse, ws=ws, dev_status=status)
+        torch.cuda.synchronize()
+        assert status.item() == 0, status.item()
+        got_c = bits16(kv_c)
+        for b in range(B):
+            i = pos[b] // m
+            _, _, vals = orc.compress_kv(kv_bits[b: b + 1], [pos[b] + 1], f32(w_s), f32(b_pos),
+                                         None, m, i, 1, N_cap, rope_dim=w.rope_dim)
+            assert_bf16_storage_close(got_c[b: b + 1, i], vals[:, i], f"step {step} seq {b} entry")
+        ro, rl = orc.mqa(bits16(q).reshape(B, 1, w.H, w.D), pos.reshape(B, 1), got_c, kv_bits,
+                         f32(qi["sink"]), m, w.W, w.rope_dim)
+        got = out.double().cpu().numpy()
+        assert np.isfinite(got).all()
+        assert_attention_close(got, ro[:, 0], f"HCA step {step}")
+        _check_lse(lse, rl[:, 0])
