@@ -312,7 +312,8 @@ class Decode:
         ]
 
     def launches_per_step(self):
-        # compress 1, (index 1, top-k 1), attention pair 1 + combine 1
+        # compress 1, (index 1, top-k 1), attention 1 + merge 1 (the decode
+        # workloads' rows always have several splits, so the merge runs)
         return 5 if self.w.csa else 3
 
     def capture(self, instrumented=False):
@@ -669,7 +670,9 @@ def run_prefill(args):
         "step_roofline": {"fp8_flops": fp8, "bf16_flops": bf16,
                           "ideal_ms": round(t_ideal * 1e3, 4),
                           "frac": round(t_ideal * 1e3 / ms, 4)},
-        "gpu_launches": 6 * K, "clocks": clocks.summary(), "device_status": int(status.item()),
+        # per chunk: compress, indexer, top-k, attention (one split per row:
+        # no merge); plus the separately timed indexer launch
+        "gpu_launches": 5 * K, "clocks": clocks.summary(), "device_status": int(status.item()),
     }
     print(json.dumps(line), flush=True)
 
@@ -746,7 +749,8 @@ def run_hca_prefill(args):
                      "unit": "TFLOP/s", "frac": round(tf / peaks["bf16_tflops"], 4),
                      "peak_source": peaks["source"], "avg_launch_ms": round(ms, 4),
                      "algorithmic_flops": flops},
-        "gpu_launches": 3 * K, "clocks": clocks.summary(), "device_status": int(status.item()),
+        # per chunk: compress, attention (one split per row: no merge)
+        "gpu_launches": 2 * K, "clocks": clocks.summary(), "device_status": int(status.item()),
     }
     print(json.dumps(line), flush=True)
 
