@@ -200,3 +200,18 @@ def test_step_algorithmic_bytes_per_query():
     per_q = (w.N_c + w.W) * w.d * 2 + w.m * w.d * 2 + w.d * 2 + 2 * w.H * w.d * 2 + w.H * 4 / w.B
     got = bench.algorithmic_bytes(w)["step"] / w.B
     assert abs(got - per_q - (w.d + w.m) * 4 / w.B) <= 8, (got, per_q)
+
+
+def test_params_for_applies_yarn_to_a_yarn_workload(L, orc):
+    import math
+
+    import numpy as np
+    from compressed_sparse_kv_04_b200 import configs
+    w = configs.CSA_FLASH_128K
+    p = binding.params_for(w)
+    tab = np.array([p.rope_inv_freq[j] for j in range(w.rope_dim // 2)])
+    assert np.allclose(tab, orc.yarn_inv_freq(w.rope_dim, *w.yarn), rtol=1e-14, atol=0)
+    assert math.isclose(p.softmax_scale, orc.yarn_logit_gain(w.yarn[0]) / math.sqrt(w.d),
+                        rel_tol=1e-6)
+    plain = binding.params_for(configs.CSA_128K)
+    assert not plain.rope_inv_freq and plain.softmax_scale == 0.0
