@@ -87,7 +87,8 @@ def _declare(L):
     L.hca_decode_step.argtypes = [P, vp, vp, i64, vp, vp, vp, vp, i64, vp, vp, vp, vp, vp, vp, vp,
                                   sz, vp, vp]
     L.csa_rope_yarn.argtypes = [i32, C.c_double, C.c_double, C.c_double, C.c_double,
-                                C.c_double, C.POINTER(C.c_double), C.POINTER(C.c_double)]
+                                C.c_double, i32, C.POINTER(C.c_double), C.POINTER(C.c_double),
+                                C.POINTER(C.c_float)]
     for name in EXPORTS[3:]:
         getattr(L, name).restype = i32
 
@@ -105,11 +106,11 @@ def make_params(B, d, H=0, H_I=0, D_I=0, k=0, window=0, rope_dim=0, m=4, eps=1e-
 def params_for(w, B=None, **kw):
     """csa_params for a Workload (compressed_sparse_kv_04_b200.configs).  A
     workload with YaRN settings gets the library's YaRN frequency table and
-    the logit scale gain / sqrt(d), unless the caller passes its own."""
+    logit scale (csa_rope_yarn), unless the caller passes its own."""
     if w.yarn is not None and w.rope_dim > 0 and "rope_inv_freq" not in kw:
-        tab, gain = rope_yarn(w.rope_dim, *w.yarn)
+        tab, _, scale = rope_yarn(w.rope_dim, *w.yarn, d=w.d)
         kw["rope_inv_freq"] = tab
-        kw.setdefault("softmax_scale", gain / w.d ** 0.5)
+        kw.setdefault("softmax_scale", scale)
     return make_params(B or w.B, w.d, w.H, w.H_I, w.D_I, w.k, w.W, w.rope_dim, w.m, **kw)
 
 
@@ -187,14 +188,16 @@ def lightning_index_topk_static(p, Q, q_idx, q_scale, w, idx_key, idx_scale, pos
         _stream(stream)))
 
 
-def rope_yarn(rope_dim, factor, beta_fast, beta_slow, original_len, base=10000.0):
-    """YaRN frequency table and logit gain (host only): returns (list of
-    rope_dim/2 frequencies for make_params(rope_inv_freq=...), logit gain)."""
-    tab = (C.c_double * (rope_dim // 2))()
+def rope_yarn(rope_dim, factor, beta_fast, beta_slow, original_len, base=10000.0, d=1):
+    """YaRN frequency table, logit gain and logit scale for head dim d (host
+    only, computed by the library): returns (list of rope_dim/2 frequencies
+    for make_params(rope_inv_freq=...), logit gain, softmax_scale)."""
+    tab = (C.c_double * max(1, rope_dim // 2))()
     gain = C.c_double()
-    _check(lib().csa_rope_yarn(rope_dim, base, factor, beta_fast, beta_slow, original_len, tab,
-                               C.byref(gain)))
-    return list(tab), gain.value
+    scale = C.c_float()
+    _check(lib().csa_rope_yarn(rope_dim, base, factor, beta_fast, beta_slow, original_len, d, tab,
+                               C.byref(gain), C.byref(scale)))
+    return list(tab)[: rope_dim // 2], gain.value, scale.value
 
 
 def lightning_index_scores(p, Q, q_idx, q_scale, w, idx_key, idx_scale, pos_q, scores,

@@ -129,13 +129,15 @@ extern "C" {
 int csa_version(void) { return 101; }
 
 csa_status csa_rope_yarn(int rope_dim, double base, double factor, double beta_fast,
-                         double beta_slow, double original_len, double* inv_freq,
-                         double* logit_gain) {
+                         double beta_slow, double original_len, int d, double* inv_freq,
+                         double* logit_gain, float* softmax_scale) {
   const char* fn = "csa_rope_yarn";
   if (rope_dim < 2 || rope_dim > 128 || rope_dim % 2)
     return fail(CSA_ERR_UNSUPPORTED_SHAPE, "%s: rope_dim=%d (supported: even, 2..128)", fn,
                 rope_dim);
   if (!inv_freq) return fail(CSA_ERR_INVALID_ARG, "%s: inv_freq is NULL", fn);
+  if (softmax_scale && d < 1)
+    return fail(CSA_ERR_INVALID_ARG, "%s: d=%d must be >= 1 for softmax_scale", fn, d);
   if (!(base > 1.0) || !std::isfinite(base) || !(factor >= 1.0) || !std::isfinite(factor) ||
       !(beta_slow >= 0.0) || !(beta_fast > beta_slow) || !std::isfinite(beta_fast) ||
       !(original_len > 0.0) || !std::isfinite(original_len))
@@ -151,10 +153,11 @@ csa_status csa_rope_yarn(int rope_dim, double base, double factor, double beta_f
     ramp = ramp < 0.0 ? 0.0 : (ramp > 1.0 ? 1.0 : ramp);
     inv_freq[j] = theta / factor + ramp * (theta - theta / factor);
   }
-  if (logit_gain) {
-    const double t = 1.0 + 0.1 * std::log(factor);
-    *logit_gain = t * t;
-  }
+  // The method's attention temperature: q and k are each scaled by
+  // 1 + 0.1 ln(factor), so the logits by its square.
+  const double t = 1.0 + 0.1 * std::log(factor);
+  if (logit_gain) *logit_gain = t * t;
+  if (softmax_scale) *softmax_scale = (float)(t * t / std::sqrt((double)d));
   return CSA_OK;
 }
 

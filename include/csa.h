@@ -105,22 +105,29 @@ const char* csa_last_error(void);
  *   turns_j  = original_len * theta_j / (2 pi)
  *   ramp_j   = clamp((turns_j - beta_slow) / (beta_fast - beta_slow), 0, 1)
  *   inv_freq[j] = ramp_j * theta_j + (1 - ramp_j) * theta_j / factor
- *   *logit_gain = (1 + 0.1 ln factor)^2   (the method's attention
- *                 temperature; multiply 1/sqrt(d) by it for softmax_scale)
+ *   *logit_gain    = (1 + 0.1 ln factor)^2   (the method's attention
+ *                    temperature: query and key are each scaled by
+ *                    1 + 0.1 ln factor)
+ *   *softmax_scale = *logit_gain / sqrt(d), rounded to binary32: the logit
+ *                    scale to put in csa_params.softmax_scale
  * Pass the table as csa_params.rope_inv_freq: compression, the window
  * rotation, the query rotation and the inverse rotation of the output all
  * use it.  (original_len = 1,048,576 / 16 = 65,536 is the reading for the
  * pages' schedule.)
- *   inv_freq   host, [rope_dim/2] doubles (written)
- *   logit_gain host, one double (written) or NULL
+ *   d             head dim of the attention calls (read only when
+ *                 softmax_scale is not NULL)
+ *   inv_freq      host, [rope_dim/2] doubles (written)
+ *   logit_gain    host, one double (written) or NULL
+ *   softmax_scale host, one float (written) or NULL
  * Errors: CSA_ERR_UNSUPPORTED_SHAPE for rope_dim odd or outside 2..128;
  *         CSA_ERR_INVALID_ARG for inv_freq NULL, base <= 1, factor < 1,
- *         beta_slow < 0, beta_fast <= beta_slow, original_len <= 0 or any
- *         non-finite value.
+ *         beta_slow < 0, beta_fast <= beta_slow, original_len <= 0, any
+ *         non-finite value, or d < 1 with softmax_scale not NULL.  Nothing
+ *         is written on error.
  * ------------------------------------------------------------------------- */
 csa_status csa_rope_yarn(int rope_dim, double base, double factor, double beta_fast,
-                         double beta_slow, double original_len, double* inv_freq,
-                         double* logit_gain);
+                         double beta_slow, double original_len, int d, double* inv_freq,
+                         double* logit_gain, float* softmax_scale);
 
 /* Workspace bytes that `op` needs for these params.
  *   Q     queries per sequence (1 for decode; T for CSA_OP_PREFILL and

@@ -18,3 +18,11 @@ def orc():
     from oracle import oracle
     oracle.lib()
     return oracle
+
+
+def pytest_terminal_summary(terminalreporter):
+    """Largest parity errors measured by the GPU tests of this session."""
+    gh = sys.modules.get("gpuhelp")
+    if gh is not None and getattr(gh, "MAX_ERR", None):
+        items = ", ".join(f"{k} {v:.3e}" for k, v in sorted(gh.MAX_ERR.items()))
+        terminalreporter.write_line(f"largest measured errors: {items}")

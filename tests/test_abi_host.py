@@ -156,9 +156,14 @@ def test_yarn_table_matches_the_oracle(L, orc, args):
     import math
 
     import numpy as np
-    tab, gain = binding.rope_yarn(*args)
+    tab, gain, scale = binding.rope_yarn(*args, d=512)
     assert np.allclose(tab, orc.yarn_inv_freq(*args), rtol=1e-14, atol=0)
     assert math.isclose(gain, orc.yarn_logit_gain(args[1]), rel_tol=1e-14)
+    # The ready logit scale (binary32) is the gain over sqrt(d).
+    ref = orc.yarn_logit_gain(args[1]) / math.sqrt(512)
+    assert abs(scale - ref) <= ref * 2.0 ** -24
+    _, _, s128 = binding.rope_yarn(*args, d=128)
+    assert abs(s128 - 2 * ref) <= 2 * ref * 2.0 ** -24
 
 
 @pytest.mark.parametrize("args,code", [((63, 16.0, 32.0, 1.0, 65536.0), 2),
@@ -174,7 +179,11 @@ def test_yarn_argument_checks(L, args, code):
     with pytest.raises(binding.CsaError) as e:
         binding.rope_yarn(*args)
     assert e.value.status == code
-    assert L.csa_rope_yarn(64, 1e4, 16.0, 32.0, 1.0, 65536.0, None, None) == 1
+    assert L.csa_rope_yarn(64, 1e4, 16.0, 32.0, 1.0, 65536.0, 512, None, None, None) == 1
+    tab = (C.c_double * 32)()
+    sc = C.c_float()
+    assert L.csa_rope_yarn(64, 1e4, 16.0, 32.0, 1.0, 65536.0, 0, tab, None, C.byref(sc)) == 1
+    assert L.csa_rope_yarn(64, 1e4, 16.0, 32.0, 1.0, 65536.0, 0, tab, None, None) == 0
 
 
 # ------------------------------------------- bench accounting (no GPU) --
@@ -211,7 +220,7 @@ def test_params_for_applies_yarn_to_a_yarn_workload(L, orc):
     p = binding.params_for(w)
     tab = np.array([p.rope_inv_freq[j] for j in range(w.rope_dim // 2)])
     assert np.allclose(tab, orc.yarn_inv_freq(w.rope_dim, *w.yarn), rtol=1e-14, atol=0)
-    assert math.isclose(p.softmax_scale, orc.yarn_logit_gain(w.yarn[0]) / math.sqrt(w.d),
-                        rel_tol=1e-6)
+    ref = orc.yarn_logit_gain(w.yarn[0]) / math.sqrt(w.d)
+    assert abs(p.softmax_scale - ref) <= ref * 2.0 ** -24
     plain = binding.params_for(configs.CSA_128K)
     assert not plain.rope_inv_freq and plain.softmax_scale == 0.0

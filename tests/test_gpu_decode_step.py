@@ -14,7 +14,8 @@ import pytest
 import torch
 
 from compressed_sparse_kv_04_b200 import binding, configs, synth
-from gpuhelp import assert_attention_close, assert_bf16_storage_close, bits8, bits16, f32
+from gpuhelp import (assert_attention_close, assert_bf16_storage_close, assert_lse_close, bits8,
+                     bits16, f32)
 from test_gpu_compress_index import check_keys
 
 pytestmark = pytest.mark.gpu
@@ -33,10 +34,7 @@ def _to_bf16(bits):
 
 
 def _check_lse(lse, rlse):
-    gl = f32(lse).astype(np.float64)
-    fin = np.isfinite(rlse)
-    assert np.array_equal(np.isfinite(gl), fin)
-    assert np.allclose(gl[fin], rlse[fin], rtol=0, atol=2e-2), np.abs(gl[fin] - rlse[fin]).max()
+    assert_lse_close(f32(lse), rlse, "decode-step LSE")
 
 
 def test_csa_decode_loop(orc):

@@ -15,7 +15,8 @@ import pytest
 import torch
 
 from compressed_sparse_kv_04_b200 import binding, configs, synth
-from gpuhelp import assert_attention_close, assert_bf16_storage_close, bits8, bits16, f32
+from gpuhelp import (assert_attention_close, assert_bf16_storage_close, assert_lse_close, bits8,
+                     bits16, f32)
 
 pytestmark = pytest.mark.gpu
 
@@ -189,7 +190,7 @@ def check_hca_prefill(orc, w, r, rows):
     assert np.isfinite(got).all()
     assert_attention_close(got, ref[0], "HCA prefill attention")
     gl, rl = r["lse"][rows], rlse[0]
-    assert np.allclose(gl, rl, rtol=0, atol=2e-2), np.abs(gl - rl).max()
+    assert_lse_close(gl, rl, "HCA prefill LSE")
 
 
 @pytest.mark.parametrize("P,T,gamma", [(128 * 10, 300, False), (0, 260, True), (128 * 3, 128, False)])

@@ -525,3 +525,75 @@ def test_frequency_table_reaches_compression_and_attention(orc):
     assert np.allclose(out, base, rtol=1e-9, atol=1e-9) and np.allclose(l2, lb, rtol=1e-9, atol=1e-9)
     plain, _ = orc.mqa(q, pos, kv_c, kv_tok, sink, m, W, r_dim, sel, cnt)
     assert not np.allclose(plain, base, rtol=1e-6, atol=1e-6)
+
+
+# --------------------------------- joint softmax over entries and window ---
+def _rms(x, gamma=None, eps=1e-6):
+    y = x / np.sqrt(np.mean(x * x, axis=-1, keepdims=True) + eps)
+    return y if gamma is None else y * gamma.astype(np.float64)
+
+
+@pytest.mark.parametrize("r_dim", [0, 16])
+def test_joint_softmax_over_entries_window_and_sink(orc, r_dim):
+    # Selected compressed entries and window tokens share ONE softmax whose
+    # denominator also holds e^z (the sink), and the output is rotated back
+    # by the query position.  Written out here as textbook attention over the
+    # concatenated key list [entries (as stored); RMSNorm'd, rotated window],
+    # with the sink as one extra logit that has no value vector.
+    B, Q, H, D, L, m, W = 1, 1, 4, 32, 64, 4, 9
+    q, kv_tok, kv_c, sink = _mqa_case(B, Q, H, D, L, m, 51)
+    sink = np.array([0.7, -1.5, 2.5, -0.2], np.float32)
+    gq = (1 + 0.2 * rng(52).standard_normal(D)).astype(np.float32)
+    gk = (1 + 0.2 * rng(53).standard_normal(D)).astype(np.float32)
+    pos = 58  # n_vis = 14; window = tokens 50..58
+    sel = np.array([[[2, 7, 11, 13, -1]]], np.int32)
+    cnt = np.array([[4]], np.int32)
+    out, lse = orc.mqa(q, np.array([[pos]]), kv_c, kv_tok, sink, m, W, r_dim, sel, cnt, gq, gk)
+
+    ents = orc.bf16_decode(kv_c)[0, [2, 7, 11, 13]]
+    toks = np.arange(pos - W + 1, pos + 1)
+    win = _rms(orc.bf16_decode(kv_tok)[0, toks], gk)
+    if r_dim:
+        win = np.stack([_rotate(win[j], float(t), r_dim) for j, t in enumerate(toks)])
+    keys = np.concatenate([ents, win], 0)  # K = V
+    qh = _rms(orc.bf16_decode(q)[0, 0], gq)
+    if r_dim:
+        qh = _rotate(qh, float(pos), r_dim)
+    logits = qh @ keys.T / math.sqrt(D)                       # [H, 4 + W]
+    full = np.concatenate([logits, sink.astype(np.float64)[:, None]], 1)
+    ref_lse = logsumexp(full, axis=1)
+    p = np.exp(logits - ref_lse[:, None])                      # sink column dropped
+    ref = p @ keys
+    if r_dim:
+        ref = _rotate(ref, -float(pos), r_dim)
+    assert np.allclose(out[0, 0], ref, rtol=1e-12, atol=1e-12)
+    assert np.allclose(lse[0, 0], ref_lse, rtol=1e-13, atol=1e-13)
+    # Two separate softmaxes (entries alone, window alone) averaged would be
+    # a different number: the case does distinguish the readings.
+    def branch(k):
+        lg = qh @ k.T / math.sqrt(D)
+        pw = np.exp(lg - lg.max(1, keepdims=True))
+        return (pw / pw.sum(1, keepdims=True)) @ k
+    assert not np.allclose(ref, 0.5 * (branch(ents) + branch(win)), rtol=1e-3, atol=1e-3)
+
+
+def test_joint_softmax_without_sink_is_sdpa_over_concatenated_keys(orc):
+    # Sink -inf, r = 0: plain scaled-dot-product attention (torch, fp64) over
+    # the selected entries followed by the window tokens.
+    B, Q, H, D, L, m, W = 1, 1, 8, 64, 96, 4, 16
+    q, kv_tok, kv_c, sink = _mqa_case(B, Q, H, D, L, m, 54)
+    sink[:] = -np.inf
+    pos = 90  # n_vis = 22; window = tokens 75..90
+    idx = [0, 5, 9, 17, 21]
+    sel = np.array([[idx + [-1, -1, -1]]], np.int32)
+    cnt = np.array([[len(idx)]], np.int32)
+    out, lse = orc.mqa(q, np.array([[pos]]), kv_c, kv_tok, sink, m, W, 0, sel, cnt)
+    ents = torch.from_numpy(orc.bf16_decode(kv_c)[0, idx])
+    win = F.rms_norm(torch.from_numpy(orc.bf16_decode(kv_tok)[0, pos - W + 1: pos + 1]), (D,),
+                     eps=1e-6)
+    keys = torch.cat([ents, win], 0)
+    qh = F.rms_norm(torch.from_numpy(orc.bf16_decode(q)[0, 0]), (D,), eps=1e-6)
+    ref = F.scaled_dot_product_attention(qh[None], keys[None], keys[None])[0]
+    assert np.allclose(out[0, 0], ref.numpy(), rtol=1e-12, atol=1e-12)
+    assert np.allclose(lse[0, 0], torch.logsumexp(qh @ keys.T / math.sqrt(D), 1).numpy(),
+                       rtol=1e-13, atol=1e-13)
