@@ -11,16 +11,20 @@ the whole hot path over one batch:
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
     python bench.py --impl reference ...   (the fp64 CPU oracle, same metric)
 
-Timing: W untimed warm-up steps, then exactly K steps replayed as CUDA graphs,
-bracketed by a barrier and torch.cuda.synchronize() on both sides, CUDA
-events on the launching stream, max over ranks.  Inputs rotate over R
-independent device-resident sets whose combined per-step traffic exceeds
-four times the 126 MB L2, so every step reads its data from HBM.  A second,
-instrumented pass over the same sets records CUDA events between the stages
-of every step; it gives each kernel's average launch time, from which the
-dominant kernel's roofline fraction is computed.  The e2e figure runs the
-same steps through the same calls with the step's new inputs copied from
+Timing: W untimed warm-up steps (plus one untimed replay of every CUDA graph
+the timed steps replay), then exactly K steps replayed as CUDA graphs of the
+public step call (csa_decode_step / hca_decode_step), bracketed by a barrier
+and torch.cuda.synchronize() on both sides, CUDA events on the launching
+stream, max over ranks.  Inputs rotate over R independent device-resident
+sets whose combined per-step traffic exceeds four times the 126 MB L2, so
+every step reads its data from HBM.  A second pass over the same sets runs
+each step as separate stage calls with CUDA events between them; it gives
+each kernel's average launch time, from which the dominant kernel's
+roofline fraction is computed.  The e2e figure runs the same steps as
+direct public calls (no graph) with the step's new inputs copied from
 pinned host memory and the output copied back, inside the timed region.
+A default run then times the other decode workloads (1M-token HCA and CSA)
+and the CSA prefill chunk the same way and reports them under "workloads".
 """
 from __future__ import annotations
 
@@ -256,6 +260,7 @@ class Decode:
                                  kv_c_src)
         tail = max(w.W, w.m)
         self.tail = tail
+        op_step = binding.OP_CSA_DECODE_STEP if w.csa else binding.OP_HCA_DECODE_STEP
         self.sets = []
         for r in range(R):
             s = {}
@@ -265,6 +270,7 @@ class Decode:
             s["kv_c"] = kv_c_src.clone()
             s["q"] = synth.normal_bf16((B, w.H, d), w.seed + 1000 + r, "q", device)
             s["out"] = torch.empty(B, w.H, d, dtype=torch.bfloat16, device=device)
+            s["ws_step"] = binding.workspace(self.p, op_step, 1, N, device)
             if w.csa:
                 s["idx_tok"] = torch.empty(B, L, w.D_I, dtype=torch.bfloat16, device=device)
                 s["idx_tok"][:, L - tail:] = idx_src[:, L - tail:]
@@ -283,7 +289,24 @@ class Decode:
         self.status = torch.zeros(1, dtype=torch.int32, device=device)
         torch.cuda.synchronize()
 
-    # The stages of one step, in order; each is one library call.
+    def step(self, s):
+        """One decode step of the whole batch: ONE public call (newest-block
+        compression, then indexer, top-k and sparse attention for CSA, or
+        dense attention for HCA)."""
+        b, w, p = self.binding, self.w, self.p
+        if w.csa:
+            b.csa_decode_step(p, self.pos, s["kv_tok"], s["idx_tok"], self.w_s, self.b_pos, None,
+                              self.w_si, self.b_pi, s["kv_c"], s["key"], s["ksc"], s["q"],
+                              s["q_idx"].view(w.B, w.H_I, w.D_I), s["q_scale"].view(w.B, w.H_I),
+                              s["w"].view(w.B, w.H_I), self.sink, s["tidx"].view(w.B, w.k),
+                              s["tcnt"].view(w.B), s["out"], ws=s["ws_step"],
+                              dev_status=self.status)
+        else:
+            b.hca_decode_step(p, self.pos, s["kv_tok"], self.w_s, self.b_pos, None, s["kv_c"],
+                              s["q"], self.sink, s["out"], ws=s["ws_step"], dev_status=self.status)
+
+    # The same step as separate calls, one per stage (for the per-stage
+    # timing pass: events between the calls).
     def stages(self, s):
         b, w, p, N = self.binding, self.w, self.p, self.w.N_c
         st = self.status
@@ -316,35 +339,30 @@ class Decode:
         # workloads' rows always have several splits, so the merge runs)
         return 5 if self.w.csa else 3
 
-    def capture(self, instrumented=False):
-        """One CUDA graph per input set (optionally with stage events)."""
+    def _warm(self):
         torch = self.torch
-        graphs, events = [], []
         stream = torch.cuda.Stream()
         stream.wait_stream(torch.cuda.current_stream())
-        with torch.cuda.stream(stream):
-            for s in self.sets:  # warm the launch path outside capture
+        with torch.cuda.stream(stream):  # warm the launch path outside capture
+            for s in self.sets:
+                self.step(s)
                 for _, fn in self.stages(s):
                     fn()
         torch.cuda.current_stream().wait_stream(stream)
         torch.cuda.synchronize()
+        return stream
+
+    def capture_steps(self):
+        """One CUDA graph per input set holding one step (one public call)."""
+        torch = self.torch
+        stream = self._warm()
+        graphs = []
         for s in self.sets:
             g = torch.cuda.CUDAGraph()
-            ev = []
             with torch.cuda.graph(g, stream=stream):
-                if instrumented:
-                    e = torch.cuda.Event(enable_timing=True, external=True)
-                    e.record()
-                    ev.append(e)
-                for _, fn in self.stages(s):
-                    fn()
-                    if instrumented:
-                        e = torch.cuda.Event(enable_timing=True, external=True)
-                        e.record()
-                        ev.append(e)
+                self.step(s)
             graphs.append(g)
-            events.append(ev)
-        return graphs, events
+        return graphs
 
     def capture_cycle(self):
         """One CUDA graph holding a step of every input set in turn (R
@@ -358,16 +376,133 @@ class Decode:
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=stream):
             for s in self.sets:
-                for _, fn in self.stages(s):
-                    fn()
+                self.step(s)
         return g
 
-    def step_input_bytes(self):
-        w = self.w
-        b = w.B * w.H * w.d * 2 + w.B * w.m * w.d * 2
-        if w.csa:
-            b += w.B * w.H_I * (w.D_I + 8) + w.B * w.m * w.D_I * 2
-        return b
+    def capture_instrumented(self):
+        """One graph per input set: the step as separate stage calls with an
+        event between consecutive stages."""
+        torch = self.torch
+        stream = self._warm()
+        graphs, events = [], []
+        for s in self.sets:
+            g = torch.cuda.CUDAGraph()
+            ev = []
+            with torch.cuda.graph(g, stream=stream):
+                e = torch.cuda.Event(enable_timing=True, external=True)
+                e.record()
+                ev.append(e)
+                for _, fn in self.stages(s):
+                    fn()
+                    e = torch.cuda.Event(enable_timing=True, external=True)
+                    e.record()
+                    ev.append(e)
+            graphs.append(g)
+            events.append(ev)
+        return graphs, events
+
+
+def measure_decode(w, K, W, dev, barrier, rmax, rsum, world, rotate=0, e2e=True):
+    """Times K decode steps of workload w (after W warm-up steps); returns
+    the per-workload record (throughput, step and dominant-kernel rooflines,
+    per-stage times, e2e)."""
+    import torch
+    ab = algorithmic_bytes(w)
+    R = rotate or max(2, math.ceil(4 * L2_BYTES / ab["step"]) + 1)
+    st = Decode(w, R, dev)
+    graphs = st.capture_steps()
+    cycle = st.capture_cycle()
+    torch.cuda.synchronize()
+
+    def plan(n):
+        """The graphs that n consecutive steps replay: whole R-step cycles,
+        then single-step graphs."""
+        return [cycle] * (n // R) + [graphs[i] for i in range(n % R)]
+
+    # Warm-up: W steps, then one untimed replay of every graph the timed
+    # region replays and the W steps did not (so no first replay, with its
+    # one-time upload, falls inside the timed region).
+    warm = plan(W)
+    for g in warm:
+        g.replay()
+    timed = plan(K)
+    for g in timed:
+        if not any(g is x for x in warm):
+            g.replay()
+            warm.append(g)
+    barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for g in timed:
+        g.replay()
+    e1.record()
+    barrier()
+    elapsed = e0.elapsed_time(e1)
+    value, t_max = aggregate(w.B * K, elapsed, world, rmax, rsum)
+    status = int(st.status.item())
+    del graphs, cycle
+
+    # Per-stage pass: K steps as separate stage calls with events between
+    # them (the events break the overlap between kernels, so the stage times
+    # add up to more than a step).
+    igraphs, ievents = st.capture_instrumented()
+    names = [n for n, _ in st.stages(st.sets[0])]
+    sums = {n: 0.0 for n in names}
+    for _ in range(max(1, W)):  # warm the instrumented graphs too
+        for g in igraphs:
+            g.replay()
+    torch.cuda.synchronize()
+    done = 0
+    while done < K:
+        batch = min(R, K - done)
+        for j in range(batch):
+            igraphs[j].replay()
+        torch.cuda.synchronize()
+        for j in range(batch):
+            ev = ievents[j]
+            for n, a, b in zip(names, ev[:-1], ev[1:]):
+                sums[n] += a.elapsed_time(b)
+        done += batch
+    stage_ms = {n: sums[n] / K for n in names}
+    del igraphs, ievents
+
+    e2e_rec = run_e2e(st, K, W, barrier, rmax, rsum, world) if e2e else None
+
+    peaks = measured_peaks()
+    dom = max(stage_ms, key=stage_ms.get)
+    dom_ms = stage_ms[dom]
+    # the attention call is the attention kernel + the split merge
+    bytes_dom = ab["mqa"] + ab["combine"] if dom == "mqa" else ab[dom]
+    achieved = bytes_dom / (dom_ms * 1e-3) / 1e9
+    ms_per_step = t_max / K
+    rec = {
+        "value": round(value, 1), "unit": "query-tokens/s", "ms_per_step": round(ms_per_step, 6),
+        "config": {"workload": w.name, "batch": w.B, "context": w.L, "compressed_entries": w.N_c,
+                   "m": w.m, "heads": w.H, "head_dim": w.d, "window": w.W,
+                   "top_k": w.k if w.csa else None,
+                   "indexer": [w.H_I, w.D_I] if w.csa else None,
+                   "call": "csa_decode_step" if w.csa else "hca_decode_step",
+                   "l2": l2_note(R, ab["step"]),
+                   "warmup": "W steps plus one untimed replay of every graph the timed steps "
+                             "replay"},
+        "roofline": {"bound": "hbm", "kernel": dom, "achieved": round(achieved, 1),
+                     "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": round(achieved / peaks["hbm_gbs"], 4),
+                     "peak_source": peaks["source"], "traffic": stored_traffic(dom, w.name),
+                     "algorithmic_bytes_per_launch": bytes_dom, "avg_launch_ms": round(dom_ms, 6)},
+        "step_roofline": {"algorithmic_bytes": ab["step"],
+                          "achieved_GBps": round(ab["step"] / (ms_per_step * 1e-3) / 1e9, 1),
+                          "frac": round(ab["step"] / (ms_per_step * 1e-3) / 1e9 /
+                                        peaks["hbm_gbs"], 4),
+                          "peak": peaks["hbm_gbs"], "peak_source": peaks["source"]},
+        "kernels_ms": {k: round(v, 6) for k, v in stage_ms.items()},
+        "gpu_launches": st.launches_per_step() * K,
+        "device_status": status,
+    }
+    if e2e_rec is not None:
+        rec["e2e"] = e2e_rec
+    return rec, st
 
 
 def run_gpu(args):
@@ -388,143 +523,104 @@ def run_gpu(args):
     barrier, rmax, rsum = make_reducers(world, dev)
 
     w = workload_for_rank(configs.BY_NAME[args.workload], rank)
-    ab = algorithmic_bytes(w)
-    R = args.rotate or max(2, math.ceil(4 * L2_BYTES / ab["step"]) + 1)
-    st = Decode(w, R, dev)
-    graphs, _ = st.capture(instrumented=False)
-    cycle = st.capture_cycle()
     K, W = args.steps, args.warmup
-    torch.cuda.synchronize()
-
-    def run_steps(n):
-        """n consecutive steps: whole R-step cycles, then single-step graphs."""
-        for _ in range(n // R):
-            cycle.replay()
-        for i in range(n % R):
-            graphs[i].replay()
-
+    extras = {}
     with ClockSampler(local) as clocks:
-        run_steps(W)
-        barrier()
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        e0.record()
-        run_steps(K)
-        e1.record()
-        barrier()
-        elapsed = e0.elapsed_time(e1)
-        value, t_max = aggregate(w.B * K, elapsed, world, rmax, rsum)
-        status = int(st.status.item())
-
-        # Instrumented pass: stage durations of K steps (events inside graphs).
-        igraphs, ievents = st.capture(instrumented=True)
-        names = [n for n, _ in st.stages(st.sets[0])]
-        sums = {n: 0.0 for n in names}
-        done = 0
-        while done < K:
-            batch = min(R, K - done)
-            for j in range(batch):
-                igraphs[j].replay()
-            torch.cuda.synchronize()
-            for j in range(batch):
-                ev = ievents[j]
-                for n, a, b in zip(names, ev[:-1], ev[1:]):
-                    sums[n] += a.elapsed_time(b)
-            done += batch
-        stage_ms = {n: sums[n] / K for n in names}
-
-        # e2e: the step's new inputs from pinned host memory, output back.
-        e2e = None
-        if not args.no_e2e:
-            e2e = run_e2e(st, graphs, K, W, barrier, rmax, rsum, world)
+        rec, st = measure_decode(w, K, W, dev, barrier, rmax, rsum, world, args.rotate,
+                                 e2e=not args.no_e2e)
+        cpu = None
+        if not args.no_cpu_baseline and world == 1:
+            cpu = cpu_baseline(w, st, args.cpu_seconds)
+        del st
+        torch.cuda.empty_cache()
+        # The other decode workloads (and the prefill chunk) in the same run,
+        # each with its own time and rooflines.
+        if not args.no_extra:
+            for name in EXTRA_WORKLOADS:
+                if name == w.name:
+                    continue
+                wx = workload_for_rank(configs.BY_NAME[name], rank)
+                if wx.kind == "csa_prefill":
+                    extras[name] = measure_prefill(wx, K, W, dev)
+                else:
+                    r, sx = measure_decode(wx, K, W, dev, barrier, rmax, rsum, world, 0,
+                                           e2e=False)
+                    extras[name] = r
+                    del sx
+                torch.cuda.empty_cache()
     clk = clocks.summary()
-
-    # Dominant kernel (largest average stage time) and its roofline.
-    peaks = measured_peaks()
-    dom = max(stage_ms, key=stage_ms.get)
-    dom_kernel = dom
-    dom_ms = stage_ms[dom]
-    if dom == "mqa":
-        # the attention call is the pair kernel + the combine kernel
-        bytes_dom = ab["mqa"] + ab["combine"]
-    else:
-        bytes_dom = ab[dom]
-    achieved = bytes_dom / (dom_ms * 1e-3) / 1e9
-    traffic = stored_traffic(dom_kernel, w.name)
-    launches = st.launches_per_step() * K
 
     if rank != 0:
         if world > 1:
             dist.destroy_process_group()
         return
-    ms_per_step = t_max / K
     line = {
         "metric": METRIC,
-        "value": round(value, 1),
+        "value": rec["value"],
         "unit": "query-tokens/s",
         "n_gpus": world,
         "steps": K,
         "warmup": W,
-        "ms_per_step": round(ms_per_step, 6),
+        "ms_per_step": rec["ms_per_step"],
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
         "dtype": "bf16+e4m3",
         "data": "synthetic (seeded N(0,1) token streams, random query/indexer inputs)",
-        "config": {"workload": w.name, "batch": w.B, "context": w.L, "compressed_entries": w.N_c,
-                   "m": w.m, "heads": w.H, "head_dim": w.d, "window": w.W,
-                   "top_k": w.k if w.csa else None, "indexer": [w.H_I, w.D_I] if w.csa else None,
-                   "parallelism": f"replicas x{world} (independent sequences per GPU)",
-                   "l2": l2_note(R, ab["step"])},
-        "roofline": {"bound": "hbm", "kernel": dom_kernel, "achieved": round(achieved, 1),
-                     "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                     "frac": round(achieved / peaks["hbm_gbs"], 4),
-                     "peak_source": peaks["source"], "traffic": traffic,
-                     "algorithmic_bytes_per_launch": bytes_dom,
-                     "avg_launch_ms": round(dom_ms, 6)},
-        "step_roofline": {"algorithmic_bytes": ab["step"],
-                          "achieved_GBps": round(ab["step"] / (ms_per_step * 1e-3) / 1e9, 1),
-                          "frac": round(ab["step"] / (ms_per_step * 1e-3) / 1e9 / peaks["hbm_gbs"], 4)},
-        "kernels_ms": {k: round(v, 6) for k, v in stage_ms.items()},
-        "e2e": e2e,
-        "gpu_launches": launches,
+        "config": dict(rec["config"],
+                       parallelism=f"replicas x{world} (independent sequences per GPU)"),
+        "roofline": rec["roofline"],
+        "step_roofline": rec["step_roofline"],
+        "kernels_ms": rec["kernels_ms"],
+        "e2e": rec.get("e2e"),
+        "gpu_launches": rec["gpu_launches"],
         "clocks": clk,
-        "device_status": status,
+        "device_status": rec["device_status"],
     }
-    if not args.no_cpu_baseline and world == 1:
-        line["cpu_baseline"] = cpu_baseline(w, st, args.cpu_seconds)
+    if extras:
+        line["workloads"] = extras
+    if cpu is not None:
+        line["cpu_baseline"] = cpu
     print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
 
 
-def run_e2e(st, graphs, K, W, barrier, rmax, rsum, world):
-    """Same steps; the new query and token rows come from pinned host memory
-    and the output goes back to it, inside the timed region."""
+# The workloads timed after the primary one in a default run.
+EXTRA_WORKLOADS = ["hca_decode_1m_b8", "csa_decode_1m_b4", "csa_prefill_4096_after_65536"]
+
+
+def run_e2e(st, K, W, barrier, rmax, rsum, world):
+    """The same K steps through the public call (csa_decode_step /
+    hca_decode_step, each step a direct call: argument checks and launches
+    included, no graph), with the step's new query and token rows copied
+    from pinned host memory and its output copied back to pinned host
+    memory, all inside the timed region."""
     torch = st.torch
     w, R = st.w, st.R
     L, m = w.L, w.m
     hq = [s["q"].cpu().pin_memory() for s in st.sets]
     hkv = [s["kv_tok"][:, L - m:].cpu().pin_memory() for s in st.sets]
-    hout = torch.empty_like(st.sets[0]["out"], device="cpu").pin_memory()
+    hout = [torch.empty_like(s["out"], device="cpu").pin_memory() for s in st.sets]
     extra = []
     if w.csa:
-        extra = [(s, s["q_idx"].cpu().pin_memory(), s["q_scale"].cpu().pin_memory(),
+        extra = [(s["q_idx"].cpu().pin_memory(), s["q_scale"].cpu().pin_memory(),
                   s["w"].cpu().pin_memory(), s["idx_tok"][:, L - m:].cpu().pin_memory())
                  for s in st.sets]
     h2d = sum(t.numel() * t.element_size() for t in (hq[0], hkv[0]))
     if w.csa:
-        h2d += sum(t.numel() * t.element_size() for t in extra[0][1:])
-    d2h = hout.numel() * hout.element_size()
+        h2d += sum(t.numel() * t.element_size() for t in extra[0])
+    d2h = hout[0].numel() * hout[0].element_size()
 
     # Copies run on their own streams: the inputs of step i+1 travel while
     # step i computes, and the output of step i returns while step i+1
-    # computes (each step has its own input set, so nothing is overwritten
-    # while in use).
+    # computes (each step has its own input set and its own host output
+    # buffer, so nothing is overwritten while in use).
     comp = torch.cuda.current_stream()
     up, down = torch.cuda.Stream(), torch.cuda.Stream()
     copied = [torch.cuda.Event() for _ in range(R)]
     done = [torch.cuda.Event() for _ in range(R)]
+    fetched = [torch.cuda.Event() for _ in range(R)]
     used = [False] * R
 
     def upload(i):
@@ -536,7 +632,7 @@ def run_e2e(st, graphs, K, W, barrier, rmax, rsum, world):
             s["q"].copy_(hq[r], non_blocking=True)
             s["kv_tok"][:, L - m:].copy_(hkv[r], non_blocking=True)
             if w.csa:
-                _, a, b, c, d = extra[r]
+                a, b, c, d = extra[r]
                 s["q_idx"].copy_(a, non_blocking=True)
                 s["q_scale"].copy_(b, non_blocking=True)
                 s["w"].copy_(c, non_blocking=True)
@@ -546,12 +642,15 @@ def run_e2e(st, graphs, K, W, barrier, rmax, rsum, world):
     def compute(i):
         r = i % R
         comp.wait_event(copied[r])
-        graphs[r].replay()
+        if used[r]:
+            comp.wait_event(fetched[r])  # the set's previous output has left
+        st.step(st.sets[r])
         done[r].record(comp)
         used[r] = True
         with torch.cuda.stream(down):
             down.wait_event(done[r])
-            hout.copy_(st.sets[r]["out"], non_blocking=True)
+            hout[r].copy_(st.sets[r]["out"], non_blocking=True)
+            fetched[r].record(down)
 
     def run(n):
         up.wait_stream(comp)
@@ -572,7 +671,9 @@ def run_e2e(st, graphs, K, W, barrier, rmax, rsum, world):
     barrier()
     val, _ = aggregate(w.B * K, e0.elapsed_time(e1), world, rmax, rsum)
     return {"value": round(val, 1), "unit": "query-tokens/s", "h2d_bytes_per_step": h2d,
-            "d2h_bytes_per_step": d2h}
+            "d2h_bytes_per_step": d2h,
+            "path": "direct public call per step (no graph); inputs from pinned host memory, "
+                    "output to pinned host memory, inside the timed region"}
 
 
 # ---------------------------------------------------------------- prefill --
@@ -590,16 +691,13 @@ def prefill_work(w):
     return fp8, bf16
 
 
-def run_prefill(args):
+def measure_prefill(w, K, W, dev):
     """One CSA prefill chunk per step (csa_prefill_chunk: compression of the
     chunk's blocks, causal indexer, top-k, sparse attention), B = 1.  The
     step's scores alone (T x N_cap fp32) exceed the L2, so no rotation."""
     import torch
 
     from compressed_sparse_kv_04_b200 import binding, synth
-    w = configs.CSA_PREFILL
-    dev = torch.device("cuda", 0)
-    torch.cuda.set_device(dev)
     b = binding
     L_cap = w.P + w.T
     N_cap = -(-L_cap // w.m)
@@ -642,25 +740,23 @@ def run_prefill(args):
         torch.cuda.synchronize()
         return e0.elapsed_time(e1) / n
 
-    K, W = args.steps, args.warmup
-    with ClockSampler(0) as clocks:
-        for _ in range(W):
-            chunk()
-        torch.cuda.synchronize()
-        ms = timed(chunk, K)
-        ms_idx = timed(index_only, K)
+    for _ in range(W):
+        chunk()
+        index_only()
+    torch.cuda.synchronize()
+    ms = timed(chunk, K)
+    ms_idx = timed(index_only, K)
     fp8, bf16 = prefill_work(w)
     peaks = measured_peaks()
     fp8_peak = 2.0 * peaks["bf16_tflops"]  # dense FP8 = 2 x dense BF16 (nominal ratio)
     idx_tf = fp8 / (ms_idx * 1e-3) / 1e12
     t_ideal = fp8 / (fp8_peak * 1e12) + bf16 / (peaks["bf16_tflops"] * 1e12)
-    line = {
+    return {
         "metric": PREFILL_METRIC, "value": round(w.T / (ms * 1e-3), 1), "unit": "query-tokens/s",
-        "n_gpus": 1, "steps": K, "warmup": W, "ms_per_step": round(ms, 4),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "e4m3+bf16",
-        "data": "synthetic (seeded N(0,1) token streams, random query/indexer inputs)",
+        "ms_per_step": round(ms, 4), "dtype": "e4m3+bf16",
         "config": {"workload": w.name, "prior_tokens": w.P, "chunk_tokens": w.T, "heads": w.H,
                    "head_dim": w.d, "top_k": w.k, "indexer": [w.H_I, w.D_I],
+                   "call": "csa_prefill_chunk",
                    "l2": "no rotation: the chunk's scores alone (T x N_cap fp32) exceed the L2"},
         "roofline": {"bound": "tensor", "kernel": "index_scores", "achieved": round(idx_tf, 1),
                      "peak": round(fp8_peak, 1), "unit": "TFLOP/s",
@@ -671,9 +767,23 @@ def run_prefill(args):
                           "ideal_ms": round(t_ideal * 1e3, 4),
                           "frac": round(t_ideal * 1e3 / ms, 4)},
         # per chunk: compress, indexer, top-k, attention (one split per row:
-        # no merge); plus the separately timed indexer launch
-        "gpu_launches": 5 * K, "clocks": clocks.summary(), "device_status": int(status.item()),
+        # no merge)
+        "gpu_launches": 4 * K, "device_status": int(status.item()),
     }
+
+
+def run_prefill(args):
+    import torch
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    K, W = args.steps, args.warmup
+    with ClockSampler(0) as clocks:
+        rec = measure_prefill(configs.CSA_PREFILL, K, W, dev)
+    line = dict(rec, n_gpus=1, steps=K, warmup=W, higher_is_better=True, scaling="weak",
+                vs_baseline=None,
+                data="synthetic (seeded N(0,1) token streams, random query/indexer inputs)",
+                clocks=clocks.summary())
+    line["gpu_launches"] = rec["gpu_launches"] + K  # plus the separately timed indexer
     print(json.dumps(line), flush=True)
 
 
@@ -692,9 +802,8 @@ def hca_prefill_flops(w):
 
 def run_hca_prefill(args):
     """One HCA prefill chunk per step (hca_prefill_chunk: compression of the
-    chunk's blocks, dense attention per query, merge), B = 1.  The step's
-    split partials and output (2 x T x H x d x 2 bytes) exceed the L2, so no
-    rotation."""
+    chunk's blocks, dense attention per query), B = 1.  The step's output
+    (T x H x d x 2 bytes) exceeds the L2, so no rotation."""
     import torch
 
     from compressed_sparse_kv_04_b200 import binding as b
@@ -743,8 +852,8 @@ def run_hca_prefill(args):
         "data": "synthetic (seeded N(0,1) token streams and queries)",
         "config": {"workload": w.name, "prior_tokens": w.P, "chunk_tokens": w.T, "heads": w.H,
                    "head_dim": w.d, "m": w.m, "window": w.W,
-                   "l2": "no rotation: the chunk's partials and output exceed the L2"},
-        "roofline": {"bound": "tensor", "kernel": "hca_prefill_chunk (compress + attention + merge)",
+                   "l2": "no rotation: the chunk's output exceeds the L2"},
+        "roofline": {"bound": "tensor", "kernel": "hca_prefill_chunk (compress + attention)",
                      "achieved": round(tf, 1), "peak": round(peaks["bf16_tflops"], 1),
                      "unit": "TFLOP/s", "frac": round(tf / peaks["bf16_tflops"], 4),
                      "peak_source": peaks["source"], "avg_launch_ms": round(ms, 4),
@@ -949,6 +1058,9 @@ def main(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="time only the primary workload (not the other decode workloads and "
+                         "the prefill chunk)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

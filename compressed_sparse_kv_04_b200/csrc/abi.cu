@@ -303,8 +303,9 @@ static csa_status index_common(const char* fn, const csa_params* p, int Q,
                                const uint8_t* q_idx, const float* q_scale, const float* w,
                                const uint8_t* idx_key, const float* idx_scale, int64_t N_cap,
                                const int64_t* pos_q, int64_t pos_base, float* scores,
-                               int32_t* dev_status, cudaStream_t stream) {
+                               int32_t* dev_status, cudaStream_t stream, int chained) {
   csa::IndexLaunch a{};
+  a.chained = chained;
   a.B = p->B;
   a.Q = Q;
   a.H_I = p->H_I;
@@ -329,8 +330,9 @@ static csa_status index_common(const char* fn, const csa_params* p, int Q,
 static csa_status topk_common(const char* fn, const csa_params* p, int Q, const float* scores,
                               int64_t N_cap, const int64_t* pos_q, int64_t pos_base,
                               int32_t* topk_idx, int32_t* topk_cnt, int32_t* dev_status,
-                              cudaStream_t stream) {
+                              cudaStream_t stream, int chained) {
   csa::TopkLaunch t{};
+  t.chained = chained;
   t.rows = p->B * Q;
   t.Q = Q;
   t.m = p->m;
@@ -352,12 +354,12 @@ static csa_status index_topk_common(const char* fn, const csa_params* p, int Q,
                                     const uint8_t* idx_key, const float* idx_scale,
                                     int64_t N_cap, const int64_t* pos_q, int64_t pos_base,
                                     int32_t* topk_idx, int32_t* topk_cnt, float* scores,
-                                    int32_t* dev_status, cudaStream_t stream) {
+                                    int32_t* dev_status, cudaStream_t stream, int chained) {
   csa_status st = index_common(fn, p, Q, q_idx, q_scale, w, idx_key, idx_scale, N_cap, pos_q,
-                               pos_base, scores, dev_status, stream);
+                               pos_base, scores, dev_status, stream, chained);
   if (st != CSA_OK) return st;
   return topk_common(fn, p, Q, scores, N_cap, pos_q, pos_base, topk_idx, topk_cnt, dev_status,
-                     stream);
+                     stream, 1);
 }
 
 static csa_status check_index_args(const char* fn, const csa_params* p, int Q, int64_t N_cap) {
@@ -404,7 +406,7 @@ csa_status lightning_index_topk(const csa_params* p, int Q, const uint8_t* q_idx
   }
   return index_topk_common(fn, p, Q, q_idx, q_scale, w, idx_key, idx_scale, N_cap, pos_q, 0,
                            topk_idx, topk_cnt, scores, dev_status,
-                           static_cast<cudaStream_t>(stream));
+                           static_cast<cudaStream_t>(stream), 0);
 }
 
 csa_status lightning_index_scores(const csa_params* p, int Q, const uint8_t* q_idx,
@@ -423,7 +425,7 @@ csa_status lightning_index_scores(const csa_params* p, int Q, const uint8_t* q_i
   REQ_PTR(scores);
   OPT_PTR4(dev_status);
   return index_common(fn, p, Q, q_idx, q_scale, w, idx_key, idx_scale, N_cap, pos_q, 0, scores,
-                      dev_status, static_cast<cudaStream_t>(stream));
+                      dev_status, static_cast<cudaStream_t>(stream), 0);
 }
 
 csa_status topk_select(const csa_params* p, int Q, const float* scores, int64_t N_cap,
@@ -438,7 +440,7 @@ csa_status topk_select(const csa_params* p, int Q, const float* scores, int64_t 
   REQ_PTR4(topk_cnt);
   OPT_PTR4(dev_status);
   return topk_common(fn, p, Q, scores, N_cap, pos_q, 0, topk_idx, topk_cnt, dev_status,
-                     static_cast<cudaStream_t>(stream));
+                     static_cast<cudaStream_t>(stream), 0);
 }
 
 static csa_status mqa_common(const char* fn, const csa_params* p, csa_op op, int rows, int Q,
@@ -447,7 +449,7 @@ static csa_status mqa_common(const char* fn, const csa_params* p, csa_op op, int
                              const int32_t* sel_cnt, const void* kv_tok, int64_t L_cap,
                              const float* sink, const float* gamma_q, const float* gamma_kv,
                              void* out, float* lse, void* ws, size_t ws_bytes,
-                             int32_t* dev_status, cudaStream_t stream) {
+                             int32_t* dev_status, cudaStream_t stream, int chained) {
   int splits = splits_for(p, op, rows, N_cap);
   size_t need = csa::mqa_workspace_bytes(rows, splits, p->H, p->d);
   if (!ws || ws_bytes < need)
@@ -485,6 +487,7 @@ static csa_status mqa_common(const char* fn, const csa_params* p, csa_op op, int
   a.part_ml = reinterpret_cast<float*>(static_cast<char*>(ws) +
                                        round_up((size_t)rows * splits * p->H * p->d * 2, 256));
   a.status = dev_status;
+  a.chained = chained;
   cudaError_t e = csa::launch_mqa(a, stream);
   if (e != cudaSuccess) return cuda_fail(fn, e);
   return CSA_OK;
@@ -533,7 +536,7 @@ csa_status sparse_mqa_decode(const csa_params* p, const void* q, const int64_t* 
   REQ_PTR4(topk_cnt);
   return mqa_common(fn, p, CSA_OP_SPARSE_MQA, p->B, 1, q, pos_q, 0, kv_c, N_cap, topk_idx,
                     topk_cnt, kv_tok, L_cap, sink, gamma_q, gamma_kv, out, lse, ws, ws_bytes,
-                    dev_status, static_cast<cudaStream_t>(stream));
+                    dev_status, static_cast<cudaStream_t>(stream), 0);
 }
 
 csa_status dense_mqa_decode(const csa_params* p, const void* q, const int64_t* pos_q,
@@ -547,7 +550,7 @@ csa_status dense_mqa_decode(const csa_params* p, const void* q, const int64_t* p
   if (st != CSA_OK) return st;
   return mqa_common(fn, p, CSA_OP_DENSE_MQA, p->B, 1, q, pos_q, 0, kv_c, N_cap, nullptr,
                     nullptr, kv_tok, L_cap, sink, gamma_q, gamma_kv, out, lse, ws, ws_bytes,
-                    dev_status, static_cast<cudaStream_t>(stream));
+                    dev_status, static_cast<cudaStream_t>(stream), 0);
 }
 
 csa_status csa_prefill_chunk(const csa_params* p, int64_t P, int T, const void* kv_tok,
@@ -603,14 +606,14 @@ csa_status csa_prefill_chunk(const csa_params* p, int64_t P, int T, const void* 
   float* scores = static_cast<float*>(ws);
   csa_params p1 = *p;
   st = index_topk_common(fn, &p1, T, q_idx, q_scale, w, idx_key, idx_scale, N_cap, nullptr, P,
-                         topk_idx, topk_cnt, scores, dev_status, s);
+                         topk_idx, topk_cnt, scores, dev_status, s, 1);
   if (st != CSA_OK) return st;
   // 4. Sparse MQA per query, each with its own causal window.
   char* rest = static_cast<char*>(ws) + scores_bytes(T, N_cap);
   size_t rest_bytes = ws_bytes - scores_bytes(T, N_cap);
   return mqa_common(fn, p, CSA_OP_SPARSE_MQA, T, T, q, nullptr, P, kv_c, N_cap, topk_idx,
                     topk_cnt, kv_tok, L_cap, sink, gamma_q, gamma_kv, out, nullptr, rest,
-                    rest_bytes, dev_status, s);
+                    rest_bytes, dev_status, s, 1);
 }
 
 csa_status csa_decode_step(const csa_params* p, const int64_t* pos_q, const void* kv_tok,
@@ -650,13 +653,13 @@ csa_status csa_decode_step(const csa_params* p, const int64_t* pos_q, const void
   // 2-3. Indexer and top-k over each sequence's visible entries.
   float* scores = static_cast<float*>(ws);
   st = index_topk_common(fn, p, 1, q_idx, q_scale, w, idx_key, idx_scale, N_cap, pos_q, 0,
-                         topk_idx, topk_cnt, scores, dev_status, s);
+                         topk_idx, topk_cnt, scores, dev_status, s, 1);
   if (st != CSA_OK) return st;
   // 4. Sparse MQA over the selection, the window and the sink.
   char* rest = static_cast<char*>(ws) + scores_bytes(p->B, N_cap);
   return mqa_common(fn, p, CSA_OP_SPARSE_MQA, p->B, 1, q, pos_q, 0, kv_c, N_cap, topk_idx,
                     topk_cnt, kv_tok, L_cap, sink, gamma_q, gamma_kv, out, lse, rest,
-                    ws_bytes - scores_bytes(p->B, N_cap), dev_status, s);
+                    ws_bytes - scores_bytes(p->B, N_cap), dev_status, s, 1);
 }
 
 csa_status hca_decode_step(const csa_params* p, const int64_t* pos_q, const void* kv_tok,
@@ -680,7 +683,7 @@ csa_status hca_decode_step(const csa_params* p, const int64_t* pos_q, const void
   if (st != CSA_OK) return st;
   return mqa_common(fn, p, CSA_OP_DENSE_MQA, p->B, 1, q, pos_q, 0, kv_c, N_cap, nullptr, nullptr,
                     kv_tok, L_cap, sink, gamma_q, gamma_kv, out, lse, ws, ws_bytes, dev_status,
-                    static_cast<cudaStream_t>(stream));
+                    static_cast<cudaStream_t>(stream), 1);
 }
 
 csa_status hca_prefill_chunk(const csa_params* p, int64_t P, int T, const void* kv_tok,
@@ -728,7 +731,7 @@ csa_status hca_prefill_chunk(const csa_params* p, int64_t P, int T, const void* 
   // 2. Dense MQA per query over its visible entries and its causal window.
   return mqa_common(fn, p, CSA_OP_DENSE_MQA, T, T, q, nullptr, P, kv_c, N_cap, nullptr, nullptr,
                     kv_tok, L_cap, sink, gamma_q, gamma_kv, out, lse, ws, ws_bytes, dev_status,
-                    static_cast<cudaStream_t>(stream));
+                    static_cast<cudaStream_t>(stream), 1);
 }
 
 }  // extern "C"

@@ -397,7 +397,7 @@ cudaError_t launch_compress(const CompressLaunch& c, cudaStream_t stream) {
   int maxdim = c.idx_tok && c.D_I > c.d ? c.D_I : c.d;
   size_t smem = G == 1 ? 0 : (size_t)kWarps * (maxdim + 2) * sizeof(float);
   dim3 grid((unsigned)grid_x, a.nstreams);
-  return launch_pdl(compress_kernel, grid, dim3(kThreads), smem, stream, 0, a);
+  return launch_pdl(compress_kernel, grid, dim3(kThreads), smem, stream, 0, c.chained, a);
 }
 
 }  // namespace csa

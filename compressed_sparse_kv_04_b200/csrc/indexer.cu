@@ -102,7 +102,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int t_begin = blockIdx.x * p.tiles_per_chunk;
   const int t_vis = (int)((nv_max + kTileRows - 1) / kTileRows);
   const int t_end = min(min(t_begin + p.tiles_per_chunk, p.ntiles), t_vis);
-  if (t_begin >= t_end) return;  // uniform over the CTA
+  if (t_begin >= t_end) {  // uniform over the CTA
+    pdl_wait();  // this grid completes only after its predecessor
+    return;
+  }
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) {
@@ -323,7 +326,7 @@ cudaError_t launch_impl(const IndexLaunch& a, cudaStream_t stream) {
                    kTileRows, DI, DI == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B);
   if (e != cudaSuccess) return e;
   dim3 grid(chunks, (unsigned)groups);
-  return launch_pdl(kern, grid, dim3(kThreads), smem, stream, 0, kmap, p);
+  return launch_pdl(kern, grid, dim3(kThreads), smem, stream, 0, a.chained, kmap, p);
 }
 
 }  // namespace

@@ -27,6 +27,7 @@ struct CompressLaunch {
   int rope_dim;             // KV entries are stored rotated to (i+1)*m - 1
   double inv_freq[64];      // rope_dim/2 entries
   int32_t* status;
+  int chained;              // see launch_pdl
 };
 cudaError_t launch_compress(const CompressLaunch& c, cudaStream_t stream);
 
@@ -45,6 +46,7 @@ struct IndexLaunch {
   float* scores;            // [B, Q, N_cap]
   int32_t* status;
   int num_sms;
+  int chained;              // see launch_pdl
 };
 cudaError_t launch_index_scores(const IndexLaunch& a, cudaStream_t stream);
 
@@ -60,6 +62,7 @@ struct TopkLaunch {
   int32_t* idx;             // [rows, k]
   int32_t* cnt;             // [rows]
   int32_t* status;
+  int chained;              // see launch_pdl
 };
 cudaError_t launch_topk(const TopkLaunch& a, cudaStream_t stream);
 
@@ -90,6 +93,7 @@ struct MqaLaunch {
   float* part_ml;           // workspace [rows, S, 2, H] fp32
   int splits;               // S
   int32_t* status;
+  int chained;              // see launch_pdl (the merge kernel is always chained)
 };
 size_t mqa_workspace_bytes(int rows, int splits, int H, int D);
 int mqa_choose_splits(int rows, int64_t compressed_max, int window, int num_sms, int H);
@@ -97,12 +101,22 @@ cudaError_t launch_mqa(const MqaLaunch& a, cudaStream_t stream);
 
 int device_sm_count();
 
-// Launches `kern` with programmatic stream serialization (the kernel may
-// overlap its predecessor in the stream up to its pdl_wait()) and, when
-// cluster_x > 0, a (cluster_x, 1, 1) cluster.
+// Launches `kern` and, when cluster_x > 0, as (cluster_x, 1, 1) clusters.
+//
+// chained != 0: with programmatic stream serialization, so the kernel may
+// start while its predecessor in the stream still runs, up to its
+// pdl_wait().  Only the second and later kernels of one entry point are
+// launched this way: their predecessor is a kernel of the same call, which
+// itself started only after everything before the call had completed.  So
+// their reads of caller inputs before pdl_wait() are safe, and their reads
+// of data written by an earlier kernel of the call come after pdl_wait().
+// chained == 0 (the first kernel of every entry point): an ordinary launch,
+// which starts after all earlier work in the stream has completed, whatever
+// that work is (a caller's kernel that lets its dependents start early
+// included).
 template <typename... KArgs, typename... Args>
 cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
-                       cudaStream_t stream, int cluster_x, Args... args) {
+                       cudaStream_t stream, int cluster_x, int chained, Args... args) {
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = grid;
   cfg.blockDim = block;
@@ -110,9 +124,11 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sme
   cfg.stream = stream;
   cudaLaunchAttribute attr[2];
   int n = 0;
-  attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[n].val.programmaticStreamSerializationAllowed = 1;
-  ++n;
+  if (chained) {
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+  }
   if (cluster_x > 0) {
     attr[n].id = cudaLaunchAttributeClusterDimension;
     attr[n].val.clusterDim.x = cluster_x;

@@ -1011,13 +1011,13 @@ cudaError_t launch_impl(const MqaLaunch& a, cudaStream_t stream) {
   e = ensure_smem_attr(reinterpret_cast<const void*>(kern), 3 + (D == 512 ? 0 : 3) + R / 32, smem);
   if (e != cudaSuccess) return e;
   dim3 grid(cps * a.splits, rows, 1);
-  e = launch_pdl(kern, grid, dim3(kThreads), smem, stream, 0, map_q, box_c, box_t, p);
+  e = launch_pdl(kern, grid, dim3(kThreads), smem, stream, 0, a.chained, map_q, box_c, box_t, p);
   if (e != cudaSuccess) return e;
   if (p.fused) return cudaSuccess;  // the attention kernel finished the rows
   const unsigned nblk = (unsigned)(((int64_t)rows * a.H + 3) / 4);
   const size_t wsm = (size_t)4 * a.splits * sizeof(float);
   auto merge = mqa_combine_kernel<D, R, 4>;
-  return launch_pdl(merge, dim3(nblk), dim3(128), wsm, stream, 0, p, rows, a.sink,
+  return launch_pdl(merge, dim3(nblk), dim3(128), wsm, stream, 0, 1, p, rows, a.sink,
                     reinterpret_cast<__nv_bfloat16*>(a.out), a.lse);
 }
 

@@ -381,7 +381,7 @@ cudaError_t launch_topk(const TopkLaunch& a, cudaStream_t stream) {
   p.cnt = a.cnt;
   p.status = a.status;
   const size_t smem = sizeof(S) + (size_t)p.slice * 4;
-  return launch_pdl(kern, dim3(C, a.rows, 1), dim3(kThreads), smem, stream, C, p);
+  return launch_pdl(kern, dim3(C, a.rows, 1), dim3(kThreads), smem, stream, C, a.chained, p);
 }
 
 }  // namespace csa

@@ -26,6 +26,14 @@
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
  *     stream).  Calls only enqueue work; they are stream-ordered, keep no
  *     state between calls and may be captured into a CUDA graph.
+ *   - Ordering: the first kernel of every call is an ordinary launch, so it
+ *     starts only after all earlier work on the stream has completed --
+ *     including a caller's kernel that lets its dependents launch early.
+ *     The later kernels of a call may start while their predecessor in the
+ *     same call still runs (programmatic dependent launch) and read the
+ *     call's inputs early; they wait for that predecessor before reading
+ *     anything it writes.  Inputs therefore only need to be complete in
+ *     stream order when the call is made.
  *   - Argument checks are synchronous and return an error before anything
  *     is enqueued.  A failed launch returns CSA_ERR_CUDA.  csa_last_error()
  *     returns a thread-local message for the last failure on that thread.
