@@ -1,5 +1,7 @@
 """Helpers shared by the GPU parity tests (tensor <-> oracle array conversion,
 tolerance checks).  Holds none of the method's arithmetic."""
+import math
+
 import numpy as np
 import torch
 
@@ -57,29 +59,48 @@ def assert_attention_close(got: np.ndarray, ref: np.ndarray, what=""):
     return mx, rl2
 
 
-# Log-sum-exp tolerance at the plain logit scale 1/sqrt(D).  The tensor cores
-# see the normalised (and rotated) query rounded to bf16, qhat_d (1 + e_d)
-# with |e_d| <= 2^-8.  Every key shares that rounding, so the log-sum-exp
-# moves by the attention-weighted mean of the logit errors,
-#     dLSE = scale * sum_d e_d qhat_d vbar_d,   vbar = sum_j p_j v_j,
-# whose standard deviation is about 2^-8/sqrt(3) * |qhat| |vbar| / sqrt(D)
-# = 2.3e-3 * |vbar| / sqrt(D) for |qhat| = sqrt(D).  |vbar| <= sqrt(D) (one
-# dominant key, the worst case: 2.3e-3), and it is far smaller when the
-# attention spreads over many keys.  5e-3 is two standard deviations of that
-# worst case; at the test data's near-uniform attention it is a wide margin.
-# A larger logit scale (YaRN's gain) scales the bound with it.
-LSE_ATOL = 5e-3
+# Log-sum-exp tolerance, per (row, head).  The tensor cores see the
+# normalised (and rotated) query rounded to bf16, qhat_d (1 + e_d) with
+# |e_d| <= 2^-8 (standard deviation about 2^-8/sqrt(3) = 2.3e-3), and a
+# window token's key, when the kernel rescales or rotates it in bf16, rounded
+# the same way.  The log-sum-exp moves by the attention-weighted mean of the
+# logit errors: for the query part
+#     dLSE = scale * sum_d e_d qhat_d obar_d,   obar = sum_j p_j v_j,
+# where p_j are the softmax weights (sink included) and obar is the output
+# before its inverse rotation, so |obar| = |o| for the head's output o.  With
+# |qhat_d| ~ 1 its standard deviation is about 2.3e-3 * scale * |o|; the key
+# part is at most as large again.  The bound is five standard deviations of
+# the two together, 5 * sqrt(2) * 2.3e-3 * scale * |o|, plus 1e-4 for the fp32
+# accumulation.  A head that attends to one key (|o| ~ sqrt(D)) gets about
+# 1.6e-2 at scale 1/sqrt(D); one that spreads over ~1000 keys, about 1e-3.
+LSE_SIGMA = 2.3e-3
 
 
-def assert_lse_close(got, ref, what="", scale_gain=1.0):
+def lse_tolerance(out_ref, scale):
+    """Per-(row, head) LSE bound from the oracle's output [..., H, D]."""
+    o = np.linalg.norm(np.asarray(out_ref, np.float64), axis=-1)
+    return 5.0 * math.sqrt(2.0) * LSE_SIGMA * scale * o + 1e-4
+
+
+def assert_lse_close(got, ref, out_ref, what="", scale=None):
+    """LSE [..., H] against the oracle's, within lse_tolerance of the oracle's
+    output out_ref [..., H, D]; scale is the logit scale (1/sqrt(D) when
+    None)."""
     got = np.asarray(got, np.float64)
     ref = np.asarray(ref, np.float64)
+    if scale is None:
+        scale = 1.0 / math.sqrt(np.asarray(out_ref).shape[-1])
     fin = np.isfinite(ref)
     assert np.array_equal(np.isfinite(got), fin), f"{what}: non-finite pattern differs"
     assert np.array_equal(got[~fin], ref[~fin]), f"{what}: infinite values differ"
     if not fin.any():
         return 0.0
-    err = float(np.abs(got[fin] - ref[fin]).max())
-    _record("lse_abs", err / scale_gain)
-    assert err <= LSE_ATOL * scale_gain, f"{what}: max LSE error {err:.3e}"
-    return err
+    tol = lse_tolerance(out_ref, scale)
+    err = np.abs(got - ref)
+    _record("lse_abs", float(err[fin].max()))
+    _record("lse_over_bound", float((err[fin] / tol[fin]).max()))
+    bad = fin & (err > tol)
+    assert not bad.any(), (f"{what}: {bad.sum()} LSE values out of tolerance, max error "
+                           f"{err[fin].max():.3e}, largest error/bound "
+                           f"{(err[fin] / tol[fin]).max():.2f}")
+    return float(err[fin].max())

@@ -33,8 +33,8 @@ def _to_bf16(bits):
     return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(DEV)
 
 
-def _check_lse(lse, rlse):
-    assert_lse_close(f32(lse), rlse, "decode-step LSE")
+def _check_lse(lse, rlse, ref):
+    assert_lse_close(f32(lse), rlse, ref, "decode-step LSE")
 
 
 def test_csa_decode_loop(orc):
@@ -105,7 +105,7 @@ def test_csa_decode_loop(orc):
         got = out.double().cpu().numpy()
         assert np.isfinite(got).all()
         assert_attention_close(got, ro[:, 0], f"step {step}")
-        _check_lse(lse, rl[:, 0])
+        _check_lse(lse, rl[:, 0], ro[:, 0])
     # The whole cache after the loop: every block of tokens up to the last
     # position, the partial newest one included.
     last = start + 5
@@ -154,4 +154,4 @@ def test_hca_decode_loop(orc):
         got = out.double().cpu().numpy()
         assert np.isfinite(got).all()
         assert_attention_close(got, ro[:, 0], f"HCA step {step}")
-        _check_lse(lse, rl[:, 0])
+        _check_lse(lse, rl[:, 0], ro[:, 0])
