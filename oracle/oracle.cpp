@@ -171,7 +171,7 @@ void rms_norm(double* v, int D, const float* gamma, double eps) {
 
 extern "C" {
 
-int orc_abi_version(void) { return 2; }
+int orc_abi_version(void) { return 3; }
 
 double orc_bf16_decode(uint16_t h) { return bf16_decode(h); }
 uint16_t orc_bf16_encode(double x) { return bf16_encode(x); }
@@ -429,6 +429,57 @@ void orc_mqa(int B, int Q, int H, int D, int m, int W, int rope_dim, double rope
       if (lse) lse[bq * H + h] = M + std::log(L);
     });
   }
+}
+
+// ------------------------------------------- f1: grouped output projection ---
+// "DeepSeek V4 technical report" (agentupdate.ai), 混合注意力机制, item
+// 分组输出投影 (grouped output projection): with head dim 512, projecting all
+// head outputs straight back to the model dim d is costly, so the n_h heads
+// are split into g groups, each group is first projected to an intermediate
+// dim d_g, and the results are then projected together back to d.  "DeepSeek
+// V4-Pro" (llm-arch-kb), "1. Hybrid attention": g = 16, d_g = 1024.
+//
+// Reading (the pages give the two projections only): for token t and group
+// j, x_j = the concatenation of the outputs of heads j*H/g .. (j+1)*H/g - 1
+// (H/g * D values, head-major); y_j = W_g[j] x_j (W_g[j]: [d_g, H/g * D],
+// rows = outputs); y = concat_j y_j ([g * d_g]); z = W_o y (W_o: [d, g * d_g]).
+// No bias and no nonlinearity between the two.  The library stores y in
+// bfloat16, so y_bf16 != 0 rounds y to bfloat16 before the second
+// projection, as the storage contract does; y_in != nullptr replaces the
+// first projection by the given bfloat16 y (a step-chained check).
+void orc_grouped_out_proj(int64_t T, int H, int D, int g, int d_g, int d_model,
+                          const uint16_t* o, const uint16_t* w_g, const uint16_t* w_o,
+                          int y_bf16, const uint16_t* y_in, double* y_out, double* z_out,
+                          int nthreads) {
+  const int hpg = H / g;             // heads per group
+  const int64_t kin = (int64_t)hpg * D;  // inputs of one group
+  const int64_t ny = (int64_t)g * d_g;
+  parallel_for(T, nthreads, [&](int64_t t) {
+    std::vector<double> y(ny);
+    if (y_in) {
+      for (int64_t i = 0; i < ny; ++i) y[i] = bf16_decode(y_in[t * ny + i]);
+    } else {
+      for (int j = 0; j < g; ++j) {
+        const uint16_t* x = o + (t * H + (int64_t)j * hpg) * D;  // heads of group j, contiguous
+        for (int r = 0; r < d_g; ++r) {
+          const uint16_t* wr = w_g + ((int64_t)j * d_g + r) * kin;
+          double acc = 0.0;
+          for (int64_t c = 0; c < kin; ++c) acc += bf16_decode(wr[c]) * bf16_decode(x[c]);
+          y[(int64_t)j * d_g + r] = acc;
+        }
+      }
+      if (y_bf16)
+        for (int64_t i = 0; i < ny; ++i) y[i] = bf16_decode(bf16_encode(y[i]));
+    }
+    if (y_out)
+      for (int64_t i = 0; i < ny; ++i) y_out[t * ny + i] = y[i];
+    for (int n = 0; n < d_model; ++n) {
+      const uint16_t* wr = w_o + (int64_t)n * ny;
+      double acc = 0.0;
+      for (int64_t i = 0; i < ny; ++i) acc += bf16_decode(wr[i]) * y[i];
+      z_out[t * d_model + n] = acc;
+    }
+  });
 }
 
 }  // extern "C"

@@ -66,6 +66,9 @@ def _declare(L):
     L.orc_mqa.argtypes = [i32, i32, i32, i32, i32, i32, i32, f64, P(f64), P(C.c_uint16), P(i64),
                           P(C.c_uint16), i64, P(C.c_int32), P(C.c_int32), i32, P(C.c_uint16),
                           i64, i64, P(f32), P(f32), P(f32), f64, f64, P(f64), P(f64), i32]
+    L.orc_grouped_out_proj.argtypes = [i64, i32, i32, i32, i32, i32, P(C.c_uint16),
+                                       P(C.c_uint16), P(C.c_uint16), i32, P(C.c_uint16),
+                                       P(f64), P(f64), i32]
 
 
 def _c(a, dt):
@@ -281,3 +284,32 @@ def hca_decode(q, pos_q, kv_c, kv_tok, sink, m, W, rope_dim, gamma_q=None, gamma
     out, lse = mqa(q.reshape((B, 1) + q.shape[-2:]), pos, kv_c, kv_tok, sink, m, W, rope_dim,
                    None, None, gamma_q, gamma_kv, nthreads=nthreads)
     return dict(out=out[:, 0], lse=lse[:, 0], out_bf16=bf16_encode(out[:, 0]))
+
+
+def grouped_out_proj(o, w_g, w_o, y_bf16=True, y_in=None, nthreads=0):
+    """Grouped output projection (f1) in fp64.
+
+    o [T, H, D] bf16 bits (the attention output); w_g [g, d_g, H/g * D] and
+    w_o [d, g * d_g] bf16 bits (rows = outputs).  y_bf16 rounds the
+    intermediate y to bf16 (the library's storage); y_in [T, g * d_g] bf16
+    bits replaces the first projection.  Returns (y fp64 [T, g*d_g], z fp64 [T, d])."""
+    o = _c(o, np.uint16)
+    T, H, D = o.shape
+    w_g = _c(w_g, np.uint16)
+    g, d_g, kin = w_g.shape
+    if H % g or kin != (H // g) * D:
+        raise ValueError("w_g must be [g, d_g, H/g * D] with g dividing H")
+    w_o = _c(w_o, np.uint16)
+    d_model = w_o.shape[0]
+    if w_o.shape[1] != g * d_g:
+        raise ValueError("w_o must be [d, g * d_g]")
+    if y_in is not None:
+        y_in = _c(y_in, np.uint16)
+        if y_in.shape != (T, g * d_g):
+            raise ValueError("y_in must be [T, g * d_g]")
+    y = np.empty((T, g * d_g), np.float64)
+    z = np.empty((T, d_model), np.float64)
+    lib().orc_grouped_out_proj(T, H, D, g, d_g, d_model, _p(o, C.c_uint16), _p(w_g, C.c_uint16),
+                               _p(w_o, C.c_uint16), 1 if y_bf16 else 0, _p(y_in, C.c_uint16),
+                               _p(y, C.c_double), _p(z, C.c_double), nthreads)
+    return y, z

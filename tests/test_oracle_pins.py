@@ -597,3 +597,85 @@ def test_joint_softmax_without_sink_is_sdpa_over_concatenated_keys(orc):
     assert np.allclose(out[0, 0], ref.numpy(), rtol=1e-12, atol=1e-12)
     assert np.allclose(lse[0, 0], torch.logsumexp(qh @ keys.T / math.sqrt(D), 1).numpy(),
                        rtol=1e-13, atol=1e-13)
+
+
+# -------------------------------------------- grouped output projection ---
+def _gop_case(T, H, D, g, d_g, d, seed):
+    r = rng(seed)
+    o = bf16_bits(r.standard_normal((T, H, D)))
+    w_g = bf16_bits(r.standard_normal((g, d_g, (H // g) * D)) / math.sqrt((H // g) * D))
+    w_o = bf16_bits(r.standard_normal((d, g * d_g)) / math.sqrt(g * d_g))
+    return o, w_g, w_o
+
+
+def test_grouped_out_proj_matches_einsum(orc):
+    # Group j reads heads j*H/g .. (j+1)*H/g - 1 (concatenated, head-major),
+    # W_g[j] maps them to d_g values, W_o maps the concatenation to d.
+    T, H, D, g, d_g, d = 3, 8, 16, 4, 8, 12
+    o, w_g, w_o = _gop_case(T, H, D, g, d_g, d, 61)
+    y, z = orc.grouped_out_proj(o, w_g, w_o, y_bf16=False)
+    of = orc.bf16_decode(o).reshape(T, g, (H // g) * D)
+    wg = orc.bf16_decode(w_g)
+    wo = orc.bf16_decode(w_o)
+    y_ref = np.einsum("tgk,gnk->tgn", of, wg).reshape(T, g * d_g)
+    assert np.allclose(y, y_ref, rtol=1e-13, atol=1e-13)
+    assert np.allclose(z, y_ref @ wo.T, rtol=1e-12, atol=1e-12)
+    # Another reading -- groups of interleaved heads (head h in group h % g) --
+    # gives another result, so the grouping is pinned.
+    inter = orc.bf16_decode(o).reshape(T, H // g, g, D).transpose(0, 2, 1, 3).reshape(T, g, -1)
+    assert not np.allclose(y, np.einsum("tgk,gnk->tgn", inter, wg).reshape(T, -1), atol=1e-3)
+
+
+def test_grouped_out_proj_single_group_is_two_matmuls(orc):
+    T, H, D, g, d_g, d = 2, 4, 8, 1, 5, 7
+    o, w_g, w_o = _gop_case(T, H, D, g, d_g, d, 62)
+    _, z = orc.grouped_out_proj(o, w_g, w_o, y_bf16=False)
+    x = torch.from_numpy(orc.bf16_decode(o).reshape(T, H * D))
+    ref = (x @ torch.from_numpy(orc.bf16_decode(w_g)[0]).T) @ torch.from_numpy(orc.bf16_decode(w_o)).T
+    assert np.allclose(z, ref.numpy(), rtol=1e-12, atol=1e-12)
+
+
+def test_grouped_out_proj_is_block_diagonal(orc):
+    # The grouped first projection equals one dense projection whose weight is
+    # block diagonal over the groups.
+    T, H, D, g, d_g, d = 2, 6, 4, 3, 5, 4
+    o, w_g, w_o = _gop_case(T, H, D, g, d_g, d, 63)
+    y, _ = orc.grouped_out_proj(o, w_g, w_o, y_bf16=False)
+    wg = orc.bf16_decode(w_g)
+    k = (H // g) * D
+    big = np.zeros((g * d_g, H * D))
+    for j in range(g):
+        big[j * d_g:(j + 1) * d_g, j * k:(j + 1) * k] = wg[j]
+    assert np.allclose(y, orc.bf16_decode(o).reshape(T, H * D) @ big.T, rtol=1e-13, atol=1e-13)
+
+
+def test_grouped_out_proj_selection_weights_are_exact(orc):
+    # 0/1 weights that pick input c_j of group j, then the identity: y and z
+    # are exactly those inputs.
+    T, H, D, g, d_g = 2, 4, 8, 2, 3
+    o, _, _ = _gop_case(T, H, D, g, d_g, 1, 64)
+    k = (H // g) * D
+    picks = [[0, 5, 15], [1, 8, 9]]
+    w = np.zeros((g, d_g, k), np.float32)
+    for j in range(g):
+        for r, c in enumerate(picks[j]):
+            w[j, r, c] = 1.0
+    w_o = np.eye(g * d_g, dtype=np.float32)
+    y, z = orc.grouped_out_proj(o, bf16_bits(w), bf16_bits(w_o))
+    of = orc.bf16_decode(o).reshape(T, g, k)
+    ref = np.stack([of[:, j, picks[j]] for j in range(g)], 1).reshape(T, -1)
+    assert np.array_equal(y, ref) and np.array_equal(z, ref)
+
+
+def test_grouped_out_proj_intermediate_storage_and_chaining(orc):
+    T, H, D, g, d_g, d = 3, 8, 16, 4, 8, 12
+    o, w_g, w_o = _gop_case(T, H, D, g, d_g, d, 65)
+    y_exact, _ = orc.grouped_out_proj(o, w_g, w_o, y_bf16=False)
+    y, z = orc.grouped_out_proj(o, w_g, w_o, y_bf16=True)
+    # y is stored in bf16: a bf16 value within half a bf16 ulp of the exact y.
+    assert np.array_equal(orc.bf16_decode(orc.bf16_encode(y)), y)
+    assert np.all(np.abs(y - y_exact) <= np.abs(y_exact) * 2.0 ** -8)
+    # Feeding that bf16 y as y_in gives the same z (the second projection alone).
+    _, z2 = orc.grouped_out_proj(o, w_g, w_o, y_in=orc.bf16_encode(y))
+    assert np.array_equal(z, z2)
+    assert np.allclose(z, y @ orc.bf16_decode(w_o).T, rtol=1e-12, atol=1e-12)
