@@ -171,7 +171,7 @@ void rms_norm(double* v, int D, const float* gamma, double eps) {
 
 extern "C" {
 
-int orc_abi_version(void) { return 3; }
+int orc_abi_version(void) { return 4; }
 
 double orc_bf16_decode(uint16_t h) { return bf16_decode(h); }
 uint16_t orc_bf16_encode(double x) { return bf16_encode(x); }
@@ -189,45 +189,52 @@ void orc_bf16_encode_array(int64_t n, const double* x, uint16_t* out) {
 // [P5] gives m = 4 for CSA and m' = 128 for HCA.
 //
 // Reading (weight form not given by the pages): for block i the present
-// tokens t = i*m + j (j < m, t < ctx_len) get scores s_j = c_t . w_s + b_pos[j];
-// the weights are the softmax of s over the present j; the pooled vector is
-// the weighted sum, followed by RMSNorm with gain gamma (this is the KV side
-// of the QK-Norm that [P5] places on the one shared compressed KV head).  Blocks do not
-// overlap for either ratio.  A block with no present token is not written.
-// `normalize` = 0 skips the RMSNorm (a test hook only).
+// tokens t = i*m - overlap + j (j < m + overlap, 0 <= t < ctx_len) get scores
+// s_j = c_t . w_s + b_pos[j]; the weights are the softmax of s over the
+// present j; the pooled vector is the weighted sum, followed by RMSNorm with
+// gain gamma (this is the KV side of the QK-Norm that [P5] places on the one
+// shared compressed KV head).  overlap = 0: blocks do not overlap ([P2] says
+// so for HCA).  overlap > 0 (a CSA variant: [P2] states "no overlap" for HCA
+// only, and gives no overlap rule): entry i also pools the last `overlap`
+// tokens of block i-1, i.e. a window of m + overlap tokens at stride m,
+// clipped at the sequence start.  A block with no present token of its own
+// range is not written.  `normalize` = 0 skips the RMSNorm (a test hook only).
 //
 // Storage reading for the KV stream ([P5] puts RoPE on the last dimensions
 // of the KV; where it is applied is not fixed): the entry is stored already
 // rotated to its own position (i+1)*m - 1, the last token of the block, so
 // that attention uses it as stored.  rope_dim = 0 stores it unrotated (the
 // indexer stream, which the pages do not rotate).
-void orc_pool(int B, int64_t L_cap, int d, int m, const uint16_t* tok, const int64_t* ctx_len,
-              const float* w_s, const float* b_pos, const float* gamma, double eps, int normalize,
-              int rope_dim, double rope_base, const double* rope_freq, int64_t first_block,
-              int64_t n_blocks,
-              int64_t N_cap, double* out, uint8_t* written, int nthreads) {
+void orc_pool(int B, int64_t L_cap, int d, int m, int overlap, const uint16_t* tok,
+              const int64_t* ctx_len, const float* w_s, const float* b_pos, const float* gamma,
+              double eps, int normalize, int rope_dim, double rope_base, const double* rope_freq,
+              int64_t first_block, int64_t n_blocks, int64_t N_cap, double* out,
+              uint8_t* written, int nthreads) {
   parallel_for((int64_t)B * n_blocks, nthreads, [&](int64_t w) {
     int64_t b = w / n_blocks, i = first_block + w % n_blocks;
     if (i < 0 || i >= N_cap) return;
     int64_t L = std::min<int64_t>(ctx_len[b], L_cap);
-    int64_t t0 = i * m;
-    int present = (int)std::max<int64_t>(0, std::min<int64_t>(m, L - t0));
-    if (present == 0) return;
-    std::vector<double> s(present);
+    if (L <= i * m) return;  // no token of the block's own range yet
+    // Window positions j = 0 .. m+overlap-1 hold token t = i*m - overlap + j.
+    int64_t t0 = i * m - overlap;
+    std::vector<int> js;
+    for (int j = 0; j < m + overlap; ++j)
+      if (t0 + j >= 0 && t0 + j < L) js.push_back(j);
+    std::vector<double> s(js.size());
     double smax = -std::numeric_limits<double>::infinity();
-    for (int j = 0; j < present; ++j) {
-      const uint16_t* row = tok + ((int64_t)b * L_cap + t0 + j) * d;
+    for (size_t q = 0; q < js.size(); ++q) {
+      const uint16_t* row = tok + ((int64_t)b * L_cap + t0 + js[q]) * d;
       double acc = 0.0;
       for (int k = 0; k < d; ++k) acc += bf16_decode(row[k]) * (double)w_s[k];
-      s[j] = acc + (double)b_pos[j];
-      smax = std::max(smax, s[j]);
+      s[q] = acc + (double)b_pos[js[q]];
+      smax = std::max(smax, s[q]);
     }
     double z = 0.0;
-    for (int j = 0; j < present; ++j) z += std::exp(s[j] - smax);
+    for (size_t q = 0; q < js.size(); ++q) z += std::exp(s[q] - smax);
     std::vector<double> p(d, 0.0);
-    for (int j = 0; j < present; ++j) {
-      double a = std::exp(s[j] - smax) / z;
-      const uint16_t* row = tok + ((int64_t)b * L_cap + t0 + j) * d;
+    for (size_t q = 0; q < js.size(); ++q) {
+      double a = std::exp(s[q] - smax) / z;
+      const uint16_t* row = tok + ((int64_t)b * L_cap + t0 + js[q]) * d;
       for (int k = 0; k < d; ++k) p[k] += a * bf16_decode(row[k]);
     }
     if (normalize) rms_norm(p.data(), d, gamma, eps);

@@ -56,9 +56,9 @@ def _declare(L):
     L.orc_e4m3_encode.argtypes = [f32]
     L.orc_e4m3_encode.restype = C.c_uint8
     L.orc_bf16_encode_array.argtypes = [i64, P(f64), P(C.c_uint16)]
-    L.orc_pool.argtypes = [i32, i64, i32, i32, P(C.c_uint16), P(i64), P(f32), P(f32), P(f32),
-                           f64, i32, i32, f64, P(f64), i64, i64, i64, P(f64), P(C.c_uint8),
-                           i32]
+    L.orc_pool.argtypes = [i32, i64, i32, i32, i32, P(C.c_uint16), P(i64), P(f32), P(f32),
+                           P(f32), f64, i32, i32, f64, P(f64), i64, i64, i64, P(f64),
+                           P(C.c_uint8), i32]
     L.orc_quant_rows_e4m3.argtypes = [i64, i32, P(f64), P(C.c_uint8), P(f32)]
     L.orc_index_scores.argtypes = [i32, i32, i32, i32, i32, P(C.c_uint8), P(f32), P(f32),
                                    P(C.c_uint8), P(f32), i64, P(i64), P(f64), i32]
@@ -143,17 +143,21 @@ def _freq(rope_freq, rope_dim):
 
 
 def pool(tok, ctx_len, w_s, b_pos, gamma, m, first_block, n_blocks, N_cap, eps=1e-6,
-         normalize=True, nthreads=0, rope_dim=0, rope_base=10000.0, rope_freq=None):
+         normalize=True, nthreads=0, rope_dim=0, rope_base=10000.0, rope_freq=None, overlap=0):
     """Compression step (a1) in fp64.  Returns (values[B,N_cap,d], written[B,N_cap]).
     rope_dim > 0: each entry is stored rotated to its position (i+1)*m - 1.
-    rope_freq [rope_dim/2] replaces the frequencies rope_base^(-2j/rope_dim)."""
+    rope_freq [rope_dim/2] replaces the frequencies rope_base^(-2j/rope_dim).
+    overlap > 0: entry i pools tokens i*m - overlap .. (i+1)*m - 1 (b_pos has
+    m + overlap values)."""
     rope_freq = _freq(rope_freq, rope_dim)
     tok = _c(tok, np.uint16)
     B, L_cap, d = tok.shape
     ctx_len = _c(ctx_len, np.int64)
+    if len(np.ravel(b_pos)) != m + overlap:
+        raise ValueError("b_pos must hold m + overlap values")
     out = np.zeros((B, N_cap, d), np.float64)
     written = np.zeros((B, N_cap), np.uint8)
-    lib().orc_pool(B, L_cap, d, m, _p(tok, C.c_uint16), _p(ctx_len, C.c_int64),
+    lib().orc_pool(B, L_cap, d, m, overlap, _p(tok, C.c_uint16), _p(ctx_len, C.c_int64),
                    _p(_c(w_s, np.float32), C.c_float), _p(_c(b_pos, np.float32), C.c_float),
                    _p(None if gamma is None else _c(gamma, np.float32), C.c_float),
                    eps, 1 if normalize else 0, rope_dim, rope_base, _p(rope_freq, C.c_double),
@@ -241,19 +245,19 @@ def mqa(q, pos_q, kv_c, kv_tok, sink, m, W, rope_dim, sel_idx=None, sel_cnt=None
 
 # --------------------------------------------------------------- composites --
 def compress_kv(tok, ctx_len, w_s, b_pos, gamma, m, first_block, n_blocks, N_cap, eps=1e-6,
-                nthreads=0, rope_dim=0, rope_base=10000.0, rope_freq=None):
+                nthreads=0, rope_dim=0, rope_base=10000.0, rope_freq=None, overlap=0):
     """a1 for the KV stream with bfloat16 storage (entries stored rotated to
     their position when rope_dim > 0): returns (bf16 bits, written mask, fp64 values)."""
     vals, written = pool(tok, ctx_len, w_s, b_pos, gamma, m, first_block, n_blocks, N_cap,
-                         eps, True, nthreads, rope_dim, rope_base, rope_freq)
+                         eps, True, nthreads, rope_dim, rope_base, rope_freq, overlap)
     return bf16_encode(vals), written, vals
 
 
 def compress_index(tok, ctx_len, w_s, b_pos, m, first_block, n_blocks, N_cap, eps=1e-6,
-                   nthreads=0):
+                   nthreads=0, overlap=0):
     """a1 for the indexer stream: pooled, RMSNorm'd, E4M3 rows (codes, scale, fp64 values, written)."""
     vals, written = pool(tok, ctx_len, w_s, b_pos, None, m, first_block, n_blocks, N_cap,
-                         eps, True, nthreads)
+                         eps, True, nthreads, overlap=overlap)
     codes, scale = quant_rows_e4m3(vals)
     return codes, scale, vals, written
 

@@ -679,3 +679,63 @@ def test_grouped_out_proj_intermediate_storage_and_chaining(orc):
     _, z2 = orc.grouped_out_proj(o, w_g, w_o, y_in=orc.bf16_encode(y))
     assert np.array_equal(z, z2)
     assert np.allclose(z, y @ orc.bf16_decode(w_o).T, rtol=1e-12, atol=1e-12)
+
+
+# ------------------------------------------ overlapping compression (CSA) ---
+def test_pool_overlap_zero_is_the_plain_pooling(orc):
+    B, L, d, m = 1, 22, 16, 4
+    tok = _tok(B, L, d, 71)
+    r = rng(72)
+    w_s = (0.3 * r.standard_normal(d)).astype(np.float32)
+    b_pos = r.standard_normal(m).astype(np.float32)
+    N = math.ceil(L / m)
+    a, _ = orc.pool(tok, np.array([L]), w_s, b_pos, None, m, 0, N, N)
+    b, _ = orc.pool(tok, np.array([L]), w_s, b_pos, None, m, 0, N, N, overlap=0)
+    assert np.array_equal(a, b)
+
+
+def test_pool_overlap_uniform_is_window_mean(orc):
+    # Uniform weights: entry i is the mean of tokens max(0, i*m - ov) .. (i+1)*m - 1
+    # (present ones): the window reaches back `ov` tokens into block i-1.
+    B, L, d, m = 1, 23, 8, 4
+    tok = _tok(B, L, d, 73)
+    x = orc.bf16_decode(tok)[0]
+    N = math.ceil(L / m)
+    for ov in (1, 2, 4):
+        vals, w = orc.pool(tok, np.array([L]), np.zeros(d), np.zeros(m + ov), None, m, 0, N, N,
+                           normalize=False, overlap=ov)
+        assert w[0].all()
+        for i in range(N):
+            lo, hi = max(0, i * m - ov), min(L, (i + 1) * m)
+            assert np.allclose(vals[0, i], x[lo:hi].mean(0), rtol=0, atol=1e-15), (ov, i)
+
+
+def test_pool_overlap_position_bias_addresses_the_window(orc):
+    # A large bias at window position j selects token i*m - ov + j: position
+    # 0 is the first borrowed token of block i-1, position ov the block's own
+    # first token.  For block 0 the borrowed positions do not exist.
+    B, L, d, m, ov = 1, 16, 8, 4, 4
+    tok = _tok(B, L, d, 74)
+    x = orc.bf16_decode(tok)[0]
+    for j in (0, 2, 4, 7):
+        b_pos = np.zeros(m + ov, np.float32)
+        b_pos[j] = 90.0
+        vals, _ = orc.pool(tok, np.array([L]), np.zeros(d), b_pos, None, m, 0, 4, 4,
+                           normalize=False, overlap=ov)
+        for i in range(1, 4):
+            assert np.allclose(vals[0, i], x[i * m - ov + j], rtol=0, atol=1e-30), (j, i)
+        if j >= ov:  # block 0: only its own tokens are present
+            assert np.allclose(vals[0, 0], x[j - ov], rtol=0, atol=1e-30)
+        else:        # the selected position is absent: uniform over tokens 0..3
+            assert np.allclose(vals[0, 0], x[0:4].mean(0), rtol=0, atol=1e-15)
+
+
+def test_pool_overlap_partial_newest_block(orc):
+    # Context ends inside block i: the window is clipped at the context end too.
+    B, L, d, m, ov = 1, 10, 8, 4, 4
+    tok = _tok(B, 12, d, 75)
+    x = orc.bf16_decode(tok)[0]
+    vals, w = orc.pool(tok, np.array([L]), np.zeros(d), np.zeros(m + ov), None, m, 0, 3, 3,
+                       normalize=False, overlap=ov)
+    assert w[0].tolist() == [True, True, True]
+    assert np.allclose(vals[0, 2], x[4:10].mean(0), rtol=0, atol=1e-15)
