@@ -539,6 +539,10 @@ def run_gpu(args):
             for name in EXTRA_WORKLOADS:
                 if name == w.name:
                     continue
+                if name in PROJ_TOKENS:
+                    extras[name] = measure_proj(name, K, W, dev)
+                    torch.cuda.empty_cache()
+                    continue
                 wx = workload_for_rank(configs.BY_NAME[name], rank)
                 if wx.kind == "csa_prefill":
                     extras[name] = measure_prefill(wx, K, W, dev)
@@ -587,7 +591,89 @@ def run_gpu(args):
 
 
 # The workloads timed after the primary one in a default run.
-EXTRA_WORKLOADS = ["hca_decode_1m_b8", "csa_decode_1m_b4", "csa_prefill_4096_after_65536"]
+EXTRA_WORKLOADS = ["hca_decode_1m_b8", "csa_decode_1m_b4", "csa_prefill_4096_after_65536",
+                   "grouped_out_proj_decode_t8", "grouped_out_proj_prefill_t4096"]
+
+# Grouped output projection ("DeepSeek V4-Pro" (llm-arch-kb), "1. Hybrid
+# attention": g = 16 groups, d_g = 1024) of the 128-head x 512 attention
+# output; d = 7168 (the pages give no model dim).  T = 8 is one decode step of
+# the 128K batch, T = 4096 the prefill chunk.
+PROJ_SHAPE = dict(H=128, D=512, g=16, d_g=1024, d_model=7168)
+PROJ_TOKENS = {"grouped_out_proj_decode_t8": 8, "grouped_out_proj_prefill_t4096": 4096}
+
+
+def measure_proj(name, K, W, dev):
+    """K calls of grouped_out_proj on one fixed input (the weights, 352 MiB,
+    exceed the L2, so every call streams them from HBM)."""
+    import torch
+
+    from compressed_sparse_kv_04_b200 import binding, synth
+    T = PROJ_TOKENS[name]
+    H, D, g, d_g, dm = (PROJ_SHAPE[k] for k in ("H", "D", "g", "d_g", "d_model"))
+    gen = torch.Generator(device=dev).manual_seed(20260008)
+    k1 = H // g * D
+    w_g = (torch.randn(g, d_g, k1, generator=gen, device=dev) / math.sqrt(k1)).to(torch.bfloat16)
+    w_o = (torch.randn(dm, g * d_g, generator=gen, device=dev) / math.sqrt(g * d_g)).to(
+        torch.bfloat16)
+    o = synth.normal_bf16((T, H, D), 20260008, "q", dev)
+    z = torch.empty(T, dm, dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(binding.grouped_out_proj_workspace_bytes(T, H, D, g, d_g, dm),
+                     dtype=torch.uint8, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    def call():
+        binding.grouped_out_proj(o, w_g, w_o, z, ws=ws, dev_status=status)
+
+    for _ in range(W):
+        call()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(K):
+        call()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / K
+    peaks = measured_peaks()
+    flops = 2.0 * T * (g * d_g * k1 + dm * g * d_g)
+    wbytes = (g * d_g * k1 + dm * g * d_g) * 2
+    abytes = wbytes + T * H * D * 2 + T * g * d_g * 2 * 2 + T * dm * 2
+    launches = 2 + sum(1 for sp in _proj_splits(T, H, D, g, d_g, dm) if sp > 1)
+    rec = {"value": round(T / (ms * 1e-3), 1), "unit": "tokens/s", "ms_per_step": round(ms, 6),
+           "config": {"workload": name, "tokens": T, **PROJ_SHAPE, "call": "grouped_out_proj",
+                      "l2": "no rotation: the weights (352 MiB) exceed the L2"},
+           "gpu_launches": launches * K, "device_status": int(status.item())}
+    tf = flops / (ms * 1e-3) / 1e12
+    gbs = abytes / (ms * 1e-3) / 1e9
+    if T <= 64:  # weight streaming: HBM-bound
+        rec["roofline"] = {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"],
+                           "unit": "GB/s", "frac": round(gbs / peaks["hbm_gbs"], 4),
+                           "peak_source": peaks["source"], "algorithmic_bytes": abytes,
+                           "avg_launch_ms": round(ms, 6), "traffic": None}
+    else:
+        rec["roofline"] = {"bound": "tensor", "achieved": round(tf, 1),
+                           "peak": round(peaks["bf16_tflops"], 1), "unit": "TFLOP/s",
+                           "frac": round(tf / peaks["bf16_tflops"], 4),
+                           "peak_source": peaks["source"], "algorithmic_flops": flops,
+                           "avg_launch_ms": round(ms, 6), "traffic": None}
+    return rec
+
+
+def _proj_splits(T, H, D, g, d_g, dm):
+    """The split-K factors the library picks (mirrors its planning, for the
+    launch count: a split projection adds one reduce launch)."""
+    import torch
+    sms = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+    bn = 16 if T <= 16 else 32 if T <= 32 else 64 if T <= 64 else 128 if T <= 128 else 256
+
+    def choose(N, groups, Kin):
+        tiles = (N // 128) * -(-T // bn) * groups
+        chunks = Kin // 64
+        s = 1
+        while tiles * s * 2 <= sms and chunks % (s * 2) == 0 and chunks // (s * 2) >= 8:
+            s *= 2
+        return s
+    return choose(d_g, g, H // g * D), choose(dm, 1, g * d_g)
 
 
 def run_e2e(st, K, W, barrier, rmax, rsum, world):

@@ -26,7 +26,8 @@ EXPORTS = ["csa_version", "csa_last_error", "csa_workspace_bytes", "hca_compress
            "csa_compress", "lightning_index_topk", "lightning_index_scores", "topk_select",
            "sparse_mqa_decode", "dense_mqa_decode", "csa_prefill_chunk",
            "lightning_index_topk_static", "csa_rope_yarn", "hca_prefill_chunk",
-           "csa_decode_step", "hca_decode_step"]
+           "csa_decode_step", "hca_decode_step", "grouped_out_proj",
+           "grouped_out_proj_workspace_bytes"]
 
 
 class CsaError(RuntimeError):
@@ -39,7 +40,7 @@ class csa_params(C.Structure):
     _fields_ = [("B", C.c_int), ("d", C.c_int), ("H", C.c_int), ("H_I", C.c_int),
                 ("D_I", C.c_int), ("k", C.c_int), ("window", C.c_int), ("rope_dim", C.c_int),
                 ("m", C.c_int), ("eps", C.c_float), ("softmax_scale", C.c_float),
-                ("rope_inv_freq", C.POINTER(C.c_double))]
+                ("rope_inv_freq", C.POINTER(C.c_double)), ("overlap", C.c_int)]
 
 
 _lib = None
@@ -89,13 +90,18 @@ def _declare(L):
     L.csa_rope_yarn.argtypes = [i32, C.c_double, C.c_double, C.c_double, C.c_double,
                                 C.c_double, i32, C.POINTER(C.c_double), C.POINTER(C.c_double),
                                 C.POINTER(C.c_float)]
+    L.grouped_out_proj.argtypes = [i32, i32, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, sz, vp,
+                                   vp]
+    L.grouped_out_proj_workspace_bytes.argtypes = [i32, i32, i32, i32, i32, i32]
+    L.grouped_out_proj_workspace_bytes.restype = sz
     for name in EXPORTS[3:]:
-        getattr(L, name).restype = i32
+        if name != "grouped_out_proj_workspace_bytes":
+            getattr(L, name).restype = i32
 
 
 def make_params(B, d, H=0, H_I=0, D_I=0, k=0, window=0, rope_dim=0, m=4, eps=1e-6,
-                softmax_scale=0.0, rope_inv_freq=None):
-    p = csa_params(B, d, H, H_I, D_I, k, window, rope_dim, m, eps, softmax_scale, None)
+                softmax_scale=0.0, rope_inv_freq=None, overlap=0):
+    p = csa_params(B, d, H, H_I, D_I, k, window, rope_dim, m, eps, softmax_scale, None, overlap)
     if rope_inv_freq is not None:
         arr = (C.c_double * len(rope_inv_freq))(*rope_inv_freq)
         p.rope_inv_freq = C.cast(arr, C.POINTER(C.c_double))
@@ -111,6 +117,7 @@ def params_for(w, B=None, **kw):
         tab, _, scale = rope_yarn(w.rope_dim, *w.yarn, d=w.d)
         kw["rope_inv_freq"] = tab
         kw.setdefault("softmax_scale", scale)
+    kw.setdefault("overlap", w.overlap)
     return make_params(B or w.B, w.d, w.H, w.H_I, w.D_I, w.k, w.W, w.rope_dim, w.m, **kw)
 
 
@@ -275,3 +282,25 @@ def hca_decode_step(p, pos_q, kv_tok, w_s, b_pos, gamma, kv_c, q, sink, out, gam
         _ptr(gamma), _ptr(kv_c), kv_c.shape[1], _ptr(q), _ptr(sink), _ptr(gamma_q),
         _ptr(gamma_kv), _ptr(out), _ptr(lse), _ptr(ws),
         0 if ws is None else ws.numel() * ws.element_size(), _ptr(dev_status), _stream(stream)))
+
+
+def grouped_out_proj_workspace_bytes(T, H, D, g, d_g, d_model):
+    n = lib().grouped_out_proj_workspace_bytes(T, H, D, g, d_g, d_model)
+    if n == 0:
+        raise CsaError(2, lib().csa_last_error().decode())
+    return n
+
+
+def grouped_out_proj(o, w_g, w_o, z, y=None, ws=None, dev_status=None, stream=None):
+    """Grouped output projection: o [T, H, D] -> y [T, g*d_g] -> z [T, d_model]
+    (w_g [g, d_g, H/g*D], w_o [d_model, g*d_g], all bf16).  The workspace is
+    allocated here when not given."""
+    T, H, D = o.shape
+    g, d_g, _ = w_g.shape
+    d_model = w_o.shape[0]
+    if ws is None:
+        ws = torch.empty(grouped_out_proj_workspace_bytes(T, H, D, g, d_g, d_model),
+                         dtype=torch.uint8, device=o.device)
+    _check(lib().grouped_out_proj(T, H, D, g, d_g, d_model, _ptr(o), _ptr(w_g), _ptr(w_o),
+                                  _ptr(y), _ptr(z), _ptr(ws), ws.numel() * ws.element_size(),
+                                  _ptr(dev_status), _stream(stream)))

@@ -31,6 +31,7 @@ class Workload:
     T: int = 0           # prefill: new tokens
     seed: int = 0
     yarn: tuple | None = None  # (factor, beta_fast, beta_slow, original_len) or plain RoPE
+    overlap: int = 0     # compression: tokens of block i-1 that entry i also pools
 
     @property
     def D(self) -> int:

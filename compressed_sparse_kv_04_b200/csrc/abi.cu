@@ -21,6 +21,7 @@ csa_status fail(csa_status s, const char* fmt, ...) {
 }
 
 constexpr int64_t kMaxIndexEntries = 262144;  // one 8-CTA cluster holds a score row
+constexpr int kMaxTopk = 2048;                // entries kept per query
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -54,6 +55,9 @@ csa_status check_common(const char* fn, const csa_params* p) {
     return fail(CSA_ERR_UNSUPPORTED_SHAPE, "%s: d=%d (supported: 128, 512)", fn, p->d);
   if (p->m < 1 || p->m > 128)
     return fail(CSA_ERR_UNSUPPORTED_SHAPE, "%s: m=%d (supported: 1..128)", fn, p->m);
+  if (p->overlap < 0 || p->overlap > p->m || p->m + p->overlap > 128)
+    return fail(CSA_ERR_UNSUPPORTED_SHAPE, "%s: overlap=%d (supported: 0..m, m + overlap <= 128)",
+                fn, p->overlap);
   if (!(p->eps > 0.f) || !std::isfinite(p->eps))
     return fail(CSA_ERR_INVALID_ARG, "%s: eps must be finite and > 0", fn);
   return CSA_OK;
@@ -64,8 +68,8 @@ csa_status check_indexer(const char* fn, const csa_params* p) {
     return fail(CSA_ERR_UNSUPPORTED_SHAPE, "%s: D_I=%d (supported: 64, 128)", fn, p->D_I);
   if (p->H_I < 1 || p->H_I > 64)
     return fail(CSA_ERR_UNSUPPORTED_SHAPE, "%s: H_I=%d (supported: 1..64)", fn, p->H_I);
-  if (p->k < 1 || p->k > 1024)
-    return fail(CSA_ERR_UNSUPPORTED_SHAPE, "%s: k=%d (supported: 1..1024)", fn, p->k);
+  if (p->k < 1 || p->k > kMaxTopk)
+    return fail(CSA_ERR_UNSUPPORTED_SHAPE, "%s: k=%d (supported: 1..%d)", fn, p->k, kMaxTopk);
   return CSA_OK;
 }
 
@@ -126,7 +130,7 @@ csa_status set_error(csa_status s, const char* fmt, ...) {
 
 extern "C" {
 
-int csa_version(void) { return 101; }
+int csa_version(void) { return 102; }
 
 csa_status csa_rope_yarn(int rope_dim, double base, double factor, double beta_fast,
                          double beta_slow, double original_len, int d, double* inv_freq,
@@ -245,6 +249,7 @@ static csa_status compress_common(const char* fn, const csa_params* p, const voi
   c.d = p->d;
   c.D_I = p->D_I;
   c.m = p->m;
+  c.overlap = p->overlap;
   c.L_cap = L_cap;
   c.N_cap = N_cap;
   c.kv_tok = kv_tok;
@@ -530,8 +535,8 @@ csa_status sparse_mqa_decode(const csa_params* p, const void* q, const int64_t* 
   csa_status st = check_mqa_args(fn, p, q, pos_q, kv_c, N_cap, kv_tok, L_cap, sink, gamma_q,
                                  gamma_kv, out, lse, dev_status);
   if (st != CSA_OK) return st;
-  if (p->k < 1 || p->k > 1024)
-    return fail(CSA_ERR_UNSUPPORTED_SHAPE, "%s: k=%d (supported: 1..1024)", fn, p->k);
+  if (p->k < 1 || p->k > kMaxTopk)
+    return fail(CSA_ERR_UNSUPPORTED_SHAPE, "%s: k=%d (supported: 1..%d)", fn, p->k, kMaxTopk);
   REQ_PTR(topk_idx);
   REQ_PTR4(topk_cnt);
   return mqa_common(fn, p, CSA_OP_SPARSE_MQA, p->B, 1, q, pos_q, 0, kv_c, N_cap, topk_idx,
@@ -631,8 +636,8 @@ csa_status csa_decode_step(const csa_params* p, const int64_t* pos_q, const void
   st = check_mqa_args(fn, p, q, pos_q, kv_c, N_cap, kv_tok, L_cap, sink, gamma_q, gamma_kv, out,
                       lse, dev_status);
   if (st != CSA_OK) return st;
-  if (p->k < 1 || p->k > 1024)
-    return fail(CSA_ERR_UNSUPPORTED_SHAPE, "%s: k=%d (supported: 1..1024)", fn, p->k);
+  if (p->k < 1 || p->k > kMaxTopk)
+    return fail(CSA_ERR_UNSUPPORTED_SHAPE, "%s: k=%d (supported: 1..%d)", fn, p->k, kMaxTopk);
   REQ_PTR(idx_tok);
   REQ_PTR(q_idx);
   REQ_PTR4(q_scale);
@@ -732,6 +737,111 @@ csa_status hca_prefill_chunk(const csa_params* p, int64_t P, int T, const void* 
   return mqa_common(fn, p, CSA_OP_DENSE_MQA, T, T, q, nullptr, P, kv_c, N_cap, nullptr, nullptr,
                     kv_tok, L_cap, sink, gamma_q, gamma_kv, out, lse, ws, ws_bytes, dev_status,
                     static_cast<cudaStream_t>(stream), 1);
+}
+
+// ------------------------------------------------- grouped output projection --
+static csa_status check_proj(const char* fn, int T, int H, int D, int g, int d_g, int d_model) {
+  if (T < 1 || H < 1 || D < 1 || g < 1 || d_g < 1 || d_model < 1)
+    return fail(CSA_ERR_INVALID_ARG, "%s: T=%d H=%d D=%d g=%d d_g=%d d=%d must be >= 1", fn, T, H, D,
+                g, d_g, d_model);
+  if (H % g)
+    return fail(CSA_ERR_UNSUPPORTED_SHAPE, "%s: g=%d must divide H=%d", fn, g, H);
+  const int64_t k1 = (int64_t)(H / g) * D, k2 = (int64_t)g * d_g;
+  if (k1 % 64 || k2 % 64 || d_g % 128 || d_model % 128 || k1 > (1 << 20) || k2 > (1 << 20) ||
+      (int64_t)H * D > ((int64_t)1 << 24) || d_model > (1 << 20))
+    return fail(CSA_ERR_UNSUPPORTED_SHAPE,
+                "%s: need (H/g)*D and g*d_g multiples of 64, d_g and d multiples of 128", fn);
+  if ((int64_t)T > (int64_t)65535 * 256)
+    return fail(CSA_ERR_UNSUPPORTED_SHAPE, "%s: T=%d too large", fn, T);
+  return CSA_OK;
+}
+
+struct ProjPlan {
+  int64_t k1, n1, k2;
+  int s1, s2;
+  size_t y_bytes, part_bytes;
+};
+
+static ProjPlan proj_plan(int T, int H, int D, int g, int d_g, int d_model) {
+  ProjPlan pl{};
+  pl.k1 = (int64_t)(H / g) * D;
+  pl.n1 = (int64_t)g * d_g;
+  pl.k2 = pl.n1;
+  const int sms = csa::device_sm_count();
+  pl.s1 = csa::proj_choose_splits(T, d_g, g, (int)pl.k1, sms);
+  pl.s2 = csa::proj_choose_splits(T, d_model, 1, (int)pl.k2, sms);
+  pl.y_bytes = round_up((size_t)T * pl.n1 * 2, 256);
+  size_t p1 = pl.s1 > 1 ? (size_t)pl.s1 * T * pl.n1 * 4 : 0;
+  size_t p2 = pl.s2 > 1 ? (size_t)pl.s2 * T * d_model * 4 : 0;
+  pl.part_bytes = round_up(p1 > p2 ? p1 : p2, 256);
+  return pl;
+}
+
+size_t grouped_out_proj_workspace_bytes(int T, int H, int D, int g, int d_g, int d_model) {
+  if (check_proj("grouped_out_proj_workspace_bytes", T, H, D, g, d_g, d_model) != CSA_OK) return 0;
+  const ProjPlan pl = proj_plan(T, H, D, g, d_g, d_model);
+  return pl.y_bytes + pl.part_bytes + 256;
+}
+
+csa_status grouped_out_proj(int T, int H, int D, int g, int d_g, int d_model, const void* o,
+                            const void* w_g, const void* w_o, void* y, void* z, void* ws,
+                            size_t ws_bytes, int32_t* dev_status, void* stream) {
+  const char* fn = "grouped_out_proj";
+  csa_status st = check_proj(fn, T, H, D, g, d_g, d_model);
+  if (st != CSA_OK) return st;
+  REQ_PTR(o);
+  REQ_PTR(w_g);
+  REQ_PTR(w_o);
+  OPT_PTR(y);
+  REQ_PTR(z);
+  OPT_PTR4(dev_status);
+  const ProjPlan pl = proj_plan(T, H, D, g, d_g, d_model);
+  const size_t need = pl.y_bytes + pl.part_bytes + 256;
+  if (!ws || ws_bytes < need)
+    return fail(CSA_ERR_WORKSPACE, "%s: workspace of %zu bytes needed, %zu given", fn, need,
+                ws ? ws_bytes : (size_t)0);
+  if (!aligned16(ws)) return fail(CSA_ERR_INVALID_ARG, "%s: ws is not 16-byte aligned", fn);
+  char* wsb = static_cast<char*>(ws);
+  void* ybuf = y ? y : static_cast<void*>(wsb);
+  float* part = reinterpret_cast<float*>(wsb + pl.y_bytes);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // 1. Per group j: y[:, j*d_g .. ] = x_j W_g[j]^T, x_j = heads j*H/g .. of o.
+  csa::ProjGemm a{};
+  a.a = o;
+  a.lda = (int64_t)H * D;
+  a.w = w_g;
+  a.w_rows = pl.n1;
+  a.K = (int)pl.k1;
+  a.N = d_g;
+  a.groups = g;
+  a.T = T;
+  a.splits = pl.s1;
+  a.c = ybuf;
+  a.ldc = (int)pl.n1;
+  a.part = part;
+  a.status = dev_status;
+  a.chained = 0;
+  cudaError_t e = csa::launch_proj_gemm(a, s);
+  if (e != cudaSuccess) return cuda_fail(fn, e);
+  // 2. z = y W_o^T.
+  csa::ProjGemm b{};
+  b.a = ybuf;
+  b.lda = pl.n1;
+  b.w = w_o;
+  b.w_rows = d_model;
+  b.K = (int)pl.k2;
+  b.N = d_model;
+  b.groups = 1;
+  b.T = T;
+  b.splits = pl.s2;
+  b.c = z;
+  b.ldc = d_model;
+  b.part = part;
+  b.status = dev_status;
+  b.chained = 1;
+  e = csa::launch_proj_gemm(b, s);
+  if (e != cudaSuccess) return cuda_fail(fn, e);
+  return CSA_OK;
 }
 
 }  // extern "C"

@@ -7,6 +7,10 @@
 // paragraph (m' = 128, no overlap); "DeepSeek V4-Pro" (llm-arch-kb), "Hybrid
 // attention" CSA / HCA bullets.  Weight form (the build's reading):
 // softmax_j(c_t . w_s + b_pos[j]) over the present tokens of the block.
+// Overlapping variant (CSA; the pages fix "no overlap" for HCA only): entry i
+// pools the window of m + overlap tokens i*m - overlap .. (i+1)*m - 1, with
+// b_pos indexed by the window position, clipped at the sequence start and at
+// the context end.
 //
 // Storage (the build's reading): a KV entry is stored already rotated (RoPE
 // on the last rope_dim dims, "DeepSeek V4-Pro" (llm-arch-kb), "Hybrid
@@ -32,7 +36,7 @@ constexpr int kWarps = kThreads / 32;
 struct StreamArgs {
   const __nv_bfloat16* tok;  // [B, L_cap, dim]
   const float* w_s;          // [dim]
-  const float* b_pos;        // [m]
+  const float* b_pos;        // [m + overlap]
   const float* gamma;        // [dim] or null
   __nv_bfloat16* out_bf16;   // [B, N_cap, dim] or null
   uint8_t* out_e4m3;         // [B, N_cap, dim] or null
@@ -45,6 +49,7 @@ struct PoolArgs {
   StreamArgs s[2];
   int nstreams;
   int B, m;
+  int overlap;             // tokens of block i-1 that entry i also pools
   int64_t L_cap, N_cap;
   const int64_t* ctx_len;  // [B] device, or null -> ctx_len_value
   int64_t ctx_len_value;
@@ -259,7 +264,10 @@ CSA_DEV void pool_stream(const PoolArgs& a, const StreamArgs& sa, float* smem) {
   constexpr int E = DIM / 32;
   using LN = Lane<DIM>;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int G = a.m <= 16 ? 1 : kWarps;           // warps per block
+  // Entry i pools the window of span = m + overlap tokens that ends with its
+  // own block: window position j holds token i*m - overlap + j.
+  const int span = a.m + a.overlap;
+  const int G = span <= 16 ? 1 : kWarps;           // warps per block
   const int per_cta = kWarps / G;                  // blocks per CTA
   const int64_t unit = (int64_t)blockIdx.x * per_cta + warp / G;  // (b, block) pair
   const int64_t total = (int64_t)a.B * a.n_blocks;
@@ -287,25 +295,30 @@ CSA_DEV void pool_stream(const PoolArgs& a, const StreamArgs& sa, float* smem) {
       L = a.ctx_len ? a.ctx_len[b] : a.ctx_len_value;
     }
     if (L > a.L_cap) L = a.L_cap;
-    int64_t rem = L - i * a.m;
-    present = rem <= 0 ? 0 : (rem < a.m ? (int)rem : a.m);
+    // Window positions [jlo, present) are present: none before token 0, none
+    // at or past the context end, and nothing at all while the block's own
+    // range is empty.
+    const int64_t rem = L - (i * a.m - a.overlap);
+    present = L - i * a.m <= 0 ? 0 : (rem < span ? (int)rem : span);
   }
+  const int jlo = active && i * a.m < a.overlap ? (int)(a.overlap - i * a.m) : 0;
   float ws[E];
 #pragma unroll
   for (int part = 0; part < LN::NPART; ++part)
 #pragma unroll
     for (int v = 0; v < LN::VEC; ++v) ws[part * LN::VEC + v] = __ldg(sa.w_s + LN::elem(lane, part, v));
 
-  const __nv_bfloat16* blk = sa.tok + ((int64_t)b * a.L_cap + i * a.m) * DIM;
+  // Row j of the window is blk + j*DIM (only rows j >= jlo are touched).
+  const __nv_bfloat16* blk = sa.tok + ((int64_t)b * a.L_cap + i * a.m - a.overlap) * DIM;
   float mx, l, acc[E];
   const int g = warp % G;
-  const int per_warp = (a.m + G - 1) / G;
+  const int per_warp = (span + G - 1) / G;
   // Rows in the buffer (fetched at once) and rows present (pooled).
-  const int64_t in_buf = active ? a.L_cap - i * a.m : 0;
-  const int avail = in_buf <= 0 ? 0 : (in_buf < a.m ? (int)in_buf : a.m);
-  const int j0 = g * per_warp;
-  const int j_load = max(j0, min(avail, j0 + per_warp));
-  const int j_use = max(j0, min(present, j0 + per_warp));
+  const int64_t in_buf = active ? a.L_cap - (i * a.m - a.overlap) : 0;
+  const int avail = in_buf <= 0 ? 0 : (in_buf < span ? (int)in_buf : span);
+  const int j0 = max(g * per_warp, jlo);
+  const int j_load = max(j0, min(avail, g * per_warp + per_warp));
+  const int j_use = max(j0, min(present, g * per_warp + per_warp));
   pool_tokens<DIM>(blk, j0, j_load, j_use, lane, ws, sa.b_pos, mx, l, acc);
 
   if (G == 1) {
@@ -379,6 +392,7 @@ cudaError_t launch_compress(const CompressLaunch& c, cudaStream_t stream) {
   for (int j = 0; j < 64; ++j) a.inv_freq[j] = c.inv_freq[j];
   a.B = c.B;
   a.m = c.m;
+  a.overlap = c.overlap;
   a.L_cap = c.L_cap;
   a.N_cap = c.N_cap;
   a.ctx_len = c.ctx_len;
@@ -388,7 +402,7 @@ cudaError_t launch_compress(const CompressLaunch& c, cudaStream_t stream) {
   a.pos_newest = c.pos_newest;
   a.eps = c.eps;
   a.status = c.status;
-  int G = c.m <= 16 ? 1 : kWarps;
+  int G = c.m + c.overlap <= 16 ? 1 : kWarps;
   int per_cta = kWarps / G;
   int64_t units = (int64_t)c.B * a.n_blocks;
   if (units == 0) return cudaSuccess;

@@ -12,6 +12,7 @@ namespace csa {
 
 struct CompressLaunch {
   int B, d, D_I, m;
+  int overlap;              // tokens of block i-1 that entry i also pools (b_pos has m + overlap)
   int64_t L_cap, N_cap;
   const void* kv_tok;
   const void* idx_tok;  // null: KV stream only
@@ -98,6 +99,26 @@ struct MqaLaunch {
 size_t mqa_workspace_bytes(int rows, int splits, int H, int D);
 int mqa_choose_splits(int rows, int64_t compressed_max, int window, int num_sms, int H);
 cudaError_t launch_mqa(const MqaLaunch& a, cudaStream_t stream);
+
+// One projection GEMM of the grouped output projection: for each group j,
+// C[t, j*N + n] = sum_k A[t, j*K + k] * W[j*N + n, k] (bf16 in, fp32
+// accumulate, bf16 out), or fp32 split-K partials reduced by a second kernel.
+struct ProjGemm {
+  const void* a;      // [T, lda] bf16 (lda >= groups * K)
+  int64_t lda;
+  const void* w;      // [w_rows, K] bf16, w_rows = groups * N
+  int64_t w_rows;
+  int K, N, groups, T;
+  int splits;         // split-K factor (partials in `part` when > 1)
+  void* c;            // [T, ldc] bf16
+  int ldc;
+  float* part;        // [splits, T, ldc] fp32 workspace (splits > 1)
+  int32_t* status;
+  int chained;        // see launch_pdl
+};
+cudaError_t launch_proj_gemm(const ProjGemm& g, cudaStream_t stream);
+int proj_token_tile(int T);
+int proj_choose_splits(int T, int N, int groups, int K, int num_sms);
 
 int device_sm_count();
 

@@ -34,9 +34,13 @@
 //     16x32bx2 TMEM access) run an online softmax with lazy rescaling (O is
 //     rescaled in TMEM only when the running max grows by more than 8) and
 //     write P (bf16) to shared memory in the MMA's K-major layout.
-// Splits of the KV list run on different CTA pairs; their (m, l, O) partials
-// are merged by mqa_combine_kernel, which also folds in the sink and applies
-// the inverse RoPE.  Every wait is bounded and reports CSA_ERR_DEVICE_TIMEOUT.
+// Splits of the KV list run on different CTAs; their (m, l, O) partials are
+// merged, with the sink folded in and the inverse RoPE applied, by the CTAs
+// themselves when the S splits of a head group form one thread-block
+// cluster (S <= 16: a cluster barrier, then each CTA merges a share of the
+// heads from L2), else by mqa_combine_kernel.  With one split per row the
+// attention CTA finishes its rows directly.  Every wait is bounded and
+// reports CSA_ERR_DEVICE_TIMEOUT.
 #include <algorithm>
 
 #include "common.cuh"
@@ -112,6 +116,11 @@ struct Params {
   // normalisation, inverse rotation, bf16 output and log-sum-exp) and no
   // merge runs.
   int fused;
+  // Several splits per row, launched as one cluster per (row, head group):
+  // after every CTA of the cluster has written its partial, the CTAs merge
+  // them themselves (each a share of the group's heads) and no merge kernel
+  // runs.
+  int cluster_merge;
   const float* sink;
   __nv_bfloat16* out;
   float* lse;
@@ -135,6 +144,138 @@ template <bool kCluster = false>
 CSA_DEV bool wait_all(uint64_t* bar, uint32_t parity, const Params& p, volatile int* abort_flag) {
   bool ok = mbar_wait<kCluster>(bar, parity, p.status, abort_flag);
   return __all_sync(0xffffffffu, ok);
+}
+
+// Merge of the split partials of one (row, head) by one warp: fold in the
+// sink, normalise, apply the inverse rotation, store bf16 (and the
+// log-sum-exp).  Lane l owns dims [l*VPL, (l+1)*VPL) (VPL = D/32), so the
+// output row leaves as one coalesced 32-lane store and the rotated pairs
+// (d, d + R/2) sit in lanes l and l ^ (R/2/VPL).  The S (max, sum) pairs
+// become one weight per split (wsplit: S floats of this warp's shared
+// memory); the partials are read G splits at a time with the next group's
+// loads in flight, the first group before the weights are known.
+// kLdg: the partials come from an earlier kernel (read-only path); otherwise
+// they were written during this kernel by other CTAs and are read from L2.
+template <int D, int R, int G, bool kLdg>
+CSA_DEV void merge_head(const Params& p, int row, int h, int lane, float* wsplit) {
+  constexpr int VPL = D / 32;     // dims per lane: 16 (D = 512) or 4 (D = 128)
+  constexpr int NW = VPL / 2;     // 32-bit words (fp16 pairs) per lane and split
+  static_assert(VPL == 16 || VPL == 4, "D must be 512 or 128");
+  const int S = p.splits;
+  const float* ml = p.part_ml + (int64_t)row * S * 2 * p.H;
+  const __half* src = p.part_o + ((int64_t)row * S * p.H + h) * D + lane * VPL;
+  const int64_t stride = (int64_t)p.H * D;
+  auto ld4 = [](const uint4* a) -> uint4 { return kLdg ? __ldg(a) : __ldcg(a); };
+  auto ld2 = [](const uint2* a) -> uint2 { return kLdg ? __ldg(a) : __ldcg(a); };
+  auto ldf = [](const float* a) -> float { return kLdg ? __ldg(a) : __ldcg(a); };
+  auto load = [&](int s, uint32_t (&v)[NW]) {
+    const __half* a = src + (int64_t)s * stride;
+    if constexpr (VPL == 16) {
+      *reinterpret_cast<uint4*>(&v[0]) = ld4(reinterpret_cast<const uint4*>(a));
+      *reinterpret_cast<uint4*>(&v[4]) = ld4(reinterpret_cast<const uint4*>(a) + 1);
+    } else {
+      *reinterpret_cast<uint2*>(&v[0]) = ld2(reinterpret_cast<const uint2*>(a));
+    }
+  };
+  uint32_t cur[G][NW], nxt[G][NW];
+#pragma unroll
+  for (int u = 0; u < G; ++u)
+    if (u < S) load(u, cur[u]);
+  const float LOG2E = 1.4426950408889634f;
+  const float z = p.sink[h];
+  const float z2 = z * LOG2E;  // log2 domain
+  float M = z2;
+  for (int s = lane; s < S; s += 32) M = fmaxf(M, ldf(ml + (int64_t)s * 2 * p.H + h));
+  M = warp_max(M);
+  const bool zero = z == INFINITY || M == -INFINITY;  // +inf sink, or nothing to attend
+  float L = 0.f;
+  if (!zero) {
+    for (int s = lane; s < S; s += 32) {
+      const float ms = ldf(ml + (int64_t)s * 2 * p.H + h);
+      const float w = ms == -INFINITY ? 0.f : ldf(ml + (int64_t)s * 2 * p.H + p.H + h) * exp2f(ms - M);
+      wsplit[s] = w;  // the split's stored output is O / l
+      L += w;
+    }
+    L = warp_sum(L);
+    if (z2 != -INFINITY) L += exp2f(z2 - M);
+  }
+  __syncwarp();
+  __nv_bfloat16* o = p.out + ((int64_t)row * p.H + h) * D + lane * VPL;
+  float acc[VPL];
+#pragma unroll
+  for (int e = 0; e < VPL; ++e) acc[e] = 0.f;
+  if (!zero) {
+    for (int s0 = 0; s0 < S; s0 += G) {
+      if (s0 + G < S) {
+#pragma unroll
+        for (int u = 0; u < G; ++u)
+          if (s0 + G + u < S) load(s0 + G + u, nxt[u]);
+      }
+#pragma unroll
+      for (int u = 0; u < G; ++u) {
+        if (s0 + u >= S) break;
+        const float w = wsplit[s0 + u];
+        if (w == 0.f) continue;  // empty split: its partial was never written
+#pragma unroll
+        for (int i = 0; i < NW; ++i) {
+          const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&cur[u][i]));
+          acc[2 * i] = fmaf(f.x, w, acc[2 * i]);
+          acc[2 * i + 1] = fmaf(f.y, w, acc[2 * i + 1]);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < G; ++u)
+#pragma unroll
+        for (int i = 0; i < NW; ++i) cur[u][i] = nxt[u][i];
+    }
+    const float invL = 1.0f / L;
+#pragma unroll
+    for (int e = 0; e < VPL; ++e) acc[e] *= invL;
+    if constexpr (R > 0) {
+      // Rotation by -pos: pair j of the last R dims is (d0 + j, d0 + j + R/2).
+      constexpr int K = R / 2 / VPL;  // lanes per rotated half
+      constexpr int L0 = 32 - 2 * K;  // first lane holding rotated dims
+      static_assert(K >= 1 && (K & (K - 1)) == 0, "rotated halves must span whole lanes");
+      const int64_t pos = row_pos(p, row);
+      float sn = 0.f, cs = 1.f;
+      if (lane < R / 2) sincos_reduced((double)pos * p.inv_freq[lane], &sn, &cs);
+      const bool rot = lane >= L0;
+      const bool first = rot && lane - L0 < K;
+      const int jb = rot ? ((lane - L0) % K) * VPL : 0;
+#pragma unroll
+      for (int e = 0; e < VPL; ++e) {
+        const float c = __shfl_sync(0xffffffffu, cs, jb + e);
+        const float sj = __shfl_sync(0xffffffffu, sn, jb + e);
+        const float other = __shfl_xor_sync(0xffffffffu, acc[e], K);
+        if (rot) acc[e] = first ? acc[e] * c + other * sj : acc[e] * c - other * sj;
+      }
+    }
+  }
+  uint32_t packed[NW];
+#pragma unroll
+  for (int i = 0; i < NW; ++i) packed[i] = pack_bf16(acc[2 * i], acc[2 * i + 1]);
+  if constexpr (VPL == 16) {
+    reinterpret_cast<uint4*>(o)[0] = *reinterpret_cast<const uint4*>(&packed[0]);
+    reinterpret_cast<uint4*>(o)[1] = *reinterpret_cast<const uint4*>(&packed[4]);
+  } else {
+    *reinterpret_cast<uint2*>(o) = *reinterpret_cast<const uint2*>(&packed[0]);
+  }
+  if (p.lse && lane == 0)
+    p.lse[(int64_t)row * p.H + h] =
+        zero ? (z == INFINITY ? INFINITY : -INFINITY) : (M + log2f(L)) / LOG2E;
+}
+
+// The split merge as its own kernel (several splits per row when the
+// in-cluster merge is not available): one warp per (row, head), four per CTA.
+template <int D, int R, int G>
+__global__ void __launch_bounds__(128) mqa_combine_kernel(const Params p, int rows) {
+  extern __shared__ float wsm[];  // [4 warps][S] split weights
+  pdl_trigger();
+  pdl_wait();  // the partials come from the attention kernel
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t gw = (int64_t)blockIdx.x * 4 + warp;
+  if (gw >= (int64_t)rows * p.H) return;
+  merge_head<D, R, G, true>(p, (int)(gw / p.H), (int)(gw % p.H), lane, wsm + warp * p.splits);
 }
 
 template <int D, int R>
@@ -165,10 +306,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   pdl_trigger();
-  // H > 64: CTAs 2s and 2s+1 of split s own heads 0..63 and 64..H-1.
+  // H > 64: CTA g*S + s (g = 0, 1) owns heads [64g, 64g+64) of split s, so
+  // the S splits of one head group are consecutive (one cluster when the
+  // partials are merged in-cluster).
   const bool pair = p.H > HC;
-  const int hg0 = pair ? (blockIdx.x & 1) * HC : 0;  // first head of this CTA
-  const int split = pair ? blockIdx.x >> 1 : blockIdx.x;
+  const int hg0 = pair ? (int)(blockIdx.x / p.splits) * HC : 0;  // first head of this CTA
+  const int split = (int)(blockIdx.x % p.splits);
   const int row = blockIdx.y;
   const int b = row / p.Q;
 
@@ -804,10 +947,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       if (head_ok) {
-        fence_proxy_async_smem();
-        bulk_store(po, ob, (D / 2) * 2);
-        bulk_commit();
-        bulk_wait_read();  // shared memory may be released; the kernel end publishes the data
+        if (p.cluster_merge && !p.fused) {
+          // Plain stores: the other CTAs of the cluster read the partial
+          // back after the cluster barrier below.
+          const uint4* s4 = reinterpret_cast<const uint4*>(ob);
+          uint4* g4 = reinterpret_cast<uint4*>(po);
+#pragma unroll 8
+          for (int i = 0; i < D / 16; ++i) g4[i] = s4[i];
+        } else {
+          fence_proxy_async_smem();
+          bulk_store(po, ob, (D / 2) * 2);
+          bulk_commit();
+          bulk_wait_read();  // shared memory may be released; the kernel end publishes the data
+        }
       }
       if (head_ok && hf == 0) {
         if (p.fused) {
@@ -831,131 +983,56 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem, C::kAlloc);
   }
+  if (p.cluster_merge) {
+    // Every CTA of the cluster (the S splits of this head group) has written
+    // its partial and its (max, sum): the release / acquire cluster barrier
+    // publishes them, and CTA `split` then merges heads split, split + S, ...
+    // of the group, one warp per head.  Every thread of every CTA reaches
+    // this point exactly once (no role returns early).
+    __threadfence();
+    __syncwarp();
+    cluster_sync();
+    const int nh = pair ? min(HC, p.H - hg0) : p.H;
+    float* wsplit = reinterpret_cast<float*>(stages) + warp * 32;  // S <= 16 weights
+    for (int j = split + p.splits * warp; j < nh; j += p.splits * (kThreads / 32))
+      merge_head<D, R, 4, false>(p, row, hg0 + j, lane, wsplit);
+  }
 }
 
-// Merge the split partials of one (row, head) per warp: fold in the sink,
-// normalise, apply the inverse rotation, store bf16 (and the log-sum-exp).
-// Lane l owns dims [l*VPL, (l+1)*VPL) (VPL = D/32), so the output row leaves
-// as one coalesced 32-lane store and the rotated pairs (d, d + R/2) sit in
-// lanes l and l ^ (R/2/VPL).  The S (max, sum) pairs become one weight per
-// split (per-warp shared memory); the partials are read G splits at a time
-// with the next group's loads in flight, the first group before the weights
-// are known.  Four warps per CTA.
-template <int D, int R, int G>
-__global__ void __launch_bounds__(128) mqa_combine_kernel(const Params p, int rows,
-                                                          const float* __restrict__ sink,
-                                                          __nv_bfloat16* __restrict__ out,
-                                                          float* __restrict__ lse) {
-  constexpr int VPL = D / 32;     // dims per lane: 16 (D = 512) or 4 (D = 128)
-  constexpr int NW = VPL / 2;     // 32-bit words (fp16 pairs) per lane and split
-  static_assert(VPL == 16 || VPL == 4, "D must be 512 or 128");
-  extern __shared__ float wsm[];  // [4 warps][S] split weights
-  pdl_trigger();
-  pdl_wait();  // the partials come from the attention kernel
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t gw = (int64_t)blockIdx.x * 4 + warp;
-  if (gw >= (int64_t)rows * p.H) return;
-  const int row = (int)(gw / p.H), h = (int)(gw % p.H);
-  const int S = p.splits;
-  float* wsplit = wsm + warp * S;
-  const float* ml = p.part_ml + (int64_t)row * S * 2 * p.H;
-  const __half* src = p.part_o + ((int64_t)row * S * p.H + h) * D + lane * VPL;
-  const int64_t stride = (int64_t)p.H * D;
-  auto load = [&](int s, uint32_t (&v)[NW]) {
-    const __half* a = src + (int64_t)s * stride;
-    if constexpr (VPL == 16) {
-      *reinterpret_cast<uint4*>(&v[0]) = __ldg(reinterpret_cast<const uint4*>(a));
-      *reinterpret_cast<uint4*>(&v[4]) = __ldg(reinterpret_cast<const uint4*>(a) + 1);
-    } else {
-      *reinterpret_cast<uint2*>(&v[0]) = __ldg(reinterpret_cast<const uint2*>(a));
-    }
-  };
-  uint32_t cur[G][NW], nxt[G][NW];
-#pragma unroll
-  for (int u = 0; u < G; ++u)
-    if (u < S) load(u, cur[u]);
-  const float LOG2E = 1.4426950408889634f;
-  const float z = sink[h];
-  const float z2 = z * LOG2E;  // log2 domain
-  float M = z2;
-  for (int s = lane; s < S; s += 32) M = fmaxf(M, ml[(int64_t)s * 2 * p.H + h]);
-  M = warp_max(M);
-  const bool zero = z == INFINITY || M == -INFINITY;  // +inf sink, or nothing to attend
-  float L = 0.f;
-  if (!zero) {
-    for (int s = lane; s < S; s += 32) {
-      const float ms = ml[(int64_t)s * 2 * p.H + h];
-      const float w = ms == -INFINITY ? 0.f : ml[(int64_t)s * 2 * p.H + p.H + h] * exp2f(ms - M);
-      wsplit[s] = w;  // the split's stored output is O / l
-      L += w;
-    }
-    L = warp_sum(L);
-    if (z2 != -INFINITY) L += exp2f(z2 - M);
+// Whether S CTAs of the attention kernel (one per SM) can run as one
+// thread-block cluster on this device: S <= 8 always can in principle, up to
+// 16 with the non-portable cluster size; the occupancy query says whether at
+// least one such cluster fits.  Cached per (device, kernel variant, S).
+bool cluster_fits(const void* kern, int variant, int S, size_t smem) {
+  static int cached[64][8][17] = {};  // 0 unknown, 1 yes, 2 no
+  if (S < 2 || S > 16) return false;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64 || variant < 0 || variant >= 8)
+    return false;
+  int& c = cached[dev][variant][S];
+  if (c) return c == 1;
+  bool ok = true;
+  if (S > 8 && cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
+                   cudaSuccess)
+    ok = false;
+  if (ok) {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(S, 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = S;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    ok = cudaOccupancyMaxActiveClusters(&n, kern, &cfg) == cudaSuccess && n >= 1;
   }
-  __syncwarp();
-  __nv_bfloat16* o = out + ((int64_t)row * p.H + h) * D + lane * VPL;
-  float acc[VPL];
-#pragma unroll
-  for (int e = 0; e < VPL; ++e) acc[e] = 0.f;
-  if (!zero) {
-    for (int s0 = 0; s0 < S; s0 += G) {
-      if (s0 + G < S) {
-#pragma unroll
-        for (int u = 0; u < G; ++u)
-          if (s0 + G + u < S) load(s0 + G + u, nxt[u]);
-      }
-#pragma unroll
-      for (int u = 0; u < G; ++u) {
-        if (s0 + u >= S) break;
-        const float w = wsplit[s0 + u];
-        if (w == 0.f) continue;  // empty split: its partial was never written
-#pragma unroll
-        for (int i = 0; i < NW; ++i) {
-          const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&cur[u][i]));
-          acc[2 * i] = fmaf(f.x, w, acc[2 * i]);
-          acc[2 * i + 1] = fmaf(f.y, w, acc[2 * i + 1]);
-        }
-      }
-#pragma unroll
-      for (int u = 0; u < G; ++u)
-#pragma unroll
-        for (int i = 0; i < NW; ++i) cur[u][i] = nxt[u][i];
-    }
-    const float invL = 1.0f / L;
-#pragma unroll
-    for (int e = 0; e < VPL; ++e) acc[e] *= invL;
-    if constexpr (R > 0) {
-      // Rotation by -pos: pair j of the last R dims is (d0 + j, d0 + j + R/2).
-      constexpr int K = R / 2 / VPL;  // lanes per rotated half
-      constexpr int L0 = 32 - 2 * K;  // first lane holding rotated dims
-      static_assert(K >= 1 && (K & (K - 1)) == 0, "rotated halves must span whole lanes");
-      const int64_t pos = row_pos(p, row);
-      float sn = 0.f, cs = 1.f;
-      if (lane < R / 2) sincos_reduced((double)pos * p.inv_freq[lane], &sn, &cs);
-      const bool rot = lane >= L0;
-      const bool first = rot && lane - L0 < K;
-      const int jb = rot ? ((lane - L0) % K) * VPL : 0;
-#pragma unroll
-      for (int e = 0; e < VPL; ++e) {
-        const float c = __shfl_sync(0xffffffffu, cs, jb + e);
-        const float sj = __shfl_sync(0xffffffffu, sn, jb + e);
-        const float other = __shfl_xor_sync(0xffffffffu, acc[e], K);
-        if (rot) acc[e] = first ? acc[e] * c + other * sj : acc[e] * c - other * sj;
-      }
-    }
-  }
-  uint32_t packed[NW];
-#pragma unroll
-  for (int i = 0; i < NW; ++i) packed[i] = pack_bf16(acc[2 * i], acc[2 * i + 1]);
-  if constexpr (VPL == 16) {
-    reinterpret_cast<uint4*>(o)[0] = *reinterpret_cast<const uint4*>(&packed[0]);
-    reinterpret_cast<uint4*>(o)[1] = *reinterpret_cast<const uint4*>(&packed[4]);
-  } else {
-    *reinterpret_cast<uint2*>(o) = *reinterpret_cast<const uint2*>(&packed[0]);
-  }
-  if (lse && lane == 0)
-    lse[(int64_t)row * p.H + h] =
-        zero ? (z == INFINITY ? INFINITY : -INFINITY) : (M + log2f(L)) / LOG2E;
+  if (!ok) cudaGetLastError();  // a refused query is not the caller's error
+  c = ok ? 1 : 2;
+  return ok;
 }
 
 template <int D, int R>
@@ -1008,17 +1085,23 @@ cudaError_t launch_impl(const MqaLaunch& a, cudaStream_t stream) {
   const size_t smem = 1024 + (size_t)C::kStages * C::kStageBytes + 2 * C::kPBytes +
                       C::kStages * sizeof(Meta) + 32 * 8 + 16;
   auto kern = mqa_heads_kernel<D, R>;
-  e = ensure_smem_attr(reinterpret_cast<const void*>(kern), 3 + (D == 512 ? 0 : 3) + R / 32, smem);
+  const int variant = (D == 512 ? 0 : 3) + R / 32;
+  e = ensure_smem_attr(reinterpret_cast<const void*>(kern), 3 + variant, smem);
   if (e != cudaSuccess) return e;
   dim3 grid(cps * a.splits, rows, 1);
+  if (!p.fused && cluster_fits(reinterpret_cast<const void*>(kern), variant, a.splits, smem)) {
+    // The splits of each head group form one cluster and merge in-kernel.
+    p.cluster_merge = 1;
+    return launch_pdl(kern, grid, dim3(kThreads), smem, stream, a.splits, a.chained, map_q, box_c,
+                      box_t, p);
+  }
   e = launch_pdl(kern, grid, dim3(kThreads), smem, stream, 0, a.chained, map_q, box_c, box_t, p);
   if (e != cudaSuccess) return e;
   if (p.fused) return cudaSuccess;  // the attention kernel finished the rows
   const unsigned nblk = (unsigned)(((int64_t)rows * a.H + 3) / 4);
   const size_t wsm = (size_t)4 * a.splits * sizeof(float);
   auto merge = mqa_combine_kernel<D, R, 4>;
-  return launch_pdl(merge, dim3(nblk), dim3(128), wsm, stream, 0, 1, p, rows, a.sink,
-                    reinterpret_cast<__nv_bfloat16*>(a.out), a.lse);
+  return launch_pdl(merge, dim3(nblk), dim3(128), wsm, stream, 0, 1, p, rows);
 }
 
 }  // namespace

@@ -6,7 +6,9 @@
 // ascending; NaN below every number; -0 == +0.  Output: ascending indices,
 // padded with -1, and the count min(k, n_vis).
 //
-// Design: one thread-block cluster of C CTAs (C = 1..8) per query row.  CTA r
+// Rows that fit in one CTA's shared memory (up to ~47K scores) are ranked by
+// topk_row_kernel, one CTA per row; longer rows by topk_kernel:
+// one thread-block cluster of C CTAs (C = 1..16) per query row.  CTA r
 // keeps its slice of the row in shared memory as order-preserving 32-bit
 // keys.  A radix select finds the exact k-th largest key over the whole row:
 //   - every exchange is a push of plain 16-byte stores: each CTA writes its
@@ -34,7 +36,7 @@ namespace {
 
 constexpr int kThreads = 1024;
 constexpr int kDigitBits = 8;  // radix digit width (256 bins)
-constexpr int kMaxK = 1024;
+constexpr int kMaxK = 2048;
 constexpr int kMaxC = 16;      // CTAs per cluster (16 needs the non-portable size)
 
 struct Params {
@@ -308,6 +310,219 @@ __global__ void __launch_bounds__(kThreads, 1) topk_kernel(const Params p) {
   if (r == 0 && tid == 0) p.cnt[row] = p.k;
 }
 
+
+// One CTA per query row, for rows whose visible scores fit in shared memory
+// (decode at 128K context, every prefill row).  The same radix select as
+// above with no cluster exchange: 1024 threads hold the row as keys in shared
+// memory, a block-wide (min, max) gives the common prefix, and each round
+// histograms the next kRowBits bits of the keys that still match the prefix
+// (shared-memory atomics) and finds the threshold digit with a block scan.
+// Rounds stop once the threshold bin is taken whole; the index-ordered
+// output is the same ballot-ranked pass.  Only __syncthreads barriers.
+constexpr int kRowBits = 12;
+
+struct RowShared {
+  uint32_t hist[1 << kRowBits];
+  uint32_t warp_a[32], warp_b[32];
+  uint32_t scan[33];
+  uint32_t bcast[4];
+};
+
+// Exclusive prefix over the block of per-thread values (1024 threads, one
+// value each); warp_tot is 33 words of shared scratch.
+CSA_DEV uint32_t block_excl_scan(uint32_t v, uint32_t* warp_tot) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint32_t incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) warp_tot[warp] = incl;
+  cta_sync();
+  if (warp == 0) {
+    const uint32_t t = warp_tot[lane];
+    uint32_t x = t;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    warp_tot[lane] = x - t;  // exclusive over warps
+  }
+  cta_sync();
+  return warp_tot[warp] + incl - v;
+}
+
+__global__ void __launch_bounds__(kThreads, 1) topk_row_kernel(const Params p) {
+  constexpr int kBins = 1 << kRowBits;
+  constexpr int kPer = kBins / kThreads;  // bins per thread in the digit scan
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  RowShared& sh = *reinterpret_cast<RowShared*>(smem_raw);
+  uint32_t* keys = reinterpret_cast<uint32_t*>(smem_raw + sizeof(RowShared));
+  const int row = blockIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int64_t pos = p.pos_q ? p.pos_q[row] : p.pos_base + row % p.Q;
+  pdl_trigger();
+  pdl_wait();  // the scores come from the indexer kernel
+  int64_t n64 = pos < 0 ? 0 : (pos + 1) / p.m;
+  if (n64 > p.N_cap) {
+    n64 = p.N_cap;
+    if (tid == 0) report(p.status, CSA_ERR_CAPACITY);
+  }
+  const int n = (int)n64;
+  int32_t* out = p.idx + (int64_t)row * p.k;
+  if (n <= p.k) {  // every visible entry is kept
+    for (int j = tid; j < p.k; j += kThreads) out[j] = j < n ? j : -1;
+    if (tid == 0) p.cnt[row] = n;
+    return;
+  }
+  // The visible scores as order-preserving keys, with this thread's min/max.
+  const float* src = p.scores + (int64_t)row * p.N_cap;
+  uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
+  const bool vec = ((reinterpret_cast<uintptr_t>(src) & 15u) == 0);
+  const int n4 = vec ? (n & ~3) : 0;
+#pragma unroll 4
+  for (int i = 4 * tid; i < n4; i += 4 * kThreads) {
+    const float4 v = __ldg(reinterpret_cast<const float4*>(src + i));
+    const uint4 u = make_uint4(orderable(v.x), orderable(v.y), orderable(v.z), orderable(v.w));
+    *reinterpret_cast<uint4*>(keys + i) = u;
+    kmin = min(kmin, min(min(u.x, u.y), min(u.z, u.w)));
+    kmax = max(kmax, max(max(u.x, u.y), max(u.z, u.w)));
+  }
+  for (int i = n4 + tid; i < n; i += kThreads) {
+    const uint32_t u = orderable(__ldg(src + i));
+    keys[i] = u;
+    kmin = min(kmin, u);
+    kmax = max(kmax, u);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
+    kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
+  }
+  if (lane == 0) {
+    sh.warp_a[warp] = kmin;
+    sh.warp_b[warp] = kmax;
+  }
+  for (int b = tid; b < kBins; b += kThreads) sh.hist[b] = 0;
+  cta_sync();
+  uint32_t gmin = sh.warp_a[lane], gmax = sh.warp_b[lane];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    gmin = min(gmin, __shfl_xor_sync(0xffffffffu, gmin, o));
+    gmax = max(gmax, __shfl_xor_sync(0xffffffffu, gmax, o));
+  }
+  cta_sync();  // every warp has read the min / max slots
+
+  uint32_t prefix, mask;
+  uint32_t k_rem = (uint32_t)p.k;
+  if (gmin == gmax) {
+    prefix = gmin;
+    mask = 0xFFFFFFFFu;
+  } else {
+    const int top = 31 - __clz(gmin ^ gmax);
+    mask = top == 31 ? 0u : (0xFFFFFFFFu << (top + 1));
+    prefix = gmin & mask;
+    int shift = top + 1;
+    while (shift > 0) {
+      const int width = shift >= kRowBits ? kRowBits : shift;
+      shift -= width;
+      const uint32_t dmask = (1u << width) - 1u;
+#pragma unroll 4
+      for (int i = tid; i < n; i += kThreads) {
+        const uint32_t key = keys[i];
+        if ((key & mask) == prefix) atomicAdd(&sh.hist[(key >> shift) & dmask], 1u);
+      }
+      cta_sync();
+      // Thread t owns digits nb-1-t*kPer down to nb-(t+1)*kPer (descending),
+      // so an exclusive scan over t counts the keys in higher digits.
+      const int nb = (int)dmask + 1;
+      uint32_t c[kPer];
+      uint32_t local = 0;
+#pragma unroll
+      for (int j = 0; j < kPer; ++j) {
+        const int d = nb - 1 - (tid * kPer + j);
+        c[j] = d >= 0 ? sh.hist[d] : 0u;
+        local += c[j];
+      }
+      uint32_t above = block_excl_scan(local, sh.scan);
+#pragma unroll
+      for (int j = 0; j < kPer; ++j) {
+        const int d = nb - 1 - (tid * kPer + j);
+        if (d >= 0 && above < k_rem && above + c[j] >= k_rem) {
+          sh.bcast[0] = (uint32_t)d;
+          sh.bcast[1] = above;
+          sh.bcast[2] = c[j];
+        }
+        above += c[j];
+      }
+      for (int b = tid; b < kBins; b += kThreads) sh.hist[b] = 0;
+      cta_sync();
+      const uint32_t d = sh.bcast[0], abv = sh.bcast[1], cnt_d = sh.bcast[2];
+      cta_sync();  // bcast is read before the next round can rewrite it
+      k_rem -= abv;
+      prefix |= d << shift;
+      mask |= dmask << shift;
+      if (cnt_d == k_rem) break;  // the whole bin is taken
+    }
+  }
+  const uint32_t T = prefix, M = mask, need_eq = k_rem;
+
+  // Index-ordered output: warp w owns positions [w*chunk, (w+1)*chunk).
+  const int chunk = (((n + 31) / 32) + 31) & ~31;
+  const int w0 = min(n, warp * chunk), w1 = min(n, w0 + chunk);
+  uint32_t n_gt = 0, n_eq = 0;
+  for (int i = w0 + lane; i < w1; i += 32) {
+    const uint32_t km = keys[i] & M;
+    n_gt += km > T;
+    n_eq += km == T;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    n_gt += __shfl_xor_sync(0xffffffffu, n_gt, o);
+    n_eq += __shfl_xor_sync(0xffffffffu, n_eq, o);
+  }
+  if (lane == 0) {
+    sh.warp_a[warp] = n_gt;
+    sh.warp_b[warp] = n_eq;
+  }
+  cta_sync();
+  if (warp == 0) {
+    const uint32_t a = sh.warp_a[lane], b = sh.warp_b[lane];
+    uint32_t sa = a, sb = b;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t ya = __shfl_up_sync(0xffffffffu, sa, o);
+      const uint32_t yb = __shfl_up_sync(0xffffffffu, sb, o);
+      if (lane >= o) {
+        sa += ya;
+        sb += yb;
+      }
+    }
+    sh.warp_a[lane] = sa - a;
+    sh.warp_b[lane] = sb - b;
+  }
+  cta_sync();
+  uint32_t gt_run = sh.warp_a[warp], eq_run = sh.warp_b[warp];
+  const uint32_t lt = (1u << lane) - 1u;
+  for (int i = w0 + lane; i - lane < w1; i += 32) {
+    const uint32_t km = i < w1 ? keys[i] & M : 0u;
+    const bool gt = i < w1 && km > T;
+    const bool eq = i < w1 && km == T;
+    const uint32_t bg = __ballot_sync(0xffffffffu, gt);
+    const uint32_t be = __ballot_sync(0xffffffffu, eq);
+    const uint32_t eq_rank = eq_run + __popc(be & lt);
+    if (gt || (eq && eq_rank < need_eq)) {
+      const uint32_t o = gt_run + __popc(bg & lt) + min(need_eq, eq_rank);
+      if (o < (uint32_t)p.k) out[o] = i;
+    }
+    gt_run += __popc(bg);
+    eq_run += __popc(be);
+  }
+  if (tid == 0) p.cnt[row] = p.k;
+}
+
 }  // namespace
 
 // Largest cluster size (8 or 16) that can be resident for this kernel and
@@ -346,9 +561,32 @@ int max_cluster(const void* kern, size_t smem) {
   return best;
 }
 
+// Rows of at most this many scores take the one-CTA-per-row kernel.
+constexpr int64_t kRowMaxScores = (200 * 1024 - (int64_t)sizeof(RowShared)) / 4;
+
 cudaError_t launch_topk(const TopkLaunch& a, cudaStream_t stream) {
   if (a.rows < 1) return cudaSuccess;
   if (a.rows > 65535 || a.k > kMaxK) return cudaErrorInvalidConfiguration;
+  if (a.N_cap <= kRowMaxScores) {
+    Params p{};
+    p.Q = a.Q;
+    p.m = a.m;
+    p.k = a.k;
+    p.C = 1;
+    p.N_cap = a.N_cap;
+    p.slice = a.N_cap;
+    p.scores = a.scores;
+    p.pos_q = a.pos_q;
+    p.pos_base = a.pos_base;
+    p.idx = a.idx;
+    p.cnt = a.cnt;
+    p.status = a.status;
+    const size_t smem = sizeof(RowShared) + (size_t)((a.N_cap + 3) / 4 * 4) * 4;
+    cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(topk_row_kernel), 3, smem);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(topk_row_kernel, dim3(a.rows), dim3(kThreads), smem, stream, 0, a.chained,
+                      p);
+  }
   const int sms = device_sm_count();
   const int need = (int)((a.N_cap + 32767) / 32768);
   if (need > 8) return cudaErrorInvalidValue;

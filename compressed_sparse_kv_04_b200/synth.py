@@ -63,11 +63,11 @@ def e4m3_codes(shape, seed, name, device="cpu") -> torch.Tensor:
 
 
 def pool_params(w, device="cpu", indexer=False):
-    """(w_s [dim], b_pos [m]) for the KV stream, or for the indexer stream."""
+    """(w_s [dim], b_pos [m + overlap]) for the KV stream, or for the indexer stream."""
     dim = w.D_I if indexer else w.d
     ns, nb = ("w_s_idx", "b_pos_idx") if indexer else ("w_s", "b_pos")
     return (normal_f32((dim,), w.seed, ns, 0.02, device),
-            normal_f32((w.m,), w.seed, nb, 0.1, device))
+            normal_f32((w.m + getattr(w, "overlap", 0),), w.seed, nb, 0.1, device))
 
 
 def token_streams(w, L_cap=None, device="cpu"):

@@ -67,9 +67,9 @@ typedef enum {
 
 /* Shapes and constants shared by the calls of one layer.
  * Supported: d in {128, 512}; 1 <= H <= 128; H_I in {1..64}, D_I in {64, 128}
- * (indexer calls only); 1 <= k <= 1024; 0 <= window <= 1024; rope_dim in
+ * (indexer calls only); 1 <= k <= 2048; 0 <= window <= 1024; rope_dim in
  * {0, 32, 64} and <= d/4 (attention calls); 1 <= m <= 128 (CSA uses 4, HCA
- * 128); eps > 0. */
+ * 128); 0 <= overlap <= m with m + overlap <= 128; eps > 0. */
 typedef struct {
   int B;               /* sequences in the batch */
   int d;               /* KV entry dim == attention head dim D ([P5]: 512) */
@@ -84,6 +84,9 @@ typedef struct {
   float softmax_scale; /* logit scale; 0 selects 1/sqrt(d) */
   const double* rope_inv_freq; /* host, [rope_dim/2] angle per position for
                                   pair j; NULL selects 10000^(-2j/rope_dim) */
+  int overlap;         /* compression: tokens of block i-1 that entry i also
+                          pools (0 = non-overlapping blocks; 0..m, see
+                          csa_compress); b_pos then holds m + overlap values */
 } csa_params;
 
 /* Operation selector for csa_workspace_bytes(). */
@@ -175,7 +178,15 @@ csa_status hca_compress(const csa_params* p, const void* kv_tok, int64_t L_cap,
 
 /* ---------------------------------------------------------------------------
  * KV compression, CSA form ([P2] CSA step 1; [P5] CSA bullet: m = 4).
- * The KV stream is pooled exactly as hca_compress does.  When idx_tok is not
+ * The KV stream is pooled exactly as hca_compress does.
+ * Overlapping variant (p->overlap > 0; [P2] states "no overlap" for HCA
+ * only and gives no rule for CSA, so this is the build's reading): entry i
+ * pools the window of m + overlap tokens t = i*m - overlap + j (j < m +
+ * overlap), those with 0 <= t < ctx_len, scored with b_pos[j]; b_pos then
+ * holds m + overlap values.  The entry is still written once its own block
+ * has a token, visible once its own block is complete, and rotated to
+ * (i+1)*m - 1.  The same holds for every call that compresses (the prefill
+ * chunks and the decode steps).  When idx_tok is not
  * NULL, the indexer-key stream idx_tok [B, L_cap, D_I] bf16 is pooled by the
  * same operation with its own w_s_idx [D_I] and b_pos_idx [m] (no gain),
  * and each pooled row x is stored in E4M3 ([P3]: the indexer is low
@@ -410,6 +421,40 @@ csa_status hca_prefill_chunk(const csa_params* p, int64_t P, int T, const void* 
                              const float* sink, const float* gamma_q, const float* gamma_kv,
                              void* out, float* lse, void* ws, size_t ws_bytes,
                              int32_t* dev_status, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Grouped output projection ("DeepSeek V4 technical report" (agentupdate.ai),
+ * 混合注意力机制, item 分组输出投影: because the head dim is 512, the heads'
+ * outputs are not projected straight back to the model dim d; the n_h heads
+ * are split into g groups, each group is projected to an intermediate dim
+ * d_g, and the concatenation is projected back to d.  "DeepSeek V4-Pro"
+ * (llm-arch-kb), "1. Hybrid attention": g = 16, d_g = 1024.)
+ *
+ * For every token t (the rows of the attention output o):
+ *   y[t, j*d_g + r] = sum_c W_g[j, r, c] * o[t, j*(H/g)*D + c]   j < g, r < d_g
+ *   z[t, n]         = sum_i W_o[n, i] * y[t, i]                  n < d_model
+ * i.e. group j reads heads j*H/g .. (j+1)*H/g - 1 of o (contiguous,
+ * head-major).  No bias and no nonlinearity between the two projections (the
+ * pages give none).  bf16 inputs, fp32 accumulation on the tensor cores, y
+ * stored in bf16 before the second projection, z stored in bf16.  The pages
+ * do not give d; any multiple of 128 is supported.
+ *
+ *   o   [T, H, D] bf16 (device)             attention output
+ *   w_g [g, d_g, (H/g)*D] bf16 (device)     rows are outputs
+ *   w_o [d_model, g*d_g] bf16 (device)      rows are outputs
+ *   y   [T, g*d_g] bf16 (device, written) or NULL (then kept in the workspace)
+ *   z   [T, d_model] bf16 (device, written)
+ * Supported: g divides H; (H/g)*D and g*d_g multiples of 64; d_g and
+ * d_model multiples of 128; T >= 1.  Anything else returns
+ * CSA_ERR_UNSUPPORTED_SHAPE (or CSA_ERR_INVALID_ARG for values < 1).
+ * Workspace: grouped_out_proj_workspace_bytes(T, H, D, g, d_g, d_model)
+ * (0 for unsupported arguments); CSA_ERR_WORKSPACE when smaller.
+ * ------------------------------------------------------------------------- */
+size_t grouped_out_proj_workspace_bytes(int T, int H, int D, int g, int d_g, int d_model);
+
+csa_status grouped_out_proj(int T, int H, int D, int g, int d_g, int d_model, const void* o,
+                            const void* w_g, const void* w_o, void* y, void* z, void* ws,
+                            size_t ws_bytes, int32_t* dev_status, void* stream);
 
 #ifdef __cplusplus
 }

@@ -80,7 +80,7 @@ def test_null_tensor_rejected_before_launch(L):
 
 
 def test_indexer_shape_limits(L):
-    for kw in (dict(D_I=96), dict(H_I=65), dict(k=1025), dict(k=0)):
+    for kw in (dict(D_I=96), dict(H_I=65), dict(k=2049), dict(k=0)):
         p = P(**kw)
         st = L.lightning_index_topk(C.byref(p), 1, None, None, None, None, None, 1024, None,
                                     None, None, None, None, 0, None, None)
@@ -128,7 +128,7 @@ def test_decode_step_argument_checks(L):
     assert L.csa_decode_step(*n) == 1            # pos_q (and the rest) NULL
     p = P(B=2, k=4096)
     n[0] = C.byref(p)
-    assert L.csa_decode_step(*n) in (1, 2)       # k outside 1..1024 or NULL pointers
+    assert L.csa_decode_step(*n) in (1, 2)       # k outside 1..2048 or NULL pointers
     h = [None] * 19
     h[0] = C.byref(P(B=2, m=128))
     h[3], h[8], h[16] = 1 << 12, 32, 0
@@ -224,3 +224,26 @@ def test_params_for_applies_yarn_to_a_yarn_workload(L, orc):
     assert abs(p.softmax_scale - ref) <= ref * 2.0 ** -24
     plain = binding.params_for(configs.CSA_128K)
     assert not plain.rope_inv_freq and plain.softmax_scale == 0.0
+
+
+# ------------------------------------------ grouped output projection (host) --
+@pytest.mark.parametrize("shape,code", [((8, 128, 512, 16, 1024, 7168), 0),
+                                        ((8, 128, 512, 12, 1024, 7168), 2),   # g does not divide H
+                                        ((8, 128, 512, 16, 1000, 7168), 2),   # d_g % 128
+                                        ((8, 128, 512, 16, 1024, 7000), 2),   # d % 128
+                                        ((0, 128, 512, 16, 1024, 7168), 1),
+                                        ((8, 128, 36, 16, 1024, 7168), 2)])   # (H/g)*D % 64
+def test_grouped_out_proj_argument_checks(L, shape, code):
+    n = L.grouped_out_proj_workspace_bytes(*shape)
+    assert (n > 0) == (code == 0)
+    # NULL tensors: the shape error wins, else the pointer check.
+    st = L.grouped_out_proj(*shape, None, None, None, None, None, None, 0, None, None)
+    assert st == (code if code else 1)
+
+
+def test_grouped_out_proj_workspace_grows_with_tokens(L):
+    a = L.grouped_out_proj_workspace_bytes(8, 128, 512, 16, 1024, 7168)
+    b = L.grouped_out_proj_workspace_bytes(4096, 128, 512, 16, 1024, 7168)
+    assert 0 < a < b
+    # At least the bf16 intermediate y.
+    assert b >= 4096 * 16 * 1024 * 2

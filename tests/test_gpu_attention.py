@@ -277,3 +277,39 @@ def test_one_split_rows_with_nothing_to_attend(orc):
     sink[7], sink[9] = float("inf"), float("-inf")
     pos = [t % 128 if t % 3 else 128 * (1 + t % 7) + 5 for t in range(B)]
     check(orc, w, q, pos, kv_c, kv_tok, sink, what="one split, empty KV sets")
+
+
+def test_sparse_csa_1m_shape(orc):
+    """C4 at full size: 4 sequences x 262144 compressed entries (indices up to
+    2^18 - 1), 1024 selected per sequence, the 128-token window at position
+    2^20 - 1.  Only the window tail of the 1M-token stream is materialised for
+    the oracle; the kernel reads the full-size device stream."""
+    w = configs.CSA_1M
+    g = torch.Generator(device=DEV).manual_seed(60)
+    kv_c = torch.randn(w.B, w.N_c, w.D, generator=g, device=DEV)
+    kv_c = (kv_c / kv_c.pow(2).mean(-1, keepdim=True).sqrt()).to(torch.bfloat16)
+    tail = torch.randn(w.B, w.W, w.D, generator=g, device=DEV).to(torch.bfloat16)
+    kv_tok = torch.empty(w.B, w.L, w.D, dtype=torch.bfloat16, device=DEV)
+    kv_tok[:, -w.W:] = tail
+    q = synth.normal_bf16((w.B, w.H, w.D), 61, "q", DEV)
+    sink = synth.normal_f32((w.H,), 62, "sink", 1.0, DEV)
+    sel, cnt = random_selection(w.B, w.k, [w.N_c] * w.B, 63)
+    assert int(sel.max()) >= 1 << 17
+    out, lse = run_attention(w, q, [w.L - 1] * w.B, kv_c, kv_tok, sink, sel, cnt)
+    del kv_tok
+    ref, rlse = oracle_attention(orc, w, q, [w.L - 1] * w.B, kv_c, tail, sink, sel, cnt,
+                                 tok_base=w.L - w.W)
+    assert_attention_close(out_values(out), ref, "CSA 1M")
+    assert_lse_close(f32(lse), rlse, ref, "CSA 1M")
+
+
+@pytest.mark.parametrize("cnt", [2048, 1500])
+def test_sparse_top_2048(orc, cnt):
+    """k = 2048 selected entries (the largest supported), full and partial."""
+    w = configs.scaled(configs.CSA_128K, B=2, k=2048)
+    B, N_cap, L_cap = 2, 4096, 4 * 4096
+    kv_c, kv_tok = random_cache(w, B, N_cap, L_cap, 70 + cnt)
+    q = synth.normal_bf16((B, w.H, w.D), 71, "q", DEV)
+    sink = synth.normal_f32((w.H,), 72, "sink", 1.0, DEV)
+    sel, c = random_selection(B, w.k, [N_cap] * B, 73, cnt=[cnt, cnt - 77])
+    check(orc, w, q, [L_cap - 1] * B, kv_c, kv_tok, sink, sel, c, what=f"k=2048 cnt={cnt}")

@@ -242,3 +242,39 @@ def test_indexer_topk_csa_1m_shape_sampled(orc):
     ridx, rcnt = orc.topk(got, np.full((w.B, 1), w.N_c), w.k)
     assert np.array_equal(tidx.cpu().numpy(), ridx)
     assert (tcnt.cpu().numpy() == w.k).all()
+
+
+@pytest.mark.parametrize("overlap,L_ctx", [(4, 4096), (4, 4094), (2, 37), (4, 3)])
+def test_csa_compress_overlapping(orc, overlap, L_ctx):
+    """Overlapping compression: entry i pools tokens i*m - overlap .. (i+1)*m - 1
+    (b_pos has m + overlap values), both streams, ragged context ends."""
+    w = configs.scaled(configs.TINY_CSA, overlap=overlap)
+    r = run_compress(w, L_ctx)
+    n = math.ceil(L_ctx / w.m)
+    _, written, vals = orc.compress_kv(bits16(r["kv_tok"]), [L_ctx], f32(r["w_s"]), f32(r["b_pos"]),
+                                       None, w.m, 0, r["N_cap"], r["N_cap"], rope_dim=w.rope_dim,
+                                       overlap=overlap)
+    assert written[0, :n].all()
+    assert_bf16_storage_close(bits16(r["kv_c"])[:, :n], vals[:, :n], f"kv_c overlap={overlap}")
+    _, _, ivals, _ = orc.compress_index(bits16(r["idx_tok"]), [L_ctx], f32(r["w_si"]), f32(r["b_pi"]),
+                                        w.m, 0, r["N_cap"], r["N_cap"], overlap=overlap)
+    check_keys(orc, bits8(r["idx_key"])[:, :n], f32(r["idx_scale"])[:, :n], ivals[:, :n],
+               f"idx_key overlap={overlap}")
+    # The overlap changes the entries (so the check above can fail).
+    _, _, plain = orc.compress_kv(bits16(r["kv_tok"]), [L_ctx], f32(r["w_s"]), f32(r["b_pos"])[:w.m],
+                                  None, w.m, 0, r["N_cap"], r["N_cap"], rope_dim=w.rope_dim)
+    if n > 1:
+        assert np.abs(plain[:, 1:n] - vals[:, 1:n]).max() > 1e-2
+
+
+def test_csa_compress_overlapping_d512_partial_range(orc):
+    """d = 512, a block range that starts mid-sequence (the borrowed tokens
+    come from the block before the range)."""
+    w = configs.scaled(configs.CSA_128K, B=2, overlap=4)
+    r = run_compress(w, [1027, 1000], first=100, nblk=157)
+    for b, L in enumerate([1027, 1000]):
+        n = math.ceil(L / w.m)
+        _, _, vals = orc.compress_kv(bits16(r["kv_tok"])[b: b + 1], [L], f32(r["w_s"]), f32(r["b_pos"]),
+                                     None, w.m, 100, n - 100, r["N_cap"], rope_dim=w.rope_dim,
+                                     overlap=4)
+        assert_bf16_storage_close(bits16(r["kv_c"])[b: b + 1, 100:n], vals[:, 100:n], f"seq {b}")

@@ -37,11 +37,13 @@ def _check_lse(lse, rlse, ref):
     assert_lse_close(f32(lse), rlse, ref, "decode-step LSE")
 
 
-def test_csa_decode_loop(orc):
+@pytest.mark.parametrize("overlap", [0, 4])
+def test_csa_decode_loop(orc, overlap):
     """Three sequences at positions 301, 514 and 127, six steps each: blocks
     complete mid-loop (at 303, 515/519, 127/131), and the third sequence
-    starts with fewer visible entries (32) than k (64)."""
-    w = configs.scaled(configs.CSA_128K, B=3, k=64, L=2048)
+    starts with fewer visible entries (32) than k (64).  overlap = 4: the
+    newest entry also pools the previous block's tokens."""
+    w = configs.scaled(configs.CSA_128K, B=3, k=64, L=2048, overlap=overlap)
     B, m, L_cap = w.B, w.m, 2048
     N_cap = L_cap // m
     start = np.array([301, 514, 127])
@@ -50,8 +52,9 @@ def test_csa_decode_loop(orc):
     w_s, b_pos = synth.pool_params(w, DEV)
     w_si, b_pi = synth.pool_params(w, DEV, indexer=True)
     kv_c0, _, _ = orc.compress_kv(kv_bits, start, f32(w_s), f32(b_pos), None, m, 0, N_cap, N_cap,
-                                  rope_dim=w.rope_dim)
-    key0, ks0, _, _ = orc.compress_index(idx_bits, start, f32(w_si), f32(b_pi), m, 0, N_cap, N_cap)
+                                  rope_dim=w.rope_dim, overlap=w.overlap)
+    key0, ks0, _, _ = orc.compress_index(idx_bits, start, f32(w_si), f32(b_pi), m, 0, N_cap, N_cap,
+                                         overlap=w.overlap)
     kv_c = _to_bf16(kv_c0)
     idx_key = torch.from_numpy(key0).to(DEV)
     idx_scale = torch.from_numpy(ks0).to(DEV)
@@ -79,10 +82,10 @@ def test_csa_decode_loop(orc):
         for b in range(B):
             i = pos[b] // m
             _, _, vals = orc.compress_kv(kv_bits[b: b + 1], [pos[b] + 1], f32(w_s), f32(b_pos),
-                                         None, m, i, 1, N_cap, rope_dim=w.rope_dim)
+                                         None, m, i, 1, N_cap, rope_dim=w.rope_dim, overlap=w.overlap)
             assert_bf16_storage_close(got_c[b: b + 1, i], vals[:, i], f"step {step} seq {b} entry")
             _, _, kvals, _ = orc.compress_index(idx_bits[b: b + 1], [pos[b] + 1], f32(w_si),
-                                                f32(b_pi), m, i, 1, N_cap)
+                                                f32(b_pi), m, i, 1, N_cap, overlap=w.overlap)
             check_keys(orc, got_k[b: b + 1, i], got_s[b: b + 1, i], kvals[:, i],
                        f"step {step} seq {b} key")
         # 2. Scores of the visible entries against the oracle on the GPU's keys.
@@ -110,7 +113,7 @@ def test_csa_decode_loop(orc):
     # position, the partial newest one included.
     last = start + 5
     _, _, vals = orc.compress_kv(kv_bits, last + 1, f32(w_s), f32(b_pos), None, m, 0, N_cap, N_cap,
-                                 rope_dim=w.rope_dim)
+                                 rope_dim=w.rope_dim, overlap=w.overlap)
     got_c = bits16(kv_c)
     for b in range(B):
         n = last[b] // m + 1

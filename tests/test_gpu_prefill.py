@@ -48,8 +48,9 @@ def run_prefill(orc, w, P, T):
     kv_bits, idx_bits = bits16(kv_tok), bits16(idx_tok)
     # Cached blocks 0 .. b0-1 from the oracle.
     kv_c0, _, _ = orc.compress_kv(kv_bits, [P], f32(w_s), f32(b_pos), None, m, 0, b0, N_cap,
-                                  rope_dim=w.rope_dim)
-    key0, ks0, _, _ = orc.compress_index(idx_bits, [P], f32(w_si), f32(b_pi), m, 0, b0, N_cap)
+                                  rope_dim=w.rope_dim, overlap=w.overlap)
+    key0, ks0, _, _ = orc.compress_index(idx_bits, [P], f32(w_si), f32(b_pi), m, 0, b0, N_cap,
+                                         overlap=w.overlap)
     kv_c = torch.from_numpy(kv_c0.view(np.int16)).view(torch.bfloat16).to(DEV)
     idx_key = torch.from_numpy(key0).to(DEV)
     idx_scale = torch.from_numpy(ks0).to(DEV)
@@ -81,10 +82,11 @@ def check_prefill(orc, w, r, rows):
     assert np.array_equal(r["kv_c"][:, :b0], r["kv_c0"][:, :b0])
     assert np.array_equal(r["idx_key"][:, :b0], r["key0"][:, :b0])
     _, _, vals = orc.compress_kv(r["kv_bits"], [P + T], f32(r["w_s"]), f32(r["b_pos"]), None, m,
-                                 b0, N_cap - b0, N_cap, rope_dim=w.rope_dim)
+                                 b0, N_cap - b0, N_cap, rope_dim=w.rope_dim, overlap=w.overlap)
     assert_bf16_storage_close(r["kv_c"][:, b0:], vals[:, b0:], "new KV entries")
     _, ks_ref, kvals, _ = orc.compress_index(r["idx_bits"], [P + T], f32(r["w_si"]),
-                                             f32(r["b_pi"]), m, b0, N_cap - b0, N_cap)
+                                             f32(r["b_pi"]), m, b0, N_cap - b0, N_cap,
+                                             overlap=w.overlap)
     sc = r["idx_scale"][:, b0:]
     assert np.allclose(sc, ks_ref[:, b0:], rtol=1e-5, atol=0), "key scales"
     deq = orc.e4m3_decode(r["idx_key"][:, b0:]) * sc[..., None].astype(np.float64)
@@ -132,6 +134,15 @@ def test_prefill_small(orc, P, T):
     w = configs.scaled(configs.CSA_PREFILL, L=P + T, P=P, T=T)
     r = run_prefill(orc, w, P, T)
     check_prefill(orc, w, r, _sample_rows(T, w.m, 24, P + T))
+
+
+@pytest.mark.parametrize("P,T", [(4096, 203), (0, 90)])
+def test_prefill_small_overlapping(orc, P, T):
+    """Overlapping compression (window of 2m tokens at stride m) through the
+    prefill chunk: the first new block borrows the last cached tokens."""
+    w = configs.scaled(configs.CSA_PREFILL, L=P + T, P=P, T=T, overlap=4)
+    r = run_prefill(orc, w, P, T)
+    check_prefill(orc, w, r, _sample_rows(T, w.m, 16, P + T + 1))
 
 
 @pytest.mark.slow

@@ -111,3 +111,22 @@ def test_topk_select_repeated_calls_same_result():
     b = run_topk(s, [131072] * 4, 1024)[0]
     assert np.array_equal(a, b)
     assert (np.diff(a, axis=-1) > 0).all()
+
+
+@pytest.mark.parametrize("N", [4096, 32768, 262144])
+def test_topk_select_k2048(orc, N):
+    """The largest supported k, on the one-CTA-per-row and cluster paths."""
+    rng = np.random.default_rng(N + 2048)
+    k = 2048
+    ns = sorted({min(N, k - 1), min(N, k), min(N, k + 1), N, (N * 2) // 3})
+    for kind in ("normal", "dups", "relu"):
+        check(orc, make_scores(kind, len(ns), N, rng), ns, k)
+
+
+def test_topk_select_row_path_boundary(orc):
+    """Capacities either side of the largest row the one-CTA kernel holds in
+    shared memory, and a ragged capacity (scalar loads)."""
+    rng = np.random.default_rng(77)
+    for N in (46000, 47000, 48000, 33333):
+        ns = [N, N - 1, 5000, 1025]
+        check(orc, make_scores("normal", len(ns), N, rng), ns, 1024)
