@@ -40,7 +40,8 @@ class csa_params(C.Structure):
     _fields_ = [("B", C.c_int), ("d", C.c_int), ("H", C.c_int), ("H_I", C.c_int),
                 ("D_I", C.c_int), ("k", C.c_int), ("window", C.c_int), ("rope_dim", C.c_int),
                 ("m", C.c_int), ("eps", C.c_float), ("softmax_scale", C.c_float),
-                ("rope_inv_freq", C.POINTER(C.c_double)), ("overlap", C.c_int)]
+                ("rope_inv_freq", C.POINTER(C.c_double)), ("overlap", C.c_int),
+                ("entry_offset", C.c_int64)]
 
 
 _lib = None
@@ -100,8 +101,9 @@ def _declare(L):
 
 
 def make_params(B, d, H=0, H_I=0, D_I=0, k=0, window=0, rope_dim=0, m=4, eps=1e-6,
-                softmax_scale=0.0, rope_inv_freq=None, overlap=0):
-    p = csa_params(B, d, H, H_I, D_I, k, window, rope_dim, m, eps, softmax_scale, None, overlap)
+                softmax_scale=0.0, rope_inv_freq=None, overlap=0, entry_offset=0):
+    p = csa_params(B, d, H, H_I, D_I, k, window, rope_dim, m, eps, softmax_scale, None, overlap,
+                   entry_offset)
     if rope_inv_freq is not None:
         arr = (C.c_double * len(rope_inv_freq))(*rope_inv_freq)
         p.rope_inv_freq = C.cast(arr, C.POINTER(C.c_double))

@@ -55,6 +55,8 @@ csa_status check_common(const char* fn, const csa_params* p) {
     return fail(CSA_ERR_UNSUPPORTED_SHAPE, "%s: d=%d (supported: 128, 512)", fn, p->d);
   if (p->m < 1 || p->m > 128)
     return fail(CSA_ERR_UNSUPPORTED_SHAPE, "%s: m=%d (supported: 1..128)", fn, p->m);
+  if (p->entry_offset < 0 || p->entry_offset > ((int64_t)1 << 40))
+    return fail(CSA_ERR_INVALID_ARG, "%s: entry_offset=%lld", fn, (long long)p->entry_offset);
   if (p->overlap < 0 || p->overlap > p->m || p->m + p->overlap > 128)
     return fail(CSA_ERR_UNSUPPORTED_SHAPE, "%s: overlap=%d (supported: 0..m, m + overlap <= 128)",
                 fn, p->overlap);
@@ -250,6 +252,7 @@ static csa_status compress_common(const char* fn, const csa_params* p, const voi
   c.D_I = p->D_I;
   c.m = p->m;
   c.overlap = p->overlap;
+  c.entry_offset = p->entry_offset;
   c.L_cap = L_cap;
   c.N_cap = N_cap;
   c.kv_tok = kv_tok;
@@ -327,6 +330,7 @@ static csa_status index_common(const char* fn, const csa_params* p, int Q,
   a.scores = scores;
   a.status = dev_status;
   a.num_sms = csa::device_sm_count();
+  a.entry_offset = p->entry_offset;
   cudaError_t e = csa::launch_index_scores(a, stream);
   if (e != cudaSuccess) return cuda_fail(fn, e);
   return CSA_OK;
@@ -349,6 +353,7 @@ static csa_status topk_common(const char* fn, const csa_params* p, int Q, const 
   t.idx = topk_idx;
   t.cnt = topk_cnt;
   t.status = dev_status;
+  t.entry_offset = p->entry_offset;
   cudaError_t e = csa::launch_topk(t, stream);
   if (e != cudaSuccess) return cuda_fail(fn, e);
   return CSA_OK;
@@ -493,6 +498,7 @@ static csa_status mqa_common(const char* fn, const csa_params* p, csa_op op, int
                                        round_up((size_t)rows * splits * p->H * p->d * 2, 256));
   a.status = dev_status;
   a.chained = chained;
+  a.entry_offset = p->entry_offset;
   cudaError_t e = csa::launch_mqa(a, stream);
   if (e != cudaSuccess) return cuda_fail(fn, e);
   return CSA_OK;

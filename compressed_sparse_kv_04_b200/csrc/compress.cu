@@ -54,6 +54,9 @@ struct PoolArgs {
   const int64_t* ctx_len;  // [B] device, or null -> ctx_len_value
   int64_t ctx_len_value;
   int64_t first_block, n_blocks;
+  // The cache holds entries entry_offset .. of the sequence: local entry i is
+  // block entry_offset + i (its tokens and its rotation position).
+  int64_t entry_offset;
   // [B] device, or null.  Set: one block per sequence, the one holding
   // position pos_newest[b], pooled over tokens up to pos_newest[b].
   const int64_t* pos_newest;
@@ -280,8 +283,8 @@ CSA_DEV void pool_stream(const PoolArgs& a, const StreamArgs& sa, float* smem) {
     if (a.pos_newest) {
       const int64_t t = a.pos_newest[b];
       L = t + 1;
-      i = t < 0 ? 0 : t / a.m;
-      if (t < 0 || i >= a.N_cap) {  // no block, or one outside the cache
+      i = t < 0 ? 0 : t / a.m - a.entry_offset;
+      if (t < 0 || i < 0 || i >= a.N_cap) {  // no block, or one outside the cache
         active = false;
         L = 0;
         i = 0;
@@ -298,10 +301,12 @@ CSA_DEV void pool_stream(const PoolArgs& a, const StreamArgs& sa, float* smem) {
     // Window positions [jlo, present) are present: none before token 0, none
     // at or past the context end, and nothing at all while the block's own
     // range is empty.
-    const int64_t rem = L - (i * a.m - a.overlap);
-    present = L - i * a.m <= 0 ? 0 : (rem < span ? (int)rem : span);
+    const int64_t gi = a.entry_offset + i;  // block index in the sequence
+    const int64_t rem = L - (gi * a.m - a.overlap);
+    present = L - gi * a.m <= 0 ? 0 : (rem < span ? (int)rem : span);
   }
-  const int jlo = active && i * a.m < a.overlap ? (int)(a.overlap - i * a.m) : 0;
+  const int64_t gblk = a.entry_offset + i;
+  const int jlo = active && gblk * a.m < a.overlap ? (int)(a.overlap - gblk * a.m) : 0;
   float ws[E];
 #pragma unroll
   for (int part = 0; part < LN::NPART; ++part)
@@ -309,12 +314,12 @@ CSA_DEV void pool_stream(const PoolArgs& a, const StreamArgs& sa, float* smem) {
     for (int v = 0; v < LN::VEC; ++v) ws[part * LN::VEC + v] = __ldg(sa.w_s + LN::elem(lane, part, v));
 
   // Row j of the window is blk + j*DIM (only rows j >= jlo are touched).
-  const __nv_bfloat16* blk = sa.tok + ((int64_t)b * a.L_cap + i * a.m - a.overlap) * DIM;
+  const __nv_bfloat16* blk = sa.tok + ((int64_t)b * a.L_cap + gblk * a.m - a.overlap) * DIM;
   float mx, l, acc[E];
   const int g = warp % G;
   const int per_warp = (span + G - 1) / G;
   // Rows in the buffer (fetched at once) and rows present (pooled).
-  const int64_t in_buf = active ? a.L_cap - (i * a.m - a.overlap) : 0;
+  const int64_t in_buf = active ? a.L_cap - (gblk * a.m - a.overlap) : 0;
   const int avail = in_buf <= 0 ? 0 : (in_buf < span ? (int)in_buf : span);
   const int j0 = max(g * per_warp, jlo);
   const int j_load = max(j0, min(avail, g * per_warp + per_warp));
@@ -325,7 +330,7 @@ CSA_DEV void pool_stream(const PoolArgs& a, const StreamArgs& sa, float* smem) {
     if (!active || present == 0) return;
 #pragma unroll
     for (int e = 0; e < E; ++e) acc[e] = acc[e] / l;
-    finish_row<DIM>(sa, a, b * a.N_cap + i, (i + 1) * a.m - 1, lane, acc, a.eps);
+    finish_row<DIM>(sa, a, b * a.N_cap + i, (gblk + 1) * a.m - 1, lane, acc, a.eps);
     return;
   }
   // Merge the G warp partials of the one block of this CTA.
@@ -361,7 +366,7 @@ CSA_DEV void pool_stream(const PoolArgs& a, const StreamArgs& sa, float* smem) {
   }
 #pragma unroll
   for (int e = 0; e < E; ++e) p[e] = p[e] / L;
-  finish_row<DIM>(sa, a, b * a.N_cap + i, (i + 1) * a.m - 1, lane, p, a.eps);
+  finish_row<DIM>(sa, a, b * a.N_cap + i, (gblk + 1) * a.m - 1, lane, p, a.eps);
 }
 
 __global__ void __launch_bounds__(kThreads) compress_kernel(const PoolArgs a) {
@@ -398,6 +403,7 @@ cudaError_t launch_compress(const CompressLaunch& c, cudaStream_t stream) {
   a.ctx_len = c.ctx_len;
   a.ctx_len_value = c.ctx_len_value;
   a.first_block = c.first_block;
+  a.entry_offset = c.entry_offset;
   a.n_blocks = c.pos_newest ? 1 : c.n_blocks;
   a.pos_newest = c.pos_newest;
   a.eps = c.eps;

@@ -43,6 +43,7 @@ struct Cfg {
 struct Params {
   int B, Q, H_I, HP, G, N, m;
   int64_t N_cap;
+  int64_t entry_offset;  // the cache holds entries entry_offset .. of the sequence
   int tiles_per_chunk, ntiles, qgroups;
   const uint8_t* q_idx;
   const float* q_scale;
@@ -95,7 +96,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   int64_t nv_max = 0;
   for (int g = 0; g < nq; ++g) {
     int64_t pos = p.pos_q ? p.pos_q[(int64_t)b * p.Q + q0 + g] : p.pos_base + q0 + g;
-    int64_t nv = pos < 0 ? 0 : (pos + 1) / p.m;
+    int64_t nv = pos < 0 ? 0 : (pos + 1) / p.m - p.entry_offset;
+    if (nv < 0) nv = 0;
     if (nv > p.N_cap) nv = p.N_cap;
     nv_max = max(nv_max, nv);
   }
@@ -216,7 +218,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int g = 0; g < 8; ++g) nv[g] = 0;
     for (int g = 0; g < nq && g < 8; ++g) {
       int64_t pos = p.pos_q ? p.pos_q[(int64_t)b * p.Q + q0 + g] : p.pos_base + q0 + g;
-      int64_t v = pos < 0 ? 0 : (pos + 1) / p.m;
+      int64_t v = pos < 0 ? 0 : (pos + 1) / p.m - p.entry_offset;
+      if (v < 0) v = 0;
       if (v > p.N_cap) {
         v = p.N_cap;
         if (row == 0 && t_begin == 0) report(p.status, CSA_ERR_CAPACITY);
@@ -290,6 +293,7 @@ cudaError_t launch_impl(const IndexLaunch& a, cudaStream_t stream) {
   p.N = p.G * p.HP;
   p.m = a.m;
   p.N_cap = a.N_cap;
+  p.entry_offset = a.entry_offset;
   p.ntiles = (int)((a.N_cap + kTileRows - 1) / kTileRows);
   p.qgroups = (a.Q + p.G - 1) / p.G;
   p.q_idx = a.q_idx;

@@ -13,6 +13,7 @@ namespace csa {
 struct CompressLaunch {
   int B, d, D_I, m;
   int overlap;              // tokens of block i-1 that entry i also pools (b_pos has m + overlap)
+  int64_t entry_offset;     // local entry i is block entry_offset + i of the sequence
   int64_t L_cap, N_cap;
   const void* kv_tok;
   const void* idx_tok;  // null: KV stream only
@@ -47,6 +48,7 @@ struct IndexLaunch {
   float* scores;            // [B, Q, N_cap]
   int32_t* status;
   int num_sms;
+  int64_t entry_offset;     // the cache holds entries entry_offset .. N_cap-1+entry_offset
   int chained;              // see launch_pdl
 };
 cudaError_t launch_index_scores(const IndexLaunch& a, cudaStream_t stream);
@@ -63,6 +65,7 @@ struct TopkLaunch {
   int32_t* idx;             // [rows, k]
   int32_t* cnt;             // [rows]
   int32_t* status;
+  int64_t entry_offset;     // score j is entry entry_offset + j of the sequence
   int chained;              // see launch_pdl
 };
 cudaError_t launch_topk(const TopkLaunch& a, cudaStream_t stream);
@@ -94,6 +97,7 @@ struct MqaLaunch {
   float* part_ml;           // workspace [rows, S, 2, H] fp32
   int splits;               // S
   int32_t* status;
+  int64_t entry_offset;     // the cache holds entries entry_offset .. of the sequence
   int chained;              // see launch_pdl (the merge kernel is always chained)
 };
 size_t mqa_workspace_bytes(int rows, int splits, int H, int D);

@@ -99,6 +99,7 @@ struct Meta {
 struct Params {
   int Q, H, m, W, R, splits;
   int64_t N_cap, L_cap;
+  int64_t entry_offset;  // the cache holds entries entry_offset .. of the sequence
   const __nv_bfloat16* q;
   const int64_t* pos_q;
   int64_t pos_base;
@@ -317,7 +318,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   // The KV list of this query row: n_c compressed entries, then the window.
   const int64_t pos = row_pos(p, row);
-  int64_t n_vis = pos < 0 ? 0 : (pos + 1) / p.m;
+  int64_t n_vis = pos < 0 ? 0 : (pos + 1) / p.m - p.entry_offset;
+  if (n_vis < 0) n_vis = 0;
   if (n_vis > p.N_cap) n_vis = p.N_cap;
   const int64_t w0 = pos - p.W + 1 < 0 ? 0 : pos - p.W + 1;
   const int nwin = (p.W > 0 && pos >= 0) ? (int)(pos - w0 + 1) : 0;
@@ -1046,6 +1048,7 @@ cudaError_t launch_impl(const MqaLaunch& a, cudaStream_t stream) {
   p.R = a.rope_dim;
   p.splits = a.splits;
   p.N_cap = a.N_cap;
+  p.entry_offset = a.entry_offset;
   p.L_cap = a.L_cap;
   p.q = reinterpret_cast<const __nv_bfloat16*>(a.q);
   p.pos_q = a.pos_q;

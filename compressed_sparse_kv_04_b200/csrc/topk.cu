@@ -42,6 +42,7 @@ constexpr int kMaxC = 16;      // CTAs per cluster (16 needs the non-portable si
 struct Params {
   int Q, m, k, C;
   int64_t N_cap, slice;
+  int64_t entry_offset;  // the scores are of entries entry_offset .. of the sequence
   const float* scores;
   const int64_t* pos_q;
   int64_t pos_base;
@@ -113,7 +114,8 @@ __global__ void __launch_bounds__(kThreads, 1) topk_kernel(const Params p) {
   const float* src = p.scores + (int64_t)row * p.N_cap + lo;
 #pragma unroll 8
   for (int i = tid; i < cap; i += kThreads) keys[i] = orderable(__ldg(src + i));
-  int64_t n = pos < 0 ? 0 : (pos + 1) / p.m;
+  int64_t n = pos < 0 ? 0 : (pos + 1) / p.m - p.entry_offset;
+  if (n < 0) n = 0;
   if (n > p.N_cap) {
     n = p.N_cap;
     if (r == 0 && tid == 0) report(p.status, CSA_ERR_CAPACITY);
@@ -365,7 +367,8 @@ __global__ void __launch_bounds__(kThreads, 1) topk_row_kernel(const Params p) {
   const int64_t pos = p.pos_q ? p.pos_q[row] : p.pos_base + row % p.Q;
   pdl_trigger();
   pdl_wait();  // the scores come from the indexer kernel
-  int64_t n64 = pos < 0 ? 0 : (pos + 1) / p.m;
+  int64_t n64 = pos < 0 ? 0 : (pos + 1) / p.m - p.entry_offset;
+  if (n64 < 0) n64 = 0;
   if (n64 > p.N_cap) {
     n64 = p.N_cap;
     if (tid == 0) report(p.status, CSA_ERR_CAPACITY);
@@ -574,6 +577,7 @@ cudaError_t launch_topk(const TopkLaunch& a, cudaStream_t stream) {
     p.k = a.k;
     p.C = 1;
     p.N_cap = a.N_cap;
+    p.entry_offset = a.entry_offset;
     p.slice = a.N_cap;
     p.scores = a.scores;
     p.pos_q = a.pos_q;
@@ -611,6 +615,7 @@ cudaError_t launch_topk(const TopkLaunch& a, cudaStream_t stream) {
   p.k = a.k;
   p.C = C;
   p.N_cap = a.N_cap;
+  p.entry_offset = a.entry_offset;
   p.slice = (a.N_cap + C - 1) / C;
   p.scores = a.scores;
   p.pos_q = a.pos_q;

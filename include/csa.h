@@ -87,6 +87,16 @@ typedef struct {
   int overlap;         /* compression: tokens of block i-1 that entry i also
                           pools (0 = non-overlapping blocks; 0..m, see
                           csa_compress); b_pos then holds m + overlap values */
+  int64_t entry_offset; /* the compressed cache (kv_c, idx_key, idx_scale and
+                          the indexer scores) holds entries entry_offset ..
+                          entry_offset + N_cap - 1 of the sequence: a shard of
+                          a context split over several devices (0 = the whole
+                          cache).  Local entry i is block entry_offset + i: its
+                          tokens and its rotation position (entry_offset + i +
+                          1)*m - 1 are the sequence's, visible counts are
+                          floor((pos+1)/m) - entry_offset clamped to 0..N_cap,
+                          and block ranges and indices are local.  Token rows
+                          (kv_tok, idx_tok) and positions stay global. */
 } csa_params;
 
 /* Operation selector for csa_workspace_bytes(). */
