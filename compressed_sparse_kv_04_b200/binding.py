@@ -27,7 +27,8 @@ EXPORTS = ["csa_version", "csa_last_error", "csa_workspace_bytes", "hca_compress
            "sparse_mqa_decode", "dense_mqa_decode", "csa_prefill_chunk",
            "lightning_index_topk_static", "csa_rope_yarn", "hca_prefill_chunk",
            "csa_decode_step", "hca_decode_step", "grouped_out_proj",
-           "grouped_out_proj_workspace_bytes"]
+           "grouped_out_proj_workspace_bytes", "csa_shard_candidates", "csa_merge_candidates",
+           "sparse_mqa_partials", "mqa_merge_partials"]
 
 
 class CsaError(RuntimeError):
@@ -95,6 +96,11 @@ def _declare(L):
                                    vp]
     L.grouped_out_proj_workspace_bytes.argtypes = [i32, i32, i32, i32, i32, i32]
     L.grouped_out_proj_workspace_bytes.restype = sz
+    L.csa_shard_candidates.argtypes = [P, i32, vp, i64, vp, vp, vp, vp, vp, vp]
+    L.csa_merge_candidates.argtypes = [P, i32, i32, vp, vp, vp, i64, vp, vp, vp, vp, vp, vp]
+    L.sparse_mqa_partials.argtypes = [P, i32, vp, vp, vp, i64, vp, vp, vp, i64, vp, vp, vp, vp,
+                                      vp, vp]
+    L.mqa_merge_partials.argtypes = [P, i32, vp, vp, vp, vp, vp, vp, vp, vp]
     for name in EXPORTS[3:]:
         if name != "grouped_out_proj_workspace_bytes":
             getattr(L, name).restype = i32
@@ -306,3 +312,35 @@ def grouped_out_proj(o, w_g, w_o, z, y=None, ws=None, dev_status=None, stream=No
     _check(lib().grouped_out_proj(T, H, D, g, d_g, d_model, _ptr(o), _ptr(w_g), _ptr(w_o),
                                   _ptr(y), _ptr(z), _ptr(ws), ws.numel() * ws.element_size(),
                                   _ptr(dev_status), _stream(stream)))
+
+
+# ------------------------------------------- context split over several devices --
+def csa_shard_candidates(p, Q, scores, topk_idx, topk_cnt, cand_score, cand_idx,
+                         dev_status=None, stream=None):
+    _check(lib().csa_shard_candidates(C.byref(p), Q, _ptr(scores), scores.shape[-1],
+                                      _ptr(topk_idx), _ptr(topk_cnt), _ptr(cand_score),
+                                      _ptr(cand_idx), _ptr(dev_status), _stream(stream)))
+
+
+def csa_merge_candidates(p, Q, G, cand_score, cand_idx, cand_cnt, N_cap, topk_idx, topk_cnt,
+                         local_idx, local_cnt, dev_status=None, stream=None):
+    _check(lib().csa_merge_candidates(C.byref(p), Q, G, _ptr(cand_score), _ptr(cand_idx),
+                                      _ptr(cand_cnt), N_cap, _ptr(topk_idx), _ptr(topk_cnt),
+                                      _ptr(local_idx), _ptr(local_cnt), _ptr(dev_status),
+                                      _stream(stream)))
+
+
+def sparse_mqa_partials(p, splits, q, pos_q, kv_c, topk_idx, topk_cnt, kv_tok, part_o, part_ml,
+                        gamma_q=None, gamma_kv=None, dev_status=None, stream=None):
+    _check(lib().sparse_mqa_partials(C.byref(p), splits, _ptr(q), _ptr(pos_q), _ptr(kv_c),
+                                     kv_c.shape[1], _ptr(topk_idx), _ptr(topk_cnt), _ptr(kv_tok),
+                                     kv_tok.shape[1], _ptr(gamma_q), _ptr(gamma_kv),
+                                     _ptr(part_o), _ptr(part_ml), _ptr(dev_status),
+                                     _stream(stream)))
+
+
+def mqa_merge_partials(p, splits, part_o, part_ml, pos_q, sink, out, lse=None, dev_status=None,
+                       stream=None):
+    _check(lib().mqa_merge_partials(C.byref(p), splits, _ptr(part_o), _ptr(part_ml), _ptr(pos_q),
+                                    _ptr(sink), _ptr(out), _ptr(lse), _ptr(dev_status),
+                                    _stream(stream)))

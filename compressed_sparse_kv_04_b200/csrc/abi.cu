@@ -850,4 +850,165 @@ csa_status grouped_out_proj(int T, int H, int D, int g, int d_g, int d_model, co
   return CSA_OK;
 }
 
+// ----------------------------------------- context split over several devices --
+csa_status csa_shard_candidates(const csa_params* p, int Q, const float* scores, int64_t N_cap,
+                                const int32_t* topk_idx, const int32_t* topk_cnt,
+                                float* cand_score, int32_t* cand_idx, int32_t* dev_status,
+                                void* stream) {
+  const char* fn = "csa_shard_candidates";
+  csa_status st = check_index_args(fn, p, Q, N_cap);
+  if (st != CSA_OK) return st;
+  REQ_PTR(scores);
+  REQ_PTR(topk_idx);
+  REQ_PTR4(topk_cnt);
+  REQ_PTR4(cand_score);
+  REQ_PTR4(cand_idx);
+  OPT_PTR4(dev_status);
+  if (p->entry_offset + N_cap > 0x7FFFFFFF)
+    return fail(CSA_ERR_UNSUPPORTED_SHAPE, "%s: sequence indices must fit in int32", fn);
+  cudaError_t e = csa::launch_shard_candidates(scores, N_cap, topk_idx, topk_cnt, p->B * Q, p->k,
+                                               p->entry_offset, cand_score, cand_idx,
+                                               static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(fn, e);
+  return CSA_OK;
+}
+
+csa_status csa_merge_candidates(const csa_params* p, int Q, int G, const float* cand_score,
+                                const int32_t* cand_idx, const int32_t* cand_cnt, int64_t N_cap,
+                                int32_t* topk_idx, int32_t* topk_cnt, int32_t* local_idx,
+                                int32_t* local_cnt, int32_t* dev_status, void* stream) {
+  const char* fn = "csa_merge_candidates";
+  csa_status st = check_index_args(fn, p, Q, N_cap);
+  if (st != CSA_OK) return st;
+  if (G < 1 || G > 64 || (size_t)G * p->k * 8 > 190 * 1024)
+    return fail(CSA_ERR_UNSUPPORTED_SHAPE, "%s: G=%d (supported: 1..64 with G*k <= 24320)", fn, G);
+  REQ_PTR4(cand_score);
+  REQ_PTR4(cand_idx);
+  REQ_PTR4(cand_cnt);
+  REQ_PTR(topk_idx);
+  REQ_PTR4(topk_cnt);
+  REQ_PTR(local_idx);
+  REQ_PTR4(local_cnt);
+  OPT_PTR4(dev_status);
+  csa::MergeLaunch a{};
+  a.G = G;
+  a.rows = p->B * Q;
+  a.k = p->k;
+  a.cand_s = cand_score;
+  a.cand_i = cand_idx;
+  a.cand_c = cand_cnt;
+  a.idx = topk_idx;
+  a.cnt = topk_cnt;
+  a.lo = p->entry_offset;
+  a.hi = p->entry_offset + N_cap;
+  a.local_idx = local_idx;
+  a.local_cnt = local_cnt;
+  a.status = dev_status;
+  a.chained = 0;
+  cudaError_t e = csa::launch_merge_candidates(a, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(fn, e);
+  return CSA_OK;
+}
+
+csa_status sparse_mqa_partials(const csa_params* p, int splits, const void* q, const int64_t* pos_q,
+                               const void* kv_c, int64_t N_cap, const int32_t* topk_idx,
+                               const int32_t* topk_cnt, const void* kv_tok, int64_t L_cap,
+                               const float* gamma_q, const float* gamma_kv, void* part_o,
+                               float* part_ml, int32_t* dev_status, void* stream) {
+  const char* fn = "sparse_mqa_partials";
+  csa_status st = check_common(fn, p);
+  if (st != CSA_OK) return st;
+  st = check_attention(fn, p);
+  if (st != CSA_OK) return st;
+  if (p->k < 1 || p->k > kMaxTopk)
+    return fail(CSA_ERR_UNSUPPORTED_SHAPE, "%s: k=%d (supported: 1..%d)", fn, p->k, kMaxTopk);
+  if (splits < 1 || splits > 64)
+    return fail(CSA_ERR_UNSUPPORTED_SHAPE, "%s: splits=%d (supported: 1..64)", fn, splits);
+  REQ_PTR(q);
+  REQ_PTR(pos_q);
+  REQ_PTR(kv_c);
+  REQ_PTR(kv_tok);
+  REQ_PTR(topk_idx);
+  REQ_PTR4(topk_cnt);
+  OPT_PTR4(gamma_q);
+  OPT_PTR4(gamma_kv);
+  REQ_PTR(part_o);
+  REQ_PTR4(part_ml);
+  OPT_PTR4(dev_status);
+  if (N_cap < 1 || L_cap < 1 || (int64_t)p->B * N_cap > ((int64_t)1 << 31) - 1 ||
+      (int64_t)p->B * L_cap > ((int64_t)1 << 31) - 1)
+    return fail(CSA_ERR_INVALID_ARG, "%s: N_cap=%lld L_cap=%lld", fn, (long long)N_cap,
+                (long long)L_cap);
+  csa::MqaLaunch a{};
+  a.B = p->B;
+  a.Q = 1;
+  a.H = p->H;
+  a.D = p->d;
+  a.m = p->m;
+  a.W = p->window;
+  a.rope_dim = p->rope_dim;
+  a.N_cap = N_cap;
+  a.L_cap = L_cap;
+  a.q = q;
+  a.pos_q = pos_q;
+  a.kv_c = kv_c;
+  a.sel_idx = topk_idx;
+  a.sel_cnt = topk_cnt;
+  a.kmax = p->k;
+  a.kv_tok = kv_tok;
+  a.sink = nullptr;
+  a.gamma_q = gamma_q;
+  a.gamma_kv = gamma_kv;
+  a.eps = p->eps;
+  a.scale = softmax_scale_of(p);
+  fill_inv_freq(p, a.inv_freq);
+  a.part_o = part_o;
+  a.part_ml = part_ml;
+  a.splits = splits;
+  a.status = dev_status;
+  a.entry_offset = p->entry_offset;
+  a.emit_partials = 1;
+  cudaError_t e = csa::launch_mqa(a, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(fn, e);
+  return CSA_OK;
+}
+
+csa_status mqa_merge_partials(const csa_params* p, int splits, const void* part_o,
+                              const float* part_ml, const int64_t* pos_q, const float* sink,
+                              void* out, float* lse, int32_t* dev_status, void* stream) {
+  const char* fn = "mqa_merge_partials";
+  csa_status st = check_common(fn, p);
+  if (st != CSA_OK) return st;
+  st = check_attention(fn, p);
+  if (st != CSA_OK) return st;
+  if (splits < 1 || splits > 4096)
+    return fail(CSA_ERR_UNSUPPORTED_SHAPE, "%s: splits=%d (supported: 1..4096)", fn, splits);
+  REQ_PTR(part_o);
+  REQ_PTR4(part_ml);
+  REQ_PTR(pos_q);
+  REQ_PTR4(sink);
+  REQ_PTR(out);
+  OPT_PTR4(lse);
+  OPT_PTR4(dev_status);
+  csa::MqaLaunch a{};
+  a.B = p->B;
+  a.Q = 1;
+  a.H = p->H;
+  a.D = p->d;
+  a.rope_dim = p->rope_dim;
+  a.pos_q = pos_q;
+  a.sink = sink;
+  fill_inv_freq(p, a.inv_freq);
+  a.out = out;
+  a.lse = lse;
+  a.part_o = const_cast<void*>(part_o);
+  a.part_ml = const_cast<float*>(part_ml);
+  a.splits = splits;
+  a.status = dev_status;
+  a.chained = 0;
+  cudaError_t e = csa::launch_mqa_merge(a, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(fn, e);
+  return CSA_OK;
+}
+
 }  // extern "C"

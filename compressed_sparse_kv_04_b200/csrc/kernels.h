@@ -70,6 +70,26 @@ struct TopkLaunch {
 };
 cudaError_t launch_topk(const TopkLaunch& a, cudaStream_t stream);
 
+// Context split over ranks: a shard's candidates (score, sequence index) and
+// the global top-k over all ranks' candidates.
+cudaError_t launch_shard_candidates(const float* scores, int64_t N_cap, const int32_t* idx,
+                                    const int32_t* cnt, int rows, int k, int64_t offset,
+                                    float* cand_s, int32_t* cand_i, cudaStream_t stream);
+struct MergeLaunch {
+  int G, rows, k;
+  const float* cand_s;      // [G, rows, k]
+  const int32_t* cand_i;    // [G, rows, k]
+  const int32_t* cand_c;    // [G, rows]
+  int32_t* idx;             // [rows, k]
+  int32_t* cnt;             // [rows]
+  int64_t lo, hi;           // this rank's entries
+  int32_t* local_idx;       // [rows, k]
+  int32_t* local_cnt;       // [rows]
+  int32_t* status;
+  int chained;
+};
+cudaError_t launch_merge_candidates(const MergeLaunch& a, cudaStream_t stream);
+
 // Shared-KV MQA decode (sparse or dense) with window and sink: one CTA per
 // (query row, split) for H <= 64, two for H > 64 (64 heads each), at the
 // full head dim;
@@ -99,10 +119,13 @@ struct MqaLaunch {
   int32_t* status;
   int64_t entry_offset;     // the cache holds entries entry_offset .. of the sequence
   int chained;              // see launch_pdl (the merge kernel is always chained)
+  int emit_partials;        // write the split partials only (no merge, no output)
 };
 size_t mqa_workspace_bytes(int rows, int splits, int H, int D);
 int mqa_choose_splits(int rows, int64_t compressed_max, int window, int num_sms, int H);
 cudaError_t launch_mqa(const MqaLaunch& a, cudaStream_t stream);
+// The split merge alone (part_o / part_ml with a.splits splits per row).
+cudaError_t launch_mqa_merge(const MqaLaunch& a, cudaStream_t stream);
 
 // One projection GEMM of the grouped output projection: for each group j,
 // C[t, j*N + n] = sum_k A[t, j*K + k] * W[j*N + n, k] (bf16 in, fp32

@@ -1064,7 +1064,7 @@ cudaError_t launch_impl(const MqaLaunch& a, cudaStream_t stream) {
   p.part_o = reinterpret_cast<__half*>(a.part_o);
   p.part_ml = a.part_ml;
   p.status = a.status;
-  p.fused = a.splits == 1 ? 1 : 0;
+  p.fused = (a.splits == 1 && !a.emit_partials) ? 1 : 0;
   p.sink = a.sink;
   p.out = reinterpret_cast<__nv_bfloat16*>(a.out);
   p.lse = a.lse;
@@ -1092,7 +1092,8 @@ cudaError_t launch_impl(const MqaLaunch& a, cudaStream_t stream) {
   e = ensure_smem_attr(reinterpret_cast<const void*>(kern), 3 + variant, smem);
   if (e != cudaSuccess) return e;
   dim3 grid(cps * a.splits, rows, 1);
-  if (!p.fused && cluster_fits(reinterpret_cast<const void*>(kern), variant, a.splits, smem)) {
+  if (!p.fused && !a.emit_partials &&
+      cluster_fits(reinterpret_cast<const void*>(kern), variant, a.splits, smem)) {
     // The splits of each head group form one cluster and merge in-kernel.
     p.cluster_merge = 1;
     return launch_pdl(kern, grid, dim3(kThreads), smem, stream, a.splits, a.chained, map_q, box_c,
@@ -1101,13 +1102,49 @@ cudaError_t launch_impl(const MqaLaunch& a, cudaStream_t stream) {
   e = launch_pdl(kern, grid, dim3(kThreads), smem, stream, 0, a.chained, map_q, box_c, box_t, p);
   if (e != cudaSuccess) return e;
   if (p.fused) return cudaSuccess;  // the attention kernel finished the rows
+  if (a.emit_partials) return cudaSuccess;  // the caller merges the partials
   const unsigned nblk = (unsigned)(((int64_t)rows * a.H + 3) / 4);
   const size_t wsm = (size_t)4 * a.splits * sizeof(float);
   auto merge = mqa_combine_kernel<D, R, 4>;
   return launch_pdl(merge, dim3(nblk), dim3(128), wsm, stream, 0, 1, p, rows);
 }
 
+template <int D, int R>
+cudaError_t launch_merge_impl(const MqaLaunch& a, cudaStream_t stream) {
+  Params p{};
+  p.Q = a.Q;
+  p.H = a.H;
+  p.R = a.rope_dim;
+  p.splits = a.splits;
+  p.pos_q = a.pos_q;
+  p.pos_base = a.pos_base;
+  p.part_o = reinterpret_cast<__half*>(a.part_o);
+  p.part_ml = a.part_ml;
+  p.status = a.status;
+  p.sink = a.sink;
+  p.out = reinterpret_cast<__nv_bfloat16*>(a.out);
+  p.lse = a.lse;
+  for (int j = 0; j < 64; ++j) p.inv_freq[j] = a.inv_freq[j];
+  const int rows = a.B * a.Q;
+  const unsigned nblk = (unsigned)(((int64_t)rows * a.H + 3) / 4);
+  const size_t wsm = (size_t)4 * a.splits * sizeof(float);
+  return launch_pdl(mqa_combine_kernel<D, R, 4>, dim3(nblk), dim3(128), wsm, stream, 0, a.chained,
+                    p, rows);
+}
+
 }  // namespace
+
+cudaError_t launch_mqa_merge(const MqaLaunch& a, cudaStream_t stream) {
+  if (a.D == 512) {
+    if (a.rope_dim == 64) return launch_merge_impl<512, 64>(a, stream);
+    if (a.rope_dim == 32) return launch_merge_impl<512, 32>(a, stream);
+    if (a.rope_dim == 0) return launch_merge_impl<512, 0>(a, stream);
+  } else if (a.D == 128) {
+    if (a.rope_dim == 32) return launch_merge_impl<128, 32>(a, stream);
+    if (a.rope_dim == 0) return launch_merge_impl<128, 0>(a, stream);
+  }
+  return cudaErrorInvalidValue;
+}
 
 cudaError_t launch_mqa(const MqaLaunch& a, cudaStream_t stream) {
   if (a.D == 512) {

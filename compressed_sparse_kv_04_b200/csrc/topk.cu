@@ -356,49 +356,17 @@ CSA_DEV uint32_t block_excl_scan(uint32_t v, uint32_t* warp_tot) {
   return warp_tot[warp] + incl - v;
 }
 
-__global__ void __launch_bounds__(kThreads, 1) topk_row_kernel(const Params p) {
+// Selects the k largest of keys[0..n) (n > k; order-preserving keys in
+// shared memory, written by this CTA) under (key descending, position
+// ascending) and calls emit(o, i) once for each output slot o < k with the
+// selected position i, slots in ascending order of i.  kmin / kmax: this
+// thread's min and max over the keys it wrote.  All 1024 threads call it.
+template <typename Emit>
+CSA_DEV void row_select(const uint32_t* keys, int n, int k, RowShared& sh, uint32_t kmin,
+                        uint32_t kmax, Emit emit) {
   constexpr int kBins = 1 << kRowBits;
   constexpr int kPer = kBins / kThreads;  // bins per thread in the digit scan
-  extern __shared__ __align__(16) uint8_t smem_raw[];
-  RowShared& sh = *reinterpret_cast<RowShared*>(smem_raw);
-  uint32_t* keys = reinterpret_cast<uint32_t*>(smem_raw + sizeof(RowShared));
-  const int row = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int64_t pos = p.pos_q ? p.pos_q[row] : p.pos_base + row % p.Q;
-  pdl_trigger();
-  pdl_wait();  // the scores come from the indexer kernel
-  int64_t n64 = pos < 0 ? 0 : (pos + 1) / p.m - p.entry_offset;
-  if (n64 < 0) n64 = 0;
-  if (n64 > p.N_cap) {
-    n64 = p.N_cap;
-    if (tid == 0) report(p.status, CSA_ERR_CAPACITY);
-  }
-  const int n = (int)n64;
-  int32_t* out = p.idx + (int64_t)row * p.k;
-  if (n <= p.k) {  // every visible entry is kept
-    for (int j = tid; j < p.k; j += kThreads) out[j] = j < n ? j : -1;
-    if (tid == 0) p.cnt[row] = n;
-    return;
-  }
-  // The visible scores as order-preserving keys, with this thread's min/max.
-  const float* src = p.scores + (int64_t)row * p.N_cap;
-  uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
-  const bool vec = ((reinterpret_cast<uintptr_t>(src) & 15u) == 0);
-  const int n4 = vec ? (n & ~3) : 0;
-#pragma unroll 4
-  for (int i = 4 * tid; i < n4; i += 4 * kThreads) {
-    const float4 v = __ldg(reinterpret_cast<const float4*>(src + i));
-    const uint4 u = make_uint4(orderable(v.x), orderable(v.y), orderable(v.z), orderable(v.w));
-    *reinterpret_cast<uint4*>(keys + i) = u;
-    kmin = min(kmin, min(min(u.x, u.y), min(u.z, u.w)));
-    kmax = max(kmax, max(max(u.x, u.y), max(u.z, u.w)));
-  }
-  for (int i = n4 + tid; i < n; i += kThreads) {
-    const uint32_t u = orderable(__ldg(src + i));
-    keys[i] = u;
-    kmin = min(kmin, u);
-    kmax = max(kmax, u);
-  }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
     kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
@@ -419,7 +387,7 @@ __global__ void __launch_bounds__(kThreads, 1) topk_row_kernel(const Params p) {
   cta_sync();  // every warp has read the min / max slots
 
   uint32_t prefix, mask;
-  uint32_t k_rem = (uint32_t)p.k;
+  uint32_t k_rem = (uint32_t)k;
   if (gmin == gmax) {
     prefix = gmin;
     mask = 0xFFFFFFFFu;
@@ -518,15 +486,201 @@ __global__ void __launch_bounds__(kThreads, 1) topk_row_kernel(const Params p) {
     const uint32_t eq_rank = eq_run + __popc(be & lt);
     if (gt || (eq && eq_rank < need_eq)) {
       const uint32_t o = gt_run + __popc(bg & lt) + min(need_eq, eq_rank);
-      if (o < (uint32_t)p.k) out[o] = i;
+      if (o < (uint32_t)k) emit(o, i);
     }
     gt_run += __popc(bg);
     eq_run += __popc(be);
   }
+}
+
+__global__ void __launch_bounds__(kThreads, 1) topk_row_kernel(const Params p) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  RowShared& sh = *reinterpret_cast<RowShared*>(smem_raw);
+  uint32_t* keys = reinterpret_cast<uint32_t*>(smem_raw + sizeof(RowShared));
+  const int row = blockIdx.x;
+  const int tid = threadIdx.x;
+  const int64_t pos = p.pos_q ? p.pos_q[row] : p.pos_base + row % p.Q;
+  pdl_trigger();
+  pdl_wait();  // the scores come from the indexer kernel
+  int64_t n64 = pos < 0 ? 0 : (pos + 1) / p.m - p.entry_offset;
+  if (n64 < 0) n64 = 0;
+  if (n64 > p.N_cap) {
+    n64 = p.N_cap;
+    if (tid == 0) report(p.status, CSA_ERR_CAPACITY);
+  }
+  const int n = (int)n64;
+  int32_t* out = p.idx + (int64_t)row * p.k;
+  if (n <= p.k) {  // every visible entry is kept
+    for (int j = tid; j < p.k; j += kThreads) out[j] = j < n ? j : -1;
+    if (tid == 0) p.cnt[row] = n;
+    return;
+  }
+  // The visible scores as order-preserving keys, with this thread's min/max.
+  const float* src = p.scores + (int64_t)row * p.N_cap;
+  uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
+  const bool vec = ((reinterpret_cast<uintptr_t>(src) & 15u) == 0);
+  const int n4 = vec ? (n & ~3) : 0;
+#pragma unroll 4
+  for (int i = 4 * tid; i < n4; i += 4 * kThreads) {
+    const float4 v = __ldg(reinterpret_cast<const float4*>(src + i));
+    const uint4 u = make_uint4(orderable(v.x), orderable(v.y), orderable(v.z), orderable(v.w));
+    *reinterpret_cast<uint4*>(keys + i) = u;
+    kmin = min(kmin, min(min(u.x, u.y), min(u.z, u.w)));
+    kmax = max(kmax, max(max(u.x, u.y), max(u.z, u.w)));
+  }
+  for (int i = n4 + tid; i < n; i += kThreads) {
+    const uint32_t u = orderable(__ldg(src + i));
+    keys[i] = u;
+    kmin = min(kmin, u);
+    kmax = max(kmax, u);
+  }
+  row_select(keys, n, p.k, sh, kmin, kmax, [&](uint32_t o, int i) { out[o] = i; });
   if (tid == 0) p.cnt[row] = p.k;
 }
 
+// ------------------------------------------------- context split over ranks --
+// Candidates of one shard: the (score, sequence index) of each entry its
+// local top-k kept; slots past the count get (NaN, -1).
+__global__ void __launch_bounds__(256) shard_candidates_kernel(
+    const float* __restrict__ scores, int64_t N_cap, const int32_t* __restrict__ idx,
+    const int32_t* __restrict__ cnt, int rows, int k, int64_t offset, float* __restrict__ cand_s,
+    int32_t* __restrict__ cand_i) {
+  pdl_trigger();
+  pdl_wait();  // the selection comes from the top-k kernel
+  const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (t >= (int64_t)rows * k) return;
+  const int row = (int)(t / k), j = (int)(t % k);
+  const int c = cnt[row];
+  const int32_t i = idx[t];
+  if (j < c && i >= 0 && i < N_cap) {
+    cand_s[t] = scores[(int64_t)row * N_cap + i];
+    cand_i[t] = (int32_t)(i + offset);
+  } else {
+    cand_s[t] = __int_as_float(0x7fffffff);
+    cand_i[t] = -1;
+  }
+}
+
+struct MergeParams {
+  int G, rows, k;
+  const float* cand_s;     // [G, rows, k]
+  const int32_t* cand_i;   // [G, rows, k] sequence indices, ascending per (rank, row)
+  const int32_t* cand_c;   // [G, rows] candidates per rank
+  int32_t* idx;            // [rows, k] sequence indices (written)
+  int32_t* cnt;            // [rows]
+  int64_t lo, hi;          // this rank's entries [lo, hi)
+  int32_t* local_idx;      // [rows, k] local indices of this rank's selected entries
+  int32_t* local_cnt;      // [rows]
+  int32_t* status;
+};
+
+// Global top-k over the candidates of all ranks (one CTA per row).  The
+// ranks' candidate lists are concatenated in rank order; each list holds
+// ascending sequence indices and rank r's indices lie below rank r+1's, so a
+// position in the concatenation orders candidates exactly as their sequence
+// index does, and the tie rule (lower position first) is the method's (lower
+// index first).  The exact top-k of the sequence lies within the union of
+// the ranks' top-k lists.  Also writes this rank's share of the selection,
+// as local indices: a contiguous run of the ascending output.
+__global__ void __launch_bounds__(kThreads, 1) merge_candidates_kernel(const MergeParams p) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  RowShared& sh = *reinterpret_cast<RowShared*>(smem_raw);
+  __shared__ int32_t s_off[65];
+  __shared__ int32_t s_first, s_nloc;
+  const int nmax = p.G * p.k;
+  uint32_t* keys = reinterpret_cast<uint32_t*>(smem_raw + sizeof(RowShared));
+  int32_t* gidx = reinterpret_cast<int32_t*>(keys + nmax);
+  const int row = blockIdx.x, tid = threadIdx.x;
+  pdl_trigger();
+  pdl_wait();
+  if (tid == 0) {
+    int o = 0;
+    for (int r = 0; r < p.G; ++r) {
+      s_off[r] = o;
+      int c = p.cand_c[(int64_t)r * p.rows + row];
+      c = c < 0 ? 0 : (c > p.k ? p.k : c);
+      o += c;
+    }
+    s_off[p.G] = o;
+    s_first = 0x7fffffff;
+    s_nloc = 0;
+  }
+  cta_sync();
+  const int n = s_off[p.G];
+  uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
+  for (int r = 0; r < p.G; ++r) {
+    const int base = s_off[r], c = s_off[r + 1] - base;
+    const int64_t src = ((int64_t)r * p.rows + row) * p.k;
+    for (int j = tid; j < c; j += kThreads) {
+      const uint32_t u = orderable(p.cand_s[src + j]);
+      keys[base + j] = u;
+      gidx[base + j] = p.cand_i[src + j];
+      kmin = min(kmin, u);
+      kmax = max(kmax, u);
+    }
+  }
+  cta_sync();
+  int32_t* out = p.idx + (int64_t)row * p.k;
+  const int total = n < p.k ? n : p.k;
+  if (n <= p.k) {
+    for (int j = tid; j < p.k; j += kThreads) out[j] = j < n ? gidx[j] : -1;
+  } else {
+    row_select(keys, n, p.k, sh, kmin, kmax, [&](uint32_t o, int i) { out[o] = gidx[i]; });
+  }
+  if (tid == 0) p.cnt[row] = total;
+  __threadfence_block();
+  cta_sync();  // the output row is complete (read back below)
+  int32_t* loc = p.local_idx + (int64_t)row * p.k;
+  for (int j = tid; j < total; j += kThreads) {
+    const int64_t g = out[j];
+    if (g >= p.lo && g < p.hi) {
+      atomicMin(&s_first, j);
+      atomicAdd(&s_nloc, 1);
+    }
+  }
+  cta_sync();
+  const int first = s_first, nloc = s_nloc;
+  for (int j = tid; j < p.k; j += kThreads)
+    loc[j] = j < nloc ? (int32_t)(out[first + j] - p.lo) : -1;
+  if (tid == 0) p.local_cnt[row] = nloc;
+}
+
 }  // namespace
+
+cudaError_t launch_shard_candidates(const float* scores, int64_t N_cap, const int32_t* idx,
+                                    const int32_t* cnt, int rows, int k, int64_t offset,
+                                    float* cand_s, int32_t* cand_i, cudaStream_t stream) {
+  const int64_t n = (int64_t)rows * k;
+  if (n <= 0) return cudaSuccess;
+  return launch_pdl(shard_candidates_kernel, dim3((unsigned)((n + 255) / 256)), dim3(256), 0,
+                    stream, 0, 0, scores, N_cap, idx, cnt, rows, k, offset, cand_s, cand_i);
+}
+
+cudaError_t launch_merge_candidates(const MergeLaunch& a, cudaStream_t stream) {
+  if (a.rows < 1) return cudaSuccess;
+  if (a.G < 1 || a.G > 64 || a.k < 1 || a.k > kMaxK || a.rows > 65535)
+    return cudaErrorInvalidConfiguration;
+  MergeParams p{};
+  p.G = a.G;
+  p.rows = a.rows;
+  p.k = a.k;
+  p.cand_s = a.cand_s;
+  p.cand_i = a.cand_i;
+  p.cand_c = a.cand_c;
+  p.idx = a.idx;
+  p.cnt = a.cnt;
+  p.lo = a.lo;
+  p.hi = a.hi;
+  p.local_idx = a.local_idx;
+  p.local_cnt = a.local_cnt;
+  p.status = a.status;
+  const size_t smem = sizeof(RowShared) + (size_t)a.G * a.k * 8;
+  if (smem > 220 * 1024) return cudaErrorInvalidValue;
+  cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(merge_candidates_kernel), 4, smem);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(merge_candidates_kernel, dim3(a.rows), dim3(kThreads), smem, stream, 0,
+                    a.chained, p);
+}
 
 // Largest cluster size (8 or 16) that can be resident for this kernel and
 // shared-memory size on the current device; cached per device.

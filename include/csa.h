@@ -466,6 +466,88 @@ csa_status grouped_out_proj(int T, int H, int D, int g, int d_g, int d_model, co
                             const void* w_g, const void* w_o, void* y, void* z, void* ws,
                             size_t ws_bytes, int32_t* dev_status, void* stream);
 
+/* ---------------------------------------------------------------------------
+ * Context split: one sequence's compressed cache over G devices.
+ *
+ * The pages give no parallel scheme for this path ("Architectural Overview
+ * of V4 Series Models" (intl.cloud.baidu.com) names only 3D-parallel
+ * training as an outlook); this is the build's.  Rank r holds the entries
+ * [lo_r, hi_r) of the compressed KV cache and of the indexer keys, a
+ * contiguous range in rank order, described to every call by
+ * csa_params.entry_offset = lo_r and N_cap = hi_r - lo_r.  One decode step:
+ *   1. every rank scores its entries and keeps its local top-k
+ *      (lightning_index_topk on its shard, scores_out given);
+ *   2. csa_shard_candidates turns that into (score, sequence index) pairs;
+ *   3. the ranks exchange the pairs and counts (an all-gather in rank order,
+ *      e.g. NCCL);
+ *   4. csa_merge_candidates ranks the G*k candidates: the exact top-k of the
+ *      whole sequence (it lies within the union of the local top-k lists;
+ *      same tie rule), and this rank's share of it as local indices;
+ *   5. sparse_mqa_partials attends over this rank's share (the window only on
+ *      the rank holding the newest tokens: csa_params.window = 0 elsewhere)
+ *      and writes split partials instead of an output;
+ *   6. the ranks exchange the partials (all-gather in rank order);
+ *   7. mqa_merge_partials folds all ranks' partials, the sink and the inverse
+ *      rotation into the output, identical on every rank.
+ * Steps 3 and 6 are the only data exchange (B*Q*k*8 bytes of candidates and
+ * B*S*H*(2d+8) bytes of partials per rank).
+ * ------------------------------------------------------------------------- */
+
+/* Candidates of one shard.  For every row (b, q) and slot j < topk_cnt:
+ *   cand_score[b,q,j] = scores[b,q,topk_idx[b,q,j]],
+ *   cand_idx[b,q,j]   = topk_idx[b,q,j] + p->entry_offset  (sequence index);
+ * slots j >= topk_cnt get (NaN, -1).  scores [B,Q,N_cap] fp32, topk_idx
+ * [B,Q,k] / topk_cnt [B,Q] int32 as lightning_index_topk writes them (all
+ * device); cand_score [B,Q,k] fp32, cand_idx [B,Q,k] int32 (written).
+ * Sequence indices must fit in int32 (CSA_ERR_UNSUPPORTED_SHAPE). */
+csa_status csa_shard_candidates(const csa_params* p, int Q, const float* scores, int64_t N_cap,
+                                const int32_t* topk_idx, const int32_t* topk_cnt,
+                                float* cand_score, int32_t* cand_idx, int32_t* dev_status,
+                                void* stream);
+
+/* Global top-k over the candidates of G ranks (concatenated in rank order).
+ *   cand_score [G,B,Q,k] fp32, cand_idx [G,B,Q,k] int32, cand_cnt [G,B,Q]
+ *   int32 (device): the all-gathered outputs of csa_shard_candidates and the
+ *   local counts.  The candidates of rank r must be ascending and below
+ *   rank r+1's (true for contiguous shards in rank order).
+ *   topk_idx [B,Q,k] / topk_cnt [B,Q] (written): the k best candidates by
+ *   (score descending, sequence index ascending; NaN lowest), as ascending
+ *   sequence indices padded with -1 -- the same selection lightning_index_topk
+ *   makes over the whole sequence.
+ *   local_idx [B,Q,k] / local_cnt [B,Q] (written): the selected entries in
+ *   this rank's range [p->entry_offset, p->entry_offset + N_cap), as local
+ *   indices (ascending, padded with -1).
+ * Supported: 1 <= G <= 64 with G*k <= 24320. */
+csa_status csa_merge_candidates(const csa_params* p, int Q, int G, const float* cand_score,
+                                const int32_t* cand_idx, const int32_t* cand_cnt, int64_t N_cap,
+                                int32_t* topk_idx, int32_t* topk_cnt, int32_t* local_idx,
+                                int32_t* local_cnt, int32_t* dev_status, void* stream);
+
+/* sparse_mqa_decode over this rank's share, stopped before the merge: the KV
+ * set is the entries local_idx (topk_idx here) of this rank's cache plus,
+ * when p->window > 0, the window of kv_tok; the list is cut into `splits`
+ * parts (1..64), and each part's unnormalised softmax state is written:
+ *   part_o  [B, splits, H, d] fp16 (device): the part's weighted sum of
+ *           values divided by its own sum (before the inverse rotation),
+ *   part_ml [B, splits, 2, H] fp32 (device): [.., 0, h] the part's largest
+ *           logit times log2(e), [.., 1, h] its sum of 2^(logit*log2 e - max);
+ *           an empty part holds (-inf, 0) and no part_o row.
+ * Other arguments as sparse_mqa_decode (no sink: the merge adds it). */
+csa_status sparse_mqa_partials(const csa_params* p, int splits, const void* q, const int64_t* pos_q,
+                               const void* kv_c, int64_t N_cap, const int32_t* topk_idx,
+                               const int32_t* topk_cnt, const void* kv_tok, int64_t L_cap,
+                               const float* gamma_q, const float* gamma_kv, void* part_o,
+                               float* part_ml, int32_t* dev_status, void* stream);
+
+/* Merge of split partials [B, splits, ...] (the concatenation, in rank
+ * order, of every rank's sparse_mqa_partials output for B = 1): the
+ * output and log-sum-exp of one joint softmax over every part's KV set and
+ * the sink, with the inverse rotation by pos_q -- what sparse_mqa_decode
+ * would write for the union of the parts.  splits 1..4096. */
+csa_status mqa_merge_partials(const csa_params* p, int splits, const void* part_o,
+                              const float* part_ml, const int64_t* pos_q, const float* sink,
+                              void* out, float* lse, int32_t* dev_status, void* stream);
+
 #ifdef __cplusplus
 }
 #endif
