@@ -329,6 +329,9 @@ struct RowShared {
   uint32_t scan[33];
   uint32_t bcast[4];
 };
+// The keys follow RowShared in dynamic shared memory, on a 16-byte boundary
+// (they are written with 16-byte stores).
+constexpr size_t kRowKeysOff = (sizeof(RowShared) + 15) / 16 * 16;
 
 // Exclusive prefix over the block of per-thread values (1024 threads, one
 // value each); warp_tot is 33 words of shared scratch.
@@ -496,7 +499,7 @@ CSA_DEV void row_select(const uint32_t* keys, int n, int k, RowShared& sh, uint3
 __global__ void __launch_bounds__(kThreads, 1) topk_row_kernel(const Params p) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
   RowShared& sh = *reinterpret_cast<RowShared*>(smem_raw);
-  uint32_t* keys = reinterpret_cast<uint32_t*>(smem_raw + sizeof(RowShared));
+  uint32_t* keys = reinterpret_cast<uint32_t*>(smem_raw + kRowKeysOff);
   const int row = blockIdx.x;
   const int tid = threadIdx.x;
   const int64_t pos = p.pos_q ? p.pos_q[row] : p.pos_base + row % p.Q;
@@ -588,7 +591,7 @@ __global__ void __launch_bounds__(kThreads, 1) merge_candidates_kernel(const Mer
   __shared__ int32_t s_off[65];
   __shared__ int32_t s_first, s_nloc;
   const int nmax = p.G * p.k;
-  uint32_t* keys = reinterpret_cast<uint32_t*>(smem_raw + sizeof(RowShared));
+  uint32_t* keys = reinterpret_cast<uint32_t*>(smem_raw + kRowKeysOff);
   int32_t* gidx = reinterpret_cast<int32_t*>(keys + nmax);
   const int row = blockIdx.x, tid = threadIdx.x;
   pdl_trigger();
@@ -674,7 +677,7 @@ cudaError_t launch_merge_candidates(const MergeLaunch& a, cudaStream_t stream) {
   p.local_idx = a.local_idx;
   p.local_cnt = a.local_cnt;
   p.status = a.status;
-  const size_t smem = sizeof(RowShared) + (size_t)a.G * a.k * 8;
+  const size_t smem = kRowKeysOff + (size_t)a.G * a.k * 8;
   if (smem > 220 * 1024) return cudaErrorInvalidValue;
   cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(merge_candidates_kernel), 4, smem);
   if (e != cudaSuccess) return e;
@@ -719,7 +722,7 @@ int max_cluster(const void* kern, size_t smem) {
 }
 
 // Rows of at most this many scores take the one-CTA-per-row kernel.
-constexpr int64_t kRowMaxScores = (200 * 1024 - (int64_t)sizeof(RowShared)) / 4;
+constexpr int64_t kRowMaxScores = (200 * 1024 - (int64_t)kRowKeysOff) / 4;
 
 cudaError_t launch_topk(const TopkLaunch& a, cudaStream_t stream) {
   if (a.rows < 1) return cudaSuccess;
@@ -739,7 +742,7 @@ cudaError_t launch_topk(const TopkLaunch& a, cudaStream_t stream) {
     p.idx = a.idx;
     p.cnt = a.cnt;
     p.status = a.status;
-    const size_t smem = sizeof(RowShared) + (size_t)((a.N_cap + 3) / 4 * 4) * 4;
+    const size_t smem = kRowKeysOff + (size_t)((a.N_cap + 3) / 4 * 4) * 4;
     cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(topk_row_kernel), 3, smem);
     if (e != cudaSuccess) return e;
     return launch_pdl(topk_row_kernel, dim3(a.rows), dim3(kThreads), smem, stream, 0, a.chained,

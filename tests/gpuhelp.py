@@ -60,32 +60,30 @@ def assert_attention_close(got: np.ndarray, ref: np.ndarray, what=""):
 
 
 # Log-sum-exp tolerance, per (row, head).  The tensor cores see the
-# normalised (and rotated) query rounded to bf16, qhat_d (1 + e_d) with
-# |e_d| <= 2^-8 (standard deviation about 2^-8/sqrt(3) = 2.3e-3), and a
-# window token's key, when the kernel rescales or rotates it in bf16, rounded
-# the same way.  The log-sum-exp moves by the attention-weighted mean of the
-# logit errors: for the query part
-#     dLSE = scale * sum_d e_d qhat_d obar_d,   obar = sum_j p_j v_j,
-# where p_j are the softmax weights (sink included) and obar is the output
-# before its inverse rotation, so |obar| = |o| for the head's output o.  With
-# |qhat_d| ~ 1 its standard deviation is about 2.3e-3 * scale * |o|; the key
-# part is at most as large again.  The bound is five standard deviations of
-# the two together, 5 * sqrt(2) * 2.3e-3 * scale * |o|, plus 1e-4 for the fp32
-# accumulation.  A head that attends to one key (|o| ~ sqrt(D)) gets about
-# 1.6e-2 at scale 1/sqrt(D); one that spreads over ~1000 keys, about 1e-3.
-LSE_SIGMA = 2.3e-3
-
-
-def lse_tolerance(out_ref, scale):
+# normalised, rotated query rounded to bf16, qhat_d (1 + e_d) with
+# |e_d| <= 2^-8, and every logit of the head shares that rounding.  To first
+# order the log-sum-exp moves by the softmax-weighted mean of the logit
+# errors,
+#     dLSE = scale * sum_d e_d qhat_d obar_d,    obar = sum_j p_j v_j,
+# the head's output before its inverse rotation (p_j: the weights, sink
+# included), so |dLSE| <= 2^-8 scale sum_d |qhat_d obar_d|
+#                       <= 2^-8 scale |qhat| |o|      (Cauchy-Schwarz; the
+# rotation keeps the norm, |obar| = |o|).  Window rows that the kernel
+# rescales or rotates in bf16 add a key-side rounding of the same order, so
+# the bound is doubled; 1e-4 covers the fp32 accumulation.  |qhat| = sqrt(D)
+# for a unit gain (qnorm_gain scales it for other gains).  On the 128K decode
+# shape the measured errors stay below 0.4 of the query term alone.
+def lse_tolerance(out_ref, scale, qnorm_gain=1.0):
     """Per-(row, head) LSE bound from the oracle's output [..., H, D]."""
     o = np.linalg.norm(np.asarray(out_ref, np.float64), axis=-1)
-    return 5.0 * math.sqrt(2.0) * LSE_SIGMA * scale * o + 1e-4
+    D = np.asarray(out_ref).shape[-1]
+    return 2.0 * 2.0 ** -8 * scale * math.sqrt(D) * qnorm_gain * o + 1e-4
 
 
-def assert_lse_close(got, ref, out_ref, what="", scale=None):
+def assert_lse_close(got, ref, out_ref, what="", scale=None, qnorm_gain=1.0):
     """LSE [..., H] against the oracle's, within lse_tolerance of the oracle's
     output out_ref [..., H, D]; scale is the logit scale (1/sqrt(D) when
-    None)."""
+    None); qnorm_gain the largest query gain (1 without gains)."""
     got = np.asarray(got, np.float64)
     ref = np.asarray(ref, np.float64)
     if scale is None:
@@ -95,7 +93,7 @@ def assert_lse_close(got, ref, out_ref, what="", scale=None):
     assert np.array_equal(got[~fin], ref[~fin]), f"{what}: infinite values differ"
     if not fin.any():
         return 0.0
-    tol = lse_tolerance(out_ref, scale)
+    tol = lse_tolerance(out_ref, scale, qnorm_gain)
     err = np.abs(got - ref)
     _record("lse_abs", float(err[fin].max()))
     _record("lse_over_bound", float((err[fin] / tol[fin]).max()))
