@@ -335,8 +335,30 @@ class Decode:
         ]
 
     def launches_per_step(self):
-        # compress 1, (index 1, top-k 1), attention 1 + merge 1 (the decode
-        # workloads' rows always have several splits, so the merge runs)
+        """Kernel launches of one step, counted from the kernel nodes of a
+        captured step graph (a separate capture kept as a cudaGraph_t);
+        falls back to the call's known sequence (compress, (indexer, top-k,)
+        attention, split merge) where the runtime does not expose nodes."""
+        torch = self.torch
+        try:
+            from cuda.bindings import runtime as rt
+            stream = torch.cuda.Stream()
+            stream.wait_stream(torch.cuda.current_stream())
+            g = torch.cuda.CUDAGraph(keep_graph=True)
+            with torch.cuda.graph(g, stream=stream):
+                self.step(self.sets[0])
+            torch.cuda.synchronize()
+            raw = g.raw_cuda_graph()
+            _, _, n = rt.cudaGraphGetNodes(raw, numNodes=0)
+            _, nodes, n = rt.cudaGraphGetNodes(raw, numNodes=n)
+            kernels = sum(1 for nd in nodes[:n]
+                          if rt.cudaGraphNodeGetType(nd)[1] ==
+                          rt.cudaGraphNodeType.cudaGraphNodeTypeKernel)
+            del g
+            if kernels > 0:
+                return kernels
+        except Exception:  # noqa: BLE001 - the count then falls back
+            pass
         return 5 if self.w.csa else 3
 
     def _warm(self):
@@ -413,6 +435,7 @@ def measure_decode(w, K, W, dev, barrier, rmax, rsum, world, rotate=0, e2e=True)
     graphs = st.capture_steps()
     cycle = st.capture_cycle()
     torch.cuda.synchronize()
+    launches_step = st.launches_per_step()
 
     def plan(n):
         """The graphs that n consecutive steps replay: whole R-step cycles,
@@ -497,7 +520,7 @@ def measure_decode(w, K, W, dev, barrier, rmax, rsum, world, rotate=0, e2e=True)
                                         peaks["hbm_gbs"], 4),
                           "peak": peaks["hbm_gbs"], "peak_source": peaks["source"]},
         "kernels_ms": {k: round(v, 6) for k, v in stage_ms.items()},
-        "gpu_launches": st.launches_per_step() * K,
+        "gpu_launches": launches_step * K,
         "device_status": status,
     }
     if e2e_rec is not None:

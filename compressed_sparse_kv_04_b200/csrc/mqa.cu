@@ -37,8 +37,9 @@
 // Splits of the KV list run on different CTAs; their (m, l, O) partials are
 // merged, with the sink folded in and the inverse RoPE applied, by the CTAs
 // themselves when the S splits of a head group form one thread-block
-// cluster (S <= 16: a cluster barrier, then each CTA merges a share of the
-// heads from L2), else by mqa_combine_kernel.  With one split per row the
+// cluster and all clusters of the launch fit at once (S <= 16: a cluster
+// barrier, then each CTA merges a share of the heads from L2), else by
+// mqa_combine_kernel.  With one split per row the
 // attention CTA finishes its rows directly.  Every wait is bounded and
 // reports CSA_ERR_DEVICE_TIMEOUT.
 #include <algorithm>
@@ -1001,18 +1002,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-// Whether S CTAs of the attention kernel (one per SM) can run as one
-// thread-block cluster on this device: S <= 8 always can in principle, up to
-// 16 with the non-portable cluster size; the occupancy query says whether at
-// least one such cluster fits.  Cached per (device, kernel variant, S).
-bool cluster_fits(const void* kern, int variant, int S, size_t smem) {
-  static int cached[64][8][17] = {};  // 0 unknown, 1 yes, 2 no
-  if (S < 2 || S > 16) return false;
+// How many clusters of S attention CTAs (one per SM) can be resident at once
+// on this device (S <= 8 portable, up to 16 with the non-portable cluster
+// size); 0 when none can.  Cached per (device, kernel variant, S).
+int clusters_resident(const void* kern, int variant, int S, size_t smem) {
+  static int cached[64][8][17] = {};  // 0 unknown, else count + 1
+  if (S < 2 || S > 16) return 0;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64 || variant < 0 || variant >= 8)
-    return false;
+    return 0;
   int& c = cached[dev][variant][S];
-  if (c) return c == 1;
+  if (c) return c - 1;
   bool ok = true;
   if (S > 8 && cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
                    cudaSuccess)
@@ -1031,10 +1031,12 @@ bool cluster_fits(const void* kern, int variant, int S, size_t smem) {
     cfg.numAttrs = 1;
     int n = 0;
     ok = cudaOccupancyMaxActiveClusters(&n, kern, &cfg) == cudaSuccess && n >= 1;
+    c = ok ? n + 1 : 1;
+  } else {
+    c = 1;
   }
   if (!ok) cudaGetLastError();  // a refused query is not the caller's error
-  c = ok ? 1 : 2;
-  return ok;
+  return c - 1;
 }
 
 template <int D, int R>
@@ -1092,9 +1094,12 @@ cudaError_t launch_impl(const MqaLaunch& a, cudaStream_t stream) {
   e = ensure_smem_attr(reinterpret_cast<const void*>(kern), 3 + variant, smem);
   if (e != cudaSuccess) return e;
   dim3 grid(cps * a.splits, rows, 1);
+  // The splits of each head group form one cluster and merge in-kernel, when
+  // every cluster of the launch can be resident at once (otherwise the
+  // clusters would run in waves: the separate merge kernel is faster).
   if (!p.fused && !a.emit_partials &&
-      cluster_fits(reinterpret_cast<const void*>(kern), variant, a.splits, smem)) {
-    // The splits of each head group form one cluster and merge in-kernel.
+      (int64_t)cps * rows <=
+          clusters_resident(reinterpret_cast<const void*>(kern), variant, a.splits, smem)) {
     p.cluster_merge = 1;
     return launch_pdl(kern, grid, dim3(kThreads), smem, stream, a.splits, a.chained, map_q, box_c,
                       box_t, p);

@@ -6,9 +6,9 @@
 // ascending; NaN below every number; -0 == +0.  Output: ascending indices,
 // padded with -1, and the count min(k, n_vis).
 //
-// Rows that fit in one CTA's shared memory (up to ~47K scores) are ranked by
-// topk_row_kernel, one CTA per row; longer rows by topk_kernel:
-// one thread-block cluster of C CTAs (C = 1..16) per query row.  CTA r
+// Many rows, or short ones, that fit in one CTA's shared memory (up to ~47K
+// scores) are ranked by topk_row_kernel, one CTA per row; the other rows by
+// topk_kernel: one thread-block cluster of C CTAs (C = 1..16) per query row.  CTA r
 // keeps its slice of the row in shared memory as order-preserving 32-bit
 // keys.  A radix select finds the exact k-th largest key over the whole row:
 //   - every exchange is a push of plain 16-byte stores: each CTA writes its
@@ -727,7 +727,9 @@ constexpr int64_t kRowMaxScores = (200 * 1024 - (int64_t)kRowKeysOff) / 4;
 cudaError_t launch_topk(const TopkLaunch& a, cudaStream_t stream) {
   if (a.rows < 1) return cudaSuccess;
   if (a.rows > 65535 || a.k > kMaxK) return cudaErrorInvalidConfiguration;
-  if (a.N_cap <= kRowMaxScores) {
+  // One CTA per row when rows fill the GPU (prefill) or are short; a few
+  // long rows (decode) spread each row over a cluster instead.
+  if (a.N_cap <= kRowMaxScores && (a.rows >= device_sm_count() / 4 || a.N_cap <= 8192)) {
     Params p{};
     p.Q = a.Q;
     p.m = a.m;
