@@ -74,7 +74,16 @@ HCA_PREFILL = Workload("hca_prefill_4096_after_65536", "hca_prefill", B=1, L=655
                        d=512, m=128, H=128, rope_dim=64, W=128, P=65536, T=4096,
                        seed=20260007)
 
-ALL = [TINY_CSA, CSA_128K, HCA_1M, CSA_1M, CSA_PREFILL, CSA_FLASH_128K, HCA_PREFILL]
+# Reduced cases for profiler captures (a few GB on the device): the 128K CSA
+# decode with a 32K context (the same per-row attention work: 1024 selected
+# entries + the window), and the HCA decode at 256K (2048 entries per row).
+CSA_32K_PROFILE = Workload("csa_decode_32k_b8", "csa_decode", B=8, L=32768, d=512, m=4, H=128,
+                           rope_dim=64, W=128, H_I=64, D_I=128, k=1024, seed=20260009)
+HCA_256K_PROFILE = Workload("hca_decode_256k_b8", "hca_decode", B=8, L=262144, d=512, m=128,
+                            H=128, rope_dim=64, W=128, seed=20260010)
+
+ALL = [TINY_CSA, CSA_128K, HCA_1M, CSA_1M, CSA_PREFILL, CSA_FLASH_128K, HCA_PREFILL,
+       CSA_32K_PROFILE, HCA_256K_PROFILE]
 BY_NAME = {w.name: w for w in ALL}
 
 

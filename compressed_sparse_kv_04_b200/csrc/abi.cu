@@ -218,7 +218,7 @@ static csa_status compress_common(const char* fn, const csa_params* p, const voi
                                   int64_t N_cap, const void* idx_tok, const float* w_s_idx,
                                   const float* b_pos_idx, uint8_t* idx_key, float* idx_scale,
                                   int32_t* dev_status, void* stream,
-                                  const int64_t* pos_newest = nullptr) {
+                                  const int64_t* pos_newest = nullptr, int pdl_head = 0) {
   csa_status st = check_common(fn, p);
   if (st != CSA_OK) return st;
   REQ_PTR(kv_tok);
@@ -274,6 +274,7 @@ static csa_status compress_common(const char* fn, const csa_params* p, const voi
   c.rope_dim = p->rope_dim;
   fill_inv_freq(p, c.inv_freq);
   c.status = dev_status;
+  c.pdl_head = pdl_head;
   cudaError_t e = csa::launch_compress(c, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(fn, e);
   return CSA_OK;
@@ -311,9 +312,13 @@ static csa_status index_common(const char* fn, const csa_params* p, int Q,
                                const uint8_t* q_idx, const float* q_scale, const float* w,
                                const uint8_t* idx_key, const float* idx_scale, int64_t N_cap,
                                const int64_t* pos_q, int64_t pos_base, float* scores,
-                               int32_t* dev_status, cudaStream_t stream, int chained) {
+                               int32_t* dev_status, cudaStream_t stream, int chained,
+                               const int64_t* safe_pos = nullptr,
+                               int64_t safe_fixed = INT64_MAX) {
   csa::IndexLaunch a{};
   a.chained = chained;
+  a.safe_pos = safe_pos;
+  a.safe_fixed = safe_fixed;
   a.B = p->B;
   a.Q = Q;
   a.H_I = p->H_I;
@@ -364,9 +369,12 @@ static csa_status index_topk_common(const char* fn, const csa_params* p, int Q,
                                     const uint8_t* idx_key, const float* idx_scale,
                                     int64_t N_cap, const int64_t* pos_q, int64_t pos_base,
                                     int32_t* topk_idx, int32_t* topk_cnt, float* scores,
-                                    int32_t* dev_status, cudaStream_t stream, int chained) {
+                                    int32_t* dev_status, cudaStream_t stream, int chained,
+                                    const int64_t* safe_pos = nullptr,
+                                    int64_t safe_fixed = INT64_MAX) {
   csa_status st = index_common(fn, p, Q, q_idx, q_scale, w, idx_key, idx_scale, N_cap, pos_q,
-                               pos_base, scores, dev_status, stream, chained);
+                               pos_base, scores, dev_status, stream, chained, safe_pos,
+                               safe_fixed);
   if (st != CSA_OK) return st;
   return topk_common(fn, p, Q, scores, N_cap, pos_q, pos_base, topk_idx, topk_cnt, dev_status,
                      stream, 1);
@@ -577,6 +585,9 @@ csa_status csa_prefill_chunk(const csa_params* p, int64_t P, int T, const void* 
   csa_status st = check_common(fn, p);
   if (st != CSA_OK) return st;
   if (p->B != 1) return fail(CSA_ERR_UNSUPPORTED_SHAPE, "%s: B=%d (supported: 1)", fn, p->B);
+  if (p->entry_offset != 0)
+    return fail(CSA_ERR_UNSUPPORTED_SHAPE, "%s: entry_offset=%lld (supported: 0)", fn,
+                (long long)p->entry_offset);
   st = check_indexer(fn, p);
   if (st != CSA_OK) return st;
   st = check_attention(fn, p);
@@ -616,8 +627,9 @@ csa_status csa_prefill_chunk(const csa_params* p, int64_t P, int T, const void* 
   // 2-3. Causal indexer and top-k for the T queries at positions P .. P+T-1.
   float* scores = static_cast<float*>(ws);
   csa_params p1 = *p;
+  // The keys of blocks before P/m were written before this call.
   st = index_topk_common(fn, &p1, T, q_idx, q_scale, w, idx_key, idx_scale, N_cap, nullptr, P,
-                         topk_idx, topk_cnt, scores, dev_status, s, 1);
+                         topk_idx, topk_cnt, scores, dev_status, s, 1, nullptr, b0);
   if (st != CSA_OK) return st;
   // 4. Sparse MQA per query, each with its own causal window.
   char* rest = static_cast<char*>(ws) + scores_bytes(T, N_cap);
@@ -659,12 +671,14 @@ csa_status csa_decode_step(const csa_params* p, const int64_t* pos_q, const void
   // 1. Each sequence's newest block: the one holding its query token,
   // pooled over the tokens up to it.
   st = compress_common(fn, p, kv_tok, L_cap, nullptr, 0, w_s, b_pos, gamma, 0, 1, kv_c, N_cap,
-                       idx_tok, w_s_idx, b_pos_idx, idx_key, idx_scale, dev_status, stream, pos_q);
+                       idx_tok, w_s_idx, b_pos_idx, idx_key, idx_scale, dev_status, stream, pos_q,
+                       1);
   if (st != CSA_OK) return st;
   // 2-3. Indexer and top-k over each sequence's visible entries.
   float* scores = static_cast<float*>(ws);
+  // Only each sequence's newest block is written by this call.
   st = index_topk_common(fn, p, 1, q_idx, q_scale, w, idx_key, idx_scale, N_cap, pos_q, 0,
-                         topk_idx, topk_cnt, scores, dev_status, s, 1);
+                         topk_idx, topk_cnt, scores, dev_status, s, 1, pos_q);
   if (st != CSA_OK) return st;
   // 4. Sparse MQA over the selection, the window and the sink.
   char* rest = static_cast<char*>(ws) + scores_bytes(p->B, N_cap);
@@ -690,7 +704,7 @@ csa_status hca_decode_step(const csa_params* p, const int64_t* pos_q, const void
   if (!aligned16(ws)) return fail(CSA_ERR_INVALID_ARG, "%s: ws is not 16-byte aligned", fn);
   // 1. Each sequence's newest block, then 2. dense MQA with window and sink.
   st = compress_common(fn, p, kv_tok, L_cap, nullptr, 0, w_s, b_pos, gamma, 0, 1, kv_c, N_cap,
-                       nullptr, nullptr, nullptr, nullptr, nullptr, dev_status, stream, pos_q);
+                       nullptr, nullptr, nullptr, nullptr, nullptr, dev_status, stream, pos_q, 1);
   if (st != CSA_OK) return st;
   return mqa_common(fn, p, CSA_OP_DENSE_MQA, p->B, 1, q, pos_q, 0, kv_c, N_cap, nullptr, nullptr,
                     kv_tok, L_cap, sink, gamma_q, gamma_kv, out, lse, ws, ws_bytes, dev_status,
@@ -707,6 +721,9 @@ csa_status hca_prefill_chunk(const csa_params* p, int64_t P, int T, const void* 
   csa_status st = check_common(fn, p);
   if (st != CSA_OK) return st;
   if (p->B != 1) return fail(CSA_ERR_UNSUPPORTED_SHAPE, "%s: B=%d (supported: 1)", fn, p->B);
+  if (p->entry_offset != 0)
+    return fail(CSA_ERR_UNSUPPORTED_SHAPE, "%s: entry_offset=%lld (supported: 0)", fn,
+                (long long)p->entry_offset);
   st = check_attention(fn, p);
   if (st != CSA_OK) return st;
   if (P < 0 || T < 1 || P % p->m != 0)

@@ -57,6 +57,10 @@ struct PoolArgs {
   // The cache holds entries entry_offset .. of the sequence: local entry i is
   // block entry_offset + i (its tokens and its rotation position).
   int64_t entry_offset;
+  // 1: launched as the first kernel of a call with programmatic serialization
+  // (it may start while the caller's previous kernel runs): every global
+  // read waits for that kernel, and dependents are let in only afterwards.
+  int pdl_head;
   // [B] device, or null.  Set: one block per sequence, the one holding
   // position pos_newest[b], pooled over tokens up to pos_newest[b].
   const int64_t* pos_newest;
@@ -371,6 +375,7 @@ CSA_DEV void pool_stream(const PoolArgs& a, const StreamArgs& sa, float* smem) {
 
 __global__ void __launch_bounds__(kThreads) compress_kernel(const PoolArgs a) {
   extern __shared__ float smem[];
+  if (a.pdl_head) pdl_wait();  // nothing of the caller's is read before its kernels end
   pdl_trigger();
   const StreamArgs& sa = a.s[blockIdx.y];
   switch (sa.dim) {
@@ -404,6 +409,7 @@ cudaError_t launch_compress(const CompressLaunch& c, cudaStream_t stream) {
   a.ctx_len_value = c.ctx_len_value;
   a.first_block = c.first_block;
   a.entry_offset = c.entry_offset;
+  a.pdl_head = c.pdl_head;
   a.n_blocks = c.pos_newest ? 1 : c.n_blocks;
   a.pos_newest = c.pos_newest;
   a.eps = c.eps;
@@ -417,7 +423,8 @@ cudaError_t launch_compress(const CompressLaunch& c, cudaStream_t stream) {
   int maxdim = c.idx_tok && c.D_I > c.d ? c.D_I : c.d;
   size_t smem = G == 1 ? 0 : (size_t)kWarps * (maxdim + 2) * sizeof(float);
   dim3 grid((unsigned)grid_x, a.nstreams);
-  return launch_pdl(compress_kernel, grid, dim3(kThreads), smem, stream, 0, c.chained, a);
+  return launch_pdl(compress_kernel, grid, dim3(kThreads), smem, stream, 0,
+                    c.chained || c.pdl_head, a);
 }
 
 }  // namespace csa

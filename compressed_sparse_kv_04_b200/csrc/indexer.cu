@@ -44,6 +44,13 @@ struct Params {
   int B, Q, H_I, HP, G, N, m;
   int64_t N_cap;
   int64_t entry_offset;  // the cache holds entries entry_offset .. of the sequence
+  // Entries below this bound were written before this call and may be read
+  // before pdl_wait(); the rest (written by the previous kernel of the
+  // call) only after it.  safe_pos: per sequence, entries below
+  // safe_pos[b] / m - entry_offset (the block holding position safe_pos[b]
+  // is the one being written); else safe_fixed for every sequence.
+  const int64_t* safe_pos;
+  int64_t safe_fixed;
   int tiles_per_chunk, ntiles, qgroups;
   const uint8_t* q_idx;
   const float* q_scale;
@@ -62,6 +69,14 @@ CSA_DEV uint64_t desc_kmajor(uint32_t saddr) {
   d &= ~(7ull << 61);
   d |= Cfg<DI>::kLayout << 61;
   return d;
+}
+
+// Entries of sequence b below this bound may be read before pdl_wait().
+CSA_DEV int64_t safe_bound(const Params& p, int b) {
+  if (!p.safe_pos) return p.safe_fixed;
+  const int64_t t = p.safe_pos[b];
+  const int64_t i = (t < 0 ? 0 : t / p.m) - p.entry_offset;
+  return i < 0 ? 0 : i;
 }
 
 template <int DI>
@@ -162,16 +177,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------- TMA producer --
     if (elect_one()) {
       tma_prefetch_desc(&kmap);
-      pdl_wait();  // the keys are written by the compression kernel
+      // Tiles of entries written before this call stream at once; the first
+      // tile with an entry that the previous kernel writes waits for it.
+      const int64_t safe = safe_bound(p, b);
+      bool waited = false;
       int it = 0;
       for (int t = t_begin; t < t_end; ++t, ++it) {
         int s = it % C::kStages;
         uint32_t ph = (it / C::kStages) & 1;
+        if (!waited && (int64_t)(t + 1) * kTileRows > safe) {
+          pdl_wait();
+          waited = true;
+        }
         if (!mbar_wait(&empty[s], ph ^ 1, p.status, abort_flag)) break;
         mbar_expect_tx(&full[s], C::kStageBytes);
         tma_load_2d(ring + s * C::kStageBytes, &kmap, &full[s], 0,
                     (int32_t)((int64_t)b * p.N_cap + (int64_t)t * kTileRows));
       }
+      if (!waited) pdl_wait();  // this grid completes only after its predecessor
       // On abort, wait for the copies still in flight before the CTA exits.
       if (*abort_flag) {
         int issued = it;
@@ -212,7 +235,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ epilogue --
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
-    pdl_wait();  // key scales are read and scores written below
+    // Key scales follow the producer's rule (read through L2: a line may
+    // hold scales from both sides of the bound); the scores are a buffer no
+    // earlier kernel of the call touches.
+    const int64_t safe = safe_bound(p, b);
+    bool waited = false;
+    auto ensure = [&](int t) {
+      if (!waited && (int64_t)(t + 1) * kTileRows > safe) {
+        pdl_wait();
+        waited = true;
+      }
+    };
     int64_t nv[8];
 #pragma unroll
     for (int g = 0; g < 8; ++g) nv[g] = 0;
@@ -230,8 +263,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     // the previous tile's work.
     auto load_ks = [&](int t) -> float {
       const int64_t e = (int64_t)t * kTileRows + row;
-      return e < p.N_cap ? __ldg(p.key_scale + (int64_t)b * p.N_cap + e) : 0.f;
+      return e < p.N_cap ? __ldcg(p.key_scale + (int64_t)b * p.N_cap + e) : 0.f;
     };
+    ensure(t_begin);
     float ks_next = load_ks(t_begin);
     int it = 0;
     for (int t = t_begin; t < t_end; ++t, ++it) {
@@ -239,7 +273,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t aph = (it >> 1) & 1;
       const int64_t entry = (int64_t)t * kTileRows + row;
       const float ks = ks_next;
-      if (t + 1 < t_end) ks_next = load_ks(t + 1);
+      if (t + 1 < t_end) {
+        ensure(t + 1);
+        ks_next = load_ks(t + 1);
+      }
       bool ok = mbar_wait(&tfull[a], aph, p.status, abort_flag);
       if (!__all_sync(0xffffffffu, ok)) break;  // keep the warp converged for tcgen05.ld
       tc_fence_after();
@@ -267,6 +304,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       mbar_arrive(&tempty[a]);
     }
+    if (!waited) pdl_wait();  // this grid completes only after its predecessor
   }
   // Teardown: every warp reports (converged) that it is done with tensor
   // memory; warp 0 frees it after all of them (bounded wait).
@@ -294,6 +332,8 @@ cudaError_t launch_impl(const IndexLaunch& a, cudaStream_t stream) {
   p.m = a.m;
   p.N_cap = a.N_cap;
   p.entry_offset = a.entry_offset;
+  p.safe_pos = a.safe_pos;
+  p.safe_fixed = a.safe_fixed;
   p.ntiles = (int)((a.N_cap + kTileRows - 1) / kTileRows);
   p.qgroups = (a.Q + p.G - 1) / p.G;
   p.q_idx = a.q_idx;

@@ -14,6 +14,10 @@ struct CompressLaunch {
   int B, d, D_I, m;
   int overlap;              // tokens of block i-1 that entry i also pools (b_pos has m + overlap)
   int64_t entry_offset;     // local entry i is block entry_offset + i of the sequence
+  // First kernel of a call, launched with programmatic serialization: it
+  // waits for the previous kernel before any global read and lets its
+  // dependents start only after that (so they may read the call's inputs).
+  int pdl_head;
   int64_t L_cap, N_cap;
   const void* kv_tok;
   const void* idx_tok;  // null: KV stream only
@@ -49,6 +53,12 @@ struct IndexLaunch {
   int32_t* status;
   int num_sms;
   int64_t entry_offset;     // the cache holds entries entry_offset .. N_cap-1+entry_offset
+  // Keys of entries below the bound were written before the call and are
+  // read before waiting on the previous kernel: safe_pos[b] / m (per
+  // sequence, the block holding that position is being written) when given,
+  // else safe_fixed.
+  const int64_t* safe_pos;
+  int64_t safe_fixed;
   int chained;              // see launch_pdl
 };
 cudaError_t launch_index_scores(const IndexLaunch& a, cudaStream_t stream);
@@ -158,10 +168,14 @@ int device_sm_count();
 // itself started only after everything before the call had completed.  So
 // their reads of caller inputs before pdl_wait() are safe, and their reads
 // of data written by an earlier kernel of the call come after pdl_wait().
-// chained == 0 (the first kernel of every entry point): an ordinary launch,
+// chained == 0 (the first kernel of an entry point): an ordinary launch,
 // which starts after all earlier work in the stream has completed, whatever
 // that work is (a caller's kernel that lets its dependents start early
-// included).
+// included).  The decode steps' first kernel (compression) instead runs in
+// a head mode: launched with programmatic serialization, it waits for the
+// previous kernel before it reads anything and triggers its dependents only
+// after that wait, which gives the same guarantee while its launch overlaps
+// the previous kernel.
 template <typename... KArgs, typename... Args>
 cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
                        cudaStream_t stream, int cluster_x, int chained, Args... args) {

@@ -26,9 +26,11 @@
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
  *     stream).  Calls only enqueue work; they are stream-ordered, keep no
  *     state between calls and may be captured into a CUDA graph.
- *   - Ordering: the first kernel of every call is an ordinary launch, so it
- *     starts only after all earlier work on the stream has completed --
- *     including a caller's kernel that lets its dependents launch early.
+ *   - Ordering: the first kernel of every call starts its work only after
+ *     all earlier work on the stream has completed -- including a caller's
+ *     kernel that lets its dependents launch early.  (It is an ordinary
+ *     launch, except in the decode steps, where it may be scheduled early
+ *     but waits for the previous kernel before reading anything.)
  *     The later kernels of a call may start while their predecessor in the
  *     same call still runs (programmatic dependent launch) and read the
  *     call's inputs early; they wait for that predecessor before reading
@@ -343,7 +345,7 @@ csa_status dense_mqa_decode(const csa_params* p, const void* q, const int64_t* p
  * (ctx_len = P+T); the Lightning Indexer for every new query t with its own
  * causal visible count floor((t+1)/m); top-k per query; and the sparse MQA
  * per query with its own window [max(0,t-W+1), t].  P must be a multiple
- * of m.
+ * of m, and the cache is a whole one (entry_offset = 0).
  *   q [T, H, d] bf16, q_idx [T, H_I, D_I] E4M3, q_scale/w [T, H_I] fp32,
  *   out [T, H, d] bf16 (written), topk_idx [T, k] / topk_cnt [T] (written).
  * ------------------------------------------------------------------------- */
