@@ -143,6 +143,9 @@ CSA_DEV void pool_tokens(const __nv_bfloat16* blk, int j0, int j_load, int j_use
   l = 0.f;
 #pragma unroll
   for (int e = 0; e < E; ++e) acc[e] = 0.f;
+  // The position biases of this warp's tokens (at most 32), one load per
+  // lane up front instead of one dependent load per token.
+  const float bp = j0 + lane < j_use ? __ldg(b_pos + j0 + lane) : 0.f;
   for (int j = j0; j < j_load; j += RB) {
     uint32_t w[RB][E / 2];
 #pragma unroll
@@ -160,7 +163,8 @@ CSA_DEV void pool_tokens(const __nv_bfloat16* blk, int j0, int j_load, int j_use
       float d4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int e = 0; e < E; ++e) d4[e & 3] = fmaf(x[e], ws[e], d4[e & 3]);
-      float s = warp_sum((d4[0] + d4[1]) + (d4[2] + d4[3])) + __ldg(b_pos + j + u);
+      float s = warp_sum((d4[0] + d4[1]) + (d4[2] + d4[3])) +
+                __shfl_sync(0xffffffffu, bp, (j + u - j0) & 31);
       float mn = fmaxf(mx, s);
       float corr = __expf(mx - mn);
       float p = __expf(s - mn);
@@ -174,7 +178,7 @@ CSA_DEV void pool_tokens(const __nv_bfloat16* blk, int j0, int j_load, int j_use
 
 template <int DIM>
 CSA_DEV void finish_row(const StreamArgs& sa, const PoolArgs& a, int64_t row, int64_t pos,
-                        int lane, float (&p)[DIM / 32], float eps) {
+                        int lane, float (&p)[DIM / 32], float eps, const float (&gam)[DIM / 32]) {
   using LN = Lane<DIM>;
   constexpr int E = DIM / 32;
   float ss = 0.f;
@@ -187,8 +191,7 @@ CSA_DEV void finish_row(const StreamArgs& sa, const PoolArgs& a, int64_t row, in
 #pragma unroll
     for (int v = 0; v < LN::VEC; ++v) {
       int e = part * LN::VEC + v;
-      float g = sa.gamma ? __ldg(sa.gamma + LN::elem(lane, part, v)) : 1.f;
-      p[e] = p[e] * inv * g;
+      p[e] = p[e] * inv * gam[e];
     }
   if (sa.rope_dim > 0) {
     // Rotate-half over the last R dims, to the entry's position.  Those dims
@@ -316,6 +319,13 @@ CSA_DEV void pool_stream(const PoolArgs& a, const StreamArgs& sa, float* smem) {
   for (int part = 0; part < LN::NPART; ++part)
 #pragma unroll
     for (int v = 0; v < LN::VEC; ++v) ws[part * LN::VEC + v] = __ldg(sa.w_s + LN::elem(lane, part, v));
+  // The gains, loaded with the other inputs (used after the pooling).
+  float gam[E];
+#pragma unroll
+  for (int part = 0; part < LN::NPART; ++part)
+#pragma unroll
+    for (int v = 0; v < LN::VEC; ++v)
+      gam[part * LN::VEC + v] = sa.gamma ? __ldg(sa.gamma + LN::elem(lane, part, v)) : 1.f;
 
   // Row j of the window is blk + j*DIM (only rows j >= jlo are touched).
   const __nv_bfloat16* blk = sa.tok + ((int64_t)b * a.L_cap + gblk * a.m - a.overlap) * DIM;
@@ -334,7 +344,7 @@ CSA_DEV void pool_stream(const PoolArgs& a, const StreamArgs& sa, float* smem) {
     if (!active || present == 0) return;
 #pragma unroll
     for (int e = 0; e < E; ++e) acc[e] = acc[e] / l;
-    finish_row<DIM>(sa, a, b * a.N_cap + i, (gblk + 1) * a.m - 1, lane, acc, a.eps);
+    finish_row<DIM>(sa, a, b * a.N_cap + i, (gblk + 1) * a.m - 1, lane, acc, a.eps, gam);
     return;
   }
   // Merge the G warp partials of the one block of this CTA.
@@ -370,7 +380,7 @@ CSA_DEV void pool_stream(const PoolArgs& a, const StreamArgs& sa, float* smem) {
   }
 #pragma unroll
   for (int e = 0; e < E; ++e) p[e] = p[e] / L;
-  finish_row<DIM>(sa, a, b * a.N_cap + i, (gblk + 1) * a.m - 1, lane, p, a.eps);
+  finish_row<DIM>(sa, a, b * a.N_cap + i, (gblk + 1) * a.m - 1, lane, p, a.eps, gam);
 }
 
 __global__ void __launch_bounds__(kThreads) compress_kernel(const PoolArgs a) {
