@@ -110,10 +110,14 @@ float softmax_scale_of(const csa_params* p) {
   return p->softmax_scale > 0.f ? p->softmax_scale : (float)(1.0 / std::sqrt((double)p->d));
 }
 
-int splits_for(const csa_params* p, csa_op op, int rows, int64_t N_cap) {
+// reserve: SMs held by a kernel that runs alongside the attention (the
+// compression of an HCA decode step, one CTA per sequence), left out so
+// that every attention CTA is resident from the start.
+int splits_for(const csa_params* p, csa_op op, int rows, int64_t N_cap, int reserve = 0) {
   const int64_t compressed_max = (op == CSA_OP_DENSE_MQA) ? N_cap : (int64_t)p->k;
-  return csa::mqa_choose_splits(rows, compressed_max, p->window, csa::device_sm_count(),
-                                p->H);
+  const int sms = csa::device_sm_count();
+  return csa::mqa_choose_splits(rows, compressed_max, p->window,
+                                sms - reserve >= 2 ? sms - reserve : sms, p->H);
 }
 
 }  // namespace
@@ -197,8 +201,8 @@ size_t csa_workspace_bytes(const csa_params* p, csa_op op, int Q, int64_t N_cap)
                                       p->d) +
              512;
     case CSA_OP_HCA_DECODE_STEP:
-      return csa::mqa_workspace_bytes(p->B, splits_for(p, CSA_OP_DENSE_MQA, p->B, N_cap), p->H,
-                                      p->d) +
+      return csa::mqa_workspace_bytes(p->B, splits_for(p, CSA_OP_DENSE_MQA, p->B, N_cap, p->B),
+                                      p->H, p->d) +
              256;
     case CSA_OP_HCA_PREFILL: {
       int rows = Q;
@@ -467,8 +471,10 @@ static csa_status mqa_common(const char* fn, const csa_params* p, csa_op op, int
                              const int32_t* sel_cnt, const void* kv_tok, int64_t L_cap,
                              const float* sink, const float* gamma_q, const float* gamma_kv,
                              void* out, float* lse, void* ws, size_t ws_bytes,
-                             int32_t* dev_status, cudaStream_t stream, int chained) {
-  int splits = splits_for(p, op, rows, N_cap);
+                             int32_t* dev_status, cudaStream_t stream, int chained,
+                             const int64_t* safe_pos = nullptr, int64_t safe_fixed = 0,
+                             int reserve = 0) {
+  int splits = splits_for(p, op, rows, N_cap, reserve);
   size_t need = csa::mqa_workspace_bytes(rows, splits, p->H, p->d);
   if (!ws || ws_bytes < need)
     return fail(CSA_ERR_WORKSPACE, "%s: workspace of %zu bytes needed, %zu given", fn, need,
@@ -507,6 +513,8 @@ static csa_status mqa_common(const char* fn, const csa_params* p, csa_op op, int
   a.status = dev_status;
   a.chained = chained;
   a.entry_offset = p->entry_offset;
+  a.safe_pos = safe_pos;
+  a.safe_fixed = safe_fixed;
   cudaError_t e = csa::launch_mqa(a, stream);
   if (e != cudaSuccess) return cuda_fail(fn, e);
   return CSA_OK;
@@ -706,9 +714,11 @@ csa_status hca_decode_step(const csa_params* p, const int64_t* pos_q, const void
   st = compress_common(fn, p, kv_tok, L_cap, nullptr, 0, w_s, b_pos, gamma, 0, 1, kv_c, N_cap,
                        nullptr, nullptr, nullptr, nullptr, nullptr, dev_status, stream, pos_q, 1);
   if (st != CSA_OK) return st;
+  // Only each sequence's newest block is written by this call: the older
+  // entries stream in while it is compressed.
   return mqa_common(fn, p, CSA_OP_DENSE_MQA, p->B, 1, q, pos_q, 0, kv_c, N_cap, nullptr, nullptr,
                     kv_tok, L_cap, sink, gamma_q, gamma_kv, out, lse, ws, ws_bytes, dev_status,
-                    static_cast<cudaStream_t>(stream), 1);
+                    static_cast<cudaStream_t>(stream), 1, pos_q, 0, p->B);
 }
 
 csa_status hca_prefill_chunk(const csa_params* p, int64_t P, int T, const void* kv_tok,
@@ -756,10 +766,11 @@ csa_status hca_prefill_chunk(const csa_params* p, int64_t P, int T, const void* 
                        nblk_total - b0, kv_c, N_cap, nullptr, nullptr, nullptr, nullptr, nullptr,
                        dev_status, stream);
   if (st != CSA_OK) return st;
-  // 2. Dense MQA per query over its visible entries and its causal window.
+  // 2. Dense MQA per query over its visible entries and its causal window
+  // (entries below b0 were written before the call).
   return mqa_common(fn, p, CSA_OP_DENSE_MQA, T, T, q, nullptr, P, kv_c, N_cap, nullptr, nullptr,
                     kv_tok, L_cap, sink, gamma_q, gamma_kv, out, lse, ws, ws_bytes, dev_status,
-                    static_cast<cudaStream_t>(stream), 1);
+                    static_cast<cudaStream_t>(stream), 1, nullptr, b0);
 }
 
 // ------------------------------------------------- grouped output projection --

@@ -130,6 +130,13 @@ struct MqaLaunch {
   int64_t entry_offset;     // the cache holds entries entry_offset .. of the sequence
   int chained;              // see launch_pdl (the merge kernel is always chained)
   int emit_partials;        // write the split partials only (no merge, no output)
+  // Without a selection, cached entries below the bound were written before
+  // the call and are read before waiting on the previous kernel:
+  // safe_pos[b] / m (per sequence, the block holding that position is being
+  // written) when given, else safe_fixed (0: every cached entry waits).
+  // Window tokens are caller inputs and never wait; a selection always does.
+  const int64_t* safe_pos = nullptr;
+  int64_t safe_fixed = 0;
 };
 size_t mqa_workspace_bytes(int rows, int splits, int H, int D);
 int mqa_choose_splits(int rows, int64_t compressed_max, int window, int num_sms, int H);

@@ -101,6 +101,10 @@ struct Params {
   int Q, H, m, W, R, splits;
   int64_t N_cap, L_cap;
   int64_t entry_offset;  // the cache holds entries entry_offset .. of the sequence
+  // Cached entries below this bound were written before the call and are
+  // read before pdl_wait(); see MqaLaunch.
+  const int64_t* safe_pos;
+  int64_t safe_fixed;
   const __nv_bfloat16* q;
   const int64_t* pos_q;
   int64_t pos_base;
@@ -305,6 +309,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* qfull = done + 1;  // the query block landed in the last stage
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(qfull + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  // The gains, staged once by the warps that use them: [0, D) gamma_q,
+  // [D, 2D) gamma_kv (ones where not given).
+  float* gam_s = reinterpret_cast<float*>(
+      (reinterpret_cast<uintptr_t>(abort_flag + 1) + 15) & ~uintptr_t(15));
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   pdl_trigger();
@@ -341,6 +349,29 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int c = p.sel_cnt[row];
     return c < 0 ? 0 : (c > p.kmax ? p.kmax : c);
   };
+  // Tiles that read nothing the previous kernel of the call writes: window
+  // tokens (caller inputs) and, without a selection, tiles whose visible
+  // entries all lie below the safe bound (written before the call).  Only
+  // the roles that read cached entries or the selection wait, just before
+  // the first tile that is not safe; a selection is never safe.
+  int64_t safe_e = 0;
+  if (!p.sel_idx) {
+    if (p.safe_pos) {
+      const int64_t sp = p.safe_pos[b];
+      safe_e = (sp < 0 ? 0 : sp / p.m) - p.entry_offset;
+    } else {
+      safe_e = p.safe_fixed;
+    }
+  }
+  auto tile_safe = [&](int t) -> bool {
+    if (t >= tiles_c) return true;
+    if (p.sel_idx) return false;
+    const int64_t end = (int64_t)(t + 1) * TN < n_vis ? (int64_t)(t + 1) * TN : n_vis;
+    return end <= safe_e;
+  };
+  // The selection count is read only by CTAs with selected tiles (after
+  // their wait).
+  const bool sel_tiles = p.sel_idx != nullptr && t0 < tiles_c;
 
   float* pml = p.part_ml + ((int64_t)row * p.splits + split) * 2 * p.H;
 
@@ -389,7 +420,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_load_2d(stages + (C::kStages - 1) * C::kStageBytes + c * C::kChunkBytes, &map_q, qfull,
                     c * 64, row * p.H + hg0);
     }
-    pdl_wait();
+    bool waited = false;
+    auto ensure = [&](int t) {
+      if (!waited && !tile_safe(t)) {
+        pdl_wait();
+        waited = true;
+      }
+    };
     // Selected indices of the next tile are loaded one tile ahead, and
     // independently of the selection count (both round trips overlap).
     auto load_idx = [&](int t, int hh) -> int64_t {
@@ -397,12 +434,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       return (p.sel_idx && t < tiles_c && j < p.kmax) ? (int64_t)p.sel_idx[(int64_t)row * p.kmax + j]
                                                        : 0;
     };
-    int64_t nxt0 = load_idx(t0, 0), nxt1 = load_idx(t0, 1);
-    const int n_c = sel_count();
+    if (t0 < t1) ensure(t0);
+    int64_t nxt0 = t0 < t1 ? load_idx(t0, 0) : 0, nxt1 = t0 < t1 ? load_idx(t0, 1) : 0;
+    const int n_c = sel_tiles ? sel_count() : (p.sel_idx ? 0 : (int)n_vis);
     int it = 0;
     for (int t = t0; t < t1; ++t, ++it) {
       const int64_t cur[2] = {nxt0, nxt1};
       if (t + 1 < t1) {
+        ensure(t + 1);
         nxt0 = load_idx(t + 1, 0);
         nxt1 = load_idx(t + 1, 1);
       }
@@ -476,6 +515,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (t0 + j >= tiles_c || p.sel_idx == nullptr)
           mbar_wait(&full[j % C::kStages], (j / C::kStages) & 1, p.status);
     }
+    // A CTA whose tiles were all safe still waits once, so that the grid
+    // does not complete before the previous kernel.
+    if (!waited) pdl_wait();
   } else if (warp == 1) {
     // -------------------------------------------------------- MMA issuer --
     constexpr int kPvN = D >= 256 ? 256 : D;  // N of one P.V instruction
@@ -534,8 +576,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     // and the KV gain in place.  Every real row: RoPE on the rotated dims.
     const int tid = threadIdx.x - 64;  // 0..127
     const int r = tid >> 1, hf = tid & 1;
-    pdl_wait();
-    const int n_c = sel_count();
+    for (int i = tid; i < D; i += 128) gam_s[D + i] = p.gamma_kv ? __ldg(p.gamma_kv + i) : 1.f;
+    named_barrier_sync(2, 128);  // the transform warps
+    if (sel_tiles) pdl_wait();  // selected rows are gathered here
+    const int n_c = sel_tiles ? sel_count() : (p.sel_idx ? 0 : (int)n_vis);
     // Tile `it`: selected entries are fetched here (thread pair r gathers
     // row r, half hf each, 16 bytes per cp.async) once the stage is free;
     // every thread then arrives on full[s] (after its copies land).
@@ -611,11 +655,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             a4[e] = fmaf(lo, lo, fmaf(hi, hi, a4[e]));
           }
           if (p.gamma_kv) {
-            const float* g = p.gamma_kv + c * 8;
+            const float* g = gam_s + D + c * 8;
 #pragma unroll
             for (int e = 0; e < 4; ++e)
-              w4[e] = pack_bf16(bf16_lo(w4[e]) * __ldg(g + 2 * e),
-                                bf16_hi(w4[e]) * __ldg(g + 2 * e + 1));
+              w4[e] = pack_bf16(bf16_lo(w4[e]) * g[2 * e], bf16_hi(w4[e]) * g[2 * e + 1]);
             *reinterpret_cast<uint4*>(st + tile_off(r, c * 8)) =
                 make_uint4(w4[0], w4[1], w4[2], w4[3]);
           }
@@ -679,6 +722,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     // columns) writes 64 dims of both halves.  The rotated dims (the last R)
     // all sit in the last 64-dim chunk of half 1.
     {
+      for (int i = threadIdx.x - 192; i < D; i += 128)
+        gam_s[i] = p.gamma_q ? __ldg(p.gamma_q + i) : 1.f;
+      named_barrier_sync(1, 128);  // the softmax warps
       // The block is in the last stage (TMA, 128-byte swizzled chunks):
       // row hl, dims [hf*D/2, hf*D/2 + D/2).
       const uint8_t* qs = stages + (C::kStages - 1) * C::kStageBytes;
@@ -712,7 +758,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       float ss = (a4[0] + a4[1]) + (a4[2] + a4[3]);
       ss += __shfl_xor_sync(0xffffffffu, ss, 16);  // the row's other half
       const float inv = (head_ok && qok) ? 1.0f / sqrtf(ss / (float)D + p.eps) : 0.f;
-      const float* gq = p.gamma_q ? p.gamma_q + hf * (D / 2) : nullptr;
+      const float* gq = gam_s + hf * (D / 2);
       constexpr int kChunks = D / 128;  // 64-dim chunks per half row
 #pragma unroll 1
       for (int c = 0; c < kChunks; ++c) {
@@ -728,10 +774,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             x[8 * u + 2 * e + 1] = bf16_hi(w4[e]) * inv;
           }
         }
-        if (gq) {
+        {
 #pragma unroll
           for (int j = 0; j < 64; j += 4) {
-            const float4 g = __ldg(reinterpret_cast<const float4*>(gq + 64 * c + j));
+            const float4 g = *reinterpret_cast<const float4*>(gq + 64 * c + j);
             x[j] *= g.x;
             x[j + 1] *= g.y;
             x[j + 2] *= g.z;
@@ -760,7 +806,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       mbar_arrive(qready);
     }
-    pdl_wait();  // the query prologue above overlaps the previous kernel
+    // (No wait: these warps read only tiles the producer and the transform
+    // warps have made ready, which waited where a tile needed it.)
 
     float m_run = -INFINITY, l_run = 0.f;
     for (int it = 0; it < ntile; ++it) {
@@ -1057,6 +1104,8 @@ cudaError_t launch_impl(const MqaLaunch& a, cudaStream_t stream) {
   p.pos_base = a.pos_base;
   p.sel_idx = a.sel_idx;
   p.sel_cnt = a.sel_cnt;
+  p.safe_pos = a.safe_pos;
+  p.safe_fixed = a.safe_fixed;
   p.kv_c = reinterpret_cast<const __nv_bfloat16*>(a.kv_c);
   p.kmax = a.kmax;
   p.gamma_q = a.gamma_q;
@@ -1088,7 +1137,7 @@ cudaError_t launch_impl(const MqaLaunch& a, cudaStream_t stream) {
   if (e != cudaSuccess) return e;
 
   const size_t smem = 1024 + (size_t)C::kStages * C::kStageBytes + 2 * C::kPBytes +
-                      C::kStages * sizeof(Meta) + 32 * 8 + 16;
+                      C::kStages * sizeof(Meta) + 32 * 8 + 16 + 16 + 2 * D * sizeof(float);
   auto kern = mqa_heads_kernel<D, R>;
   const int variant = (D == 512 ? 0 : 3) + R / 32;
   e = ensure_smem_attr(reinterpret_cast<const void*>(kern), 3 + variant, smem);

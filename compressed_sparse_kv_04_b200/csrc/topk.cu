@@ -92,45 +92,20 @@ CSA_DEV void st_remote_v4(uint32_t caddr, uint4 v) {
                : "memory");
 }
 
+// The radix select over the cluster and the index-ordered emission.  The
+// slice is keys[0..len) at row positions lo.. (keys follow the Shared block
+// in dynamic shared memory); the selection goes to out[0..k).
+// (Out of line: the exchange rounds measured faster that way.)
 template <int kBits, bool kAggregate>
-__global__ void __launch_bounds__(kThreads, 1) topk_kernel(const Params p) {
+__device__ __noinline__ void cluster_select(uint8_t* smem_raw, int C, uint32_t r, int k, int len,
+                                            int64_t lo, int32_t* out) {
   constexpr int kBins = 1 << kBits;
   using S = Shared<kBins>;
-  extern __shared__ __align__(16) uint8_t smem_raw[];
   S& sh = *reinterpret_cast<S*>(smem_raw);
-  uint32_t* keys = reinterpret_cast<uint32_t*>(smem_raw + sizeof(S));
-
-  const int row = blockIdx.y;
-  const int C = p.C;
-  const uint32_t r = cluster_ctarank();
+  const uint32_t* keys = reinterpret_cast<const uint32_t*>(smem_raw + sizeof(S));
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  pdl_trigger();
-  const int64_t pos = p.pos_q ? p.pos_q[row] : p.pos_base + row % p.Q;
-  pdl_wait();  // the scores come from the indexer kernel
-  // The slice's scores are loaded before the visible count is known (the
-  // row holds N_cap scores, so every address is in bounds).
-  const int64_t lo = (int64_t)r * p.slice;
-  const int cap = (int)(p.N_cap - lo < p.slice ? (p.N_cap - lo > 0 ? p.N_cap - lo : 0) : p.slice);
-  const float* src = p.scores + (int64_t)row * p.N_cap + lo;
-#pragma unroll 8
-  for (int i = tid; i < cap; i += kThreads) keys[i] = orderable(__ldg(src + i));
-  int64_t n = pos < 0 ? 0 : (pos + 1) / p.m - p.entry_offset;
-  if (n < 0) n = 0;
-  if (n > p.N_cap) {
-    n = p.N_cap;
-    if (r == 0 && tid == 0) report(p.status, CSA_ERR_CAPACITY);
-  }
-  int32_t* out = p.idx + (int64_t)row * p.k;
-  if (n <= p.k) {  // every visible entry is kept (the whole cluster returns)
-    if (r == 0) {
-      for (int j = tid; j < p.k; j += kThreads) out[j] = j < n ? j : -1;
-      if (tid == 0) p.cnt[row] = (int32_t)n;
-    }
-    return;
-  }
   cluster_arrive();  // paired with the wait before the first remote store
 
-  const int len = (int)(n - lo < cap ? (n - lo > 0 ? n - lo : 0) : cap);
   for (int b = tid; b < kBins; b += kThreads) sh.local[0][b] = 0;
   uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
   for (int i = tid; i < len; i += kThreads) {  // the keys this thread wrote
@@ -169,7 +144,7 @@ __global__ void __launch_bounds__(kThreads, 1) topk_kernel(const Params p) {
 
   // Radix rounds below the common prefix.
   uint32_t prefix, mask;
-  uint32_t k_rem = (uint32_t)p.k;
+  uint32_t k_rem = (uint32_t)k;
   if (gmin == gmax) {
     prefix = gmin;
     mask = 0xFFFFFFFFu;
@@ -304,11 +279,50 @@ __global__ void __launch_bounds__(kThreads, 1) topk_kernel(const Params p) {
     const uint32_t eq_rank = eq_run + __popc(be & lt);
     if (gt || (eq && eq_rank < need_eq)) {
       const uint32_t o = gt_run + __popc(bg & lt) + min(need_eq, eq_rank);
-      if (o < (uint32_t)p.k) out[o] = (int32_t)(lo + i);
+      if (o < (uint32_t)k) out[o] = (int32_t)(lo + i);
     }
     gt_run += __popc(bg);
     eq_run += __popc(be);
   }
+}
+
+template <int kBits, bool kAggregate>
+__global__ void __launch_bounds__(kThreads, 1) topk_kernel(const Params p) {
+  constexpr int kBins = 1 << kBits;
+  using S = Shared<kBins>;
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  uint32_t* keys = reinterpret_cast<uint32_t*>(smem_raw + sizeof(S));
+
+  const int row = blockIdx.y;
+  const int C = p.C;
+  const uint32_t r = cluster_ctarank();
+  const int tid = threadIdx.x;
+  pdl_trigger();
+  const int64_t pos = p.pos_q ? p.pos_q[row] : p.pos_base + row % p.Q;
+  const int64_t lo = (int64_t)r * p.slice;
+  pdl_wait();  // the scores come from the indexer kernel
+  // The slice's scores are loaded before the visible count is known (the
+  // row holds N_cap scores, so every address is in bounds).
+  const int cap = (int)(p.N_cap - lo < p.slice ? (p.N_cap - lo > 0 ? p.N_cap - lo : 0) : p.slice);
+  const float* src = p.scores + (int64_t)row * p.N_cap + lo;
+#pragma unroll 8
+  for (int i = tid; i < cap; i += kThreads) keys[i] = orderable(__ldg(src + i));
+  int64_t n = pos < 0 ? 0 : (pos + 1) / p.m - p.entry_offset;
+  if (n < 0) n = 0;
+  if (n > p.N_cap) {
+    n = p.N_cap;
+    if (r == 0 && tid == 0) report(p.status, CSA_ERR_CAPACITY);
+  }
+  int32_t* out = p.idx + (int64_t)row * p.k;
+  if (n <= p.k) {  // every visible entry is kept (the whole cluster returns)
+    if (r == 0) {
+      for (int j = tid; j < p.k; j += kThreads) out[j] = j < n ? j : -1;
+      if (tid == 0) p.cnt[row] = (int32_t)n;
+    }
+    return;
+  }
+  const int len = (int)(n - lo < cap ? (n - lo > 0 ? n - lo : 0) : cap);
+  cluster_select<kBits, kAggregate>(smem_raw, C, r, p.k, len, lo, out);
   if (r == 0 && tid == 0) p.cnt[row] = p.k;
 }
 
