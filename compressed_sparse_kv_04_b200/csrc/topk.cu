@@ -693,7 +693,7 @@ cudaError_t launch_merge_candidates(const MergeLaunch& a, cudaStream_t stream) {
   p.status = a.status;
   const size_t smem = kRowKeysOff + (size_t)a.G * a.k * 8;
   if (smem > 220 * 1024) return cudaErrorInvalidValue;
-  cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(merge_candidates_kernel), 4, smem);
+  cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(merge_candidates_kernel), 9, smem);
   if (e != cudaSuccess) return e;
   return launch_pdl(merge_candidates_kernel, dim3(a.rows), dim3(kThreads), smem, stream, 0,
                     a.chained, p);
@@ -759,7 +759,7 @@ cudaError_t launch_topk(const TopkLaunch& a, cudaStream_t stream) {
     p.cnt = a.cnt;
     p.status = a.status;
     const size_t smem = kRowKeysOff + (size_t)((a.N_cap + 3) / 4 * 4) * 4;
-    cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(topk_row_kernel), 3, smem);
+    cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(topk_row_kernel), 8, smem);
     if (e != cudaSuccess) return e;
     return launch_pdl(topk_row_kernel, dim3(a.rows), dim3(kThreads), smem, stream, 0, a.chained,
                       p);

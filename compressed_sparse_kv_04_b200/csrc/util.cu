@@ -21,10 +21,10 @@ int device_sm_count() {
 }
 
 cudaError_t ensure_smem_attr(const void* func, int slot, size_t bytes) {
-  static size_t done[64][16] = {};
+  static size_t done[64][32] = {};
   static std::mutex mu;
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64 || slot < 0 || slot >= 16)
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64 || slot < 0 || slot >= 32)
     return cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
   std::lock_guard<std::mutex> lock(mu);
   if (done[dev][slot] >= bytes) return cudaSuccess;
