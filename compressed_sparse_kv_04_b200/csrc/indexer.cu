@@ -29,7 +29,6 @@ namespace csa {
 namespace {
 
 constexpr int kTileRows = 128;
-constexpr int kThreads = 192;
 
 template <int DI>
 struct Cfg {
@@ -79,8 +78,12 @@ CSA_DEV int64_t safe_bound(const Params& p, int b) {
   return i < 0 ? 0 : i;
 }
 
-template <int DI>
-__global__ void __launch_bounds__(kThreads, 1)
+// EW epilogue warps: 4 (one per TMEM lane quarter), or 8 when the group
+// holds several queries (two warps per quarter, queries alternating), which
+// halves the epilogue's work per thread where it bounds the kernel
+// (prefill: four queries x 64 heads per entry and tile).
+template <int DI, int EW>
+__global__ void __launch_bounds__(64 + 32 * EW, 1)
     index_score_kernel(const __grid_constant__ CUtensorMap kmap, const Params p) {
   using C = Cfg<DI>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -131,10 +134,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 128);
+      mbar_init(&tempty[a], 32 * EW);
     }
     mbar_init(drain, 1);
-    mbar_init(done, kThreads / 32);
+    mbar_init(done, 2 + EW);
     *abort_flag = 0;
     *consumed = 0;
     fence_mbar_init();
@@ -147,7 +150,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // Query tile (B operand): row g*HP + h holds head h of query q0+g; rows of
   // padding heads / absent queries are zero.  Written with the swizzle the
   // MMA descriptor expects.
-  for (int c = threadIdx.x; c < p.N * (DI / 16); c += kThreads) {
+  for (int c = threadIdx.x; c < p.N * (DI / 16); c += 64 + 32 * EW) {
     int row = c / (DI / 16), chunk = c % (DI / 16);
     int g = row / p.HP, h = row % p.HP;
     uint4 v = make_uint4(0, 0, 0, 0);
@@ -158,7 +161,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t phys = lin ^ (((lin >> 7) & C::kSwzMask) << 4);
     *reinterpret_cast<uint4*>(qtile + phys) = v;
   }
-  for (int r = threadIdx.x; r < p.N; r += kThreads) {
+  for (int r = threadIdx.x; r < p.N; r += 64 + 32 * EW) {
     int g = r / p.HP, h = r % p.HP;
     float v = 0.f;
     if (g < nq && h < p.H_I) {
@@ -235,6 +238,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ epilogue --
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
+    const int wg = (warp - 2) / 4;  // queries wg, wg + EW/4, ... of the group
     // Key scales follow the producer's rule (read through L2: a line may
     // hold scales from both sides of the bound); the scores are a buffer no
     // earlier kernel of the call touches.
@@ -280,7 +284,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = mbar_wait(&tfull[a], aph, p.status, abort_flag);
       if (!__all_sync(0xffffffffu, ok)) break;  // keep the warp converged for tcgen05.ld
       tc_fence_after();
-      for (int g = 0; g < nq; ++g) {
+      for (int g = wg; g < nq; g += EW / 4) {
         // All of this query's head columns (<= 64) in flight, one wait.
         uint32_t v[4][16];
         const uint32_t col = tmem_addr(tmem, quarter * 32, a * p.N + g * p.HP);
@@ -319,7 +323,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int DI>
+template <int DI, int EW>
 cudaError_t launch_impl(const IndexLaunch& a, cudaStream_t stream) {
   using C = Cfg<DI>;
   Params p{};
@@ -350,13 +354,14 @@ cudaError_t launch_impl(const IndexLaunch& a, cudaStream_t stream) {
 
   size_t smem = 1024 + (size_t)C::kStages * C::kStageBytes + (size_t)p.N * DI + 256 * 4 +
                 (2 * C::kStages + 6) * 8 + 16;
-  auto kern = index_score_kernel<DI>;
-  cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kern), DI == 128 ? 0 : 1,
-                                   smem);
+  auto kern = index_score_kernel<DI, EW>;
+  cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kern),
+                                   (DI == 128 ? 0 : 1) + (EW == 8 ? 19 : 0), smem);
   if (e != cudaSuccess) return e;
   // Two CTAs per SM when shared memory allows it (228 KB per SM).
   int occ = (2 * (smem + 1024) <= 228 * 1024) ? 2 : 1;
   if (2 * cols > 512) occ = 1;  // two CTAs would contend for tensor memory
+  if (EW == 8) occ = 1;  // 320 threads x ~130 registers: one CTA per SM
   int64_t groups = (int64_t)a.B * p.qgroups;
   if (groups > 65535) return cudaErrorInvalidConfiguration;
   int64_t slots = (int64_t)a.num_sms * occ;
@@ -370,15 +375,18 @@ cudaError_t launch_impl(const IndexLaunch& a, cudaStream_t stream) {
                    kTileRows, DI, DI == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B);
   if (e != cudaSuccess) return e;
   dim3 grid(chunks, (unsigned)groups);
-  return launch_pdl(kern, grid, dim3(kThreads), smem, stream, 0, a.chained, kmap, p);
+  return launch_pdl(kern, grid, dim3(64 + 32 * EW), smem, stream, 0, a.chained, kmap, p);
 }
 
 }  // namespace
 
 cudaError_t launch_index_scores(const IndexLaunch& a, cudaStream_t stream) {
   if (a.B * (int64_t)a.N_cap > 0x7FFFFFFF) return cudaErrorInvalidValue;
-  if (a.D_I == 128) return launch_impl<128>(a, stream);
-  if (a.D_I == 64) return launch_impl<64>(a, stream);
+  // Groups of several queries (prefill) take eight epilogue warps.
+  const int HP = (a.H_I + 15) / 16 * 16;
+  const bool wide = std::min(std::min(a.Q, 256 / HP), 8) >= 2;
+  if (a.D_I == 128) return wide ? launch_impl<128, 8>(a, stream) : launch_impl<128, 4>(a, stream);
+  if (a.D_I == 64) return wide ? launch_impl<64, 8>(a, stream) : launch_impl<64, 4>(a, stream);
   return cudaErrorInvalidValue;
 }
 

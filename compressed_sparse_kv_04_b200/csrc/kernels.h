@@ -218,7 +218,7 @@ csa_status set_error(csa_status s, const char* fmt, ...);
 // Sets the dynamic shared-memory limit of `func` once per device (the call
 // is then skipped, which keeps launches legal inside CUDA-graph capture).
 // `slot` (0..31) identifies the kernel: each kernel instance has its own
-// (indexer 0-1, top-k 2 and 8-9, attention 3-7, projection 10-14).
+// (indexer 0-1 and 19-20, top-k 2 and 8-9, attention 3-7, projection 10-14).
 cudaError_t ensure_smem_attr(const void* func, int slot, size_t bytes);
 
 }  // namespace csa
