@@ -365,6 +365,16 @@ CSA_DEV void st_cluster_v4(uint32_t caddr, float a, float b, float c, float d) {
 }
 
 // ------------------------------------------------------------ small helpers --
+// d = a * b + c on both lanes of a pair (two fp32 FMAs, each rounded once).
+CSA_DEV float2 fma_f32x2(float2 a, float2 b, float2 c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;"
+      : "=l"(d)
+      : "l"(*reinterpret_cast<const uint64_t*>(&a)), "l"(*reinterpret_cast<const uint64_t*>(&b)),
+        "l"(*reinterpret_cast<const uint64_t*>(&c)));
+  return *reinterpret_cast<const float2*>(&d);
+}
+
 CSA_DEV float warp_sum(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);

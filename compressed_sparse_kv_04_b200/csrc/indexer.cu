@@ -78,12 +78,12 @@ CSA_DEV int64_t safe_bound(const Params& p, int b) {
   return i < 0 ? 0 : i;
 }
 
-// EW epilogue warps: 4 (one per TMEM lane quarter), or 8 when the group
-// holds several queries (two warps per quarter, queries alternating), which
-// halves the epilogue's work per thread where it bounds the kernel
-// (prefill: four queries x 64 heads per entry and tile).
+// EW epilogue warps: 4 (one per TMEM lane quarter; two CTAs per SM), or 8
+// when the group holds several queries (two warps per quarter, queries
+// alternating), which halves the epilogue's work per thread where it bounds
+// the kernel (prefill: four queries x 64 heads per entry and tile).
 template <int DI, int EW>
-__global__ void __launch_bounds__(64 + 32 * EW, 1)
+__global__ void __launch_bounds__(64 + 32 * EW, EW == 4 ? 2 : 1)
     index_score_kernel(const __grid_constant__ CUtensorMap kmap, const Params p) {
   using C = Cfg<DI>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -285,6 +285,30 @@ __global__ void __launch_bounds__(64 + 32 * EW, 1)
       if (!__all_sync(0xffffffffu, ok)) break;  // keep the warp converged for tcgen05.ld
       tc_fence_after();
       for (int g = wg; g < nq; g += EW / 4) {
+        if (p.HP == 64) {
+          // 64 head columns in two loads; the weighted sum in packed fp32
+          // FMAs (lane pairs = chains j & 3 of the generic path below, in
+          // the same order: the same number).
+          const uint32_t col = tmem_addr(tmem, quarter * 32, a * p.N + g * 64);
+          const float2* wg2 = reinterpret_cast<const float2*>(wq + g * 64);
+          float2 acc2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+#pragma unroll
+          for (int h0 = 0; h0 < 64; h0 += 32) {
+            uint32_t v[32];
+            tmem_ld32(col + h0, v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 32; j += 2)
+              acc2[(j >> 1) & 1] = fma_f32x2(wg2[(h0 + j) >> 1],
+                                             make_float2(fmaxf(__uint_as_float(v[j]), 0.f),
+                                                         fmaxf(__uint_as_float(v[j + 1]), 0.f)),
+                                             acc2[(j >> 1) & 1]);
+          }
+          const float acc = (acc2[0].x + acc2[0].y) + (acc2[1].x + acc2[1].y);
+          if (entry < nv[g < 8 ? g : 7])
+            p.scores[((int64_t)b * p.Q + q0 + g) * p.N_cap + entry] = acc * ks;
+          continue;
+        }
         // All of this query's head columns (<= 64) in flight, one wait.
         uint32_t v[4][16];
         const uint32_t col = tmem_addr(tmem, quarter * 32, a * p.N + g * p.HP);
