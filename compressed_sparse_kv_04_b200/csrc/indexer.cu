@@ -290,7 +290,7 @@ __global__ void __launch_bounds__(64 + 32 * EW, EW == 4 ? 2 : 1)
           // FMAs (lane pairs = chains j & 3 of the generic path below, in
           // the same order: the same number).
           const uint32_t col = tmem_addr(tmem, quarter * 32, a * p.N + g * 64);
-          const float2* wg2 = reinterpret_cast<const float2*>(wq + g * 64);
+          const float4* wg4 = reinterpret_cast<const float4*>(wq + g * 64);
           float2 acc2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
           for (int h0 = 0; h0 < 64; h0 += 32) {
@@ -298,11 +298,17 @@ __global__ void __launch_bounds__(64 + 32 * EW, EW == 4 ? 2 : 1)
             tmem_ld32(col + h0, v);
             tmem_wait_ld();
 #pragma unroll
-            for (int j = 0; j < 32; j += 2)
-              acc2[(j >> 1) & 1] = fma_f32x2(wg2[(h0 + j) >> 1],
-                                             make_float2(fmaxf(__uint_as_float(v[j]), 0.f),
-                                                         fmaxf(__uint_as_float(v[j + 1]), 0.f)),
-                                             acc2[(j >> 1) & 1]);
+            for (int j = 0; j < 32; j += 4) {
+              const float4 w4 = wg4[(h0 + j) >> 2];
+              acc2[0] = fma_f32x2(make_float2(w4.x, w4.y),
+                                  make_float2(fmaxf(__uint_as_float(v[j]), 0.f),
+                                              fmaxf(__uint_as_float(v[j + 1]), 0.f)),
+                                  acc2[0]);
+              acc2[1] = fma_f32x2(make_float2(w4.z, w4.w),
+                                  make_float2(fmaxf(__uint_as_float(v[j + 2]), 0.f),
+                                              fmaxf(__uint_as_float(v[j + 3]), 0.f)),
+                                  acc2[1]);
+            }
           }
           const float acc = (acc2[0].x + acc2[0].y) + (acc2[1].x + acc2[1].y);
           if (entry < nv[g < 8 ? g : 7])
