@@ -186,7 +186,8 @@ def test_indexer_topk_tiny_end_to_end(orc):
         assert abs(ref[0, 0, i] - kth) <= 1e-6 * abs(kth) or flipped[i], i
 
 
-@pytest.mark.parametrize("H_I,D_I,Q", [(64, 128, 37), (4, 64, 5), (64, 64, 1), (7, 128, 9)])
+@pytest.mark.parametrize("H_I,D_I,Q", [(64, 128, 37), (4, 64, 5), (64, 64, 1), (7, 128, 9),
+                                        (64, 128, 2), (64, 128, 3)])
 def test_indexer_causal_multi_query(orc, H_I, D_I, Q):
     w = configs.scaled(configs.CSA_128K, B=2, H_I=H_I, D_I=D_I, k=100)
     N_cap = 2048 + 13 if D_I == 128 else 2048 + 14
