@@ -163,7 +163,9 @@ def workspace_bytes(p, op, Q, N_cap):
 
 
 def workspace(p, op, Q, N_cap, device=None):
-    return torch.empty(workspace_bytes(p, op, Q, N_cap), dtype=torch.uint8,
+    """A zero-filled workspace (the decode step's score histogram starts
+    cleared; each call leaves it so)."""
+    return torch.zeros(workspace_bytes(p, op, Q, N_cap), dtype=torch.uint8,
                        device=device or torch.cuda.current_device())
 
 

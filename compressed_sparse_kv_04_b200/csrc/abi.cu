@@ -98,6 +98,12 @@ size_t scores_bytes(int64_t rows, int64_t N_cap) {
   return round_up((size_t)rows * (size_t)N_cap * sizeof(float), 256);
 }
 
+// The decode step's score histogram ([B, kScoreHistBins] u32, left zeroed by
+// each call) and the top-k path word per sequence, after the scores.
+size_t hist_bytes(int64_t B) {
+  return (size_t)B * csa::kScoreHistBins * sizeof(uint32_t) + round_up((size_t)B * 4, 256);
+}
+
 void fill_inv_freq(const csa_params* p, double* out) {
   int half = p->rope_dim / 2;
   for (int j = 0; j < 64; ++j) out[j] = 0.0;
@@ -196,7 +202,7 @@ size_t csa_workspace_bytes(const csa_params* p, csa_op op, int Q, int64_t N_cap)
              512;
     }
     case CSA_OP_CSA_DECODE_STEP:
-      return scores_bytes(p->B, N_cap) +
+      return scores_bytes(p->B, N_cap) + hist_bytes(p->B) +
              csa::mqa_workspace_bytes(p->B, splits_for(p, CSA_OP_SPARSE_MQA, p->B, N_cap), p->H,
                                       p->d) +
              512;
@@ -318,9 +324,10 @@ static csa_status index_common(const char* fn, const csa_params* p, int Q,
                                const int64_t* pos_q, int64_t pos_base, float* scores,
                                int32_t* dev_status, cudaStream_t stream, int chained,
                                const int64_t* safe_pos = nullptr,
-                               int64_t safe_fixed = INT64_MAX) {
+                               int64_t safe_fixed = INT64_MAX, uint32_t* hist = nullptr) {
   csa::IndexLaunch a{};
   a.chained = chained;
+  a.hist = hist;
   a.safe_pos = safe_pos;
   a.safe_fixed = safe_fixed;
   a.B = p->B;
@@ -348,9 +355,12 @@ static csa_status index_common(const char* fn, const csa_params* p, int Q,
 static csa_status topk_common(const char* fn, const csa_params* p, int Q, const float* scores,
                               int64_t N_cap, const int64_t* pos_q, int64_t pos_base,
                               int32_t* topk_idx, int32_t* topk_cnt, int32_t* dev_status,
-                              cudaStream_t stream, int chained) {
+                              cudaStream_t stream, int chained, uint32_t* hist = nullptr,
+                              int32_t* path = nullptr) {
   csa::TopkLaunch t{};
   t.chained = chained;
+  t.hist = hist;
+  t.path = path;
   t.rows = p->B * Q;
   t.Q = Q;
   t.m = p->m;
@@ -375,13 +385,14 @@ static csa_status index_topk_common(const char* fn, const csa_params* p, int Q,
                                     int32_t* topk_idx, int32_t* topk_cnt, float* scores,
                                     int32_t* dev_status, cudaStream_t stream, int chained,
                                     const int64_t* safe_pos = nullptr,
-                                    int64_t safe_fixed = INT64_MAX) {
+                                    int64_t safe_fixed = INT64_MAX, uint32_t* hist = nullptr,
+                                    int32_t* path = nullptr) {
   csa_status st = index_common(fn, p, Q, q_idx, q_scale, w, idx_key, idx_scale, N_cap, pos_q,
                                pos_base, scores, dev_status, stream, chained, safe_pos,
-                               safe_fixed);
+                               safe_fixed, hist);
   if (st != CSA_OK) return st;
   return topk_common(fn, p, Q, scores, N_cap, pos_q, pos_base, topk_idx, topk_cnt, dev_status,
-                     stream, 1);
+                     stream, 1, hist, path);
 }
 
 static csa_status check_index_args(const char* fn, const csa_params* p, int Q, int64_t N_cap) {
@@ -682,17 +693,25 @@ csa_status csa_decode_step(const csa_params* p, const int64_t* pos_q, const void
                        idx_tok, w_s_idx, b_pos_idx, idx_key, idx_scale, dev_status, stream, pos_q,
                        1);
   if (st != CSA_OK) return st;
-  // 2-3. Indexer and top-k over each sequence's visible entries.
+  // 2-3. Indexer and top-k over each sequence's visible entries.  Where the
+  // top-k spreads a row over a cluster, the indexer also counts the scores
+  // by their top key bits, which seeds the selection.
   float* scores = static_cast<float*>(ws);
+  char* hist_at = static_cast<char*>(ws) + scores_bytes(p->B, N_cap);
+  uint32_t* hist = csa::topk_uses_hist(p->B, N_cap) ? reinterpret_cast<uint32_t*>(hist_at) : nullptr;
+  int32_t* path = hist ? reinterpret_cast<int32_t*>(hist + (size_t)p->B * csa::kScoreHistBins)
+                       : nullptr;
   // Only each sequence's newest block is written by this call.
   st = index_topk_common(fn, p, 1, q_idx, q_scale, w, idx_key, idx_scale, N_cap, pos_q, 0,
-                         topk_idx, topk_cnt, scores, dev_status, s, 1, pos_q);
+                         topk_idx, topk_cnt, scores, dev_status, s, 1, pos_q, INT64_MAX, hist,
+                         path);
   if (st != CSA_OK) return st;
   // 4. Sparse MQA over the selection, the window and the sink.
-  char* rest = static_cast<char*>(ws) + scores_bytes(p->B, N_cap);
+  const size_t head = scores_bytes(p->B, N_cap) + hist_bytes(p->B);
+  char* rest = static_cast<char*>(ws) + head;
   return mqa_common(fn, p, CSA_OP_SPARSE_MQA, p->B, 1, q, pos_q, 0, kv_c, N_cap, topk_idx,
                     topk_cnt, kv_tok, L_cap, sink, gamma_q, gamma_kv, out, lse, rest,
-                    ws_bytes - scores_bytes(p->B, N_cap), dev_status, s, 1);
+                    ws_bytes - head, dev_status, s, 1);
 }
 
 csa_status hca_decode_step(const csa_params* p, const int64_t* pos_q, const void* kv_tok,

@@ -365,6 +365,16 @@ CSA_DEV void st_cluster_v4(uint32_t caddr, float a, float b, float c, float d) {
 }
 
 // ------------------------------------------------------------ small helpers --
+// Order-preserving 32-bit key of an indexer score (a larger score has a
+// larger key; NaN below every number; -0 == +0).  The indexer's score
+// histogram bins and the top-k's radix digits are bits of this key.
+CSA_DEV uint32_t score_key(float s) {
+  if (isnan(s)) return 0u;
+  uint32_t u = __float_as_uint(s);
+  if ((u & 0x7FFFFFFFu) == 0u) u = 0u;
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
 // d = a * b + c on both lanes of a pair (two fp32 FMAs, each rounded once).
 CSA_DEV float2 fma_f32x2(float2 a, float2 b, float2 c) {
   uint64_t d;

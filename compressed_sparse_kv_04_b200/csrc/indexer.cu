@@ -30,10 +30,12 @@ namespace {
 
 constexpr int kTileRows = 128;
 
-template <int DI>
+// kHist: the histogram's 16 KB of shared memory come out of the key ring
+// (five stages instead of six at D_I = 128), which keeps two CTAs per SM.
+template <int DI, bool kHist = false>
 struct Cfg {
   static constexpr int kStageBytes = kTileRows * DI;
-  static constexpr int kStages = DI == 128 ? 6 : 8;
+  static constexpr int kStages = DI == 128 ? (kHist ? 5 : 6) : 8;
   static constexpr uint32_t kSBO = 8 * DI;               // 8 rows per swizzle atom
   static constexpr uint32_t kSwzMask = DI == 128 ? 7 : 3;  // 128B / 64B swizzle
   static constexpr uint64_t kLayout = DI == 128 ? 2 : 4;   // descriptor layout type
@@ -58,6 +60,7 @@ struct Params {
   const int64_t* pos_q;
   int64_t pos_base;
   float* scores;
+  uint32_t* hist;  // [B, kScoreHistBins] (kHist launches)
   int32_t* status;
   uint32_t tmem_cols;
 };
@@ -82,10 +85,15 @@ CSA_DEV int64_t safe_bound(const Params& p, int b) {
 // when the group holds several queries (two warps per quarter, queries
 // alternating), which halves the epilogue's work per thread where it bounds
 // the kernel (prefill: four queries x 64 heads per entry and tile).
-template <int DI, int EW>
+// kHist (one query per sequence): the epilogue also counts each visible
+// score by the top kScoreHistBits bits of its key in a shared-memory
+// histogram, added to the sequence's global histogram when the CTA is done
+// (only the non-zero bins), so that the top-k that follows knows which bin
+// holds its threshold before it reads a score.
+template <int DI, int EW, bool kHist>
 __global__ void __launch_bounds__(64 + 32 * EW, EW == 4 ? 2 : 1)
     index_score_kernel(const __grid_constant__ CUtensorMap kmap, const Params p) {
-  using C = Cfg<DI>;
+  using C = Cfg<DI, kHist>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -101,7 +109,11 @@ __global__ void __launch_bounds__(64 + 32 * EW, EW == 4 ? 2 : 1)
   uint64_t* done = drain + 1;  // one arrival per warp when its role is over
   uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_slot + 1);
-  int* consumed = const_cast<int*>(abort_flag + 1);
+  // kHist: the lowest and highest bin any score of the CTA fell in, then
+  // the histogram on the next 16-byte boundary.
+  uint32_t* hrange = reinterpret_cast<uint32_t*>(const_cast<int*>(abort_flag + 1));
+  uint32_t* shist = reinterpret_cast<uint32_t*>(
+      (reinterpret_cast<uintptr_t>(hrange + 2) + 15) & ~uintptr_t(15));
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   pdl_trigger();
@@ -139,7 +151,8 @@ __global__ void __launch_bounds__(64 + 32 * EW, EW == 4 ? 2 : 1)
     mbar_init(drain, 1);
     mbar_init(done, 2 + EW);
     *abort_flag = 0;
-    *consumed = 0;
+    hrange[0] = kScoreHistBins;
+    hrange[1] = 0u;
     fence_mbar_init();
   }
   __syncwarp();
@@ -170,6 +183,8 @@ __global__ void __launch_bounds__(64 + 32 * EW, EW == 4 ? 2 : 1)
     }
     wq[r] = v;
   }
+  if (kHist)
+    for (int i = threadIdx.x; i < kScoreHistBins; i += 64 + 32 * EW) shist[i] = 0u;
   fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
@@ -263,23 +278,36 @@ __global__ void __launch_bounds__(64 + 32 * EW, EW == 4 ? 2 : 1)
       }
       nv[g] = v;
     }
-    // Key scales are loaded a tile ahead so that their latency hides behind
-    // the previous tile's work.
+    // Key scales of the next kKsAhead tiles are in flight (a register queue):
+    // a tile's own work is far shorter than a load's latency, so one tile
+    // ahead would leave the loop waiting on every load.  Tiles past the safe
+    // bound load theirs on use, after the wait.
+    constexpr int kKsAhead = 8;
+    auto tile_safe = [&](int t) { return (int64_t)(t + 1) * kTileRows <= safe; };
     auto load_ks = [&](int t) -> float {
       const int64_t e = (int64_t)t * kTileRows + row;
       return e < p.N_cap ? __ldcg(p.key_scale + (int64_t)b * p.N_cap + e) : 0.f;
     };
-    ensure(t_begin);
-    float ks_next = load_ks(t_begin);
+    uint32_t hlo = kScoreHistBins, hhi = 0;  // kHist: this thread's bins
+    float ksq[kKsAhead];
+#pragma unroll
+    for (int j = 0; j < kKsAhead; ++j)
+      ksq[j] = (t_begin + j < t_end && tile_safe(t_begin + j)) ? load_ks(t_begin + j) : 0.f;
     int it = 0;
     for (int t = t_begin; t < t_end; ++t, ++it) {
       const int a = it & 1;
       const uint32_t aph = (it >> 1) & 1;
       const int64_t entry = (int64_t)t * kTileRows + row;
-      const float ks = ks_next;
-      if (t + 1 < t_end) {
-        ensure(t + 1);
-        ks_next = load_ks(t + 1);
+      float ks = ksq[0];
+#pragma unroll
+      for (int j = 0; j + 1 < kKsAhead; ++j) ksq[j] = ksq[j + 1];
+      {
+        const int tn = t + kKsAhead;
+        ksq[kKsAhead - 1] = (tn < t_end && tile_safe(tn)) ? load_ks(tn) : 0.f;
+      }
+      if (!tile_safe(t)) {
+        ensure(t);
+        ks = load_ks(t);
       }
       bool ok = mbar_wait(&tfull[a], aph, p.status, abort_flag);
       if (!__all_sync(0xffffffffu, ok)) break;  // keep the warp converged for tcgen05.ld
@@ -311,8 +339,16 @@ __global__ void __launch_bounds__(64 + 32 * EW, EW == 4 ? 2 : 1)
             }
           }
           const float acc = (acc2[0].x + acc2[0].y) + (acc2[1].x + acc2[1].y);
-          if (entry < nv[g < 8 ? g : 7])
-            p.scores[((int64_t)b * p.Q + q0 + g) * p.N_cap + entry] = acc * ks;
+          if (entry < nv[g < 8 ? g : 7]) {
+            const float sc = acc * ks;
+            p.scores[((int64_t)b * p.Q + q0 + g) * p.N_cap + entry] = sc;
+            if (kHist) {
+              const uint32_t bin = score_key(sc) >> (32 - kScoreHistBits);
+              atomicAdd(&shist[bin], 1u);
+              hlo = min(hlo, bin);
+              hhi = max(hhi, bin);
+            }
+          }
           continue;
         }
         // All of this query's head columns (<= 64) in flight, one wait.
@@ -332,13 +368,39 @@ __global__ void __launch_bounds__(64 + 32 * EW, EW == 4 ? 2 : 1)
               a4[j & 3] = fmaf(wg[c * 16 + j], fmaxf(__uint_as_float(v[c][j]), 0.f), a4[j & 3]);
           }
         const float acc = (a4[0] + a4[1]) + (a4[2] + a4[3]);
-        if (entry < nv[g < 8 ? g : 7])
-          p.scores[((int64_t)b * p.Q + q0 + g) * p.N_cap + entry] = acc * ks;
+        if (entry < nv[g < 8 ? g : 7]) {
+          const float sc = acc * ks;
+          p.scores[((int64_t)b * p.Q + q0 + g) * p.N_cap + entry] = sc;
+          if (kHist) {
+            const uint32_t bin = score_key(sc) >> (32 - kScoreHistBits);
+            atomicAdd(&shist[bin], 1u);
+            hlo = min(hlo, bin);
+            hhi = max(hhi, bin);
+          }
+        }
       }
       tc_fence_before();
       mbar_arrive(&tempty[a]);
     }
     if (!waited) pdl_wait();  // this grid completes only after its predecessor
+    if (kHist) {
+      // Every epilogue warp has counted its last score: add the non-zero
+      // bins (within the range the CTA's scores fell in) to the sequence's
+      // histogram.
+      hlo = __reduce_min_sync(0xffffffffu, hlo);
+      hhi = __reduce_max_sync(0xffffffffu, hhi);
+      if (lane == 0) {
+        atomicMin(&hrange[0], hlo);
+        atomicMax(&hrange[1], hhi);
+      }
+      named_barrier_sync(1, 32 * EW);
+      uint32_t* gh = p.hist + (int64_t)b * kScoreHistBins;
+      const int lo = (int)hrange[0], hi = (int)hrange[1];
+      for (int i = lo + threadIdx.x - 64; i <= hi; i += 32 * EW) {
+        const uint32_t v = shist[i];
+        if (v) atomicAdd(gh + i, v);
+      }
+    }
   }
   // Teardown: every warp reports (converged) that it is done with tensor
   // memory; warp 0 frees it after all of them (bounded wait).
@@ -353,9 +415,9 @@ __global__ void __launch_bounds__(64 + 32 * EW, EW == 4 ? 2 : 1)
   }
 }
 
-template <int DI, int EW>
+template <int DI, int EW, bool kHist>
 cudaError_t launch_impl(const IndexLaunch& a, cudaStream_t stream) {
-  using C = Cfg<DI>;
+  using C = Cfg<DI, kHist>;
   Params p{};
   p.B = a.B;
   p.Q = a.Q;
@@ -377,6 +439,7 @@ cudaError_t launch_impl(const IndexLaunch& a, cudaStream_t stream) {
   p.pos_q = a.pos_q;
   p.pos_base = a.pos_base;
   p.scores = a.scores;
+  p.hist = a.hist;
   p.status = a.status;
   uint32_t cols = 32;
   while (cols < (uint32_t)(2 * p.N)) cols <<= 1;
@@ -384,9 +447,11 @@ cudaError_t launch_impl(const IndexLaunch& a, cudaStream_t stream) {
 
   size_t smem = 1024 + (size_t)C::kStages * C::kStageBytes + (size_t)p.N * DI + 256 * 4 +
                 (2 * C::kStages + 6) * 8 + 16;
-  auto kern = index_score_kernel<DI, EW>;
+  if (kHist) smem += 16 + kScoreHistBins * 4;  // range words + histogram
+  auto kern = index_score_kernel<DI, EW, kHist>;
   cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kern),
-                                   (DI == 128 ? 0 : 1) + (EW == 8 ? 19 : 0), smem);
+                                   (DI == 128 ? 0 : 1) + (EW == 8 ? 19 : 0) + (kHist ? 15 : 0),
+                                   smem);
   if (e != cudaSuccess) return e;
   // Two CTAs per SM when shared memory allows it (228 KB per SM).
   int occ = (2 * (smem + 1024) <= 228 * 1024) ? 2 : 1;
@@ -415,8 +480,16 @@ cudaError_t launch_index_scores(const IndexLaunch& a, cudaStream_t stream) {
   // Groups of several queries (prefill) take eight epilogue warps.
   const int HP = (a.H_I + 15) / 16 * 16;
   const bool wide = std::min(std::min(a.Q, 256 / HP), 8) >= 2;
-  if (a.D_I == 128) return wide ? launch_impl<128, 8>(a, stream) : launch_impl<128, 4>(a, stream);
-  if (a.D_I == 64) return wide ? launch_impl<64, 8>(a, stream) : launch_impl<64, 4>(a, stream);
+  if (a.hist) {  // one query per sequence
+    if (a.Q != 1) return cudaErrorInvalidValue;
+    if (a.D_I == 128) return launch_impl<128, 4, true>(a, stream);
+    if (a.D_I == 64) return launch_impl<64, 4, true>(a, stream);
+    return cudaErrorInvalidValue;
+  }
+  if (a.D_I == 128)
+    return wide ? launch_impl<128, 8, false>(a, stream) : launch_impl<128, 4, false>(a, stream);
+  if (a.D_I == 64)
+    return wide ? launch_impl<64, 8, false>(a, stream) : launch_impl<64, 4, false>(a, stream);
   return cudaErrorInvalidValue;
 }
 

@@ -60,8 +60,16 @@ struct IndexLaunch {
   const int64_t* safe_pos;
   int64_t safe_fixed;
   int chained;              // see launch_pdl
+  // One query per sequence only (Q == 1): adds, per sequence, the count of
+  // its visible scores by the top kScoreHistBits bits of their keys
+  // (score_key) to hist[b * kScoreHistBins ..].  Null: no histogram.
+  uint32_t* hist = nullptr;
 };
 cudaError_t launch_index_scores(const IndexLaunch& a, cudaStream_t stream);
+
+// Score histogram of the decode chain: bins of the top 12 key bits.
+constexpr int kScoreHistBits = 12;
+constexpr int kScoreHistBins = 1 << kScoreHistBits;
 
 // Exact top-k over fp32 scores, one cluster of CTAs per query row.
 struct TopkLaunch {
@@ -77,8 +85,17 @@ struct TopkLaunch {
   int32_t* status;
   int64_t entry_offset;     // score j is entry entry_offset + j of the sequence
   int chained;              // see launch_pdl
+  // [rows, kScoreHistBins] histogram of each row's visible scores, written
+  // by the indexer kernel (IndexLaunch::hist), or null.  Used as a guess of
+  // the threshold bin; the selection is exact whatever it holds.  Every bin
+  // is zero when the kernel ends.
+  uint32_t* hist = nullptr;
+  int32_t* path = nullptr;  // [rows] or null: 0 all kept, 1 histogram, 2 radix rounds
 };
 cudaError_t launch_topk(const TopkLaunch& a, cudaStream_t stream);
+// True when launch_topk takes the histogram path for these rows (one
+// cluster of CTAs per row): only then should the indexer build one.
+bool topk_uses_hist(int rows, int64_t N_cap);
 
 // Context split over ranks: a shard's candidates (score, sequence index) and
 // the global top-k over all ranks' candidates.
@@ -218,7 +235,7 @@ csa_status set_error(csa_status s, const char* fmt, ...);
 // Sets the dynamic shared-memory limit of `func` once per device (the call
 // is then skipped, which keeps launches legal inside CUDA-graph capture).
 // `slot` (0..31) identifies the kernel: each kernel instance has its own
-// (indexer 0-1 and 19-20, top-k 2 and 8-9, attention 3-7, projection 10-14).
+// (indexer 0-1, 15-16 and 19-20, top-k 2, 8-9 and 17, attention 3-7, projection 10-14).
 cudaError_t ensure_smem_attr(const void* func, int slot, size_t bytes);
 
 }  // namespace csa

@@ -49,14 +49,12 @@ struct Params {
   int32_t* idx;
   int32_t* cnt;
   int32_t* status;
+  uint32_t* hist;     // topk_hist_kernel: [rows, kScoreHistBins]
+  int32_t* path;      // [rows] or null
+  uint32_t hist_off;  // topk_hist_kernel: byte offset of HistShared
 };
 
-CSA_DEV uint32_t orderable(float s) {
-  if (isnan(s)) return 0u;
-  uint32_t u = __float_as_uint(s);
-  if ((u & 0x7FFFFFFFu) == 0u) u = 0u;  // -0 == +0
-  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
+CSA_DEV uint32_t orderable(float s) { return score_key(s); }
 
 template <int kBins>
 struct Shared {
@@ -373,91 +371,76 @@ CSA_DEV uint32_t block_excl_scan(uint32_t v, uint32_t* warp_tot) {
   return warp_tot[warp] + incl - v;
 }
 
-// Selects the k largest of keys[0..n) (n > k; order-preserving keys in
-// shared memory, written by this CTA) under (key descending, position
-// ascending) and calls emit(o, i) once for each output slot o < k with the
-// selected position i, slots in ascending order of i.  kmin / kmax: this
-// thread's min and max over the keys it wrote.  All 1024 threads call it.
-template <typename Emit>
-CSA_DEV void row_select(const uint32_t* keys, int n, int k, RowShared& sh, uint32_t kmin,
-                        uint32_t kmax, Emit emit) {
-  constexpr int kBins = 1 << kRowBits;
+// Radix rounds over keys[0..n): the keys whose bits under `mask` equal
+// `prefix` take part, and the digits start at bit `shift`, kRowBits per
+// round, until the threshold digit's bin is taken whole.  sh.hist must be
+// zero on entry (it is zero again on return).  On return prefix / mask are
+// the threshold key T and the mask M of its decided bits; the selection is
+// every key above T (under M) and the first need_eq keys equal to it, where
+// need_eq is the return value and k_rem the number of keys still to choose
+// among those taking part.  All 1024 threads call it.
+template <int kBits = kRowBits>
+CSA_DEV uint32_t row_rounds(const uint32_t* keys, int n, uint32_t k_rem, RowShared& sh,
+                            uint32_t& prefix, uint32_t& mask, int shift) {
+  static_assert(kBits >= 10 && kBits <= kRowBits, "1 to 4 bins per thread");
+  constexpr int kBins = 1 << kBits;
   constexpr int kPer = kBins / kThreads;  // bins per thread in the digit scan
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
-    kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
-  }
-  if (lane == 0) {
-    sh.warp_a[warp] = kmin;
-    sh.warp_b[warp] = kmax;
-  }
-  for (int b = tid; b < kBins; b += kThreads) sh.hist[b] = 0;
-  cta_sync();
-  uint32_t gmin = sh.warp_a[lane], gmax = sh.warp_b[lane];
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    gmin = min(gmin, __shfl_xor_sync(0xffffffffu, gmin, o));
-    gmax = max(gmax, __shfl_xor_sync(0xffffffffu, gmax, o));
-  }
-  cta_sync();  // every warp has read the min / max slots
-
-  uint32_t prefix, mask;
-  uint32_t k_rem = (uint32_t)k;
-  if (gmin == gmax) {
-    prefix = gmin;
-    mask = 0xFFFFFFFFu;
-  } else {
-    const int top = 31 - __clz(gmin ^ gmax);
-    mask = top == 31 ? 0u : (0xFFFFFFFFu << (top + 1));
-    prefix = gmin & mask;
-    int shift = top + 1;
-    while (shift > 0) {
-      const int width = shift >= kRowBits ? kRowBits : shift;
-      shift -= width;
-      const uint32_t dmask = (1u << width) - 1u;
+  const int tid = threadIdx.x;
+  while (shift > 0) {
+    const int width = shift >= kBits ? kBits : shift;
+    shift -= width;
+    const uint32_t dmask = (1u << width) - 1u;
 #pragma unroll 4
-      for (int i = tid; i < n; i += kThreads) {
-        const uint32_t key = keys[i];
-        if ((key & mask) == prefix) atomicAdd(&sh.hist[(key >> shift) & dmask], 1u);
-      }
-      cta_sync();
-      // Thread t owns digits nb-1-t*kPer down to nb-(t+1)*kPer (descending),
-      // so an exclusive scan over t counts the keys in higher digits.
-      const int nb = (int)dmask + 1;
-      uint32_t c[kPer];
-      uint32_t local = 0;
-#pragma unroll
-      for (int j = 0; j < kPer; ++j) {
-        const int d = nb - 1 - (tid * kPer + j);
-        c[j] = d >= 0 ? sh.hist[d] : 0u;
-        local += c[j];
-      }
-      uint32_t above = block_excl_scan(local, sh.scan);
-#pragma unroll
-      for (int j = 0; j < kPer; ++j) {
-        const int d = nb - 1 - (tid * kPer + j);
-        if (d >= 0 && above < k_rem && above + c[j] >= k_rem) {
-          sh.bcast[0] = (uint32_t)d;
-          sh.bcast[1] = above;
-          sh.bcast[2] = c[j];
-        }
-        above += c[j];
-      }
-      for (int b = tid; b < kBins; b += kThreads) sh.hist[b] = 0;
-      cta_sync();
-      const uint32_t d = sh.bcast[0], abv = sh.bcast[1], cnt_d = sh.bcast[2];
-      cta_sync();  // bcast is read before the next round can rewrite it
-      k_rem -= abv;
-      prefix |= d << shift;
-      mask |= dmask << shift;
-      if (cnt_d == k_rem) break;  // the whole bin is taken
+    for (int i = tid; i < n; i += kThreads) {
+      const uint32_t key = keys[i];
+      if ((key & mask) == prefix) atomicAdd(&sh.hist[(key >> shift) & dmask], 1u);
     }
+    cta_sync();
+    // Thread t owns digits nb-1-t*kPer down to nb-(t+1)*kPer (descending),
+    // so an exclusive scan over t counts the keys in higher digits.
+    const int nb = (int)dmask + 1;
+    uint32_t c[kPer];
+    uint32_t local = 0;
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+      const int d = nb - 1 - (tid * kPer + j);
+      c[j] = d >= 0 ? sh.hist[d] : 0u;
+      local += c[j];
+    }
+    uint32_t above = block_excl_scan(local, sh.scan);
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+      const int d = nb - 1 - (tid * kPer + j);
+      if (d >= 0 && above < k_rem && above + c[j] >= k_rem) {
+        sh.bcast[0] = (uint32_t)d;
+        sh.bcast[1] = above;
+        sh.bcast[2] = c[j];
+      }
+      above += c[j];
+    }
+    for (int b = tid; b < kBins; b += kThreads) sh.hist[b] = 0;
+    cta_sync();
+    const uint32_t d = sh.bcast[0], abv = sh.bcast[1], cnt_d = sh.bcast[2];
+    cta_sync();  // bcast is read before the next round can rewrite it
+    k_rem -= abv;
+    prefix |= d << shift;
+    mask |= dmask << shift;
+    if (cnt_d == k_rem) break;  // the whole bin is taken
   }
-  const uint32_t T = prefix, M = mask, need_eq = k_rem;
+  return k_rem;
+}
 
-  // Index-ordered output: warp w owns positions [w*chunk, (w+1)*chunk).
+// Index-ordered output of a selection (threshold T under mask M, need_eq
+// equal keys): calls emit(o, i) for each selected position i of keys[0..n)
+// with its output slot o < k, given gt_base / eq_base keys above / equal to
+// T that precede keys[0] in index order.  Warp w owns positions
+// [w*chunk, (w+1)*chunk) (chunk a multiple of 32); lane l takes element
+// j*32 + l of the chunk, so a ballot ranks it.  All 1024 threads call it.
+template <typename Emit>
+CSA_DEV void ordered_emit(const uint32_t* keys, int n, int k, uint32_t T, uint32_t M,
+                          uint32_t need_eq, uint32_t gt_base, uint32_t eq_base, RowShared& sh,
+                          Emit emit) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int chunk = (((n + 31) / 32) + 31) & ~31;
   const int w0 = min(n, warp * chunk), w1 = min(n, w0 + chunk);
   uint32_t n_gt = 0, n_eq = 0;
@@ -492,7 +475,7 @@ CSA_DEV void row_select(const uint32_t* keys, int n, int k, RowShared& sh, uint3
     sh.warp_b[lane] = sb - b;
   }
   cta_sync();
-  uint32_t gt_run = sh.warp_a[warp], eq_run = sh.warp_b[warp];
+  uint32_t gt_run = gt_base + sh.warp_a[warp], eq_run = eq_base + sh.warp_b[warp];
   const uint32_t lt = (1u << lane) - 1u;
   for (int i = w0 + lane; i - lane < w1; i += 32) {
     const uint32_t km = i < w1 ? keys[i] & M : 0u;
@@ -508,6 +491,49 @@ CSA_DEV void row_select(const uint32_t* keys, int n, int k, RowShared& sh, uint3
     gt_run += __popc(bg);
     eq_run += __popc(be);
   }
+}
+
+// Selects the k largest of keys[0..n) (n > k; order-preserving keys in
+// shared memory, written by this CTA) under (key descending, position
+// ascending) and calls emit(o, i) once for each output slot o < k with the
+// selected position i, slots in ascending order of i.  kmin / kmax: this
+// thread's min and max over the keys it wrote.  All 1024 threads call it.
+template <typename Emit>
+CSA_DEV void row_select(const uint32_t* keys, int n, int k, RowShared& sh, uint32_t kmin,
+                        uint32_t kmax, Emit emit) {
+  constexpr int kBins = 1 << kRowBits;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
+    kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
+  }
+  if (lane == 0) {
+    sh.warp_a[warp] = kmin;
+    sh.warp_b[warp] = kmax;
+  }
+  for (int b = tid; b < kBins; b += kThreads) sh.hist[b] = 0;
+  cta_sync();
+  uint32_t gmin = sh.warp_a[lane], gmax = sh.warp_b[lane];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    gmin = min(gmin, __shfl_xor_sync(0xffffffffu, gmin, o));
+    gmax = max(gmax, __shfl_xor_sync(0xffffffffu, gmax, o));
+  }
+  cta_sync();  // every warp has read the min / max slots
+
+  uint32_t prefix, mask;
+  uint32_t k_rem = (uint32_t)k;
+  if (gmin == gmax) {
+    prefix = gmin;
+    mask = 0xFFFFFFFFu;
+  } else {
+    const int top = 31 - __clz(gmin ^ gmax);
+    mask = top == 31 ? 0u : (0xFFFFFFFFu << (top + 1));
+    prefix = gmin & mask;
+    k_rem = row_rounds(keys, n, k_rem, sh, prefix, mask, top + 1);
+  }
+  ordered_emit(keys, n, k, prefix, mask, k_rem, 0u, 0u, sh, emit);
 }
 
 __global__ void __launch_bounds__(kThreads, 1) topk_row_kernel(const Params p) {
@@ -553,6 +579,218 @@ __global__ void __launch_bounds__(kThreads, 1) topk_row_kernel(const Params p) {
   }
   row_select(keys, n, p.k, sh, kmin, kmax, [&](uint32_t o, int i) { out[o] = i; });
   if (tid == 0) p.cnt[row] = p.k;
+}
+
+// --------------------------------------------- histogram-seeded selection --
+// Decode chain (a few long rows): the indexer kernel has counted each row's
+// visible scores by the top kScoreHistBits bits of their keys, so the bin
+// b* holding the k-th largest key is known from the histogram alone, and
+// one exchange replaces the (min, max) round and the first digit rounds.
+// One cluster of C CTAs per row, each with its slice of the row in shared
+// memory as keys (the layout of topk_kernel, whose select is the fallback):
+//   - every CTA reads the whole histogram and finds b* (a block scan);
+//   - each CTA counts its keys above b* and copies its keys in b* (the
+//     candidates, at most kScoreHistBins / C) into its slot of a candidate
+//     buffer; one push sends both to every CTA, then one cluster barrier;
+//   - the counts are the keys' own, so whether b* holds the threshold is
+//     checked, not assumed (A above b* < k <= A + candidates); if not, or
+//     if a slot overflowed, the cluster runs the full radix select;
+//   - otherwise each CTA ranks the candidates of all slots locally (radix
+//     rounds below b*), which gives the threshold key, and from the
+//     per-slot counts above / equal to it its offset in the index-ordered
+//     output, then emits its slice.
+// The histogram is cleared (each CTA its share) once every CTA has read it.
+struct HistShared {
+  alignas(16) uint32_t cbuf[kScoreHistBins];  // candidates, slot c at [c*cap, (c+1)*cap)
+  alignas(16) uint32_t cn[kMaxC][2];           // per-slot (above b*, candidates)
+  uint32_t gq[kMaxC][2];                       // per-slot (above T, equal to T)
+  uint32_t cand_n, above_n, bstar, pad_;
+  RowShared row;                               // rounds over the candidates
+};
+
+__global__ void __launch_bounds__(kThreads, 1) topk_hist_kernel(const Params p) {
+  using S = Shared<(1 << kDigitBits)>;
+  constexpr int kShift = 32 - kScoreHistBits;
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  uint32_t* keys = reinterpret_cast<uint32_t*>(smem_raw + sizeof(S));
+  HistShared& hs = *reinterpret_cast<HistShared*>(smem_raw + p.hist_off);
+
+  const int row = blockIdx.y;
+  const int C = p.C;
+  const int cap = kScoreHistBins / C;  // candidate slots per CTA
+  const uint32_t r = cluster_ctarank();
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  pdl_trigger();
+  const int64_t pos = p.pos_q ? p.pos_q[row] : p.pos_base + row % p.Q;
+  const int64_t lo = (int64_t)r * p.slice;
+  int64_t n = pos < 0 ? 0 : (pos + 1) / p.m - p.entry_offset;
+  if (n < 0) n = 0;
+  if (tid == 0) {
+    hs.cand_n = 0;
+    hs.above_n = 0;
+    hs.bstar = 0xFFFFFFFFu;  // no bin found
+  }
+  cluster_arrive();  // paired with the wait before the first remote store
+  pdl_wait();  // the scores and the histogram come from the indexer kernel
+  uint32_t* gh = p.hist + (int64_t)row * kScoreHistBins;
+  const int zb = kScoreHistBins / C;  // bins this CTA clears, from r * zb
+  int32_t* out = p.idx + (int64_t)row * p.k;
+  if (n > p.N_cap) {
+    n = p.N_cap;
+    if (r == 0 && tid == 0) report(p.status, CSA_ERR_CAPACITY);
+  }
+  if (n <= p.k) {  // every visible entry is kept; nobody reads the histogram
+    if (r == 0) {
+      for (int j = tid; j < p.k; j += kThreads) out[j] = j < n ? j : -1;
+      if (tid == 0) {
+        p.cnt[row] = (int32_t)n;
+        if (p.path) p.path[row] = 0;
+      }
+    }
+    for (int j = tid; j < zb; j += kThreads) gh[r * zb + j] = 0u;
+    cluster_wait();
+    return;
+  }
+  // Thread t's four bins, highest first (kScoreHistBins == 4 * kThreads),
+  // and the first kPer of its slice's scores, both in flight during the scan.
+  const uint4 h4 = __ldcg(reinterpret_cast<const uint4*>(gh) + (kThreads - 1 - tid));
+  const int cap_n = (int)(p.N_cap - lo < p.slice ? (p.N_cap - lo > 0 ? p.N_cap - lo : 0) : p.slice);
+  const float* src = p.scores + (int64_t)row * p.N_cap + lo;
+  const int len = (int)(n - lo < cap_n ? (n - lo > 0 ? n - lo : 0) : cap_n);
+  constexpr int kPer = 8;  // scores per thread per pass (slices up to 8192 in one)
+  float sv[kPer];
+#pragma unroll
+  for (int j = 0; j < kPer; ++j) {
+    const int i = tid + j * kThreads;
+    sv[j] = i < len ? __ldg(src + i) : 0.f;
+  }
+
+  // b*: an exclusive scan over threads counts the scores in higher bins.
+  {
+    const uint32_t c4[4] = {h4.w, h4.z, h4.y, h4.x};
+    uint32_t above = block_excl_scan(c4[0] + c4[1] + c4[2] + c4[3], hs.row.scan);
+    const uint32_t k = (uint32_t)p.k;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      // (The lowest such bin: with a histogram that does not add up, the
+      // CTAs of the cluster still agree on b*.)
+      if (above < k && above + c4[j] >= k)
+        atomicMin(&hs.bstar, (uint32_t)(kScoreHistBins - 1 - 4 * tid - j));
+      above += c4[j];
+    }
+  }
+  cta_sync();
+  const uint32_t bstar = hs.bstar;
+
+  // This CTA's keys (to shared memory) above b* (counted) and in b* (copied
+  // to its slot), pass by pass over the visible part of the slice.
+  uint32_t n_above = 0;
+  uint32_t* mine = hs.cbuf + r * cap;
+  for (int base_i = 0; base_i < len; base_i += kPer * kThreads) {
+    if (base_i > 0) {
+#pragma unroll
+      for (int j = 0; j < kPer; ++j) {
+        const int i = base_i + tid + j * kThreads;
+        sv[j] = i < len ? __ldg(src + i) : 0.f;
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+      const int i = base_i + tid + j * kThreads;  // warp-uniform range per j
+      const uint32_t key = orderable(sv[j]);
+      if (i < len) keys[i] = key;
+      const uint32_t bin = key >> kShift;
+      n_above += (i < len && bin > bstar) ? 1u : 0u;
+      const bool cand = i < len && bin == bstar;
+      const uint32_t bal = __ballot_sync(0xffffffffu, cand);
+      if (bal) {
+        uint32_t at = 0;
+        if (lane == 0) at = atomicAdd(&hs.cand_n, (uint32_t)__popc(bal));
+        at = __shfl_sync(0xffffffffu, at, 0);
+        const uint32_t o = at + __popc(bal & ((1u << lane) - 1u));
+        if (cand && o < (uint32_t)cap) mine[o] = key;
+      }
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) n_above += __shfl_xor_sync(0xffffffffu, n_above, o);
+  if (lane == 0 && n_above) atomicAdd(&hs.above_n, n_above);
+  cta_sync();
+  cluster_wait();  // every CTA of the cluster is running
+
+  // One exchange: counts and candidates into slot r of every CTA.
+  const uint32_t my_a = hs.above_n, my_c = hs.cand_n;
+  if (tid < C) st_remote_v2(mapa(smem_u32(&hs.cn[r][0]), tid), my_a, my_c);
+  const int nv4 = ((int)min(my_c, (uint32_t)cap) + 3) / 4;
+  for (int t = tid; t < C * nv4; t += kThreads) {
+    const int c = t / nv4, j = t % nv4;
+    if (c == (int)r) continue;
+    const uint4 v = reinterpret_cast<const uint4*>(mine)[j];
+    st_remote_v4(mapa(smem_u32(mine + 4 * j), c), v);
+  }
+  cluster_arrive();
+  cluster_wait();
+  // Every CTA has read the histogram: clear this CTA's share.
+  for (int j = tid; j < zb / 4; j += kThreads)
+    reinterpret_cast<uint4*>(gh + r * zb)[j] = make_uint4(0u, 0u, 0u, 0u);
+
+  uint32_t A = 0, Mc = 0;
+  bool ovf = false;
+  for (int c = 0; c < C; ++c) {
+    A += hs.cn[c][0];
+    Mc += hs.cn[c][1];
+    ovf = ovf || hs.cn[c][1] > (uint32_t)cap;
+  }
+  const uint32_t k = (uint32_t)p.k;
+  if (bstar == 0xFFFFFFFFu || ovf || A >= k || A + Mc < k) {
+    // The histogram did not hold this row's scores: the full select.
+    cluster_select<kDigitBits, false>(smem_raw, C, r, p.k, len, lo, out);
+    if (r == 0 && tid == 0) {
+      p.cnt[row] = p.k;
+      if (p.path) p.path[row] = 2;
+    }
+    return;
+  }
+
+  // The threshold among the candidates (unused slots hold a key outside b*).
+  const uint32_t pad = (bstar ^ 1u) << kShift;
+  for (int i = tid; i < kScoreHistBins; i += kThreads)
+    if ((uint32_t)(i % cap) >= hs.cn[i / cap][1]) hs.cbuf[i] = pad;
+  for (int b = tid; b < (1 << 10); b += kThreads) hs.row.hist[b] = 0u;
+  cta_sync();
+  uint32_t T = bstar << kShift, M = 0xFFFFFFFFu << kShift;
+  const uint32_t need_eq = row_rounds<10>(hs.cbuf, kScoreHistBins, k - A, hs.row, T, M, kShift);
+  // Per slot: keys above T (those above b* included) and equal to it.
+  if (warp < C) {
+    const uint32_t nc = hs.cn[warp][1];
+    uint32_t gt = 0, eq = 0;
+    for (uint32_t j = lane; j < nc; j += 32) {
+      const uint32_t km = hs.cbuf[warp * cap + j] & M;
+      gt += km > T;
+      eq += km == T;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      gt += __shfl_xor_sync(0xffffffffu, gt, o);
+      eq += __shfl_xor_sync(0xffffffffu, eq, o);
+    }
+    if (lane == 0) {
+      hs.gq[warp][0] = hs.cn[warp][0] + gt;
+      hs.gq[warp][1] = eq;
+    }
+  }
+  cta_sync();
+  uint32_t gt_base = 0, eq_base = 0;
+  for (int c = 0; c < (int)r; ++c) {
+    gt_base += hs.gq[c][0];
+    eq_base += hs.gq[c][1];
+  }
+  ordered_emit(keys, len, p.k, T, M, need_eq, gt_base, eq_base, hs.row,
+               [&](uint32_t o, int i) { out[o] = (int32_t)(lo + i); });
+  if (r == 0 && tid == 0) {
+    p.cnt[row] = p.k;
+    if (p.path) p.path[row] = 1;
+  }
 }
 
 // ------------------------------------------------- context split over ranks --
@@ -700,13 +938,15 @@ cudaError_t launch_merge_candidates(const MergeLaunch& a, cudaStream_t stream) {
 }
 
 // Largest cluster size (8 or 16) that can be resident for this kernel and
-// shared-memory size on the current device; cached per device.
-int max_cluster(const void* kern, size_t smem) {
-  static int cached[64][2] = {};
-  static size_t cached_smem[64] = {};
+// shared-memory size on the current device; cached per device and kernel
+// (`which`: 0 topk_kernel, 1 topk_hist_kernel).  Also allows the 16-CTA
+// size on the kernel.
+int max_cluster(const void* kern, size_t smem, int which) {
+  static int cached[64][2][2] = {};
+  static size_t cached_smem[64][2] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 8;
-  if (cached[dev][0] && cached_smem[dev] == smem) return cached[dev][1];
+  if (cached[dev][which][0] && cached_smem[dev][which] == smem) return cached[dev][which][1];
   int best = 8;
   bool failed = true;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
@@ -729,21 +969,29 @@ int max_cluster(const void* kern, size_t smem) {
     }
   }
   if (failed) cudaGetLastError();  // a refused query is not the caller's error
-  cached[dev][0] = 1;
-  cached[dev][1] = best;
-  cached_smem[dev] = smem;
+  cached[dev][which][0] = 1;
+  cached[dev][which][1] = best;
+  cached_smem[dev][which] = smem;
   return best;
 }
 
 // Rows of at most this many scores take the one-CTA-per-row kernel.
 constexpr int64_t kRowMaxScores = (200 * 1024 - (int64_t)kRowKeysOff) / 4;
 
-cudaError_t launch_topk(const TopkLaunch& a, cudaStream_t stream) {
+// One CTA per row when rows fill the GPU (prefill) or are short; a few
+// long rows (decode) spread each row over a cluster instead.
+static bool row_path(int rows, int64_t N_cap) {
+  return N_cap <= kRowMaxScores && (rows >= device_sm_count() / 4 || N_cap <= 8192);
+}
+
+bool topk_uses_hist(int rows, int64_t N_cap) {
+  return rows >= 1 && rows <= 65535 && !row_path(rows, N_cap) && N_cap <= 8 * 32768;
+}
+
+static cudaError_t launch_topk_impl(const TopkLaunch& a, cudaStream_t stream) {
   if (a.rows < 1) return cudaSuccess;
   if (a.rows > 65535 || a.k > kMaxK) return cudaErrorInvalidConfiguration;
-  // One CTA per row when rows fill the GPU (prefill) or are short; a few
-  // long rows (decode) spread each row over a cluster instead.
-  if (a.N_cap <= kRowMaxScores && (a.rows >= device_sm_count() / 4 || a.N_cap <= 8192)) {
+  if (row_path(a.rows, a.N_cap)) {
     Params p{};
     p.Q = a.Q;
     p.m = a.m;
@@ -767,15 +1015,19 @@ cudaError_t launch_topk(const TopkLaunch& a, cudaStream_t stream) {
   const int sms = device_sm_count();
   const int need = (int)((a.N_cap + 32767) / 32768);
   if (need > 8) return cudaErrorInvalidValue;
-  auto kern = topk_kernel<kDigitBits, false>;
+  const bool hist = a.hist != nullptr;
+  auto kern = hist ? topk_hist_kernel : topk_kernel<kDigitBits, false>;
   using S = Shared<(1 << kDigitBits)>;
   // Slices of at most 32768 scores; small batches spread each row over more
   // CTAs (slices of at least 4096 scores), up to 16 where 16-CTA clusters fit.
+  // The histogram kernel's HistShared follows the largest slice.
   const int64_t slice_max = (a.N_cap + need - 1) / need;
-  cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kern), 2,
-                                   sizeof(S) + (size_t)slice_max * 4);
+  const size_t hist_off = (sizeof(S) + (size_t)slice_max * 4 + 15) / 16 * 16;
+  const size_t smem_max = hist ? hist_off + sizeof(HistShared) : sizeof(S) + (size_t)slice_max * 4;
+  cudaError_t e =
+      ensure_smem_attr(reinterpret_cast<const void*>(kern), hist ? 17 : 2, smem_max);
   if (e != cudaSuccess) return e;
-  const int limit = max_cluster(reinterpret_cast<const void*>(kern), sizeof(S) + slice_max * 4);
+  const int limit = max_cluster(reinterpret_cast<const void*>(kern), smem_max, hist ? 1 : 0);
   int C = 1;
   while (C < need) C <<= 1;
   if (a.rows < sms) {
@@ -796,8 +1048,19 @@ cudaError_t launch_topk(const TopkLaunch& a, cudaStream_t stream) {
   p.idx = a.idx;
   p.cnt = a.cnt;
   p.status = a.status;
-  const size_t smem = sizeof(S) + (size_t)p.slice * 4;
+  p.hist = a.hist;
+  p.path = a.path;
+  size_t smem = sizeof(S) + (size_t)p.slice * 4;
+  if (hist) {
+    p.hist_off = (uint32_t)((smem + 15) / 16 * 16);
+    smem = p.hist_off + sizeof(HistShared);
+  }
   return launch_pdl(kern, dim3(C, a.rows, 1), dim3(kThreads), smem, stream, C, a.chained, p);
+}
+
+cudaError_t launch_topk(const TopkLaunch& a, cudaStream_t stream) {
+  if (a.hist && !topk_uses_hist(a.rows, a.N_cap)) return cudaErrorInvalidValue;
+  return launch_topk_impl(a, stream);
 }
 
 }  // namespace csa

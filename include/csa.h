@@ -378,7 +378,14 @@ csa_status csa_prefill_chunk(const csa_params* p, int64_t P, int T, const void* 
  *   [B, H_I]; topk_idx [B, k], topk_cnt [B] (written); out [B, H, d] bf16
  *   and lse [B, H] or NULL (written); other tensors as csa_compress and
  *   sparse_mqa_decode.
- * Workspace: csa_workspace_bytes(p, CSA_OP_CSA_DECODE_STEP, 1, N_cap).
+ * Workspace: csa_workspace_bytes(p, CSA_OP_CSA_DECODE_STEP, 1, N_cap).  It
+ * carries state between calls that only affects speed: where the top-k
+ * spreads a row over a cluster of CTAs (a few long rows), the indexer
+ * counts each row's scores by their top 12 key bits into a histogram in the
+ * workspace, which the top-k reads and clears.  A zero-filled workspace, or
+ * one that the previous call of this function left, takes the fast path;
+ * other contents cost that call a full radix selection, never a different
+ * result.
  * Device errors: a newest block at or beyond N_cap -> CSA_ERR_DEVICE_INDEX
  * (not written).
  * ------------------------------------------------------------------------- */

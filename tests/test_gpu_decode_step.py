@@ -158,3 +158,153 @@ def test_hca_decode_loop(orc):
         assert np.isfinite(got).all()
         assert_attention_close(got, ro[:, 0], f"HCA step {step}")
         _check_lse(lse, rl[:, 0], ro[:, 0])
+
+
+# ----------------------------------------------------------------------------
+# The histogram-seeded top-k of the decode step (a few long rows: one cluster
+# of CTAs per row).  The workspace holds the scores [B, N_cap] fp32 from byte
+# 0, then the score histogram [B, 4096] u32 and one path word per sequence
+# (0 every visible entry kept, 1 histogram path, 2 full radix select).
+
+def _ws_layout(B, N_cap):
+    sb = (B * N_cap * 4 + 255) // 256 * 256
+    return sb, sb + B * 4096 * 4
+
+
+def _hist_and_path(ws, B, N_cap):
+    h0, p0 = _ws_layout(B, N_cap)
+    hist = ws[h0:p0].view(torch.int32).view(B, 4096).cpu().numpy()
+    path = ws[p0:p0 + 4 * B].view(torch.int32).cpu().numpy()
+    return hist, path
+
+
+class _Step:
+    """A decode step over caches compressed from random token streams (the
+    construction of the timed workload), or over given caches."""
+
+    def __init__(self, w, L_cap, seed=0):
+        w = configs.scaled(w, seed=w.seed + seed)
+        self.w, self.B, self.N = w, w.B, L_cap // w.m
+        B, d = w.B, w.d
+        self.kv_tok, self.idx_tok = synth.token_streams(w, L_cap=L_cap, device=DEV)
+        self.w_s, self.b_pos = synth.pool_params(w, DEV)
+        self.w_si, self.b_pi = synth.pool_params(w, DEV, indexer=True)
+        self.p = binding.params_for(w, B=B)
+        self.kv_c = torch.zeros(B, self.N, d, dtype=torch.bfloat16, device=DEV)
+        self.key = torch.zeros(B, self.N, w.D_I, dtype=torch.uint8, device=DEV)
+        self.ksc = torch.zeros(B, self.N, dtype=torch.float32, device=DEV)
+        self.ws = binding.workspace(self.p, binding.OP_CSA_DECODE_STEP, 1, self.N)
+        self.status = torch.zeros(1, dtype=torch.int32, device=DEV)
+
+    def compress_all(self, L):
+        ctx = torch.full((self.B,), L, dtype=torch.int64, device=DEV)
+        binding.csa_compress(self.p, self.kv_tok, ctx, self.w_s, self.b_pos, None, 0, self.N,
+                             self.kv_c, self.idx_tok, self.w_si, self.b_pi, self.key, self.ksc,
+                             dev_status=self.status)
+
+    def run(self, pos, qseed):
+        w, B = self.w, self.B
+        qi = synth.queries(configs.scaled(w, seed=qseed), Q=1, device=DEV)
+        out = torch.empty(B, w.H, w.D, dtype=torch.bfloat16, device=DEV)
+        tidx = torch.full((B, w.k), -7, dtype=torch.int32, device=DEV)
+        tcnt = torch.full((B,), -7, dtype=torch.int32, device=DEV)
+        pos_t = torch.as_tensor(pos, dtype=torch.int64, device=DEV)
+        binding.csa_decode_step(self.p, pos_t, self.kv_tok, self.idx_tok, self.w_s, self.b_pos,
+                                None, self.w_si, self.b_pi, self.kv_c, self.key, self.ksc,
+                                qi["q"][:, 0].contiguous(), qi["q_idx"][:, 0].contiguous(),
+                                qi["q_scale"][:, 0].contiguous(), qi["w"][:, 0].contiguous(),
+                                qi["sink"], tidx, tcnt, out, ws=self.ws, dev_status=self.status)
+        torch.cuda.synchronize()
+        assert self.status.item() == 0, self.status.item()
+        return qi, tidx, tcnt
+
+    def check(self, orc, pos, qi, tidx, tcnt, path_expect, n_sample=256):
+        """Scores (sampled) against the oracle on the GPU's keys; the top-k
+        bit-exact against the oracle ranking the GPU's scores; the path
+        taken; the histogram cleared."""
+        w, B, N = self.w, self.B, self.N
+        pos = np.asarray(pos)
+        nv = (pos + 1) // w.m
+        scores = self.ws[: B * N * 4].view(torch.float32).view(B, N).cpu().numpy().astype(np.float64)
+        keys, ks = bits8(self.key), f32(self.ksc)
+        rng = np.random.default_rng(int(pos.sum()))
+        for b in range(B):
+            smp = np.union1d(rng.choice(nv[b], min(n_sample, nv[b]), replace=False),
+                             [0, nv[b] - 1])
+            ref = orc.index_scores(bits8(qi["q_idx"][b: b + 1]), f32(qi["q_scale"][b: b + 1]),
+                                   f32(qi["w"][b: b + 1]), keys[b: b + 1, smp], ks[b: b + 1, smp],
+                                   np.array([[len(smp) * w.m - 1]]), w.m)[0, 0]
+            g = scores[b, smp]
+            assert np.allclose(g, ref, rtol=2e-5, atol=1e-6 * np.abs(ref).mean()), b
+        gs = np.full((B, N), -np.inf)
+        for b in range(B):
+            gs[b, : nv[b]] = scores[b, : nv[b]]
+        ridx, rcnt = orc.topk(gs, nv, w.k)
+        assert np.array_equal(tcnt.cpu().numpy(), rcnt)
+        assert np.array_equal(tidx.cpu().numpy(), ridx)
+        hist, path = _hist_and_path(self.ws, B, N)
+        assert not hist.any(), "histogram not cleared"
+        assert path.tolist() == list(path_expect), path
+
+
+def test_histogram_topk_csa_128k_shape(orc):
+    """The timed 128K workload (8 sequences x 32768 entries, k = 1024):
+    every row takes the histogram path, on a fresh workspace and on the one
+    the previous step left.  The indexer adds its counts to what the
+    workspace holds: N spurious counts in the top bin (keys no finite score
+    has) make that bin the guess, which the keys' own counts refute, so every
+    row takes the full select, with the same result; counts below the
+    threshold change nothing."""
+    w = configs.CSA_128K
+    st = _Step(w, w.L, seed=1)
+    st.compress_all(w.L)
+    pos = np.full(w.B, w.L - 1)
+    for step in range(2):
+        qi, tidx, tcnt = st.run(pos, w.seed + 1000 + step)
+        st.check(orc, pos, qi, tidx, tcnt, [1] * w.B)
+    h0, _ = _ws_layout(w.B, st.N)
+    for top_bin, path in ((4095, 2), (0, 1)):
+        bad = torch.zeros(w.B, 4096, dtype=torch.int32, device=DEV)
+        bad[:, top_bin] = st.N
+        st.ws[h0: h0 + bad.numel() * 4].copy_(bad.view(-1).view(torch.uint8))
+        qi, tidx, tcnt = st.run(pos, w.seed + 1002 + top_bin)
+        st.check(orc, pos, qi, tidx, tcnt, [path] * w.B)
+
+
+def test_histogram_topk_csa_1m_shape(orc):
+    """The timed 1M workload (4 sequences x 262144 entries, 16-CTA clusters
+    of 256 candidate slots each): the histogram path, bit-exact."""
+    w = configs.CSA_1M
+    st = _Step(w, w.L, seed=2)
+    st.compress_all(w.L)
+    pos = np.full(w.B, w.L - 1)
+    qi, tidx, tcnt = st.run(pos, w.seed + 1000)
+    st.check(orc, pos, qi, tidx, tcnt, [1] * w.B)
+
+
+@pytest.mark.parametrize("case", ["ties", "all_equal", "few_visible"])
+def test_histogram_topk_structures(orc, case):
+    """Two sequences x 16384 entries, k = 512 (4-CTA clusters, 1024 slots):
+    ties: one key row for every entry and 64 key scales, so scores take 64
+    values and the threshold bin holds 8 of them (the tie rule across CTAs);
+    all_equal: one score everywhere, more candidates than slots (the full
+    select, lowest indices); few_visible: one sequence with fewer visible
+    entries than k next to one on the histogram path."""
+    w = configs.scaled(configs.CSA_128K, B=2, k=512, L=65536)
+    st = _Step(w, w.L, seed=5)
+    N = st.N
+    row = synth.e4m3_codes((1, 1, w.D_I), 6, "q_idx", DEV)
+    st.key.copy_(row.expand(w.B, N, w.D_I))
+    if case == "ties":
+        vals = 1.0 + torch.arange(64, device=DEV, dtype=torch.float32) / 64
+        rng = torch.Generator(device=DEV).manual_seed(7)
+        st.ksc.copy_(vals[torch.randint(0, 64, (w.B, N), generator=rng, device=DEV)] / 64)
+    else:
+        st.ksc.fill_(1.0 / 64)
+    pos = np.full(w.B, w.L - 1)
+    expect = [1, 1] if case == "ties" else [2, 2]
+    if case == "few_visible":
+        pos[0] = 4 * 400 - 1
+        expect = [0, 2]
+    qi, tidx, tcnt = st.run(pos, w.seed + 1000)
+    st.check(orc, pos, qi, tidx, tcnt, expect)
