@@ -158,8 +158,9 @@ CSA_DEV bool wait_all(uint64_t* bar, uint32_t parity, const Params& p, volatile 
 // output row leaves as one coalesced 32-lane store and the rotated pairs
 // (d, d + R/2) sit in lanes l and l ^ (R/2/VPL).  The S (max, sum) pairs
 // become one weight per split (wsplit: S floats of this warp's shared
-// memory); the partials are read G splits at a time with the next group's
-// loads in flight, the first group before the weights are known.
+// memory).  The first G splits' partials are loaded together with the
+// (max, sum) pairs, so that with S <= G the warp waits on one round of L2
+// reads; further groups of G follow one round each.
 // kLdg: the partials come from an earlier kernel (read-only path); otherwise
 // they were written during this kernel by other CTAs and are read from L2.
 template <int D, int R, int G, bool kLdg>
@@ -183,22 +184,29 @@ CSA_DEV void merge_head(const Params& p, int row, int h, int lane, float* wsplit
       *reinterpret_cast<uint2*>(&v[0]) = ld2(reinterpret_cast<const uint2*>(a));
     }
   };
-  uint32_t cur[G][NW], nxt[G][NW];
+  uint32_t buf[G][NW];
 #pragma unroll
   for (int u = 0; u < G; ++u)
-    if (u < S) load(u, cur[u]);
+    if (u < S) load(u, buf[u]);
+  // Split `lane`'s (max, sum) pair, in flight with the partials.
+  float m0 = -INFINITY, l0 = 0.f;
+  if (lane < S) {
+    m0 = ldf(ml + (int64_t)lane * 2 * p.H + h);
+    l0 = ldf(ml + (int64_t)lane * 2 * p.H + p.H + h);
+  }
   const float LOG2E = 1.4426950408889634f;
   const float z = p.sink[h];
   const float z2 = z * LOG2E;  // log2 domain
-  float M = z2;
-  for (int s = lane; s < S; s += 32) M = fmaxf(M, ldf(ml + (int64_t)s * 2 * p.H + h));
+  float M = fmaxf(z2, m0);
+  for (int s = lane + 32; s < S; s += 32) M = fmaxf(M, ldf(ml + (int64_t)s * 2 * p.H + h));
   M = warp_max(M);
   const bool zero = z == INFINITY || M == -INFINITY;  // +inf sink, or nothing to attend
   float L = 0.f;
   if (!zero) {
     for (int s = lane; s < S; s += 32) {
-      const float ms = ldf(ml + (int64_t)s * 2 * p.H + h);
-      const float w = ms == -INFINITY ? 0.f : ldf(ml + (int64_t)s * 2 * p.H + p.H + h) * exp2f(ms - M);
+      const float ms = s == lane ? m0 : ldf(ml + (int64_t)s * 2 * p.H + h);
+      const float ls = s == lane ? l0 : ldf(ml + (int64_t)s * 2 * p.H + p.H + h);
+      const float w = ms == -INFINITY ? 0.f : ls * exp2f(ms - M);
       wsplit[s] = w;  // the split's stored output is O / l
       L += w;
     }
@@ -212,10 +220,10 @@ CSA_DEV void merge_head(const Params& p, int row, int h, int lane, float* wsplit
   for (int e = 0; e < VPL; ++e) acc[e] = 0.f;
   if (!zero) {
     for (int s0 = 0; s0 < S; s0 += G) {
-      if (s0 + G < S) {
+      if (s0 > 0) {
 #pragma unroll
         for (int u = 0; u < G; ++u)
-          if (s0 + G + u < S) load(s0 + G + u, nxt[u]);
+          if (s0 + u < S) load(s0 + u, buf[u]);
       }
 #pragma unroll
       for (int u = 0; u < G; ++u) {
@@ -224,15 +232,11 @@ CSA_DEV void merge_head(const Params& p, int row, int h, int lane, float* wsplit
         if (w == 0.f) continue;  // empty split: its partial was never written
 #pragma unroll
         for (int i = 0; i < NW; ++i) {
-          const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&cur[u][i]));
+          const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&buf[u][i]));
           acc[2 * i] = fmaf(f.x, w, acc[2 * i]);
           acc[2 * i + 1] = fmaf(f.y, w, acc[2 * i + 1]);
         }
       }
-#pragma unroll
-      for (int u = 0; u < G; ++u)
-#pragma unroll
-        for (int i = 0; i < NW; ++i) cur[u][i] = nxt[u][i];
     }
     const float invL = 1.0f / L;
 #pragma unroll
@@ -1159,7 +1163,9 @@ cudaError_t launch_impl(const MqaLaunch& a, cudaStream_t stream) {
   if (a.emit_partials) return cudaSuccess;  // the caller merges the partials
   const unsigned nblk = (unsigned)(((int64_t)rows * a.H + 3) / 4);
   const size_t wsm = (size_t)4 * a.splits * sizeof(float);
-  auto merge = mqa_combine_kernel<D, R, 4>;
+  // Groups of 8 or 16 splits (the first group's loads go out with the
+  // (max, sum) pairs).
+  auto merge = a.splits <= 8 ? mqa_combine_kernel<D, R, 8> : mqa_combine_kernel<D, R, 16>;
   return launch_pdl(merge, dim3(nblk), dim3(128), wsm, stream, 0, 1, p, rows);
 }
 
@@ -1182,8 +1188,8 @@ cudaError_t launch_merge_impl(const MqaLaunch& a, cudaStream_t stream) {
   const int rows = a.B * a.Q;
   const unsigned nblk = (unsigned)(((int64_t)rows * a.H + 3) / 4);
   const size_t wsm = (size_t)4 * a.splits * sizeof(float);
-  return launch_pdl(mqa_combine_kernel<D, R, 4>, dim3(nblk), dim3(128), wsm, stream, 0, a.chained,
-                    p, rows);
+  auto merge = a.splits <= 8 ? mqa_combine_kernel<D, R, 8> : mqa_combine_kernel<D, R, 16>;
+  return launch_pdl(merge, dim3(nblk), dim3(128), wsm, stream, 0, a.chained, p, rows);
 }
 
 }  // namespace
