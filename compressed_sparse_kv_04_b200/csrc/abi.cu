@@ -228,7 +228,8 @@ static csa_status compress_common(const char* fn, const csa_params* p, const voi
                                   int64_t N_cap, const void* idx_tok, const float* w_s_idx,
                                   const float* b_pos_idx, uint8_t* idx_key, float* idx_scale,
                                   int32_t* dev_status, void* stream,
-                                  const int64_t* pos_newest = nullptr, int pdl_head = 0) {
+                                  const int64_t* pos_newest = nullptr, int pdl_head = 0,
+                                  int* ctas = nullptr) {
   csa_status st = check_common(fn, p);
   if (st != CSA_OK) return st;
   REQ_PTR(kv_tok);
@@ -285,6 +286,7 @@ static csa_status compress_common(const char* fn, const csa_params* p, const voi
   fill_inv_freq(p, c.inv_freq);
   c.status = dev_status;
   c.pdl_head = pdl_head;
+  if (ctas) *ctas = csa::compress_ctas(c);
   cudaError_t e = csa::launch_compress(c, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(fn, e);
   return CSA_OK;
@@ -324,10 +326,12 @@ static csa_status index_common(const char* fn, const csa_params* p, int Q,
                                const int64_t* pos_q, int64_t pos_base, float* scores,
                                int32_t* dev_status, cudaStream_t stream, int chained,
                                const int64_t* safe_pos = nullptr,
-                               int64_t safe_fixed = INT64_MAX, uint32_t* hist = nullptr) {
+                               int64_t safe_fixed = INT64_MAX, uint32_t* hist = nullptr,
+                               int reserve_slots = 0) {
   csa::IndexLaunch a{};
   a.chained = chained;
   a.hist = hist;
+  a.reserve_slots = reserve_slots;
   a.safe_pos = safe_pos;
   a.safe_fixed = safe_fixed;
   a.B = p->B;
@@ -386,10 +390,10 @@ static csa_status index_topk_common(const char* fn, const csa_params* p, int Q,
                                     int32_t* dev_status, cudaStream_t stream, int chained,
                                     const int64_t* safe_pos = nullptr,
                                     int64_t safe_fixed = INT64_MAX, uint32_t* hist = nullptr,
-                                    int32_t* path = nullptr) {
+                                    int32_t* path = nullptr, int reserve_slots = 0) {
   csa_status st = index_common(fn, p, Q, q_idx, q_scale, w, idx_key, idx_scale, N_cap, pos_q,
                                pos_base, scores, dev_status, stream, chained, safe_pos,
-                               safe_fixed, hist);
+                               safe_fixed, hist, reserve_slots);
   if (st != CSA_OK) return st;
   return topk_common(fn, p, Q, scores, N_cap, pos_q, pos_base, topk_idx, topk_cnt, dev_status,
                      stream, 1, hist, path);
@@ -689,11 +693,13 @@ csa_status csa_decode_step(const csa_params* p, const int64_t* pos_q, const void
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   // 1. Each sequence's newest block: the one holding its query token,
   // pooled over the tokens up to it.
+  int compress_ctas = 0;
   st = compress_common(fn, p, kv_tok, L_cap, nullptr, 0, w_s, b_pos, gamma, 0, 1, kv_c, N_cap,
                        idx_tok, w_s_idx, b_pos_idx, idx_key, idx_scale, dev_status, stream, pos_q,
-                       1);
+                       1, &compress_ctas);
   if (st != CSA_OK) return st;
-  // 2-3. Indexer and top-k over each sequence's visible entries.  Where the
+  // 2-3. Indexer and top-k over each sequence's visible entries (the indexer
+  // grid leaves out the slots the compression CTAs hold).  Where the
   // top-k spreads a row over a cluster, the indexer also counts the scores
   // by their top key bits, which seeds the selection.
   float* scores = static_cast<float*>(ws);
@@ -704,7 +710,7 @@ csa_status csa_decode_step(const csa_params* p, const int64_t* pos_q, const void
   // Only each sequence's newest block is written by this call.
   st = index_topk_common(fn, p, 1, q_idx, q_scale, w, idx_key, idx_scale, N_cap, pos_q, 0,
                          topk_idx, topk_cnt, scores, dev_status, s, 1, pos_q, INT64_MAX, hist,
-                         path);
+                         path, compress_ctas);
   if (st != CSA_OK) return st;
   // 4. Sparse MQA over the selection, the window and the sink.
   const size_t head = scores_bytes(p->B, N_cap) + hist_bytes(p->B);

@@ -24,6 +24,8 @@
 // per block, 8 blocks per 256-thread CTA.  m > 16: 8 warps per block, merged
 // through shared memory.  Both streams of csa_compress run in one launch
 // (blockIdx.y selects the stream).
+#include <algorithm>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -400,6 +402,13 @@ __global__ void __launch_bounds__(kThreads) compress_kernel(const PoolArgs a) {
 }
 
 }  // namespace
+
+int compress_ctas(const CompressLaunch& c) {
+  const int G = c.m + c.overlap <= 16 ? 1 : kWarps;
+  const int per_cta = kWarps / G;
+  const int64_t units = (int64_t)c.B * (c.pos_newest ? 1 : c.n_blocks);
+  return (int)std::min<int64_t>((units + per_cta - 1) / per_cta * (c.idx_tok ? 2 : 1), 1 << 30);
+}
 
 cudaError_t launch_compress(const CompressLaunch& c, cudaStream_t stream) {
   PoolArgs a{};

@@ -52,7 +52,7 @@ struct Params {
   // is the one being written); else safe_fixed for every sequence.
   const int64_t* safe_pos;
   int64_t safe_fixed;
-  int tiles_per_chunk, ntiles, qgroups;
+  int nchunks, ntiles, qgroups;  // chunk c: tiles [c*ntiles/nchunks, (c+1)*ntiles/nchunks)
   const uint8_t* q_idx;
   const float* q_scale;
   const float* w;
@@ -79,6 +79,15 @@ CSA_DEV int64_t safe_bound(const Params& p, int b) {
   const int64_t t = p.safe_pos[b];
   const int64_t i = (t < 0 ? 0 : t / p.m) - p.entry_offset;
   return i < 0 ? 0 : i;
+}
+
+// Tiles the set-up issues into the key ring: the CTA's first tiles, up to
+// one per stage, while their entries lie below the safe bound.
+CSA_DEV int early_tiles(const Params& p, int b, int t_begin, int t_end, int stages) {
+  const int64_t safe = safe_bound(p, b);
+  int n = 0;
+  while (n < stages && t_begin + n < t_end && (int64_t)(t_begin + n + 1) * kTileRows <= safe) ++n;
+  return n;
 }
 
 // EW epilogue warps: 4 (one per TMEM lane quarter; two CTAs per SM), or 8
@@ -121,6 +130,39 @@ __global__ void __launch_bounds__(64 + 32 * EW, EW == 4 ? 2 : 1)
   const int b = group / p.qgroups;
   const int q0 = (group % p.qgroups) * p.G;
   const int nq = min(p.G, p.Q - q0);
+  constexpr int kThr = 64 + 32 * EW;
+
+  // The query tile's codes (B operand; row g*HP + h holds head h of query
+  // q0+g, zero for padding heads and absent queries) and the head weights
+  // are caller inputs, loaded first: the key stream, started below before
+  // the rest of the set-up, would otherwise queue ahead of them.
+  constexpr int kQPre = 3;  // chunks per thread held in registers (decode: all)
+  const int nchunk = p.N * (DI / 16);
+  auto q_chunk = [&](int c) -> uint4 {
+    const int row = c / (DI / 16), chunk = c % (DI / 16);
+    const int g = row / p.HP, h = row % p.HP;
+    if (g >= nq || h >= p.H_I) return make_uint4(0, 0, 0, 0);
+    return __ldg(reinterpret_cast<const uint4*>(
+        p.q_idx + (((int64_t)b * p.Q + q0 + g) * p.H_I + h) * DI + chunk * 16));
+  };
+  uint4 qpre[kQPre];
+#pragma unroll
+  for (int j = 0; j < kQPre; ++j) {
+    const int c = threadIdx.x + j * kThr;
+    qpre[j] = c < nchunk ? q_chunk(c) : make_uint4(0, 0, 0, 0);
+  }
+  float wpre[2], spre[2];
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    const int r = threadIdx.x + j * kThr;
+    const int g = r / p.HP, h = r % p.HP;
+    wpre[j] = spre[j] = 0.f;
+    if (r < p.N && g < nq && h < p.H_I) {
+      const int64_t o = ((int64_t)b * p.Q + q0 + g) * p.H_I + h;
+      wpre[j] = __ldg(p.w + o);
+      spre[j] = __ldg(p.q_scale + o);
+    }
+  }
 
   // Visible entries per query of the group (causal), clamped to capacity.
   int64_t nv_max = 0;
@@ -131,9 +173,9 @@ __global__ void __launch_bounds__(64 + 32 * EW, EW == 4 ? 2 : 1)
     if (nv > p.N_cap) nv = p.N_cap;
     nv_max = max(nv_max, nv);
   }
-  const int t_begin = blockIdx.x * p.tiles_per_chunk;
+  const int t_begin = (int)((int64_t)blockIdx.x * p.ntiles / p.nchunks);
   const int t_vis = (int)((nv_max + kTileRows - 1) / kTileRows);
-  const int t_end = min(min(t_begin + p.tiles_per_chunk, p.ntiles), t_vis);
+  const int t_end = min((int)((int64_t)(blockIdx.x + 1) * p.ntiles / p.nchunks), t_vis);
   if (t_begin >= t_end) {  // uniform over the CTA
     pdl_wait();  // this grid completes only after its predecessor
     return;
@@ -154,34 +196,40 @@ __global__ void __launch_bounds__(64 + 32 * EW, EW == 4 ? 2 : 1)
     hrange[0] = kScoreHistBins;
     hrange[1] = 0u;
     fence_mbar_init();
+    fence_proxy_async_smem();
+    // The key stream starts here: the ring's stages take the CTA's first
+    // tiles of entries written before this call (the producer continues
+    // after them), so their latency overlaps the rest of the set-up.
+    tma_prefetch_desc(&kmap);
+    const int n_early = early_tiles(p, b, t_begin, t_end, C::kStages);
+    for (int j = 0; j < n_early; ++j) {
+      mbar_expect_tx(&full[j], C::kStageBytes);
+      tma_load_2d(ring + j * C::kStageBytes, &kmap, &full[j], 0,
+                  (int32_t)((int64_t)b * p.N_cap + (int64_t)(t_begin + j) * kTileRows));
+    }
   }
   __syncwarp();
   if (warp == 0) {
     tmem_alloc(tmem_base_slot, p.tmem_cols);
     tmem_relinquish();
   }
-  // Query tile (B operand): row g*HP + h holds head h of query q0+g; rows of
-  // padding heads / absent queries are zero.  Written with the swizzle the
-  // MMA descriptor expects.
-  for (int c = threadIdx.x; c < p.N * (DI / 16); c += 64 + 32 * EW) {
-    int row = c / (DI / 16), chunk = c % (DI / 16);
-    int g = row / p.HP, h = row % p.HP;
-    uint4 v = make_uint4(0, 0, 0, 0);
-    if (g < nq && h < p.H_I)
-      v = __ldg(reinterpret_cast<const uint4*>(
-          p.q_idx + (((int64_t)b * p.Q + q0 + g) * p.H_I + h) * DI + chunk * 16));
-    uint32_t lin = row * DI + chunk * 16;
-    uint32_t phys = lin ^ (((lin >> 7) & C::kSwzMask) << 4);
+  // The query tile in shared memory, with the swizzle the MMA descriptor
+  // expects (chunks past the registers' share are loaded here).
+  auto put_chunk = [&](int c, uint4 v) {
+    const uint32_t lin = (c / (DI / 16)) * DI + (c % (DI / 16)) * 16;
+    const uint32_t phys = lin ^ (((lin >> 7) & C::kSwzMask) << 4);
     *reinterpret_cast<uint4*>(qtile + phys) = v;
+  };
+#pragma unroll
+  for (int j = 0; j < kQPre; ++j) {
+    const int c = threadIdx.x + j * kThr;
+    if (c < nchunk) put_chunk(c, qpre[j]);
   }
-  for (int r = threadIdx.x; r < p.N; r += 64 + 32 * EW) {
-    int g = r / p.HP, h = r % p.HP;
-    float v = 0.f;
-    if (g < nq && h < p.H_I) {
-      int64_t o = ((int64_t)b * p.Q + q0 + g) * p.H_I + h;
-      v = __ldg(p.w + o) * __ldg(p.q_scale + o);
-    }
-    wq[r] = v;
+  for (int c = threadIdx.x + kQPre * kThr; c < nchunk; c += kThr) put_chunk(c, q_chunk(c));
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    const int r = threadIdx.x + j * kThr;
+    if (r < p.N) wq[r] = wpre[j] * spre[j];
   }
   if (kHist)
     for (int i = threadIdx.x; i < kScoreHistBins; i += 64 + 32 * EW) shist[i] = 0u;
@@ -194,13 +242,13 @@ __global__ void __launch_bounds__(64 + 32 * EW, EW == 4 ? 2 : 1)
   if (warp == 0) {
     // ------------------------------------------------------- TMA producer --
     if (elect_one()) {
-      tma_prefetch_desc(&kmap);
-      // Tiles of entries written before this call stream at once; the first
-      // tile with an entry that the previous kernel writes waits for it.
+      // Tiles of entries written before this call stream at once (the first
+      // ones were issued during the set-up); the first tile with an entry
+      // that the previous kernel writes waits for it.
       const int64_t safe = safe_bound(p, b);
       bool waited = false;
-      int it = 0;
-      for (int t = t_begin; t < t_end; ++t, ++it) {
+      int it = early_tiles(p, b, t_begin, t_end, C::kStages);
+      for (int t = t_begin + it; t < t_end; ++t, ++it) {
         int s = it % C::kStages;
         uint32_t ph = (it / C::kStages) & 1;
         if (!waited && (int64_t)(t + 1) * kTileRows > safe) {
@@ -459,11 +507,13 @@ cudaError_t launch_impl(const IndexLaunch& a, cudaStream_t stream) {
   if (EW == 8) occ = 1;  // 320 threads x ~130 registers: one CTA per SM
   int64_t groups = (int64_t)a.B * p.qgroups;
   if (groups > 65535) return cudaErrorInvalidConfiguration;
-  int64_t slots = (int64_t)a.num_sms * occ;
+  // Every CTA resident at once: the slots the call's earlier kernel holds
+  // (reserve_slots) are left out, so that no CTA starts only when it ends.
+  // The tiles are split evenly (chunk sizes differ by at most one).
+  const int64_t slots = std::max<int64_t>(1, (int64_t)a.num_sms * occ - a.reserve_slots);
   int chunks = 1;
   if (groups < slots) chunks = (int)std::max<int64_t>(1, std::min<int64_t>(p.ntiles, slots / groups));
-  p.tiles_per_chunk = (p.ntiles + chunks - 1) / chunks;
-  chunks = (p.ntiles + p.tiles_per_chunk - 1) / p.tiles_per_chunk;
+  p.nchunks = chunks;
 
   CUtensorMap kmap;
   e = make_tmap_2d(&kmap, a.key, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)a.B * a.N_cap, DI,

@@ -36,6 +36,8 @@ struct CompressLaunch {
   int chained;              // see launch_pdl
 };
 cudaError_t launch_compress(const CompressLaunch& c, cudaStream_t stream);
+// CTAs of launch_compress for these arguments.
+int compress_ctas(const CompressLaunch& c);
 
 // Lightning Indexer scores (tcgen05 kind::f8f6f4) over every (query, entry
 // tile).  Queries are grouped G per MMA (N = G * H_I <= 256).
@@ -64,6 +66,9 @@ struct IndexLaunch {
   // its visible scores by the top kScoreHistBits bits of their keys
   // (score_key) to hist[b * kScoreHistBins ..].  Null: no histogram.
   uint32_t* hist = nullptr;
+  // Slots (CTAs of this kernel's size) that the call's previous kernel keeps
+  // busy while this one starts: the grid leaves them out.
+  int reserve_slots = 0;
 };
 cudaError_t launch_index_scores(const IndexLaunch& a, cudaStream_t stream);
 
