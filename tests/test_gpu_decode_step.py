@@ -9,6 +9,8 @@ against the oracle's compression of the tokens up to its position; scores
 against the oracle fed the GPU's E4M3 keys; the top-k bit-exact against the
 oracle ranking the GPU's scores; attention against the oracle fed the GPU's
 selection and cache.  After the loop the whole cache is checked."""
+import math
+
 import numpy as np
 import pytest
 import torch
@@ -205,7 +207,8 @@ class _Step:
     def run(self, pos, qseed):
         w, B = self.w, self.B
         qi = synth.queries(configs.scaled(w, seed=qseed), Q=1, device=DEV)
-        out = torch.empty(B, w.H, w.D, dtype=torch.bfloat16, device=DEV)
+        out = torch.full((B, w.H, w.D), float("nan"), dtype=torch.bfloat16, device=DEV)
+        lse = torch.full((B, w.H), float("nan"), dtype=torch.float32, device=DEV)
         tidx = torch.full((B, w.k), -7, dtype=torch.int32, device=DEV)
         tcnt = torch.full((B,), -7, dtype=torch.int32, device=DEV)
         pos_t = torch.as_tensor(pos, dtype=torch.int64, device=DEV)
@@ -213,9 +216,11 @@ class _Step:
                                 None, self.w_si, self.b_pi, self.kv_c, self.key, self.ksc,
                                 qi["q"][:, 0].contiguous(), qi["q_idx"][:, 0].contiguous(),
                                 qi["q_scale"][:, 0].contiguous(), qi["w"][:, 0].contiguous(),
-                                qi["sink"], tidx, tcnt, out, ws=self.ws, dev_status=self.status)
+                                qi["sink"], tidx, tcnt, out, lse=lse, ws=self.ws,
+                                dev_status=self.status)
         torch.cuda.synchronize()
         assert self.status.item() == 0, self.status.item()
+        self.out, self.lse = out, lse
         return qi, tidx, tcnt
 
     def check(self, orc, pos, qi, tidx, tcnt, path_expect, n_sample=256):
@@ -246,6 +251,30 @@ class _Step:
         assert not hist.any(), "histogram not cleared"
         assert path.tolist() == list(path_expect), path
 
+    def check_attention(self, orc, pos, qi, tidx, tcnt):
+        """The step's attention output and LSE against the oracle fed the
+        GPU's selection and cache (the window tail of the token stream)."""
+        w, B = self.w, self.B
+        pos = np.asarray(pos)
+        lo = int(pos.min()) - w.W + 1
+        hi = int(pos.max()) + 1
+        tail = bits16(self.kv_tok[:, lo:hi])
+        q = qi["q"][:, 0].contiguous()
+        kw = {}
+        if w.yarn:  # the oracle's own YaRN table and logit gain
+            kw = dict(rope_freq=orc.yarn_inv_freq(w.rope_dim, *w.yarn),
+                      scale=orc.yarn_logit_gain(w.yarn[0]) / math.sqrt(w.d))
+        ro, rl = orc.mqa(bits16(q).reshape(B, 1, w.H, w.D), pos.reshape(B, 1), bits16(self.kv_c),
+                         tail, f32(qi["sink"]), w.m, w.W, w.rope_dim, tidx.cpu().numpy()[:, None],
+                         tcnt.cpu().numpy()[:, None], tok_base=lo, **kw)
+        got = self.out.double().cpu().numpy()
+        assert np.isfinite(got).all()
+        assert_attention_close(got, ro[:, 0], "decode step, Qhat from the top-k")
+        if w.yarn:
+            assert_lse_close(f32(self.lse), rl[:, 0], ro[:, 0], "decode-step LSE", kw["scale"])
+        else:
+            _check_lse(self.lse, rl[:, 0], ro[:, 0])
+
 
 def test_histogram_topk_csa_128k_shape(orc):
     """The timed 128K workload (8 sequences x 32768 entries, k = 1024):
@@ -262,6 +291,8 @@ def test_histogram_topk_csa_128k_shape(orc):
     for step in range(2):
         qi, tidx, tcnt = st.run(pos, w.seed + 1000 + step)
         st.check(orc, pos, qi, tidx, tcnt, [1] * w.B)
+        if step == 0:
+            st.check_attention(orc, pos, qi, tidx, tcnt)
     h0, _ = _ws_layout(w.B, st.N)
     for top_bin, path in ((4095, 2), (0, 1)):
         bad = torch.zeros(w.B, 4096, dtype=torch.int32, device=DEV)
@@ -280,6 +311,7 @@ def test_histogram_topk_csa_1m_shape(orc):
     pos = np.full(w.B, w.L - 1)
     qi, tidx, tcnt = st.run(pos, w.seed + 1000)
     st.check(orc, pos, qi, tidx, tcnt, [1] * w.B)
+    st.check_attention(orc, pos, qi, tidx, tcnt)
 
 
 @pytest.mark.parametrize("case", ["ties", "all_equal", "few_visible"])
@@ -308,3 +340,18 @@ def test_histogram_topk_structures(orc, case):
         expect = [0, 2]
     qi, tidx, tcnt = st.run(pos, w.seed + 1000)
     st.check(orc, pos, qi, tidx, tcnt, expect)
+    st.check_attention(orc, pos, qi, tidx, tcnt)
+
+
+def test_histogram_topk_flash_yarn(orc):
+    """V4-Flash shapes through the decode step ("DeepSeek V4-Pro" (llm-arch-kb),
+    "Family": 64 heads, top-512; YaRN RoPE): two sequences x 16384 entries at
+    different positions, on the histogram path, with the attention's Qhat
+    formed by the top-k kernel (one attention CTA per row and split)."""
+    w = configs.scaled(configs.CSA_FLASH_128K, B=2, L=65536)
+    st = _Step(w, w.L, seed=9)
+    st.compress_all(w.L)
+    pos = np.array([w.L - 1, w.L - 1 - 37])
+    qi, tidx, tcnt = st.run(pos, w.seed + 1000)
+    st.check(orc, pos, qi, tidx, tcnt, [1, 1])
+    st.check_attention(orc, pos, qi, tidx, tcnt)
