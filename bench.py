@@ -268,7 +268,7 @@ class Decode:
             s["kv_tok"] = torch.empty(B, L, d, dtype=torch.bfloat16, device=device)
             s["kv_tok"][:, L - tail:] = kv_src[:, L - tail:]
             s["kv_c"] = kv_c_src.clone()
-            s["q"] = synth.normal_bf16((B, w.H, d), w.seed + 1000 + r, "q", device)
+            q = synth.normal_bf16((B, w.H, d), w.seed + 1000 + r, "q", device)
             s["out"] = torch.empty(B, w.H, d, dtype=torch.bfloat16, device=device)
             s["ws_step"] = binding.workspace(self.p, op_step, 1, N, device)
             if w.csa:
@@ -277,12 +277,30 @@ class Decode:
                 s["key"] = key_src.clone()
                 s["ksc"] = ksc_src.clone()
                 qr = synth.queries(configs.scaled(w, seed=w.seed + 1000 + r), Q=1, device=device)
-                s["q_idx"], s["q_scale"], s["w"] = qr["q_idx"], qr["q_scale"], qr["w"]
+                # The step's query-side inputs in one buffer (one copy per
+                # step on the end-to-end path).
+                parts = [q, qr["q_idx"], qr["q_scale"], qr["w"]]
+                offs, o = [], 0
+                for t in parts:
+                    offs.append(o)
+                    o += (t.numel() * t.element_size() + 255) // 256 * 256
+                s["qin"] = torch.empty(o, dtype=torch.uint8, device=device)
+                views = []
+                for t, o0 in zip(parts, offs):
+                    nb = t.numel() * t.element_size()
+                    v = s["qin"][o0:o0 + nb].view(t.dtype).view(t.shape)
+                    v.copy_(t)
+                    views.append(v)
+                s["q"], s["q_idx"], s["q_scale"], s["w"] = views
+                s["q_idx3"] = s["q_idx"].view(B, w.H_I, w.D_I)
+                s["q_scale2"] = s["q_scale"].view(B, w.H_I)
+                s["w2"] = s["w"].view(B, w.H_I)
                 s["scores"] = torch.empty(B, 1, N, dtype=torch.float32, device=device)
                 s["tidx"] = torch.empty(B, 1, w.k, dtype=torch.int32, device=device)
                 s["tcnt"] = torch.empty(B, 1, dtype=torch.int32, device=device)
                 s["ws"] = binding.workspace(self.p, binding.OP_SPARSE_MQA, 1, N, device)
             else:
+                s["q"] = q
                 s["ws"] = binding.workspace(self.p, binding.OP_DENSE_MQA, 1, N, device)
             self.sets.append(s)
         del kv_src, idx_src
@@ -297,10 +315,9 @@ class Decode:
         if w.csa:
             b.csa_decode_step(p, self.pos, s["kv_tok"], s["idx_tok"], self.w_s, self.b_pos, None,
                               self.w_si, self.b_pi, s["kv_c"], s["key"], s["ksc"], s["q"],
-                              s["q_idx"].view(w.B, w.H_I, w.D_I), s["q_scale"].view(w.B, w.H_I),
-                              s["w"].view(w.B, w.H_I), self.sink, s["tidx"].view(w.B, w.k),
-                              s["tcnt"].view(w.B), s["out"], ws=s["ws_step"],
-                              dev_status=self.status)
+                              s["q_idx3"], s["q_scale2"], s["w2"], self.sink,
+                              s["tidx"].view(w.B, w.k), s["tcnt"].view(w.B), s["out"],
+                              ws=s["ws_step"], dev_status=self.status)
         else:
             b.hca_decode_step(p, self.pos, s["kv_tok"], self.w_s, self.b_pos, None, s["kv_c"],
                               s["q"], self.sink, s["out"], ws=s["ws_step"], dev_status=self.status)
@@ -333,6 +350,22 @@ class Decode:
             ("mqa", lambda: b.dense_mqa_decode(p, s["q"], self.pos, s["kv_c"], s["kv_tok"],
                                                self.sink, s["out"], ws=s["ws"], dev_status=st)),
         ]
+
+    def prepared_step(self, s):
+        """The step of input set s as a prepared public call (binding
+        CsaDecodeStep / HcaDecodeStep: the unchanging arguments converted
+        once); returns f(stream) that runs one step."""
+        b, w, p = self.binding, self.w, self.p
+        if w.csa:
+            f = b.CsaDecodeStep(p, s["kv_tok"], s["idx_tok"], self.w_s, self.b_pos, None, self.w_si,
+                                self.b_pi, s["kv_c"], s["key"], s["ksc"], self.sink,
+                                s["tidx"].view(w.B, w.k), s["tcnt"].view(w.B), s["ws_step"],
+                                dev_status=self.status)
+            return lambda stream: f(self.pos, s["q"], s["q_idx3"], s["q_scale2"], s["w2"],
+                                    s["out"], stream=stream)
+        f = b.HcaDecodeStep(p, s["kv_tok"], self.w_s, self.b_pos, None, s["kv_c"], self.sink,
+                            s["ws_step"], dev_status=self.status)
+        return lambda stream: f(self.pos, s["q"], s["out"], stream=stream)
 
     def launches_per_step(self):
         """Kernel launches of one step, counted from the kernel nodes of a
@@ -707,19 +740,20 @@ def run_e2e(st, K, W, barrier, rmax, rsum, world):
     memory, all inside the timed region."""
     torch = st.torch
     w, R = st.w, st.R
-    L, m = w.L, w.m
-    hq = [s["q"].cpu().pin_memory() for s in st.sets]
-    hkv = [s["kv_tok"][:, L - m:].cpu().pin_memory() for s in st.sets]
+    L = w.L
+    # CSA: the query-side inputs are one buffer (qin); HCA: the query.
+    qkey = "qin" if w.csa else "q"
+    hq = [s[qkey].cpu().pin_memory() for s in st.sets]
+    # The step's new token: one KV (and indexer) row per sequence at the
+    # step's position L - 1 (the block's earlier rows came with earlier steps).
+    hkv = [s["kv_tok"][:, L - 1:].cpu().pin_memory() for s in st.sets]
     hout = [torch.empty_like(s["out"], device="cpu").pin_memory() for s in st.sets]
-    extra = []
-    if w.csa:
-        extra = [(s["q_idx"].cpu().pin_memory(), s["q_scale"].cpu().pin_memory(),
-                  s["w"].cpu().pin_memory(), s["idx_tok"][:, L - m:].cpu().pin_memory())
-                 for s in st.sets]
+    hidx = [s["idx_tok"][:, L - 1:].cpu().pin_memory() for s in st.sets] if w.csa else []
     h2d = sum(t.numel() * t.element_size() for t in (hq[0], hkv[0]))
     if w.csa:
-        h2d += sum(t.numel() * t.element_size() for t in extra[0])
+        h2d += hidx[0].numel() * hidx[0].element_size()
     d2h = hout[0].numel() * hout[0].element_size()
+    steps = [st.prepared_step(s) for s in st.sets]
 
     # Copies run on their own streams: the inputs of step i+1 travel while
     # step i computes, and the output of step i returns while step i+1
@@ -738,14 +772,10 @@ def run_e2e(st, K, W, barrier, rmax, rsum, world):
         with torch.cuda.stream(up):
             if used[r]:
                 up.wait_event(done[r])  # the set's previous step has finished
-            s["q"].copy_(hq[r], non_blocking=True)
-            s["kv_tok"][:, L - m:].copy_(hkv[r], non_blocking=True)
+            s[qkey].copy_(hq[r], non_blocking=True)
+            s["kv_tok"][:, L - 1:].copy_(hkv[r], non_blocking=True)
             if w.csa:
-                a, b, c, d = extra[r]
-                s["q_idx"].copy_(a, non_blocking=True)
-                s["q_scale"].copy_(b, non_blocking=True)
-                s["w"].copy_(c, non_blocking=True)
-                s["idx_tok"][:, L - m:].copy_(d, non_blocking=True)
+                s["idx_tok"][:, L - 1:].copy_(hidx[r], non_blocking=True)
             copied[r].record(up)
 
     def compute(i):
@@ -753,7 +783,7 @@ def run_e2e(st, K, W, barrier, rmax, rsum, world):
         comp.wait_event(copied[r])
         if used[r]:
             comp.wait_event(fetched[r])  # the set's previous output has left
-        st.step(st.sets[r])
+        steps[r](comp)
         done[r].record(comp)
         used[r] = True
         with torch.cuda.stream(down):
@@ -781,8 +811,9 @@ def run_e2e(st, K, W, barrier, rmax, rsum, world):
     val, _ = aggregate(w.B * K, e0.elapsed_time(e1), world, rmax, rsum)
     return {"value": round(val, 1), "unit": "query-tokens/s", "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h,
-            "path": "direct public call per step (no graph); inputs from pinned host memory, "
-                    "output to pinned host memory, inside the timed region"}
+            "path": "direct public call per step (no graph; the binding's prepared "
+                    "CsaDecodeStep / HcaDecodeStep); inputs from pinned host memory, output to "
+                    "pinned host memory, inside the timed region"}
 
 
 # ---------------------------------------------------------------- prefill --

@@ -283,6 +283,50 @@ def csa_decode_step(p, pos_q, kv_tok, idx_tok, w_s, b_pos, gamma, w_s_idx, b_pos
         _stream(stream)))
 
 
+class CsaDecodeStep:
+    """csa_decode_step for a fixed set of sequences: the arguments that stay
+    the same from step to step (token buffers, caches, weights, sink and
+    gains, the selection outputs, workspace and status word) are checked and
+    converted once; each call passes the step's positions, queries and
+    outputs.  Same C entry point and the same device-side work as
+    csa_decode_step (argument marshalling only)."""
+
+    def __init__(self, p, kv_tok, idx_tok, w_s, b_pos, gamma, w_s_idx, b_pos_idx, kv_c, idx_key,
+                 idx_scale, sink, topk_idx, topk_cnt, ws, gamma_q=None, gamma_kv=None,
+                 dev_status=None):
+        self._fn = lib().csa_decode_step
+        self._keep = (p, kv_tok, idx_tok, w_s, b_pos, gamma, w_s_idx, b_pos_idx, kv_c, idx_key,
+                      idx_scale, sink, topk_idx, topk_cnt, ws, gamma_q, gamma_kv, dev_status)
+        self._head = (C.byref(p),)
+        self._mid = (_ptr(kv_tok), _ptr(idx_tok), kv_tok.shape[1], _ptr(w_s), _ptr(b_pos),
+                     _ptr(gamma), _ptr(w_s_idx), _ptr(b_pos_idx), _ptr(kv_c), _ptr(idx_key),
+                     _ptr(idx_scale), kv_c.shape[1])
+        self._sink = (_ptr(sink), _ptr(gamma_q), _ptr(gamma_kv), _ptr(topk_idx), _ptr(topk_cnt))
+        self._tail = (_ptr(ws), ws.numel() * ws.element_size(), _ptr(dev_status))
+
+    def __call__(self, pos_q, q, q_idx, q_scale, w, out, lse=None, stream=None):
+        _check(self._fn(*self._head, _ptr(pos_q), *self._mid, _ptr(q), _ptr(q_idx), _ptr(q_scale),
+                        _ptr(w), *self._sink, _ptr(out), _ptr(lse), *self._tail, _stream(stream)))
+
+
+class HcaDecodeStep:
+    """hca_decode_step for a fixed set of sequences (see CsaDecodeStep)."""
+
+    def __init__(self, p, kv_tok, w_s, b_pos, gamma, kv_c, sink, ws, gamma_q=None, gamma_kv=None,
+                 dev_status=None):
+        self._fn = lib().hca_decode_step
+        self._keep = (p, kv_tok, w_s, b_pos, gamma, kv_c, sink, ws, gamma_q, gamma_kv, dev_status)
+        self._head = (C.byref(p),)
+        self._mid = (_ptr(kv_tok), kv_tok.shape[1], _ptr(w_s), _ptr(b_pos), _ptr(gamma),
+                     _ptr(kv_c), kv_c.shape[1])
+        self._gains = (_ptr(sink), _ptr(gamma_q), _ptr(gamma_kv))
+        self._tail = (_ptr(ws), ws.numel() * ws.element_size(), _ptr(dev_status))
+
+    def __call__(self, pos_q, q, out, lse=None, stream=None):
+        _check(self._fn(*self._head, _ptr(pos_q), *self._mid, _ptr(q), *self._gains, _ptr(out),
+                        _ptr(lse), *self._tail, _stream(stream)))
+
+
 def hca_decode_step(p, pos_q, kv_tok, w_s, b_pos, gamma, kv_c, q, sink, out, gamma_q=None,
                     gamma_kv=None, lse=None, ws=None, dev_status=None, stream=None):
     """One HCA decode step (newest-block compression, dense MQA) for B

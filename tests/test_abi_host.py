@@ -247,3 +247,17 @@ def test_grouped_out_proj_workspace_grows_with_tokens(L):
     assert 0 < a < b
     # At least the bf16 intermediate y.
     assert b >= 4096 * 16 * 1024 * 2
+
+
+def test_prepared_decode_steps_reject_host_tensors(L):
+    """CsaDecodeStep / HcaDecodeStep check their tensors like the plain calls
+    (host tensors are refused before anything reaches the library)."""
+    import torch
+    from compressed_sparse_kv_04_b200 import configs
+    w = configs.scaled(configs.CSA_128K, B=1, L=64)
+    p = binding.params_for(w)
+    t = torch.zeros(16)
+    with pytest.raises(ValueError):
+        binding.CsaDecodeStep(p, t, t, t, t, None, t, t, t, t, t, t, t, t, t)
+    with pytest.raises(ValueError):
+        binding.HcaDecodeStep(p, t, t, t, None, t, t, t)

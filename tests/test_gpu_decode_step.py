@@ -355,3 +355,70 @@ def test_histogram_topk_flash_yarn(orc):
     qi, tidx, tcnt = st.run(pos, w.seed + 1000)
     st.check(orc, pos, qi, tidx, tcnt, [1, 1])
     st.check_attention(orc, pos, qi, tidx, tcnt)
+
+
+def test_prepared_decode_steps_match_the_plain_calls():
+    """binding.CsaDecodeStep / HcaDecodeStep (the unchanging arguments
+    converted once) run the same C entry points: the same outputs, bit for
+    bit, as csa_decode_step / hca_decode_step."""
+    for csa in (True, False):
+        w = configs.scaled(configs.CSA_128K if csa else configs.HCA_1M, B=2, L=4096)
+        p = binding.params_for(w)
+        kv_tok, idx_tok = synth.token_streams(w, device=DEV)
+        w_s, b_pos = synth.pool_params(w, DEV)
+        N = w.L // w.m
+        kv_c = torch.zeros(w.B, N, w.d, dtype=torch.bfloat16, device=DEV)
+        qi = synth.queries(w, Q=1, device=DEV)
+        q = qi["q"][:, 0].contiguous()
+        pos = torch.tensor([w.L - 1, w.L - 7], dtype=torch.int64, device=DEV)
+        status = torch.zeros(1, dtype=torch.int32, device=DEV)
+        outs = []
+        if csa:
+            w_si, b_pi = synth.pool_params(w, DEV, indexer=True)
+            key = torch.zeros(w.B, N, w.D_I, dtype=torch.uint8, device=DEV)
+            ksc = torch.zeros(w.B, N, dtype=torch.float32, device=DEV)
+            ctx = torch.full((w.B,), w.L, dtype=torch.int64, device=DEV)
+            binding.csa_compress(p, kv_tok, ctx, w_s, b_pos, None, 0, N, kv_c, idx_tok, w_si, b_pi,
+                                 key, ksc, dev_status=status)
+            ws = binding.workspace(p, binding.OP_CSA_DECODE_STEP, 1, N)
+            args = (q, qi["q_idx"][:, 0].contiguous(), qi["q_scale"][:, 0].contiguous(),
+                    qi["w"][:, 0].contiguous())
+            tidx = torch.zeros(w.B, w.k, dtype=torch.int32, device=DEV)
+            tcnt = torch.zeros(w.B, dtype=torch.int32, device=DEV)
+            for prepared in (False, True):
+                out = torch.full((w.B, w.H, w.D), float("nan"), dtype=torch.bfloat16, device=DEV)
+                lse = torch.full((w.B, w.H), float("nan"), dtype=torch.float32, device=DEV)
+                if prepared:
+                    f = binding.CsaDecodeStep(p, kv_tok, idx_tok, w_s, b_pos, None, w_si, b_pi,
+                                              kv_c, key, ksc, qi["sink"], tidx, tcnt, ws,
+                                              dev_status=status)
+                    f(pos, *args, out, lse=lse)
+                else:
+                    binding.csa_decode_step(p, pos, kv_tok, idx_tok, w_s, b_pos, None, w_si, b_pi,
+                                            kv_c, key, ksc, *args, qi["sink"], tidx, tcnt, out,
+                                            lse=lse, ws=ws, dev_status=status)
+                torch.cuda.synchronize()
+                outs.append((out.clone(), lse.clone(), tidx.clone()))
+        else:
+            ctx = torch.full((w.B,), w.L, dtype=torch.int64, device=DEV)
+            binding.hca_compress(p, kv_tok, ctx, w_s, b_pos, None, 0, N, kv_c, dev_status=status)
+            ws = binding.workspace(p, binding.OP_HCA_DECODE_STEP, 1, N)
+            for prepared in (False, True):
+                out = torch.full((w.B, w.H, w.D), float("nan"), dtype=torch.bfloat16, device=DEV)
+                lse = torch.full((w.B, w.H), float("nan"), dtype=torch.float32, device=DEV)
+                if prepared:
+                    f = binding.HcaDecodeStep(p, kv_tok, w_s, b_pos, None, kv_c, qi["sink"], ws,
+                                              dev_status=status)
+                    f(pos, q, out, lse=lse)
+                else:
+                    binding.hca_decode_step(p, pos, kv_tok, w_s, b_pos, None, kv_c, q, qi["sink"],
+                                            out, lse=lse, ws=ws, dev_status=status)
+                torch.cuda.synchronize()
+                outs.append((out.clone(), lse.clone(), None))
+        assert status.item() == 0
+        (o0, l0, t0), (o1, l1, t1) = outs
+        assert torch.isfinite(o0.float()).all()
+        assert torch.equal(o0.view(torch.int16), o1.view(torch.int16))
+        assert torch.equal(l0, l1)
+        if csa:
+            assert torch.equal(t0, t1)
