@@ -422,3 +422,16 @@ def test_prepared_decode_steps_match_the_plain_calls():
         assert torch.equal(l0, l1)
         if csa:
             assert torch.equal(t0, t1)
+
+
+def test_histogram_topk_single_sequence(orc):
+    """One sequence x 16384 entries, k = 512: the widest top-k cluster per row
+    and one indexer chunk per tile; the histogram path, bit-exact, with the
+    step's attention against the oracle."""
+    w = configs.scaled(configs.CSA_128K, B=1, k=512, L=65536)
+    st = _Step(w, w.L, seed=11)
+    st.compress_all(w.L)
+    pos = np.array([w.L - 2])
+    qi, tidx, tcnt = st.run(pos, w.seed + 1000)
+    st.check(orc, pos, qi, tidx, tcnt, [1])
+    st.check_attention(orc, pos, qi, tidx, tcnt)
