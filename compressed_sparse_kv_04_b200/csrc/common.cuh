@@ -385,6 +385,15 @@ CSA_DEV float2 fma_f32x2(float2 a, float2 b, float2 c) {
   return *reinterpret_cast<const float2*>(&d);
 }
 
+// d = a * b on both lanes of a pair (two fp32 multiplies, each rounded once).
+CSA_DEV float2 mul_f32x2(float2 a, float2 b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;"
+      : "=l"(d)
+      : "l"(*reinterpret_cast<const uint64_t*>(&a)), "l"(*reinterpret_cast<const uint64_t*>(&b)));
+  return *reinterpret_cast<const float2*>(&d);
+}
+
 CSA_DEV float warp_sum(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);

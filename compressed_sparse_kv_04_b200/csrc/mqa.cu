@@ -748,44 +748,46 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
       }
       const bool qok = wait_all(qfull, 0, p, abort_flag);
-      float a4[4] = {0.f, 0.f, 0.f, 0.f};  // independent chains, loads in flight
+      // Sum of squares in packed FMAs: word e of each 16-byte unit in pair
+      // accumulator e (its low and high halves in the two lanes).
+      float2 a2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                      make_float2(0.f, 0.f)};
 #pragma unroll 8
       for (int c = 0; c < NU; ++c) {
         const uint4 v = *reinterpret_cast<const uint4*>(qs + tile_off(hl, d_half + 8 * c));
         const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const float lo = bf16_lo(w4[e]), hi = bf16_hi(w4[e]);
-          a4[e] = fmaf(lo, lo, fmaf(hi, hi, a4[e]));
+          const float2 x = make_float2(bf16_lo(w4[e]), bf16_hi(w4[e]));
+          a2[e] = fma_f32x2(x, x, a2[e]);
         }
       }
-      float ss = (a4[0] + a4[1]) + (a4[2] + a4[3]);
+      float ss = ((a2[0].x + a2[0].y) + (a2[1].x + a2[1].y)) +
+                 ((a2[2].x + a2[2].y) + (a2[3].x + a2[3].y));
       ss += __shfl_xor_sync(0xffffffffu, ss, 16);  // the row's other half
       const float inv = (head_ok && qok) ? 1.0f / sqrtf(ss / (float)D + p.eps) : 0.f;
       const float* gq = gam_s + hf * (D / 2);
       constexpr int kChunks = D / 128;  // 64-dim chunks per half row
 #pragma unroll 1
       for (int c = 0; c < kChunks; ++c) {
+        // x = (q * inv) * gamma, two dims per packed multiply.
         float x[64];
+        const float2 inv2 = make_float2(inv, inv);
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
           const uint4 v =
               *reinterpret_cast<const uint4*>(qs + tile_off(hl, d_half + 64 * c + 8 * u));
           const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+          const float4 ga = *reinterpret_cast<const float4*>(gq + 64 * c + 8 * u);
+          const float4 gb = *reinterpret_cast<const float4*>(gq + 64 * c + 8 * u + 4);
+          const float2 g2[4] = {make_float2(ga.x, ga.y), make_float2(ga.z, ga.w),
+                                make_float2(gb.x, gb.y), make_float2(gb.z, gb.w)};
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            x[8 * u + 2 * e] = bf16_lo(w4[e]) * inv;
-            x[8 * u + 2 * e + 1] = bf16_hi(w4[e]) * inv;
-          }
-        }
-        {
-#pragma unroll
-          for (int j = 0; j < 64; j += 4) {
-            const float4 g = *reinterpret_cast<const float4*>(gq + 64 * c + j);
-            x[j] *= g.x;
-            x[j + 1] *= g.y;
-            x[j + 2] *= g.z;
-            x[j + 3] *= g.w;
+            const float2 y =
+                mul_f32x2(mul_f32x2(make_float2(bf16_lo(w4[e]), bf16_hi(w4[e])), inv2), g2[e]);
+            x[8 * u + 2 * e] = y.x;
+            x[8 * u + 2 * e + 1] = y.y;
           }
         }
         if constexpr (R > 0) {
