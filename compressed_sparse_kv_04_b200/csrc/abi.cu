@@ -126,6 +126,21 @@ int splits_for(const csa_params* p, csa_op op, int rows, int64_t N_cap, int rese
                                 sms - reserve >= 2 ? sms - reserve : sms, p->H);
 }
 
+// SMs the CSA decode step's attention leaves to its top-k.  The attention
+// is launched while the top-k still runs; CTAs beyond the SMs the top-k
+// leaves free start only when it ends.  Where every attention CTA fits
+// beside the top-k at the cost of at most one more 64-entry tile per CTA,
+// the splits are sized for the free SMs.
+int decode_step_reserve(const csa_params* p, int64_t N_cap) {
+  const int r = csa::topk_hist_ctas(p->B, N_cap);
+  if (r <= 0) return 0;
+  const int s0 = splits_for(p, CSA_OP_SPARSE_MQA, p->B, N_cap);
+  const int s1 = splits_for(p, CSA_OP_SPARSE_MQA, p->B, N_cap, r);
+  const int64_t tiles = ((int64_t)p->k + 63) / 64 + (p->window + 63) / 64;
+  const int64_t t0 = (tiles + s0 - 1) / s0, t1 = (tiles + s1 - 1) / s1;
+  return (s1 < s0 && t1 <= t0 + 1) ? r : 0;
+}
+
 }  // namespace
 
 namespace csa {
@@ -203,8 +218,10 @@ size_t csa_workspace_bytes(const csa_params* p, csa_op op, int Q, int64_t N_cap)
     }
     case CSA_OP_CSA_DECODE_STEP:
       return scores_bytes(p->B, N_cap) + hist_bytes(p->B) +
-             csa::mqa_workspace_bytes(p->B, splits_for(p, CSA_OP_SPARSE_MQA, p->B, N_cap), p->H,
-                                      p->d) +
+             csa::mqa_workspace_bytes(p->B,
+                                      splits_for(p, CSA_OP_SPARSE_MQA, p->B, N_cap,
+                                                 decode_step_reserve(p, N_cap)),
+                                      p->H, p->d) +
              512;
     case CSA_OP_HCA_DECODE_STEP:
       return csa::mqa_workspace_bytes(p->B, splits_for(p, CSA_OP_DENSE_MQA, p->B, N_cap, p->B),
@@ -717,7 +734,8 @@ csa_status csa_decode_step(const csa_params* p, const int64_t* pos_q, const void
   char* rest = static_cast<char*>(ws) + head;
   return mqa_common(fn, p, CSA_OP_SPARSE_MQA, p->B, 1, q, pos_q, 0, kv_c, N_cap, topk_idx,
                     topk_cnt, kv_tok, L_cap, sink, gamma_q, gamma_kv, out, lse, rest,
-                    ws_bytes - head, dev_status, s, 1);
+                    ws_bytes - head, dev_status, s, 1, nullptr, 0,
+                    decode_step_reserve(p, N_cap));
 }
 
 csa_status hca_decode_step(const csa_params* p, const int64_t* pos_q, const void* kv_tok,

@@ -101,6 +101,9 @@ cudaError_t launch_topk(const TopkLaunch& a, cudaStream_t stream);
 // True when launch_topk takes the histogram path for these rows (one
 // cluster of CTAs per row): only then should the indexer build one.
 bool topk_uses_hist(int rows, int64_t N_cap);
+// CTAs (one SM each) of the histogram top-k for these rows; 0 when it does
+// not run.
+int topk_hist_ctas(int rows, int64_t N_cap);
 
 // Context split over ranks: a shard's candidates (score, sequence index) and
 // the global top-k over all ranks' candidates.

@@ -988,6 +988,38 @@ bool topk_uses_hist(int rows, int64_t N_cap) {
   return rows >= 1 && rows <= 65535 && !row_path(rows, N_cap) && N_cap <= 8 * 32768;
 }
 
+// Cluster size of the radix (hist false) or histogram kernel for these rows,
+// with the kernel's shared-memory limit set on the way; 0 if the rows do not
+// fit.  Slices of at most 32768 scores; small batches spread each row over
+// more CTAs (slices of at least 4096 scores), up to 16 where 16-CTA clusters
+// fit.  The histogram kernel's HistShared follows the largest slice.
+static int cluster_size(int rows, int64_t N_cap, bool hist) {
+  const int need = (int)((N_cap + 32767) / 32768);
+  if (need > 8 || rows < 1) return 0;
+  auto kern = hist ? topk_hist_kernel : topk_kernel<kDigitBits, false>;
+  using S = Shared<(1 << kDigitBits)>;
+  const int64_t slice_max = (N_cap + need - 1) / need;
+  const size_t hist_off = (sizeof(S) + (size_t)slice_max * 4 + 15) / 16 * 16;
+  const size_t smem_max = hist ? hist_off + sizeof(HistShared) : sizeof(S) + (size_t)slice_max * 4;
+  if (ensure_smem_attr(reinterpret_cast<const void*>(kern), hist ? 17 : 2, smem_max) !=
+      cudaSuccess)
+    return 0;
+  const int limit = max_cluster(reinterpret_cast<const void*>(kern), smem_max, hist ? 1 : 0);
+  int C = 1;
+  while (C < need) C <<= 1;
+  const int sms = device_sm_count();
+  if (rows < sms) {
+    const int fill = std::max(1, sms / rows);
+    while (C * 2 <= limit && C * 2 <= fill && N_cap / (C * 2) >= 4096) C *= 2;
+  }
+  return C;
+}
+
+int topk_hist_ctas(int rows, int64_t N_cap) {
+  if (!topk_uses_hist(rows, N_cap)) return 0;
+  return rows * cluster_size(rows, N_cap, true);
+}
+
 static cudaError_t launch_topk_impl(const TopkLaunch& a, cudaStream_t stream) {
   if (a.rows < 1) return cudaSuccess;
   if (a.rows > 65535 || a.k > kMaxK) return cudaErrorInvalidConfiguration;
@@ -1012,28 +1044,11 @@ static cudaError_t launch_topk_impl(const TopkLaunch& a, cudaStream_t stream) {
     return launch_pdl(topk_row_kernel, dim3(a.rows), dim3(kThreads), smem, stream, 0, a.chained,
                       p);
   }
-  const int sms = device_sm_count();
-  const int need = (int)((a.N_cap + 32767) / 32768);
-  if (need > 8) return cudaErrorInvalidValue;
   const bool hist = a.hist != nullptr;
   auto kern = hist ? topk_hist_kernel : topk_kernel<kDigitBits, false>;
   using S = Shared<(1 << kDigitBits)>;
-  // Slices of at most 32768 scores; small batches spread each row over more
-  // CTAs (slices of at least 4096 scores), up to 16 where 16-CTA clusters fit.
-  // The histogram kernel's HistShared follows the largest slice.
-  const int64_t slice_max = (a.N_cap + need - 1) / need;
-  const size_t hist_off = (sizeof(S) + (size_t)slice_max * 4 + 15) / 16 * 16;
-  const size_t smem_max = hist ? hist_off + sizeof(HistShared) : sizeof(S) + (size_t)slice_max * 4;
-  cudaError_t e =
-      ensure_smem_attr(reinterpret_cast<const void*>(kern), hist ? 17 : 2, smem_max);
-  if (e != cudaSuccess) return e;
-  const int limit = max_cluster(reinterpret_cast<const void*>(kern), smem_max, hist ? 1 : 0);
-  int C = 1;
-  while (C < need) C <<= 1;
-  if (a.rows < sms) {
-    const int fill = std::max(1, sms / a.rows);
-    while (C * 2 <= limit && C * 2 <= fill && a.N_cap / (C * 2) >= 4096) C *= 2;
-  }
+  const int C = cluster_size(a.rows, a.N_cap, hist);
+  if (C == 0) return cudaErrorInvalidValue;
   Params p{};
   p.Q = a.Q;
   p.m = a.m;
