@@ -351,21 +351,21 @@ class Decode:
                                                self.sink, s["out"], ws=s["ws"], dev_status=st)),
         ]
 
-    def prepared_step(self, s):
-        """The step of input set s as a prepared public call (binding
-        CsaDecodeStep / HcaDecodeStep: the unchanging arguments converted
-        once); returns f(stream) that runs one step."""
+    def prepared_step(self, s, stream):
+        """The step of input set s as a prepared public call bound to its
+        buffers (binding CsaDecodeStep / HcaDecodeStep .bind: arguments
+        converted once); returns f() that runs one step on `stream`."""
         b, w, p = self.binding, self.w, self.p
         if w.csa:
             f = b.CsaDecodeStep(p, s["kv_tok"], s["idx_tok"], self.w_s, self.b_pos, None, self.w_si,
                                 self.b_pi, s["kv_c"], s["key"], s["ksc"], self.sink,
                                 s["tidx"].view(w.B, w.k), s["tcnt"].view(w.B), s["ws_step"],
                                 dev_status=self.status)
-            return lambda stream: f(self.pos, s["q"], s["q_idx3"], s["q_scale2"], s["w2"],
-                                    s["out"], stream=stream)
+            return f.bind(self.pos, s["q"], s["q_idx3"], s["q_scale2"], s["w2"], s["out"],
+                          stream=stream)
         f = b.HcaDecodeStep(p, s["kv_tok"], self.w_s, self.b_pos, None, s["kv_c"], self.sink,
                             s["ws_step"], dev_status=self.status)
-        return lambda stream: f(self.pos, s["q"], s["out"], stream=stream)
+        return f.bind(self.pos, s["q"], s["out"], stream=stream)
 
     def launches_per_step(self):
         """Kernel launches of one step, counted from the kernel nodes of a
@@ -749,18 +749,26 @@ def run_e2e(st, K, W, barrier, rmax, rsum, world):
     hkv = [s["kv_tok"][:, L - 1:].cpu().pin_memory() for s in st.sets]
     hout = [torch.empty_like(s["out"], device="cpu").pin_memory() for s in st.sets]
     hidx = [s["idx_tok"][:, L - 1:].cpu().pin_memory() for s in st.sets] if w.csa else []
-    h2d = sum(t.numel() * t.element_size() for t in (hq[0], hkv[0]))
-    if w.csa:
-        h2d += hidx[0].numel() * hidx[0].element_size()
-    d2h = hout[0].numel() * hout[0].element_size()
-    steps = [st.prepared_step(s) for s in st.sets]
 
     # Copies run on their own streams: the inputs of step i+1 travel while
     # step i computes, and the output of step i returns while step i+1
     # computes (each step has its own input set and its own host output
-    # buffer, so nothing is overwritten while in use).
+    # buffer, so nothing is overwritten while in use).  Copies and steps are
+    # the binding's prepared calls (csa_copy_async / csa_copy_rows_async and
+    # the bound decode step): one library call each, arguments converted once.
     comp = torch.cuda.current_stream()
     up, down = torch.cuda.Stream(), torch.cuda.Stream()
+    PC = st.binding.PreparedCopy
+    ups = []
+    for r, s in enumerate(st.sets):
+        c = [PC(s[qkey], hq[r], up), PC(s["kv_tok"][:, L - 1:], hkv[r], up)]
+        if w.csa:
+            c.append(PC(s["idx_tok"][:, L - 1:], hidx[r], up))
+        ups.append(c)
+    downs = [PC(hout[r], s["out"], down) for r, s in enumerate(st.sets)]
+    h2d = sum(c.bytes for c in ups[0])
+    d2h = downs[0].bytes
+    steps = [st.prepared_step(s, comp) for s in st.sets]
     copied = [torch.cuda.Event() for _ in range(R)]
     done = [torch.cuda.Event() for _ in range(R)]
     fetched = [torch.cuda.Event() for _ in range(R)]
@@ -768,28 +776,23 @@ def run_e2e(st, K, W, barrier, rmax, rsum, world):
 
     def upload(i):
         r = i % R
-        s = st.sets[r]
-        with torch.cuda.stream(up):
-            if used[r]:
-                up.wait_event(done[r])  # the set's previous step has finished
-            s[qkey].copy_(hq[r], non_blocking=True)
-            s["kv_tok"][:, L - 1:].copy_(hkv[r], non_blocking=True)
-            if w.csa:
-                s["idx_tok"][:, L - 1:].copy_(hidx[r], non_blocking=True)
-            copied[r].record(up)
+        if used[r]:
+            up.wait_event(done[r])  # the set's previous step has finished
+        for c in ups[r]:
+            c()
+        copied[r].record(up)
 
     def compute(i):
         r = i % R
         comp.wait_event(copied[r])
         if used[r]:
             comp.wait_event(fetched[r])  # the set's previous output has left
-        steps[r](comp)
+        steps[r]()
         done[r].record(comp)
         used[r] = True
-        with torch.cuda.stream(down):
-            down.wait_event(done[r])
-            hout[r].copy_(st.sets[r]["out"], non_blocking=True)
-            fetched[r].record(down)
+        down.wait_event(done[r])
+        downs[r]()
+        fetched[r].record(down)
 
     def run(n):
         up.wait_stream(comp)
@@ -811,9 +814,11 @@ def run_e2e(st, K, W, barrier, rmax, rsum, world):
     val, _ = aggregate(w.B * K, e0.elapsed_time(e1), world, rmax, rsum)
     return {"value": round(val, 1), "unit": "query-tokens/s", "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h,
-            "path": "direct public call per step (no graph; the binding's prepared "
-                    "CsaDecodeStep / HcaDecodeStep); inputs from pinned host memory, output to "
-                    "pinned host memory, inside the timed region"}
+            "path": "direct public calls per step (no graph): the binding's prepared "
+                    "CsaDecodeStep / HcaDecodeStep bound to the set's buffers, and prepared "
+                    "copies (csa_copy_async / csa_copy_rows_async) of the inputs from pinned "
+                    "host memory and of the output to pinned host memory, inside the timed "
+                    "region"}
 
 
 # ---------------------------------------------------------------- prefill --

@@ -28,7 +28,7 @@ EXPORTS = ["csa_version", "csa_last_error", "csa_workspace_bytes", "hca_compress
            "lightning_index_topk_static", "csa_rope_yarn", "hca_prefill_chunk",
            "csa_decode_step", "hca_decode_step", "grouped_out_proj",
            "grouped_out_proj_workspace_bytes", "csa_shard_candidates", "csa_merge_candidates",
-           "sparse_mqa_partials", "mqa_merge_partials"]
+           "sparse_mqa_partials", "mqa_merge_partials", "csa_copy_async", "csa_copy_rows_async"]
 
 
 class CsaError(RuntimeError):
@@ -101,6 +101,8 @@ def _declare(L):
     L.sparse_mqa_partials.argtypes = [P, i32, vp, vp, vp, i64, vp, vp, vp, i64, vp, vp, vp, vp,
                                       vp, vp]
     L.mqa_merge_partials.argtypes = [P, i32, vp, vp, vp, vp, vp, vp, vp, vp]
+    L.csa_copy_async.argtypes = [vp, vp, sz, vp]
+    L.csa_copy_rows_async.argtypes = [vp, sz, vp, sz, sz, sz, vp]
     for name in EXPORTS[3:]:
         if name != "grouped_out_proj_workspace_bytes":
             getattr(L, name).restype = i32
@@ -304,9 +306,23 @@ class CsaDecodeStep:
         self._sink = (_ptr(sink), _ptr(gamma_q), _ptr(gamma_kv), _ptr(topk_idx), _ptr(topk_cnt))
         self._tail = (_ptr(ws), ws.numel() * ws.element_size(), _ptr(dev_status))
 
+    def _args(self, pos_q, q, q_idx, q_scale, w, out, lse, stream):
+        return (*self._head, _ptr(pos_q), *self._mid, _ptr(q), _ptr(q_idx), _ptr(q_scale),
+                _ptr(w), *self._sink, _ptr(out), _ptr(lse), *self._tail, _stream(stream))
+
     def __call__(self, pos_q, q, q_idx, q_scale, w, out, lse=None, stream=None):
-        _check(self._fn(*self._head, _ptr(pos_q), *self._mid, _ptr(q), _ptr(q_idx), _ptr(q_scale),
-                        _ptr(w), *self._sink, _ptr(out), _ptr(lse), *self._tail, _stream(stream)))
+        _check(self._fn(*self._args(pos_q, q, q_idx, q_scale, w, out, lse, stream)))
+
+    def bind(self, pos_q, q, q_idx, q_scale, w, out, lse=None, stream=None):
+        """The step with its per-step buffers fixed as well (a decode loop
+        that writes each step's positions and queries into the same
+        buffers): returns f() that runs one step on `stream`."""
+        fn, args = self._fn, self._args(pos_q, q, q_idx, q_scale, w, out, lse, stream)
+        keep = (self, pos_q, q, q_idx, q_scale, w, out, lse, stream)
+
+        def run(_keep=keep):
+            _check(fn(*args))
+        return run
 
 
 class HcaDecodeStep:
@@ -322,9 +338,67 @@ class HcaDecodeStep:
         self._gains = (_ptr(sink), _ptr(gamma_q), _ptr(gamma_kv))
         self._tail = (_ptr(ws), ws.numel() * ws.element_size(), _ptr(dev_status))
 
+    def _args(self, pos_q, q, out, lse, stream):
+        return (*self._head, _ptr(pos_q), *self._mid, _ptr(q), *self._gains, _ptr(out),
+                _ptr(lse), *self._tail, _stream(stream))
+
     def __call__(self, pos_q, q, out, lse=None, stream=None):
-        _check(self._fn(*self._head, _ptr(pos_q), *self._mid, _ptr(q), *self._gains, _ptr(out),
-                        _ptr(lse), *self._tail, _stream(stream)))
+        _check(self._fn(*self._args(pos_q, q, out, lse, stream)))
+
+    def bind(self, pos_q, q, out, lse=None, stream=None):
+        """The step with its per-step buffers fixed (see CsaDecodeStep.bind)."""
+        fn, args = self._fn, self._args(pos_q, q, out, lse, stream)
+        keep = (self, pos_q, q, out, lse, stream)
+
+        def run(_keep=keep):
+            _check(fn(*args))
+        return run
+
+
+def _rows_of(t):
+    """(rows, row_bytes, pitch_bytes) of a tensor whose first dimension
+    strides over rows that are each contiguous."""
+    if t.dim() == 0:
+        return 1, t.element_size(), t.element_size()
+    inner = t[0] if t.shape[0] > 0 else t
+    if t.shape[0] > 0 and not inner.is_contiguous():
+        raise ValueError("each row (first-dimension slice) must be contiguous")
+    row = (t.numel() // max(1, t.shape[0])) * t.element_size()
+    pitch = t.stride(0) * t.element_size() if t.shape[0] > 1 else row
+    return t.shape[0], row, pitch
+
+
+class PreparedCopy:
+    """One asynchronous copy between two tensors of the same shape and dtype
+    (page-locked host <-> device, either direction) with its addresses and
+    stream fixed: csa_copy_async when both are contiguous, else
+    csa_copy_rows_async over the first dimension (each row contiguous, e.g.
+    kv_tok[:, pos:pos+1] of a [B, L_cap, d] token buffer).  f() enqueues it."""
+
+    def __init__(self, dst, src, stream=None):
+        if dst.shape != src.shape or dst.dtype != src.dtype:
+            raise ValueError(f"copy between {tuple(src.shape)} {src.dtype} and "
+                             f"{tuple(dst.shape)} {dst.dtype}")
+        for t in (dst, src):
+            if not t.is_cuda and not t.is_pinned():
+                raise ValueError("host tensors of a prepared copy must be page-locked")
+        self._keep = (dst, src, stream)
+        L = lib()
+        st = _stream(stream)
+        if dst.is_contiguous() and src.is_contiguous():
+            fn = L.csa_copy_async
+            args = (C.c_void_p(dst.data_ptr()), C.c_void_p(src.data_ptr()),
+                    dst.numel() * dst.element_size(), st)
+        else:
+            rows, row, dp = _rows_of(dst)
+            _, srow, sp = _rows_of(src)
+            fn = L.csa_copy_rows_async
+            args = (C.c_void_p(dst.data_ptr()), dp, C.c_void_p(src.data_ptr()), sp, row, rows, st)
+        self.bytes = dst.numel() * dst.element_size()
+        self._fn, self._args = fn, args
+
+    def __call__(self):
+        _check(self._fn(*self._args))
 
 
 def hca_decode_step(p, pos_q, kv_tok, w_s, b_pos, gamma, kv_c, q, sink, out, gamma_q=None,

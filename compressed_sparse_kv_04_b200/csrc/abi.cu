@@ -194,6 +194,31 @@ csa_status csa_rope_yarn(int rope_dim, double base, double factor, double beta_f
 
 const char* csa_last_error(void) { return g_err; }
 
+csa_status csa_copy_async(void* dst, const void* src, size_t bytes, void* stream) {
+  if (bytes == 0) return CSA_OK;
+  if (!dst || !src)
+    return fail(CSA_ERR_INVALID_ARG, "csa_copy_async: NULL address for %zu bytes", bytes);
+  cudaError_t e = cudaMemcpyAsync(dst, src, bytes, cudaMemcpyDefault,
+                                  static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess)
+    return fail(CSA_ERR_CUDA, "csa_copy_async: %s", cudaGetErrorString(e));
+  return CSA_OK;
+}
+
+csa_status csa_copy_rows_async(void* dst, size_t dst_pitch, const void* src, size_t src_pitch,
+                               size_t row_bytes, size_t rows, void* stream) {
+  const char* fn = "csa_copy_rows_async";
+  if (row_bytes == 0 || rows == 0) return CSA_OK;
+  if (!dst || !src) return fail(CSA_ERR_INVALID_ARG, "%s: NULL address", fn);
+  if (dst_pitch < row_bytes || src_pitch < row_bytes)
+    return fail(CSA_ERR_INVALID_ARG, "%s: pitches %zu / %zu below the row of %zu bytes", fn,
+                dst_pitch, src_pitch, row_bytes);
+  cudaError_t e = cudaMemcpy2DAsync(dst, dst_pitch, src, src_pitch, row_bytes, rows,
+                                    cudaMemcpyDefault, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(CSA_ERR_CUDA, "%s: %s", fn, cudaGetErrorString(e));
+  return CSA_OK;
+}
+
 size_t csa_workspace_bytes(const csa_params* p, csa_op op, int Q, int64_t N_cap) {
   const char* fn = "csa_workspace_bytes";
   if (check_common(fn, p) != CSA_OK) return 0;

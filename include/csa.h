@@ -119,6 +119,26 @@ int csa_version(void);
 const char* csa_last_error(void);
 
 /* ---------------------------------------------------------------------------
+ * Transfers for a decode loop (no counterpart in the method: plumbing for a
+ * caller that keeps its inputs and outputs in host memory).  One
+ * asynchronous copy on `stream`, in whichever direction the two addresses
+ * imply (host or device memory; unified addressing); page-locked host memory
+ * makes it overlap with kernels.  Ordering: stream order only, so the
+ * caller orders the copy against the step that reads or writes the device
+ * side (same stream, or events).  Nothing is owned or kept.
+ *   csa_copy_async: `bytes` contiguous bytes.
+ *   csa_copy_rows_async: `rows` rows of `row_bytes` bytes each, row r at
+ *   dst + r * dst_pitch and src + r * src_pitch (pitches >= row_bytes), e.g.
+ *   the new token's row of every sequence in a [B, L_cap, d] token buffer.
+ * Errors: a NULL address with a non-zero size or a pitch below row_bytes ->
+ * CSA_ERR_INVALID_ARG; a refused copy -> CSA_ERR_CUDA.  Zero bytes or rows
+ * enqueue nothing.
+ * ------------------------------------------------------------------------- */
+csa_status csa_copy_async(void* dst, const void* src, size_t bytes, void* stream);
+csa_status csa_copy_rows_async(void* dst, size_t dst_pitch, const void* src, size_t src_pitch,
+                               size_t row_bytes, size_t rows, void* stream);
+
+/* ---------------------------------------------------------------------------
  * YaRN RoPE frequency table (host only; no device work).  [P5] "5. 1M
  * context, gradually": the context is extended to 1,048,576 tokens with
  * YaRN, factor 16, beta_fast 32, beta_slow 1.  The pages give no formula;

@@ -249,6 +249,34 @@ def test_grouped_out_proj_workspace_grows_with_tokens(L):
     assert b >= 4096 * 16 * 1024 * 2
 
 
+def test_copy_entry_points_check_arguments(L):
+    """csa_copy_async / csa_copy_rows_async refuse NULL addresses and pitches
+    below the row before any copy is enqueued; empty copies do nothing."""
+    import ctypes as C
+    buf = (C.c_char * 64)()
+    a = C.cast(buf, C.c_void_p)
+    assert L.csa_copy_async(a, a, 0, None) == 0
+    assert L.csa_copy_async(None, a, 16, None) == 1
+    assert L.csa_copy_async(a, None, 16, None) == 1
+    assert L.csa_copy_rows_async(a, 64, a, 64, 0, 3, None) == 0
+    assert L.csa_copy_rows_async(a, 64, a, 64, 16, 0, None) == 0
+    assert L.csa_copy_rows_async(a, 8, a, 64, 16, 2, None) == 1
+    assert L.csa_copy_rows_async(a, 64, a, 8, 16, 2, None) == 1
+    assert L.csa_copy_rows_async(None, 64, a, 64, 16, 2, None) == 1
+    assert b"pitch" in L.csa_last_error() or b"NULL" in L.csa_last_error()
+
+
+def test_prepared_copy_checks_its_tensors(L):
+    """PreparedCopy wants equal shapes and dtypes and page-locked host
+    memory (checked before the library is called)."""
+    import torch
+    a, b = torch.zeros(4, 8), torch.zeros(4, 9)
+    with pytest.raises(ValueError):
+        binding.PreparedCopy(a, b)
+    with pytest.raises(ValueError):
+        binding.PreparedCopy(a, a.clone())  # neither side on a device nor pinned
+
+
 def test_prepared_decode_steps_reject_host_tensors(L):
     """CsaDecodeStep / HcaDecodeStep check their tensors like the plain calls
     (host tensors are refused before anything reaches the library)."""

@@ -359,8 +359,9 @@ def test_histogram_topk_flash_yarn(orc):
 
 def test_prepared_decode_steps_match_the_plain_calls():
     """binding.CsaDecodeStep / HcaDecodeStep (the unchanging arguments
-    converted once) run the same C entry points: the same outputs, bit for
-    bit, as csa_decode_step / hca_decode_step."""
+    converted once), called per step or bound to the step's buffers, run the
+    same C entry points: the same outputs, bit for bit, as csa_decode_step /
+    hca_decode_step."""
     for csa in (True, False):
         w = configs.scaled(configs.CSA_128K if csa else configs.HCA_1M, B=2, L=4096)
         p = binding.params_for(w)
@@ -385,14 +386,17 @@ def test_prepared_decode_steps_match_the_plain_calls():
                     qi["w"][:, 0].contiguous())
             tidx = torch.zeros(w.B, w.k, dtype=torch.int32, device=DEV)
             tcnt = torch.zeros(w.B, dtype=torch.int32, device=DEV)
-            for prepared in (False, True):
+            for mode in ("plain", "prepared", "bound"):
                 out = torch.full((w.B, w.H, w.D), float("nan"), dtype=torch.bfloat16, device=DEV)
                 lse = torch.full((w.B, w.H), float("nan"), dtype=torch.float32, device=DEV)
-                if prepared:
+                if mode != "plain":
                     f = binding.CsaDecodeStep(p, kv_tok, idx_tok, w_s, b_pos, None, w_si, b_pi,
                                               kv_c, key, ksc, qi["sink"], tidx, tcnt, ws,
                                               dev_status=status)
-                    f(pos, *args, out, lse=lse)
+                    if mode == "bound":
+                        f.bind(pos, *args, out, lse=lse)()
+                    else:
+                        f(pos, *args, out, lse=lse)
                 else:
                     binding.csa_decode_step(p, pos, kv_tok, idx_tok, w_s, b_pos, None, w_si, b_pi,
                                             kv_c, key, ksc, *args, qi["sink"], tidx, tcnt, out,
@@ -403,25 +407,59 @@ def test_prepared_decode_steps_match_the_plain_calls():
             ctx = torch.full((w.B,), w.L, dtype=torch.int64, device=DEV)
             binding.hca_compress(p, kv_tok, ctx, w_s, b_pos, None, 0, N, kv_c, dev_status=status)
             ws = binding.workspace(p, binding.OP_HCA_DECODE_STEP, 1, N)
-            for prepared in (False, True):
+            for mode in ("plain", "prepared", "bound"):
                 out = torch.full((w.B, w.H, w.D), float("nan"), dtype=torch.bfloat16, device=DEV)
                 lse = torch.full((w.B, w.H), float("nan"), dtype=torch.float32, device=DEV)
-                if prepared:
+                if mode != "plain":
                     f = binding.HcaDecodeStep(p, kv_tok, w_s, b_pos, None, kv_c, qi["sink"], ws,
                                               dev_status=status)
-                    f(pos, q, out, lse=lse)
+                    if mode == "bound":
+                        f.bind(pos, q, out, lse=lse)()
+                    else:
+                        f(pos, q, out, lse=lse)
                 else:
                     binding.hca_decode_step(p, pos, kv_tok, w_s, b_pos, None, kv_c, q, qi["sink"],
                                             out, lse=lse, ws=ws, dev_status=status)
                 torch.cuda.synchronize()
                 outs.append((out.clone(), lse.clone(), None))
         assert status.item() == 0
-        (o0, l0, t0), (o1, l1, t1) = outs
+        o0, l0, t0 = outs[0]
         assert torch.isfinite(o0.float()).all()
-        assert torch.equal(o0.view(torch.int16), o1.view(torch.int16))
-        assert torch.equal(l0, l1)
-        if csa:
-            assert torch.equal(t0, t1)
+        for o1, l1, t1 in outs[1:]:
+            assert torch.equal(o0.view(torch.int16), o1.view(torch.int16))
+            assert torch.equal(l0, l1)
+            if csa:
+                assert torch.equal(t0, t1)
+
+
+def test_prepared_copies_round_trip():
+    """binding.PreparedCopy (csa_copy_async / csa_copy_rows_async): pinned
+    host rows into one strided row per sequence of a device token buffer, a
+    contiguous upload, and a download, each on its own stream; every byte
+    arrives and no other byte of the buffer changes."""
+    g = torch.Generator().manual_seed(5)
+    B, L_cap, d = 3, 37, 512
+    buf = torch.randn(B, L_cap, d, generator=g).to(torch.bfloat16).to(DEV)
+    before = buf.clone()
+    rows = torch.randn(B, 1, d, generator=g).to(torch.bfloat16).pin_memory()
+    flat = torch.randint(0, 256, (4099,), dtype=torch.uint8, generator=g).pin_memory()
+    dflat = torch.zeros(4099, dtype=torch.uint8, device=DEV)
+    back = torch.zeros(B, L_cap, d, dtype=torch.bfloat16).pin_memory()
+    up, down = torch.cuda.Stream(), torch.cuda.Stream()
+    c_rows = binding.PreparedCopy(buf[:, 11:12], rows, up)
+    c_flat = binding.PreparedCopy(dflat, flat, up)
+    c_back = binding.PreparedCopy(back, buf, down)
+    assert c_rows.bytes == B * d * 2 and c_flat.bytes == 4099
+    c_rows()
+    c_flat()
+    down.wait_stream(up)
+    c_back()
+    torch.cuda.synchronize()
+    want = before.clone()
+    want[:, 11:12] = rows.to(DEV)
+    assert torch.equal(buf.view(torch.int16), want.view(torch.int16))
+    assert torch.equal(back.view(torch.int16), want.cpu().view(torch.int16))
+    assert torch.equal(dflat.cpu(), flat)
 
 
 def test_histogram_topk_single_sequence(orc):
