@@ -436,6 +436,41 @@ CSA_DEV uint32_t row_rounds(const uint32_t* keys, int n, uint32_t k_rem, RowShar
 // T that precede keys[0] in index order.  Warp w owns positions
 // [w*chunk, (w+1)*chunk) (chunk a multiple of 32); lane l takes element
 // j*32 + l of the chunk, so a ballot ranks it.  All 1024 threads call it.
+// Sums each warp's (a, b) over its lanes and returns, to every thread of
+// the warp, the sums of the warps before it (block exclusive prefix in warp
+// order).  All 1024 threads call it.
+CSA_DEV void warp_excl_prefix(uint32_t a, uint32_t b, RowShared& sh, uint32_t& pa, uint32_t& pb) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    a += __shfl_xor_sync(0xffffffffu, a, o);
+    b += __shfl_xor_sync(0xffffffffu, b, o);
+  }
+  if (lane == 0) {
+    sh.warp_a[warp] = a;
+    sh.warp_b[warp] = b;
+  }
+  cta_sync();
+  if (warp == 0) {
+    const uint32_t x = sh.warp_a[lane], y = sh.warp_b[lane];
+    uint32_t sa = x, sb = y;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t ya = __shfl_up_sync(0xffffffffu, sa, o);
+      const uint32_t yb = __shfl_up_sync(0xffffffffu, sb, o);
+      if (lane >= o) {
+        sa += ya;
+        sb += yb;
+      }
+    }
+    sh.warp_a[lane] = sa - x;
+    sh.warp_b[lane] = sb - y;
+  }
+  cta_sync();
+  pa = sh.warp_a[warp];
+  pb = sh.warp_b[warp];
+}
+
 template <typename Emit>
 CSA_DEV void ordered_emit(const uint32_t* keys, int n, int k, uint32_t T, uint32_t M,
                           uint32_t need_eq, uint32_t gt_base, uint32_t eq_base, RowShared& sh,
@@ -449,38 +484,51 @@ CSA_DEV void ordered_emit(const uint32_t* keys, int n, int k, uint32_t T, uint32
     n_gt += km > T;
     n_eq += km == T;
   }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    n_gt += __shfl_xor_sync(0xffffffffu, n_gt, o);
-    n_eq += __shfl_xor_sync(0xffffffffu, n_eq, o);
-  }
-  if (lane == 0) {
-    sh.warp_a[warp] = n_gt;
-    sh.warp_b[warp] = n_eq;
-  }
-  cta_sync();
-  if (warp == 0) {
-    const uint32_t a = sh.warp_a[lane], b = sh.warp_b[lane];
-    uint32_t sa = a, sb = b;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const uint32_t ya = __shfl_up_sync(0xffffffffu, sa, o);
-      const uint32_t yb = __shfl_up_sync(0xffffffffu, sb, o);
-      if (lane >= o) {
-        sa += ya;
-        sb += yb;
-      }
-    }
-    sh.warp_a[lane] = sa - a;
-    sh.warp_b[lane] = sb - b;
-  }
-  cta_sync();
-  uint32_t gt_run = gt_base + sh.warp_a[warp], eq_run = eq_base + sh.warp_b[warp];
+  uint32_t gt_run, eq_run;
+  warp_excl_prefix(n_gt, n_eq, sh, gt_run, eq_run);
+  gt_run += gt_base;
+  eq_run += eq_base;
   const uint32_t lt = (1u << lane) - 1u;
   for (int i = w0 + lane; i - lane < w1; i += 32) {
     const uint32_t km = i < w1 ? keys[i] & M : 0u;
     const bool gt = i < w1 && km > T;
     const bool eq = i < w1 && km == T;
+    const uint32_t bg = __ballot_sync(0xffffffffu, gt);
+    const uint32_t be = __ballot_sync(0xffffffffu, eq);
+    const uint32_t eq_rank = eq_run + __popc(be & lt);
+    if (gt || (eq && eq_rank < need_eq)) {
+      const uint32_t o = gt_run + __popc(bg & lt) + min(need_eq, eq_rank);
+      if (o < (uint32_t)k) emit(o, i);
+    }
+    gt_run += __popc(bg);
+    eq_run += __popc(be);
+  }
+}
+
+// The same output as ordered_emit when every key the selection can take
+// is listed: warp w passes its list of n_list positions (ascending, and all
+// of them below those of warp w + 1), so only the listed keys are read.
+template <typename Emit>
+CSA_DEV void list_emit(const uint32_t* keys, const uint16_t* list, int n_list, int k, uint32_t T,
+                       uint32_t M, uint32_t need_eq, uint32_t gt_base, uint32_t eq_base,
+                       RowShared& sh, Emit emit) {
+  const int lane = threadIdx.x & 31;
+  uint32_t n_gt = 0, n_eq = 0;
+  for (int e = lane; e < n_list; e += 32) {
+    const uint32_t km = keys[list[e]] & M;
+    n_gt += km > T;
+    n_eq += km == T;
+  }
+  uint32_t gt_run, eq_run;
+  warp_excl_prefix(n_gt, n_eq, sh, gt_run, eq_run);
+  gt_run += gt_base;
+  eq_run += eq_base;
+  const uint32_t lt = (1u << lane) - 1u;
+  for (int e = lane; e - lane < n_list; e += 32) {
+    const int i = e < n_list ? (int)list[e] : 0;
+    const uint32_t km = e < n_list ? keys[i] & M : 0u;
+    const bool gt = e < n_list && km > T;
+    const bool eq = e < n_list && km == T;
     const uint32_t bg = __ballot_sync(0xffffffffu, gt);
     const uint32_t be = __ballot_sync(0xffffffffu, eq);
     const uint32_t eq_rank = eq_run + __popc(be & lt);
@@ -598,13 +646,20 @@ __global__ void __launch_bounds__(kThreads, 1) topk_row_kernel(const Params p) {
 //   - otherwise each CTA ranks the candidates of all slots locally (radix
 //     rounds below b*), which gives the threshold key, and from the
 //     per-slot counts above / equal to it its offset in the index-ordered
-//     output, then emits its slice.
+//     output, then emits its slice.  Each warp owns a contiguous chunk of
+//     the slice and lists, in order, the positions of its keys in b* or
+//     above (every key the selection can take), so the emission reads only
+//     those; a warp whose list overflows sends the CTA through the emission
+//     over its whole slice.
 // The histogram is cleared (each CTA its share) once every CTA has read it.
+constexpr int kListCap = 64;  // listed positions per warp
 struct HistShared {
   alignas(16) uint32_t cbuf[kScoreHistBins];  // candidates, slot c at [c*cap, (c+1)*cap)
   alignas(16) uint32_t cn[kMaxC][2];           // per-slot (above b*, candidates)
   uint32_t gq[kMaxC][2];                       // per-slot (above T, equal to T)
-  uint32_t cand_n, above_n, bstar, pad_;
+  uint32_t cand_n, above_n, bstar, list_ovf;
+  uint32_t list_n[32];                         // per-warp list lengths
+  uint16_t list[32][kListCap];                 // per-warp positions at or above b*
   RowShared row;                               // rounds over the candidates
 };
 
@@ -629,6 +684,7 @@ __global__ void __launch_bounds__(kThreads, 1) topk_hist_kernel(const Params p) 
     hs.cand_n = 0;
     hs.above_n = 0;
     hs.bstar = 0xFFFFFFFFu;  // no bin found
+    hs.list_ovf = 0;
   }
   cluster_arrive();  // paired with the wait before the first remote store
   pdl_wait();  // the scores and the histogram come from the indexer kernel
@@ -657,12 +713,16 @@ __global__ void __launch_bounds__(kThreads, 1) topk_hist_kernel(const Params p) 
   const int cap_n = (int)(p.N_cap - lo < p.slice ? (p.N_cap - lo > 0 ? p.N_cap - lo : 0) : p.slice);
   const float* src = p.scores + (int64_t)row * p.N_cap + lo;
   const int len = (int)(n - lo < cap_n ? (n - lo > 0 ? n - lo : 0) : cap_n);
+  // Warp w owns positions [w*ch, (w+1)*ch) of the slice (ch a multiple of
+  // 32); lane l reads position w*ch + 32*j + l at step j, kPer steps per pass.
+  const int ch = (((len + 31) / 32) + 31) & ~31;
+  const int wbase = warp * ch;
   constexpr int kPer = 8;  // scores per thread per pass (slices up to 8192 in one)
   float sv[kPer];
 #pragma unroll
   for (int j = 0; j < kPer; ++j) {
-    const int i = tid + j * kThreads;
-    sv[j] = i < len ? __ldg(src + i) : 0.f;
+    const int i = wbase + 32 * j + lane;
+    sv[j] = (32 * j < ch && i < len) ? __ldg(src + i) : 0.f;
   }
 
   // b*: an exclusive scan over threads counts the scores in higher bins.
@@ -682,39 +742,70 @@ __global__ void __launch_bounds__(kThreads, 1) topk_hist_kernel(const Params p) 
   cta_sync();
   const uint32_t bstar = hs.bstar;
 
-  // This CTA's keys (to shared memory) above b* (counted) and in b* (copied
-  // to its slot), pass by pass over the visible part of the slice.
-  uint32_t n_above = 0;
+  // This CTA's keys (to shared memory) above b* (counted), pass by pass
+  // over the visible part of the slice; each warp lists the positions of its
+  // keys in b* or above, in order.
+  uint32_t n_above = 0, n_list = 0;
   uint32_t* mine = hs.cbuf + r * cap;
-  for (int base_i = 0; base_i < len; base_i += kPer * kThreads) {
-    if (base_i > 0) {
+  uint16_t* my_list = hs.list[warp];
+  const uint32_t lt = (1u << lane) - 1u;
+  for (int j0 = 0; 32 * j0 < ch; j0 += kPer) {
+    if (j0 > 0) {
 #pragma unroll
       for (int j = 0; j < kPer; ++j) {
-        const int i = base_i + tid + j * kThreads;
-        sv[j] = i < len ? __ldg(src + i) : 0.f;
+        const int i = wbase + 32 * (j0 + j) + lane;
+        sv[j] = (32 * (j0 + j) < ch && i < len) ? __ldg(src + i) : 0.f;
       }
     }
 #pragma unroll
     for (int j = 0; j < kPer; ++j) {
-      const int i = base_i + tid + j * kThreads;  // warp-uniform range per j
+      const int i = wbase + 32 * (j0 + j) + lane;
+      const bool in = 32 * (j0 + j) < ch && i < len;
       const uint32_t key = orderable(sv[j]);
-      if (i < len) keys[i] = key;
+      if (in) keys[i] = key;
       const uint32_t bin = key >> kShift;
-      n_above += (i < len && bin > bstar) ? 1u : 0u;
-      const bool cand = i < len && bin == bstar;
-      const uint32_t bal = __ballot_sync(0xffffffffu, cand);
-      if (bal) {
-        uint32_t at = 0;
-        if (lane == 0) at = atomicAdd(&hs.cand_n, (uint32_t)__popc(bal));
-        at = __shfl_sync(0xffffffffu, at, 0);
-        const uint32_t o = at + __popc(bal & ((1u << lane) - 1u));
-        if (cand && o < (uint32_t)cap) mine[o] = key;
-      }
+      n_above += (in && bin > bstar) ? 1u : 0u;
+      const bool ge = in && bin >= bstar;
+      const uint32_t bge = __ballot_sync(0xffffffffu, ge);
+      const uint32_t o = n_list + __popc(bge & lt);
+      if (ge && o < (uint32_t)kListCap) my_list[o] = (uint16_t)i;
+      n_list += __popc(bge);
+    }
+  }
+  // The keys in b* (the candidates) to this CTA's slot, from the warp's list
+  // or, where it overflowed, from its chunk of keys.
+  __syncwarp();  // the warp's keys are in shared memory
+  auto append = [&](bool cand, uint32_t key) {
+    const uint32_t bal = __ballot_sync(0xffffffffu, cand);
+    if (bal) {
+      uint32_t at = 0;
+      if (lane == 0) at = atomicAdd(&hs.cand_n, (uint32_t)__popc(bal));
+      at = __shfl_sync(0xffffffffu, at, 0);
+      const uint32_t o = at + __popc(bal & lt);
+      if (cand && o < (uint32_t)cap) mine[o] = key;
+    }
+  };
+  if (n_list <= (uint32_t)kListCap) {
+    for (int e0 = 0; e0 < (int)n_list; e0 += 32) {
+      const int e = e0 + lane;
+      const uint32_t key = e < (int)n_list ? keys[my_list[e]] : 0u;
+      append(e < (int)n_list && (key >> kShift) == bstar, key);
+    }
+  } else {
+    const int wend = min(len, wbase + ch);
+    for (int i0 = wbase; i0 < wend; i0 += 32) {
+      const int i = i0 + lane;
+      const uint32_t key = i < wend ? keys[i] : 0u;
+      append(i < wend && (key >> kShift) == bstar, key);
     }
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) n_above += __shfl_xor_sync(0xffffffffu, n_above, o);
-  if (lane == 0 && n_above) atomicAdd(&hs.above_n, n_above);
+  if (lane == 0) {
+    if (n_above) atomicAdd(&hs.above_n, n_above);
+    hs.list_n[warp] = n_list;
+    if (n_list > (uint32_t)kListCap) hs.list_ovf = 1;
+  }
   cta_sync();
   cluster_wait();  // every CTA of the cluster is running
 
@@ -785,8 +876,12 @@ __global__ void __launch_bounds__(kThreads, 1) topk_hist_kernel(const Params p) 
     gt_base += hs.gq[c][0];
     eq_base += hs.gq[c][1];
   }
-  ordered_emit(keys, len, p.k, T, M, need_eq, gt_base, eq_base, hs.row,
-               [&](uint32_t o, int i) { out[o] = (int32_t)(lo + i); });
+  auto put = [&](uint32_t o, int i) { out[o] = (int32_t)(lo + i); };
+  if (hs.list_ovf)
+    ordered_emit(keys, len, p.k, T, M, need_eq, gt_base, eq_base, hs.row, put);
+  else
+    list_emit(keys, hs.list[warp], (int)hs.list_n[warp], p.k, T, M, need_eq, gt_base, eq_base,
+              hs.row, put);
   if (r == 0 && tid == 0) {
     p.cnt[row] = p.k;
     if (p.path) p.path[row] = 1;
