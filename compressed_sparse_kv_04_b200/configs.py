@@ -76,14 +76,19 @@ HCA_PREFILL = Workload("hca_prefill_4096_after_65536", "hca_prefill", B=1, L=655
 
 # Reduced cases for profiler captures (a few GB on the device): the 128K CSA
 # decode with a 32K context (the same per-row attention work: 1024 selected
-# entries + the window), and the HCA decode at 256K (2048 entries per row).
+# entries + the window), the HCA decode at 256K (2048 entries per row), and
+# the 1M CSA decode's batch of 4 at 32K.
 CSA_32K_PROFILE = Workload("csa_decode_32k_b8", "csa_decode", B=8, L=32768, d=512, m=4, H=128,
                            rope_dim=64, W=128, H_I=64, D_I=128, k=1024, seed=20260009)
 HCA_256K_PROFILE = Workload("hca_decode_256k_b8", "hca_decode", B=8, L=262144, d=512, m=128,
                             H=128, rope_dim=64, W=128, seed=20260010)
+# The 1M CSA decode's attention work (4 sequences x (1024 selected entries +
+# the window)) with a 32K context.
+CSA_32K_B4_PROFILE = Workload("csa_decode_32k_b4", "csa_decode", B=4, L=32768, d=512, m=4, H=128,
+                              rope_dim=64, W=128, H_I=64, D_I=128, k=1024, seed=20260011)
 
 ALL = [TINY_CSA, CSA_128K, HCA_1M, CSA_1M, CSA_PREFILL, CSA_FLASH_128K, HCA_PREFILL,
-       CSA_32K_PROFILE, HCA_256K_PROFILE]
+       CSA_32K_PROFILE, HCA_256K_PROFILE, CSA_32K_B4_PROFILE]
 BY_NAME = {w.name: w for w in ALL}
 
 

@@ -314,27 +314,44 @@ def test_histogram_topk_csa_1m_shape(orc):
     st.check_attention(orc, pos, qi, tidx, tcnt)
 
 
-@pytest.mark.parametrize("case", ["ties", "all_equal", "few_visible"])
+@pytest.mark.parametrize("case", ["ties", "all_equal", "few_visible", "recent_block"])
 def test_histogram_topk_structures(orc, case):
     """Two sequences x 16384 entries, k = 512 (4-CTA clusters, 1024 slots):
     ties: one key row for every entry and 64 key scales, so scores take 64
     values and the threshold bin holds 8 of them (the tie rule across CTAs);
     all_equal: one score everywhere, more candidates than slots (the full
     select, lowest indices); few_visible: one sequence with fewer visible
-    entries than k next to one on the histogram path."""
+    entries than k next to one on the histogram path; recent_block: the 600
+    highest scores on the last 600 entries (each warp chunk there holds more
+    keys at or above the threshold bin than its position list: the emission
+    over the whole slice, on the histogram path)."""
     w = configs.scaled(configs.CSA_128K, B=2, k=512, L=65536)
     st = _Step(w, w.L, seed=5)
     N = st.N
     row = synth.e4m3_codes((1, 1, w.D_I), 6, "q_idx", DEV)
     st.key.copy_(row.expand(w.B, N, w.D_I))
-    if case == "ties":
+    if case == "recent_block":
+        # The sign of each sequence's score for this key row (its query and
+        # head weights), so that the block holds the largest scores.
+        qi0 = synth.queries(configs.scaled(st.w, seed=w.seed + 1000), Q=1, device=DEV)
+        t = torch.arange(N, device=DEV, dtype=torch.float32)
+        blk = (t - (N - 600)).clamp(min=0) / 600
+        for b in range(w.B):
+            c = orc.index_scores(bits8(qi0["q_idx"][b: b + 1]), f32(qi0["q_scale"][b: b + 1]),
+                                 f32(qi0["w"][b: b + 1]), bits8(row), np.ones((1, 1)),
+                                 np.array([[w.m - 1]]), w.m)[0, 0][0]
+            assert c != 0
+            base = (1 + t / N) / 64
+            top = (4 + 3.9 * blk) / 64 if c > 0 else (0.49 - 0.24 * blk) / 64
+            st.ksc[b].copy_(torch.where(t >= N - 600, top, base))
+    elif case == "ties":
         vals = 1.0 + torch.arange(64, device=DEV, dtype=torch.float32) / 64
         rng = torch.Generator(device=DEV).manual_seed(7)
         st.ksc.copy_(vals[torch.randint(0, 64, (w.B, N), generator=rng, device=DEV)] / 64)
     else:
         st.ksc.fill_(1.0 / 64)
     pos = np.full(w.B, w.L - 1)
-    expect = [1, 1] if case == "ties" else [2, 2]
+    expect = [1, 1] if case in ("ties", "recent_block") else [2, 2]
     if case == "few_visible":
         pos[0] = 4 * 400 - 1
         expect = [0, 2]
