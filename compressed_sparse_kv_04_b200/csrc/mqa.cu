@@ -324,9 +324,23 @@ __global__ void __launch_bounds__(kThreads, 1)
   // the S splits of one head group are consecutive (one cluster when the
   // partials are merged in-cluster).
   const bool pair = p.H > HC;
-  const int hg0 = pair ? (int)(blockIdx.x / p.splits) * HC : 0;  // first head of this CTA
-  const int split = (int)(blockIdx.x % p.splits);
-  const int row = blockIdx.y;
+  // Sparse decode without the in-cluster merge: the CTAs of every head
+  // group's last split (the window tiles, which wait for no other kernel of
+  // the call) come first in launch order, so CTAs that start late, on SMs the
+  // top-k frees, hold only selected tiles.
+  int gx = (int)blockIdx.x, gy = (int)blockIdx.y;
+  if (p.Q == 1 && p.sel_idx != nullptr && !p.cluster_merge && p.splits > 1) {
+    const int64_t G = (int64_t)gridDim.x / p.splits;  // head groups per row
+    const int64_t ng = G * gridDim.y;
+    const int64_t L = (int64_t)blockIdx.x + (int64_t)gridDim.x * blockIdx.y;
+    const int64_t grp = L < ng ? L : (L - ng) / (p.splits - 1);
+    const int64_t sp = L < ng ? p.splits - 1 : (L - ng) % (p.splits - 1);
+    gy = (int)(grp / G);
+    gx = (int)((grp % G) * p.splits + sp);
+  }
+  const int hg0 = pair ? (gx / p.splits) * HC : 0;  // first head of this CTA
+  const int split = gx % p.splits;
+  const int row = gy;
   const int b = row / p.Q;
 
   // The KV list of this query row: n_c compressed entries, then the window.
