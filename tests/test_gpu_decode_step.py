@@ -449,6 +449,32 @@ def test_prepared_decode_steps_match_the_plain_calls():
                 assert torch.equal(t0, t1)
 
 
+def test_decode_step_newest_entries_match_compress():
+    """The decode step's newest entry of each sequence (KV row, indexer key
+    and scale) has the same bits as csa_compress over the same tokens.
+    Positions: a complete block, a partial one, and a partial block that
+    opens an indexer tile past the visible ones."""
+    w = configs.scaled(configs.CSA_128K, B=3, L=8192)
+    st = _Step(w, w.L, seed=13)
+    st.compress_all(w.L)
+    pos = np.array([w.L - 1, w.L - 3, 4096])
+    st.run(pos, w.seed + 1000)
+    N = st.N
+    kv_c = torch.zeros_like(st.kv_c)
+    key = torch.zeros_like(st.key)
+    ksc = torch.zeros_like(st.ksc)
+    ctx = torch.from_numpy(pos + 1).to(DEV)
+    binding.csa_compress(st.p, st.kv_tok, ctx, st.w_s, st.b_pos, None, 0, N, kv_c, st.idx_tok,
+                         st.w_si, st.b_pi, key, ksc, dev_status=st.status)
+    torch.cuda.synchronize()
+    assert st.status.item() == 0
+    for b in range(w.B):
+        i = int(pos[b]) // w.m
+        assert torch.equal(st.kv_c[b, i].view(torch.int16), kv_c[b, i].view(torch.int16)), b
+        assert torch.equal(st.key[b, i], key[b, i]), b
+        assert torch.equal(st.ksc[b, i], ksc[b, i]), b
+
+
 def test_prepared_copies_round_trip():
     """binding.PreparedCopy (csa_copy_async / csa_copy_rows_async): pinned
     host rows into one strided row per sequence of a device token buffer, a
