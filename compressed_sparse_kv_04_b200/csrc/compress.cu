@@ -5,14 +5,14 @@
 // "DeepSeek V4 technical report" (agentupdate.ai), hybrid attention: CSA step
 // 1 (m tokens merged with learned attention-like weights) and the HCA
 // paragraph (m' = 128, no overlap); "DeepSeek V4-Pro" (llm-arch-kb), "Hybrid
-// attention" CSA / HCA bullets.  Weight form (the build's reading):
+// attention" CSA / HCA bullets.  Weight form (the reading taken here):
 // softmax_j(c_t . w_s + b_pos[j]) over the present tokens of the block.
 // Overlapping variant (CSA; the pages fix "no overlap" for HCA only): entry i
 // pools the window of m + overlap tokens i*m - overlap .. (i+1)*m - 1, with
 // b_pos indexed by the window position, clipped at the sequence start and at
 // the context end.
 //
-// Storage (the build's reading): a KV entry is stored already rotated (RoPE
+// Storage (the reading taken here): a KV entry is stored already rotated (RoPE
 // on the last rope_dim dims, "DeepSeek V4-Pro" (llm-arch-kb), "Hybrid
 // attention") to its own position (i+1)*m - 1, so attention uses it as
 // stored; indexer keys are not rotated.

@@ -2,7 +2,7 @@
 //
 // "DeepSeek V4 technical report" (agentupdate.ai), CSA step 2 keeps the k
 // highest-scoring compressed blocks per query; "DeepSeek V4-Pro" (llm-arch-kb)
-// sets k = 1024.  Tie rule (the build's): score descending, then index
+// sets k = 1024.  Tie rule (chosen here): score descending, then index
 // ascending; NaN below every number; -0 == +0.  Output: ascending indices,
 // padded with -1, and the count min(k, n_vis).
 //

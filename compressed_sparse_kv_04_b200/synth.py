@@ -6,7 +6,7 @@ Generator seeded from the workload seed plus a fixed per-tensor offset, so the
 same call gives the same bits on any machine (CPU generator) or on any device
 of one kind (CUDA generator).
 
-Distributions (the pages fix none; these are the build's choices):
+Distributions (the pages fix none; these are this library's choices):
   token KV / indexer streams  N(0, 1)          -> bfloat16
   pooling w_s                 N(0, 0.02)       fp32 [d]
   pooling b_pos               N(0, 0.1)        fp32 [m]

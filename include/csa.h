@@ -82,7 +82,7 @@ typedef struct {
   int window;          /* uncompressed sliding window W ([P5]: 128) */
   int rope_dim;        /* rotated trailing dims r ([P5]: 64) */
   int m;               /* compression ratio ([P5]: 4 for CSA, 128 for HCA) */
-  float eps;           /* RMSNorm epsilon (1e-6 in the build's tests) */
+  float eps;           /* RMSNorm epsilon (1e-6 in the tests) */
   float softmax_scale; /* logit scale; 0 selects 1/sqrt(d) */
   const double* rope_inv_freq; /* host, [rope_dim/2] angle per position for
                                   pair j; NULL selects 10000^(-2j/rope_dim) */
@@ -193,7 +193,7 @@ size_t csa_workspace_bytes(const csa_params* p, csa_op op, int Q, int64_t N_cap)
  * position of the block's last token ([P5]: RoPE on the last 64 dims of the
  * KV) -- is stored as bf16 in kv_c[b,i,:], so that attention uses entries
  * as stored.  A block with no present token is left untouched.  (The weight
- * form and the place of the rotation are the build's readings: the pages
+ * form and the place of the rotation are the readings taken here: the pages
  * fix neither.)  rope_dim must be 0, 32 or 64 and at most d/4.
  *
  *   kv_tok  [B, L_cap, d] bf16 (device)     token KV stream
@@ -212,7 +212,7 @@ csa_status hca_compress(const csa_params* p, const void* kv_tok, int64_t L_cap,
  * KV compression, CSA form ([P2] CSA step 1; [P5] CSA bullet: m = 4).
  * The KV stream is pooled exactly as hca_compress does.
  * Overlapping variant (p->overlap > 0; [P2] states "no overlap" for HCA
- * only and gives no rule for CSA, so this is the build's reading): entry i
+ * only and gives no rule for CSA, so this is the reading taken here): entry i
  * pools the window of m + overlap tokens t = i*m - overlap + j (j < m +
  * overlap), those with 0 <= t < ctx_len, scored with b_pos[j]; b_pos then
  * holds m + overlap values.  The entry is still written once its own block
@@ -500,7 +500,7 @@ csa_status grouped_out_proj(int T, int H, int D, int g, int d_g, int d_model, co
  *
  * The pages give no parallel scheme for this path ("Architectural Overview
  * of V4 Series Models" (intl.cloud.baidu.com) names only 3D-parallel
- * training as an outlook); this is the build's.  Rank r holds the entries
+ * training as an outlook); this is this library's.  Rank r holds the entries
  * [lo_r, hi_r) of the compressed KV cache and of the indexer keys, a
  * contiguous range in rank order, described to every call by
  * csa_params.entry_offset = lo_r and N_cap = hi_r - lo_r.  One decode step:
