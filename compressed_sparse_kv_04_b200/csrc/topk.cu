@@ -505,24 +505,35 @@ CSA_DEV void ordered_emit(const uint32_t* keys, int n, int k, uint32_t T, uint32
   }
 }
 
+// Keys above T and equal to T (under mask M) among a warp's listed
+// positions, summed over the warp (every lane gets the sums).
+CSA_DEV void list_counts(const uint32_t* keys, const uint16_t* list, int n_list, uint32_t T,
+                         uint32_t M, uint32_t& gt, uint32_t& eq) {
+  const int lane = threadIdx.x & 31;
+  gt = 0;
+  eq = 0;
+  for (int e = lane; e < n_list; e += 32) {
+    const uint32_t km = keys[list[e]] & M;
+    gt += km > T;
+    eq += km == T;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    gt += __shfl_xor_sync(0xffffffffu, gt, o);
+    eq += __shfl_xor_sync(0xffffffffu, eq, o);
+  }
+}
+
 // The same output as ordered_emit when every key the selection can take
 // is listed: warp w passes its list of n_list positions (ascending, and all
 // of them below those of warp w + 1), so only the listed keys are read.
+// gt_run / eq_run: keys above / equal to T before the warp's first position
+// in index order (the slice's base plus the warps before it).
 template <typename Emit>
 CSA_DEV void list_emit(const uint32_t* keys, const uint16_t* list, int n_list, int k, uint32_t T,
-                       uint32_t M, uint32_t need_eq, uint32_t gt_base, uint32_t eq_base,
-                       RowShared& sh, Emit emit) {
+                       uint32_t M, uint32_t need_eq, uint32_t gt_run, uint32_t eq_run,
+                       Emit emit) {
   const int lane = threadIdx.x & 31;
-  uint32_t n_gt = 0, n_eq = 0;
-  for (int e = lane; e < n_list; e += 32) {
-    const uint32_t km = keys[list[e]] & M;
-    n_gt += km > T;
-    n_eq += km == T;
-  }
-  uint32_t gt_run, eq_run;
-  warp_excl_prefix(n_gt, n_eq, sh, gt_run, eq_run);
-  gt_run += gt_base;
-  eq_run += eq_base;
   const uint32_t lt = (1u << lane) - 1u;
   for (int e = lane; e - lane < n_list; e += 32) {
     const int i = e < n_list ? (int)list[e] : 0;
@@ -851,7 +862,19 @@ __global__ void __launch_bounds__(kThreads, 1) topk_hist_kernel(const Params p) 
   cta_sync();
   uint32_t T = bstar << kShift, M = 0xFFFFFFFFu << kShift;
   const uint32_t need_eq = row_rounds<10>(hs.cbuf, kScoreHistBins, k - A, hs.row, T, M, kShift);
-  // Per slot: keys above T (those above b* included) and equal to it.
+  // Per slot: keys above T (those above b* included) and equal to it; for
+  // the emission over the lists, each warp's own counts (read by every warp
+  // after the barrier below, which serves both).
+  const bool lists = hs.list_ovf == 0;
+  const int n_mine = (int)hs.list_n[warp];
+  if (lists) {
+    uint32_t gt, eq;
+    list_counts(keys, hs.list[warp], n_mine, T, M, gt, eq);
+    if (lane == 0) {
+      hs.row.warp_a[warp] = gt;
+      hs.row.warp_b[warp] = eq;
+    }
+  }
   if (warp < C) {
     const uint32_t nc = hs.cn[warp][1];
     uint32_t gt = 0, eq = 0;
@@ -877,11 +900,26 @@ __global__ void __launch_bounds__(kThreads, 1) topk_hist_kernel(const Params p) 
     eq_base += hs.gq[c][1];
   }
   auto put = [&](uint32_t o, int i) { out[o] = (int32_t)(lo + i); };
-  if (hs.list_ovf)
+  if (!lists) {
     ordered_emit(keys, len, p.k, T, M, need_eq, gt_base, eq_base, hs.row, put);
-  else
-    list_emit(keys, hs.list[warp], (int)hs.list_n[warp], p.k, T, M, need_eq, gt_base, eq_base,
-              hs.row, put);
+  } else {
+    // This warp's offset: the counts of the warps before it (a scan over
+    // the 32 warps' counts, in every warp).
+    const uint32_t a = hs.row.warp_a[lane], b = hs.row.warp_b[lane];
+    uint32_t sa = a, sb = b;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t ya = __shfl_up_sync(0xffffffffu, sa, o);
+      const uint32_t yb = __shfl_up_sync(0xffffffffu, sb, o);
+      if (lane >= o) {
+        sa += ya;
+        sb += yb;
+      }
+    }
+    const uint32_t pa = __shfl_sync(0xffffffffu, sa - a, warp);
+    const uint32_t pb = __shfl_sync(0xffffffffu, sb - b, warp);
+    list_emit(keys, hs.list[warp], n_mine, p.k, T, M, need_eq, gt_base + pa, eq_base + pb, put);
+  }
   if (r == 0 && tid == 0) {
     p.cnt[row] = p.k;
     if (p.path) p.path[row] = 1;
