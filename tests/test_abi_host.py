@@ -277,6 +277,21 @@ def test_prepared_copy_checks_its_tensors(L):
         binding.PreparedCopy(a, a.clone())  # neither side on a device nor pinned
 
 
+def test_prepared_copy_row_layout():
+    """The (rows, row bytes, pitch) that PreparedCopy passes to
+    csa_copy_rows_async: one row per first-dimension slice of a strided
+    view, its bytes contiguous, the pitch the first dimension's stride."""
+    import torch
+    buf = torch.zeros(3, 37, 512, dtype=torch.bfloat16)
+    assert binding._rows_of(buf[:, 11:12]) == (3, 1024, 37 * 512 * 2)
+    assert binding._rows_of(buf[:, 5:9]) == (3, 4 * 1024, 37 * 512 * 2)
+    host = torch.zeros(3, 1, 512, dtype=torch.bfloat16)
+    assert binding._rows_of(host) == (3, 1024, 1024)
+    assert binding._rows_of(torch.zeros(1, 7, dtype=torch.uint8)) == (1, 7, 7)
+    with pytest.raises(ValueError):  # rows that are not contiguous
+        binding._rows_of(buf[:, :, ::2])
+
+
 def test_prepared_decode_steps_reject_host_tensors(L):
     """CsaDecodeStep / HcaDecodeStep check their tensors like the plain calls
     (host tensors are refused before anything reaches the library)."""
